@@ -1,0 +1,165 @@
+/*
+ * nsa.h -- C ABI of libnsa, a B200 (sm_100a) implementation of the Native
+ * Sparse Attention (NSA) per-layer attention operator.
+ *
+ * What the operator computes (page "硬件对齐+原生训练！DeepSeek NSA打造高效稀疏
+ * Attention", section 二 NSA核心工作; explainer "DeepseekNativelySparseAttention",
+ * sections on compressed / selected / sliding-window attention and the gated
+ * fusion):  for every query token t and query head h of a causal GQA context
+ *
+ *     out[t,h] = g_cmp[t,h] * Attn(q[t,h], K~cmp, V~cmp)
+ *              + g_slc[t,h] * Attn(q[t,h], K[selected blocks], V[...])
+ *              + g_win[t,h] * Attn(q[t,h], K[t-w+1 .. t], V[...])
+ *
+ * with Attn(q, K, V) = softmax(scale * q K^T) V over the keys that branch
+ * remaps (token compression, top-n block selection, sliding window):
+ *   - compressed keys/values: K~[i] = phi(k[i*d .. i*d+l-1]) for blocks of
+ *     length l at stride d (phi = mean-pool, or a linear map of the flattened
+ *     block plus an intra-block position embedding), rounded to bf16; block i
+ *     is visible to t once complete (i*d + l - 1 <= t);
+ *   - selected blocks: selection blocks of l' tokens; importance
+ *     p'[t,g,j] = sum over the heads h of group g of sum_i w(i,j) p_cmp[t,h,i],
+ *     where p_cmp is the compressed branch's softmax and w(i,j) counts the
+ *     stride-d segments compressed block i shares with selection block j;
+ *     the first `forced_initial` blocks and the `forced_local` blocks ending
+ *     at floor(t/l') are always kept, the remaining n - forced are the
+ *     highest-scoring other candidates (ties to the lower index); when at most
+ *     n candidate blocks exist all are taken;
+ *   - window: the last w tokens up to and including t.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers to contiguous row-major arrays
+ *     owned by the caller; libnsa never allocates, frees or synchronises
+ *     device memory during a call.  Scratch memory is the caller-provided
+ *     workspace (size from nsa_workspace_size), 256-byte aligned.
+ *   - bf16 tensors (q, k, v, phi parameters, caches, dout) are bfloat16;
+ *     gates, out, lse and gradients are fp32; indices int32; offsets int64.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream).  The returned status covers argument validation and
+ *     kernel launch.  A device-side failure (a bounded wait that expired) is
+ *     reported by nsa_sync_status().
+ *   - Invalid arguments return NSA_ERR_INVALID_ARG and launch nothing.
+ *     Valid but unimplemented shapes return NSA_ERR_UNSUPPORTED.
+ */
+#ifndef NSA_H_
+#define NSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NSA_OK = 0,
+    NSA_ERR_INVALID_ARG = 1,   /* null pointer, inconsistent sizes, bad hyperparameters */
+    NSA_ERR_UNSUPPORTED = 2,   /* valid, but no kernel instantiated for these sizes */
+    NSA_ERR_WORKSPACE = 3,     /* workspace missing, misaligned or too small */
+    NSA_ERR_CUDA = 4,          /* a CUDA runtime/driver call or launch failed */
+    NSA_ERR_DEVICE_TIMEOUT = 5 /* a kernel's bounded wait expired (see nsa_sync_status) */
+} nsa_status_t;
+
+typedef enum { NSA_PHI_MEAN = 0, NSA_PHI_LINEAR = 1 } nsa_phi_t;
+
+typedef enum { NSA_MODE_FORWARD = 0, NSA_MODE_DECODE = 1, NSA_MODE_BACKWARD = 2 } nsa_mode_t;
+
+/* Operator configuration.  Token compression: block length l = cmp_block,
+ * stride d = cmp_stride.  Selection: block length l' = sel_block, n =
+ * sel_count blocks of which forced_initial + forced_local are always kept.
+ * Window: w = window tokens.  Requirements (validated): d divides l and l';
+ * l <= l'; n >= forced_initial + forced_local; num_q_heads a multiple of
+ * num_kv_groups.  Implemented sizes: (d_k, d_v) in {(64,64), (192,128)},
+ * heads per group in {4, 16}, l/d in {1, 2}, l'/d in {1, 2, 4}, score_map 0.
+ * For nsa_decode, `batch` is the number of sequences and `seqlen` the largest
+ * context length (they size the workspace). */
+typedef struct {
+    int32_t batch, seqlen, num_q_heads, num_kv_groups, d_k, d_v;
+    int32_t cmp_block, cmp_stride, sel_block, sel_count, forced_initial, forced_local, window;
+    int32_t phi;       /* nsa_phi_t */
+    int32_t score_map; /* 0: overlap-weighted mapping of compressed to selection blocks */
+    float scale;       /* softmax scale; 0 selects 1/sqrt(d_k) */
+} nsa_config_t;
+
+/* Linear phi parameters (bf16, device): w_k [d_k, l*d_k], e_k [l, d_k],
+ * w_v [d_v, l*d_v], e_v [l, d_v].  The flattened block is position-major:
+ * x[j*d_k + c] = k[i*d + j][c] + e_k[j][c], K~[i] = w_k x.  Unused (may be
+ * NULL) for NSA_PHI_MEAN. */
+typedef struct {
+    const void* w_k;
+    const void* e_k;
+    const void* w_v;
+    const void* e_v;
+} nsa_phi_params_t;
+
+/* Bytes of device workspace an entry point needs for this configuration. */
+size_t nsa_workspace_size(const nsa_config_t* cfg, int32_t mode);
+
+/* Number of compressed blocks over a context of `len` tokens:
+ * floor((len - l)/d) + 1, or 0 when len < l (token compression section). */
+int64_t nsa_num_cmp_blocks(const nsa_config_t* cfg, int64_t len);
+
+/* Token compression alone (page 2, 令牌压缩; explainer 2.2-2.3).
+ * k [B,T,G,d_k], v [B,T,G,d_v] -> kc [B,C,G,d_k], vc [B,C,G,d_v] (bf16,
+ * round-to-nearest-even), C = nsa_num_cmp_blocks(cfg, T).  Needs the FORWARD
+ * workspace. */
+nsa_status_t nsa_compress(const nsa_config_t* cfg, const void* k, const void* v,
+                          const nsa_phi_params_t* phi, void* kc, void* vc, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/* Prefill forward (page 2, sections 整体框架 / 算法设计 / 最终输出计算).
+ * In:  q [B,T,H,d_k], k [B,T,G,d_k], v [B,T,G,d_v] bf16; gates [B,T,H,3] fp32
+ *      in the order (compressed, selected, window), the sigmoid outputs.
+ * Out: out [B,T,H,d_v] fp32; sel_idx [B,T,G,n] int32 (ascending, -1 padded);
+ *      lse [B,T,H,3] fp32 natural-log log-sum-exp of each branch's scaled
+ *      logits (-inf where a branch sees no key) or NULL;
+ *      kc_out [B,C,G,d_k] / vc_out [B,C,G,d_v] bf16 compressed keys/values or
+ *      NULL.  sel_idx is required. */
+nsa_status_t nsa_forward(const nsa_config_t* cfg, const void* q, const void* k, const void* v,
+                         const float* gates, const nsa_phi_params_t* phi, float* out,
+                         int32_t* sel_idx, float* lse, void* kc_out, void* vc_out,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* Batched decode step (page 2, 效率分析 解码速度): one query per sequence at
+ * position t = L_s - 1 over caches that already hold the current token.
+ * q [S,H,d_k] bf16; k_cache [sumL,G,d_k], v_cache [sumL,G,d_v] bf16 with
+ * sequence s in rows [kv_offsets[s], kv_offsets[s+1]); kc_cache [sumC,G,d_k],
+ * vc_cache [sumC,G,d_v] bf16 with sequence s in rows [cmp_offsets[s],
+ * cmp_offsets[s+1]), which must number nsa_num_cmp_blocks(cfg, L_s);
+ * offsets are int64 device arrays of S+1 entries; gates [S,H,3] fp32.
+ * Out: out [S,H,d_v] fp32, sel_idx [S,G,n] int32, lse [S,H,3] fp32 or NULL.
+ * num_seqs must not exceed cfg->batch and no L_s may exceed cfg->seqlen (the
+ * workspace was sized from them); a wrong cache length is not detected on the
+ * device: the result for that sequence is undefined. */
+nsa_status_t nsa_decode(const nsa_config_t* cfg, int32_t num_seqs, const void* q,
+                        const void* k_cache, const void* v_cache, const int64_t* kv_offsets,
+                        const void* kc_cache, const void* vc_cache, const int64_t* cmp_offsets,
+                        const float* gates, float* out, int32_t* sel_idx, float* lse,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward with the block selection held fixed (pages: natively trainable
+ * design; training-speed paragraph of 效率分析).  In: the forward inputs, the
+ * upstream gradient dout [B,T,H,d_v] bf16 and sel_idx [B,T,G,n] (normally the
+ * forward's).  Out (fp32, overwritten): dq [B,T,H,d_k], dk [B,T,G,d_k],
+ * dv [B,T,G,d_v] (through all three branches and, for the compressed branch,
+ * through phi), dgates [B,T,H,3] = <dout, o_branch>.  The per-branch softmax
+ * statistics are recomputed.  No gradient flows into the importance scores,
+ * the phi parameters or the gate MLP. */
+nsa_status_t nsa_backward(const nsa_config_t* cfg, const void* q, const void* k, const void* v,
+                          const float* gates, const nsa_phi_params_t* phi, const void* dout,
+                          const int32_t* sel_idx, float* dq, float* dk, float* dv, float* dgates,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronise `stream`, then read and clear the device error word of the
+ * current device.  Returns NSA_ERR_DEVICE_TIMEOUT if a kernel's bounded wait
+ * expired since the last call, NSA_ERR_CUDA if synchronisation failed. */
+nsa_status_t nsa_sync_status(void* stream);
+
+/* Static description of a status code. */
+const char* nsa_status_string(nsa_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NSA_H_ */

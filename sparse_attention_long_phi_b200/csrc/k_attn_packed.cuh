@@ -1,0 +1,460 @@
+// k_attn_packed.cuh -- tcgen05 attention over a contiguous key range for a
+// tile of 128 query rows packed as (128/HG tokens) x (HG heads of one GQA
+// group).  Three modes:
+//
+//   kModeLse  compressed attention, pass 1: per-row log-sum-exp of the scaled
+//             logits over the visible compressed keys (explainer, compressed
+//             attention 2.4: A = Q K~^T / sqrt(d_k), softmax).
+//   kModeCmp  compressed attention, pass 2: with the row LSE known,
+//             P = exp(S - LSE) is the exact compressed-branch probability;
+//             O = P V~ needs no rescaling.  The same P feeds the selection
+//             importance scores (page 2, 重要性分数计算 / shared GQA scores):
+//             each row's probabilities are mapped to selection blocks with the
+//             overlap weights and summed over the HG heads of the token, then
+//             written to the score table [B,T,G,NSp].  out = g_cmp * O.
+//   kModeWin  sliding window (page 2, 滑动窗口): keys t-w+1 .. t, online softmax
+//             with lazy rescaling of the TMEM accumulator (only when a row's
+//             running max grows by more than 8 in log2 units).
+//             out += g_win * O / l.
+//
+// Warp roles: warps 0-3 softmax/epilogue (thread = query row), warp 4 TMA
+// producer, warp 5 MMA issuer and TMEM owner.  Key tiles of 64 keys.
+// S = Q K^T  (M=128, N=64, K=DK) into one of two TMEM buffers;
+// O += P V   (M=128, N=DV, K=64) with P staged in shared memory (bf16).
+#pragma once
+#include "nsa_dev.cuh"
+
+namespace nsa {
+
+enum { kModeLse = 0, kModeCmp = 1, kModeWin = 2 };
+
+struct PackedParams {
+    int B, T, H, G;
+    int l, d, lp, w;
+    float scale_log2;          // softmax scale * log2(e)
+    const float* gates;        // [B,T,H,3]
+    float* out;                // [B,T,H,DV]
+    float* lse_user;           // [B,T,H,3] or null
+    float* lse_cmp;            // [B,T,H] natural log (pass 1 writes, pass 2 reads)
+    float* pscore;             // [B,T,G,NSp]
+    int NSp;
+    int n_qtiles;
+};
+
+template <int DK, int DV, int HG, int MODE>
+struct PackedCfg {
+    static constexpr int TOK = 128 / HG;
+    static constexpr int BN = 64;
+    static constexpr int NQB = DK / 64;
+    static constexpr int kQBytes = 128 * DK * 2;
+    static constexpr int kKBox = BN * 128;            // 64 rows x 128 B
+    static constexpr int kKBytes = NQB * kKBox;
+    static constexpr int kVBytes = DV * 128;          // DV rows x 64 keys
+    static constexpr int kPBytes = 128 * 128;         // 128 rows x 64 keys
+    static constexpr int NSK = 3;
+    static constexpr int NSV = MODE == kModeLse ? 0 : 3;
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = kOffQ + kQBytes;
+    static constexpr int kOffV = kOffK + NSK * kKBytes;
+    static constexpr int kOffP = kOffV + NSV * kVBytes;
+    static constexpr int kOffBar = kOffP + (MODE == kModeLse ? 0 : kPBytes);
+    static constexpr int kSmem = kOffBar + 256 + 1024;
+    static constexpr uint32_t kTmemCols = 256;        // S0 [0,64) S1 [64,128) O [128,128+DV)
+};
+
+// Reduce `N` per-row values over the HG lanes of a token (lanes differing in
+// the low log2(HG) bits) and scatter: afterwards value v of this lane holds
+// the group sum of index `base + v`, with base given by bits of the lane id.
+template <int N, int HG>
+__device__ __forceinline__ int reduce_scatter_heads(float (&x)[N], int lane) {
+    int base = 0;
+    int cnt = N;
+#pragma unroll
+    for (int m = HG / 2; m >= 1; m >>= 1) {
+        const bool hi = (lane & m) != 0;
+        const int half = cnt / 2;
+#pragma unroll
+        for (int i = 0; i < N / 2; ++i) {
+            if (i < half) {
+                float send = hi ? x[i] : x[i + half];
+                float keep = hi ? x[i + half] : x[i];
+                x[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+            }
+        }
+        if (hi) base += half;
+        cnt = half;
+    }
+    return base;
+}
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, unsigned site,
+                                              volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 15u) == 15u) {
+            if (*abort_flag) return false;
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                record_timeout(site);
+                *abort_flag = 1;
+                return false;
+            }
+        }
+    }
+}
+
+template <int DK, int DV, int HG, int MODE, int CPS, int SPB>
+__global__ void __launch_bounds__(192, 1)
+    attn_packed_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
+                       const __grid_constant__ CUtensorMap mapV, const PackedParams p) {
+    using Cfg = PackedCfg<DK, DV, HG, MODE>;
+    constexpr int TOK = Cfg::TOK;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
+    uint64_t* qfull = bars + 0;
+    uint64_t* kfull = bars + 1;           // [NSK]
+    uint64_t* kempty = bars + 4;          // [NSK]
+    uint64_t* vfull = bars + 7;           // [NSV]
+    uint64_t* vempty = bars + 10;         // [NSV]
+    uint64_t* sfull = bars + 13;          // [2]
+    uint64_t* sfree = bars + 15;          // [2]
+    uint64_t* pfull = bars + 17;
+    uint64_t* pvdone = bars + 18;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 21);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int qt = p.n_qtiles - 1 - (int)blockIdx.x;   // heavy tiles first
+    const int g = blockIdx.y, b = blockIdx.z;
+    const int t0 = qt * TOK;
+    const int t_last = min(t0 + TOK, p.T) - 1;
+
+    // key range of this tile
+    int key0, ntiles;
+    if (MODE == kModeWin) {
+        int klo = max(0, t0 - p.w + 1);
+        key0 = (klo / 64) * 64;
+        ntiles = (t_last - key0) / 64 + 1;
+    } else {
+        int kend = (t_last + 1 >= p.l) ? (t_last + 1 - p.l) / p.d + 1 : 0;
+        key0 = 0;
+        ntiles = (kend + 63) / 64;
+    }
+
+    if (threadIdx.x == 0) {
+        mbar_init(qfull, 1);
+        for (int s = 0; s < 3; ++s) {
+            mbar_init(&kfull[s], 1);
+            mbar_init(&kempty[s], 1);
+            mbar_init(&vfull[s], 1);
+            mbar_init(&vempty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sfull[s], 1);
+            mbar_init(&sfree[s], 4);
+        }
+        mbar_init(pfull, 128);
+        mbar_init(pvdone, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(tmem_slot, Cfg::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 4) {
+        // ------------------------------------------------------ producer
+        if (lane == 0 && ntiles > 0) {
+            tma_prefetch_desc(&mapQ);
+            tma_prefetch_desc(&mapK);
+            if (MODE != kModeLse) tma_prefetch_desc(&mapV);
+            mbar_expect_tx(qfull, Cfg::kQBytes);
+#pragma unroll
+            for (int bx = 0; bx < Cfg::NQB; ++bx)
+                tma_load_4d(smem + Cfg::kOffQ + bx * 16384, &mapQ, qfull, bx * 64, g * HG, t0, b);
+            for (int jt = 0; jt < ntiles; ++jt) {
+                const int kb = key0 + jt * 64;
+                const int s = jt % Cfg::NSK;
+                if (jt >= Cfg::NSK &&
+                    !wait_or_abort(&kempty[s], ((jt / Cfg::NSK) - 1) & 1, 0x201, abort_flag))
+                    break;
+                uint8_t* ks = smem + Cfg::kOffK + s * Cfg::kKBytes;
+                mbar_expect_tx(&kfull[s], Cfg::kKBytes);
+#pragma unroll
+                for (int bx = 0; bx < Cfg::NQB; ++bx)
+                    tma_load_4d(ks + bx * Cfg::kKBox, &mapK, &kfull[s], bx * 64, g, kb, b);
+                if (MODE != kModeLse) {
+                    const int sv = jt % 3;
+                    if (jt >= 3 && !wait_or_abort(&vempty[sv], ((jt / 3) - 1) & 1, 0x202, abort_flag))
+                        break;
+                    uint8_t* vs = smem + Cfg::kOffV + sv * Cfg::kVBytes;
+                    mbar_expect_tx(&vfull[sv], Cfg::kVBytes);
+                    tma_load_4d(vs, &mapV, &vfull[sv], kb, 0, g, b);
+                }
+            }
+        }
+    } else if (warp == 5) {
+        // ----------------------------------------------------------- MMA
+        if (lane == 0 && ntiles > 0) {
+            constexpr uint32_t idS = idesc_bf16(128, 64);
+            constexpr uint32_t idO = idesc_bf16(128, DV);
+            const uint32_t sQ = smem_u32(smem + Cfg::kOffQ);
+            bool ok = wait_or_abort(qfull, 0, 0x203, abort_flag);
+            auto issue_S = [&](int jt) -> bool {
+                const int s = jt % Cfg::NSK, buf = jt & 1;
+                if (!wait_or_abort(&kfull[s], (jt / Cfg::NSK) & 1, 0x204, abort_flag)) return false;
+                if (jt >= 2 && !wait_or_abort(&sfree[buf], ((jt - 2) >> 1) & 1, 0x205, abort_flag))
+                    return false;
+                tc_fence_after();
+                const uint32_t sK = smem_u32(smem + Cfg::kOffK + s * Cfg::kKBytes);
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk)
+                    umma_bf16_ss(tmem + buf * 64, sdesc_sw128(sQ + (kk / 4) * 16384 + (kk % 4) * 32),
+                                 sdesc_sw128(sK + (kk / 4) * Cfg::kKBox + (kk % 4) * 32), idS,
+                                 kk > 0 ? 1u : 0u);
+                umma_commit(&sfull[buf]);
+                umma_commit(&kempty[s]);
+                return true;
+            };
+            auto issue_PV = [&](int jt) -> bool {
+                if (!wait_or_abort(pfull, jt & 1, 0x206, abort_flag)) return false;
+                const int sv = jt % 3;
+                if (!wait_or_abort(&vfull[sv], (jt / 3) & 1, 0x207, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t sP = smem_u32(smem + Cfg::kOffP);
+                const uint32_t sV = smem_u32(smem + Cfg::kOffV + sv * Cfg::kVBytes);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_bf16_ss(tmem + 128, sdesc_sw128(sP + kk * 32), sdesc_sw128(sV + kk * 32),
+                                 idO, (jt > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(pvdone);
+                umma_commit(&vempty[sv]);
+                return true;
+            };
+            if (ok) ok = issue_S(0);
+            for (int jt = 0; jt < ntiles && ok; ++jt) {
+                if (jt + 1 < ntiles) ok = issue_S(jt + 1);
+                if (ok && MODE != kModeLse) ok = issue_PV(jt);
+            }
+        }
+    } else {
+        // ------------------------------------------------ softmax / epilogue
+        const int r = threadIdx.x;
+        const int t = t0 + r / HG;
+        const int hh = r % HG;
+        const int h = g * HG + hh;
+        const bool row_ok = t < p.T;
+        const size_t rowid = ((size_t)b * p.T + (row_ok ? t : 0)) * p.H + h;
+        const uint32_t lanebase = tmem + ((uint32_t)(warp * 32) << 16);
+        // visible-key bound for this row
+        int vis_hi;   // exclusive upper bound (cmp) / inclusive t (win)
+        int vis_lo = 0;
+        if (MODE == kModeWin) {
+            vis_hi = t + 1;
+            vis_lo = t - p.w + 1;
+        } else {
+            vis_hi = (t + 1 >= p.l) ? (t + 1 - p.l) / p.d + 1 : 0;
+        }
+        if (!row_ok) vis_hi = vis_lo = -1 << 30;
+        float m_run = -INFINITY, l_run = 0.f;
+        float lse2 = -INFINITY;
+        if (MODE == kModeCmp && row_ok) lse2 = p.lse_cmp[rowid] * kLog2e;
+        constexpr int NB = 64 / SPB;                        // complete blocks per tile
+        constexpr int NJ = (63 + CPS - 1) / SPB + 1;        // partial blocks touched per tile
+        constexpr int NC = NJ - NB;                         // carried into the next tile
+        float carry[NC > 0 ? NC : 1];
+#pragma unroll
+        for (int c = 0; c < (NC > 0 ? NC : 1); ++c) carry[c] = 0.f;
+        bool ok = true;
+
+        for (int jt = 0; jt < ntiles; ++jt) {
+            const int buf = jt & 1;
+            const int kb = key0 + jt * 64;
+            if (ok) ok = wait_or_abort(&sfull[buf], (jt >> 1) & 1, 0x208, abort_flag);
+            tc_fence_after();
+            uint32_t ra[32], rb[32];
+            tmem_ld32(lanebase + buf * 64, ra);
+            tmem_ld32(lanebase + buf * 64 + 32, rb);
+            tmem_wait_ld32(ra);
+            tmem_wait_ld32(rb);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sfree[buf]);
+            float s[64];
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                s[k] = __uint_as_float(ra[k]) * p.scale_log2;
+                s[k + 32] = __uint_as_float(rb[k]) * p.scale_log2;
+            }
+#pragma unroll
+            for (int k = 0; k < 64; ++k) {
+                const int key = kb + k;
+                if (!(key >= vis_lo && key < vis_hi)) s[k] = -INFINITY;
+            }
+            if (MODE == kModeLse) {
+                float mt = -INFINITY;
+#pragma unroll
+                for (int k = 0; k < 64; ++k) mt = fmaxf(mt, s[k]);
+                const float mn = fmaxf(m_run, mt);
+                if (mn != -INFINITY) {
+                    float acc = 0.f;
+#pragma unroll
+                    for (int k = 0; k < 64; ++k) acc += exp2f(s[k] - mn);
+                    l_run = l_run * exp2f(m_run - mn) + acc;
+                    m_run = mn;
+                }
+                continue;
+            }
+            float pr[64];
+            float alpha = 1.f;
+            bool need_rescale = false;
+            if (MODE == kModeCmp) {
+#pragma unroll
+                for (int k = 0; k < 64; ++k) pr[k] = (s[k] == -INFINITY) ? 0.f : exp2f(s[k] - lse2);
+            } else {
+                float mt = -INFINITY;
+#pragma unroll
+                for (int k = 0; k < 64; ++k) mt = fmaxf(mt, s[k]);
+                if (mt > m_run + 8.f) {
+                    const float mn = mt;
+                    alpha = exp2f(m_run - mn);       // 0 when m_run = -inf
+                    l_run *= alpha;
+                    m_run = mn;
+                    need_rescale = true;
+                }
+                float acc = 0.f;
+#pragma unroll
+                for (int k = 0; k < 64; ++k) {
+                    pr[k] = (s[k] == -INFINITY) ? 0.f : exp2f(s[k] - m_run);
+                    acc += pr[k];
+                }
+                l_run += acc;
+            }
+            if (MODE == kModeCmp) {
+                // importance scores of selection blocks kb/SPB .. kb/SPB + NB - 1
+                float part[NJ];
+#pragma unroll
+                for (int m = 0; m < NJ; ++m) part[m] = 0.f;
+#pragma unroll
+                for (int c = 0; c < NC; ++c) part[c] += carry[c];
+#pragma unroll
+                for (int k = 0; k < 64; ++k)
+#pragma unroll
+                    for (int u = 0; u < CPS; ++u) part[(k + u) / SPB] += pr[k];
+#pragma unroll
+                for (int c = 0; c < NC; ++c) carry[c] = part[NB + c];
+                float red[NB];
+#pragma unroll
+                for (int m = 0; m < NB; ++m) red[m] = part[m];
+                const int base = reduce_scatter_heads<NB, HG>(red, lane);
+                if (row_ok) {
+                    const int j0 = kb / SPB;
+                    float* dst = p.pscore + (((size_t)b * p.T + t) * p.G + g) * p.NSp;
+#pragma unroll
+                    for (int v = 0; v < NB / HG; ++v)
+                        if (j0 + base + v < p.NSp) dst[j0 + base + v] = red[v];
+                }
+            }
+            // P -> shared memory (after the previous P.V has consumed it)
+            if (jt > 0 && ok) ok = wait_or_abort(pvdone, (jt - 1) & 1, 0x209, abort_flag);
+            tc_fence_after();
+            if (MODE == kModeWin && jt > 0 && __any_sync(0xffffffffu, need_rescale)) {
+                const float a = need_rescale ? alpha : 1.f;
+#pragma unroll 1
+                for (int c0 = 0; c0 < DV; c0 += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(lanebase + 128 + c0, o);
+                    tmem_wait_ld32(o);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * a);
+                    tmem_st32(lanebase + 128 + c0, o);
+                }
+                tmem_wait_st();
+            }
+            const uint32_t sP = smem_u32(smem + Cfg::kOffP);
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                st_shared_v4(sP + sw128_off(r, c), pack_bf16x2(pr[8 * c + 0], pr[8 * c + 1]),
+                             pack_bf16x2(pr[8 * c + 2], pr[8 * c + 3]),
+                             pack_bf16x2(pr[8 * c + 4], pr[8 * c + 5]),
+                             pack_bf16x2(pr[8 * c + 6], pr[8 * c + 7]));
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(pfull);
+        }
+
+        // ------------------------------------------------------- epilogue
+        if (MODE == kModeLse) {
+            if (row_ok) {
+                const float lse = (l_run > 0.f) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+                p.lse_cmp[rowid] = lse;
+                if (p.lse_user) p.lse_user[rowid * 3 + 0] = lse;
+            }
+        } else {
+            if (MODE == kModeCmp && NC > 0) {
+                // flush the carried partial scores of the block after the last tile
+                const int jn = (key0 + ntiles * 64) / SPB;
+#pragma unroll
+                for (int c = 0; c < (NC > 0 ? NC : 1); ++c) {
+                    float v = carry[c];
+#pragma unroll
+                    for (int m = HG / 2; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+                    if (row_ok && hh == 0 && ntiles > 0 && jn + c < p.NSp)
+                        p.pscore[(((size_t)b * p.T + t) * p.G + g) * p.NSp + jn + c] = v;
+                }
+            }
+            if (ntiles > 0 && ok) ok = wait_or_abort(pvdone, (ntiles - 1) & 1, 0x20A, abort_flag);
+            tc_fence_after();
+            const float gate = row_ok ? p.gates[rowid * 3 + (MODE == kModeCmp ? 0 : 2)] : 0.f;
+            const float inv = (MODE == kModeWin) ? (l_run > 0.f ? 1.f / l_run : 0.f) : 1.f;
+#pragma unroll 1
+            for (int c0 = 0; c0 < DV; c0 += 32) {
+                uint32_t o[32];
+                if (ntiles > 0) {
+                    tmem_ld32(lanebase + 128 + c0, o);
+                    tmem_wait_ld32(o);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = 0u;
+                }
+                if (row_ok && ok) {
+                    float4* dst = reinterpret_cast<float4*>(p.out + rowid * DV + c0);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        float4 v;
+                        v.x = gate * __uint_as_float(o[4 * e + 0]) * inv;
+                        v.y = gate * __uint_as_float(o[4 * e + 1]) * inv;
+                        v.z = gate * __uint_as_float(o[4 * e + 2]) * inv;
+                        v.w = gate * __uint_as_float(o[4 * e + 3]) * inv;
+                        if (MODE == kModeWin) {
+                            float4 prev = dst[e];
+                            v.x += prev.x;
+                            v.y += prev.y;
+                            v.z += prev.z;
+                            v.w += prev.w;
+                        }
+                        dst[e] = v;
+                    }
+                }
+            }
+            if (MODE == kModeWin && row_ok && p.lse_user)
+                p.lse_user[rowid * 3 + 2] = (m_run + log2f(l_run)) * kLn2;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, Cfg::kTmemCols);
+    }
+}
+
+}  // namespace nsa

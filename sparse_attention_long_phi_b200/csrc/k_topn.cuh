@@ -1,0 +1,99 @@
+// k_topn.cuh -- top-n block selection (page "硬件对齐+原生训练！DeepSeek NSA打造高效
+// 稀疏Attention", Top-n 块选择; hyperparameter paragraph: 1 initial + 2 local
+// blocks always active).
+//
+// One warp per (batch, token, group).  Candidates are the selection blocks
+// 0 .. b_t = floor(t/l').  With at most n candidates all are taken.
+// Otherwise blocks 0..fi-1 and b_t-fl+1..b_t are kept and the remaining
+// n - fi - fl are the highest importance scores among the other candidates,
+// ties to the lower block index (decision taken on the fp32 scores).  The
+// output row is ascending and padded with -1.
+#pragma once
+#include "nsa_dev.cuh"
+
+namespace nsa {
+
+constexpr int kTopnPerLane = 64;   // up to 2048 scored candidates per row
+
+__device__ __forceinline__ int warp_sort_asc(int v, int lane) {
+    // bitonic sort of one int per lane across the warp, ascending by lane
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            int o = __shfl_xor_sync(0xffffffffu, v, j);
+            bool up = ((lane & k) == 0);
+            bool lower = ((lane & j) == 0);
+            int mn = min(v, o), mx = max(v, o);
+            v = (lower == up) ? mn : mx;
+        }
+    }
+    return v;
+}
+
+// Top-n of one row of importance scores `row` (global or shared memory) for
+// query t, by one warp; writes n ascending indices (-1 padded) to `out`.
+__device__ __forceinline__ void topn_row_warp(const float* row, int t, int n, int lp, int fi, int fl,
+                                              int32_t* out, int lane) {
+    const int bt = t / lp;
+    const int ncand = bt + 1;
+    if (ncand <= n) {
+        if (lane < n) out[lane] = lane < ncand ? lane : -1;
+        return;
+    }
+    const int lo = fi, hi = bt - fl;             // scored candidates lo..hi
+    const int R = n - fi - fl;
+    float v[kTopnPerLane];
+#pragma unroll
+    for (int k = 0; k < kTopnPerLane; ++k) {
+        const int j = lo + lane + 32 * k;
+        v[k] = (j <= hi) ? row[j] : -1.f;        // scores are >= 0
+    }
+    int mine = 0x7fffffff;
+    for (int it = 0; it < R; ++it) {
+        float bv = -2.f;
+        int bk = 0;
+#pragma unroll
+        for (int k = 0; k < kTopnPerLane; ++k)
+            if (v[k] > bv) {                     // strict: first (lowest j) wins ties
+                bv = v[k];
+                bk = k;
+            }
+        int bj = lo + lane + 32 * bk;
+        if (bv < -0.5f) bj = 0x7fffffff;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+            if (ov > bv || (ov == bv && oj < bj)) {
+                bv = ov;
+                bj = oj;
+            }
+        }
+        if (bj != 0x7fffffff && ((bj - lo) & 31) == lane) {
+            const int kk = (bj - lo) >> 5;
+#pragma unroll
+            for (int k = 0; k < kTopnPerLane; ++k)
+                if (k == kk) v[k] = -1.f;
+        }
+        if (lane == it) mine = bj;
+    }
+    // lanes R .. R+fi+fl-1 carry the forced blocks
+    if (lane >= R && lane < R + fi) mine = lane - R;
+    if (lane >= R + fi && lane < R + fi + fl) mine = bt - fl + 1 + (lane - R - fi);
+    const int srt = warp_sort_asc(mine, lane);
+    if (lane < n) out[lane] = (srt == 0x7fffffff) ? -1 : srt;
+}
+
+// one warp per (batch, token, group) item; scores [items, NSp]
+__global__ void __launch_bounds__(256)
+    topn_kernel(const float* __restrict__ pscore, long long items, int T, int G, int NSp, int n,
+                int lp, int fi, int fl, int32_t* __restrict__ idx) {
+    const int lane = threadIdx.x & 31;
+    const long long item = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (item >= items) return;
+    const int t = (int)((item / G) % T);
+    topn_row_warp(pscore + item * NSp, t, n, lp, fi, fl, idx + item * n, lane);
+}
+
+}  // namespace nsa

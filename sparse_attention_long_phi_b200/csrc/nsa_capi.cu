@@ -1,0 +1,699 @@
+// nsa_capi.cu -- libnsa: the C ABI declared in include/nsa.h.
+//
+// Host side only: argument validation, workspace carving, TMA descriptor
+// encoding and kernel launches on the caller's stream.  Every step of the
+// operator runs in the kernels included below; nothing here touches tensor
+// data.  The whole library is one translation unit so that the device error
+// word is shared by every kernel.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/nsa.h"
+#include "k_attn_packed.cuh"
+#include "k_attn_sel.cuh"
+#include "k_decode.cuh"
+#include "k_backward.cuh"
+#include "k_phi.cuh"
+#include "k_topn.cuh"
+
+using namespace nsa;
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool encode_fn() {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode != nullptr;
+}
+
+// bf16 tiled map with 128-byte swizzle (box inner extent must be 64 elements)
+bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+              const uint64_t* strides, const uint32_t* box) {
+    if (!encode_fn()) return false;
+    cuuint64_t gd[5], gs[4];
+    cuuint32_t bx[5], es[5];
+    for (int i = 0; i < rank; ++i) {
+        gd[i] = dims[i];
+        bx[i] = box[i];
+        es[i] = 1;
+        if (i < rank - 1) gs[i] = strides[i];
+    }
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
+                          gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+struct Shape {
+    int64_t B, T, H, G, DK, DV, HG, l, d, lp, n, fi, fl, w;
+    int64_t C, Cp, Tp, DVP, NS, NSp;
+    int phi;
+    float scale;
+};
+
+nsa_status_t derive(const nsa_config_t* c, Shape& s) {
+    if (!c) return NSA_ERR_INVALID_ARG;
+    s.B = c->batch;
+    s.T = c->seqlen;
+    s.H = c->num_q_heads;
+    s.G = c->num_kv_groups;
+    s.DK = c->d_k;
+    s.DV = c->d_v;
+    s.l = c->cmp_block;
+    s.d = c->cmp_stride;
+    s.lp = c->sel_block;
+    s.n = c->sel_count;
+    s.fi = c->forced_initial;
+    s.fl = c->forced_local;
+    s.w = c->window;
+    s.phi = c->phi;
+    if (s.B <= 0 || s.T <= 0 || s.H <= 0 || s.G <= 0 || s.DK <= 0 || s.DV <= 0) return NSA_ERR_INVALID_ARG;
+    if (s.H % s.G) return NSA_ERR_INVALID_ARG;
+    if (s.l <= 0 || s.d <= 0 || s.lp <= 0 || s.w <= 0 || s.n <= 0) return NSA_ERR_INVALID_ARG;
+    if (s.l % s.d || s.lp % s.d || s.l > s.lp) return NSA_ERR_INVALID_ARG;
+    if (s.fi < 0 || s.fl < 0 || s.n < s.fi + s.fl) return NSA_ERR_INVALID_ARG;
+    if (c->phi != NSA_PHI_MEAN && c->phi != NSA_PHI_LINEAR) return NSA_ERR_INVALID_ARG;
+    if (c->score_map != 0 && c->score_map != 1) return NSA_ERR_INVALID_ARG;
+    if (!(c->scale >= 0.f)) return NSA_ERR_INVALID_ARG;
+    s.HG = s.H / s.G;
+    s.scale = c->scale > 0.f ? c->scale : 1.0f / std::sqrt((float)s.DK);
+    s.C = s.T >= s.l ? (s.T - s.l) / s.d + 1 : 0;
+    s.Cp = ceil_div(std::max<int64_t>(s.C, 1), 8) * 8;
+    s.Tp = ceil_div(s.T, 8) * 8;
+    s.DVP = std::max<int64_t>(s.DV, 128);
+    s.NS = ceil_div(s.T, s.lp);
+    s.NSp = ceil_div(s.NS, 4) * 4;
+    return NSA_OK;
+}
+
+// kernels exist for these sizes only
+nsa_status_t supported(const Shape& s) {
+    const bool dims = (s.DK == 64 && s.DV == 64 && s.HG == 4) || (s.DK == 192 && s.DV == 128 && s.HG == 16);
+    if (!dims) return NSA_ERR_UNSUPPORTED;
+    if (s.lp != 64 || s.n > 16) return NSA_ERR_UNSUPPORTED;
+    const int64_t cps = s.l / s.d, spb = s.lp / s.d;
+    const bool blk = (cps == 2 && spb == 4) || (cps == 1 && spb == 1) || (cps == 1 && spb == 4) ||
+                     (cps == 2 && spb == 2);
+    if (!blk) return NSA_ERR_UNSUPPORTED;
+    if (s.T > 131072 || s.B * s.T * s.H > (int64_t)1 << 31) return NSA_ERR_UNSUPPORTED;
+    return NSA_OK;
+}
+
+struct FwdWs {
+    size_t off_kc, off_vct, off_vt, off_bias, off_lse, off_ps, off_fix, total;
+};
+
+// phi fix-up list: two counters (K, V), then one entry per K~ and V~ element
+inline size_t fix_bytes(const Shape& s) {
+    return 256 + (size_t)s.B * std::max<int64_t>(s.C, 1) * s.G * (s.DK + s.DV) * 4;
+}
+
+FwdWs fwd_layout(const Shape& s) {
+    FwdWs w{};
+    size_t o = 0;
+    w.off_kc = o;
+    o = align256(o + (size_t)s.B * std::max<int64_t>(s.C, 1) * s.G * s.DK * 2);
+    w.off_vct = o;
+    o = align256(o + (size_t)s.B * s.G * s.DV * s.Cp * 2);
+    w.off_vt = o;
+    o = align256(o + (size_t)s.B * s.G * s.DVP * s.Tp * 2);
+    w.off_bias = o;
+    o = align256(o + (size_t)(s.DK + s.DV) * 4);
+    w.off_lse = o;
+    o = align256(o + (size_t)s.B * s.T * s.H * 4);
+    w.off_ps = o;
+    o = align256(o + (size_t)s.B * s.T * s.G * s.NSp * 4);
+    w.off_fix = o;
+    o = align256(o + fix_bytes(s));
+    w.total = o;
+    return w;
+}
+
+inline nsa_status_t last_launch() {
+    return cudaGetLastError() == cudaSuccess ? NSA_OK : NSA_ERR_CUDA;
+}
+
+#define NSA_TRY(x)                              \
+    do {                                        \
+        nsa_status_t _st = (x);                 \
+        if (_st != NSA_OK) return _st;          \
+    } while (0)
+
+template <typename K>
+nsa_status_t set_smem(K kernel, int bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+                   cudaSuccess
+               ? NSA_OK
+               : NSA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------- phi
+template <int D>
+nsa_status_t launch_phi_linear(const Shape& s, const void* x, const void* W, const void* E,
+                               const float* bias, void* y, void* yT, uint32_t* fix_list,
+                               unsigned int* fix_count, cudaStream_t st) {
+    CUtensorMap mA, mW;
+    const uint64_t dA[5] = {(uint64_t)D, (uint64_t)s.G, (uint64_t)s.d, (uint64_t)(s.T / s.d), (uint64_t)s.B};
+    const uint64_t sA[4] = {(uint64_t)D * 2, (uint64_t)s.G * D * 2, (uint64_t)s.d * s.G * D * 2,
+                            (uint64_t)s.T * s.G * D * 2};
+    const uint32_t bA[5] = {64, 1, 1, 128, 1};
+    const uint64_t dW[2] = {(uint64_t)s.l * D, (uint64_t)D};
+    const uint64_t sW[1] = {(uint64_t)s.l * D * 2};
+    const uint32_t bW[2] = {64, (uint32_t)D};
+    if (!make_map(&mA, x, 5, dA, sA, bA) || !make_map(&mW, W, 2, dW, sW, bW)) return NSA_ERR_CUDA;
+    NSA_TRY(set_smem(phi_linear_kernel<D>, PhiGemmCfg<D>::kSmem));
+    dim3 grid((unsigned)ceil_div(s.C, 128), (unsigned)s.G, (unsigned)s.B);
+    phi_linear_kernel<D><<<grid, 192, PhiGemmCfg<D>::kSmem, st>>>(
+        mA, mW, bias, (int)s.l, (int)s.d, (int)s.C, (int)s.Cp, (int)s.G,
+        reinterpret_cast<__nv_bfloat16*>(y), reinterpret_cast<__nv_bfloat16*>(yT), fix_list, fix_count);
+    NSA_TRY(last_launch());
+    phi_fixup_kernel<D><<<148 * 4, 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(x), reinterpret_cast<const __nv_bfloat16*>(W),
+        reinterpret_cast<const __nv_bfloat16*>(E), (int)s.T, (int)s.G, (int)s.l, (int)s.d, (int)s.C,
+        (int)s.Cp, fix_list, fix_count, reinterpret_cast<__nv_bfloat16*>(y),
+        reinterpret_cast<__nv_bfloat16*>(yT));
+    return last_launch();
+}
+
+// K~ -> kc [B,C,G,DK]; V~ -> vcT [B,G,DV,Cp] (+ vc [B,C,G,DV] if given)
+nsa_status_t run_phi(const Shape& s, const void* k, const void* v, const nsa_phi_params_t* phi,
+                     void* kc, void* vc, void* vcT, float* bias, uint8_t* fix, cudaStream_t st) {
+    if (s.C == 0) return NSA_OK;
+    if (s.phi == NSA_PHI_MEAN) {
+        dim3 grid((unsigned)s.C, (unsigned)s.G, (unsigned)s.B);
+        phi_mean_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(k), (int)s.T,
+                                              (int)s.G, (int)s.DK, (int)s.l, (int)s.d, (int)s.C,
+                                              (int)s.Cp, reinterpret_cast<__nv_bfloat16*>(kc), nullptr);
+        NSA_TRY(last_launch());
+        phi_mean_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(v), (int)s.T,
+                                              (int)s.G, (int)s.DV, (int)s.l, (int)s.d, (int)s.C,
+                                              (int)s.Cp, reinterpret_cast<__nv_bfloat16*>(vc),
+                                              reinterpret_cast<__nv_bfloat16*>(vcT));
+        return last_launch();
+    }
+    if (!phi || !phi->w_k || !phi->e_k || !phi->w_v || !phi->e_v) return NSA_ERR_INVALID_ARG;
+    if (!aligned16(phi->w_k) || !aligned16(phi->w_v)) return NSA_ERR_INVALID_ARG;
+    phi_bias_kernel<<<(unsigned)s.DK, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(phi->w_k),
+                                                    reinterpret_cast<const __nv_bfloat16*>(phi->e_k),
+                                                    (int)(s.l * s.DK), bias);
+    NSA_TRY(last_launch());
+    phi_bias_kernel<<<(unsigned)s.DV, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(phi->w_v),
+                                                    reinterpret_cast<const __nv_bfloat16*>(phi->e_v),
+                                                    (int)(s.l * s.DV), bias + s.DK);
+    NSA_TRY(last_launch());
+    unsigned int* cnt = reinterpret_cast<unsigned int*>(fix);
+    uint32_t* lk = reinterpret_cast<uint32_t*>(fix + 256);
+    uint32_t* lv = lk + (size_t)s.B * s.C * s.G * s.DK;
+    if (cudaMemsetAsync(cnt, 0, 8, st) != cudaSuccess) return NSA_ERR_CUDA;
+    if (s.DK == 192) {
+        NSA_TRY(launch_phi_linear<192>(s, k, phi->w_k, phi->e_k, bias, kc, nullptr, lk, cnt, st));
+        return launch_phi_linear<128>(s, v, phi->w_v, phi->e_v, bias + s.DK, vc, vcT, lv, cnt + 1, st);
+    }
+    NSA_TRY(launch_phi_linear<64>(s, k, phi->w_k, phi->e_k, bias, kc, nullptr, lk, cnt, st));
+    return launch_phi_linear<64>(s, v, phi->w_v, phi->e_v, bias + s.DK, vc, vcT, lv, cnt + 1, st);
+}
+
+__global__ void cmp_empty_kernel(float* out, float* lse, long long rows, int DV) {
+    long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < rows * DV) out[i] = 0.f;
+    if (lse && i < rows) lse[i * 3] = -INFINITY;
+}
+
+// ----------------------------------------------------------- attention
+template <int DK, int DV, int HG, int MODE, int CPS, int SPB>
+nsa_status_t launch_packed(const Shape& s, const CUtensorMap& mQ, const CUtensorMap& mK,
+                           const CUtensorMap& mV, const PackedParams& p, cudaStream_t st) {
+    using Cfg = PackedCfg<DK, DV, HG, MODE>;
+    auto kern = attn_packed_kernel<DK, DV, HG, MODE, CPS, SPB>;
+    NSA_TRY(set_smem(kern, Cfg::kSmem));
+    dim3 grid((unsigned)p.n_qtiles, (unsigned)s.G, (unsigned)s.B);
+    kern<<<grid, 192, Cfg::kSmem, st>>>(mQ, mK, mV, p);
+    return last_launch();
+}
+
+template <int DK, int DV, int HG, int MODE>
+nsa_status_t launch_packed_blk(const Shape& s, const CUtensorMap& mQ, const CUtensorMap& mK,
+                               const CUtensorMap& mV, const PackedParams& p, cudaStream_t st) {
+    const int64_t cps = s.l / s.d, spb = s.lp / s.d;
+    if (MODE != kModeCmp) return launch_packed<DK, DV, HG, MODE, 2, 4>(s, mQ, mK, mV, p, st);
+    if (cps == 2 && spb == 4) return launch_packed<DK, DV, HG, MODE, 2, 4>(s, mQ, mK, mV, p, st);
+    if (cps == 1 && spb == 1) return launch_packed<DK, DV, HG, MODE, 1, 1>(s, mQ, mK, mV, p, st);
+    if (cps == 1 && spb == 4) return launch_packed<DK, DV, HG, MODE, 1, 4>(s, mQ, mK, mV, p, st);
+    if (cps == 2 && spb == 2) return launch_packed<DK, DV, HG, MODE, 2, 2>(s, mQ, mK, mV, p, st);
+    return NSA_ERR_UNSUPPORTED;
+}
+
+template <int DK, int DV, int HG>
+nsa_status_t forward_impl(const Shape& s, const void* q, const void* k, const void* v,
+                          const float* gates, const nsa_phi_params_t* phi, float* out,
+                          int32_t* sel_idx, float* lse, void* kc_out, void* vc_out, uint8_t* ws,
+                          cudaStream_t st) {
+    const FwdWs L = fwd_layout(s);
+    void* kc = kc_out ? kc_out : ws + L.off_kc;
+    void* vcT = ws + L.off_vct;
+    void* vT = ws + L.off_vt;
+    float* bias = reinterpret_cast<float*>(ws + L.off_bias);
+    float* lse_cmp = reinterpret_cast<float*>(ws + L.off_lse);
+    float* pscore = reinterpret_cast<float*>(ws + L.off_ps);
+
+    // 1. token compression
+    NSA_TRY(run_phi(s, k, v, phi, kc, vc_out, vcT, bias, ws + L.off_fix, st));
+    // 2. v transposed for the P.V products of the selected and window branches
+    {
+        dim3 grid((unsigned)ceil_div(s.Tp, 64), (unsigned)s.G, (unsigned)s.B);
+        transpose_v_kernel<<<grid, dim3(64, 4), 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(v),
+                                                         (int)s.T, (int)s.G, (int)s.DV, (int)s.DVP,
+                                                         (int)s.Tp, reinterpret_cast<__nv_bfloat16*>(vT));
+        NSA_TRY(last_launch());
+    }
+    // tensor maps
+    CUtensorMap mQ, mQs, mKc, mVc, mK, mVT, mVTs;
+    {
+        const uint64_t dQ[4] = {(uint64_t)s.DK, (uint64_t)s.H, (uint64_t)s.T, (uint64_t)s.B};
+        const uint64_t sQ[3] = {(uint64_t)s.DK * 2, (uint64_t)s.H * s.DK * 2, (uint64_t)s.T * s.H * s.DK * 2};
+        const uint32_t bQ[4] = {64, (uint32_t)HG, (uint32_t)(128 / HG), 1};
+        const uint32_t bQs[4] = {64, 16, 1, 1};
+        const uint64_t dK[4] = {(uint64_t)s.DK, (uint64_t)s.G, (uint64_t)s.T, (uint64_t)s.B};
+        const uint64_t sK[3] = {(uint64_t)s.DK * 2, (uint64_t)s.G * s.DK * 2, (uint64_t)s.T * s.G * s.DK * 2};
+        const uint32_t bK[4] = {64, 1, 64, 1};
+        const uint64_t dVT[4] = {(uint64_t)s.T, (uint64_t)s.DVP, (uint64_t)s.G, (uint64_t)s.B};
+        const uint64_t sVT[3] = {(uint64_t)s.Tp * 2, (uint64_t)s.DVP * s.Tp * 2, (uint64_t)s.G * s.DVP * s.Tp * 2};
+        const uint32_t bVT[4] = {64, (uint32_t)s.DV, 1, 1};
+        const uint32_t bVTs[4] = {64, 128, 1, 1};
+        if (!make_map(&mQ, q, 4, dQ, sQ, bQ) || !make_map(&mQs, q, 4, dQ, sQ, bQs) ||
+            !make_map(&mK, k, 4, dK, sK, bK) || !make_map(&mVT, vT, 4, dVT, sVT, bVT) ||
+            !make_map(&mVTs, vT, 4, dVT, sVT, bVTs))
+            return NSA_ERR_CUDA;
+        if (s.C > 0) {
+            const uint64_t dKc[4] = {(uint64_t)s.DK, (uint64_t)s.G, (uint64_t)s.C, (uint64_t)s.B};
+            const uint64_t sKc[3] = {(uint64_t)s.DK * 2, (uint64_t)s.G * s.DK * 2, (uint64_t)s.C * s.G * s.DK * 2};
+            const uint64_t dVc[4] = {(uint64_t)s.C, (uint64_t)s.DV, (uint64_t)s.G, (uint64_t)s.B};
+            const uint64_t sVc[3] = {(uint64_t)s.Cp * 2, (uint64_t)s.DV * s.Cp * 2, (uint64_t)s.G * s.DV * s.Cp * 2};
+            const uint32_t bVc[4] = {64, (uint32_t)s.DV, 1, 1};
+            if (!make_map(&mKc, kc, 4, dKc, sKc, bK) || !make_map(&mVc, vcT, 4, dVc, sVc, bVc))
+                return NSA_ERR_CUDA;
+        }
+    }
+    PackedParams pp{};
+    pp.B = (int)s.B;
+    pp.T = (int)s.T;
+    pp.H = (int)s.H;
+    pp.G = (int)s.G;
+    pp.l = (int)s.l;
+    pp.d = (int)s.d;
+    pp.lp = (int)s.lp;
+    pp.w = (int)s.w;
+    pp.scale_log2 = s.scale * kLog2e;
+    pp.gates = gates;
+    pp.out = out;
+    pp.lse_user = lse;
+    pp.lse_cmp = lse_cmp;
+    pp.pscore = pscore;
+    pp.NSp = (int)s.NSp;
+    pp.n_qtiles = (int)ceil_div(s.T, 128 / HG);
+    // 3-4. compressed attention: LSE pass, then P.V~ with importance scores
+    if (s.C > 0) {
+        NSA_TRY((launch_packed_blk<DK, DV, HG, kModeLse>(s, mQ, mKc, mVc, pp, st)));
+        NSA_TRY((launch_packed_blk<DK, DV, HG, kModeCmp>(s, mQ, mKc, mVc, pp, st)));
+    } else {
+        const long long rows = s.B * s.T * s.H;
+        cmp_empty_kernel<<<(unsigned)ceil_div(rows * s.DV, 256), 256, 0, st>>>(out, lse, rows, (int)s.DV);
+        NSA_TRY(last_launch());
+    }
+    // 5. top-n selection
+    {
+        const long long items = s.B * s.T * s.G;
+        topn_kernel<<<(unsigned)ceil_div(items, 8), 256, 0, st>>>(pscore, items, (int)s.T, (int)s.G,
+                                                                   (int)s.NSp, (int)s.n, (int)s.lp,
+                                                                   (int)s.fi, (int)s.fl, sel_idx);
+        NSA_TRY(last_launch());
+    }
+    // 6. selected attention
+    {
+        SelParams sp{};
+        sp.B = (int)s.B;
+        sp.T = (int)s.T;
+        sp.H = (int)s.H;
+        sp.G = (int)s.G;
+        sp.n = (int)s.n;
+        sp.scale_log2 = s.scale * kLog2e;
+        sp.idx = sel_idx;
+        sp.gates = gates;
+        sp.out = out;
+        sp.lse_user = lse;
+        int64_t tpc = (s.B * s.T * s.G) / (148 * 8);
+        sp.tpc = (int)std::min<int64_t>(64, std::max<int64_t>(4, tpc));
+        using Cfg = SelCfg<DK, DV>;
+        NSA_TRY(set_smem(attn_sel_kernel<DK, DV>, Cfg::kSmem));
+        dim3 grid((unsigned)ceil_div(s.T, sp.tpc), (unsigned)s.G, (unsigned)s.B);
+        attn_sel_kernel<DK, DV><<<grid, 192, Cfg::kSmem, st>>>(mQs, mK, mVTs, sp);
+        NSA_TRY(last_launch());
+    }
+    // 7. sliding window
+    NSA_TRY((launch_packed_blk<DK, DV, HG, kModeWin>(s, mQ, mK, mVT, pp, st)));
+    return NSA_OK;
+}
+
+
+// -------------------------------------------------------------- backward
+struct BwdWs {
+    size_t off_kc, off_vc, off_vct, off_bias, off_lse2, off_dlt, off_dkc, off_dvc, off_cnt,
+        off_cur, off_off, off_choff, off_list, off_fix, total;
+};
+
+BwdWs bwd_layout(const Shape& s) {
+    BwdWs w{};
+    const int64_t C1 = std::max<int64_t>(s.C, 1);
+    const int64_t NE = s.B * s.G * s.NS;
+    size_t o = 0;
+    w.off_kc = o;
+    o = align256(o + (size_t)s.B * C1 * s.G * s.DK * 2);
+    w.off_vc = o;
+    o = align256(o + (size_t)s.B * C1 * s.G * s.DV * 2);
+    w.off_vct = o;
+    o = align256(o + (size_t)s.B * s.G * s.DV * s.Cp * 2);
+    w.off_bias = o;
+    o = align256(o + (size_t)(s.DK + s.DV) * 4);
+    w.off_lse2 = o;
+    o = align256(o + (size_t)s.B * s.T * s.H * 3 * 4);
+    w.off_dlt = o;
+    o = align256(o + (size_t)s.B * s.T * s.H * 3 * 4);
+    w.off_dkc = o;
+    o = align256(o + (size_t)s.B * C1 * s.G * s.DK * 4);
+    w.off_dvc = o;
+    o = align256(o + (size_t)s.B * C1 * s.G * s.DV * 4);
+    w.off_cnt = o;
+    o = align256(o + (size_t)NE * 4);
+    w.off_cur = o;
+    o = align256(o + (size_t)NE * 4);
+    w.off_off = o;
+    o = align256(o + (size_t)(NE + 1) * 4);
+    w.off_choff = o;
+    o = align256(o + (size_t)(NE + 1) * 4);
+    w.off_list = o;
+    o = align256(o + (size_t)s.B * s.T * s.G * s.n * 4);
+    w.off_fix = o;
+    o = align256(o + fix_bytes(s));
+    w.total = o;
+    return w;
+}
+
+template <int DK, int DV>
+nsa_status_t backward_impl(const Shape& s, const void* q, const void* k, const void* v,
+                           const float* gates, const nsa_phi_params_t* phi, const void* dout,
+                           const int32_t* sel_idx, float* dq, float* dk, float* dv, float* dgates,
+                           uint8_t* ws, cudaStream_t st) {
+    const BwdWs L = bwd_layout(s);
+    const int64_t NE = s.B * s.G * s.NS;
+    BwdParams p{};
+    p.B = (int)s.B;
+    p.T = (int)s.T;
+    p.H = (int)s.H;
+    p.G = (int)s.G;
+    p.HG = (int)s.HG;
+    p.DK = DK;
+    p.DV = DV;
+    p.l = (int)s.l;
+    p.d = (int)s.d;
+    p.lp = (int)s.lp;
+    p.n = (int)s.n;
+    p.w = (int)s.w;
+    p.C = (int)s.C;
+    p.NSb = (int)s.NS;
+    p.scale = s.scale;
+    p.scale_log2 = s.scale * kLog2e;
+    p.q = reinterpret_cast<const __nv_bfloat16*>(q);
+    p.k = reinterpret_cast<const __nv_bfloat16*>(k);
+    p.v = reinterpret_cast<const __nv_bfloat16*>(v);
+    p.kc = reinterpret_cast<const __nv_bfloat16*>(ws + L.off_kc);
+    p.vc = reinterpret_cast<const __nv_bfloat16*>(ws + L.off_vc);
+    p.dout = reinterpret_cast<const __nv_bfloat16*>(dout);
+    p.wk = phi ? reinterpret_cast<const __nv_bfloat16*>(phi->w_k) : nullptr;
+    p.wv = phi ? reinterpret_cast<const __nv_bfloat16*>(phi->w_v) : nullptr;
+    p.gates = gates;
+    p.idx = sel_idx;
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dv;
+    p.dgates = dgates;
+    p.lse2 = reinterpret_cast<float*>(ws + L.off_lse2);
+    p.dlt = reinterpret_cast<float*>(ws + L.off_dlt);
+    p.dkc = reinterpret_cast<float*>(ws + L.off_dkc);
+    p.dvc = reinterpret_cast<float*>(ws + L.off_dvc);
+    p.cnt = reinterpret_cast<int*>(ws + L.off_cnt);
+    p.cursor = reinterpret_cast<int*>(ws + L.off_cur);
+    p.off = reinterpret_cast<int*>(ws + L.off_off);
+    p.chunk_off = reinterpret_cast<int*>(ws + L.off_choff);
+    p.list = reinterpret_cast<int*>(ws + L.off_list);
+    p.phi = s.phi;
+
+    // compressed keys/values of the forward (row layout)
+    NSA_TRY(run_phi(s, k, v, phi, ws + L.off_kc, ws + L.off_vc, ws + L.off_vct,
+                    reinterpret_cast<float*>(ws + L.off_bias), ws + L.off_fix, st));
+    if (cudaMemsetAsync(dk, 0, (size_t)s.B * s.T * s.G * DK * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(dv, 0, (size_t)s.B * s.T * s.G * DV * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(ws + L.off_dkc, 0, L.off_cnt - L.off_dkc, st) != cudaSuccess ||
+        cudaMemsetAsync(ws + L.off_cnt, 0, L.off_off - L.off_cnt, st) != cudaSuccess)
+        return NSA_ERR_CUDA;
+    // per-query statistics, d(gates), dq
+    {
+        const int smem = (16 * (DK + 1) + 16 * (DV + 1) + 64 * (DK + 1) + 64 * (DV + 1) + 16 * 64 + 16) * 4;
+        NSA_TRY(set_smem(bwd_query_kernel<DK, DV>, smem));
+        bwd_query_kernel<DK, DV><<<dim3((unsigned)s.T, (unsigned)s.G, (unsigned)s.B), 256, smem, st>>>(p);
+        NSA_TRY(last_launch());
+    }
+    // inverse index of the selection: block -> tokens
+    {
+        const long long N = s.B * s.T * s.G * s.n;
+        bwd_sel_count<<<(unsigned)ceil_div(N, 256), 256, 0, st>>>(p);
+        NSA_TRY(last_launch());
+        bwd_sel_scan<<<1, 1024, 0, st>>>(p);
+        NSA_TRY(last_launch());
+        bwd_sel_fill<<<(unsigned)ceil_div(N, 256), 256, 0, st>>>(p);
+        NSA_TRY(last_launch());
+    }
+    // key-centric dK/dV
+    {
+        dim3 gw((unsigned)ceil_div(s.T, 64), (unsigned)ceil_div(64 + s.w - 1, kBwdChunk), (unsigned)(s.B * s.G));
+        bwd_kv_kernel<DK, DV, kBrWin><<<gw, 256, 0, st>>>(p);
+        NSA_TRY(last_launch());
+        const int64_t maxch = NE + ceil_div(s.B * s.T * s.G * s.n, kBwdChunk);
+        bwd_kv_kernel<DK, DV, kBrSlc><<<(unsigned)maxch, 256, 0, st>>>(p);
+        NSA_TRY(last_launch());
+        if (s.C > 0) {
+            dim3 gc((unsigned)ceil_div(s.C, 64), (unsigned)ceil_div(s.T, kBwdChunk), (unsigned)(s.B * s.G));
+            bwd_kv_kernel<DK, DV, kBrCmp><<<gc, 256, 0, st>>>(p);
+            NSA_TRY(last_launch());
+            dim3 gp((unsigned)s.T, (unsigned)s.G, (unsigned)s.B);
+            bwd_phiT_kernel<DK><<<gp, DK, 0, st>>>(p, p.dkc, p.wk, dk);
+            NSA_TRY(last_launch());
+            bwd_phiT_kernel<DV><<<gp, DV, 0, st>>>(p, p.dvc, p.wv, dv);
+            NSA_TRY(last_launch());
+        }
+    }
+    return NSA_OK;
+}
+
+// ---------------------------------------------------------------- decode
+nsa_status_t decode_impl(const Shape& s, int S, const void* q, const void* kcache, const void* vcache,
+                         const int64_t* kv_off, const void* kccache, const void* vccache,
+                         const int64_t* cmp_off, const float* gates, float* out, int32_t* sel_idx,
+                         float* lse, uint8_t* ws, cudaStream_t st) {
+    DecParams p{};
+    p.S = S;
+    p.H = (int)s.H;
+    p.G = (int)s.G;
+    p.HG = (int)s.HG;
+    p.DK = (int)s.DK;
+    p.DV = (int)s.DV;
+    p.l = (int)s.l;
+    p.d = (int)s.d;
+    p.lp = (int)s.lp;
+    p.n = (int)s.n;
+    p.fi = (int)s.fi;
+    p.fl = (int)s.fl;
+    p.w = (int)s.w;
+    p.scale_log2 = s.scale * kLog2e;
+    p.q = reinterpret_cast<const __nv_bfloat16*>(q);
+    p.kcache = reinterpret_cast<const __nv_bfloat16*>(kcache);
+    p.vcache = reinterpret_cast<const __nv_bfloat16*>(vcache);
+    p.kccache = reinterpret_cast<const __nv_bfloat16*>(kccache);
+    p.vccache = reinterpret_cast<const __nv_bfloat16*>(vccache);
+    p.kv_off = kv_off;
+    p.cmp_off = cmp_off;
+    p.gates = gates;
+    p.out = out;
+    p.sel_idx = sel_idx;
+    p.lse = lse;
+    p.Cmax = (int)(s.T >= s.l ? (s.T - s.l) / s.d + 1 : 1);
+    p.NSPL = (int)ceil_div(p.Cmax, kDecCH);
+    p.NU = (int)(s.n + ceil_div(s.w, s.lp) + 1);
+    p.NSmax = (int)ceil_div(s.T, s.lp);
+    size_t o = 0;
+    auto carve = [&](size_t bytes) {
+        float* r = reinterpret_cast<float*>(ws + o);
+        o = align256(o + bytes);
+        return r;
+    };
+    p.logits = carve((size_t)S * s.G * 16 * p.Cmax * 4);
+    p.part1 = carve((size_t)S * s.G * p.NSPL * 16 * (2 + s.DV) * 4);
+    p.ocmp = carve((size_t)S * s.G * 16 * s.DV * 4);
+    p.lsecmp = carve((size_t)S * s.G * 16 * 4);
+    p.part2 = carve((size_t)S * s.G * p.NU * 2 * 16 * (2 + s.DV) * 4);
+    dec_cmp_partial<<<dim3((unsigned)p.NSPL, (unsigned)s.G, (unsigned)S), 256, 0, st>>>(p);
+    NSA_TRY(last_launch());
+    const int smem2 = (p.Cmax + p.NSmax) * 4;
+    NSA_TRY(set_smem(dec_cmp_combine, smem2));
+    dec_cmp_combine<<<dim3((unsigned)s.G, (unsigned)S), 256, smem2, st>>>(p);
+    NSA_TRY(last_launch());
+    dec_slcwin_partial<<<dim3((unsigned)p.NU, (unsigned)s.G, (unsigned)S), 256, 0, st>>>(p);
+    NSA_TRY(last_launch());
+    dec_final<<<dim3((unsigned)s.G, (unsigned)S), 256, 0, st>>>(p);
+    return last_launch();
+}
+
+}  // namespace
+
+// ==================================================================== C ABI
+
+extern "C" {
+
+const char* nsa_status_string(nsa_status_t st) {
+    switch (st) {
+        case NSA_OK: return "ok";
+        case NSA_ERR_INVALID_ARG: return "invalid argument";
+        case NSA_ERR_UNSUPPORTED: return "unsupported configuration";
+        case NSA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case NSA_ERR_CUDA: return "CUDA call or kernel launch failed";
+        case NSA_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait expired";
+    }
+    return "unknown status";
+}
+
+int64_t nsa_num_cmp_blocks(const nsa_config_t* cfg, int64_t len) {
+    if (!cfg || cfg->cmp_stride <= 0 || cfg->cmp_block <= 0 || len < cfg->cmp_block) return 0;
+    return (len - cfg->cmp_block) / cfg->cmp_stride + 1;
+}
+
+size_t nsa_workspace_size(const nsa_config_t* cfg, int32_t mode) {
+    Shape s;
+    if (derive(cfg, s) != NSA_OK) return 0;
+    if (mode == NSA_MODE_FORWARD) return fwd_layout(s).total;
+    if (mode == NSA_MODE_DECODE) return decode_ws_bytes(s.B, s.T, s.G, s.l, s.d, s.lp, s.w, s.n, s.DV);
+    if (mode == NSA_MODE_BACKWARD) return bwd_layout(s).total;
+    return 0;
+}
+
+nsa_status_t nsa_compress(const nsa_config_t* cfg, const void* k, const void* v,
+                          const nsa_phi_params_t* phi, void* kc, void* vc, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+    Shape s;
+    NSA_TRY(derive(cfg, s));
+    NSA_TRY(supported(s));
+    if (!k || !v || !kc || !vc) return NSA_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(kc) || !aligned16(vc)) return NSA_ERR_INVALID_ARG;
+    const FwdWs L = fwd_layout(s);
+    if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return NSA_ERR_WORKSPACE;
+    uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+    return run_phi(s, k, v, phi, kc, vc, ws + L.off_vct, reinterpret_cast<float*>(ws + L.off_bias),
+                   ws + L.off_fix, reinterpret_cast<cudaStream_t>(stream));
+}
+
+nsa_status_t nsa_forward(const nsa_config_t* cfg, const void* q, const void* k, const void* v,
+                         const float* gates, const nsa_phi_params_t* phi, float* out,
+                         int32_t* sel_idx, float* lse, void* kc_out, void* vc_out, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+    Shape s;
+    NSA_TRY(derive(cfg, s));
+    NSA_TRY(supported(s));
+    if (cfg->score_map != 0) return NSA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !gates || !out || !sel_idx) return NSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        (kc_out && !aligned16(kc_out)) || (vc_out && !aligned16(vc_out)))
+        return NSA_ERR_INVALID_ARG;
+    const FwdWs L = fwd_layout(s);
+    if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return NSA_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+    if (s.DK == 192)
+        return forward_impl<192, 128, 16>(s, q, k, v, gates, phi, out, sel_idx, lse, kc_out, vc_out, ws, st);
+    return forward_impl<64, 64, 4>(s, q, k, v, gates, phi, out, sel_idx, lse, kc_out, vc_out, ws, st);
+}
+
+nsa_status_t nsa_decode(const nsa_config_t* cfg, int32_t num_seqs, const void* q,
+                        const void* k_cache, const void* v_cache, const int64_t* kv_offsets,
+                        const void* kc_cache, const void* vc_cache, const int64_t* cmp_offsets,
+                        const float* gates, float* out, int32_t* sel_idx, float* lse,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+    Shape s;
+    NSA_TRY(derive(cfg, s));
+    NSA_TRY(supported(s));
+    if (cfg->score_map != 0) return NSA_ERR_UNSUPPORTED;
+    if (num_seqs < 0 || num_seqs > cfg->batch) return NSA_ERR_INVALID_ARG;
+    if (num_seqs == 0) return NSA_OK;
+    if (!q || !k_cache || !v_cache || !kv_offsets || !kc_cache || !vc_cache || !cmp_offsets ||
+        !gates || !out || !sel_idx)
+        return NSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(kc_cache) ||
+        !aligned16(vc_cache))
+        return NSA_ERR_INVALID_ARG;
+    const size_t need = decode_ws_bytes(s.B, s.T, s.G, s.l, s.d, s.lp, s.w, s.n, s.DV);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return NSA_ERR_WORKSPACE;
+    return decode_impl(s, num_seqs, q, k_cache, v_cache, kv_offsets, kc_cache, vc_cache, cmp_offsets,
+                       gates, out, sel_idx, lse, reinterpret_cast<uint8_t*>(workspace),
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+nsa_status_t nsa_backward(const nsa_config_t* cfg, const void* q, const void* k, const void* v,
+                          const float* gates, const nsa_phi_params_t* phi, const void* dout,
+                          const int32_t* sel_idx, float* dq, float* dk, float* dv, float* dgates,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+    Shape s;
+    NSA_TRY(derive(cfg, s));
+    NSA_TRY(supported(s));
+    if (!q || !k || !v || !gates || !dout || !sel_idx || !dq || !dk || !dv || !dgates)
+        return NSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout)) return NSA_ERR_INVALID_ARG;
+    const BwdWs L = bwd_layout(s);
+    if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return NSA_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+    if (s.DK == 192)
+        return backward_impl<192, 128>(s, q, k, v, gates, phi, dout, sel_idx, dq, dk, dv, dgates, ws, st);
+    return backward_impl<64, 64>(s, q, k, v, gates, phi, dout, sel_idx, dq, dk, dv, dgates, ws, st);
+}
+
+nsa_status_t nsa_sync_status(void* stream) {
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return NSA_ERR_CUDA;
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_nsa_error, sizeof(v)) != cudaSuccess) return NSA_ERR_CUDA;
+    if (v) {
+        unsigned int z = 0;
+        cudaMemcpyToSymbol(g_nsa_error, &z, sizeof(z));
+        return (v & 1u) ? NSA_ERR_DEVICE_TIMEOUT : NSA_ERR_INVALID_ARG;
+    }
+    return NSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,232 @@
+"""Python binding of libnsa (include/nsa.h): argument marshalling only.
+
+Every step of the operator runs in the library's CUDA kernels; this module
+allocates outputs and the workspace with torch (device memory, streams) and
+passes raw pointers through ctypes.  There is no fallback: if libnsa.so is
+missing or a call fails, it raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SO = os.path.join(_HERE, "libnsa.so")
+
+NSA_MODE_FORWARD, NSA_MODE_DECODE, NSA_MODE_BACKWARD = 0, 1, 2
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "workspace",
+          4: "CUDA error", 5: "device timeout"}
+
+
+class NsaError(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__(f"{fn}: {STATUS.get(code, code)} ({code})")
+        self.code = code
+
+
+class CConfig(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("batch", "seqlen", "num_q_heads", "num_kv_groups", "d_k", "d_v", "cmp_block",
+                 "cmp_stride", "sel_block", "sel_count", "forced_initial", "forced_local", "window",
+                 "phi", "score_map")] + [("scale", ctypes.c_float)]
+
+
+class CPhi(ctypes.Structure):
+    _fields_ = [("w_k", ctypes.c_void_p), ("e_k", ctypes.c_void_p), ("w_v", ctypes.c_void_p),
+                ("e_v", ctypes.c_void_p)]
+
+
+_lib = None
+_P = ctypes.c_void_p
+
+
+def library_path() -> str:
+    return _SO
+
+
+def lib():
+    """Load libnsa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_SO):
+            raise ImportError(f"libnsa.so not found at {_SO}: build it with "
+                              "`python -m sparse_attention_long_phi_b200.build`")
+        L = ctypes.CDLL(_SO)
+        pc = ctypes.POINTER(CConfig)
+        pp = ctypes.POINTER(CPhi)
+        L.nsa_workspace_size.restype = ctypes.c_size_t
+        L.nsa_workspace_size.argtypes = [pc, ctypes.c_int32]
+        L.nsa_num_cmp_blocks.restype = ctypes.c_int64
+        L.nsa_num_cmp_blocks.argtypes = [pc, ctypes.c_int64]
+        L.nsa_compress.restype = ctypes.c_int
+        L.nsa_compress.argtypes = [pc, _P, _P, pp, _P, _P, _P, ctypes.c_size_t, _P]
+        L.nsa_forward.restype = ctypes.c_int
+        L.nsa_forward.argtypes = [pc, _P, _P, _P, _P, pp, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+        L.nsa_decode.restype = ctypes.c_int
+        L.nsa_decode.argtypes = [pc, ctypes.c_int32] + [_P] * 12 + [ctypes.c_size_t, _P]
+        L.nsa_backward.restype = ctypes.c_int
+        L.nsa_backward.argtypes = [pc, _P, _P, _P, _P, pp, _P, _P, _P, _P, _P, _P, _P,
+                                   ctypes.c_size_t, _P]
+        L.nsa_sync_status.restype = ctypes.c_int
+        L.nsa_sync_status.argtypes = [_P]
+        L.nsa_status_string.restype = ctypes.c_char_p
+        L.nsa_status_string.argtypes = [ctypes.c_int]
+        _lib = L
+    return _lib
+
+
+def make_config(c: dict, batch=None, seqlen=None) -> CConfig:
+    """nsa_config_t from a workload dict (keys B, T, H, G, dk, dv, l, d, lp, n, fi, fl, w, phi)."""
+    phi = c.get("phi", "mean")
+    phi = {"mean": 0, "linear": 1}.get(phi, phi)
+    return CConfig(int(batch if batch is not None else c.get("B", 1)),
+                   int(seqlen if seqlen is not None else c.get("T", 0)), int(c["H"]), int(c["G"]),
+                   int(c["dk"]), int(c["dv"]), int(c["l"]), int(c["d"]), int(c["lp"]), int(c["n"]),
+                   int(c.get("fi", 1)), int(c.get("fl", 2)), int(c["w"]), int(phi),
+                   int(c.get("score_map", 0)), float(c.get("scale", 0.0)))
+
+
+def _p(t):
+    if t is None:
+        return None
+    assert t.is_contiguous(), "libnsa tensors must be contiguous"
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn, code):
+    if code != 0:
+        raise NsaError(fn, code)
+
+
+def _phi(phi):
+    if phi is None:
+        return None
+    return ctypes.byref(CPhi(*(ctypes.c_void_p(phi[k].data_ptr()) for k in ("wk", "ek", "wv", "ev"))))
+
+
+def workspace_size(c: dict, mode: int, batch=None, seqlen=None) -> int:
+    return int(lib().nsa_workspace_size(ctypes.byref(make_config(c, batch, seqlen)), mode))
+
+
+def num_cmp_blocks(c: dict, length: int) -> int:
+    return int(lib().nsa_num_cmp_blocks(ctypes.byref(make_config(c)), int(length)))
+
+
+def alloc_workspace(c: dict, mode: int, device, batch=None, seqlen=None) -> torch.Tensor:
+    n = workspace_size(c, mode, batch, seqlen)
+    if n == 0:
+        raise NsaError("nsa_workspace_size", 1)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+@dataclass
+class ForwardBuffers:
+    out: torch.Tensor
+    idx: torch.Tensor
+    lse: torch.Tensor | None
+    kc: torch.Tensor | None
+    vc: torch.Tensor | None
+    ws: torch.Tensor
+
+
+def forward_buffers(c: dict, device, want_lse=True, want_kc=False) -> ForwardBuffers:
+    B, T, H, G, dk, dv = c["B"], c["T"], c["H"], c["G"], c["dk"], c["dv"]
+    C = num_cmp_blocks(c, T)
+    f32 = dict(dtype=torch.float32, device=device)
+    return ForwardBuffers(
+        out=torch.empty(B, T, H, dv, **f32),
+        idx=torch.empty(B, T, G, c["n"], dtype=torch.int32, device=device),
+        lse=torch.empty(B, T, H, 3, **f32) if want_lse else None,
+        kc=torch.empty(B, max(C, 1), G, dk, dtype=torch.bfloat16, device=device) if want_kc else None,
+        vc=torch.empty(B, max(C, 1), G, dv, dtype=torch.bfloat16, device=device) if want_kc else None,
+        ws=alloc_workspace(c, NSA_MODE_FORWARD, device))
+
+
+def forward_into(c: dict, q, k, v, gates, phi, buf: ForwardBuffers, stream=None):
+    """nsa_forward into preallocated buffers (asynchronous on the stream)."""
+    cfg = make_config(c)
+    _check("nsa_forward", lib().nsa_forward(
+        ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(gates), _phi(phi), _p(buf.out), _p(buf.idx),
+        _p(buf.lse), _p(buf.kc), _p(buf.vc), _p(buf.ws), buf.ws.numel(), _stream(stream)))
+
+
+def forward(c: dict, q, k, v, gates, phi=None, want_lse=True, want_kc=False, stream=None) -> dict:
+    """Prefill forward.  q [B,T,H,dk], k [B,T,G,dk], v [B,T,G,dv] bf16; gates [B,T,H,3] fp32;
+    phi = dict(wk, ek, wv, ev) for the linear map.  Returns out, idx, lse, kc, vc."""
+    buf = forward_buffers(c, q.device, want_lse, want_kc)
+    forward_into(c, q, k, v, gates, phi, buf, stream)
+    return {"out": buf.out, "idx": buf.idx, "lse": buf.lse, "kc": buf.kc, "vc": buf.vc}
+
+
+def compress(c: dict, k, v, phi=None, stream=None):
+    B, T, G = c["B"], c["T"], c["G"]
+    C = num_cmp_blocks(c, T)
+    kc = torch.empty(B, max(C, 1), G, c["dk"], dtype=torch.bfloat16, device=k.device)
+    vc = torch.empty(B, max(C, 1), G, c["dv"], dtype=torch.bfloat16, device=k.device)
+    ws = alloc_workspace(c, NSA_MODE_FORWARD, k.device)
+    _check("nsa_compress", lib().nsa_compress(ctypes.byref(make_config(c)), _p(k), _p(v), _phi(phi),
+                                              _p(kc), _p(vc), _p(ws), ws.numel(), _stream(stream)))
+    return kc[:, :C], vc[:, :C]
+
+
+@dataclass
+class DecodeBuffers:
+    out: torch.Tensor
+    idx: torch.Tensor
+    lse: torch.Tensor | None
+    ws: torch.Tensor
+
+
+def decode_buffers(c: dict, num_seqs: int, max_len: int, device, want_lse=True) -> DecodeBuffers:
+    f32 = dict(dtype=torch.float32, device=device)
+    return DecodeBuffers(
+        out=torch.empty(num_seqs, c["H"], c["dv"], **f32),
+        idx=torch.empty(num_seqs, c["G"], c["n"], dtype=torch.int32, device=device),
+        lse=torch.empty(num_seqs, c["H"], 3, **f32) if want_lse else None,
+        ws=alloc_workspace(c, NSA_MODE_DECODE, device, batch=num_seqs, seqlen=max_len))
+
+
+def decode_into(c: dict, max_len: int, q, k_cache, v_cache, kv_off, kc_cache, vc_cache, cmp_off,
+                gates, buf: DecodeBuffers, stream=None):
+    S = q.shape[0]
+    cfg = make_config(c, batch=S, seqlen=max_len)
+    _check("nsa_decode", lib().nsa_decode(
+        ctypes.byref(cfg), S, _p(q), _p(k_cache), _p(v_cache), _p(kv_off), _p(kc_cache),
+        _p(vc_cache), _p(cmp_off), _p(gates), _p(buf.out), _p(buf.idx), _p(buf.lse), _p(buf.ws),
+        buf.ws.numel(), _stream(stream)))
+
+
+def decode(c: dict, q, k_cache, v_cache, kv_off, kc_cache, vc_cache, cmp_off, gates, max_len: int,
+           want_lse=True, stream=None) -> dict:
+    """One decode step: q [S,H,dk]; packed caches with int64 device offsets [S+1]."""
+    buf = decode_buffers(c, q.shape[0], max_len, q.device, want_lse)
+    decode_into(c, max_len, q, k_cache, v_cache, kv_off, kc_cache, vc_cache, cmp_off, gates, buf,
+                stream)
+    return {"out": buf.out, "idx": buf.idx, "lse": buf.lse}
+
+
+def backward(c: dict, q, k, v, gates, dout, idx, phi=None, stream=None) -> dict:
+    """Gradients with the selection idx [B,T,G,n] held fixed: dq, dk, dv, dgates (fp32)."""
+    B, T, H, G, dk, dv = c["B"], c["T"], c["H"], c["G"], c["dk"], c["dv"]
+    f32 = dict(dtype=torch.float32, device=q.device)
+    res = {"dq": torch.empty(B, T, H, dk, **f32), "dk": torch.empty(B, T, G, dk, **f32),
+           "dv": torch.empty(B, T, G, dv, **f32), "dgates": torch.empty(B, T, H, 3, **f32)}
+    ws = alloc_workspace(c, NSA_MODE_BACKWARD, q.device)
+    _check("nsa_backward", lib().nsa_backward(
+        ctypes.byref(make_config(c)), _p(q), _p(k), _p(v), _p(gates), _phi(phi), _p(dout), _p(idx),
+        _p(res["dq"]), _p(res["dk"]), _p(res["dv"]), _p(res["dgates"]), _p(ws), ws.numel(),
+        _stream(stream)))
+    return res
+
+
+def sync_status(stream=None):
+    """Synchronise and raise if a kernel's bounded wait expired since the last check."""
+    _check("nsa_sync_status", lib().nsa_sync_status(_stream(stream)))

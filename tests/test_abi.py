@@ -1,0 +1,84 @@
+"""The C-ABI library builds, exports every entry point include/nsa.h declares,
+and validates its arguments on the host (no GPU needed: every case below is
+rejected before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_attention_long_phi_b200 import build as nbuild
+from sparse_attention_long_phi_b200 import inputs as I
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    nbuild.build()
+    from sparse_attention_long_phi_b200 import nsa
+    return nsa
+
+
+def declared_functions():
+    txt = open(os.path.join(ROOT, "include", "nsa.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(nsa_[a-z_]+)\s*\(", txt)))
+
+
+def test_library_exports_every_declared_entry_point(L):
+    names = declared_functions()
+    assert {"nsa_forward", "nsa_decode", "nsa_backward", "nsa_workspace_size",
+            "nsa_status_string", "nsa_compress", "nsa_sync_status", "nsa_num_cmp_blocks"} <= set(names)
+    lib = ctypes.CDLL(L.library_path())
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings_and_shape_helpers(L):
+    lib = L.lib()
+    for code in range(6):
+        assert lib.nsa_status_string(code)
+    c = I.WORKLOADS["prefill_fwd_T65536"]
+    assert L.num_cmp_blocks(c, 65536) == 4095
+    assert L.num_cmp_blocks(c, 31) == 0 and L.num_cmp_blocks(c, 32) == 1
+    for mode in (0, 1, 2):
+        assert L.workspace_size(c, mode) > 0
+
+
+def _fwd(L, c, ptrs=True, ws_bytes=1 << 30):
+    lib = L.lib()
+    cfg = L.make_config(c)
+    fake = ctypes.c_void_p(1 << 20) if ptrs else None     # never dereferenced: rejected first
+    return lib.nsa_forward(ctypes.byref(cfg), fake, fake, fake, fake, None, fake, fake, None, None,
+                           None, ctypes.c_void_p(1 << 20), ws_bytes, None)
+
+
+def test_forward_argument_validation_on_host(L):
+    base = dict(I.WORKLOADS["prefill_fwd_T8192"], phi="mean")
+    assert _fwd(L, dict(base, d=12)) == 1                   # d does not divide l
+    assert _fwd(L, dict(base, l=128)) == 1                  # l > l'
+    assert _fwd(L, dict(base, n=2)) == 1                    # n < forced blocks
+    assert _fwd(L, dict(base, H=63)) == 1                   # heads not a multiple of groups
+    assert _fwd(L, dict(base, T=0)) == 1
+    assert _fwd(L, base, ptrs=False) == 1                   # null tensors
+    assert _fwd(L, dict(base, dk=128)) == 2                 # no kernel for d_k = 128
+    assert _fwd(L, dict(base, lp=32, l=16)) == 2            # selection block != 64
+    assert _fwd(L, dict(base, n=17)) == 2
+    assert _fwd(L, base, ws_bytes=1024) == 3                # workspace too small
+
+
+def test_decode_and_backward_validation_on_host(L):
+    lib = L.lib()
+    c = dict(I.WORKLOADS["decode_S32_L8k_64k"], B=32, T=65536)
+    cfg = L.make_config(c, batch=32, seqlen=65536)
+    fake = ctypes.c_void_p(1 << 20)
+    args = [fake] * 12
+    assert lib.nsa_decode(ctypes.byref(cfg), 33, *args, 1 << 30, None) == 1   # more seqs than sized
+    assert lib.nsa_decode(ctypes.byref(cfg), 8, *args, 16, None) == 3         # workspace too small
+    assert lib.nsa_decode(ctypes.byref(cfg), 0, *args, 16, None) == 0         # nothing to do
+    cb = L.make_config(I.WORKLOADS["train_fwd_bwd_B2_T16384"])
+    assert lib.nsa_backward(ctypes.byref(cb), fake, fake, fake, fake, None, fake, fake, fake, fake,
+                            fake, fake, fake, 64, None) == 3
+    assert lib.nsa_backward(ctypes.byref(cb), None, fake, fake, fake, None, fake, fake, fake, fake,
+                            fake, fake, fake, 1 << 40, None) == 1

@@ -1,0 +1,482 @@
+"""Benchmark of the NSA per-layer attention operator on B200 (one JSON line).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl nsa|reference]
+
+A step is one nsa_forward (token compression, compressed attention with score
+emission, top-n selection, selected and window attention, gated merge) over one
+sequence of the prefill workload (default: T=65536, 64 heads in 4 GQA groups,
+d_k=192, d_v=128, l=32, d=16, l'=64, n=16, w=512, linear phi), inputs resident
+in HBM.  Under torchrun every rank runs its own sequence (weak scaling, no
+data-path collective); rank 0 prints.  The line also carries, from the same
+run: the roofline of the dominant kernel, an end-to-end figure through host
+buffers, the clocks seen during the timed region, the number of kernel
+launches, the CPU baseline (the fp64 oracle on a bounded sample) and the
+decode and backward measurements of their own workloads.
+
+--impl reference times the oracle (the reference of this build) on host cores
+with the same metric, each step a bounded sample extrapolated to a full step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_attention_long_phi_b200 import inputs as I  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------ work accounting
+def branch_counts(c, T):
+    """keys read per query by each branch, per token t (numpy, all t < T)"""
+    t = np.arange(T, dtype=np.int64)
+    ncmp = np.where(t + 1 >= c["l"], (t + 1 - c["l"]) // c["d"] + 1, 0)
+    few = t // c["lp"] + 1 <= c["n"]
+    nslc = np.where(few, t + 1, (c["n"] - 1) * c["lp"] + t % c["lp"] + 1)
+    nwin = np.minimum(c["w"], t + 1)
+    return ncmp, nslc, nwin
+
+
+def forward_flops(c):
+    """algorithmic FLOPs of one forward per kernel (2 FLOP per multiply-add)"""
+    B, T, H, G, dk, dv, l = c["B"], c["T"], c["H"], c["G"], c["dk"], c["dv"], c["l"]
+    ncmp, nslc, nwin = branch_counts(c, T)
+    C = (T - l) // c["d"] + 1 if T >= l else 0
+    f = {
+        "attn_cmp_lse": 2.0 * dk * H * ncmp.sum() * B,          # logits for the row LSE
+        "attn_cmp_pv_scores": 2.0 * dv * H * ncmp.sum() * B,    # P.V~ (logits recomputed)
+        "attn_sel_kernel": 2.0 * (dk + dv) * H * nslc.sum() * B,
+        "attn_window": 2.0 * (dk + dv) * H * nwin.sum() * B,
+    }
+    if c.get("phi") == "linear":
+        f["phi_linear_kernel"] = 2.0 * B * C * G * l * (dk * dk + dv * dv)
+    total_attn = 2.0 * (dk + dv) * H * (ncmp.sum() + nslc.sum() + nwin.sum()) * B
+    return f, total_attn
+
+
+def csrc_sha():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "sparse_attention_long_phi_b200", "csrc")
+    for n in sorted(os.listdir(d)):
+        h.update(open(os.path.join(d, n), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if the
+    kernel sources have not changed since it was captured (else None)."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.md")
+    if not os.path.exists(p):
+        return None
+    sha = csrc_sha()
+    for line in open(p):
+        parts = line.strip().split()
+        if len(parts) == 4 and parts[0] == "traffic:" and parts[1] == kernel and parts[3] == sha:
+            return float(parts[2])
+    return None
+
+
+# -------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.gpu = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.gpu = str(device.index or 0)
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        self.proc.wait()
+        rows = []
+        for line in open(self.path):
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 8:
+                continue
+            try:
+                rows.append((float(p[0]), float(p[1]), p[2], p[3:]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        smax = max(r[1] for r in rows)
+        load = [r for r in rows if r[0] > 0.5 * smax] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in load for i, v in enumerate(r[3][1:5]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in load), "sm_max_mhz": smax,
+                "reasons": reasons, "samples": len(load)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_sample(c, x_host, rows_per_step, phi_fraction, seed):
+    """Time the fp64 oracle on a bounded sample of one forward step: phi over
+    a slice of the compressed blocks and the full forward of rows drawn
+    uniformly over t.  Returns (seconds for a full step by extrapolation,
+    description)."""
+    import oracle
+    T = c["T"]
+    C = oracle.num_cmp_blocks(c, T)
+    # phi over a contiguous slice of ~phi_fraction of the blocks (timed),
+    # then the whole phi (untimed) for the rows' compressed branch
+    nb = max(1, int(C * phi_fraction))
+    cut = min(T, (nb - 1) * c["d"] + c["l"])
+    cs = dict(c, T=cut)
+    t0 = time.perf_counter()
+    oracle.phi(cs, x_host["k"][:, :cut], x_host["v"][:, :cut], x_host.get("wk"), x_host.get("ek"),
+               x_host.get("wv"), x_host.get("ev"))
+    t_phi = time.perf_counter() - t0
+    if "_kc" not in x_host:
+        x_host["_kc"] = oracle.phi(c, x_host["k"], x_host["v"], x_host.get("wk"), x_host.get("ek"),
+                                   x_host.get("wv"), x_host.get("ev"))
+    kc, vc = x_host["_kc"]
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.integers(0, c["B"] * T, rows_per_step))
+    t0 = time.perf_counter()
+    oracle.forward_rows(c, x_host["q"], x_host["k"], x_host["v"], x_host["gates"], kc, vc, rows)
+    t_rows = time.perf_counter() - t0
+    full = t_phi * (C / nb) + t_rows * (c["B"] * T / rows_per_step)
+    desc = (f"fp64 oracle: phi over {nb}/{C} compressed blocks and the forward of "
+            f"{rows_per_step} rows drawn uniformly over t, extrapolated to one full step "
+            f"({t_phi + t_rows:.1f} s measured)")
+    return full, desc
+
+
+def host_inputs(x):
+    return {k: (I.bits(v) if v.dtype == torch.bfloat16 else v.detach().cpu().numpy())
+            for k, v in x.items()}
+
+
+# --------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="nsa", choices=["nsa", "reference"])
+    ap.add_argument("--workload", default="prefill_fwd_T65536")
+    ap.add_argument("--seq-len", type=int, default=0, help="override T (smaller profiling cases)")
+    ap.add_argument("--no-extras", action="store_true", help="skip e2e, CPU, decode, backward")
+    args = ap.parse_args()
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    c = dict(I.WORKLOADS[args.workload])
+    if args.seq_len:
+        c["T"] = args.seq_len
+    tokens_per_step = c["B"] * c["T"]
+
+    if args.impl == "reference":
+        run_reference(args, c, rank, world, tokens_per_step)
+        return
+
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    from sparse_attention_long_phi_b200 import nsa
+    peaks, peak_src = load_peaks()
+
+    # inputs: per-rank seed (independent sequences), resident in HBM
+    cr = dict(c, seed=c["seed"] + 7919 * rank)
+    x = I.make_forward_inputs(cr, dev)
+    phi = {k: x[k] for k in ("wk", "ek", "wv", "ev")} if "wk" in x else None
+    buf = nsa.forward_buffers(cr, dev, want_lse=False)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        nsa.forward_into(cr, x["q"], x["k"], x["v"], x["gates"], phi, buf, stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier(device_ids=[local])
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    nsa.sync_status()
+    nsa.profile_read()                      # drop warm-up records
+    clocks = ClockSampler(dev)
+    clocks.start()
+    nsa.profile_enable(True)
+    barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    barrier()
+    nsa.profile_enable(False)
+    clk = clocks.stop()
+    nsa.sync_status()
+    ms = ev0.elapsed_time(ev1)
+    prof = nsa.profile_read()
+    if dist is not None:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    value = world * tokens_per_step * args.steps / (ms / 1e3)
+
+    # roofline of the dominant kernel (largest device time in the timed region)
+    flops, attn_total = forward_flops(cr)
+    launches = sum(n for n, _ in prof.values())
+    dom = max(prof, key=lambda k: prof[k][1])
+    n_dom, t_dom = prof[dom]
+    peak_tf = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    if dom in flops:
+        per_launch = flops[dom] * args.steps / n_dom
+        achieved = per_launch / (t_dom / n_dom / 1e3) / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak_tf,
+                "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4),
+                "traffic": ncu_traffic(dom), "peak_source": f"{peak_src} bf16 sustained"}
+    else:
+        roof = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": None, "traffic": ncu_traffic(dom)}
+    kernels = {k: {"launches": n, "ms_per_step": round(t / args.steps, 4),
+                   "share": round(t / sum(v[1] for v in prof.values()), 4)} for k, (n, t) in prof.items()}
+    step_tflops = attn_total / (ms_step / 1e3) / 1e12
+
+    line = {
+        "metric": "NSA prefill tokens/s @64k (% BF16 TC peak); decode tokens/s @64k (% HBM BW)",
+        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "batch": cr["B"], "seq_len": cr["T"],
+                   "q_heads": cr["H"], "kv_groups": cr["G"], "d_k": cr["dk"], "d_v": cr["dv"],
+                   "l": cr["l"], "d": cr["d"], "l_sel": cr["lp"], "n": cr["n"], "w": cr["w"],
+                   "phi": cr["phi"], "parallelism": f"replicas x{world}",
+                   "l2": "no flush: inputs and outputs per step (q 1.6 GB, out 2.1 GB) exceed L2"},
+        "attn_tflops": round(step_tflops, 1),
+        "attn_frac_of_peak": round(step_tflops / peaks.get("bf16_tflops", 1590.0), 4),
+        "roofline": roof, "kernels": kernels, "gpu_launches": launches, "clocks": clk,
+    }
+
+    if not args.no_extras:
+        line["e2e"] = e2e_forward(cr, x, phi, dev, stream, nsa, min(args.steps, 5), world, dist, local)
+        line["decode"] = bench_decode(dev, nsa, peaks, peak_src)
+        line["backward"] = bench_backward(dev, nsa, peaks)
+        if rank == 0 and world == 1:
+            try:
+                hx = host_inputs(x)
+                full, desc = oracle_sample(cr, hx, rows_per_step=24, phi_fraction=1 / 8, seed=1)
+                import oracle
+                line["cpu_baseline"] = {"value": round(tokens_per_step / full, 3), "unit": "tokens/s",
+                                        "cores": oracle.num_threads(), "kind": "oracle",
+                                        "sample": desc}
+            except Exception as e:  # the baseline is reported, never the product path
+                line["cpu_baseline"] = {"value": None, "unit": "tokens/s", "kind": "oracle",
+                                        "cores": None, "sample": f"failed: {e}"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+
+
+def e2e_forward(c, x, phi, dev, stream, nsa, steps, world, dist, local):
+    """Same metric through the public API with host buffers: pinned host
+    inputs copied in, nsa_forward, output and selection copied back."""
+    names = ["q", "k", "v", "gates"] + (["wk", "ek", "wv", "ev"] if phi else [])
+    hin = {k: x[k].detach().cpu().pin_memory() for k in names}
+    din = {k: torch.empty_like(x[k]) for k in names}
+    buf = nsa.forward_buffers(c, dev, want_lse=False)
+    hout = torch.empty(buf.out.shape, dtype=buf.out.dtype).pin_memory()
+    hidx = torch.empty(buf.idx.shape, dtype=buf.idx.dtype).pin_memory()
+    bi = sum(t.numel() * t.element_size() for t in hin.values())
+    bo = hout.numel() * hout.element_size() + hidx.numel() * hidx.element_size()
+
+    def one():
+        for k in names:
+            din[k].copy_(hin[k], non_blocking=True)
+        p = {k: din[k] for k in ("wk", "ek", "wv", "ev")} if phi else None
+        nsa.forward_into(c, din["q"], din["k"], din["v"], din["gates"], p, buf, stream)
+        hout.copy_(buf.out, non_blocking=True)
+        hidx.copy_(buf.idx, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": round(world * c["B"] * c["T"] * steps / (ms / 1e3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": steps}
+
+
+def bench_decode(dev, nsa, peaks, peak_src, steps=50, warmup=5):
+    """Batched decode (32 sequences, L ~ U[8192, 65536]) against HBM bandwidth."""
+    c = dict(I.WORKLOADS["decode_S32_L8k_64k"])
+    x = I.make_decode_inputs(c, lambda L: nsa.num_cmp_blocks(c, L), dev)
+    Lmax = int(x["lengths"].max())
+    kv_off = torch.from_numpy(x["kv_off"]).to(dev)
+    cmp_off = torch.from_numpy(x["cmp_off"]).to(dev)
+    buf = nsa.decode_buffers(c, c["S"], Lmax, dev, want_lse=False)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        nsa.decode_into(c, Lmax, x["q"], x["k_cache"], x["v_cache"], kv_off, x["kc_cache"],
+                        x["vc_cache"], cmp_off, x["gates"], buf, stream)
+
+    # each timed step reads a fresh copy of the caches: flush L2 with a 512 MB write
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    nsa.sync_status()
+    times = []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    # unique bytes read: compressed cache rows + the tokens of (selected U window) blocks
+    idx = buf.idx.cpu().numpy()
+    G, dk, dv, H, lp, w = c["G"], c["dk"], c["dv"], c["H"], c["lp"], c["w"]
+    row = (dk + dv) * 2
+    nbytes = 0
+    for s, L in enumerate(x["lengths"]):
+        C = nsa.num_cmp_blocks(c, int(L))
+        blocks = set()
+        for g in range(G):
+            bl = set(int(j) for j in idx[s, g] if j >= 0) | set(range(max(0, L - w) // lp, (L - 1) // lp + 1))
+            toks = sum(min(lp, int(L) - j * lp) for j in bl)
+            nbytes += (C + toks) * row
+            blocks |= bl
+        nbytes += H * dk * 2 + H * 3 * 4 + H * dv * 4
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"workload": "decode_S32_L8k_64k", "value": round(c["S"] / (ms / 1e3), 1),
+            "unit": "tokens/s", "ms_per_step": round(ms, 4), "unique_bytes_per_step": int(nbytes),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                         "peak_source": f"{peak_src} copy bandwidth", "frac_of_8TBs": round(gbs / 8000, 4)},
+            "l2": "flushed (512 MB write) before each timed step"}
+
+
+def bench_backward(dev, nsa, peaks, steps=2, warmup=1):
+    """Forward + backward of the training workload (B=2, T=16384)."""
+    c = dict(I.WORKLOADS["train_fwd_bwd_B2_T16384"])
+    x = I.make_forward_inputs(c, dev, with_dout=True)
+    phi = {k: x[k] for k in ("wk", "ek", "wv", "ev")}
+    stream = torch.cuda.current_stream(dev)
+    fb = nsa.forward_buffers(c, dev, want_lse=False)
+    nsa.forward_into(c, x["q"], x["k"], x["v"], x["gates"], phi, fb, stream)
+    for _ in range(warmup):
+        nsa.backward(c, x["q"], x["k"], x["v"], x["gates"], x["dout"], fb.idx, phi)
+    torch.cuda.synchronize(dev)
+    nsa.sync_status()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        nsa.forward_into(c, x["q"], x["k"], x["v"], x["gates"], phi, fb, stream)
+    e1.record(stream)
+    for _ in range(steps):
+        nsa.backward(c, x["q"], x["k"], x["v"], x["gates"], x["dout"], fb.idx, phi)
+    e2.record(stream)
+    torch.cuda.synchronize(dev)
+    f_ms, b_ms = e0.elapsed_time(e1) / steps, e1.elapsed_time(e2) / steps
+    _, fwd = forward_flops(c)
+    bwd = 2 * fwd                               # dP, dV, dQ, dK
+    return {"workload": "train_fwd_bwd_B2_T16384", "fwd_ms": round(f_ms, 3), "bwd_ms": round(b_ms, 3),
+            "tokens_per_s": round(c["B"] * c["T"] / ((f_ms + b_ms) / 1e3), 1),
+            "bwd_tflops_algorithmic": round(bwd / (b_ms / 1e3) / 1e12, 2),
+            "bwd_frac_of_peak": round(bwd / (b_ms / 1e3) / 1e12 / peaks.get("bf16_tflops", 1590.0), 4)}
+
+
+def run_reference(args, c, rank, world, tokens_per_step):
+    """The oracle (fp64, host cores) as the reference arm: rank 0 only."""
+    if rank != 0:
+        return
+    import oracle
+    x = I.make_forward_inputs(c, "cuda" if torch.cuda.is_available() else "cpu")
+    hx = host_inputs(x)
+    for i in range(args.warmup):
+        oracle_sample(c, hx, rows_per_step=2, phi_fraction=1 / 64, seed=100 + i)
+    fulls = []
+    t0 = time.perf_counter()
+    desc = ""
+    for i in range(args.steps):
+        full, desc = oracle_sample(c, hx, rows_per_step=2, phi_fraction=1 / 64, seed=i)
+        fulls.append(full)
+    wall = time.perf_counter() - t0
+    sec = float(np.mean(fulls))
+    v = tokens_per_step / sec
+    line = {"metric": "NSA prefill tokens/s @64k (% BF16 TC peak); decode tokens/s @64k (% HBM BW)",
+            "value": round(v, 4), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": args.workload, "batch": c["B"], "seq_len": c["T"]},
+            "cpu_baseline": {"value": round(v, 4), "unit": "tokens/s", "kind": "oracle",
+                             "cores": oracle.num_threads(),
+                             "sample": desc + f"; {args.steps} steps in {wall:.1f} s"},
+            "e2e": {"value": round(v, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -129,8 +129,10 @@ nsa_status_t nsa_forward(const nsa_config_t* cfg, const void* q, const void* k, 
  * offsets are int64 device arrays of S+1 entries; gates [S,H,3] fp32.
  * Out: out [S,H,d_v] fp32, sel_idx [S,G,n] int32, lse [S,H,3] fp32 or NULL.
  * num_seqs must not exceed cfg->batch and no L_s may exceed cfg->seqlen (the
- * workspace was sized from them); a wrong cache length is not detected on the
- * device: the result for that sequence is undefined. */
+ * workspace was sized from them): a longer context is skipped on the device
+ * and reported as NSA_ERR_INVALID_ARG by nsa_sync_status().  A compressed
+ * cache of the wrong length is not detected: that sequence's result is
+ * undefined. */
 nsa_status_t nsa_decode(const nsa_config_t* cfg, int32_t num_seqs, const void* q,
                         const void* k_cache, const void* v_cache, const int64_t* kv_offsets,
                         const void* kc_cache, const void* vc_cache, const int64_t* cmp_offsets,
@@ -154,6 +156,18 @@ nsa_status_t nsa_backward(const nsa_config_t* cfg, const void* q, const void* k,
  * current device.  Returns NSA_ERR_DEVICE_TIMEOUT if a kernel's bounded wait
  * expired since the last call, NSA_ERR_CUDA if synchronisation failed. */
 nsa_status_t nsa_sync_status(void* stream);
+
+/* Per-kernel timing, for diagnostics and benchmarking.  While enabled (on =
+ * 1), every kernel launch made by the entry points is bracketed by two CUDA
+ * events recorded on the call's stream (events are created by the library,
+ * no device memory is allocated).  nsa_profile_read() waits for the recorded
+ * events and fills, per kernel name (at most max_kernels, 48-byte
+ * NUL-terminated names), the number of launches and the total device time in
+ * ms since the previous read, then clears the records; it returns the number
+ * of names written, or -1 on a CUDA error.  Not thread-safe against
+ * concurrent entry-point calls from other host threads. */
+nsa_status_t nsa_profile_enable(int32_t on);
+int32_t nsa_profile_read(int32_t max_kernels, char* names, int32_t* launches, float* total_ms);
 
 /* Static description of a status code. */
 const char* nsa_status_string(nsa_status_t status);

@@ -10,7 +10,10 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <string>
+#include <vector>
 
 #include "../../include/nsa.h"
 #include "k_attn_packed.cuh"
@@ -56,6 +59,54 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
+
+
+// ---------------------------------------------------------- launch timing
+struct ProfRec {
+    const char* name;
+    cudaEvent_t a, b;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof_recs;
+std::vector<cudaEvent_t> g_prof_pool;
+
+cudaEvent_t prof_event() {
+    if (!g_prof_pool.empty()) {
+        cudaEvent_t e = g_prof_pool.back();
+        g_prof_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+// brackets the launches in its scope with events on `st` when timing is on
+struct ProfScope {
+    const char* name;
+    cudaStream_t st;
+    cudaEvent_t a = nullptr, b = nullptr;
+    ProfScope(const char* n, cudaStream_t s) : name(n), st(s) {
+        if (!g_prof_on) return;
+        std::lock_guard<std::mutex> lk(g_prof_mu);
+        a = prof_event();
+        b = prof_event();
+        cudaEventRecord(a, st);
+    }
+    ~ProfScope() {
+        if (!a) return;
+        cudaEventRecord(b, st);
+        std::lock_guard<std::mutex> lk(g_prof_mu);
+        g_prof_recs.push_back({name, a, b});
+    }
+};
+
+#define NSA_LAUNCH(name, st, ...)        \
+    do {                                 \
+        ProfScope _prof_scope(name, st); \
+        __VA_ARGS__;                     \
+    } while (0)
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -180,15 +231,15 @@ nsa_status_t launch_phi_linear(const Shape& s, const void* x, const void* W, con
     if (!make_map(&mA, x, 5, dA, sA, bA) || !make_map(&mW, W, 2, dW, sW, bW)) return NSA_ERR_CUDA;
     NSA_TRY(set_smem(phi_linear_kernel<D>, PhiGemmCfg<D>::kSmem));
     dim3 grid((unsigned)ceil_div(s.C, 128), (unsigned)s.G, (unsigned)s.B);
-    phi_linear_kernel<D><<<grid, 192, PhiGemmCfg<D>::kSmem, st>>>(
+    NSA_LAUNCH("phi_linear_kernel", st, phi_linear_kernel<D><<<grid, 192, PhiGemmCfg<D>::kSmem, st>>>(
         mA, mW, bias, (int)s.l, (int)s.d, (int)s.C, (int)s.Cp, (int)s.G,
-        reinterpret_cast<__nv_bfloat16*>(y), reinterpret_cast<__nv_bfloat16*>(yT), fix_list, fix_count);
+        reinterpret_cast<__nv_bfloat16*>(y), reinterpret_cast<__nv_bfloat16*>(yT), fix_list, fix_count));
     NSA_TRY(last_launch());
-    phi_fixup_kernel<D><<<148 * 4, 256, 0, st>>>(
+    NSA_LAUNCH("phi_fixup_kernel", st, phi_fixup_kernel<D><<<148 * 4, 256, 0, st>>>(
         reinterpret_cast<const __nv_bfloat16*>(x), reinterpret_cast<const __nv_bfloat16*>(W),
         reinterpret_cast<const __nv_bfloat16*>(E), (int)s.T, (int)s.G, (int)s.l, (int)s.d, (int)s.C,
         (int)s.Cp, fix_list, fix_count, reinterpret_cast<__nv_bfloat16*>(y),
-        reinterpret_cast<__nv_bfloat16*>(yT));
+        reinterpret_cast<__nv_bfloat16*>(yT)));
     return last_launch();
 }
 
@@ -198,25 +249,25 @@ nsa_status_t run_phi(const Shape& s, const void* k, const void* v, const nsa_phi
     if (s.C == 0) return NSA_OK;
     if (s.phi == NSA_PHI_MEAN) {
         dim3 grid((unsigned)s.C, (unsigned)s.G, (unsigned)s.B);
-        phi_mean_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(k), (int)s.T,
+        NSA_LAUNCH("phi_mean_kernel", st, phi_mean_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(k), (int)s.T,
                                               (int)s.G, (int)s.DK, (int)s.l, (int)s.d, (int)s.C,
-                                              (int)s.Cp, reinterpret_cast<__nv_bfloat16*>(kc), nullptr);
+                                              (int)s.Cp, reinterpret_cast<__nv_bfloat16*>(kc), nullptr));
         NSA_TRY(last_launch());
-        phi_mean_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(v), (int)s.T,
+        NSA_LAUNCH("phi_mean_kernel", st, phi_mean_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(v), (int)s.T,
                                               (int)s.G, (int)s.DV, (int)s.l, (int)s.d, (int)s.C,
                                               (int)s.Cp, reinterpret_cast<__nv_bfloat16*>(vc),
-                                              reinterpret_cast<__nv_bfloat16*>(vcT));
+                                              reinterpret_cast<__nv_bfloat16*>(vcT)));
         return last_launch();
     }
     if (!phi || !phi->w_k || !phi->e_k || !phi->w_v || !phi->e_v) return NSA_ERR_INVALID_ARG;
     if (!aligned16(phi->w_k) || !aligned16(phi->w_v)) return NSA_ERR_INVALID_ARG;
-    phi_bias_kernel<<<(unsigned)s.DK, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(phi->w_k),
+    NSA_LAUNCH("phi_bias_kernel", st, phi_bias_kernel<<<(unsigned)s.DK, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(phi->w_k),
                                                     reinterpret_cast<const __nv_bfloat16*>(phi->e_k),
-                                                    (int)(s.l * s.DK), bias);
+                                                    (int)(s.l * s.DK), bias));
     NSA_TRY(last_launch());
-    phi_bias_kernel<<<(unsigned)s.DV, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(phi->w_v),
+    NSA_LAUNCH("phi_bias_kernel", st, phi_bias_kernel<<<(unsigned)s.DV, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(phi->w_v),
                                                     reinterpret_cast<const __nv_bfloat16*>(phi->e_v),
-                                                    (int)(s.l * s.DV), bias + s.DK);
+                                                    (int)(s.l * s.DV), bias + s.DK));
     NSA_TRY(last_launch());
     unsigned int* cnt = reinterpret_cast<unsigned int*>(fix);
     uint32_t* lk = reinterpret_cast<uint32_t*>(fix + 256);
@@ -242,9 +293,10 @@ nsa_status_t launch_packed(const Shape& s, const CUtensorMap& mQ, const CUtensor
                            const CUtensorMap& mV, const PackedParams& p, cudaStream_t st) {
     using Cfg = PackedCfg<DK, DV, HG, MODE>;
     auto kern = attn_packed_kernel<DK, DV, HG, MODE, CPS, SPB>;
+    const char* kern_name = MODE == kModeLse ? "attn_cmp_lse" : MODE == kModeCmp ? "attn_cmp_pv_scores" : "attn_window";
     NSA_TRY(set_smem(kern, Cfg::kSmem));
     dim3 grid((unsigned)p.n_qtiles, (unsigned)s.G, (unsigned)s.B);
-    kern<<<grid, 192, Cfg::kSmem, st>>>(mQ, mK, mV, p);
+    NSA_LAUNCH(kern_name, st, kern<<<grid, 192, Cfg::kSmem, st>>>(mQ, mK, mV, p));
     return last_launch();
 }
 
@@ -278,9 +330,9 @@ nsa_status_t forward_impl(const Shape& s, const void* q, const void* k, const vo
     // 2. v transposed for the P.V products of the selected and window branches
     {
         dim3 grid((unsigned)ceil_div(s.Tp, 64), (unsigned)s.G, (unsigned)s.B);
-        transpose_v_kernel<<<grid, dim3(64, 4), 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(v),
+        NSA_LAUNCH("transpose_v_kernel", st, transpose_v_kernel<<<grid, dim3(64, 4), 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(v),
                                                          (int)s.T, (int)s.G, (int)s.DV, (int)s.DVP,
-                                                         (int)s.Tp, reinterpret_cast<__nv_bfloat16*>(vT));
+                                                         (int)s.Tp, reinterpret_cast<__nv_bfloat16*>(vT)));
         NSA_TRY(last_launch());
     }
     // tensor maps
@@ -334,15 +386,15 @@ nsa_status_t forward_impl(const Shape& s, const void* q, const void* k, const vo
         NSA_TRY((launch_packed_blk<DK, DV, HG, kModeCmp>(s, mQ, mKc, mVc, pp, st)));
     } else {
         const long long rows = s.B * s.T * s.H;
-        cmp_empty_kernel<<<(unsigned)ceil_div(rows * s.DV, 256), 256, 0, st>>>(out, lse, rows, (int)s.DV);
+        NSA_LAUNCH("cmp_empty_kernel", st, cmp_empty_kernel<<<(unsigned)ceil_div(rows * s.DV, 256), 256, 0, st>>>(out, lse, rows, (int)s.DV));
         NSA_TRY(last_launch());
     }
     // 5. top-n selection
     {
         const long long items = s.B * s.T * s.G;
-        topn_kernel<<<(unsigned)ceil_div(items, 8), 256, 0, st>>>(pscore, items, (int)s.T, (int)s.G,
+        NSA_LAUNCH("topn_kernel", st, topn_kernel<<<(unsigned)ceil_div(items, 8), 256, 0, st>>>(pscore, items, (int)s.T, (int)s.G,
                                                                    (int)s.NSp, (int)s.n, (int)s.lp,
-                                                                   (int)s.fi, (int)s.fl, sel_idx);
+                                                                   (int)s.fi, (int)s.fl, sel_idx));
         NSA_TRY(last_launch());
     }
     // 6. selected attention
@@ -363,7 +415,7 @@ nsa_status_t forward_impl(const Shape& s, const void* q, const void* k, const vo
         using Cfg = SelCfg<DK, DV>;
         NSA_TRY(set_smem(attn_sel_kernel<DK, DV>, Cfg::kSmem));
         dim3 grid((unsigned)ceil_div(s.T, sp.tpc), (unsigned)s.G, (unsigned)s.B);
-        attn_sel_kernel<DK, DV><<<grid, 192, Cfg::kSmem, st>>>(mQs, mK, mVTs, sp);
+        NSA_LAUNCH("attn_sel_kernel", st, attn_sel_kernel<DK, DV><<<grid, 192, Cfg::kSmem, st>>>(mQs, mK, mVTs, sp));
         NSA_TRY(last_launch());
     }
     // 7. sliding window
@@ -476,35 +528,35 @@ nsa_status_t backward_impl(const Shape& s, const void* q, const void* k, const v
     {
         const int smem = (16 * (DK + 1) + 16 * (DV + 1) + 64 * (DK + 1) + 64 * (DV + 1) + 16 * 64 + 16) * 4;
         NSA_TRY(set_smem(bwd_query_kernel<DK, DV>, smem));
-        bwd_query_kernel<DK, DV><<<dim3((unsigned)s.T, (unsigned)s.G, (unsigned)s.B), 256, smem, st>>>(p);
+        NSA_LAUNCH("bwd_query_kernel", st, bwd_query_kernel<DK, DV><<<dim3((unsigned)s.T, (unsigned)s.G, (unsigned)s.B), 256, smem, st>>>(p));
         NSA_TRY(last_launch());
     }
     // inverse index of the selection: block -> tokens
     {
         const long long N = s.B * s.T * s.G * s.n;
-        bwd_sel_count<<<(unsigned)ceil_div(N, 256), 256, 0, st>>>(p);
+        NSA_LAUNCH("bwd_sel_count", st, bwd_sel_count<<<(unsigned)ceil_div(N, 256), 256, 0, st>>>(p));
         NSA_TRY(last_launch());
-        bwd_sel_scan<<<1, 1024, 0, st>>>(p);
+        NSA_LAUNCH("bwd_sel_scan", st, bwd_sel_scan<<<1, 1024, 0, st>>>(p));
         NSA_TRY(last_launch());
-        bwd_sel_fill<<<(unsigned)ceil_div(N, 256), 256, 0, st>>>(p);
+        NSA_LAUNCH("bwd_sel_fill", st, bwd_sel_fill<<<(unsigned)ceil_div(N, 256), 256, 0, st>>>(p));
         NSA_TRY(last_launch());
     }
     // key-centric dK/dV
     {
         dim3 gw((unsigned)ceil_div(s.T, 64), (unsigned)ceil_div(64 + s.w - 1, kBwdChunk), (unsigned)(s.B * s.G));
-        bwd_kv_kernel<DK, DV, kBrWin><<<gw, 256, 0, st>>>(p);
+        NSA_LAUNCH("bwd_kv_kernel", st, bwd_kv_kernel<DK, DV, kBrWin><<<gw, 256, 0, st>>>(p));
         NSA_TRY(last_launch());
         const int64_t maxch = NE + ceil_div(s.B * s.T * s.G * s.n, kBwdChunk);
-        bwd_kv_kernel<DK, DV, kBrSlc><<<(unsigned)maxch, 256, 0, st>>>(p);
+        NSA_LAUNCH("bwd_kv_kernel", st, bwd_kv_kernel<DK, DV, kBrSlc><<<(unsigned)maxch, 256, 0, st>>>(p));
         NSA_TRY(last_launch());
         if (s.C > 0) {
             dim3 gc((unsigned)ceil_div(s.C, 64), (unsigned)ceil_div(s.T, kBwdChunk), (unsigned)(s.B * s.G));
-            bwd_kv_kernel<DK, DV, kBrCmp><<<gc, 256, 0, st>>>(p);
+            NSA_LAUNCH("bwd_kv_kernel", st, bwd_kv_kernel<DK, DV, kBrCmp><<<gc, 256, 0, st>>>(p));
             NSA_TRY(last_launch());
             dim3 gp((unsigned)s.T, (unsigned)s.G, (unsigned)s.B);
-            bwd_phiT_kernel<DK><<<gp, DK, 0, st>>>(p, p.dkc, p.wk, dk);
+            NSA_LAUNCH("bwd_phiT_kernel", st, bwd_phiT_kernel<DK><<<gp, DK, 0, st>>>(p, p.dkc, p.wk, dk));
             NSA_TRY(last_launch());
-            bwd_phiT_kernel<DV><<<gp, DV, 0, st>>>(p, p.dvc, p.wv, dv);
+            NSA_LAUNCH("bwd_phiT_kernel", st, bwd_phiT_kernel<DV><<<gp, DV, 0, st>>>(p, p.dvc, p.wv, dv));
             NSA_TRY(last_launch());
         }
     }
@@ -557,15 +609,15 @@ nsa_status_t decode_impl(const Shape& s, int S, const void* q, const void* kcach
     p.ocmp = carve((size_t)S * s.G * 16 * s.DV * 4);
     p.lsecmp = carve((size_t)S * s.G * 16 * 4);
     p.part2 = carve((size_t)S * s.G * p.NU * 2 * 16 * (2 + s.DV) * 4);
-    dec_cmp_partial<<<dim3((unsigned)p.NSPL, (unsigned)s.G, (unsigned)S), 256, 0, st>>>(p);
+    NSA_LAUNCH("dec_cmp_partial", st, dec_cmp_partial<<<dim3((unsigned)p.NSPL, (unsigned)s.G, (unsigned)S), 256, 0, st>>>(p));
     NSA_TRY(last_launch());
     const int smem2 = (p.Cmax + p.NSmax) * 4;
     NSA_TRY(set_smem(dec_cmp_combine, smem2));
-    dec_cmp_combine<<<dim3((unsigned)s.G, (unsigned)S), 256, smem2, st>>>(p);
+    NSA_LAUNCH("dec_cmp_combine", st, dec_cmp_combine<<<dim3((unsigned)s.G, (unsigned)S), 256, smem2, st>>>(p));
     NSA_TRY(last_launch());
-    dec_slcwin_partial<<<dim3((unsigned)p.NU, (unsigned)s.G, (unsigned)S), 256, 0, st>>>(p);
+    NSA_LAUNCH("dec_slcwin_partial", st, dec_slcwin_partial<<<dim3((unsigned)p.NU, (unsigned)s.G, (unsigned)S), 256, 0, st>>>(p));
     NSA_TRY(last_launch());
-    dec_final<<<dim3((unsigned)s.G, (unsigned)S), 256, 0, st>>>(p);
+    NSA_LAUNCH("dec_final", st, dec_final<<<dim3((unsigned)s.G, (unsigned)S), 256, 0, st>>>(p));
     return last_launch();
 }
 
@@ -682,6 +734,52 @@ nsa_status_t nsa_backward(const nsa_config_t* cfg, const void* q, const void* k,
     if (s.DK == 192)
         return backward_impl<192, 128>(s, q, k, v, gates, phi, dout, sel_idx, dq, dk, dv, dgates, ws, st);
     return backward_impl<64, 64>(s, q, k, v, gates, phi, dout, sel_idx, dq, dk, dv, dgates, ws, st);
+}
+
+nsa_status_t nsa_profile_enable(int32_t on) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_on = on != 0;
+    return NSA_OK;
+}
+
+int32_t nsa_profile_read(int32_t max_kernels, char* names, int32_t* launches, float* total_ms) {
+    std::vector<ProfRec> recs;
+    {
+        std::lock_guard<std::mutex> lk(g_prof_mu);
+        recs.swap(g_prof_recs);
+    }
+    std::vector<std::string> order;
+    std::map<std::string, std::pair<int, double>> agg;
+    int err = 0;
+    for (auto& r : recs) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess)
+            err = 1;
+        std::string n(r.name);
+        if (!agg.count(n)) order.push_back(n);
+        agg[n].first += 1;
+        agg[n].second += ms;
+    }
+    {
+        std::lock_guard<std::mutex> lk(g_prof_mu);
+        for (auto& r : recs) {
+            g_prof_pool.push_back(r.a);
+            g_prof_pool.push_back(r.b);
+        }
+    }
+    if (err) return -1;
+    int32_t k = 0;
+    for (auto& n : order) {
+        if (k >= max_kernels) break;
+        if (names) {
+            std::strncpy(names + 48 * k, n.c_str(), 47);
+            names[48 * k + 47] = 0;
+        }
+        if (launches) launches[k] = agg[n].first;
+        if (total_ms) total_ms[k] = (float)agg[n].second;
+        ++k;
+    }
+    return k;
 }
 
 nsa_status_t nsa_sync_status(void* stream) {

@@ -72,6 +72,10 @@ def lib():
                                    ctypes.c_size_t, _P]
         L.nsa_sync_status.restype = ctypes.c_int
         L.nsa_sync_status.argtypes = [_P]
+        L.nsa_profile_enable.restype = ctypes.c_int
+        L.nsa_profile_enable.argtypes = [ctypes.c_int32]
+        L.nsa_profile_read.restype = ctypes.c_int32
+        L.nsa_profile_read.argtypes = [ctypes.c_int32, ctypes.c_char_p, _P, _P]
         L.nsa_status_string.restype = ctypes.c_char_p
         L.nsa_status_string.argtypes = [ctypes.c_int]
         _lib = L
@@ -230,3 +234,23 @@ def backward(c: dict, q, k, v, gates, dout, idx, phi=None, stream=None) -> dict:
 def sync_status(stream=None):
     """Synchronise and raise if a kernel's bounded wait expired since the last check."""
     _check("nsa_sync_status", lib().nsa_sync_status(_stream(stream)))
+
+
+def profile_enable(on: bool = True):
+    """Bracket every kernel launch of the entry points with CUDA events."""
+    lib().nsa_profile_enable(1 if on else 0)
+
+
+def profile_read(max_kernels: int = 64) -> dict:
+    """{kernel name: (launches, total device ms)} since the previous read."""
+    names = ctypes.create_string_buffer(48 * max_kernels)
+    launches = (ctypes.c_int32 * max_kernels)()
+    ms = (ctypes.c_float * max_kernels)()
+    n = lib().nsa_profile_read(max_kernels, names, ctypes.cast(launches, _P), ctypes.cast(ms, _P))
+    if n < 0:
+        raise NsaError("nsa_profile_read", 4)
+    out = {}
+    for k in range(n):
+        name = names.raw[48 * k:48 * (k + 1)].split(b"\0", 1)[0].decode()
+        out[name] = (int(launches[k]), float(ms[k]))
+    return out

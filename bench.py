@@ -383,6 +383,8 @@ def bench_decode(dev, nsa, peaks, peak_src, steps=50, warmup=5):
     torch.cuda.synchronize(dev)
     nsa.sync_status()
     times = []
+    nsa.profile_read()
+    nsa.profile_enable(True)
     for _ in range(steps):
         flush.zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -391,6 +393,8 @@ def bench_decode(dev, nsa, peaks, peak_src, steps=50, warmup=5):
         e1.record(stream)
         e1.synchronize()
         times.append(e0.elapsed_time(e1))
+    nsa.profile_enable(False)
+    prof = nsa.profile_read()
     ms = statistics.median(times)
     # unique bytes read: compressed cache rows + the tokens of (selected U window) blocks
     idx = buf.idx.cpu().numpy()
@@ -412,6 +416,7 @@ def bench_decode(dev, nsa, peaks, peak_src, steps=50, warmup=5):
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
                          "peak_source": f"{peak_src} copy bandwidth", "frac_of_8TBs": round(gbs / 8000, 4)},
+            "kernels": {k: {"launches": n, "us_per_step": round(1e3 * t / steps, 2)} for k, (n, t) in prof.items()},
             "l2": "flushed (512 MB write) before each timed step"}
 
 
@@ -433,17 +438,22 @@ def bench_backward(dev, nsa, peaks, steps=2, warmup=1):
     for _ in range(steps):
         nsa.forward_into(c, x["q"], x["k"], x["v"], x["gates"], phi, fb, stream)
     e1.record(stream)
+    nsa.profile_read()
+    nsa.profile_enable(True)
     for _ in range(steps):
         nsa.backward(c, x["q"], x["k"], x["v"], x["gates"], x["dout"], fb.idx, phi)
     e2.record(stream)
     torch.cuda.synchronize(dev)
+    nsa.profile_enable(False)
+    prof = nsa.profile_read()
     f_ms, b_ms = e0.elapsed_time(e1) / steps, e1.elapsed_time(e2) / steps
     _, fwd = forward_flops(c)
     bwd = 2 * fwd                               # dP, dV, dQ, dK
     return {"workload": "train_fwd_bwd_B2_T16384", "fwd_ms": round(f_ms, 3), "bwd_ms": round(b_ms, 3),
             "tokens_per_s": round(c["B"] * c["T"] / ((f_ms + b_ms) / 1e3), 1),
             "bwd_tflops_algorithmic": round(bwd / (b_ms / 1e3) / 1e12, 2),
-            "bwd_frac_of_peak": round(bwd / (b_ms / 1e3) / 1e12 / peaks.get("bf16_tflops", 1590.0), 4)}
+            "bwd_frac_of_peak": round(bwd / (b_ms / 1e3) / 1e12 / peaks.get("bf16_tflops", 1590.0), 4),
+            "kernels": {k: {"launches": n, "ms_per_step": round(t / steps, 3)} for k, (n, t) in prof.items()}}
 
 
 def run_reference(args, c, rank, world, tokens_per_step):

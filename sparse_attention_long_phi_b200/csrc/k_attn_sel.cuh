@@ -11,11 +11,13 @@
 // One softmax runs over the union of the selected blocks' tokens u <= t.
 // out[t, h] += g_slc * O / l;  lse[..., 1] = natural-log LSE.
 //
-// A CTA walks a range of tokens of one group.  Warp 4 streams Q_t and the
-// K/V block pairs through a ring; warp 5 issues MMAs in the skewed order
-// S(0) S(1) O(0) S(2) O(1) ... so the next token's S^T overlaps the current
-// token's softmax; warps 0-3 run the softmax (thread = key of a pair for S^T,
-// value channel for O^T) and the epilogue.
+// A CTA walks a range of tokens of one group (CTAs ordered group-major so a
+// group's keys/values stay in L2).  Warp 8 streams Q_t and the K/V block
+// pairs through a ring; warp 9 issues the MMAs in the skewed order
+// S(0) S(1) O(0) S(2) O(1) ...; two softmax warpgroups (warps 0-3 and 4-7)
+// take alternate tokens, each with its own S^T / O^T TMEM buffers and P^T
+// tile, so one group's softmax and epilogue overlap the other's.  In a
+// softmax warpgroup thread = key of a pair for S^T, value channel for O^T.
 #pragma once
 #include "nsa_dev.cuh"
 #include "k_attn_packed.cuh"
@@ -31,6 +33,7 @@ struct SelParams {
     float* out;                 // [B,T,H,DV] accumulated
     float* lse_user;            // [B,T,H,3] or null
     int tpc;                    // tokens per CTA
+    int nchunks;                // token chunks per group: grid.x = G * nchunks, group-major
 };
 
 template <int DK, int DV>
@@ -46,23 +49,30 @@ struct SelCfg {
     static constexpr int kOffKV = ((2 * kQSlot + 1023) / 1024) * 1024;
     static constexpr int kOffP = kOffKV + NSLOT * kSlot;
     static constexpr int kPBytes = 16 * 2048;             // 16 heads x 1024 keys
-    static constexpr int kOffRed = kOffP + kPBytes;
-    static constexpr int kOffBar = kOffRed + 2 * 4 * 16 * 4;
+    static constexpr int kOffRed = kOffP + 2 * kPBytes;   // one P^T tile per warpgroup
+    static constexpr int kRedBytes = 2 * (2 * 4 * 16 * 4 + 16 * 4);
+    static constexpr int kOffBar = kOffRed + kRedBytes;
     static constexpr int kSmem = kOffBar + 256 + 1024;
+    static constexpr int kThreads = 320;
 };
 
-__device__ __forceinline__ int load_units(const int32_t* row, int n, int (&u)[16]) {
+// order-preserving map of fp32 to u32 (for integer max reductions)
+__device__ __forceinline__ uint32_t f2ord(float f) {
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float ord2f(uint32_t u) {
+    return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+
+__device__ __forceinline__ int count_units(const int32_t* row, int n) {
     int nu = 0;
-#pragma unroll
-    for (int a = 0; a < 16; ++a) {
-        int j = a < n ? row[a] : -1;
-        if (j >= 0) u[nu++] = j;
-    }
+    for (int a = 0; a < n; ++a) nu += row[a] >= 0;
     return nu;
 }
 
-template <int DK, int DV>
-__global__ void __launch_bounds__(192, 1)
+template <int DK, int DV, int HG>
+__global__ void __launch_bounds__(320, 1)
     attn_sel_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                     const __grid_constant__ CUtensorMap mapV, const SelParams p) {
     using Cfg = SelCfg<DK, DV>;
@@ -70,24 +80,22 @@ __global__ void __launch_bounds__(192, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
-    uint64_t* qfull = bars + 0;    // [2]
+    uint64_t* qfull = bars + 0;    // [2]  per token parity
     uint64_t* qempty = bars + 2;   // [2]
     uint64_t* full = bars + 4;     // [NSLOT]
     uint64_t* empty = bars + 7;    // [NSLOT]
-    uint64_t* sfull = bars + 10;   // [2]
+    uint64_t* sfull = bars + 10;   // [2]  per warpgroup
     uint64_t* sfree = bars + 12;   // [2]
-    uint64_t* pfull = bars + 14;
-    uint64_t* ofull = bars + 15;   // [2]
-    uint64_t* ofree = bars + 17;   // [2]
+    uint64_t* pfull = bars + 14;   // [2]
+    uint64_t* ofull = bars + 16;   // [2]
+    uint64_t* ofree = bars + 18;   // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 21);
-    float* redm = reinterpret_cast<float*>(smem + Cfg::kOffRed);
-    float* redl = redm + 64;
+    int* npairs_ring = reinterpret_cast<int*>(bars + 22);   // [4] producer -> MMA
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int g = blockIdx.y, b = blockIdx.z;
-    const int HG = p.H / p.G;
-    const int tb = blockIdx.x * p.tpc;
+    const int g = blockIdx.x / p.nchunks, b = blockIdx.z;
+    const int tb = (blockIdx.x % p.nchunks) * p.tpc;
     const int N = min(p.tpc, p.T - tb);
 
     if (threadIdx.x == 0) {
@@ -96,6 +104,7 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(&qempty[s], 1);
             mbar_init(&sfull[s], 1);
             mbar_init(&sfree[s], 4);
+            mbar_init(&pfull[s], 128);
             mbar_init(&ofull[s], 1);
             mbar_init(&ofree[s], 4);
         }
@@ -103,11 +112,10 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(pfull, 128);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == 9) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
@@ -117,14 +125,13 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t tmem = *tmem_slot;
     const int32_t* idx_base = p.idx + ((size_t)b * p.T * p.G + g) * p.n;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ------------------------------------------------------ producer
         if (lane == 0 && N > 0) {
             tma_prefetch_desc(&mapQ);
             tma_prefetch_desc(&mapK);
             tma_prefetch_desc(&mapV);
             uint32_t cnt = 0;
-            bool ok = true;
             auto slot_acquire = [&](uint32_t c) -> uint8_t* {
                 const int sl = c % Cfg::NSLOT;
                 if (c >= Cfg::NSLOT &&
@@ -132,59 +139,68 @@ __global__ void __launch_bounds__(192, 1)
                     return nullptr;
                 return smem + Cfg::kOffKV + sl * Cfg::kSlot;
             };
-            auto load_S = [&](int i) -> bool {
-                const int t = tb + i;
-                const int qs = i & 1;
-                if (i >= 2 && !wait_or_abort(&qempty[qs], ((i - 2) >> 1) & 1, 0x302, abort_flag))
-                    return false;
-                mbar_expect_tx(&qfull[qs], Cfg::kQSlot);
-                for (int bx = 0; bx < Cfg::NQB; ++bx)
-                    tma_load_4d(smem + Cfg::kOffQ + qs * Cfg::kQSlot + bx * 2048, &mapQ, &qfull[qs],
-                                bx * 64, g * HG, t, b);
+            auto load_pairs = [&](int i, bool kv_is_k) -> bool {
+                const int32_t* row = idx_base + (size_t)(tb + i) * p.G * p.n;
                 int u[16];
-                const int nu = load_units(idx_base + (size_t)t * p.G * p.n, p.n, u);
+                int nu = 0;
+#pragma unroll
+                for (int a = 0; a < 16; ++a) {
+                    const int j = a < p.n ? row[a] : -1;
+                    u[a] = j;
+                    nu += j >= 0;
+                }
+                // the selection is ascending with -1 padding: valid entries come first
                 for (int pp = 0; pp < (nu + 1) / 2; ++pp) {
-                    const int ja = u[2 * pp], jb = (2 * pp + 1 < nu) ? u[2 * pp + 1] : ja;
+                    int ja = 0, jb = 0;
+#pragma unroll
+                    for (int a = 0; a < 16; ++a) {
+                        if (a == 2 * pp) ja = u[a];
+                        if (a == 2 * pp + 1) jb = u[a];
+                    }
+                    if (2 * pp + 1 >= nu) jb = ja;
                     uint8_t* sl = slot_acquire(cnt);
                     if (!sl) return false;
                     uint64_t* bar = &full[cnt % Cfg::NSLOT];
-                    mbar_expect_tx(bar, Cfg::kKPair);
-                    for (int bx = 0; bx < Cfg::NQB; ++bx) {
-                        tma_load_4d(sl + bx * 16384, &mapK, bar, bx * 64, g, ja * 64, b);
-                        tma_load_4d(sl + bx * 16384 + 8192, &mapK, bar, bx * 64, g, jb * 64, b);
+                    if (kv_is_k) {
+                        mbar_expect_tx(bar, Cfg::kKPair);
+                        for (int bx = 0; bx < Cfg::NQB; ++bx) {
+                            tma_load_4d(sl + bx * 16384, &mapK, bar, bx * 64, g, ja * 64, b);
+                            tma_load_4d(sl + bx * 16384 + 8192, &mapK, bar, bx * 64, g, jb * 64, b);
+                        }
+                    } else {
+                        mbar_expect_tx(bar, Cfg::kVPair);
+                        tma_load_4d(sl, &mapV, bar, ja * 64, 0, g, b);
+                        tma_load_4d(sl + Cfg::DVM * 128, &mapV, bar, jb * 64, 0, g, b);
                     }
                     ++cnt;
                 }
                 return true;
             };
-            auto load_O = [&](int i) -> bool {
-                const int t = tb + i;
-                int u[16];
-                const int nu = load_units(idx_base + (size_t)t * p.G * p.n, p.n, u);
-                for (int pp = 0; pp < (nu + 1) / 2; ++pp) {
-                    const int ja = u[2 * pp], jb = (2 * pp + 1 < nu) ? u[2 * pp + 1] : ja;
-                    uint8_t* sl = slot_acquire(cnt);
-                    if (!sl) return false;
-                    uint64_t* bar = &full[cnt % Cfg::NSLOT];
-                    mbar_expect_tx(bar, Cfg::kVPair);
-                    tma_load_4d(sl, &mapV, bar, ja * 64, 0, g, b);
-                    tma_load_4d(sl + Cfg::DVM * 128, &mapV, bar, jb * 64, 0, g, b);
-                    ++cnt;
-                }
-                return true;
+            auto load_S = [&](int i) -> bool {
+                const int qs = i & 1;
+                if (i >= 2 && !wait_or_abort(&qempty[qs], ((i - 2) >> 1) & 1, 0x302, abort_flag))
+                    return false;
+                const int32_t* row = idx_base + (size_t)(tb + i) * p.G * p.n;
+                npairs_ring[i & 3] = (count_units(row, p.n) + 1) / 2;   // read by the MMA warp
+                mbar_expect_tx(&qfull[qs], Cfg::kQSlot);                // (release)
+                for (int bx = 0; bx < Cfg::NQB; ++bx)
+                    tma_load_4d(smem + Cfg::kOffQ + qs * Cfg::kQSlot + bx * 2048, &mapQ, &qfull[qs],
+                                bx * 64, g * HG, tb + i, b);
+                return load_pairs(i, true);
             };
-            ok = load_S(0);
+            bool ok = load_S(0);
             for (int i = 1; i < N && ok; ++i) {
                 ok = load_S(i);
-                if (ok) ok = load_O(i - 1);
+                if (ok) ok = load_pairs(i - 1, false);
             }
-            if (ok) load_O(N - 1);
+            if (ok) load_pairs(N - 1, false);
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ----------------------------------------------------------- MMA
         if (lane == 0 && N > 0) {
             constexpr uint32_t id16 = idesc_bf16(128, 16);
             uint32_t cnt = 0;
+            int np_of[2] = {0, 0};
             auto slot_wait = [&](uint32_t c) -> uint32_t {
                 const int sl = c % Cfg::NSLOT;
                 if (!wait_or_abort(&full[sl], (c / Cfg::NSLOT) & 1, 0x303, abort_flag)) return 0;
@@ -192,54 +208,51 @@ __global__ void __launch_bounds__(192, 1)
                 return smem_u32(smem + Cfg::kOffKV + sl * Cfg::kSlot);
             };
             auto do_S = [&](int i) -> bool {
-                const int t = tb + i;
-                const int qs = i & 1;
+                const int qs = i & 1, wg = i & 1;
                 if (!wait_or_abort(&qfull[qs], (i >> 1) & 1, 0x304, abort_flag)) return false;
-                if (i >= 2 && !wait_or_abort(&sfree[qs], ((i - 2) >> 1) & 1, 0x305, abort_flag))
+                const int np = npairs_ring[i & 3];
+                np_of[i & 1] = np;
+                if (i >= 2 && !wait_or_abort(&sfree[wg], ((i - 2) >> 1) & 1, 0x305, abort_flag))
                     return false;
                 tc_fence_after();
                 const uint32_t sQ = smem_u32(smem + Cfg::kOffQ + qs * Cfg::kQSlot);
-                int u[16];
-                const int nu = load_units(idx_base + (size_t)t * p.G * p.n, p.n, u);
-                for (int pp = 0; pp < (nu + 1) / 2; ++pp) {
+                for (int pp = 0; pp < np; ++pp) {
                     const uint32_t sK = slot_wait(cnt);
                     if (!sK) return false;
 #pragma unroll
                     for (int kk = 0; kk < DK / 16; ++kk)
-                        umma_bf16_ss(tmem + qs * 128 + pp * 16,
+                        umma_bf16_ss(tmem + wg * 128 + pp * 16,
                                      sdesc_sw128(sK + (kk / 4) * 16384 + (kk % 4) * 32),
                                      sdesc_sw128(sQ + (kk / 4) * 2048 + (kk % 4) * 32), id16,
                                      kk > 0 ? 1u : 0u);
                     umma_commit(&empty[cnt % Cfg::NSLOT]);
                     ++cnt;
                 }
-                umma_commit(&sfull[qs]);
+                umma_commit(&sfull[wg]);
                 umma_commit(&qempty[qs]);
                 return true;
             };
             auto do_O = [&](int i) -> bool {
-                const int t = tb + i;
-                const int ob = i & 1;
-                if (!wait_or_abort(pfull, i & 1, 0x306, abort_flag)) return false;
-                if (i >= 2 && !wait_or_abort(&ofree[ob], ((i - 2) >> 1) & 1, 0x307, abort_flag))
+                const int wg = i & 1;
+                if (!wait_or_abort(&pfull[wg], (i >> 1) & 1, 0x306, abort_flag)) return false;
+                if (i >= 2 && !wait_or_abort(&ofree[wg], ((i - 2) >> 1) & 1, 0x307, abort_flag))
                     return false;
                 tc_fence_after();
-                const uint32_t sP = smem_u32(smem + Cfg::kOffP);
-                int u[16];
-                const int nu = load_units(idx_base + (size_t)t * p.G * p.n, p.n, u);
-                for (int pp = 0; pp < (nu + 1) / 2; ++pp) {
+                const uint32_t sP = smem_u32(smem + Cfg::kOffP + wg * Cfg::kPBytes);
+                const int np = np_of[i & 1];
+                for (int pp = 0; pp < np; ++pp) {
                     const uint32_t sV = slot_wait(cnt);
                     if (!sV) return false;
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        umma_bf16_ss(tmem + 256 + ob * 16,
+                        umma_bf16_ss(tmem + 256 + wg * 16,
                                      sdesc_sw128(sV + (kk / 4) * (Cfg::DVM * 128) + (kk % 4) * 32),
                                      sdesc_sw128(sP + (2 * pp + kk / 4) * 2048 + (kk % 4) * 32),
                                      id16, (pp > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&empty[cnt % Cfg::NSLOT]);
                     ++cnt;
                 }
-                umma_commit(&ofull[ob]);
+                umma_commit(&ofull[wg]);
                 return true;
             };
             bool ok = do_S(0);
@@ -250,62 +263,76 @@ __global__ void __launch_bounds__(192, 1)
             if (ok) do_O(N - 1);
         }
     } else {
-        // ------------------------------------------------ softmax / epilogue
-        const int kl = threadIdx.x;                  // key within a pair / value channel
+        // ------------------------------------- softmax / epilogue (2 groups)
+        const int wg = warp >> 2;                 // warpgroup: tokens i with i % 2 == wg
+        const int wq = warp & 3;                  // TMEM lane quadrant
+        const int kl = wq * 32 + lane;            // key within a pair / value channel
         const int unit_off = kl >> 6, tok_off = kl & 63;
-        const uint32_t lanebase = tmem + ((uint32_t)(warp * 32) << 16);
-        const uint32_t sP = smem_u32(smem + Cfg::kOffP);
+        const uint32_t lanebase = tmem + ((uint32_t)(wq * 32) << 16);
+        const uint32_t sP = smem_u32(smem + Cfg::kOffP + wg * Cfg::kPBytes);
+        float* redm = reinterpret_cast<float*>(smem + Cfg::kOffRed + wg * (Cfg::kRedBytes / 2));
+        float* redl = redm + 64;
+        int* su = reinterpret_cast<int*>(redl + 64);          // [16] block ids of the token
+        const uint32_t bar_id = 1 + wg;
         bool ok = true;
-        for (int i = 0; i < N; ++i) {
+        int it = 0;
+        for (int i = wg; i < N; i += 2, ++it) {
             const int t = tb + i;
-            const int sb = i & 1;
-            int u[16];
-            const int nu = load_units(idx_base + (size_t)t * p.G * p.n, p.n, u);
+            const int32_t* row = idx_base + (size_t)t * p.G * p.n;
+            if (kl < 16) su[kl] = kl < p.n ? row[kl] : -1;
+            // per-head gates of the token (loaded early, used in the epilogue)
+            float gate[HG];
+            const size_t rowbase = ((size_t)b * p.T + t) * p.H + (size_t)g * HG;
+#pragma unroll
+            for (int h = 0; h < HG; ++h) gate[h] = __ldg(p.gates + (rowbase + h) * 3 + 1);
+            named_bar_sync(bar_id, 128);
+            int nu = 0;
+#pragma unroll
+            for (int a = 0; a < 16; ++a) nu += su[a] >= 0;
             const int npairs = (nu + 1) / 2;
-            if (ok) ok = wait_or_abort(&sfull[sb], (i >> 1) & 1, 0x308, abort_flag);
+            if (ok) ok = wait_or_abort(&sfull[wg], it & 1, 0x308, abort_flag);
             tc_fence_after();
+            // pass A: per-head max over the valid keys
             float mx[16];
 #pragma unroll
             for (int h = 0; h < 16; ++h) mx[h] = -INFINITY;
             for (int pp = 0; pp < npairs; ++pp) {
                 uint32_t r[16];
-                tmem_ld16(lanebase + sb * 128 + pp * 16, r);
+                tmem_ld16(lanebase + wg * 128 + pp * 16, r);
                 tmem_wait_ld16(r);
                 const int un = 2 * pp + unit_off;
-                const bool valid = un < nu && (un < 16 ? (u[un] * 64 + tok_off <= t) : false);
+                const bool valid = un < nu && su[un] * 64 + tok_off <= t;
                 if (valid) {
 #pragma unroll
-                    for (int h = 0; h < 16; ++h) mx[h] = fmaxf(mx[h], __uint_as_float(r[h]) * p.scale_log2);
+                    for (int h = 0; h < 16; ++h) mx[h] = fmaxf(mx[h], __uint_as_float(r[h]));
                 }
             }
 #pragma unroll
-            for (int h = 0; h < 16; ++h) {
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], o));
+            for (int h = 0; h < HG; ++h) {
+                const uint32_t m = __reduce_max_sync(0xffffffffu, f2ord(mx[h]));
+                if (lane == 0) redm[wq * 16 + h] = ord2f(m);
             }
-            if (lane == 0)
+            named_bar_sync(bar_id, 128);
 #pragma unroll
-                for (int h = 0; h < 16; ++h) redm[warp * 16 + h] = mx[h];
-            named_bar_sync(1, 128);
-#pragma unroll
-            for (int h = 0; h < 16; ++h)
-                mx[h] = fmaxf(fmaxf(redm[h], redm[16 + h]), fmaxf(redm[32 + h], redm[48 + h]));
+            for (int h = 0; h < HG; ++h)
+                mx[h] = fmaxf(fmaxf(redm[h], redm[16 + h]), fmaxf(redm[32 + h], redm[48 + h])) * p.scale_log2;
+            // pass B: P = exp2(s - m), P^T to shared memory (bf16), per-head sums
             float ls[16];
 #pragma unroll
             for (int h = 0; h < 16; ++h) ls[h] = 0.f;
             for (int pp = 0; pp < npairs; ++pp) {
                 uint32_t r[16];
-                tmem_ld16(lanebase + sb * 128 + pp * 16, r);
+                tmem_ld16(lanebase + wg * 128 + pp * 16, r);
                 tmem_wait_ld16(r);
                 const int un = 2 * pp + unit_off;
-                const bool valid = un < nu && (un < 16 ? (u[un] * 64 + tok_off <= t) : false);
+                const bool valid = un < nu && su[un] * 64 + tok_off <= t;
                 const int key = pp * 128 + kl;
                 const uint32_t cbase = sP + (key >> 6) * 2048;
                 const int kk = key & 63;
 #pragma unroll
                 for (int h = 0; h < 16; ++h) {
                     float e = 0.f;
-                    if (valid && mx[h] != -INFINITY) e = exp2f(__uint_as_float(r[h]) * p.scale_log2 - mx[h]);
+                    if (h < HG && valid) e = exp2f(__uint_as_float(r[h]) * p.scale_log2 - mx[h]);
                     ls[h] += e;
                     __nv_bfloat16 eb = __float2bfloat16_rn(e);
                     st_shared_u16(cbase + sw128_off(h, kk >> 3) + (kk & 7) * 2,
@@ -314,47 +341,51 @@ __global__ void __launch_bounds__(192, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sfree[sb]);
+            if (lane == 0) mbar_arrive(&sfree[wg]);
             fence_proxy_async_smem();
-            mbar_arrive(pfull);
-#pragma unroll
-            for (int h = 0; h < 16; ++h) {
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) ls[h] += __shfl_xor_sync(0xffffffffu, ls[h], o);
+            mbar_arrive(&pfull[wg]);
+            // per-head sums: reduce-scatter over the warp, then across the 4 warps
+            {
+                const int base = reduce_scatter_heads<16, 16>(ls, lane);   // lanes l, l^16 hold head base
+                const float v = ls[0] + __shfl_xor_sync(0xffffffffu, ls[0], 16);
+                if (lane < 16) redl[wq * 16 + base] = v;
             }
-            if (lane == 0)
+            named_bar_sync(bar_id, 128);
 #pragma unroll
-                for (int h = 0; h < 16; ++h) redl[warp * 16 + h] = ls[h];
-            named_bar_sync(1, 128);
-#pragma unroll
-            for (int h = 0; h < 16; ++h) ls[h] = redl[h] + redl[16 + h] + redl[32 + h] + redl[48 + h];
+            for (int h = 0; h < HG; ++h) ls[h] = redl[h] + redl[16 + h] + redl[32 + h] + redl[48 + h];
 
             // O^T: lane = value channel kl, columns = heads
-            if (ok) ok = wait_or_abort(&ofull[sb], (i >> 1) & 1, 0x309, abort_flag);
+            if (ok) ok = wait_or_abort(&ofull[wg], it & 1, 0x309, abort_flag);
             tc_fence_after();
             uint32_t r[16];
-            tmem_ld16(lanebase + 256 + sb * 16, r);
+            tmem_ld16(lanebase + 256 + wg * 16, r);
             tmem_wait_ld16(r);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&ofree[sb]);
+            if (lane == 0) mbar_arrive(&ofree[wg]);
             if (ok && kl < DV) {
+                float prev[HG];
+#pragma unroll
+                for (int h = 0; h < HG; ++h) prev[h] = p.out[(rowbase + h) * DV + kl];
+#pragma unroll
                 for (int h = 0; h < HG; ++h) {
-                    const size_t rowid = ((size_t)b * p.T + t) * p.H + g * HG + h;
-                    const float gate = p.gates[rowid * 3 + 1];
                     const float o = ls[h] > 0.f ? __uint_as_float(r[h]) / ls[h] : 0.f;
-                    p.out[rowid * DV + kl] += gate * o;
+                    p.out[(rowbase + h) * DV + kl] = prev[h] + gate[h] * o;
                 }
             }
-            if (ok && kl < HG && p.lse_user) {
-                const size_t rowid = ((size_t)b * p.T + t) * p.H + g * HG + kl;
-                p.lse_user[rowid * 3 + 1] = ls[kl] > 0.f ? (mx[kl] + log2f(ls[kl])) * kLn2 : -INFINITY;
+            if (ok && p.lse_user && kl < HG) {
+                float lv = -INFINITY;
+#pragma unroll
+                for (int h = 0; h < HG; ++h)
+                    if (h == kl) lv = ls[h] > 0.f ? (mx[h] + log2f(ls[h])) * kLn2 : -INFINITY;
+                p.lse_user[(rowbase + kl) * 3 + 1] = lv;
             }
+            named_bar_sync(bar_id, 128);   // su / red reuse by the next token
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }

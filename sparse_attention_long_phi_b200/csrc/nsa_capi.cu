@@ -186,7 +186,7 @@ FwdWs fwd_layout(const Shape& s) {
     w.off_vt = o;
     o = align256(o + (size_t)s.B * s.G * s.DVP * s.Tp * 2);
     w.off_bias = o;
-    o = align256(o + (size_t)(s.DK + s.DV) * 4);
+    o = align256(o + (size_t)(s.DK + s.DV) * 8);
     w.off_lse = o;
     o = align256(o + (size_t)s.B * s.T * s.H * 4);
     w.off_ps = o;
@@ -218,7 +218,7 @@ nsa_status_t set_smem(K kernel, int bytes) {
 // ------------------------------------------------------------------- phi
 template <int D>
 nsa_status_t launch_phi_linear(const Shape& s, const void* x, const void* W, const void* E,
-                               const float* bias, void* y, void* yT, uint32_t* fix_list,
+                               const double* bias, void* y, void* yT, uint32_t* fix_list,
                                unsigned int* fix_count, cudaStream_t st) {
     CUtensorMap mA, mW;
     const uint64_t dA[5] = {(uint64_t)D, (uint64_t)s.G, (uint64_t)s.d, (uint64_t)(s.T / s.d), (uint64_t)s.B};
@@ -227,10 +227,10 @@ nsa_status_t launch_phi_linear(const Shape& s, const void* x, const void* W, con
     const uint32_t bA[5] = {64, 1, 1, 128, 1};
     const uint64_t dW[2] = {(uint64_t)s.l * D, (uint64_t)D};
     const uint64_t sW[1] = {(uint64_t)s.l * D * 2};
-    const uint32_t bW[2] = {64, (uint32_t)D};
+    const uint32_t bW[2] = {64, (uint32_t)(D / 2)};
     if (!make_map(&mA, x, 5, dA, sA, bA) || !make_map(&mW, W, 2, dW, sW, bW)) return NSA_ERR_CUDA;
     NSA_TRY(set_smem(phi_linear_kernel<D>, PhiGemmCfg<D>::kSmem));
-    dim3 grid((unsigned)ceil_div(s.C, 128), (unsigned)s.G, (unsigned)s.B);
+    dim3 grid((unsigned)ceil_div(s.C, 128), (unsigned)(2 * s.G), (unsigned)s.B);
     NSA_LAUNCH("phi_linear_kernel", st, phi_linear_kernel<D><<<grid, 192, PhiGemmCfg<D>::kSmem, st>>>(
         mA, mW, bias, (int)s.l, (int)s.d, (int)s.C, (int)s.Cp, (int)s.G,
         reinterpret_cast<__nv_bfloat16*>(y), reinterpret_cast<__nv_bfloat16*>(yT), fix_list, fix_count));
@@ -245,7 +245,7 @@ nsa_status_t launch_phi_linear(const Shape& s, const void* x, const void* W, con
 
 // K~ -> kc [B,C,G,DK]; V~ -> vcT [B,G,DV,Cp] (+ vc [B,C,G,DV] if given)
 nsa_status_t run_phi(const Shape& s, const void* k, const void* v, const nsa_phi_params_t* phi,
-                     void* kc, void* vc, void* vcT, float* bias, uint8_t* fix, cudaStream_t st) {
+                     void* kc, void* vc, void* vcT, double* bias, uint8_t* fix, cudaStream_t st) {
     if (s.C == 0) return NSA_OK;
     if (s.phi == NSA_PHI_MEAN) {
         dim3 grid((unsigned)s.C, (unsigned)s.G, (unsigned)s.B);
@@ -321,7 +321,7 @@ nsa_status_t forward_impl(const Shape& s, const void* q, const void* k, const vo
     void* kc = kc_out ? kc_out : ws + L.off_kc;
     void* vcT = ws + L.off_vct;
     void* vT = ws + L.off_vt;
-    float* bias = reinterpret_cast<float*>(ws + L.off_bias);
+    double* bias = reinterpret_cast<double*>(ws + L.off_bias);
     float* lse_cmp = reinterpret_cast<float*>(ws + L.off_lse);
     float* pscore = reinterpret_cast<float*>(ws + L.off_ps);
 
@@ -413,9 +413,10 @@ nsa_status_t forward_impl(const Shape& s, const void* q, const void* k, const vo
         int64_t tpc = (s.B * s.T * s.G) / (148 * 8);
         sp.tpc = (int)std::min<int64_t>(64, std::max<int64_t>(4, tpc));
         using Cfg = SelCfg<DK, DV>;
-        NSA_TRY(set_smem(attn_sel_kernel<DK, DV>, Cfg::kSmem));
-        dim3 grid((unsigned)ceil_div(s.T, sp.tpc), (unsigned)s.G, (unsigned)s.B);
-        NSA_LAUNCH("attn_sel_kernel", st, attn_sel_kernel<DK, DV><<<grid, 192, Cfg::kSmem, st>>>(mQs, mK, mVTs, sp));
+        NSA_TRY(set_smem(attn_sel_kernel<DK, DV, HG>, Cfg::kSmem));
+        sp.nchunks = (int)ceil_div(s.T, sp.tpc);
+        dim3 grid((unsigned)(sp.nchunks * s.G), 1, (unsigned)s.B);
+        NSA_LAUNCH("attn_sel_kernel", st, attn_sel_kernel<DK, DV, HG><<<grid, Cfg::kThreads, Cfg::kSmem, st>>>(mQs, mK, mVTs, sp));
         NSA_TRY(last_launch());
     }
     // 7. sliding window
@@ -442,7 +443,7 @@ BwdWs bwd_layout(const Shape& s) {
     w.off_vct = o;
     o = align256(o + (size_t)s.B * s.G * s.DV * s.Cp * 2);
     w.off_bias = o;
-    o = align256(o + (size_t)(s.DK + s.DV) * 4);
+    o = align256(o + (size_t)(s.DK + s.DV) * 8);
     w.off_lse2 = o;
     o = align256(o + (size_t)s.B * s.T * s.H * 3 * 4);
     w.off_dlt = o;
@@ -518,7 +519,7 @@ nsa_status_t backward_impl(const Shape& s, const void* q, const void* k, const v
 
     // compressed keys/values of the forward (row layout)
     NSA_TRY(run_phi(s, k, v, phi, ws + L.off_kc, ws + L.off_vc, ws + L.off_vct,
-                    reinterpret_cast<float*>(ws + L.off_bias), ws + L.off_fix, st));
+                    reinterpret_cast<double*>(ws + L.off_bias), ws + L.off_fix, st));
     if (cudaMemsetAsync(dk, 0, (size_t)s.B * s.T * s.G * DK * 4, st) != cudaSuccess ||
         cudaMemsetAsync(dv, 0, (size_t)s.B * s.T * s.G * DV * 4, st) != cudaSuccess ||
         cudaMemsetAsync(ws + L.off_dkc, 0, L.off_cnt - L.off_dkc, st) != cudaSuccess ||
@@ -665,7 +666,7 @@ nsa_status_t nsa_compress(const nsa_config_t* cfg, const void* k, const void* v,
     if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
         return NSA_ERR_WORKSPACE;
     uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
-    return run_phi(s, k, v, phi, kc, vc, ws + L.off_vct, reinterpret_cast<float*>(ws + L.off_bias),
+    return run_phi(s, k, v, phi, kc, vc, ws + L.off_vct, reinterpret_cast<double*>(ws + L.off_bias),
                    ws + L.off_fix, reinterpret_cast<cudaStream_t>(stream));
 }
 

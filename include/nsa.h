@@ -107,6 +107,28 @@ nsa_status_t nsa_compress(const nsa_config_t* cfg, const void* k, const void* v,
                           const nsa_phi_params_t* phi, void* kc, void* vc, void* workspace,
                           size_t workspace_bytes, void* stream);
 
+/* Token compression without any device allocation.  No counterpart in the
+ * paper: this entry point exists for callers that cannot call cudaMalloc or
+ * hand over a workspace -- code running inside CUDA graph capture, plugins
+ * hosted by a framework that owns all device memory, or a serving loop that
+ * must not allocate per step while it appends compressed blocks to its
+ * cache.  It computes exactly what nsa_compress computes (same kernels, same
+ * outputs), with its scratch in a fixed 16 MiB device array compiled into
+ * the library (held by every GPU that loads it, until process exit):
+ *   - sizes: 8*(d_k + d_v) rounded up to 256, plus 256 + 4*B*C*G*(d_k + d_v)
+ *     bytes must fit in 16 MiB, otherwise NSA_ERR_WORKSPACE is returned and
+ *     nothing is launched (e.g. B=1, G=4, d_k+d_v=320 allows up to about
+ *     T=52k tokens);
+ *   - the first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before
+ *     any stream capture;
+ *   - all calls share the array: two calls whose kernels overlap on the GPU
+ *     (different streams, or different host threads on one device) race;
+ *     serialise them.  Each call clears the counters it needs.
+ * Arguments as in nsa_compress, without the workspace. */
+nsa_status_t nsa_compress_static(const nsa_config_t* cfg, const void* k, const void* v,
+                                 const nsa_phi_params_t* phi, void* kc, void* vc, void* stream);
+
 /* Prefill forward (page 2, sections 整体框架 / 算法设计 / 最终输出计算).
  * In:  q [B,T,H,d_k], k [B,T,G,d_k], v [B,T,G,d_v] bf16; gates [B,T,H,3] fp32
  *      in the order (compressed, selected, window), the sigmoid outputs.

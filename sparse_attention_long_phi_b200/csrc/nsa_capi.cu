@@ -796,3 +796,52 @@ nsa_status_t nsa_sync_status(void* stream) {
 }
 
 }  // extern "C"
+
+// ===================================================== allocation-free compress
+//
+// nsa_compress_static: token compression for callers that cannot allocate
+// device memory.  Its scratch (the fp64 position-embedding bias and the list
+// of elements re-rounded exactly) lives in the fixed array below instead of a
+// caller workspace.  The array is a host-side stand-in in host code; its
+// device address is fetched with cudaGetSymbolAddress once per device, the
+// first time the entry point runs with that device current.
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;   // 16 MiB on every device that loads the library
+__device__ __align__(256) uint8_t g_compress_scratch[kStaticScratchBytes];
+
+std::mutex g_static_mu;
+void* g_static_scratch[128] = {};
+
+nsa_status_t static_scratch_ptr(void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return NSA_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_static_mu);
+    if (!g_static_scratch[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_compress_scratch) != cudaSuccess || !p) return NSA_ERR_CUDA;
+        g_static_scratch[dev] = p;
+    }
+    *out = g_static_scratch[dev];
+    return NSA_OK;
+}
+
+}  // namespace
+
+extern "C" nsa_status_t nsa_compress_static(const nsa_config_t* cfg, const void* k, const void* v,
+                                            const nsa_phi_params_t* phi, void* kc, void* vc,
+                                            void* stream) {
+    Shape s;
+    NSA_TRY(derive(cfg, s));
+    NSA_TRY(supported(s));
+    if (!k || !v || !kc || !vc) return NSA_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(kc) || !aligned16(vc)) return NSA_ERR_INVALID_ARG;
+    const size_t bias_bytes = align256((size_t)(s.DK + s.DV) * 8);
+    if (bias_bytes + fix_bytes(s) > kStaticScratchBytes) return NSA_ERR_WORKSPACE;
+    void* base = nullptr;
+    NSA_TRY(static_scratch_ptr(&base));
+    uint8_t* sc = reinterpret_cast<uint8_t*>(base);
+    // run_phi clears the fix-up counters at the start of every call
+    return run_phi(s, k, v, phi, kc, vc, nullptr, reinterpret_cast<double*>(sc), sc + bias_bytes,
+                   reinterpret_cast<cudaStream_t>(stream));
+}

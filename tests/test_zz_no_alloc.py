@@ -1,0 +1,63 @@
+"""nsa_compress_static: token compression for callers that cannot allocate
+device memory (graph-captured loops, plugins whose host framework owns all
+device memory).  It must produce exactly what nsa_compress produces, call
+after call, while sharing one fixed device scratch array."""
+import ctypes
+
+import pytest
+import torch
+
+from sparse_attention_long_phi_b200 import inputs as I
+
+pytestmark = pytest.mark.gpu
+
+
+def _static_fn(nsa):
+    lib = nsa.lib()
+    fn = lib.nsa_compress_static
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.POINTER(nsa.CConfig)] + [ctypes.c_void_p] * 2 + \
+                  [ctypes.POINTER(nsa.CPhi)] + [ctypes.c_void_p] * 3
+    return fn
+
+
+def _call_static(nsa, c, x):
+    fn = _static_fn(nsa)
+    B, T, G = c["B"], c["T"], c["G"]
+    C = nsa.num_cmp_blocks(c, T)
+    kc = torch.full((B, C, G, c["dk"]), float("nan"), dtype=torch.bfloat16, device="cuda")
+    vc = torch.full((B, C, G, c["dv"]), float("nan"), dtype=torch.bfloat16, device="cuda")
+    phi = None
+    if "wk" in x:
+        phi = ctypes.byref(nsa.CPhi(*(ctypes.c_void_p(x[n].data_ptr()) for n in ("wk", "ek", "wv", "ev"))))
+    rc = fn(ctypes.byref(nsa.make_config(c)), ctypes.c_void_p(x["k"].data_ptr()),
+            ctypes.c_void_p(x["v"].data_ptr()), phi, ctypes.c_void_p(kc.data_ptr()),
+            ctypes.c_void_p(vc.data_ptr()), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    return rc, kc, vc
+
+
+@pytest.mark.parametrize("name,T,seed", [("prefill_fwd_T8192", 8192, 5000), ("tiny_fwd_T1024", 1024, 5001)])
+def test_static_compress_matches_workspace_compress_twice(name, T, seed):
+    from sparse_attention_long_phi_b200 import nsa
+    for call in range(2):   # two calls in a row: the shared scratch must not leak state
+        c = dict(I.WORKLOADS[name], T=T, seed=seed + call)
+        x = I.make_forward_inputs(c, "cuda")
+        phi = {n: x[n] for n in ("wk", "ek", "wv", "ev")} if "wk" in x else None
+        rc, kc, vc = _call_static(nsa, c, x)
+        assert rc == 0, rc
+        kref, vref = nsa.compress(c, x["k"], x["v"], phi)
+        torch.cuda.synchronize()
+        nsa.sync_status()
+        assert torch.equal(kc.view(torch.int16), kref.contiguous().view(torch.int16))
+        assert torch.equal(vc.view(torch.int16), vref.contiguous().view(torch.int16))
+
+
+def test_static_compress_rejects_sizes_beyond_its_scratch():
+    from sparse_attention_long_phi_b200 import nsa
+    c = dict(I.WORKLOADS["prefill_fwd_T65536"])     # 5.2M compressed elements > 16 MiB of scratch
+    x = {k: torch.empty(0, device="cuda") for k in ("k", "v", "wk", "ek", "wv", "ev")}
+    fn = _static_fn(nsa)
+    fake = ctypes.c_void_p(1 << 20)
+    rc = fn(ctypes.byref(nsa.make_config(c)), fake, fake,
+            ctypes.byref(nsa.CPhi(fake, fake, fake, fake)), fake, fake, None)
+    assert rc == 3

@@ -98,6 +98,22 @@ def ncu_traffic(kernel):
     return None
 
 
+# ------------------------------------------------------------- multi-rank
+def max_over_ranks(ms: float, dist=None, device=None) -> float:
+    """The slowest rank's time (every rank gets the same value)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(tokens_per_rank: int, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job tokens/s: every rank processes its own sequences; the job
+    takes as long as the slowest rank."""
+    return world * tokens_per_rank * steps / (max_ms / 1e3)
+
+
 # -------------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -262,12 +278,9 @@ def main():
     nsa.sync_status()
     ms = ev0.elapsed_time(ev1)
     prof = nsa.profile_read()
-    if dist is not None:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dist, dev)
     ms_step = ms / args.steps
-    value = world * tokens_per_step * args.steps / (ms / 1e3)
+    value = weak_scaling_value(tokens_per_step, args.steps, world, ms)
 
     # roofline of the dominant kernel (largest device time in the timed region)
     flops, attn_total = forward_flops(cr)
@@ -353,12 +366,8 @@ def e2e_forward(c, x, phi, dev, stream, nsa, steps, world, dist, local):
         one()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": round(world * c["B"] * c["T"] * steps / (ms / 1e3), 1), "unit": "tokens/s",
+    ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    return {"value": round(weak_scaling_value(c["B"] * c["T"], steps, world, ms), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": steps}
 
 

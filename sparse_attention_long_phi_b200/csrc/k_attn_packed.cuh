@@ -1,6 +1,6 @@
-// k_attn_packed.cuh -- tcgen05 attention over a contiguous key range for a
-// tile of 128 query rows packed as (128/HG tokens) x (HG heads of one GQA
-// group).  Three modes:
+// k_attn_packed.cuh -- tcgen05 attention over a contiguous key range for
+// query tiles packed as (128/HG tokens) x (HG heads of one GQA group).
+// Three modes:
 //
 //   kModeLse  compressed attention, pass 1: per-row log-sum-exp of the scaled
 //             logits over the visible compressed keys (explainer, compressed
@@ -17,10 +17,16 @@
 //             running max grows by more than 8 in log2 units).
 //             out += g_win * O / l.
 //
-// Warp roles: warps 0-3 softmax/epilogue (thread = query row), warp 4 TMA
-// producer, warp 5 MMA issuer and TMEM owner.  Key tiles of 64 keys.
-// S = Q K^T  (M=128, N=64, K=DK) into one of two TMEM buffers;
-// O += P V   (M=128, N=DV, K=64) with P staged in shared memory (bf16).
+// One CTA takes two adjacent query tiles A and B (256 rows) that read the
+// same key tiles.  Warps 0-3 run the softmax and epilogue of tile A, warps
+// 4-7 those of tile B (thread = query row), warp 8 is the TMA producer and
+// warp 9 the MMA issuer and TMEM owner.  Key tiles of 64 keys:
+//   S_x = Q_x K^T (M=128, N=64, K=DK) into one of two TMEM buffers per tile,
+//   O_x += P_x V  (M=128, N=DV, K=64) with P_x staged bf16 in shared memory.
+// The MMA order S_A(j+1) S_B(j+1) PV_A(j) PV_B(j) lets each tile's softmax
+// overlap the other tile's products.  The softmax is issue-bound, so it is
+// kept to about one FFMA + one MUFU + one add per logit, and the causal /
+// window masks are applied only on the key tiles that cross a row's bound.
 #pragma once
 #include "nsa_dev.cuh"
 
@@ -38,29 +44,39 @@ struct PackedParams {
     float* lse_cmp;            // [B,T,H] natural log (pass 1 writes, pass 2 reads)
     float* pscore;             // [B,T,G,NSp]
     int NSp;
-    int n_qtiles;
+    int n_ctas;                // CTAs along the token axis (two query tiles each)
 };
 
 template <int DK, int DV, int HG, int MODE>
 struct PackedCfg {
-    static constexpr int TOK = 128 / HG;
+    static constexpr int TOK = 128 / HG;              // tokens per query tile
     static constexpr int BN = 64;
     static constexpr int NQB = DK / 64;
-    static constexpr int kQBytes = 128 * DK * 2;
+    static constexpr int kQBytes = 128 * DK * 2;      // one tile
     static constexpr int kKBox = BN * 128;            // 64 rows x 128 B
     static constexpr int kKBytes = NQB * kKBox;
     static constexpr int kVBytes = DV * 128;          // DV rows x 64 keys
     static constexpr int kPBytes = 128 * 128;         // 128 rows x 64 keys
-    static constexpr int NSK = 3;
-    static constexpr int NSV = MODE == kModeLse ? 0 : 3;
+    static constexpr int NSK = MODE == kModeLse ? 3 : 2;
+    static constexpr int NSV = MODE == kModeLse ? 0 : 2;
     static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kOffQ + kQBytes;
+    static constexpr int kOffK = kOffQ + 2 * kQBytes;
     static constexpr int kOffV = kOffK + NSK * kKBytes;
     static constexpr int kOffP = kOffV + NSV * kVBytes;
-    static constexpr int kOffBar = kOffP + (MODE == kModeLse ? 0 : kPBytes);
+    static constexpr int kOffBar = kOffP + (MODE == kModeLse ? 0 : 2 * kPBytes);
     static constexpr int kSmem = kOffBar + 256 + 1024;
-    static constexpr uint32_t kTmemCols = 256;        // S0 [0,64) S1 [64,128) O [128,128+DV)
+    // TMEM: S tile A [0,128) (2 buffers of 64), S tile B [128,256), O_A, O_B
+    static constexpr uint32_t kTmemCols = (MODE == kModeLse) ? 256 : 512;
+    static constexpr int kThreads = 320;
 };
+
+// 2^x with one MUFU instruction (ex2.approx.ftz: relative error below 2^-22,
+// ex2(-inf) = +0, so masked logits need no branch)
+__device__ __forceinline__ float ex2a(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 // Reduce `N` per-row values over the HG lanes of a token (lanes differing in
 // the low log2(HG) bits) and scatter: afterwards value v of this lane holds
@@ -105,41 +121,43 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, un
 }
 
 template <int DK, int DV, int HG, int MODE, int CPS, int SPB>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     attn_packed_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                        const __grid_constant__ CUtensorMap mapV, const PackedParams p) {
     using Cfg = PackedCfg<DK, DV, HG, MODE>;
     constexpr int TOK = Cfg::TOK;
+    constexpr int NSK = Cfg::NSK, NSV = Cfg::NSV;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
     uint64_t* qfull = bars + 0;
-    uint64_t* kfull = bars + 1;           // [NSK]
-    uint64_t* kempty = bars + 4;          // [NSK]
-    uint64_t* vfull = bars + 7;           // [NSV]
-    uint64_t* vempty = bars + 10;         // [NSV]
-    uint64_t* sfull = bars + 13;          // [2]
-    uint64_t* sfree = bars + 15;          // [2]
-    uint64_t* pfull = bars + 17;
-    uint64_t* pvdone = bars + 18;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 21);
+    uint64_t* kfull = bars + 1;           // [3]
+    uint64_t* kempty = bars + 4;          // [3]
+    uint64_t* vfull = bars + 7;           // [2]
+    uint64_t* vempty = bars + 9;          // [2]
+    uint64_t* sfull = bars + 11;          // [tile][buf] = 11 + 2*tile + buf
+    uint64_t* sfree = bars + 15;          // [tile][buf]
+    uint64_t* pfull = bars + 19;          // [tile]
+    uint64_t* pvdone = bars + 21;         // [tile]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 23);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 24);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int qt = p.n_qtiles - 1 - (int)blockIdx.x;   // heavy tiles first
+    const int cta = p.n_ctas - 1 - (int)blockIdx.x;   // heavy tiles first
     const int g = blockIdx.y, b = blockIdx.z;
-    const int t0 = qt * TOK;
-    const int t_last = min(t0 + TOK, p.T) - 1;
+    const int t0 = cta * 2 * TOK;                       // first token of tile A
+    if (t0 >= p.T) return;
+    const int t_last = min(t0 + 2 * TOK, p.T) - 1;      // last token of tile B
 
-    // key range of this tile
+    // key range shared by both tiles
     int key0, ntiles;
     if (MODE == kModeWin) {
-        int klo = max(0, t0 - p.w + 1);
+        const int klo = max(0, t0 - p.w + 1);
         key0 = (klo / 64) * 64;
         ntiles = (t_last - key0) / 64 + 1;
     } else {
-        int kend = (t_last + 1 >= p.l) ? (t_last + 1 - p.l) / p.d + 1 : 0;
+        const int kend = (t_last + 1 >= p.l) ? (t_last + 1 - p.l) / p.d + 1 : 0;
         key0 = 0;
         ntiles = (kend + 63) / 64;
     }
@@ -149,19 +167,21 @@ __global__ void __launch_bounds__(192, 1)
         for (int s = 0; s < 3; ++s) {
             mbar_init(&kfull[s], 1);
             mbar_init(&kempty[s], 1);
-            mbar_init(&vfull[s], 1);
-            mbar_init(&vempty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
+            mbar_init(&vfull[s], 1);
+            mbar_init(&vempty[s], 1);
+            mbar_init(&pfull[s], 128);
+            mbar_init(&pvdone[s], 1);
+        }
+        for (int s = 0; s < 4; ++s) {
             mbar_init(&sfull[s], 1);
             mbar_init(&sfree[s], 4);
         }
-        mbar_init(pfull, 128);
-        mbar_init(pvdone, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == 9) {
         tmem_alloc(tmem_slot, Cfg::kTmemCols);
         tmem_relinquish();
     }
@@ -170,21 +190,23 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ------------------------------------------------------ producer
         if (lane == 0 && ntiles > 0) {
             tma_prefetch_desc(&mapQ);
             tma_prefetch_desc(&mapK);
             if (MODE != kModeLse) tma_prefetch_desc(&mapV);
-            mbar_expect_tx(qfull, Cfg::kQBytes);
+            mbar_expect_tx(qfull, 2 * Cfg::kQBytes);
 #pragma unroll
-            for (int bx = 0; bx < Cfg::NQB; ++bx)
-                tma_load_4d(smem + Cfg::kOffQ + bx * 16384, &mapQ, qfull, bx * 64, g * HG, t0, b);
+            for (int tile = 0; tile < 2; ++tile)
+#pragma unroll
+                for (int bx = 0; bx < Cfg::NQB; ++bx)
+                    tma_load_4d(smem + Cfg::kOffQ + tile * Cfg::kQBytes + bx * 16384, &mapQ, qfull,
+                                bx * 64, g * HG, t0 + tile * TOK, b);
             for (int jt = 0; jt < ntiles; ++jt) {
                 const int kb = key0 + jt * 64;
-                const int s = jt % Cfg::NSK;
-                if (jt >= Cfg::NSK &&
-                    !wait_or_abort(&kempty[s], ((jt / Cfg::NSK) - 1) & 1, 0x201, abort_flag))
+                const int s = jt % NSK;
+                if (jt >= NSK && !wait_or_abort(&kempty[s], ((jt / NSK) - 1) & 1, 0x201, abort_flag))
                     break;
                 uint8_t* ks = smem + Cfg::kOffK + s * Cfg::kKBytes;
                 mbar_expect_tx(&kfull[s], Cfg::kKBytes);
@@ -192,8 +214,8 @@ __global__ void __launch_bounds__(192, 1)
                 for (int bx = 0; bx < Cfg::NQB; ++bx)
                     tma_load_4d(ks + bx * Cfg::kKBox, &mapK, &kfull[s], bx * 64, g, kb, b);
                 if (MODE != kModeLse) {
-                    const int sv = jt % 3;
-                    if (jt >= 3 && !wait_or_abort(&vempty[sv], ((jt / 3) - 1) & 1, 0x202, abort_flag))
+                    const int sv = jt % NSV;
+                    if (jt >= NSV && !wait_or_abort(&vempty[sv], ((jt / NSV) - 1) & 1, 0x202, abort_flag))
                         break;
                     uint8_t* vs = smem + Cfg::kOffV + sv * Cfg::kVBytes;
                     mbar_expect_tx(&vfull[sv], Cfg::kVBytes);
@@ -201,41 +223,49 @@ __global__ void __launch_bounds__(192, 1)
                 }
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ----------------------------------------------------------- MMA
         if (lane == 0 && ntiles > 0) {
             constexpr uint32_t idS = idesc_bf16(128, 64);
             constexpr uint32_t idO = idesc_bf16(128, DV);
-            const uint32_t sQ = smem_u32(smem + Cfg::kOffQ);
             bool ok = wait_or_abort(qfull, 0, 0x203, abort_flag);
             auto issue_S = [&](int jt) -> bool {
-                const int s = jt % Cfg::NSK, buf = jt & 1;
-                if (!wait_or_abort(&kfull[s], (jt / Cfg::NSK) & 1, 0x204, abort_flag)) return false;
-                if (jt >= 2 && !wait_or_abort(&sfree[buf], ((jt - 2) >> 1) & 1, 0x205, abort_flag))
-                    return false;
-                tc_fence_after();
+                const int s = jt % NSK, buf = jt & 1;
+                if (!wait_or_abort(&kfull[s], (jt / NSK) & 1, 0x204, abort_flag)) return false;
                 const uint32_t sK = smem_u32(smem + Cfg::kOffK + s * Cfg::kKBytes);
 #pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk)
-                    umma_bf16_ss(tmem + buf * 64, sdesc_sw128(sQ + (kk / 4) * 16384 + (kk % 4) * 32),
-                                 sdesc_sw128(sK + (kk / 4) * Cfg::kKBox + (kk % 4) * 32), idS,
-                                 kk > 0 ? 1u : 0u);
-                umma_commit(&sfull[buf]);
+                for (int tile = 0; tile < 2; ++tile) {
+                    if (jt >= 2 &&
+                        !wait_or_abort(&sfree[2 * tile + buf], ((jt - 2) >> 1) & 1, 0x205, abort_flag))
+                        return false;
+                    tc_fence_after();
+                    const uint32_t sQ = smem_u32(smem + Cfg::kOffQ + tile * Cfg::kQBytes);
+#pragma unroll
+                    for (int kk = 0; kk < DK / 16; ++kk)
+                        umma_bf16_ss(tmem + tile * 128 + buf * 64,
+                                     sdesc_sw128(sQ + (kk / 4) * 16384 + (kk % 4) * 32),
+                                     sdesc_sw128(sK + (kk / 4) * Cfg::kKBox + (kk % 4) * 32), idS,
+                                     kk > 0 ? 1u : 0u);
+                    umma_commit(&sfull[2 * tile + buf]);
+                }
                 umma_commit(&kempty[s]);
                 return true;
             };
             auto issue_PV = [&](int jt) -> bool {
-                if (!wait_or_abort(pfull, jt & 1, 0x206, abort_flag)) return false;
-                const int sv = jt % 3;
-                if (!wait_or_abort(&vfull[sv], (jt / 3) & 1, 0x207, abort_flag)) return false;
-                tc_fence_after();
-                const uint32_t sP = smem_u32(smem + Cfg::kOffP);
+                const int sv = jt % NSV;
+                if (!wait_or_abort(&vfull[sv], (jt / NSV) & 1, 0x207, abort_flag)) return false;
                 const uint32_t sV = smem_u32(smem + Cfg::kOffV + sv * Cfg::kVBytes);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_bf16_ss(tmem + 128, sdesc_sw128(sP + kk * 32), sdesc_sw128(sV + kk * 32),
-                                 idO, (jt > 0 || kk > 0) ? 1u : 0u);
-                umma_commit(pvdone);
+                for (int tile = 0; tile < 2; ++tile) {
+                    if (!wait_or_abort(&pfull[tile], jt & 1, 0x206, abort_flag)) return false;
+                    tc_fence_after();
+                    const uint32_t sP = smem_u32(smem + Cfg::kOffP + tile * Cfg::kPBytes);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_bf16_ss(tmem + 256 + tile * DV, sdesc_sw128(sP + kk * 32),
+                                     sdesc_sw128(sV + kk * 32), idO, (jt > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&pvdone[tile]);
+                }
                 umma_commit(&vempty[sv]);
                 return true;
             };
@@ -247,16 +277,18 @@ __global__ void __launch_bounds__(192, 1)
         }
     } else {
         // ------------------------------------------------ softmax / epilogue
-        const int r = threadIdx.x;
-        const int t = t0 + r / HG;
+        const int tile = warp >> 2;                 // 0: tile A, 1: tile B
+        const int wq = warp & 3;                    // TMEM lane quadrant
+        const int r = wq * 32 + lane;               // row within the tile
+        const int t = t0 + tile * TOK + r / HG;
         const int hh = r % HG;
         const int h = g * HG + hh;
         const bool row_ok = t < p.T;
         const size_t rowid = ((size_t)b * p.T + (row_ok ? t : 0)) * p.H + h;
-        const uint32_t lanebase = tmem + ((uint32_t)(warp * 32) << 16);
-        // visible-key bound for this row
-        int vis_hi;   // exclusive upper bound (cmp) / inclusive t (win)
-        int vis_lo = 0;
+        const uint32_t lanebase = tmem + ((uint32_t)(wq * 32) << 16);
+        const uint32_t sbase = lanebase + tile * 128;         // S buffers of this tile
+        const uint32_t obase = lanebase + 256 + tile * DV;    // O of this tile
+        int vis_hi, vis_lo = 0;
         if (MODE == kModeWin) {
             vis_hi = t + 1;
             vis_lo = t - p.w + 1;
@@ -264,6 +296,10 @@ __global__ void __launch_bounds__(192, 1)
             vis_hi = (t + 1 >= p.l) ? (t + 1 - p.l) / p.d + 1 : 0;
         }
         if (!row_ok) vis_hi = vis_lo = -1 << 30;
+        // bounds shared by every row of this query tile (visibility grows with t)
+        const int tile_first = t0 + tile * TOK;
+        const int tile_last = min(tile_first + TOK, p.T) - 1;
+        const int vis_first = (tile_first + 1 >= p.l) ? (tile_first + 1 - p.l) / p.d + 1 : 0;
         float m_run = -INFINITY, l_run = 0.f;
         float lse2 = -INFINITY;
         if (MODE == kModeCmp && row_ok) lse2 = p.lse_cmp[rowid] * kLog2e;
@@ -278,37 +314,47 @@ __global__ void __launch_bounds__(192, 1)
         for (int jt = 0; jt < ntiles; ++jt) {
             const int buf = jt & 1;
             const int kb = key0 + jt * 64;
-            if (ok) ok = wait_or_abort(&sfull[buf], (jt >> 1) & 1, 0x208, abort_flag);
+            if (ok) ok = wait_or_abort(&sfull[2 * tile + buf], (jt >> 1) & 1, 0x208, abort_flag);
             tc_fence_after();
             uint32_t ra[32], rb[32];
-            tmem_ld32(lanebase + buf * 64, ra);
-            tmem_ld32(lanebase + buf * 64 + 32, rb);
+            tmem_ld32(sbase + buf * 64, ra);
+            tmem_ld32(sbase + buf * 64 + 32, rb);
             tmem_wait_ld32(ra);
             tmem_wait_ld32(rb);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sfree[buf]);
+            if (lane == 0) mbar_arrive(&sfree[2 * tile + buf]);
             float s[64];
 #pragma unroll
             for (int k = 0; k < 32; ++k) {
-                s[k] = __uint_as_float(ra[k]) * p.scale_log2;
-                s[k + 32] = __uint_as_float(rb[k]) * p.scale_log2;
+                s[k] = __uint_as_float(ra[k]);
+                s[k + 32] = __uint_as_float(rb[k]);
             }
+            // masks only where the key tile crosses a row bound of this query tile
+            const bool interior = (MODE == kModeWin)
+                                      ? (kb >= tile_last - p.w + 1 && kb + 63 <= tile_first)
+                                      : (kb + 64 <= vis_first);
+            if (!interior) {
 #pragma unroll
-            for (int k = 0; k < 64; ++k) {
-                const int key = kb + k;
-                if (!(key >= vis_lo && key < vis_hi)) s[k] = -INFINITY;
+                for (int k = 0; k < 64; ++k) {
+                    const int key = kb + k;
+                    if (!(key >= vis_lo && key < vis_hi)) s[k] = -INFINITY;
+                }
             }
+            const float c = p.scale_log2;
             if (MODE == kModeLse) {
-                float mt = -INFINITY;
+                float mr = -INFINITY;
 #pragma unroll
-                for (int k = 0; k < 64; ++k) mt = fmaxf(mt, s[k]);
-                const float mn = fmaxf(m_run, mt);
+                for (int k = 0; k < 64; ++k) mr = fmaxf(mr, s[k]);
+                const float mn = fmaxf(m_run, mr * c);
                 if (mn != -INFINITY) {
-                    float acc = 0.f;
+                    float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-                    for (int k = 0; k < 64; ++k) acc += exp2f(s[k] - mn);
-                    l_run = l_run * exp2f(m_run - mn) + acc;
+                    for (int k = 0; k < 64; k += 2) {
+                        acc0 += ex2a(fmaf(s[k], c, -mn));
+                        acc1 += ex2a(fmaf(s[k + 1], c, -mn));
+                    }
+                    l_run = l_run * ex2a(m_run - mn) + (acc0 + acc1);
                     m_run = mn;
                 }
                 continue;
@@ -317,26 +363,32 @@ __global__ void __launch_bounds__(192, 1)
             float alpha = 1.f;
             bool need_rescale = false;
             if (MODE == kModeCmp) {
+                // a row with no visible key has LSE = -inf and only masked logits
+                const float nl = lse2 == -INFINITY ? 0.f : -lse2;
 #pragma unroll
-                for (int k = 0; k < 64; ++k) pr[k] = (s[k] == -INFINITY) ? 0.f : exp2f(s[k] - lse2);
+                for (int k = 0; k < 64; ++k) pr[k] = ex2a(fmaf(s[k], c, nl));
             } else {
-                float mt = -INFINITY;
+                float mr = -INFINITY;
 #pragma unroll
-                for (int k = 0; k < 64; ++k) mt = fmaxf(mt, s[k]);
+                for (int k = 0; k < 64; ++k) mr = fmaxf(mr, s[k]);
+                const float mt = mr * c;
                 if (mt > m_run + 8.f) {
-                    const float mn = mt;
-                    alpha = exp2f(m_run - mn);       // 0 when m_run = -inf
+                    alpha = ex2a(m_run - mt);        // 0 when m_run = -inf
                     l_run *= alpha;
-                    m_run = mn;
+                    m_run = mt;
                     need_rescale = true;
                 }
-                float acc = 0.f;
+                // m_run stays -inf while every key so far is masked for this row
+                const float nm = m_run == -INFINITY ? 0.f : -m_run;
+                float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-                for (int k = 0; k < 64; ++k) {
-                    pr[k] = (s[k] == -INFINITY) ? 0.f : exp2f(s[k] - m_run);
-                    acc += pr[k];
+                for (int k = 0; k < 64; k += 2) {
+                    pr[k] = ex2a(fmaf(s[k], c, nm));
+                    pr[k + 1] = ex2a(fmaf(s[k + 1], c, nm));
+                    acc0 += pr[k];
+                    acc1 += pr[k + 1];
                 }
-                l_run += acc;
+                l_run += acc0 + acc1;
             }
             if (MODE == kModeCmp) {
                 // importance scores of selection blocks kb/SPB .. kb/SPB + NB - 1
@@ -363,23 +415,23 @@ __global__ void __launch_bounds__(192, 1)
                         if (j0 + base + v < p.NSp) dst[j0 + base + v] = red[v];
                 }
             }
-            // P -> shared memory (after the previous P.V has consumed it)
-            if (jt > 0 && ok) ok = wait_or_abort(pvdone, (jt - 1) & 1, 0x209, abort_flag);
+            // P -> shared memory (after the previous P.V of this tile has consumed it)
+            if (jt > 0 && ok) ok = wait_or_abort(&pvdone[tile], (jt - 1) & 1, 0x209, abort_flag);
             tc_fence_after();
             if (MODE == kModeWin && jt > 0 && __any_sync(0xffffffffu, need_rescale)) {
                 const float a = need_rescale ? alpha : 1.f;
 #pragma unroll 1
                 for (int c0 = 0; c0 < DV; c0 += 32) {
                     uint32_t o[32];
-                    tmem_ld32(lanebase + 128 + c0, o);
+                    tmem_ld32(obase + c0, o);
                     tmem_wait_ld32(o);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * a);
-                    tmem_st32(lanebase + 128 + c0, o);
+                    tmem_st32(obase + c0, o);
                 }
                 tmem_wait_st();
             }
-            const uint32_t sP = smem_u32(smem + Cfg::kOffP);
+            const uint32_t sP = smem_u32(smem + Cfg::kOffP + tile * Cfg::kPBytes);
 #pragma unroll
             for (int c = 0; c < 8; ++c)
                 st_shared_v4(sP + sw128_off(r, c), pack_bf16x2(pr[8 * c + 0], pr[8 * c + 1]),
@@ -388,7 +440,7 @@ __global__ void __launch_bounds__(192, 1)
                              pack_bf16x2(pr[8 * c + 6], pr[8 * c + 7]));
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(pfull);
+            mbar_arrive(&pfull[tile]);
         }
 
         // ------------------------------------------------------- epilogue
@@ -411,7 +463,7 @@ __global__ void __launch_bounds__(192, 1)
                         p.pscore[(((size_t)b * p.T + t) * p.G + g) * p.NSp + jn + c] = v;
                 }
             }
-            if (ntiles > 0 && ok) ok = wait_or_abort(pvdone, (ntiles - 1) & 1, 0x20A, abort_flag);
+            if (ntiles > 0 && ok) ok = wait_or_abort(&pvdone[tile], (ntiles - 1) & 1, 0x20A, abort_flag);
             tc_fence_after();
             const float gate = row_ok ? p.gates[rowid * 3 + (MODE == kModeCmp ? 0 : 2)] : 0.f;
             const float inv = (MODE == kModeWin) ? (l_run > 0.f ? 1.f / l_run : 0.f) : 1.f;
@@ -419,7 +471,7 @@ __global__ void __launch_bounds__(192, 1)
             for (int c0 = 0; c0 < DV; c0 += 32) {
                 uint32_t o[32];
                 if (ntiles > 0) {
-                    tmem_ld32(lanebase + 128 + c0, o);
+                    tmem_ld32(obase + c0, o);
                     tmem_wait_ld32(o);
                 } else {
 #pragma unroll
@@ -427,6 +479,11 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 if (row_ok && ok) {
                     float4* dst = reinterpret_cast<float4*>(p.out + rowid * DV + c0);
+                    float4 prev[8];
+                    if (MODE == kModeWin) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) prev[e] = dst[e];
+                    }
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         float4 v;
@@ -435,11 +492,10 @@ __global__ void __launch_bounds__(192, 1)
                         v.z = gate * __uint_as_float(o[4 * e + 2]) * inv;
                         v.w = gate * __uint_as_float(o[4 * e + 3]) * inv;
                         if (MODE == kModeWin) {
-                            float4 prev = dst[e];
-                            v.x += prev.x;
-                            v.y += prev.y;
-                            v.z += prev.z;
-                            v.w += prev.w;
+                            v.x += prev[e].x;
+                            v.y += prev[e].y;
+                            v.z += prev[e].z;
+                            v.w += prev[e].w;
                         }
                         dst[e] = v;
                     }
@@ -451,7 +507,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, Cfg::kTmemCols);
     }

@@ -332,7 +332,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
                 for (int h = 0; h < 16; ++h) {
                     float e = 0.f;
-                    if (h < HG && valid) e = exp2f(__uint_as_float(r[h]) * p.scale_log2 - mx[h]);
+                    if (h < HG && valid) e = ex2a(fmaf(__uint_as_float(r[h]), p.scale_log2, -mx[h]));
                     ls[h] += e;
                     __nv_bfloat16 eb = __float2bfloat16_rn(e);
                     st_shared_u16(cbase + sw128_off(h, kk >> 3) + (kk & 7) * 2,

@@ -295,8 +295,8 @@ nsa_status_t launch_packed(const Shape& s, const CUtensorMap& mQ, const CUtensor
     auto kern = attn_packed_kernel<DK, DV, HG, MODE, CPS, SPB>;
     const char* kern_name = MODE == kModeLse ? "attn_cmp_lse" : MODE == kModeCmp ? "attn_cmp_pv_scores" : "attn_window";
     NSA_TRY(set_smem(kern, Cfg::kSmem));
-    dim3 grid((unsigned)p.n_qtiles, (unsigned)s.G, (unsigned)s.B);
-    NSA_LAUNCH(kern_name, st, kern<<<grid, 192, Cfg::kSmem, st>>>(mQ, mK, mV, p));
+    dim3 grid((unsigned)p.n_ctas, (unsigned)s.G, (unsigned)s.B);
+    NSA_LAUNCH(kern_name, st, kern<<<grid, Cfg::kThreads, Cfg::kSmem, st>>>(mQ, mK, mV, p));
     return last_launch();
 }
 
@@ -379,7 +379,7 @@ nsa_status_t forward_impl(const Shape& s, const void* q, const void* k, const vo
     pp.lse_cmp = lse_cmp;
     pp.pscore = pscore;
     pp.NSp = (int)s.NSp;
-    pp.n_qtiles = (int)ceil_div(s.T, 128 / HG);
+    pp.n_ctas = (int)ceil_div(s.T, 2 * (128 / HG));
     // 3-4. compressed attention: LSE pass, then P.V~ with importance scores
     if (s.C > 0) {
         NSA_TRY((launch_packed_blk<DK, DV, HG, kModeLse>(s, mQ, mKc, mVc, pp, st)));

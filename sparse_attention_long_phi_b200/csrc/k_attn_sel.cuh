@@ -139,25 +139,38 @@ __global__ void __launch_bounds__(320, 1)
                     return nullptr;
                 return smem + Cfg::kOffKV + sl * Cfg::kSlot;
             };
-            auto load_pairs = [&](int i, bool kv_is_k) -> bool {
+            // a token's selection row: 16 ints (ascending, -1 padded) in four
+            // 16-byte loads; rows are read once and prefetched one token ahead
+            auto load_row = [&](int i, int4 (&r)[4]) {
+                if (i >= N) return;
                 const int32_t* row = idx_base + (size_t)(tb + i) * p.G * p.n;
-                int u[16];
+                if (p.n == 16 && (reinterpret_cast<uintptr_t>(row) & 15) == 0) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) r[q] = __ldg(reinterpret_cast<const int4*>(row) + q);
+                } else {
+                    int tmp[16];
+#pragma unroll
+                    for (int a = 0; a < 16; ++a) tmp[a] = a < p.n ? row[a] : -1;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) r[q] = make_int4(tmp[4 * q], tmp[4 * q + 1], tmp[4 * q + 2], tmp[4 * q + 3]);
+                }
+            };
+            auto unit_of = [](const int4 (&r)[4], int a) -> int {
+                const int4 v = r[a >> 2];
+                const int k = a & 3;
+                return k == 0 ? v.x : k == 1 ? v.y : k == 2 ? v.z : v.w;
+            };
+            auto count_row = [&](const int4 (&r)[4]) -> int {
                 int nu = 0;
 #pragma unroll
-                for (int a = 0; a < 16; ++a) {
-                    const int j = a < p.n ? row[a] : -1;
-                    u[a] = j;
-                    nu += j >= 0;
-                }
-                // the selection is ascending with -1 padding: valid entries come first
+                for (int q = 0; q < 4; ++q) nu += (r[q].x >= 0) + (r[q].y >= 0) + (r[q].z >= 0) + (r[q].w >= 0);
+                return nu;
+            };
+            auto load_pairs = [&](const int4 (&r)[4], bool kv_is_k) -> bool {
+                const int nu = count_row(r);
                 for (int pp = 0; pp < (nu + 1) / 2; ++pp) {
-                    int ja = 0, jb = 0;
-#pragma unroll
-                    for (int a = 0; a < 16; ++a) {
-                        if (a == 2 * pp) ja = u[a];
-                        if (a == 2 * pp + 1) jb = u[a];
-                    }
-                    if (2 * pp + 1 >= nu) jb = ja;
+                    const int ja = unit_of(r, 2 * pp);
+                    const int jb = (2 * pp + 1 < nu) ? unit_of(r, 2 * pp + 1) : ja;
                     uint8_t* sl = slot_acquire(cnt);
                     if (!sl) return false;
                     uint64_t* bar = &full[cnt % Cfg::NSLOT];
@@ -176,24 +189,32 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 return true;
             };
-            auto load_S = [&](int i) -> bool {
+            auto load_S = [&](int i, const int4 (&r)[4]) -> bool {
                 const int qs = i & 1;
                 if (i >= 2 && !wait_or_abort(&qempty[qs], ((i - 2) >> 1) & 1, 0x302, abort_flag))
                     return false;
-                const int32_t* row = idx_base + (size_t)(tb + i) * p.G * p.n;
-                npairs_ring[i & 3] = (count_units(row, p.n) + 1) / 2;   // read by the MMA warp
+                npairs_ring[i & 3] = (count_row(r) + 1) / 2;          // read by the MMA warp
                 mbar_expect_tx(&qfull[qs], Cfg::kQSlot);                // (release)
                 for (int bx = 0; bx < Cfg::NQB; ++bx)
                     tma_load_4d(smem + Cfg::kOffQ + qs * Cfg::kQSlot + bx * 2048, &mapQ, &qfull[qs],
                                 bx * 64, g * HG, tb + i, b);
-                return load_pairs(i, true);
+                return load_pairs(r, true);
             };
-            bool ok = load_S(0);
+            int4 cur[4], prev[4], nxt[4];
+            load_row(0, cur);
+            load_row(1, nxt);
+            bool ok = load_S(0, cur);
             for (int i = 1; i < N && ok; ++i) {
-                ok = load_S(i);
-                if (ok) ok = load_pairs(i - 1, false);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    prev[q] = cur[q];
+                    cur[q] = nxt[q];
+                }
+                load_row(i + 1, nxt);                                  // in flight during token i
+                ok = load_S(i, cur);
+                if (ok) ok = load_pairs(prev, false);
             }
-            if (ok) load_pairs(N - 1, false);
+            if (ok) load_pairs(cur, false);
         }
     } else if (warp == 9) {
         // ----------------------------------------------------------- MMA
@@ -276,16 +297,28 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t bar_id = 1 + wg;
         bool ok = true;
         int it = 0;
+        // the token's selection entry (threads kl < 16) and gates, prefetched
+        // one token ahead so their latency overlaps the previous token
+        int idx_nx = -1;
+        float gate_nx[HG];
+        auto prefetch = [&](int i) {
+            if (i >= N) return;
+            const int32_t* row = idx_base + (size_t)(tb + i) * p.G * p.n;
+            if (kl < 16) idx_nx = kl < p.n ? __ldg(row + kl) : -1;
+            const size_t rb2 = ((size_t)b * p.T + tb + i) * p.H + (size_t)g * HG;
+#pragma unroll
+            for (int h = 0; h < HG; ++h) gate_nx[h] = __ldg(p.gates + (rb2 + h) * 3 + 1);
+        };
+        prefetch(wg);
         for (int i = wg; i < N; i += 2, ++it) {
             const int t = tb + i;
-            const int32_t* row = idx_base + (size_t)t * p.G * p.n;
-            if (kl < 16) su[kl] = kl < p.n ? row[kl] : -1;
-            // per-head gates of the token (loaded early, used in the epilogue)
+            if (kl < 16) su[kl] = idx_nx;
             float gate[HG];
-            const size_t rowbase = ((size_t)b * p.T + t) * p.H + (size_t)g * HG;
 #pragma unroll
-            for (int h = 0; h < HG; ++h) gate[h] = __ldg(p.gates + (rowbase + h) * 3 + 1);
+            for (int h = 0; h < HG; ++h) gate[h] = gate_nx[h];
+            const size_t rowbase = ((size_t)b * p.T + t) * p.H + (size_t)g * HG;
             named_bar_sync(bar_id, 128);
+            prefetch(i + 2);
             int nu = 0;
 #pragma unroll
             for (int a = 0; a < 16; ++a) nu += su[a] >= 0;

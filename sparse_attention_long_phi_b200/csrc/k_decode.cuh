@@ -3,13 +3,18 @@
 // selected blocks and the window, not the whole cache).
 //
 // One query per sequence at t = L-1 over packed varlen caches.  The step is
-// HBM-bound; the kernels stream each cache row once:
-//   1. dec_cmp_partial  split-K over the compressed cache: logits for the HG
-//                       heads of a group (kept for step 2), split max/sum and
-//                       the split's P.V~.
-//   2. dec_cmp_combine  merge the splits -> o_cmp and the row LSE; normalised
-//                       compressed probabilities summed over heads, mapped to
-//                       selection blocks; top-n by one warp -> sel_idx.
+// HBM-bound; every cache row is read once, with 16-byte coalesced loads into
+// shared memory, and the 16 heads of a GQA group are the M = 16 side of
+// warp-level bf16 tensor-core products (mma.sync m16n8k16, fp32 accumulate):
+//   1. dec_cmp_partial  split-K over the compressed cache (128 keys per CTA,
+//                       32 per warp): logits, split max / sum, P.V~, and the
+//                       per-head selection-block sums of exp(logit - split max)
+//                       (mapped with the overlap weights), so the scores can be
+//                       normalised exactly once the row LSE is known.
+//   2. dec_cmp_combine  merge the splits -> o_cmp and the row LSE; group
+//                       importance scores = sum over heads and splits of the
+//                       block sums rescaled by exp(split max - LSE); top-n by
+//                       one warp -> sel_idx.
 //   3. dec_slcwin_partial  one CTA per 64-token unit of (selected blocks U
 //                       window blocks): logits once, partial softmax of the
 //                       selected and window branches over the unit.
@@ -20,8 +25,11 @@
 
 namespace nsa {
 
-constexpr int kDecCH = 128;    // compressed keys per split
-constexpr int kDecUnit = 64;   // tokens per selected/window unit
+constexpr int kDecCH = 128;     // compressed keys per split (4 warps x 32)
+constexpr int kDecUnit = 64;    // tokens per selected/window unit (2 warps x 32)
+constexpr int kDecNJB = 132;    // block-score slots per split (>= 128/SPB + 1)
+constexpr int kDecWJB = 34;     // block-score slots per warp of 32 keys (>= 32/SPB + 2)
+constexpr int kDecMaxSplits = 64;  // compressed-cache splits per sequence (Lmax <= 8192 * 16 + l)
 
 struct DecParams {
     int S, H, G, HG, DK, DV;
@@ -33,27 +41,328 @@ struct DecParams {
     float* out;
     int32_t* sel_idx;
     float* lse;
-    float* logits;   // [S][G][16][Cmax]     log2-scaled logits
-    float* part1;    // [S][G][NSPL][16][2+DV]
+    float* part1;    // [S][G][NSPL][16][2+DV]   split max (log2 units), sum, unnormalised O
+    float* bsc;      // [S][G][NSPL][16][kDecNJB] block sums of exp2(s - split max)
     float* ocmp;     // [S][G][16][DV]
-    float* lsecmp;   // [S][G][16]            log2 units
+    float* lsecmp;   // [S][G][16]               log2 units
     float* part2;    // [S][G][NU][2][16][2+DV]
     int Cmax, NSPL, NU, NSmax;
 };
 
-__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&f)[8]) {
-    uint4 u = *reinterpret_cast<const uint4*>(p);
-    const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&u);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) f[e] = __bfloat162float(h[e]);
+// ------------------------------------------------------------ mma helpers
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
 }
 
-// q of the group's heads into shared memory as fp32 [16][DK] (rows >= HG zero)
-__device__ __forceinline__ void dec_load_q(const DecParams& p, int s, int g, float* qs) {
-    for (int e = threadIdx.x; e < 16 * p.DK; e += blockDim.x) {
-        const int h = e / p.DK, c = e % p.DK;
-        qs[e] = h < p.HG ? __bfloat162float(p.q[((size_t)s * p.H + g * p.HG + h) * p.DK + c]) : 0.f;
+// Q of the group's 16 heads (rows >= HG zero) as A fragments for DK/16 k-steps
+template <int DK>
+__device__ __forceinline__ void load_q_frags(const DecParams& p, int s, int g, uint32_t (&qa)[DK / 16][4]) {
+    const int lane = threadIdx.x & 31, gr = lane >> 2, tg = lane & 3;
+    const __nv_bfloat16* q = p.q + ((size_t)s * p.H + (size_t)g * p.HG) * DK;
+#pragma unroll
+    for (int kk = 0; kk < DK / 16; ++kk) {
+        const int c = kk * 16 + tg * 2;
+        auto ld = [&](int row, int col) -> uint32_t {
+            return row < p.HG ? *reinterpret_cast<const uint32_t*>(q + (size_t)row * DK + col) : 0u;
+        };
+        qa[kk][0] = ld(gr, c);
+        qa[kk][1] = ld(gr + 8, c);
+        qa[kk][2] = ld(gr, c + 8);
+        qa[kk][3] = ld(gr + 8, c + 8);
     }
+}
+
+// copy `rows` rows of `width` bf16 (row stride src_stride elements) into
+// shared memory with a padded pitch: 16-byte cp.async chunks, all in flight
+// at once; rows >= nvalid are zero-filled.  Caller waits with cp_async_wait.
+__device__ __forceinline__ void warp_copy_rows(uint8_t* dst, int pitch, const __nv_bfloat16* src,
+                                               size_t src_stride, int rows, int nvalid, int width) {
+    const int lane = threadIdx.x & 31;
+    const int cpr = width / 8;   // 16-byte chunks per row
+    for (int e = lane; e < rows * cpr; e += 32) {
+        const int r = e / cpr, c = e % cpr;
+        const bool ok = r < nvalid;
+        const __nv_bfloat16* sp = ok ? src + (size_t)r * src_stride + c * 8 : src;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst + r * pitch + c * 16)),
+                     "l"(sp), "r"(ok ? 16 : 0)
+                     : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// S[16 heads x 32 keys] = Q K^T for the warp's 32 keys staged at `ks` (pitch
+// DK*2+16), logits scaled to log2 units; sfr[nt][0..3] in accumulator layout
+template <int DK>
+__device__ __forceinline__ void warp_logits(const uint32_t (&qa)[DK / 16][4], uint32_t ks, float (&sfr)[4][4]) {
+    const int lane = threadIdx.x & 31;
+    constexpr int pitch = DK * 2 + 16;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sfr[nt][e] = 0.f;
+    // ldmatrix x4 (non-transposed): matrices (keys 8nt..+7, dims 16kk..+7),
+    // (same keys, dims +8), then the same for n-tile nt+1
+    const int mi = lane >> 3, rr = lane & 7;
+#pragma unroll
+    for (int kk = 0; kk < DK / 16; ++kk) {
+#pragma unroll
+        for (int nt = 0; nt < 4; nt += 2) {
+            const int key = (nt + (mi >> 1)) * 8 + rr;
+            const int dim = kk * 16 + (mi & 1) * 8;
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4(ks + key * pitch + dim * 2, b0, b1, b2, b3);
+            mma16816(sfr[nt], qa[kk], b0, b1);
+            mma16816(sfr[nt + 1], qa[kk], b2, b3);
+        }
+    }
+}
+
+// O[16 x DV] += P[16 x 32] V[32 x DV] for the warp's 32 keys staged at `vs`
+// (pitch DV*2+16); P given in accumulator layout (fp32), converted to bf16 A
+// fragments (two n-tiles of S form one k-step of P)
+template <int DV>
+__device__ __forceinline__ void warp_pv(const float (&pf)[4][4], uint32_t vs, float (&o)[DV / 8][4]) {
+    const int lane = threadIdx.x & 31;
+    constexpr int pitch = DV * 2 + 16;
+    const int mi = lane >> 3, rr = lane & 7;
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk) {
+        uint32_t a[4];
+        a[0] = pack_bf16x2(pf[2 * kk][0], pf[2 * kk][1]);
+        a[1] = pack_bf16x2(pf[2 * kk][2], pf[2 * kk][3]);
+        a[2] = pack_bf16x2(pf[2 * kk + 1][0], pf[2 * kk + 1][1]);
+        a[3] = pack_bf16x2(pf[2 * kk + 1][2], pf[2 * kk + 1][3]);
+#pragma unroll
+        for (int nt = 0; nt < DV / 8; nt += 2) {
+            // ldmatrix x4 .trans: matrices (keys 16kk..+7, ch 8nt..), (keys +8, ch 8nt..),
+            // (keys 16kk.., ch 8nt+8..), (keys +8, ch 8nt+8..)
+            const int key = kk * 16 + (mi & 1) * 8 + rr;
+            const int ch = nt * 8 + (mi >> 1) * 8;
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4_t(vs + key * pitch + ch * 2, b0, b1, b2, b3);
+            mma16816(o[nt], a, b0, b1);
+            mma16816(o[nt + 1], a, b2, b3);
+        }
+    }
+}
+
+// -------------------------------------------------------------- step 1
+template <int DK, int DV>
+__global__ void __launch_bounds__(128) dec_cmp_partial(const DecParams p) {
+    constexpr int KP = DK * 2 + 16, VP = DV * 2 + 16;
+    extern __shared__ __align__(16) uint8_t dsm[];
+    __shared__ float redm[4][16], redl[4][16];
+    __shared__ float bsw[4][16][kDecWJB];
+    const int sp = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gr = lane >> 2, tg = lane & 3;
+    const int64_t cbase = p.cmp_off[s];
+    const int C = (int)(p.cmp_off[s + 1] - cbase);
+    if (C > p.Cmax) {
+        if (threadIdx.x == 0 && sp == 0) atomicOr(&g_nsa_error, 4u);
+        return;
+    }
+    const int c0 = sp * kDecCH;
+    if (c0 >= C) return;
+    uint8_t* ks = dsm + warp * 32 * (KP + VP);
+    uint8_t* vs = ks + 32 * KP;
+    const int k0 = c0 + warp * 32;                       // first key of this warp
+    const int nval = max(0, min(32, C - k0));
+    warp_copy_rows(ks, KP, p.kccache + ((cbase + k0) * p.G + g) * DK, (size_t)p.G * DK, 32, nval, DK);
+    warp_copy_rows(vs, VP, p.vccache + ((cbase + k0) * p.G + g) * DV, (size_t)p.G * DV, 32, nval, DV);
+    uint32_t qa[DK / 16][4];
+    load_q_frags<DK>(p, s, g, qa);
+    cp_async_wait();
+    __syncwarp();
+    float sf[4][4];
+    warp_logits<DK>(qa, smem_u32(ks), sf);
+    // scale, mask keys past the cache, warp max per head row (rows gr, gr+8)
+    float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int key = nt * 8 + tg * 2 + (e & 1);
+            float v = key < nval ? sf[nt][e] * p.scale_log2 : -INFINITY;
+            sf[nt][e] = v;
+            if (e < 2) m0 = fmaxf(m0, v);
+            else m1 = fmaxf(m1, v);
+        }
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
+        m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
+    }
+    if (tg == 0) {
+        redm[warp][gr] = m0;
+        redm[warp][gr + 8] = m1;
+    }
+    __syncthreads();
+    m0 = fmaxf(fmaxf(redm[0][gr], redm[1][gr]), fmaxf(redm[2][gr], redm[3][gr]));
+    m1 = fmaxf(fmaxf(redm[0][gr + 8], redm[1][gr + 8]), fmaxf(redm[2][gr + 8], redm[3][gr + 8]));
+    // P = exp2(s - split max); row sums; per-head block sums (overlap weights)
+    const int cps = p.l / p.d, spb = p.lp / p.d;
+    const int nj = kDecCH / spb + (cps + spb - 2) / spb + 1;   // blocks this split touches
+    for (int e = lane; e < 16 * kDecWJB; e += 32) bsw[warp][e / kDecWJB][e % kDecWJB] = 0.f;
+    const int wj0 = (warp * 32) / spb;                        // first block this warp touches
+    __syncwarp();
+    float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float mm = e < 2 ? m0 : m1;
+            const float pv = sf[nt][e] == -INFINITY ? 0.f : exp2f(sf[nt][e] - mm);
+            sf[nt][e] = pv;
+            if (e < 2) l0 += pv;
+            else l1 += pv;
+        }
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+    }
+    // block sums: lanes of a quad own disjoint keys of the same two heads;
+    // accumulate per key in a fixed order (deterministic)
+    for (int q = 0; q < 4; ++q) {
+        if (tg == q) {
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int kl = nt * 8 + tg * 2 + (e & 1);
+                    const int row = e < 2 ? gr : gr + 8;
+                    const int ig = warp * 32 + kl;            // key index within the split
+                    for (int u = 0; u < cps; ++u) {
+                        const int jl = (ig + u) / spb - wj0;
+                        bsw[warp][row][jl] += sf[nt][e];
+                    }
+                }
+        }
+        __syncwarp();
+    }
+    if (tg == 0) {
+        redl[warp][gr] = l0;
+        redl[warp][gr + 8] = l1;
+    }
+    // P.V~ of this warp's keys
+    float o[DV / 8][4];
+#pragma unroll
+    for (int nt = 0; nt < DV / 8; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+    warp_pv<DV>(sf, smem_u32(vs), o);
+    __syncthreads();
+    // sum the 4 warps' O in shared memory (reusing the staging area), fixed order
+    float* ored = reinterpret_cast<float*>(dsm);          // [4][16][DV]
+#pragma unroll
+    for (int nt = 0; nt < DV / 8; ++nt) {
+        const int ch = nt * 8 + tg * 2;
+        ored[(warp * 16 + gr) * DV + ch] = o[nt][0];
+        ored[(warp * 16 + gr) * DV + ch + 1] = o[nt][1];
+        ored[(warp * 16 + gr + 8) * DV + ch] = o[nt][2];
+        ored[(warp * 16 + gr + 8) * DV + ch + 1] = o[nt][3];
+    }
+    __syncthreads();
+    float* dst = p.part1 + (((size_t)s * p.G + g) * p.NSPL + sp) * 16 * (2 + DV);
+    for (int e = threadIdx.x; e < 16 * DV; e += 128) {
+        const int h = e / DV, c = e % DV;
+        dst[h * (2 + DV) + 2 + c] = ored[h * DV + c] + ored[(16 + h) * DV + c] + ored[(32 + h) * DV + c] +
+                                    ored[(48 + h) * DV + c];
+    }
+    if (threadIdx.x < 16) {
+        const int h = threadIdx.x;
+        dst[h * (2 + DV)] = fmaxf(fmaxf(redm[0][h], redm[1][h]), fmaxf(redm[2][h], redm[3][h]));
+        dst[h * (2 + DV) + 1] = redl[0][h] + redl[1][h] + redl[2][h] + redl[3][h];
+    }
+    float* bdst = p.bsc + (((size_t)s * p.G + g) * p.NSPL + sp) * 16 * kDecNJB;
+    for (int e = threadIdx.x; e < 16 * kDecNJB; e += 128) {
+        const int h = e / kDecNJB, j = e % kDecNJB;
+        float acc = 0.f;
+        if (j < nj) {
+#pragma unroll
+            for (int w2 = 0; w2 < 4; ++w2) {      // fixed order: deterministic
+                const int jl = j - (w2 * 32) / spb;
+                if (jl >= 0 && jl < kDecWJB) acc += bsw[w2][h][jl];
+            }
+        }
+        bdst[e] = acc;
+    }
+}
+
+// -------------------------------------------------------------- step 2
+template <int DV>
+__global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
+    extern __shared__ float pg[];                      // [NSmax]
+    __shared__ float lse2[16];
+    __shared__ float fac[kDecMaxSplits][16];           // per split scale exp2(m_split - LSE)
+    const int g = blockIdx.x, s = blockIdx.y;
+    const int64_t cbase = p.cmp_off[s];
+    const int C = (int)(p.cmp_off[s + 1] - cbase);
+    const int L = (int)(p.kv_off[s + 1] - p.kv_off[s]);
+    const int t = L - 1;
+    if (C > p.Cmax || L <= 0) return;
+    const int nspl = (C + kDecCH - 1) / kDecCH;
+    const float* part = p.part1 + (((size_t)s * p.G + g) * p.NSPL) * 16 * (2 + DV);
+    if (threadIdx.x < 16) {
+        const int h = threadIdx.x;
+        float M = -INFINITY;
+        for (int i = 0; i < nspl; ++i) M = fmaxf(M, part[((size_t)i * 16 + h) * (2 + DV)]);
+        float Ls = 0.f;
+        for (int i = 0; i < nspl; ++i) {
+            const float* pr = part + ((size_t)i * 16 + h) * (2 + DV);
+            if (pr[0] != -INFINITY) Ls += pr[1] * exp2f(pr[0] - M);
+        }
+        const float l2 = Ls > 0.f ? M + log2f(Ls) : -INFINITY;
+        lse2[h] = l2;
+        p.lsecmp[((size_t)s * p.G + g) * 16 + h] = l2;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < nspl * 16; e += blockDim.x) {
+        const int i = e / 16, h = e % 16;
+        const float m = part[((size_t)i * 16 + h) * (2 + DV)];
+        fac[i][h] = (h < p.HG && m != -INFINITY && lse2[h] != -INFINITY) ? exp2f(m - lse2[h]) : 0.f;
+    }
+    __syncthreads();
+    // o_cmp = sum_i O_i * exp2(m_i - LSE)
+    for (int e = threadIdx.x; e < 16 * DV; e += blockDim.x) {
+        const int h = e / DV, c = e % DV;
+        float acc = 0.f;
+        for (int i = 0; i < nspl; ++i) acc += part[((size_t)i * 16 + h) * (2 + DV) + 2 + c] * fac[i][h];
+        p.ocmp[(((size_t)s * p.G + g) * 16 + h) * DV + c] = acc;
+    }
+    // group scores: block j lies in split j / (128/spb) and, through the
+    // overlap of its last compressed block, in the split before it
+    const int spb = p.lp / p.d;
+    const int per = kDecCH / spb;
+    const int NSs = (L + p.lp - 1) / p.lp;
+    const float* bs = p.bsc + (((size_t)s * p.G + g) * p.NSPL) * 16 * kDecNJB;
+    for (int j = threadIdx.x; j < NSs; j += blockDim.x) {
+        float acc = 0.f;
+        for (int i = max(0, j / per - 1); i <= min(nspl - 1, j / per); ++i) {
+            const int jl = j - i * per;
+            if (jl < 0 || jl >= kDecNJB) continue;
+            for (int h = 0; h < p.HG; ++h) acc += bs[((size_t)i * 16 + h) * kDecNJB + jl] * fac[i][h];
+        }
+        pg[j] = acc;
+    }
+    __syncthreads();
+    if (threadIdx.x < 32)
+        topn_row_warp(pg, t, p.n, p.lp, p.fi, p.fl, p.sel_idx + ((size_t)s * p.G + g) * p.n, threadIdx.x);
 }
 
 // sorted union of the selected blocks and the blocks overlapping the window
@@ -73,156 +382,16 @@ __device__ __forceinline__ int dec_units(const DecParams& p, const int32_t* sel,
     return cnt;
 }
 
-// -------------------------------------------------------------- step 1
-__global__ void __launch_bounds__(256) dec_cmp_partial(const DecParams p) {
-    __shared__ float qs[16 * 192];
-    __shared__ float Sm[16][kDecCH];
-    const int sp = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
-    const int64_t cbase = p.cmp_off[s];
-    const int C = (int)(p.cmp_off[s + 1] - cbase);
-    if (C > p.Cmax) {
-        if (threadIdx.x == 0 && sp == 0) atomicOr(&g_nsa_error, 4u);
-        return;
-    }
-    const int c0 = sp * kDecCH;
-    if (c0 >= C) return;
-    const int nk = min(kDecCH, C - c0);
-    dec_load_q(p, s, g, qs);
-    __syncthreads();
-    {
-        const int k = threadIdx.x & 127, hb = (threadIdx.x >> 7) * 8;
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (k < nk) {
-            const __nv_bfloat16* row = p.kccache + ((cbase + c0 + k) * p.G + g) * p.DK;
-            for (int c = 0; c < p.DK; c += 8) {
-                float kv[8];
-                load8(row + c, kv);
-#pragma unroll
-                for (int h = 0; h < 8; ++h)
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) acc[h] += qs[(hb + h) * p.DK + c + e] * kv[e];
-            }
-        }
-        float* lg = p.logits + (((size_t)s * p.G + g) * 16) * p.Cmax;
-#pragma unroll
-        for (int h = 0; h < 8; ++h) {
-            const float v = k < nk ? acc[h] * p.scale_log2 : -INFINITY;
-            Sm[hb + h][k] = v;
-            if (k < nk) lg[(size_t)(hb + h) * p.Cmax + c0 + k] = v;
-        }
-    }
-    __syncthreads();
-    const int h = threadIdx.x >> 4, sub = threadIdx.x & 15;
-    float m = -INFINITY;
-    for (int k = sub; k < kDecCH; k += 16) m = fmaxf(m, Sm[h][k]);
-#pragma unroll
-    for (int o = 8; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float l = 0.f;
-    for (int k = sub; k < kDecCH; k += 16) {
-        const float e = Sm[h][k] == -INFINITY ? 0.f : exp2f(Sm[h][k] - m);
-        Sm[h][k] = e;
-        l += e;
-    }
-#pragma unroll
-    for (int o = 8; o >= 1; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    __syncthreads();
-    // P.V~: thread (h, channel group)
-    const int cw = p.DV / 16, cg = sub;
-    float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int k = 0; k < nk; ++k) {
-        const float pk = Sm[h][k];
-        const __nv_bfloat16* vr = p.vccache + ((cbase + c0 + k) * p.G + g) * p.DV + cg * cw;
-        if (cw == 8) {
-            float vv[8];
-            load8(vr, vv);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) o[e] += pk * vv[e];
-        } else {
-            for (int e = 0; e < cw; ++e) o[e] += pk * __bfloat162float(vr[e]);
-        }
-    }
-    float* dst = p.part1 + ((((size_t)s * p.G + g) * p.NSPL + sp) * 16 + h) * (2 + p.DV);
-    if (sub == 0) {
-        dst[0] = m;
-        dst[1] = l;
-    }
-    for (int e = 0; e < cw; ++e) dst[2 + cg * cw + e] = o[e];
-}
-
-// -------------------------------------------------------------- step 2
-__global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
-    extern __shared__ float dsm[];
-    float* psum = dsm;                    // [Cmax]
-    float* pg = dsm + p.Cmax;             // [NSmax]
-    __shared__ float lse2[16];
-    const int g = blockIdx.x, s = blockIdx.y;
-    const int64_t cbase = p.cmp_off[s];
-    const int C = (int)(p.cmp_off[s + 1] - cbase);
-    const int L = (int)(p.kv_off[s + 1] - p.kv_off[s]);
-    const int t = L - 1;
-    if (C > p.Cmax || L <= 0) return;
-    const int nspl = (C + kDecCH - 1) / kDecCH;
-    const int h = threadIdx.x >> 4, sub = threadIdx.x & 15;
-    const float* part = p.part1 + (((size_t)s * p.G + g) * p.NSPL) * 16 * (2 + p.DV);
-    float M = -INFINITY;
-    for (int i = 0; i < nspl; ++i) M = fmaxf(M, part[((size_t)i * 16 + h) * (2 + p.DV)]);
-    float Lsum = 0.f;
-    for (int i = 0; i < nspl; ++i) {
-        const float* pr = part + ((size_t)i * 16 + h) * (2 + p.DV);
-        if (pr[0] != -INFINITY) Lsum += pr[1] * exp2f(pr[0] - M);
-    }
-    const int cw = p.DV / 16;
-    for (int e = 0; e < cw; ++e) {
-        const int c = sub * cw + e;
-        float acc = 0.f;
-        for (int i = 0; i < nspl; ++i) {
-            const float* pr = part + ((size_t)i * 16 + h) * (2 + p.DV);
-            if (pr[0] != -INFINITY) acc += pr[2 + c] * exp2f(pr[0] - M);
-        }
-        p.ocmp[(((size_t)s * p.G + g) * 16 + h) * p.DV + c] = Lsum > 0.f ? acc / Lsum : 0.f;
-    }
-    const float l2 = Lsum > 0.f ? M + log2f(Lsum) : -INFINITY;
-    if (sub == 0) {
-        lse2[h] = l2;
-        p.lsecmp[((size_t)s * p.G + g) * 16 + h] = l2;
-    }
-    __syncthreads();
-    // compressed probabilities summed over the group's heads
-    const float* lg = p.logits + (((size_t)s * p.G + g) * 16) * p.Cmax;
-    for (int i = threadIdx.x; i < C; i += blockDim.x) {
-        float acc = 0.f;
-        for (int hh = 0; hh < p.HG; ++hh)
-            if (lse2[hh] != -INFINITY) acc += exp2f(lg[(size_t)hh * p.Cmax + i] - lse2[hh]);
-        psum[i] = acc;
-    }
-    __syncthreads();
-    // mapped to selection blocks with the overlap weights
-    const int cps = p.l / p.d, spb = p.lp / p.d;
-    const int NSs = (L + p.lp - 1) / p.lp;
-    for (int j = threadIdx.x; j < NSs; j += blockDim.x) {
-        float acc = 0.f;
-        for (int i = j * spb - cps + 1; i <= j * spb + spb - 1; ++i) {
-            if (i < 0 || i >= C) continue;
-            int wgt = 0;
-            for (int u = 0; u < cps; ++u) wgt += ((i + u) / spb == j);
-            acc += (float)wgt * psum[i];
-        }
-        pg[j] = acc;
-    }
-    __syncthreads();
-    if (threadIdx.x < 32)
-        topn_row_warp(pg, t, p.n, p.lp, p.fi, p.fl, p.sel_idx + ((size_t)s * p.G + g) * p.n,
-                      threadIdx.x);
-}
-
 // -------------------------------------------------------------- step 3
-__global__ void __launch_bounds__(256) dec_slcwin_partial(const DecParams p) {
-    __shared__ float qs[16 * 192];
-    __shared__ float Sm[16][kDecUnit];
-    __shared__ float P0[16][kDecUnit], P1[16][kDecUnit];
+template <int DK, int DV>
+__global__ void __launch_bounds__(64) dec_slcwin_partial(const DecParams p) {
+    constexpr int KP = DK * 2 + 16, VP = DV * 2 + 16;
+    extern __shared__ __align__(16) uint8_t dsm[];
+    __shared__ float red[2][2][2][16];     // [branch][max|sum][warp][head]
     __shared__ int list[48];
     __shared__ int nlist;
     const int ui = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gr = lane >> 2, tg = lane & 3;
     const int64_t kb = p.kv_off[s];
     const int L = (int)(p.kv_off[s + 1] - kb);
     if (L <= 0) return;
@@ -233,136 +402,162 @@ __global__ void __launch_bounds__(256) dec_slcwin_partial(const DecParams p) {
     const int blk = list[ui];
     bool in_sel = false;
     for (int a = 0; a < p.n; ++a) in_sel |= (sel[a] == blk);
-    dec_load_q(p, s, g, qs);
-    __syncthreads();
-    {
-        const int k = threadIdx.x & 63, hb = (threadIdx.x >> 6) * 4;
-        const int u = blk * p.lp + k;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        if (u < L) {
-            const __nv_bfloat16* row = p.kcache + ((kb + u) * p.G + g) * p.DK;
-            for (int c = 0; c < p.DK; c += 8) {
-                float kv[8];
-                load8(row + c, kv);
+    uint8_t* ks = dsm + warp * 32 * (KP + VP);
+    uint8_t* vs = ks + 32 * KP;
+    const int u0 = blk * p.lp + warp * 32;                    // first token of this warp
+    const int nval = max(0, min(32, L - u0));
+    warp_copy_rows(ks, KP, p.kcache + ((kb + u0) * p.G + g) * DK, (size_t)p.G * DK, 32, nval, DK);
+    warp_copy_rows(vs, VP, p.vcache + ((kb + u0) * p.G + g) * DV, (size_t)p.G * DV, 32, nval, DV);
+    uint32_t qa[DK / 16][4];
+    load_q_frags<DK>(p, s, g, qa);
+    cp_async_wait();
+    __syncwarp();
+    float sf[4][4];
+    warp_logits<DK>(qa, smem_u32(ks), sf);
+    float mx[2][2];
 #pragma unroll
-                for (int h = 0; h < 4; ++h)
+    for (int br = 0; br < 2; ++br) mx[br][0] = mx[br][1] = -INFINITY;
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) acc[h] += qs[(hb + h) * p.DK + c + e] * kv[e];
-            }
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int u = u0 + nt * 8 + tg * 2 + (e & 1);
+            const float v = u < L ? sf[nt][e] * p.scale_log2 : -INFINITY;
+            sf[nt][e] = v;
+            if (in_sel) mx[0][e >> 1] = fmaxf(mx[0][e >> 1], v);
+            if (u >= L - p.w) mx[1][e >> 1] = fmaxf(mx[1][e >> 1], v);
         }
 #pragma unroll
-        for (int h = 0; h < 4; ++h) Sm[hb + h][k] = u < L ? acc[h] * p.scale_log2 : -INFINITY;
+    for (int br = 0; br < 2; ++br)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+            for (int o = 1; o <= 2; o <<= 1) mx[br][hf] = fmaxf(mx[br][hf], __shfl_xor_sync(0xffffffffu, mx[br][hf], o));
+    if (tg == 0) {
+#pragma unroll
+        for (int br = 0; br < 2; ++br) {
+            red[br][0][warp][gr] = mx[br][0];
+            red[br][0][warp][gr + 8] = mx[br][1];
+        }
     }
     __syncthreads();
-    const int h = threadIdx.x >> 4, sub = threadIdx.x & 15;
-    float mb[2], lb[2];
 #pragma unroll
     for (int br = 0; br < 2; ++br) {
-        float m = -INFINITY;
-        for (int k = sub; k < kDecUnit; k += 16) {
-            const int u = blk * p.lp + k;
-            const bool f = br == 0 ? (in_sel && u < L) : (u < L && u >= L - p.w);
-            if (f) m = fmaxf(m, Sm[h][k]);
-        }
-#pragma unroll
-        for (int o = 8; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        float l = 0.f;
-        for (int k = sub; k < kDecUnit; k += 16) {
-            const int u = blk * p.lp + k;
-            const bool f = br == 0 ? (in_sel && u < L) : (u < L && u >= L - p.w);
-            const float e = (f && m != -INFINITY) ? exp2f(Sm[h][k] - m) : 0.f;
-            (br == 0 ? P0 : P1)[h][k] = e;
-            l += e;
-        }
-#pragma unroll
-        for (int o = 8; o >= 1; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-        mb[br] = m;
-        lb[br] = l;
+        mx[br][0] = fmaxf(red[br][0][0][gr], red[br][0][1][gr]);
+        mx[br][1] = fmaxf(red[br][0][0][gr + 8], red[br][0][1][gr + 8]);
     }
-    __syncthreads();
-    const int cw = p.DV / 16, cg = sub;
-    float o0[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, o1[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    const int nk = min(kDecUnit, L - blk * p.lp);
-    for (int k = 0; k < nk; ++k) {
-        const float a0 = P0[h][k], a1 = P1[h][k];
-        const __nv_bfloat16* vr = p.vcache + ((kb + blk * p.lp + k) * p.G + g) * p.DV + cg * cw;
-        if (cw == 8) {
-            float vv[8];
-            load8(vr, vv);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                o0[e] += a0 * vv[e];
-                o1[e] += a1 * vv[e];
-            }
-        } else {
-            for (int e = 0; e < cw; ++e) {
-                const float vv = __bfloat162float(vr[e]);
-                o0[e] += a0 * vv;
-                o1[e] += a1 * vv;
-            }
-        }
-    }
+    float ls[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+    float o[2][DV / 8][4];
 #pragma unroll
     for (int br = 0; br < 2; ++br) {
-        float* dst = p.part2 + (((((size_t)s * p.G + g) * p.NU + ui) * 2 + br) * 16 + h) * (2 + p.DV);
-        if (sub == 0) {
-            dst[0] = mb[br];
-            dst[1] = lb[br];
+        float pf[4][4];
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int u = u0 + nt * 8 + tg * 2 + (e & 1);
+                const bool f = br == 0 ? (in_sel && u < L) : (u < L && u >= L - p.w);
+                const float m = mx[br][e >> 1];
+                const float pv = (f && m != -INFINITY) ? exp2f(sf[nt][e] - m) : 0.f;
+                pf[nt][e] = pv;
+                ls[br][e >> 1] += pv;
+            }
+#pragma unroll
+        for (int nt = 0; nt < DV / 8; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[br][nt][e] = 0.f;
+        warp_pv<DV>(pf, smem_u32(vs), o[br]);
+    }
+#pragma unroll
+    for (int br = 0; br < 2; ++br)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+            for (int q2 = 1; q2 <= 2; q2 <<= 1) ls[br][hf] += __shfl_xor_sync(0xffffffffu, ls[br][hf], q2);
+    if (tg == 0) {
+#pragma unroll
+        for (int br = 0; br < 2; ++br) {
+            red[br][1][warp][gr] = ls[br][0];
+            red[br][1][warp][gr + 8] = ls[br][1];
         }
-        for (int e = 0; e < cw; ++e) dst[2 + cg * cw + e] = br == 0 ? o0[e] : o1[e];
+    }
+    __syncthreads();
+    float* ored = reinterpret_cast<float*>(dsm);            // [2 br][2 warps][16][DV]
+#pragma unroll
+    for (int br = 0; br < 2; ++br)
+#pragma unroll
+        for (int nt = 0; nt < DV / 8; ++nt) {
+            const int ch = nt * 8 + tg * 2;
+            float* base = ored + ((br * 2 + warp) * 16) * DV;
+            base[gr * DV + ch] = o[br][nt][0];
+            base[gr * DV + ch + 1] = o[br][nt][1];
+            base[(gr + 8) * DV + ch] = o[br][nt][2];
+            base[(gr + 8) * DV + ch + 1] = o[br][nt][3];
+        }
+    __syncthreads();
+#pragma unroll
+    for (int br = 0; br < 2; ++br) {
+        float* dst = p.part2 + (((((size_t)s * p.G + g) * p.NU + ui) * 2 + br) * 16) * (2 + DV);
+        for (int e = threadIdx.x; e < 16 * DV; e += 64) {
+            const int h = e / DV, c = e % DV;
+            dst[h * (2 + DV) + 2 + c] = ored[((br * 2 + 0) * 16 + h) * DV + c] + ored[((br * 2 + 1) * 16 + h) * DV + c];
+        }
+        if (threadIdx.x < 16) {
+            const int h = threadIdx.x;
+            dst[h * (2 + DV)] = fmaxf(red[br][0][0][h], red[br][0][1][h]);
+            dst[h * (2 + DV) + 1] = red[br][1][0][h] + red[br][1][1][h];
+        }
     }
 }
 
 // -------------------------------------------------------------- step 4
+template <int DV>
 __global__ void __launch_bounds__(256) dec_final(const DecParams p) {
     __shared__ int list[48];
     __shared__ int nlist;
+    __shared__ float fac[2][48][16];
+    __shared__ float Lb[2][16];
     const int g = blockIdx.x, s = blockIdx.y;
     const int L = (int)(p.kv_off[s + 1] - p.kv_off[s]);
     if (L <= 0) return;
     const int32_t* sel = p.sel_idx + ((size_t)s * p.G + g) * p.n;
     if (threadIdx.x == 0) nlist = dec_units(p, sel, L, list);
     __syncthreads();
-    const int h = threadIdx.x >> 4, sub = threadIdx.x & 15;
-    const int cw = p.DV / 16;
-    float Mb[2], Lb[2];
-#pragma unroll
-    for (int br = 0; br < 2; ++br) {
+    const float* part = p.part2 + ((((size_t)s * p.G + g) * p.NU) * 2) * 16 * (2 + DV);
+    if (threadIdx.x < 32) {
+        const int br = threadIdx.x / 16, h = threadIdx.x % 16;
         float M = -INFINITY;
-        for (int u = 0; u < nlist; ++u)
-            M = fmaxf(M, p.part2[(((((size_t)s * p.G + g) * p.NU + u) * 2 + br) * 16 + h) * (2 + p.DV)]);
+        for (int u = 0; u < nlist; ++u) M = fmaxf(M, part[(((size_t)u * 2 + br) * 16 + h) * (2 + DV)]);
         float Ls = 0.f;
         for (int u = 0; u < nlist; ++u) {
-            const float* pr = p.part2 + (((((size_t)s * p.G + g) * p.NU + u) * 2 + br) * 16 + h) * (2 + p.DV);
-            if (pr[0] != -INFINITY) Ls += pr[1] * exp2f(pr[0] - M);
+            const float* pr = part + (((size_t)u * 2 + br) * 16 + h) * (2 + DV);
+            const float f = pr[0] != -INFINITY ? exp2f(pr[0] - M) : 0.f;
+            fac[br][u][h] = f;
+            Ls += pr[1] * f;
         }
-        Mb[br] = M;
-        Lb[br] = Ls;
-    }
-    if (h < p.HG) {
-        const size_t row = (size_t)s * p.H + g * p.HG + h;
-        const float g0 = p.gates[row * 3 + 0], g1 = p.gates[row * 3 + 1], g2 = p.gates[row * 3 + 2];
-        for (int e = 0; e < cw; ++e) {
-            const int c = sub * cw + e;
-            float ob[2];
-#pragma unroll
-            for (int br = 0; br < 2; ++br) {
-                float acc = 0.f;
-                for (int u = 0; u < nlist; ++u) {
-                    const float* pr = p.part2 + (((((size_t)s * p.G + g) * p.NU + u) * 2 + br) * 16 + h) * (2 + p.DV);
-                    if (pr[0] != -INFINITY) acc += pr[2 + c] * exp2f(pr[0] - Mb[br]);
-                }
-                ob[br] = Lb[br] > 0.f ? acc / Lb[br] : 0.f;
+        Lb[br][h] = Ls;
+        if (h < p.HG && p.lse) {
+            const size_t row = (size_t)s * p.H + g * p.HG + h;
+            p.lse[row * 3 + 1 + br] = Ls > 0.f ? (M + log2f(Ls)) * kLn2 : -INFINITY;
+            if (br == 0) {
+                const float lc = p.lsecmp[((size_t)s * p.G + g) * 16 + h];
+                p.lse[row * 3] = lc == -INFINITY ? -INFINITY : lc * kLn2;
             }
-            const float oc = p.ocmp[(((size_t)s * p.G + g) * 16 + h) * p.DV + c];
-            p.out[row * p.DV + c] = g0 * oc + g1 * ob[0] + g2 * ob[1];
         }
-        if (sub == 0 && p.lse) {
-            const float lc = p.lsecmp[((size_t)s * p.G + g) * 16 + h];
-            p.lse[row * 3 + 0] = lc == -INFINITY ? -INFINITY : lc * kLn2;
-            p.lse[row * 3 + 1] = Lb[0] > 0.f ? (Mb[0] + log2f(Lb[0])) * kLn2 : -INFINITY;
-            p.lse[row * 3 + 2] = Lb[1] > 0.f ? (Mb[1] + log2f(Lb[1])) * kLn2 : -INFINITY;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < p.HG * DV; e += blockDim.x) {
+        const int h = e / DV, c = e % DV;
+        float ob[2];
+#pragma unroll
+        for (int br = 0; br < 2; ++br) {
+            float acc = 0.f;
+            for (int u = 0; u < nlist; ++u) acc += part[(((size_t)u * 2 + br) * 16 + h) * (2 + DV) + 2 + c] * fac[br][u][h];
+            ob[br] = Lb[br][h] > 0.f ? acc / Lb[br][h] : 0.f;
         }
+        const size_t row = (size_t)s * p.H + g * p.HG + h;
+        const float oc = p.ocmp[(((size_t)s * p.G + g) * 16 + h) * DV + c];   // normalised
+        p.out[row * DV + c] = p.gates[row * 3] * oc + p.gates[row * 3 + 1] * ob[0] + p.gates[row * 3 + 2] * ob[1];
     }
 }
 
@@ -374,8 +569,8 @@ inline size_t decode_ws_bytes(int64_t S, int64_t Lmax, int64_t G, int64_t l, int
     const int64_t NU = n + (w + lp - 1) / lp + 1;
     auto a = [](size_t x) { return (x + 255) & ~size_t(255); };
     size_t o = 0;
-    o += a((size_t)S * G * 16 * Cmax * 4);
     o += a((size_t)S * G * NSPL * 16 * (2 + DV) * 4);
+    o += a((size_t)S * G * NSPL * 16 * kDecNJB * 4);
     o += a((size_t)S * G * 16 * DV * 4);
     o += a((size_t)S * G * 16 * 4);
     o += a((size_t)S * G * NU * 2 * 16 * (2 + DV) * 4);

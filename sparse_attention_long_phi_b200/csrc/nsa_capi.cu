@@ -565,6 +565,23 @@ nsa_status_t backward_impl(const Shape& s, const void* q, const void* k, const v
 }
 
 // ---------------------------------------------------------------- decode
+template <int DK, int DV>
+nsa_status_t decode_launch(const DecParams& p, const Shape& s, int S, cudaStream_t st) {
+    const int rows_bytes = 32 * ((DK * 2 + 16) + (DV * 2 + 16));
+    NSA_TRY(set_smem(dec_cmp_partial<DK, DV>, 4 * rows_bytes));
+    NSA_LAUNCH("dec_cmp_partial", st, dec_cmp_partial<DK, DV><<<dim3((unsigned)p.NSPL, (unsigned)s.G, (unsigned)S), 128, 4 * rows_bytes, st>>>(p));
+    NSA_TRY(last_launch());
+    const int smem2 = p.NSmax * 4;
+    NSA_TRY(set_smem(dec_cmp_combine<DV>, smem2));
+    NSA_LAUNCH("dec_cmp_combine", st, dec_cmp_combine<DV><<<dim3((unsigned)s.G, (unsigned)S), 256, smem2, st>>>(p));
+    NSA_TRY(last_launch());
+    NSA_TRY(set_smem(dec_slcwin_partial<DK, DV>, 2 * rows_bytes));
+    NSA_LAUNCH("dec_slcwin_partial", st, dec_slcwin_partial<DK, DV><<<dim3((unsigned)p.NU, (unsigned)s.G, (unsigned)S), 64, 2 * rows_bytes, st>>>(p));
+    NSA_TRY(last_launch());
+    NSA_LAUNCH("dec_final", st, dec_final<DV><<<dim3((unsigned)s.G, (unsigned)S), 256, 0, st>>>(p));
+    return last_launch();
+}
+
 nsa_status_t decode_impl(const Shape& s, int S, const void* q, const void* kcache, const void* vcache,
                          const int64_t* kv_off, const void* kccache, const void* vccache,
                          const int64_t* cmp_off, const float* gates, float* out, int32_t* sel_idx,
@@ -599,27 +616,20 @@ nsa_status_t decode_impl(const Shape& s, int S, const void* q, const void* kcach
     p.NSPL = (int)ceil_div(p.Cmax, kDecCH);
     p.NU = (int)(s.n + ceil_div(s.w, s.lp) + 1);
     p.NSmax = (int)ceil_div(s.T, s.lp);
+    if (p.NSPL > kDecMaxSplits || p.NU > 48) return NSA_ERR_UNSUPPORTED;
     size_t o = 0;
     auto carve = [&](size_t bytes) {
         float* r = reinterpret_cast<float*>(ws + o);
         o = align256(o + bytes);
         return r;
     };
-    p.logits = carve((size_t)S * s.G * 16 * p.Cmax * 4);
     p.part1 = carve((size_t)S * s.G * p.NSPL * 16 * (2 + s.DV) * 4);
+    p.bsc = carve((size_t)S * s.G * p.NSPL * 16 * kDecNJB * 4);
     p.ocmp = carve((size_t)S * s.G * 16 * s.DV * 4);
     p.lsecmp = carve((size_t)S * s.G * 16 * 4);
     p.part2 = carve((size_t)S * s.G * p.NU * 2 * 16 * (2 + s.DV) * 4);
-    NSA_LAUNCH("dec_cmp_partial", st, dec_cmp_partial<<<dim3((unsigned)p.NSPL, (unsigned)s.G, (unsigned)S), 256, 0, st>>>(p));
-    NSA_TRY(last_launch());
-    const int smem2 = (p.Cmax + p.NSmax) * 4;
-    NSA_TRY(set_smem(dec_cmp_combine, smem2));
-    NSA_LAUNCH("dec_cmp_combine", st, dec_cmp_combine<<<dim3((unsigned)s.G, (unsigned)S), 256, smem2, st>>>(p));
-    NSA_TRY(last_launch());
-    NSA_LAUNCH("dec_slcwin_partial", st, dec_slcwin_partial<<<dim3((unsigned)p.NU, (unsigned)s.G, (unsigned)S), 256, 0, st>>>(p));
-    NSA_TRY(last_launch());
-    NSA_LAUNCH("dec_final", st, dec_final<<<dim3((unsigned)s.G, (unsigned)S), 256, 0, st>>>(p));
-    return last_launch();
+    if (s.DK == 192) return decode_launch<192, 128>(p, s, S, st);
+    return decode_launch<64, 64>(p, s, S, st);
 }
 
 }  // namespace

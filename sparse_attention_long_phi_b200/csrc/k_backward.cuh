@@ -9,8 +9,12 @@
 // member token; linear: W^T dK~ scattered over the overlapping blocks).
 //
 // Kernels (SIMT, fp32 accumulation):
-//   bwd_query_kernel     one CTA per (b, t, g): recomputes every branch's LSE
-//                        and o_c, writes dgates and D_c, accumulates dq.
+//   bwd_query_mma        one CTA per (b, t, g) on warp-level bf16 tensor cores
+//                        (the 16 heads of the group are the M side): pass 1
+//                        recomputes every branch's LSE and o_c (online softmax
+//                        per warp, merged across warps) and writes dgates and
+//                        D_c; pass 2 recomputes S and dP = dO_c V^T, forms dS
+//                        and accumulates dq = scale dS K.
 //   bwd_kv_kernel<BR>    key-centric: a tile of 64 keys (raw tokens for the
 //                        window and selected branches, compressed blocks for
 //                        the compressed one) accumulates over the queries that
@@ -20,6 +24,7 @@
 //   bwd_phiT_kernel      dk/dv += phi^T(dK~/dV~).
 #pragma once
 #include "nsa_dev.cuh"
+#include "k_mma.cuh"
 
 namespace nsa {
 
@@ -43,196 +48,258 @@ __device__ __forceinline__ int ncmp_vis(const BwdParams& p, int t) {
     return (t + 1 >= p.l) ? (t + 1 - p.l) / p.d + 1 : 0;
 }
 
-// ------------------------------------------------------------ per query
+// ------------------------------------------------ per query, tensor cores
+// Shared memory: 4 warps x (32 K rows + 32 V rows) staging (reused for the
+// cross-warp merges), then dO_t of the group as a [16][DV] bf16 tile.
 template <int DK, int DV>
-__global__ void __launch_bounds__(256) bwd_query_kernel(const BwdParams p) {
-    extern __shared__ float sm[];
-    float* qf = sm;                                // [16][DK+1]
-    float* dof = qf + 16 * (DK + 1);               // [16][DV+1]
-    float* Kc = dof + 16 * (DV + 1);               // [64][DK+1]
-    float* Vc = Kc + 64 * (DK + 1);                // [64][DV+1]
-    float* Sb = Vc + 64 * (DV + 1);                // [16][64]
-    float* hl = Sb + 16 * 64;                      // [16] lse2 of the branch
+constexpr int bwd_query_mma_smem() {
+    return 4 * 32 * ((DK * 2 + 16) + (DV * 2 + 16)) + 16 * (DV * 2 + 16);
+}
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(128) bwd_query_mma(const BwdParams p) {
+    constexpr int KP = DK * 2 + 16, VP = DV * 2 + 16;
+    constexpr int STAGE = 4 * 32 * (KP + VP);
+    static_assert(4 * 16 * DK * 4 <= STAGE && 4 * 16 * DV * 4 <= STAGE, "merge buffers");
+    extern __shared__ __align__(16) uint8_t bsm[];
+    __shared__ float wm[4][16], wl[4][16], Lsum[16];
+    __shared__ float lse2s[3][16], Ds[3][16], gs[3][16];
     __shared__ int units[16];
     __shared__ int nunits;
-    constexpr int DKT = DK / 16, DVT = DV / 16;
-
     const int t = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-    const int tid = threadIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gr = lane >> 2, tg = lane & 3;
     const size_t rowbase = ((size_t)b * p.T + t) * p.H + (size_t)g * p.HG;
-    for (int e = tid; e < 16 * DK; e += 256) {
-        const int h = e / DK, c = e % DK;
-        qf[h * (DK + 1) + c] = h < p.HG ? __bfloat162float(p.q[(rowbase + h) * DK + c]) : 0.f;
-    }
-    for (int e = tid; e < 16 * DV; e += 256) {
-        const int h = e / DV, c = e % DV;
-        dof[h * (DV + 1) + c] = h < p.HG ? __bfloat162float(p.dout[(rowbase + h) * DV + c]) : 0.f;
-    }
-    if (tid == 0) {
+    uint8_t* ks = bsm + warp * 32 * (KP + VP);
+    uint8_t* vs = ks + 32 * KP;
+    uint8_t* dos = bsm + STAGE;
+    if (threadIdx.x == 0) {
         int nu = 0;
         const int32_t* r = p.idx + (((size_t)b * p.T + t) * p.G + g) * p.n;
         for (int a = 0; a < p.n; ++a)
             if (r[a] >= 0) units[nu++] = r[a];
         nunits = nu;
     }
+    for (int e = threadIdx.x; e < 16 * (DV / 8); e += 128) {     // dO tile, zero rows past HG
+        const int h = e / (DV / 8), cc = e % (DV / 8);
+        int4 v = make_int4(0, 0, 0, 0);
+        if (h < p.HG) v = *reinterpret_cast<const int4*>(p.dout + (rowbase + h) * DV + cc * 8);
+        *reinterpret_cast<int4*>(dos + h * VP + cc * 16) = v;
+    }
+    if (threadIdx.x < 48) {
+        const int br = threadIdx.x / 16, h = threadIdx.x % 16;
+        gs[br][h] = h < p.HG ? p.gates[(rowbase + h) * 3 + br] : 0.f;
+    }
     __syncthreads();
+    uint32_t qa[DK / 16][4];
+    load_a_frags<DK>(p.q + rowbase * DK, p.HG, qa);
+    const float c = p.scale_log2;
 
-    const int hq = tid >> 4, cg = tid & 15;        // (head, channel group) layout
-    const int kk = tid >> 2, part = tid & 3;       // (key, head quarter) layout
-    float dq[DKT];
-#pragma unroll
-    for (int e = 0; e < DKT; ++e) dq[e] = 0.f;
+    // key range of a branch; row pointers (nullptr: not seen by the query)
+    auto branch_keys = [&](int br, int& lo) -> int {
+        lo = 0;
+        if (br == kBrCmp) return ncmp_vis(p, t);
+        if (br == kBrSlc) return nunits * p.lp;
+        lo = max(0, t - p.w + 1);
+        return t - lo + 1;
+    };
+    auto token_of = [&](int br, int lo, int key) -> int {
+        return br == kBrSlc ? units[key / p.lp] * p.lp + key % p.lp : lo + key;
+    };
+    auto stage = [&](int br, int lo, int nk, int k0) {
+        warp_copy_rows_ptr(ks, KP, [&](int r) -> const __nv_bfloat16* {
+            const int key = k0 + r;
+            if (key >= nk) return nullptr;
+            if (br == kBrCmp) return p.kc + (((size_t)b * p.C + key) * p.G + g) * DK;
+            const int u = token_of(br, lo, key);
+            return u > t ? nullptr : p.k + (((size_t)b * p.T + u) * p.G + g) * DK;
+        }, 32, DK);
+        warp_copy_rows_ptr(vs, VP, [&](int r) -> const __nv_bfloat16* {
+            const int key = k0 + r;
+            if (key >= nk) return nullptr;
+            if (br == kBrCmp) return p.vc + (((size_t)b * p.C + key) * p.G + g) * DV;
+            const int u = token_of(br, lo, key);
+            return u > t ? nullptr : p.v + (((size_t)b * p.T + u) * p.G + g) * DV;
+        }, 32, DV);
+        cp_async_wait();
+        __syncwarp();
+    };
+    // does key `key` of the branch take part (inside the range, causal)?
+    auto seen = [&](int br, int lo, int nk, int key) -> bool {
+        if (key >= nk) return false;
+        return br != kBrSlc || token_of(br, lo, key) <= t;
+    };
 
+    // ---------------- pass 1, every branch: LSE, o_c, dgates, D
     for (int br = 0; br < 3; ++br) {
-        int nk, lo = 0;
-        if (br == kBrCmp) nk = ncmp_vis(p, t);
-        else if (br == kBrSlc) nk = nunits * p.lp;
-        else {
-            lo = max(0, t - p.w + 1);
-            nk = t - lo + 1;
-        }
-        const float gc = p.gates[(rowbase + min(hq, p.HG - 1)) * 3 + br];
-        // row pointers of a key of this branch; false for keys the query does not
-        // see (tokens after t, which may lie past the end of the sequence)
-        auto key_rows = [&](int key, const __nv_bfloat16*& kr, const __nv_bfloat16*& vr) -> bool {
-            if (br == kBrCmp) {
-                kr = p.kc + (((size_t)b * p.C + key) * p.G + g) * DK;
-                vr = p.vc + (((size_t)b * p.C + key) * p.G + g) * DV;
-                return true;
-            }
-            int u = (br == kBrSlc) ? units[key / p.lp] * p.lp + key % p.lp : lo + key;
-            kr = p.k + (((size_t)b * p.T + u) * p.G + g) * DK;
-            vr = p.v + (((size_t)b * p.T + u) * p.G + g) * DV;
-            return u <= t;
-        };
-        auto load_chunk = [&](int c0) {
-            for (int e = tid; e < 64 * DK; e += 256) {
-                const int key = e / DK, c = e % DK;
-                float val = 0.f;
-                if (c0 + key < nk) {
-                    const __nv_bfloat16 *kr, *vr;
-                    if (key_rows(c0 + key, kr, vr)) val = __bfloat162float(kr[c]);
+        int lo;
+        const int nk = branch_keys(br, lo);
+        const int nch = (nk + 31) / 32;
+        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+        float o[DV / 8][4];
+#pragma unroll
+        for (int nt = 0; nt < DV / 8; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+        for (int ch = warp; ch < nch; ch += 4) {
+            const int k0 = ch * 32;
+            stage(br, lo, nk, k0);
+            float sf[4][4];
+            warp_logits<DK>(qa, smem_u32(ks), sf);
+            float cm0 = -INFINITY, cm1 = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float v = seen(br, lo, nk, k0 + nt * 8 + tg * 2 + (e & 1)) ? sf[nt][e] * c : -INFINITY;
+                    sf[nt][e] = v;
+                    if (e < 2) cm0 = fmaxf(cm0, v);
+                    else cm1 = fmaxf(cm1, v);
                 }
-                Kc[key * (DK + 1) + c] = val;
+#pragma unroll
+            for (int q2 = 1; q2 <= 2; q2 <<= 1) {
+                cm0 = fmaxf(cm0, __shfl_xor_sync(0xffffffffu, cm0, q2));
+                cm1 = fmaxf(cm1, __shfl_xor_sync(0xffffffffu, cm1, q2));
             }
-            for (int e = tid; e < 64 * DV; e += 256) {
-                const int key = e / DV, c = e % DV;
-                float val = 0.f;
-                if (c0 + key < nk) {
-                    const __nv_bfloat16 *kr, *vr;
-                    if (key_rows(c0 + key, kr, vr)) val = __bfloat162float(vr[c]);
+            const float n0 = fmaxf(m0, cm0), n1 = fmaxf(m1, cm1);
+            const float a0 = n0 == -INFINITY ? 1.f : exp2f(m0 - n0);
+            const float a1 = n1 == -INFINITY ? 1.f : exp2f(m1 - n1);
+            m0 = n0;
+            m1 = n1;
+            float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float mm = e < 2 ? m0 : m1;
+                    const float pv = sf[nt][e] == -INFINITY ? 0.f : exp2f(sf[nt][e] - mm);
+                    sf[nt][e] = pv;
+                    if (e < 2) s0 += pv;
+                    else s1 += pv;
                 }
-                Vc[key * (DV + 1) + c] = val;
-            }
-        };
-        auto logits = [&](int c0) {
-            // thread (key kk, heads part*4 .. part*4+3)
-            bool valid = false;
-            if (c0 + kk < nk) {
-                const __nv_bfloat16 *kr, *vr;
-                valid = key_rows(c0 + kk, kr, vr);
-            }
 #pragma unroll
-            for (int hh = 0; hh < 4; ++hh) {
-                const int h = part * 4 + hh;
-                float s = 0.f;
-                for (int c = 0; c < DK; ++c) s += qf[h * (DK + 1) + c] * Kc[kk * (DK + 1) + c];
-                Sb[h * 64 + kk] = valid ? s * p.scale_log2 : -INFINITY;
+            for (int q2 = 1; q2 <= 2; q2 <<= 1) {
+                s0 += __shfl_xor_sync(0xffffffffu, s0, q2);
+                s1 += __shfl_xor_sync(0xffffffffu, s1, q2);
             }
-        };
-        // ---- pass 1: LSE and o_c
-        float m = -INFINITY, l = 0.f;
-        float o[DVT];
+            l0 = l0 * a0 + s0;
+            l1 = l1 * a1 + s1;
 #pragma unroll
-        for (int e = 0; e < DVT; ++e) o[e] = 0.f;
-        for (int c0 = 0; c0 < nk; c0 += 64) {
-            load_chunk(c0);
-            __syncthreads();
-            logits(c0);
-            __syncthreads();
-            float cm = -INFINITY;
-            for (int q2 = cg; q2 < 64; q2 += 16) cm = fmaxf(cm, Sb[hq * 64 + q2]);
-#pragma unroll
-            for (int s2 = 8; s2 >= 1; s2 >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, s2));
-            const float mn = fmaxf(m, cm);
-            const float alpha = (mn == -INFINITY) ? 1.f : exp2f(m - mn);
-            float ls = 0.f;
-            __syncthreads();
-            for (int q2 = cg; q2 < 64; q2 += 16) {
-                const float sv = Sb[hq * 64 + q2];
-                const float e = sv == -INFINITY ? 0.f : exp2f(sv - mn);
-                Sb[hq * 64 + q2] = e;
-                ls += e;
+            for (int nt = 0; nt < DV / 8; ++nt) {
+                o[nt][0] *= a0;
+                o[nt][1] *= a0;
+                o[nt][2] *= a1;
+                o[nt][3] *= a1;
             }
-#pragma unroll
-            for (int s2 = 8; s2 >= 1; s2 >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, s2);
-            l = l * alpha + ls;
-            m = mn;
-            __syncthreads();
-#pragma unroll
-            for (int e = 0; e < DVT; ++e) {
-                float acc = 0.f;
-                for (int q2 = 0; q2 < 64; ++q2) acc += Sb[hq * 64 + q2] * Vc[q2 * (DV + 1) + cg * DVT + e];
-                o[e] = o[e] * alpha + acc;
-            }
-            __syncthreads();
+            warp_pv<DV>(sf, smem_u32(vs), o);
+            __syncwarp();
         }
-        float dg = 0.f;
-#pragma unroll
-        for (int e = 0; e < DVT; ++e) {
-            o[e] = l > 0.f ? o[e] / l : 0.f;
-            dg += o[e] * dof[hq * (DV + 1) + cg * DVT + e];
+        // merge the 4 warps (fixed order): LSE and o_c per head
+        if (tg == 0) {
+            wm[warp][gr] = m0;
+            wm[warp][gr + 8] = m1;
+            wl[warp][gr] = l0;
+            wl[warp][gr + 8] = l1;
         }
+        __syncthreads();                                      // also: staging idle
+        float* ored = reinterpret_cast<float*>(bsm);          // [4][16][DV]
+        {
+            const float M0 = fmaxf(fmaxf(wm[0][gr], wm[1][gr]), fmaxf(wm[2][gr], wm[3][gr]));
+            const float M1 = fmaxf(fmaxf(wm[0][gr + 8], wm[1][gr + 8]), fmaxf(wm[2][gr + 8], wm[3][gr + 8]));
+            const float f0 = m0 == -INFINITY ? 0.f : exp2f(m0 - M0);
+            const float f1 = m1 == -INFINITY ? 0.f : exp2f(m1 - M1);
 #pragma unroll
-        for (int s2 = 8; s2 >= 1; s2 >>= 1) dg += __shfl_xor_sync(0xffffffffu, dg, s2);
-        const float l2 = l > 0.f ? m + log2f(l) : -INFINITY;
-        const float Dc = gc * dg;
-        if (cg == 0) {
-            hl[hq] = l2;
-            if (hq < p.HG) {
-                p.dgates[(rowbase + hq) * 3 + br] = dg;
-                p.lse2[(rowbase + hq) * 3 + br] = l2;
-                p.dlt[(rowbase + hq) * 3 + br] = Dc;
+            for (int nt = 0; nt < DV / 8; ++nt) {
+                const int cc = nt * 8 + tg * 2;
+                *reinterpret_cast<float2*>(ored + (warp * 16 + gr) * DV + cc) = make_float2(o[nt][0] * f0, o[nt][1] * f0);
+                *reinterpret_cast<float2*>(ored + (warp * 16 + gr + 8) * DV + cc) =
+                    make_float2(o[nt][2] * f1, o[nt][3] * f1);
             }
         }
-        // D_c of head part*4+hh for the (key, head quarter) layout
+        if (threadIdx.x < 16) {
+            const int h = threadIdx.x;
+            float M = -INFINITY;
+            for (int w2 = 0; w2 < 4; ++w2) M = fmaxf(M, wm[w2][h]);
+            float L = 0.f;
+            for (int w2 = 0; w2 < 4; ++w2)
+                if (wm[w2][h] != -INFINITY) L += wl[w2][h] * exp2f(wm[w2][h] - M);
+            lse2s[br][h] = L > 0.f ? M + log2f(L) : -INFINITY;
+            Lsum[h] = L;
+        }
         __syncthreads();
-        float Dq[4], gq[4];
+        // dgate_h = <dO_h, o_c,h>, 8 threads per head; D_c = gate * dgate
+        {
+            const int h = threadIdx.x >> 3, part = threadIdx.x & 7;
+            float acc = 0.f;
+            const float L = Lsum[h];
+            if (h < p.HG && L > 0.f) {
+                const __nv_bfloat16* dor = reinterpret_cast<const __nv_bfloat16*>(dos + h * VP);
+                for (int cc = part; cc < DV; cc += 8) {
+                    const float oc = (ored[h * DV + cc] + ored[(16 + h) * DV + cc] + ored[(32 + h) * DV + cc] +
+                                      ored[(48 + h) * DV + cc]) / L;
+                    acc += oc * __bfloat162float(dor[cc]);
+                }
+            }
 #pragma unroll
-        for (int hh = 0; hh < 4; ++hh) {
-            const int h = part * 4 + hh;
-            Dq[hh] = h < p.HG ? p.dlt[(rowbase + h) * 3 + br] : 0.f;
-            gq[hh] = h < p.HG ? p.gates[(rowbase + h) * 3 + br] : 0.f;
+            for (int q2 = 1; q2 <= 4; q2 <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, q2);
+            if (part == 0) {
+                Ds[br][h] = gs[br][h] * acc;
+                if (h < p.HG) {
+                    p.dgates[(rowbase + h) * 3 + br] = acc;
+                    p.lse2[(rowbase + h) * 3 + br] = lse2s[br][h];
+                    p.dlt[(rowbase + h) * 3 + br] = gs[br][h] * acc;
+                }
+            }
         }
-        // ---- pass 2: dS and dq
-        for (int c0 = 0; c0 < nk; c0 += 64) {
-            load_chunk(c0);
-            __syncthreads();
-            logits(c0);
-            __syncthreads();
+        __syncthreads();                                      // ored dead, staging free
+    }
+
+    // ---------------- pass 2, every branch: dS = P (g dP - D), dq += dS K
+    float dq[DK / 8][4];
 #pragma unroll
-            for (int hh = 0; hh < 4; ++hh) {
-                const int h = part * 4 + hh;
-                const float sv = Sb[h * 64 + kk];
-                const float P = (sv == -INFINITY || hl[h] == -INFINITY) ? 0.f : exp2f(sv - hl[h]);
-                float dP = 0.f;
-                for (int c = 0; c < DV; ++c) dP += dof[h * (DV + 1) + c] * Vc[kk * (DV + 1) + c];
-                dP *= gq[hh];
-                Sb[h * 64 + kk] = P * (dP - Dq[hh]);
-            }
-            __syncthreads();
+    for (int nt = 0; nt < DK / 8; ++nt)
 #pragma unroll
-            for (int e = 0; e < DKT; ++e) {
-                float acc = 0.f;
-                for (int q2 = 0; q2 < 64; ++q2) acc += Sb[hq * 64 + q2] * Kc[q2 * (DK + 1) + cg * DKT + e];
-                dq[e] += p.scale * acc;
-            }
-            __syncthreads();
+        for (int e = 0; e < 4; ++e) dq[nt][e] = 0.f;
+    for (int br = 0; br < 3; ++br) {
+        int lo;
+        const int nk = branch_keys(br, lo);
+        const int nch = (nk + 31) / 32;
+        const float L0 = lse2s[br][gr], L1 = lse2s[br][gr + 8];
+        const float D0 = Ds[br][gr], D1 = Ds[br][gr + 8];
+        const float g0 = gs[br][gr], g1 = gs[br][gr + 8];
+        for (int ch = warp; ch < nch; ch += 4) {
+            const int k0 = ch * 32;
+            stage(br, lo, nk, k0);
+            float sf[4][4], dp[4][4];
+            warp_logits<DK>(qa, smem_u32(ks), sf);
+            warp_logits_sa<DV>(smem_u32(dos), smem_u32(vs), dp);
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const bool hi = e >= 2;
+                    const float Lr = hi ? L1 : L0;
+                    const bool ok = seen(br, lo, nk, k0 + nt * 8 + tg * 2 + (e & 1)) && Lr != -INFINITY;
+                    const float P = ok ? exp2f(sf[nt][e] * c - Lr) : 0.f;
+                    sf[nt][e] = P * ((hi ? g1 : g0) * dp[nt][e] - (hi ? D1 : D0));
+                }
+            warp_pv<DK>(sf, smem_u32(ks), dq);
+            __syncwarp();
         }
     }
-    if (hq < p.HG) {
+    __syncthreads();
+    // merge dq over the 4 warps, fixed order
+    float* qred = reinterpret_cast<float*>(bsm);               // [4][16][DK]
 #pragma unroll
-        for (int e = 0; e < DKT; ++e) p.dq[(rowbase + hq) * DK + cg * DKT + e] = dq[e];
+    for (int nt = 0; nt < DK / 8; ++nt) {
+        const int cc = nt * 8 + tg * 2;
+        *reinterpret_cast<float2*>(qred + (warp * 16 + gr) * DK + cc) = make_float2(dq[nt][0], dq[nt][1]);
+        *reinterpret_cast<float2*>(qred + (warp * 16 + gr + 8) * DK + cc) = make_float2(dq[nt][2], dq[nt][3]);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < p.HG * DK; e += 128) {
+        const int h = e / DK, cc = e % DK;
+        p.dq[(rowbase + h) * DK + cc] =
+            p.scale * (qred[h * DK + cc] + qred[(16 + h) * DK + cc] + qred[(32 + h) * DK + cc] + qred[(48 + h) * DK + cc]);
     }
 }
 

@@ -22,6 +22,7 @@
 #pragma once
 #include "nsa_dev.cuh"
 #include "k_topn.cuh"
+#include "k_mma.cuh"
 
 namespace nsa {
 
@@ -49,25 +50,6 @@ struct DecParams {
     int Cmax, NSPL, NU, NSmax;
 };
 
-// ------------------------------------------------------------ mma helpers
-__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
-}
-
 // Q of the group's 16 heads (rows >= HG zero) as A fragments for DK/16 k-steps
 template <int DK>
 __device__ __forceinline__ void load_q_frags(const DecParams& p, int s, int g, uint32_t (&qa)[DK / 16][4]) {
@@ -83,81 +65,6 @@ __device__ __forceinline__ void load_q_frags(const DecParams& p, int s, int g, u
         qa[kk][1] = ld(gr + 8, c);
         qa[kk][2] = ld(gr, c + 8);
         qa[kk][3] = ld(gr + 8, c + 8);
-    }
-}
-
-// copy `rows` rows of `width` bf16 (row stride src_stride elements) into
-// shared memory with a padded pitch: 16-byte cp.async chunks, all in flight
-// at once; rows >= nvalid are zero-filled.  Caller waits with cp_async_wait.
-__device__ __forceinline__ void warp_copy_rows(uint8_t* dst, int pitch, const __nv_bfloat16* src,
-                                               size_t src_stride, int rows, int nvalid, int width) {
-    const int lane = threadIdx.x & 31;
-    const int cpr = width / 8;   // 16-byte chunks per row
-    for (int e = lane; e < rows * cpr; e += 32) {
-        const int r = e / cpr, c = e % cpr;
-        const bool ok = r < nvalid;
-        const __nv_bfloat16* sp = ok ? src + (size_t)r * src_stride + c * 8 : src;
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst + r * pitch + c * 16)),
-                     "l"(sp), "r"(ok ? 16 : 0)
-                     : "memory");
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
-// S[16 heads x 32 keys] = Q K^T for the warp's 32 keys staged at `ks` (pitch
-// DK*2+16), logits scaled to log2 units; sfr[nt][0..3] in accumulator layout
-template <int DK>
-__device__ __forceinline__ void warp_logits(const uint32_t (&qa)[DK / 16][4], uint32_t ks, float (&sfr)[4][4]) {
-    const int lane = threadIdx.x & 31;
-    constexpr int pitch = DK * 2 + 16;
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sfr[nt][e] = 0.f;
-    // ldmatrix x4 (non-transposed): matrices (keys 8nt..+7, dims 16kk..+7),
-    // (same keys, dims +8), then the same for n-tile nt+1
-    const int mi = lane >> 3, rr = lane & 7;
-#pragma unroll
-    for (int kk = 0; kk < DK / 16; ++kk) {
-#pragma unroll
-        for (int nt = 0; nt < 4; nt += 2) {
-            const int key = (nt + (mi >> 1)) * 8 + rr;
-            const int dim = kk * 16 + (mi & 1) * 8;
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4(ks + key * pitch + dim * 2, b0, b1, b2, b3);
-            mma16816(sfr[nt], qa[kk], b0, b1);
-            mma16816(sfr[nt + 1], qa[kk], b2, b3);
-        }
-    }
-}
-
-// O[16 x DV] += P[16 x 32] V[32 x DV] for the warp's 32 keys staged at `vs`
-// (pitch DV*2+16); P given in accumulator layout (fp32), converted to bf16 A
-// fragments (two n-tiles of S form one k-step of P)
-template <int DV>
-__device__ __forceinline__ void warp_pv(const float (&pf)[4][4], uint32_t vs, float (&o)[DV / 8][4]) {
-    const int lane = threadIdx.x & 31;
-    constexpr int pitch = DV * 2 + 16;
-    const int mi = lane >> 3, rr = lane & 7;
-#pragma unroll
-    for (int kk = 0; kk < 2; ++kk) {
-        uint32_t a[4];
-        a[0] = pack_bf16x2(pf[2 * kk][0], pf[2 * kk][1]);
-        a[1] = pack_bf16x2(pf[2 * kk][2], pf[2 * kk][3]);
-        a[2] = pack_bf16x2(pf[2 * kk + 1][0], pf[2 * kk + 1][1]);
-        a[3] = pack_bf16x2(pf[2 * kk + 1][2], pf[2 * kk + 1][3]);
-#pragma unroll
-        for (int nt = 0; nt < DV / 8; nt += 2) {
-            // ldmatrix x4 .trans: matrices (keys 16kk..+7, ch 8nt..), (keys +8, ch 8nt..),
-            // (keys 16kk.., ch 8nt+8..), (keys +8, ch 8nt+8..)
-            const int key = kk * 16 + (mi & 1) * 8 + rr;
-            const int ch = nt * 8 + (mi >> 1) * 8;
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4_t(vs + key * pitch + ch * 2, b0, b1, b2, b3);
-            mma16816(o[nt], a, b0, b1);
-            mma16816(o[nt + 1], a, b2, b3);
-        }
     }
 }
 

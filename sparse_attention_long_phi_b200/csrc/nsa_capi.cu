@@ -525,11 +525,11 @@ nsa_status_t backward_impl(const Shape& s, const void* q, const void* k, const v
         cudaMemsetAsync(ws + L.off_dkc, 0, L.off_cnt - L.off_dkc, st) != cudaSuccess ||
         cudaMemsetAsync(ws + L.off_cnt, 0, L.off_off - L.off_cnt, st) != cudaSuccess)
         return NSA_ERR_CUDA;
-    // per-query statistics, d(gates), dq
+    // per-query statistics, d(gates), dq (tensor cores, 16 heads = M)
     {
-        const int smem = (16 * (DK + 1) + 16 * (DV + 1) + 64 * (DK + 1) + 64 * (DV + 1) + 16 * 64 + 16) * 4;
-        NSA_TRY(set_smem(bwd_query_kernel<DK, DV>, smem));
-        NSA_LAUNCH("bwd_query_kernel", st, bwd_query_kernel<DK, DV><<<dim3((unsigned)s.T, (unsigned)s.G, (unsigned)s.B), 256, smem, st>>>(p));
+        const int smem = bwd_query_mma_smem<DK, DV>();
+        NSA_TRY(set_smem(bwd_query_mma<DK, DV>, smem));
+        NSA_LAUNCH("bwd_query_mma", st, bwd_query_mma<DK, DV><<<dim3((unsigned)s.T, (unsigned)s.G, (unsigned)s.B), 128, smem, st>>>(p));
         NSA_TRY(last_launch());
     }
     // inverse index of the selection: block -> tokens

@@ -3,22 +3,31 @@
 // selected blocks and the window, not the whole cache).
 //
 // One query per sequence at t = L-1 over packed varlen caches.  The step is
-// HBM-bound; every cache row is read once, with 16-byte coalesced loads into
-// shared memory, and the 16 heads of a GQA group are the M = 16 side of
-// warp-level bf16 tensor-core products (mma.sync m16n8k16, fp32 accumulate):
-//   1. dec_cmp_partial  split-K over the compressed cache (128 keys per CTA,
-//                       32 per warp): logits, split max / sum, P.V~, and the
-//                       per-head selection-block sums of exp(logit - split max)
-//                       (mapped with the overlap weights), so the scores can be
+// HBM-bound: every cache row is read once.  The 16 heads of a GQA group are
+// the M = 16 side of warp-level bf16 tensor-core products (mma.sync
+// m16n8k16, fp32 accumulate).  The two streaming kernels are persistent (one
+// CTA of 8 warps per SM).  The chunks of 32 cache rows of all (seq, group)
+// pairs form one sequence that is cut into equal contiguous ranges, one per
+// CTA; a CTA walks its range one (seq, group) segment at a time, its warps
+// taking the segment's chunks round-robin.  Each warp pipelines K and V
+// separately (the next chunk's K is in flight while this chunk's softmax and
+// P.V run, its V while the next logits run) and keeps an online softmax; the
+// warps merge once per segment into one record, stored at slot
+// (CTA index + seq*G + group), which is unique because consecutive pairs
+// share at most one CTA.
+//   1. dec_cmp_stream   compressed cache: per segment (max, sum, unnormalised
+//                       O); per chunk the head max and the per-head selection-
+//                       block sums of exp(logit - chunk max), mapped with the
+//                       overlap weights, so the importance scores can be
 //                       normalised exactly once the row LSE is known.
-//   2. dec_cmp_combine  merge the splits -> o_cmp and the row LSE; group
-//                       importance scores = sum over heads and splits of the
-//                       block sums rescaled by exp(split max - LSE); top-n by
-//                       one warp -> sel_idx.
-//   3. dec_slcwin_partial  one CTA per 64-token unit of (selected blocks U
-//                       window blocks): logits once, partial softmax of the
-//                       selected and window branches over the unit.
-//   4. dec_final        merge units per branch; out = sum_c g_c o_c; lse.
+//   2. dec_cmp_combine  per (seq, group): LSE, o_cmp, group importance scores
+//                       (sum over heads and chunks of the block sums rescaled
+//                       by exp(chunk max - LSE)), top-n by one warp.
+//   3. dec_slcwin_stream  the sorted union of the selected blocks and the
+//                       window blocks (a fixed number of unit slots per pair,
+//                       the unused ones empty): logits once, online softmax of
+//                       the selected and the window branch.
+//   4. dec_final        merge the records per branch; out = sum_c g_c o_c; lse.
 #pragma once
 #include "nsa_dev.cuh"
 #include "k_topn.cuh"
@@ -26,15 +35,17 @@
 
 namespace nsa {
 
-constexpr int kDecCH = 128;     // compressed keys per split (4 warps x 32)
-constexpr int kDecUnit = 64;    // tokens per selected/window unit (2 warps x 32)
-constexpr int kDecNJB = 132;    // block-score slots per split (>= 128/SPB + 1)
-constexpr int kDecWJB = 34;     // block-score slots per warp of 32 keys (>= 32/SPB + 2)
-constexpr int kDecMaxSplits = 64;  // compressed-cache splits per sequence (Lmax <= 8192 * 16 + l)
+constexpr int kDecW = 8;             // warps per streaming CTA
+constexpr int kDecNBS = 33;          // block-sum slots per chunk (>= (31 + l/d - 1) / (l'/d) + 1)
+constexpr int kDecMaxSeqs = 2048;    // sequences per call (chunk prefix held in shared memory)
+constexpr int kDecMaxChunks = 256;   // compressed chunks per sequence (T <= 131072, d = 16)
+constexpr int kDecMaxUnits = 48;     // units in a (selected U window) list
+constexpr int kDecMaxGrid = 1024;    // CTAs of a streaming kernel
 
 struct DecParams {
     int S, H, G, HG, DK, DV;
     int l, d, lp, n, fi, fl, w;
+    int spb, cps, nbs;       // l'/d, l/d, block-sum slots used per chunk
     float scale_log2;
     const __nv_bfloat16 *q, *kcache, *vcache, *kccache, *vccache;
     const int64_t *kv_off, *cmp_off;
@@ -42,248 +53,433 @@ struct DecParams {
     float* out;
     int32_t* sel_idx;
     float* lse;
-    float* part1;    // [S][G][NSPL][16][2+DV]   split max (log2 units), sum, unnormalised O
-    float* bsc;      // [S][G][NSPL][16][kDecNJB] block sums of exp2(s - split max)
-    float* ocmp;     // [S][G][16][DV]
-    float* lsecmp;   // [S][G][16]               log2 units
-    float* part2;    // [S][G][NU][2][16][2+DV]
-    int Cmax, NSPL, NU, NSmax;
+    float* cmax;     // [S*G][NCH][16]            chunk max per head (log2 units)
+    float* bsum;     // [S*G][NCH][kDecNBS][16]   per-head block sums of exp2(s - chunk max)
+    float* part1;    // [grid1 + S*G][16][DV+4]   segment max, sum, -, -, unnormalised O
+    float* ocmp;     // [S*G][16][DV]             normalised compressed-branch output
+    float* lsecmp;   // [S*G][16]                 log2 units
+    float* part2;    // [grid3 + S*G][2][16][DV+4] per segment and branch (selected, window)
+    int* cpre;       // [S+1] compressed chunks (x G) before sequence s
+    int Lmax, Cmax, NCH, NUV, NSmax;
+    int grid1, grid3;
 };
+
+template <int DK, int DV>
+__host__ __device__ constexpr int dec_stage_bytes() {      // one warp: 32 K rows + 32 V rows
+    return 32 * ((DK * 2 + 16) + (DV * 2 + 16));
+}
+template <int DK, int DV>
+__host__ __device__ constexpr int dec_stream_smem() {      // staging (merge area aliased) + P tiles
+    return kDecW * dec_stage_bytes<DK, DV>() + kDecW * 16 * 33 * 4;
+}
 
 // Q of the group's 16 heads (rows >= HG zero) as A fragments for DK/16 k-steps
 template <int DK>
 __device__ __forceinline__ void load_q_frags(const DecParams& p, int s, int g, uint32_t (&qa)[DK / 16][4]) {
-    const int lane = threadIdx.x & 31, gr = lane >> 2, tg = lane & 3;
-    const __nv_bfloat16* q = p.q + ((size_t)s * p.H + (size_t)g * p.HG) * DK;
-#pragma unroll
-    for (int kk = 0; kk < DK / 16; ++kk) {
-        const int c = kk * 16 + tg * 2;
-        auto ld = [&](int row, int col) -> uint32_t {
-            return row < p.HG ? *reinterpret_cast<const uint32_t*>(q + (size_t)row * DK + col) : 0u;
-        };
-        qa[kk][0] = ld(gr, c);
-        qa[kk][1] = ld(gr + 8, c);
-        qa[kk][2] = ld(gr, c + 8);
-        qa[kk][3] = ld(gr + 8, c + 8);
+    load_a_frags<DK>(p.q + ((size_t)s * p.H + (size_t)g * p.HG) * DK, p.HG, qa);
+}
+
+// lengths of sequence s; false when it is empty or exceeds the sizes the
+// workspace was laid out for
+__device__ __forceinline__ bool dec_seq_ok(const DecParams& p, int s, int& L, int& C) {
+    L = (int)(p.kv_off[s + 1] - p.kv_off[s]);
+    C = (int)(p.cmp_off[s + 1] - p.cmp_off[s]);
+    return L > 0 && L <= p.Lmax && C <= p.Cmax;
+}
+
+// range of CTA b when N items are cut into `grid` contiguous ranges, and the
+// CTA whose range holds item x
+__device__ __forceinline__ long long dec_range_start(int b, long long N, int grid) {
+    return (long long)b * N / grid;
+}
+__device__ __forceinline__ int dec_cta_of(long long x, long long N, int grid) {
+    return (int)(((x + 1) * grid - 1) / N);
+}
+// record slots of items [X0, X1) (X1 > X0): CTAs with a non-empty range
+// among those holding them; returns the count, slots b + sg into out[]
+__device__ __forceinline__ int dec_record_ctas(long long X0, long long X1, long long N, int grid, int* out, int cap) {
+    const int bf = dec_cta_of(X0, N, grid), bl = dec_cta_of(X1 - 1, N, grid);
+    int cnt = 0;
+    for (int b = bf; b <= bl && cnt < cap; ++b)
+        if (dec_range_start(b + 1, N, grid) > dec_range_start(b, N, grid)) out[cnt++] = b;
+    return cnt;
+}
+
+// Merge the 8 warps' online-softmax states (rows gr, gr+8 per lane) into one
+// record [16][DV+4] = (max, sum, -, -, O relative to max).  `mrg` is a
+// [8][16][DV] fp32 scratch; wm/wl [8][16].  Ends with a barrier.
+template <int DV>
+__device__ __forceinline__ void dec_merge_record(float m0, float m1, float l0, float l1, const float (&o)[DV / 8][4],
+                                                 float* mrg, float (*wm)[16], float (*wl)[16], float* rec) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gr = lane >> 2, tg = lane & 3;
+    if (tg == 0) {
+        wm[warp][gr] = m0;
+        wm[warp][gr + 8] = m1;
+        wl[warp][gr] = l0;
+        wl[warp][gr + 8] = l1;
     }
+    __syncthreads();
+    {
+        float M0 = -INFINITY, M1 = -INFINITY;
+#pragma unroll
+        for (int w2 = 0; w2 < kDecW; ++w2) {
+            M0 = fmaxf(M0, wm[w2][gr]);
+            M1 = fmaxf(M1, wm[w2][gr + 8]);
+        }
+        const float f0 = m0 == -INFINITY ? 0.f : exp2f(m0 - M0);
+        const float f1 = m1 == -INFINITY ? 0.f : exp2f(m1 - M1);
+#pragma unroll
+        for (int nt = 0; nt < DV / 8; ++nt) {
+            const int cc = nt * 8 + tg * 2;
+            *reinterpret_cast<float2*>(mrg + (warp * 16 + gr) * DV + cc) = make_float2(o[nt][0] * f0, o[nt][1] * f0);
+            *reinterpret_cast<float2*>(mrg + (warp * 16 + gr + 8) * DV + cc) = make_float2(o[nt][2] * f1, o[nt][3] * f1);
+        }
+    }
+    __syncthreads();
+    constexpr int REC = DV + 4;
+    for (int e = threadIdx.x; e < 16 * (DV / 4); e += blockDim.x) {
+        const int h = e / (DV / 4), c4 = (e % (DV / 4)) * 4;
+        float4 a = *reinterpret_cast<const float4*>(mrg + h * DV + c4);
+#pragma unroll
+        for (int w2 = 1; w2 < kDecW; ++w2) {       // fixed order: deterministic
+            const float4 b = *reinterpret_cast<const float4*>(mrg + (w2 * 16 + h) * DV + c4);
+            a.x += b.x;
+            a.y += b.y;
+            a.z += b.z;
+            a.w += b.w;
+        }
+        *reinterpret_cast<float4*>(rec + h * REC + 4 + c4) = a;
+    }
+    if (threadIdx.x < 16) {
+        const int h = threadIdx.x;
+        float M = -INFINITY;
+        for (int w2 = 0; w2 < kDecW; ++w2) M = fmaxf(M, wm[w2][h]);
+        float Ls = 0.f;
+        for (int w2 = 0; w2 < kDecW; ++w2)
+            if (wm[w2][h] != -INFINITY) Ls += wl[w2][h] * exp2f(wm[w2][h] - M);
+        rec[h * REC] = M;
+        rec[h * REC + 1] = Ls;
+    }
+    __syncthreads();
 }
 
 // -------------------------------------------------------------- step 1
 template <int DK, int DV>
-__global__ void __launch_bounds__(128) dec_cmp_partial(const DecParams p) {
-    constexpr int KP = DK * 2 + 16, VP = DV * 2 + 16;
+__global__ void __launch_bounds__(256, 1) dec_cmp_stream(const DecParams p) {
+    constexpr int KP = DK * 2 + 16, STG = dec_stage_bytes<DK, DV>();
     extern __shared__ __align__(16) uint8_t dsm[];
-    __shared__ float redm[4][16], redl[4][16];
-    __shared__ float bsw[4][16][kDecWJB];
-    const int sp = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
+    float* mrg = reinterpret_cast<float*>(dsm);                                  // [8][16][DV] at merges
+    float(*pt)[16][33] = reinterpret_cast<float(*)[16][33]>(dsm + kDecW * STG);  // [8][16][33]
+    __shared__ float wm[kDecW][16], wl[kDecW][16];
+    __shared__ int pre[kDecMaxSeqs + 1];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gr = lane >> 2, tg = lane & 3;
-    const int64_t cbase = p.cmp_off[s];
-    const int C = (int)(p.cmp_off[s + 1] - cbase);
-    if (C > p.Cmax) {
-        if (threadIdx.x == 0 && sp == 0) atomicOr(&g_nsa_error, 4u);
-        return;
-    }
-    const int c0 = sp * kDecCH;
-    if (c0 >= C) return;
-    uint8_t* ks = dsm + warp * 32 * (KP + VP);
+    uint8_t* ks = dsm + warp * STG;
     uint8_t* vs = ks + 32 * KP;
-    const int k0 = c0 + warp * 32;                       // first key of this warp
-    const int nval = max(0, min(32, C - k0));
-    warp_copy_rows(ks, KP, p.kccache + ((cbase + k0) * p.G + g) * DK, (size_t)p.G * DK, 32, nval, DK);
-    warp_copy_rows(vs, VP, p.vccache + ((cbase + k0) * p.G + g) * DV, (size_t)p.G * DV, 32, nval, DV);
-    uint32_t qa[DK / 16][4];
-    load_q_frags<DK>(p, s, g, qa);
-    cp_async_wait();
-    __syncwarp();
-    float sf[4][4];
-    warp_logits<DK>(qa, smem_u32(ks), sf);
-    // scale, mask keys past the cache, warp max per head row (rows gr, gr+8)
-    float m0 = -INFINITY, m1 = -INFINITY;
+
+    // chunks (x G) before sequence s: exclusive prefix by warp 0
+    if (warp == 0) {
+        int run = 0;
+        for (int b0 = 0; b0 < p.S; b0 += 32) {
+            const int s = b0 + lane;
+            int cnt = 0;
+            if (s < p.S) {
+                int L, C;
+                if (dec_seq_ok(p, s, L, C)) cnt = p.G * ((C + 31) / 32);
+            }
+            int inc = cnt;
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int key = nt * 8 + tg * 2 + (e & 1);
-            float v = key < nval ? sf[nt][e] * p.scale_log2 : -INFINITY;
-            sf[nt][e] = v;
-            if (e < 2) m0 = fmaxf(m0, v);
-            else m1 = fmaxf(m1, v);
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += v;
+            }
+            if (s < p.S) pre[s] = run + inc - cnt;
+            run += __shfl_sync(0xffffffffu, inc, 31);
         }
-#pragma unroll
-    for (int o = 1; o <= 2; o <<= 1) {
-        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
-        m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
-    }
-    if (tg == 0) {
-        redm[warp][gr] = m0;
-        redm[warp][gr + 8] = m1;
+        if (lane == 0) pre[p.S] = run;
     }
     __syncthreads();
-    m0 = fmaxf(fmaxf(redm[0][gr], redm[1][gr]), fmaxf(redm[2][gr], redm[3][gr]));
-    m1 = fmaxf(fmaxf(redm[0][gr + 8], redm[1][gr + 8]), fmaxf(redm[2][gr + 8], redm[3][gr + 8]));
-    // P = exp2(s - split max); row sums; per-head block sums (overlap weights)
-    const int cps = p.l / p.d, spb = p.lp / p.d;
-    const int nj = kDecCH / spb + (cps + spb - 2) / spb + 1;   // blocks this split touches
-    for (int e = lane; e < 16 * kDecWJB; e += 32) bsw[warp][e / kDecWJB][e % kDecWJB] = 0.f;
-    const int wj0 = (warp * 32) / spb;                        // first block this warp touches
-    __syncwarp();
-    float l0 = 0.f, l1 = 0.f;
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float mm = e < 2 ? m0 : m1;
-            const float pv = sf[nt][e] == -INFINITY ? 0.f : exp2f(sf[nt][e] - mm);
-            sf[nt][e] = pv;
-            if (e < 2) l0 += pv;
-            else l1 += pv;
+    if (blockIdx.x == 0)
+        for (int s = threadIdx.x; s <= p.S; s += blockDim.x) p.cpre[s] = pre[s];
+    const long long N = pre[p.S];
+    const int b = blockIdx.x;
+    long long x = dec_range_start(b, N, gridDim.x);
+    const long long x1 = dec_range_start(b + 1, N, gridDim.x);
+    const float cl = p.scale_log2;
+    const bool fast = p.spb == 4 && p.cps == 2;
+    while (x < x1) {
+        // segment: consecutive chunks of one (seq, group)
+        int lo = 0, hi = p.S;                       // largest lo with pre[lo] <= x
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (pre[mid] <= x) lo = mid;
+            else hi = mid;
         }
+        const int s = lo;
+        const int64_t cbase = p.cmp_off[s];
+        const int C = (int)(p.cmp_off[s + 1] - cbase);
+        const int nch = (C + 31) / 32;
+        const int r = (int)(x - pre[s]);
+        const int g = r / nch, cfirst = r - g * nch;
+        const int n = (int)min((long long)(nch - cfirst), x1 - x);
+        const size_t sg = (size_t)s * p.G + g;
+        const size_t kst = (size_t)p.G * DK, vst = (size_t)p.G * DV;
+        const __nv_bfloat16* kb = p.kccache + ((size_t)cbase * p.G + g) * DK;
+        const __nv_bfloat16* vb = p.vccache + ((size_t)cbase * p.G + g) * DV;
+        auto issue_k = [&](int c) {
+            warp_issue_32rows<DK>(ks, kb + (size_t)c * 32 * kst, kst, C - c * 32);
+            cp_async_commit();
+        };
+        auto issue_v = [&](int c) {
+            warp_issue_32rows<DV>(vs, vb + (size_t)c * 32 * vst, vst, C - c * 32);
+            cp_async_commit();
+        };
+        uint32_t qa[DK / 16][4];
+        load_q_frags<DK>(p, s, g, qa);
+        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+        float o[DV / 8][4];
 #pragma unroll
-    for (int o = 1; o <= 2; o <<= 1) {
-        l0 += __shfl_xor_sync(0xffffffffu, l0, o);
-        l1 += __shfl_xor_sync(0xffffffffu, l1, o);
-    }
-    // block sums: lanes of a quad own disjoint keys of the same two heads;
-    // accumulate per key in a fixed order (deterministic)
-    for (int q = 0; q < 4; ++q) {
-        if (tg == q) {
+        for (int nt = 0; nt < DV / 8; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+        int i = warp;
+        if (i < n) {
+            issue_k(cfirst + i);
+            issue_v(cfirst + i);
+        }
+        for (; i < n; i += kDecW) {
+            const int c = cfirst + i;
+            const bool more = i + kDecW < n;
+            cp_async_wait_1();                      // K of chunk c
+            __syncwarp();
+            float sf[4][4];
+            warp_logits<DK>(qa, smem_u32(ks), sf);
+            __syncwarp();
+            if (more) issue_k(c + kDecW);
+            const int nval = min(32, C - c * 32);
+            float mc0 = -INFINITY, mc1 = -INFINITY;
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int kl = nt * 8 + tg * 2 + (e & 1);
-                    const int row = e < 2 ? gr : gr + 8;
-                    const int ig = warp * 32 + kl;            // key index within the split
-                    for (int u = 0; u < cps; ++u) {
-                        const int jl = (ig + u) / spb - wj0;
-                        bsw[warp][row][jl] += sf[nt][e];
+                    const int key = nt * 8 + tg * 2 + (e & 1);
+                    const float v = key < nval ? sf[nt][e] * cl : -INFINITY;
+                    sf[nt][e] = v;
+                    if (e < 2) mc0 = fmaxf(mc0, v);
+                    else mc1 = fmaxf(mc1, v);
+                }
+#pragma unroll
+            for (int q2 = 1; q2 <= 2; q2 <<= 1) {
+                mc0 = fmaxf(mc0, __shfl_xor_sync(0xffffffffu, mc0, q2));
+                mc1 = fmaxf(mc1, __shfl_xor_sync(0xffffffffu, mc1, q2));
+            }
+            // P relative to the chunk max (key 0 is valid, so the max is finite)
+            float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float pv = exp2f(sf[nt][e] - (e < 2 ? mc0 : mc1));
+                    sf[nt][e] = pv;
+                    if (e < 2) s0 += pv;
+                    else s1 += pv;
+                }
+#pragma unroll
+            for (int q2 = 1; q2 <= 2; q2 <<= 1) {
+                s0 += __shfl_xor_sync(0xffffffffu, s0, q2);
+                s1 += __shfl_xor_sync(0xffffffffu, s1, q2);
+            }
+            // per-head selection-block sums of this chunk: slot jl = block 32c/spb + jl
+            // takes chunk key i with weight |[i, i+cps) n [jl*spb, jl*spb+spb)|
+            const size_t cr = sg * p.NCH + c;
+            float* bdst = p.bsum + cr * kDecNBS * 16;
+            if (fast) {
+                // spb = 4, cps = 2: slot jl = 2 A_jl - P(4jl+3) + P(4jl-1), A = sum of the
+                // block's 4 keys; slot 8 = P(31).  Lane pair (tg 0,1) holds block 2nt,
+                // pair (2,3) block 2nt+1 of n-tile nt.
+#pragma unroll
+                for (int rh = 0; rh < 2; ++rh) {
+                    float prev3 = 0.f;
+#pragma unroll
+                    for (int nt = 0; nt < 4; ++nt) {
+                        const float x0 = sf[nt][2 * rh], x1v = sf[nt][2 * rh + 1];
+                        const float ps = x0 + x1v;
+                        const float A = ps + __shfl_xor_sync(0xffffffffu, ps, 1);
+                        const float last = __shfl_sync(0xffffffffu, x1v, lane | 1);
+                        const float l1q = __shfl_sync(0xffffffffu, x1v, (lane & ~3) | 1);
+                        const float l3q = __shfl_sync(0xffffffffu, x1v, (lane & ~3) | 3);
+                        const float prev = (tg >> 1) ? l1q : prev3;
+                        const float v = 2.f * A - last + prev;
+                        if ((tg & 1) == 0 && gr + 8 * rh < p.HG)
+                            bdst[(2 * nt + (tg >> 1)) * 16 + gr + 8 * rh] = v;
+                        prev3 = l3q;
+                    }
+                    if (tg == 0 && gr + 8 * rh < p.HG) bdst[8 * 16 + gr + 8 * rh] = prev3;
+                }
+            } else {
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) pt[warp][e < 2 ? gr : gr + 8][nt * 8 + tg * 2 + (e & 1)] = sf[nt][e];
+                __syncwarp();
+                if (lane < p.nbs) {
+                    const int jk0 = lane * p.spb;
+                    const int ilo = max(0, jk0 - p.cps + 1), ihi = min(32, jk0 + p.spb);
+                    for (int rr = 0; rr < p.HG; ++rr) {
+                        float a = 0.f;
+                        for (int k2 = ilo; k2 < ihi; ++k2)
+                            a += (float)(min(k2 + p.cps, jk0 + p.spb) - max(k2, jk0)) * pt[warp][rr][k2];
+                        bdst[lane * 16 + rr] = a;
                     }
                 }
-        }
-        __syncwarp();
-    }
-    if (tg == 0) {
-        redl[warp][gr] = l0;
-        redl[warp][gr + 8] = l1;
-    }
-    // P.V~ of this warp's keys
-    float o[DV / 8][4];
-#pragma unroll
-    for (int nt = 0; nt < DV / 8; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
-    warp_pv<DV>(sf, smem_u32(vs), o);
-    __syncthreads();
-    // sum the 4 warps' O in shared memory (reusing the staging area), fixed order
-    float* ored = reinterpret_cast<float*>(dsm);          // [4][16][DV]
-#pragma unroll
-    for (int nt = 0; nt < DV / 8; ++nt) {
-        const int ch = nt * 8 + tg * 2;
-        ored[(warp * 16 + gr) * DV + ch] = o[nt][0];
-        ored[(warp * 16 + gr) * DV + ch + 1] = o[nt][1];
-        ored[(warp * 16 + gr + 8) * DV + ch] = o[nt][2];
-        ored[(warp * 16 + gr + 8) * DV + ch + 1] = o[nt][3];
-    }
-    __syncthreads();
-    float* dst = p.part1 + (((size_t)s * p.G + g) * p.NSPL + sp) * 16 * (2 + DV);
-    for (int e = threadIdx.x; e < 16 * DV; e += 128) {
-        const int h = e / DV, c = e % DV;
-        dst[h * (2 + DV) + 2 + c] = ored[h * DV + c] + ored[(16 + h) * DV + c] + ored[(32 + h) * DV + c] +
-                                    ored[(48 + h) * DV + c];
-    }
-    if (threadIdx.x < 16) {
-        const int h = threadIdx.x;
-        dst[h * (2 + DV)] = fmaxf(fmaxf(redm[0][h], redm[1][h]), fmaxf(redm[2][h], redm[3][h]));
-        dst[h * (2 + DV) + 1] = redl[0][h] + redl[1][h] + redl[2][h] + redl[3][h];
-    }
-    float* bdst = p.bsc + (((size_t)s * p.G + g) * p.NSPL + sp) * 16 * kDecNJB;
-    for (int e = threadIdx.x; e < 16 * kDecNJB; e += 128) {
-        const int h = e / kDecNJB, j = e % kDecNJB;
-        float acc = 0.f;
-        if (j < nj) {
-#pragma unroll
-            for (int w2 = 0; w2 < 4; ++w2) {      // fixed order: deterministic
-                const int jl = j - (w2 * 32) / spb;
-                if (jl >= 0 && jl < kDecWJB) acc += bsw[w2][h][jl];
+                __syncwarp();
             }
+            if (tg == 0) {
+                p.cmax[cr * 16 + gr] = mc0;
+                p.cmax[cr * 16 + gr + 8] = mc1;
+            }
+            if (more) cp_async_wait_1();            // V of chunk c
+            else cp_async_wait();
+            __syncwarp();
+            // online softmax for O: rescale to the new running max
+            const float mn0 = fmaxf(m0, mc0), mn1 = fmaxf(m1, mc1);
+            const float a0 = exp2f(m0 - mn0), a1 = exp2f(m1 - mn1);
+            const float f0 = exp2f(mc0 - mn0), f1 = exp2f(mc1 - mn1);
+            m0 = mn0;
+            m1 = mn1;
+            l0 = l0 * a0 + s0 * f0;
+            l1 = l1 * a1 + s1 * f1;
+#pragma unroll
+            for (int nt = 0; nt < DV / 8; ++nt) {
+                o[nt][0] *= a0;
+                o[nt][1] *= a0;
+                o[nt][2] *= a1;
+                o[nt][3] *= a1;
+            }
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                sf[nt][0] *= f0;
+                sf[nt][1] *= f0;
+                sf[nt][2] *= f1;
+                sf[nt][3] *= f1;
+            }
+            warp_pv<DV>(sf, smem_u32(vs), o);
+            __syncwarp();
+            if (more) issue_v(c + kDecW);
         }
-        bdst[e] = acc;
+        // no copy is in flight: the staging area becomes the merge scratch
+        dec_merge_record<DV>(m0, m1, l0, l1, o, mrg, wm, wl, p.part1 + ((size_t)b + sg) * 16 * (DV + 4));
+        x += n;
     }
 }
 
 // -------------------------------------------------------------- step 2
 template <int DV>
 __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
-    extern __shared__ float pg[];                      // [NSmax]
+    constexpr int REC = DV + 4;
+    extern __shared__ float csm[];                     // ifac [256][16], fac [NCH][16], pg [NSmax]
     __shared__ float lse2[16];
-    __shared__ float fac[kDecMaxSplits][16];           // per split scale exp2(m_split - LSE)
+    __shared__ int recb[kDecMaxChunks];
+    __shared__ int nrec;
     const int g = blockIdx.x, s = blockIdx.y;
-    const int64_t cbase = p.cmp_off[s];
-    const int C = (int)(p.cmp_off[s + 1] - cbase);
-    const int L = (int)(p.kv_off[s + 1] - p.kv_off[s]);
+    int L, C;
+    if (!dec_seq_ok(p, s, L, C)) {
+        if (threadIdx.x == 0 && g == 0 && L > 0) atomicOr(&g_nsa_error, 4u);
+        return;
+    }
     const int t = L - 1;
-    if (C > p.Cmax || L <= 0) return;
-    const int nspl = (C + kDecCH - 1) / kDecCH;
-    const float* part = p.part1 + (((size_t)s * p.G + g) * p.NSPL) * 16 * (2 + DV);
+    const int nch = (C + 31) / 32;
+    const size_t sg = (size_t)s * p.G + g;
+    if (threadIdx.x == 0) {
+        int cnt = 0;
+        if (nch > 0) {
+            const long long X0 = (long long)p.cpre[s] + (long long)g * nch;
+            cnt = dec_record_ctas(X0, X0 + nch, p.cpre[p.S], p.grid1, recb, kDecMaxChunks);
+        }
+        nrec = cnt;
+    }
+    __syncthreads();
+    const int nr = nrec;
+    float* ifac = csm;
+    float* fac = csm + kDecMaxChunks * 16;
+    float* pg = fac + p.NCH * 16;
     if (threadIdx.x < 16) {
         const int h = threadIdx.x;
         float M = -INFINITY;
-        for (int i = 0; i < nspl; ++i) M = fmaxf(M, part[((size_t)i * 16 + h) * (2 + DV)]);
+        for (int i = 0; i < nr; ++i) M = fmaxf(M, p.part1[((size_t)(recb[i] + sg) * 16 + h) * REC]);
         float Ls = 0.f;
-        for (int i = 0; i < nspl; ++i) {
-            const float* pr = part + ((size_t)i * 16 + h) * (2 + DV);
-            if (pr[0] != -INFINITY) Ls += pr[1] * exp2f(pr[0] - M);
+        for (int i = 0; i < nr; ++i) {
+            const float* r = p.part1 + ((size_t)(recb[i] + sg) * 16 + h) * REC;
+            if (r[0] != -INFINITY) Ls += r[1] * exp2f(r[0] - M);
         }
         const float l2 = Ls > 0.f ? M + log2f(Ls) : -INFINITY;
         lse2[h] = l2;
-        p.lsecmp[((size_t)s * p.G + g) * 16 + h] = l2;
+        p.lsecmp[sg * 16 + h] = l2;
+        for (int i = 0; i < nr; ++i) {
+            const float m = p.part1[((size_t)(recb[i] + sg) * 16 + h) * REC];
+            ifac[i * 16 + h] = (m != -INFINITY && l2 != -INFINITY) ? exp2f(m - l2) : 0.f;
+        }
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < nspl * 16; e += blockDim.x) {
-        const int i = e / 16, h = e % 16;
-        const float m = part[((size_t)i * 16 + h) * (2 + DV)];
-        fac[i][h] = (h < p.HG && m != -INFINITY && lse2[h] != -INFINITY) ? exp2f(m - lse2[h]) : 0.f;
+    // o_cmp = sum over records of O exp2(m - LSE)
+    for (int e = threadIdx.x; e < 16 * (DV / 4); e += blockDim.x) {
+        const int h = e / (DV / 4), c4 = (e % (DV / 4)) * 4;
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i = 0; i < nr; ++i) {
+            const float4 v = *reinterpret_cast<const float4*>(p.part1 + ((size_t)(recb[i] + sg) * 16 + h) * REC + 4 + c4);
+            const float f = ifac[i * 16 + h];
+            a.x += v.x * f;
+            a.y += v.y * f;
+            a.z += v.z * f;
+            a.w += v.w * f;
+        }
+        *reinterpret_cast<float4*>(p.ocmp + (sg * 16 + h) * DV + c4) = a;
+    }
+    // per chunk and head: exp2(chunk max - LSE); heads past HG do not score
+    const float* cm = p.cmax + sg * p.NCH * 16;
+    for (int e = threadIdx.x; e < nch * 16; e += blockDim.x) {
+        const int h = e & 15;
+        fac[e] = (h < p.HG && lse2[h] != -INFINITY) ? exp2f(cm[e] - lse2[h]) : 0.f;
     }
     __syncthreads();
-    // o_cmp = sum_i O_i * exp2(m_i - LSE)
-    for (int e = threadIdx.x; e < 16 * DV; e += blockDim.x) {
-        const int h = e / DV, c = e % DV;
-        float acc = 0.f;
-        for (int i = 0; i < nspl; ++i) acc += part[((size_t)i * 16 + h) * (2 + DV) + 2 + c] * fac[i][h];
-        p.ocmp[(((size_t)s * p.G + g) * 16 + h) * DV + c] = acc;
-    }
-    // group scores: block j lies in split j / (128/spb) and, through the
-    // overlap of its last compressed block, in the split before it
-    const int spb = p.lp / p.d;
-    const int per = kDecCH / spb;
-    const int NSs = (L + p.lp - 1) / p.lp;
-    const float* bs = p.bsc + (((size_t)s * p.G + g) * p.NSPL) * 16 * kDecNJB;
+    // group score of selection block j: the chunks holding keys j*spb-cps+1 .. j*spb+spb-1
+    const int NSs = t / p.lp + 1;
+    const int bpc = 32 / p.spb;                        // blocks starting in one chunk
+    const float* bs = p.bsum + sg * p.NCH * kDecNBS * 16;
     for (int j = threadIdx.x; j < NSs; j += blockDim.x) {
         float acc = 0.f;
-        for (int i = max(0, j / per - 1); i <= min(nspl - 1, j / per); ++i) {
-            const int jl = j - i * per;
-            if (jl < 0 || jl >= kDecNJB) continue;
-            for (int h = 0; h < p.HG; ++h) acc += bs[((size_t)i * 16 + h) * kDecNJB + jl] * fac[i][h];
+        const int ilo = max(0, j * p.spb - p.cps + 1), ihi = min(C - 1, j * p.spb + p.spb - 1);
+        for (int cc = ilo >> 5; ilo <= ihi && cc <= (ihi >> 5); ++cc) {
+            const int jl = j - cc * bpc;
+            if (jl < 0 || jl >= p.nbs) continue;
+            const float* bp = bs + ((size_t)cc * kDecNBS + jl) * 16;
+            for (int h = 0; h < p.HG; ++h) acc += bp[h] * fac[cc * 16 + h];
         }
         pg[j] = acc;
     }
     __syncthreads();
-    if (threadIdx.x < 32)
-        topn_row_warp(pg, t, p.n, p.lp, p.fi, p.fl, p.sel_idx + ((size_t)s * p.G + g) * p.n, threadIdx.x);
+    if (threadIdx.x < 32) topn_row_warp(pg, t, p.n, p.lp, p.fi, p.fl, p.sel_idx + sg * p.n, threadIdx.x);
 }
 
-// sorted union of the selected blocks and the blocks overlapping the window
-__device__ __forceinline__ int dec_units(const DecParams& p, const int32_t* sel, int L, int* list) {
+// sorted union of the selected blocks (sel: n entries, -1 padded, ascending)
+// and the blocks overlapping the window; flag[i] = 1 when list[i] is selected
+__device__ __forceinline__ int dec_units(const DecParams& p, const int32_t* sel, int L, int* list, int* flag) {
     const int wlo = max(0, L - p.w) / p.lp, whi = (L - 1) / p.lp;
     int i = 0, j = wlo, cnt = 0, last = -1;
-    while (true) {
+    while (cnt < kDecMaxUnits) {
         const int a = (i < p.n && sel[i] >= 0) ? sel[i] : 0x7fffffff;
         const int b = j <= whi ? j : 0x7fffffff;
         const int m = min(a, b);
         if (m == 0x7fffffff) break;
+        const bool from_sel = m == a;
         if (m == a) ++i;
         if (m == b) ++j;
-        if (m != last) list[cnt++] = m;
+        if (m != last) {
+            list[cnt] = m;
+            flag[cnt] = from_sel ? 1 : 0;
+            ++cnt;
+        } else if (from_sel) {
+            flag[cnt - 1] = 1;
+        }
         last = m;
     }
     return cnt;
@@ -291,180 +487,222 @@ __device__ __forceinline__ int dec_units(const DecParams& p, const int32_t* sel,
 
 // -------------------------------------------------------------- step 3
 template <int DK, int DV>
-__global__ void __launch_bounds__(64) dec_slcwin_partial(const DecParams p) {
-    constexpr int KP = DK * 2 + 16, VP = DV * 2 + 16;
+__global__ void __launch_bounds__(256, 1) dec_slcwin_stream(const DecParams p) {
+    constexpr int KP = DK * 2 + 16, STG = dec_stage_bytes<DK, DV>();
     extern __shared__ __align__(16) uint8_t dsm[];
-    __shared__ float red[2][2][2][16];     // [branch][max|sum][warp][head]
-    __shared__ int list[48];
-    __shared__ int nlist;
-    const int ui = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gr = lane >> 2, tg = lane & 3;
-    const int64_t kb = p.kv_off[s];
-    const int L = (int)(p.kv_off[s + 1] - kb);
-    if (L <= 0) return;
-    const int32_t* sel = p.sel_idx + ((size_t)s * p.G + g) * p.n;
-    if (threadIdx.x == 0) nlist = dec_units(p, sel, L, list);
-    __syncthreads();
-    if (ui >= nlist) return;
-    const int blk = list[ui];
-    bool in_sel = false;
-    for (int a = 0; a < p.n; ++a) in_sel |= (sel[a] == blk);
-    uint8_t* ks = dsm + warp * 32 * (KP + VP);
+    float* mrg = reinterpret_cast<float*>(dsm);
+    uint8_t* qs = dsm + kDecW * STG;                      // [16][DK] Q tile, pitch DK*2+16
+    static_assert(16 * (DK * 2 + 16) <= kDecW * 16 * 33 * 4, "Q tile");
+    __shared__ float wm[kDecW][16], wl[kDecW][16];
+    __shared__ int ulist[kDecMaxUnits], uflag[kDecMaxUnits];
+    __shared__ int selbuf[32];
+    __shared__ int nunits;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tg = lane & 3;
+    uint8_t* ks = dsm + warp * STG;
     uint8_t* vs = ks + 32 * KP;
-    const int u0 = blk * p.lp + warp * 32;                    // first token of this warp
-    const int nval = max(0, min(32, L - u0));
-    warp_copy_rows(ks, KP, p.kcache + ((kb + u0) * p.G + g) * DK, (size_t)p.G * DK, 32, nval, DK);
-    warp_copy_rows(vs, VP, p.vcache + ((kb + u0) * p.G + g) * DV, (size_t)p.G * DV, 32, nval, DV);
-    uint32_t qa[DK / 16][4];
-    load_q_frags<DK>(p, s, g, qa);
-    cp_async_wait();
-    __syncwarp();
-    float sf[4][4];
-    warp_logits<DK>(qa, smem_u32(ks), sf);
-    float mx[2][2];
-#pragma unroll
-    for (int br = 0; br < 2; ++br) mx[br][0] = mx[br][1] = -INFINITY;
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int u = u0 + nt * 8 + tg * 2 + (e & 1);
-            const float v = u < L ? sf[nt][e] * p.scale_log2 : -INFINITY;
-            sf[nt][e] = v;
-            if (in_sel) mx[0][e >> 1] = fmaxf(mx[0][e >> 1], v);
-            if (u >= L - p.w) mx[1][e >> 1] = fmaxf(mx[1][e >> 1], v);
+    const long long U = (long long)p.S * p.G * p.NUV;     // unit slots, NUV per (seq, group)
+    const int b = blockIdx.x;
+    long long x = dec_range_start(b, U, gridDim.x);
+    const long long x1 = dec_range_start(b + 1, U, gridDim.x);
+    const float cl = p.scale_log2;
+    while (x < x1) {
+        const size_t sg = (size_t)(x / p.NUV);
+        const int ua = (int)(x % p.NUV);
+        const int nslot = (int)min((long long)(p.NUV - ua), x1 - x);
+        const int s = (int)(sg / p.G), g = (int)(sg % p.G);
+        int L, C;
+        const bool ok = dec_seq_ok(p, s, L, C);
+        if (warp == 0) {                                  // unit list of (s, g)
+            if (ok && lane < p.n) selbuf[lane] = p.sel_idx[sg * p.n + lane];
+            __syncwarp();
+            if (lane == 0) nunits = ok ? dec_units(p, selbuf, L, ulist, uflag) : 0;
         }
-#pragma unroll
-    for (int br = 0; br < 2; ++br)
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf)
-#pragma unroll
-            for (int o = 1; o <= 2; o <<= 1) mx[br][hf] = fmaxf(mx[br][hf], __shfl_xor_sync(0xffffffffu, mx[br][hf], o));
-    if (tg == 0) {
+        // Q of the group as a [16][DK] tile (rows >= HG zero), read with ldmatrix
+        for (int e = threadIdx.x; e < 16 * (DK / 8); e += blockDim.x) {
+            const int h = e / (DK / 8), c8 = e % (DK / 8);
+            int4 v = make_int4(0, 0, 0, 0);
+            if (h < p.HG) v = *reinterpret_cast<const int4*>(p.q + ((size_t)s * p.H + (size_t)g * p.HG + h) * DK + c8 * 8);
+            *reinterpret_cast<int4*>(qs + h * KP + c8 * 16) = v;
+        }
+        __syncthreads();
+        const int n = 2 * max(0, min(ua + nslot, nunits) - ua);   // chunks of 32 tokens
+        const int64_t kvb = ok ? p.kv_off[s] : 0;
+        const size_t kst = (size_t)p.G * DK, vst = (size_t)p.G * DV;
+        auto tok0 = [&](int i) { return ulist[ua + (i >> 1)] * p.lp + (i & 1) * 32; };
+        // rows past the cache are not read; the source stays inside the sequence
+        auto issue_k = [&](int i) {
+            const int u0 = tok0(i), nv = min(32, L - u0);
+            warp_issue_32rows<DK>(ks, p.kcache + ((size_t)(kvb + (nv > 0 ? u0 : 0)) * p.G + g) * DK, kst, nv);
+            cp_async_commit();
+        };
+        auto issue_v = [&](int i) {
+            const int u0 = tok0(i), nv = min(32, L - u0);
+            warp_issue_32rows<DV>(vs, p.vcache + ((size_t)(kvb + (nv > 0 ? u0 : 0)) * p.G + g) * DV, vst, nv);
+            cp_async_commit();
+        };
+        float m[2][2], l[2][2];
+        float o[2][DV / 8][4];
 #pragma unroll
         for (int br = 0; br < 2; ++br) {
-            red[br][0][warp][gr] = mx[br][0];
-            red[br][0][warp][gr + 8] = mx[br][1];
+            m[br][0] = m[br][1] = -INFINITY;
+            l[br][0] = l[br][1] = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < DV / 8; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) o[br][nt][e] = 0.f;
         }
-    }
-    __syncthreads();
+        const int wlo = L - p.w;
+        int i = warp;
+        if (i < n) {
+            issue_k(i);
+            issue_v(i);
+        }
+        for (; i < n; i += kDecW) {
+            const bool more = i + kDecW < n;
+            const int u0 = tok0(i);
+            const bool insel = uflag[ua + (i >> 1)] != 0;
+            const int nval = min(32, L - u0);
+            // warp-uniform: does the chunk hold keys of each branch?
+            const bool has_sel = insel && nval > 0;
+            const bool has_win = nval > 0 && u0 + nval - 1 >= wlo;
+            cp_async_wait_1();                          // K of chunk i
+            __syncwarp();
+            float sf[4][4];
+            if (has_sel || has_win) warp_logits_sa<DK>(smem_u32(qs), smem_u32(ks), sf);
+            __syncwarp();
+            if (more) issue_k(i + kDecW);
+            if (more) cp_async_wait_1();                // V of chunk i
+            else cp_async_wait();
+            __syncwarp();
 #pragma unroll
-    for (int br = 0; br < 2; ++br) {
-        mx[br][0] = fmaxf(red[br][0][0][gr], red[br][0][1][gr]);
-        mx[br][1] = fmaxf(red[br][0][0][gr + 8], red[br][0][1][gr + 8]);
-    }
-    float ls[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-    float o[2][DV / 8][4];
+            for (int br = 0; br < 2; ++br) {
+                if (br == 0 ? !has_sel : !has_win) continue;
+                float pf4[4][4];
+                float mc0 = -INFINITY, mc1 = -INFINITY;
 #pragma unroll
-    for (int br = 0; br < 2; ++br) {
-        float pf[4][4];
+                for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
+                    for (int e = 0; e < 4; ++e) {
+                        const int key = nt * 8 + tg * 2 + (e & 1);
+                        const bool okk = key < nval && (br == 0 || u0 + key >= wlo);
+                        const float v = okk ? sf[nt][e] * cl : -INFINITY;
+                        pf4[nt][e] = v;
+                        if (e < 2) mc0 = fmaxf(mc0, v);
+                        else mc1 = fmaxf(mc1, v);
+                    }
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int u = u0 + nt * 8 + tg * 2 + (e & 1);
-                const bool f = br == 0 ? (in_sel && u < L) : (u < L && u >= L - p.w);
-                const float m = mx[br][e >> 1];
-                const float pv = (f && m != -INFINITY) ? exp2f(sf[nt][e] - m) : 0.f;
-                pf[nt][e] = pv;
-                ls[br][e >> 1] += pv;
+                for (int q2 = 1; q2 <= 2; q2 <<= 1) {
+                    mc0 = fmaxf(mc0, __shfl_xor_sync(0xffffffffu, mc0, q2));
+                    mc1 = fmaxf(mc1, __shfl_xor_sync(0xffffffffu, mc1, q2));
+                }
+                const float mn0 = fmaxf(m[br][0], mc0), mn1 = fmaxf(m[br][1], mc1);
+                float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float v = pf4[nt][e];
+                        const float pv = v == -INFINITY ? 0.f : exp2f(v - (e < 2 ? mn0 : mn1));
+                        pf4[nt][e] = pv;
+                        if (e < 2) s0 += pv;
+                        else s1 += pv;
+                    }
+#pragma unroll
+                for (int q2 = 1; q2 <= 2; q2 <<= 1) {
+                    s0 += __shfl_xor_sync(0xffffffffu, s0, q2);
+                    s1 += __shfl_xor_sync(0xffffffffu, s1, q2);
+                }
+                const float a0 = mn0 == -INFINITY ? 1.f : exp2f(m[br][0] - mn0);
+                const float a1 = mn1 == -INFINITY ? 1.f : exp2f(m[br][1] - mn1);
+                m[br][0] = mn0;
+                m[br][1] = mn1;
+                l[br][0] = l[br][0] * a0 + s0;
+                l[br][1] = l[br][1] * a1 + s1;
+#pragma unroll
+                for (int nt = 0; nt < DV / 8; ++nt) {
+                    o[br][nt][0] *= a0;
+                    o[br][nt][1] *= a0;
+                    o[br][nt][2] *= a1;
+                    o[br][nt][3] *= a1;
+                }
+                warp_pv<DV>(pf4, smem_u32(vs), o[br]);
             }
-#pragma unroll
-        for (int nt = 0; nt < DV / 8; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) o[br][nt][e] = 0.f;
-        warp_pv<DV>(pf, smem_u32(vs), o[br]);
-    }
-#pragma unroll
-    for (int br = 0; br < 2; ++br)
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf)
-#pragma unroll
-            for (int q2 = 1; q2 <= 2; q2 <<= 1) ls[br][hf] += __shfl_xor_sync(0xffffffffu, ls[br][hf], q2);
-    if (tg == 0) {
-#pragma unroll
-        for (int br = 0; br < 2; ++br) {
-            red[br][1][warp][gr] = ls[br][0];
-            red[br][1][warp][gr + 8] = ls[br][1];
+            __syncwarp();
+            if (more) issue_v(i + kDecW);
         }
-    }
-    __syncthreads();
-    float* ored = reinterpret_cast<float*>(dsm);            // [2 br][2 warps][16][DV]
-#pragma unroll
-    for (int br = 0; br < 2; ++br)
-#pragma unroll
-        for (int nt = 0; nt < DV / 8; ++nt) {
-            const int ch = nt * 8 + tg * 2;
-            float* base = ored + ((br * 2 + warp) * 16) * DV;
-            base[gr * DV + ch] = o[br][nt][0];
-            base[gr * DV + ch + 1] = o[br][nt][1];
-            base[(gr + 8) * DV + ch] = o[br][nt][2];
-            base[(gr + 8) * DV + ch + 1] = o[br][nt][3];
-        }
-    __syncthreads();
-#pragma unroll
-    for (int br = 0; br < 2; ++br) {
-        float* dst = p.part2 + (((((size_t)s * p.G + g) * p.NU + ui) * 2 + br) * 16) * (2 + DV);
-        for (int e = threadIdx.x; e < 16 * DV; e += 64) {
-            const int h = e / DV, c = e % DV;
-            dst[h * (2 + DV) + 2 + c] = ored[((br * 2 + 0) * 16 + h) * DV + c] + ored[((br * 2 + 1) * 16 + h) * DV + c];
-        }
-        if (threadIdx.x < 16) {
-            const int h = threadIdx.x;
-            dst[h * (2 + DV)] = fmaxf(red[br][0][0][h], red[br][0][1][h]);
-            dst[h * (2 + DV) + 1] = red[br][1][0][h] + red[br][1][1][h];
-        }
+        float* rec = p.part2 + ((size_t)b + sg) * 2 * 16 * (DV + 4);
+        dec_merge_record<DV>(m[0][0], m[0][1], l[0][0], l[0][1], o[0], mrg, wm, wl, rec);
+        dec_merge_record<DV>(m[1][0], m[1][1], l[1][0], l[1][1], o[1], mrg, wm, wl, rec + 16 * (DV + 4));
+        x += nslot;
     }
 }
 
 // -------------------------------------------------------------- step 4
 template <int DV>
 __global__ void __launch_bounds__(256) dec_final(const DecParams p) {
-    __shared__ int list[48];
-    __shared__ int nlist;
-    __shared__ float fac[2][48][16];
-    __shared__ float Lb[2][16];
+    constexpr int REC = DV + 4;
+    __shared__ float fac[2][kDecMaxUnits][16];
+    __shared__ int recb[kDecMaxUnits];
+    __shared__ int nrec;
     const int g = blockIdx.x, s = blockIdx.y;
-    const int L = (int)(p.kv_off[s + 1] - p.kv_off[s]);
-    if (L <= 0) return;
-    const int32_t* sel = p.sel_idx + ((size_t)s * p.G + g) * p.n;
-    if (threadIdx.x == 0) nlist = dec_units(p, sel, L, list);
+    int L, C;
+    if (!dec_seq_ok(p, s, L, C)) return;
+    const size_t sg = (size_t)s * p.G + g;
+    if (threadIdx.x == 0) {
+        const long long X0 = (long long)sg * p.NUV;
+        nrec = dec_record_ctas(X0, X0 + p.NUV, (long long)p.S * p.G * p.NUV, p.grid3, recb, kDecMaxUnits);
+    }
     __syncthreads();
-    const float* part = p.part2 + ((((size_t)s * p.G + g) * p.NU) * 2) * 16 * (2 + DV);
+    const int nr = nrec;
+    auto recp = [&](int i, int br) { return p.part2 + (((size_t)recb[i] + sg) * 2 + br) * 16 * REC; };
     if (threadIdx.x < 32) {
         const int br = threadIdx.x / 16, h = threadIdx.x % 16;
         float M = -INFINITY;
-        for (int u = 0; u < nlist; ++u) M = fmaxf(M, part[(((size_t)u * 2 + br) * 16 + h) * (2 + DV)]);
+        for (int i = 0; i < nr; ++i) M = fmaxf(M, recp(i, br)[h * REC]);
         float Ls = 0.f;
-        for (int u = 0; u < nlist; ++u) {
-            const float* pr = part + (((size_t)u * 2 + br) * 16 + h) * (2 + DV);
-            const float f = pr[0] != -INFINITY ? exp2f(pr[0] - M) : 0.f;
-            fac[br][u][h] = f;
-            Ls += pr[1] * f;
+        for (int i = 0; i < nr; ++i) {
+            const float* r = recp(i, br) + h * REC;
+            const float f = r[0] != -INFINITY ? exp2f(r[0] - M) : 0.f;
+            fac[br][i][h] = f;
+            Ls += r[1] * f;
         }
-        Lb[br][h] = Ls;
+        const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+        for (int i = 0; i < nr; ++i) fac[br][i][h] *= inv;
         if (h < p.HG && p.lse) {
             const size_t row = (size_t)s * p.H + g * p.HG + h;
             p.lse[row * 3 + 1 + br] = Ls > 0.f ? (M + log2f(Ls)) * kLn2 : -INFINITY;
             if (br == 0) {
-                const float lc = p.lsecmp[((size_t)s * p.G + g) * 16 + h];
+                const float lc = p.lsecmp[sg * 16 + h];
                 p.lse[row * 3] = lc == -INFINITY ? -INFINITY : lc * kLn2;
             }
         }
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < p.HG * DV; e += blockDim.x) {
-        const int h = e / DV, c = e % DV;
-        float ob[2];
+    for (int e = threadIdx.x; e < p.HG * (DV / 4); e += blockDim.x) {
+        const int h = e / (DV / 4), c4 = (e % (DV / 4)) * 4;
+        float4 ob[2];
 #pragma unroll
         for (int br = 0; br < 2; ++br) {
-            float acc = 0.f;
-            for (int u = 0; u < nlist; ++u) acc += part[(((size_t)u * 2 + br) * 16 + h) * (2 + DV) + 2 + c] * fac[br][u][h];
-            ob[br] = Lb[br][h] > 0.f ? acc / Lb[br][h] : 0.f;
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int i = 0; i < nr; ++i) {
+                const float4 v = *reinterpret_cast<const float4*>(recp(i, br) + h * REC + 4 + c4);
+                const float f = fac[br][i][h];
+                a.x += v.x * f;
+                a.y += v.y * f;
+                a.z += v.z * f;
+                a.w += v.w * f;
+            }
+            ob[br] = a;
         }
         const size_t row = (size_t)s * p.H + g * p.HG + h;
-        const float oc = p.ocmp[(((size_t)s * p.G + g) * 16 + h) * DV + c];   // normalised
-        p.out[row * DV + c] = p.gates[row * 3] * oc + p.gates[row * 3 + 1] * ob[0] + p.gates[row * 3 + 2] * ob[1];
+        const float4 oc = *reinterpret_cast<const float4*>(p.ocmp + (sg * 16 + h) * DV + c4);
+        const float g0 = p.gates[row * 3], g1 = p.gates[row * 3 + 1], g2 = p.gates[row * 3 + 2];
+        float4 r;
+        r.x = g0 * oc.x + g1 * ob[0].x + g2 * ob[1].x;
+        r.y = g0 * oc.y + g1 * ob[0].y + g2 * ob[1].y;
+        r.z = g0 * oc.z + g1 * ob[0].z + g2 * ob[1].z;
+        r.w = g0 * oc.w + g1 * ob[0].w + g2 * ob[1].w;
+        *reinterpret_cast<float4*>(p.out + row * DV + c4) = r;
     }
 }
 
@@ -472,15 +710,18 @@ __global__ void __launch_bounds__(256) dec_final(const DecParams p) {
 inline size_t decode_ws_bytes(int64_t S, int64_t Lmax, int64_t G, int64_t l, int64_t d, int64_t lp,
                               int64_t w, int64_t n, int64_t DV) {
     const int64_t Cmax = Lmax >= l ? (Lmax - l) / d + 1 : 1;
-    const int64_t NSPL = (Cmax + kDecCH - 1) / kDecCH;
-    const int64_t NU = n + (w + lp - 1) / lp + 1;
+    const int64_t NCH = (Cmax + 31) / 32;
+    const int64_t NUV = n + (w + lp - 1) / lp + 1;
     auto a = [](size_t x) { return (x + 255) & ~size_t(255); };
     size_t o = 0;
-    o += a((size_t)S * G * NSPL * 16 * (2 + DV) * 4);
-    o += a((size_t)S * G * NSPL * 16 * kDecNJB * 4);
+    o += a((size_t)S * G * NCH * 16 * 4);
+    o += a((size_t)S * G * NCH * kDecNBS * 16 * 4);
+    o += a((size_t)(kDecMaxGrid + S * G) * 16 * (DV + 4) * 4);
     o += a((size_t)S * G * 16 * DV * 4);
     o += a((size_t)S * G * 16 * 4);
-    o += a((size_t)S * G * NU * 2 * 16 * (2 + DV) * 4);
+    o += a((size_t)(kDecMaxGrid + S * G) * 2 * 16 * (DV + 4) * 4);
+    o += a((size_t)(S + 1) * 4);
+    (void)NUV;
     return o;
 }
 

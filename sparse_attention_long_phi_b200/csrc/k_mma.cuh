@@ -30,9 +30,10 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
 
 // copy `rows` rows of `width` bf16 (row stride src_stride elements) into
 // shared memory with a padded pitch: 16-byte cp.async chunks, all in flight
-// at once; rows >= nvalid are zero-filled.  Caller waits with cp_async_wait.
-__device__ __forceinline__ void warp_copy_rows(uint8_t* dst, int pitch, const __nv_bfloat16* src,
-                                               size_t src_stride, int rows, int nvalid, int width) {
+// at once; rows >= nvalid are zero-filled.  No commit: the caller groups the
+// copies with cp_async_commit and waits with cp_async_wait / cp_async_wait_1.
+__device__ __forceinline__ void warp_issue_rows(uint8_t* dst, int pitch, const __nv_bfloat16* src,
+                                                size_t src_stride, int rows, int nvalid, int width) {
     const int lane = threadIdx.x & 31;
     const int cpr = width / 8;   // 16-byte chunks per row
     for (int e = lane; e < rows * cpr; e += 32) {
@@ -43,9 +44,43 @@ __device__ __forceinline__ void warp_copy_rows(uint8_t* dst, int pitch, const __
                      "l"(sp), "r"(ok ? 16 : 0)
                      : "memory");
     }
-    asm volatile("cp.async.commit_group;" ::: "memory");
 }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+// all but the most recent group complete
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// 32 rows of W bf16 (W a multiple of 64; row stride `stride` elements) into
+// shared memory with pitch W*2+16, rows >= nvalid zero-filled; lane (r0, c0) =
+// (lane / 8, lane % 8) copies columns c0, c0+8, ... of rows r0, r0+4, ...,
+// so every offset but the row step is a compile-time immediate.  `src` must
+// be a valid address even when nvalid <= 0.  No commit.
+template <int W>
+__device__ __forceinline__ void warp_issue_32rows(uint8_t* dst, const __nv_bfloat16* src, size_t stride, int nvalid) {
+    constexpr int PITCH = W * 2 + 16, J = W / 64;
+    const int lane = threadIdx.x & 31, c0 = lane & 7, r0 = lane >> 3;
+    const uint32_t d = smem_u32(dst) + r0 * PITCH + c0 * 16;
+    const __nv_bfloat16* s = src + (size_t)r0 * stride + c0 * 8;
+    const size_t step = 4 * stride;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const bool ok = r0 + 4 * k < nvalid;
+        const __nv_bfloat16* sk = ok ? s + k * step : src;
+        const uint32_t n = ok ? 16u : 0u;
+#pragma unroll
+        for (int j = 0; j < J; ++j)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d + (4 * k * PITCH + j * 128)),
+                         "l"(sk + j * 64), "r"(n)
+                         : "memory");
+    }
+}
+
+// issue + commit as one group
+__device__ __forceinline__ void warp_copy_rows(uint8_t* dst, int pitch, const __nv_bfloat16* src,
+                                               size_t src_stride, int rows, int nvalid, int width) {
+    warp_issue_rows(dst, pitch, src, src_stride, rows, nvalid, width);
+    cp_async_commit();
+}
 
 // the same with a per-row source pointer (nullptr rows are zero-filled)
 template <typename RowPtr>

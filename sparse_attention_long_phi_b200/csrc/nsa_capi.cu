@@ -565,18 +565,40 @@ nsa_status_t backward_impl(const Shape& s, const void* q, const void* k, const v
 }
 
 // ---------------------------------------------------------------- decode
+// SMs of the current device (cached per device)
+int device_sm_count() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev < 0 || dev >= 64) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
 template <int DK, int DV>
-nsa_status_t decode_launch(const DecParams& p, const Shape& s, int S, cudaStream_t st) {
-    const int rows_bytes = 32 * ((DK * 2 + 16) + (DV * 2 + 16));
-    NSA_TRY(set_smem(dec_cmp_partial<DK, DV>, 4 * rows_bytes));
-    NSA_LAUNCH("dec_cmp_partial", st, dec_cmp_partial<DK, DV><<<dim3((unsigned)p.NSPL, (unsigned)s.G, (unsigned)S), 128, 4 * rows_bytes, st>>>(p));
+nsa_status_t decode_launch(DecParams& p, const Shape& s, int S, cudaStream_t st) {
+    constexpr int smem = dec_stream_smem<DK, DV>();
+    const int nsm = device_sm_count();
+    // persistent streaming kernels: as many CTAs as fit on the device at once
+    int occ1 = 1, occ3 = 1;
+    NSA_TRY(set_smem(dec_cmp_stream<DK, DV>, smem));
+    NSA_TRY(set_smem(dec_slcwin_stream<DK, DV>, smem));
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ1, dec_cmp_stream<DK, DV>, 256, smem) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ3, dec_slcwin_stream<DK, DV>, 256, smem) != cudaSuccess)
+        return NSA_ERR_CUDA;
+    p.grid1 = std::min(kDecMaxGrid, nsm * std::max(1, occ1));
+    p.grid3 = std::min(kDecMaxGrid, nsm * std::max(1, occ3));
+    NSA_LAUNCH("dec_cmp_stream", st, dec_cmp_stream<DK, DV><<<(unsigned)p.grid1, 256, smem, st>>>(p));
     NSA_TRY(last_launch());
-    const int smem2 = p.NSmax * 4;
+    const int smem2 = (kDecMaxChunks * 16 + p.NCH * 16 + p.NSmax) * 4;
     NSA_TRY(set_smem(dec_cmp_combine<DV>, smem2));
     NSA_LAUNCH("dec_cmp_combine", st, dec_cmp_combine<DV><<<dim3((unsigned)s.G, (unsigned)S), 256, smem2, st>>>(p));
     NSA_TRY(last_launch());
-    NSA_TRY(set_smem(dec_slcwin_partial<DK, DV>, 2 * rows_bytes));
-    NSA_LAUNCH("dec_slcwin_partial", st, dec_slcwin_partial<DK, DV><<<dim3((unsigned)p.NU, (unsigned)s.G, (unsigned)S), 64, 2 * rows_bytes, st>>>(p));
+    NSA_LAUNCH("dec_slcwin_stream", st, dec_slcwin_stream<DK, DV><<<(unsigned)p.grid3, 256, smem, st>>>(p));
     NSA_TRY(last_launch());
     NSA_LAUNCH("dec_final", st, dec_final<DV><<<dim3((unsigned)s.G, (unsigned)S), 256, 0, st>>>(p));
     return last_launch();
@@ -600,6 +622,9 @@ nsa_status_t decode_impl(const Shape& s, int S, const void* q, const void* kcach
     p.fi = (int)s.fi;
     p.fl = (int)s.fl;
     p.w = (int)s.w;
+    p.spb = (int)(s.lp / s.d);
+    p.cps = (int)(s.l / s.d);
+    p.nbs = (31 + p.cps - 1) / p.spb + 1;
     p.scale_log2 = s.scale * kLog2e;
     p.q = reinterpret_cast<const __nv_bfloat16*>(q);
     p.kcache = reinterpret_cast<const __nv_bfloat16*>(kcache);
@@ -612,22 +637,27 @@ nsa_status_t decode_impl(const Shape& s, int S, const void* q, const void* kcach
     p.out = out;
     p.sel_idx = sel_idx;
     p.lse = lse;
+    p.Lmax = (int)s.T;
     p.Cmax = (int)(s.T >= s.l ? (s.T - s.l) / s.d + 1 : 1);
-    p.NSPL = (int)ceil_div(p.Cmax, kDecCH);
-    p.NU = (int)(s.n + ceil_div(s.w, s.lp) + 1);
+    p.NCH = (int)ceil_div(p.Cmax, 32);
+    p.NUV = (int)(s.n + ceil_div(s.w, s.lp) + 1);
     p.NSmax = (int)ceil_div(s.T, s.lp);
-    if (p.NSPL > kDecMaxSplits || p.NU > 48) return NSA_ERR_UNSUPPORTED;
+    if (S > kDecMaxSeqs || p.NCH > kDecMaxChunks || p.NUV > kDecMaxUnits || p.nbs > kDecNBS || 32 % p.spb != 0)
+        return NSA_ERR_UNSUPPORTED;
     size_t o = 0;
     auto carve = [&](size_t bytes) {
         float* r = reinterpret_cast<float*>(ws + o);
         o = align256(o + bytes);
         return r;
     };
-    p.part1 = carve((size_t)S * s.G * p.NSPL * 16 * (2 + s.DV) * 4);
-    p.bsc = carve((size_t)S * s.G * p.NSPL * 16 * kDecNJB * 4);
-    p.ocmp = carve((size_t)S * s.G * 16 * s.DV * 4);
-    p.lsecmp = carve((size_t)S * s.G * 16 * 4);
-    p.part2 = carve((size_t)S * s.G * p.NU * 2 * 16 * (2 + s.DV) * 4);
+    const size_t SG = (size_t)S * s.G;
+    p.cmax = carve(SG * p.NCH * 16 * 4);
+    p.bsum = carve(SG * p.NCH * kDecNBS * 16 * 4);
+    p.part1 = carve((kDecMaxGrid + SG) * 16 * (s.DV + 4) * 4);
+    p.ocmp = carve(SG * 16 * s.DV * 4);
+    p.lsecmp = carve(SG * 16 * 4);
+    p.part2 = carve((kDecMaxGrid + SG) * 2 * 16 * (s.DV + 4) * 4);
+    p.cpre = reinterpret_cast<int*>(carve((size_t)(S + 1) * 4));
     if (s.DK == 192) return decode_launch<192, 128>(p, s, S, st);
     return decode_launch<64, 64>(p, s, S, st);
 }

@@ -402,19 +402,25 @@ __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
     float* ifac = csm;
     float* fac = csm + kDecMaxChunks * 16;
     float* pg = fac + p.NCH * 16;
-    if (threadIdx.x < 16) {
-        const int h = threadIdx.x;
+    {   // LSE per head over the records: 16 threads per head
+        const int h = threadIdx.x >> 4, sub = threadIdx.x & 15;
         float M = -INFINITY;
-        for (int i = 0; i < nr; ++i) M = fmaxf(M, p.part1[((size_t)(recb[i] + sg) * 16 + h) * REC]);
+        for (int i = sub; i < nr; i += 16) M = fmaxf(M, p.part1[((size_t)(recb[i] + sg) * 16 + h) * REC]);
+#pragma unroll
+        for (int o = 8; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
         float Ls = 0.f;
-        for (int i = 0; i < nr; ++i) {
+        for (int i = sub; i < nr; i += 16) {
             const float* r = p.part1 + ((size_t)(recb[i] + sg) * 16 + h) * REC;
             if (r[0] != -INFINITY) Ls += r[1] * exp2f(r[0] - M);
         }
+#pragma unroll
+        for (int o = 8; o >= 1; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
         const float l2 = Ls > 0.f ? M + log2f(Ls) : -INFINITY;
-        lse2[h] = l2;
-        p.lsecmp[sg * 16 + h] = l2;
-        for (int i = 0; i < nr; ++i) {
+        if (sub == 0) {
+            lse2[h] = l2;
+            p.lsecmp[sg * 16 + h] = l2;
+        }
+        for (int i = sub; i < nr; i += 16) {
             const float m = p.part1[((size_t)(recb[i] + sg) * 16 + h) * REC];
             ifac[i * 16 + h] = (m != -INFINITY && l2 != -INFINITY) ? exp2f(m - l2) : 0.f;
         }
@@ -424,6 +430,7 @@ __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
     for (int e = threadIdx.x; e < 16 * (DV / 4); e += blockDim.x) {
         const int h = e / (DV / 4), c4 = (e % (DV / 4)) * 4;
         float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
         for (int i = 0; i < nr; ++i) {
             const float4 v = *reinterpret_cast<const float4*>(p.part1 + ((size_t)(recb[i] + sg) * 16 + h) * REC + 4 + c4);
             const float f = ifac[i * 16 + h];
@@ -441,18 +448,36 @@ __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
         fac[e] = (h < p.HG && lse2[h] != -INFINITY) ? exp2f(cm[e] - lse2[h]) : 0.f;
     }
     __syncthreads();
-    // group score of selection block j: the chunks holding keys j*spb-cps+1 .. j*spb+spb-1
+    // group score of selection block j: the chunks holding keys j*spb-cps+1 ..
+    // j*spb+spb-1 (at most two); 16 heads per slot as four float4 loads, all
+    // issued before use
     const int NSs = t / p.lp + 1;
     const int bpc = 32 / p.spb;                        // blocks starting in one chunk
     const float* bs = p.bsum + sg * p.NCH * kDecNBS * 16;
     for (int j = threadIdx.x; j < NSs; j += blockDim.x) {
-        float acc = 0.f;
         const int ilo = max(0, j * p.spb - p.cps + 1), ihi = min(C - 1, j * p.spb + p.spb - 1);
-        for (int cc = ilo >> 5; ilo <= ihi && cc <= (ihi >> 5); ++cc) {
-            const int jl = j - cc * bpc;
-            if (jl < 0 || jl >= p.nbs) continue;
-            const float* bp = bs + ((size_t)cc * kDecNBS + jl) * 16;
-            for (int h = 0; h < p.HG; ++h) acc += bp[h] * fac[cc * 16 + h];
+        float acc = 0.f;
+        if (ilo <= ihi) {
+            const int ca = ilo >> 5, cb = ihi >> 5;    // cb - ca <= 1
+            float4 v[2][4];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int cc = ca + q, jl = j - cc * bpc;
+                const bool use = cc <= cb && jl >= 0 && jl < p.nbs;
+                const float4* bp = reinterpret_cast<const float4*>(bs + ((size_t)(use ? cc : ca) * kDecNBS + (use ? jl : 0)) * 16);
+#pragma unroll
+                for (int h4 = 0; h4 < 4; ++h4)
+                    v[q][h4] = (use && h4 * 4 < p.HG) ? bp[h4] : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int cc = min(ca + q, cb);
+                const float* f = fac + cc * 16;
+#pragma unroll
+                for (int h4 = 0; h4 < 4; ++h4)
+                    acc += v[q][h4].x * f[h4 * 4] + v[q][h4].y * f[h4 * 4 + 1] + v[q][h4].z * f[h4 * 4 + 2] +
+                           v[q][h4].w * f[h4 * 4 + 3];
+            }
         }
         pg[j] = acc;
     }
@@ -655,20 +680,25 @@ __global__ void __launch_bounds__(256) dec_final(const DecParams p) {
     __syncthreads();
     const int nr = nrec;
     auto recp = [&](int i, int br) { return p.part2 + (((size_t)recb[i] + sg) * 2 + br) * 16 * REC; };
-    if (threadIdx.x < 32) {
-        const int br = threadIdx.x / 16, h = threadIdx.x % 16;
+    {   // per branch and head: 8 threads over the records
+        const int bh = threadIdx.x >> 3, sub = threadIdx.x & 7;
+        const int br = bh >> 4, h = bh & 15;
         float M = -INFINITY;
-        for (int i = 0; i < nr; ++i) M = fmaxf(M, recp(i, br)[h * REC]);
+        for (int i = sub; i < nr; i += 8) M = fmaxf(M, recp(i, br)[h * REC]);
+#pragma unroll
+        for (int o = 4; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
         float Ls = 0.f;
-        for (int i = 0; i < nr; ++i) {
+        for (int i = sub; i < nr; i += 8) {
             const float* r = recp(i, br) + h * REC;
             const float f = r[0] != -INFINITY ? exp2f(r[0] - M) : 0.f;
             fac[br][i][h] = f;
             Ls += r[1] * f;
         }
+#pragma unroll
+        for (int o = 4; o >= 1; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
         const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-        for (int i = 0; i < nr; ++i) fac[br][i][h] *= inv;
-        if (h < p.HG && p.lse) {
+        for (int i = sub; i < nr; i += 8) fac[br][i][h] *= inv;
+        if (sub == 0 && h < p.HG && p.lse) {
             const size_t row = (size_t)s * p.H + g * p.HG + h;
             p.lse[row * 3 + 1 + br] = Ls > 0.f ? (M + log2f(Ls)) * kLn2 : -INFINITY;
             if (br == 0) {
@@ -684,6 +714,7 @@ __global__ void __launch_bounds__(256) dec_final(const DecParams p) {
 #pragma unroll
         for (int br = 0; br < 2; ++br) {
             float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
             for (int i = 0; i < nr; ++i) {
                 const float4 v = *reinterpret_cast<const float4*>(recp(i, br) + h * REC + 4 + c4);
                 const float f = fac[br][i][h];

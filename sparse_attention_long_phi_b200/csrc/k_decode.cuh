@@ -172,9 +172,15 @@ __global__ void __launch_bounds__(256, 1) dec_cmp_stream(const DecParams p) {
     float(*pt)[16][33] = reinterpret_cast<float(*)[16][33]>(dsm + kDecW * STG);  // [8][16][33]
     __shared__ float wm[kDecW][16], wl[kDecW][16];
     __shared__ int pre[kDecMaxSeqs + 1];
+    __shared__ uint64_t kbar[kDecW], vbar[kDecW];    // per warp: its K / V rows landed
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gr = lane >> 2, tg = lane & 3;
     uint8_t* ks = dsm + warp * STG;
     uint8_t* vs = ks + 32 * KP;
+    if (threadIdx.x < kDecW) {
+        mbar_init(&kbar[threadIdx.x], 1);
+        mbar_init(&vbar[threadIdx.x], 1);
+    }
+    fence_mbar_init();
 
     // chunks (x G) before sequence s: exclusive prefix by warp 0
     if (warp == 0) {
@@ -206,6 +212,8 @@ __global__ void __launch_bounds__(256, 1) dec_cmp_stream(const DecParams p) {
     const long long x1 = dec_range_start(b + 1, N, gridDim.x);
     const float cl = p.scale_log2;
     const bool fast = p.spb == 4 && p.cps == 2;
+    uint32_t kph = 0, vph = 0;
+    const uint64_t pol = l2_evict_first();
     while (x < x1) {
         // segment: consecutive chunks of one (seq, group)
         int lo = 0, hi = p.S;                       // largest lo with pre[lo] <= x
@@ -225,14 +233,8 @@ __global__ void __launch_bounds__(256, 1) dec_cmp_stream(const DecParams p) {
         const size_t kst = (size_t)p.G * DK, vst = (size_t)p.G * DV;
         const __nv_bfloat16* kb = p.kccache + ((size_t)cbase * p.G + g) * DK;
         const __nv_bfloat16* vb = p.vccache + ((size_t)cbase * p.G + g) * DV;
-        auto issue_k = [&](int c) {
-            warp_issue_32rows<DK>(ks, kb + (size_t)c * 32 * kst, kst, C - c * 32);
-            cp_async_commit();
-        };
-        auto issue_v = [&](int c) {
-            warp_issue_32rows<DV>(vs, vb + (size_t)c * 32 * vst, vst, C - c * 32);
-            cp_async_commit();
-        };
+        auto issue_k = [&](int c) { warp_bulk_rows<DK>(ks, kb + (size_t)c * 32 * kst, kst, C - c * 32, &kbar[warp], pol); };
+        auto issue_v = [&](int c) { warp_bulk_rows<DV>(vs, vb + (size_t)c * 32 * vst, vst, C - c * 32, &vbar[warp], pol); };
         uint32_t qa[DK / 16][4];
         load_q_frags<DK>(p, s, g, qa);
         float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
@@ -249,7 +251,8 @@ __global__ void __launch_bounds__(256, 1) dec_cmp_stream(const DecParams p) {
         for (; i < n; i += kDecW) {
             const int c = cfirst + i;
             const bool more = i + kDecW < n;
-            cp_async_wait_1();                      // K of chunk c
+            if (!mbar_wait(&kbar[warp], kph, 0x401)) break;   // K of chunk c
+            kph ^= 1;
             __syncwarp();
             float sf[4][4];
             warp_logits<DK>(qa, smem_u32(ks), sf);
@@ -337,8 +340,8 @@ __global__ void __launch_bounds__(256, 1) dec_cmp_stream(const DecParams p) {
                 p.cmax[cr * 16 + gr] = mc0;
                 p.cmax[cr * 16 + gr + 8] = mc1;
             }
-            if (more) cp_async_wait_1();            // V of chunk c
-            else cp_async_wait();
+            if (!mbar_wait(&vbar[warp], vph, 0x402)) break;   // V of chunk c
+            vph ^= 1;
             __syncwarp();
             // online softmax for O: rescale to the new running max
             const float mn0 = fmaxf(m0, mc0), mn1 = fmaxf(m1, mc1);
@@ -373,6 +376,9 @@ __global__ void __launch_bounds__(256, 1) dec_cmp_stream(const DecParams p) {
 }
 
 // -------------------------------------------------------------- step 2
+// Every load that does not need the row LSE (records, chunk maxima, this
+// thread's block sums) is issued before the first barrier, so the kernel
+// waits about one memory round trip; the top-n runs on all 8 warps.
 template <int DV>
 __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
     constexpr int REC = DV + 4;
@@ -380,6 +386,8 @@ __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
     __shared__ float lse2[16];
     __shared__ int recb[kDecMaxChunks];
     __shared__ int nrec;
+    __shared__ float tsv[8 * 16];
+    __shared__ int tsi[8 * 16];
     const int g = blockIdx.x, s = blockIdx.y;
     int L, C;
     if (!dec_seq_ok(p, s, L, C)) {
@@ -397,11 +405,39 @@ __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
         }
         nrec = cnt;
     }
-    __syncthreads();
-    const int nr = nrec;
     float* ifac = csm;
     float* fac = csm + kDecMaxChunks * 16;
     float* pg = fac + p.NCH * 16;
+    // chunk maxima (log2 units) and this thread's block sums: independent of the LSE
+    const float* cm = p.cmax + sg * p.NCH * 16;
+    for (int e = threadIdx.x; e < nch * 16; e += blockDim.x) fac[e] = cm[e];
+    const int NSs = t / p.lp + 1;
+    const int bpc = 32 / p.spb;                        // blocks starting in one chunk
+    const float* bs = p.bsum + sg * p.NCH * kDecNBS * 16;
+    // block j takes the chunks holding keys j*spb-cps+1 .. j*spb+spb-1 (at most two)
+    auto block_chunks = [&](int j, int& ca, int& cb) {
+        const int ilo = max(0, j * p.spb - p.cps + 1), ihi = min(C - 1, j * p.spb + p.spb - 1);
+        ca = ilo >> 5;
+        cb = ilo <= ihi ? (ihi >> 5) : ca - 1;
+    };
+    float4 bv[4][2][4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int j = threadIdx.x + q * blockDim.x;
+        int ca, cb;
+        block_chunks(j, ca, cb);
+#pragma unroll
+        for (int qq = 0; qq < 2; ++qq) {
+            const int cc = ca + qq, jl = j - cc * bpc;
+            const bool use = j < NSs && cc <= cb && jl >= 0 && jl < p.nbs;
+            const float4* bp = reinterpret_cast<const float4*>(bs + ((size_t)(use ? cc : 0) * kDecNBS + (use ? jl : 0)) * 16);
+#pragma unroll
+            for (int h4 = 0; h4 < 4; ++h4)
+                bv[q][qq][h4] = (use && h4 * 4 < p.HG) ? bp[h4] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    __syncthreads();                                   // nrec, recb, fac (raw)
+    const int nr = nrec;
     {   // LSE per head over the records: 16 threads per head
         const int h = threadIdx.x >> 4, sub = threadIdx.x & 15;
         float M = -INFINITY;
@@ -426,6 +462,11 @@ __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
         }
     }
     __syncthreads();
+    // per chunk and head: exp2(chunk max - LSE); heads past HG do not score
+    for (int e = threadIdx.x; e < nch * 16; e += blockDim.x) {
+        const int h = e & 15;
+        fac[e] = (h < p.HG && lse2[h] != -INFINITY) ? exp2f(fac[e] - lse2[h]) : 0.f;
+    }
     // o_cmp = sum over records of O exp2(m - LSE)
     for (int e = threadIdx.x; e < 16 * (DV / 4); e += blockDim.x) {
         const int h = e / (DV / 4), c4 = (e % (DV / 4)) * 4;
@@ -441,48 +482,43 @@ __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
         }
         *reinterpret_cast<float4*>(p.ocmp + (sg * 16 + h) * DV + c4) = a;
     }
-    // per chunk and head: exp2(chunk max - LSE); heads past HG do not score
-    const float* cm = p.cmax + sg * p.NCH * 16;
-    for (int e = threadIdx.x; e < nch * 16; e += blockDim.x) {
-        const int h = e & 15;
-        fac[e] = (h < p.HG && lse2[h] != -INFINITY) ? exp2f(cm[e] - lse2[h]) : 0.f;
-    }
     __syncthreads();
-    // group score of selection block j: the chunks holding keys j*spb-cps+1 ..
-    // j*spb+spb-1 (at most two); 16 heads per slot as four float4 loads, all
-    // issued before use
-    const int NSs = t / p.lp + 1;
-    const int bpc = 32 / p.spb;                        // blocks starting in one chunk
-    const float* bs = p.bsum + sg * p.NCH * kDecNBS * 16;
-    for (int j = threadIdx.x; j < NSs; j += blockDim.x) {
-        const int ilo = max(0, j * p.spb - p.cps + 1), ihi = min(C - 1, j * p.spb + p.spb - 1);
+    auto dot16 = [&](const float4 (&v)[4], const float* f) {
         float acc = 0.f;
-        if (ilo <= ihi) {
-            const int ca = ilo >> 5, cb = ihi >> 5;    // cb - ca <= 1
-            float4 v[2][4];
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                const int cc = ca + q, jl = j - cc * bpc;
-                const bool use = cc <= cb && jl >= 0 && jl < p.nbs;
-                const float4* bp = reinterpret_cast<const float4*>(bs + ((size_t)(use ? cc : ca) * kDecNBS + (use ? jl : 0)) * 16);
+        for (int h4 = 0; h4 < 4; ++h4)
+            acc += v[h4].x * f[h4 * 4] + v[h4].y * f[h4 * 4 + 1] + v[h4].z * f[h4 * 4 + 2] + v[h4].w * f[h4 * 4 + 3];
+        return acc;
+    };
 #pragma unroll
-                for (int h4 = 0; h4 < 4; ++h4)
-                    v[q][h4] = (use && h4 * 4 < p.HG) ? bp[h4] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int q = 0; q < 4; ++q) {
+        const int j = threadIdx.x + q * blockDim.x;
+        if (j < NSs) {
+            int ca, cb;
+            block_chunks(j, ca, cb);
+            float acc = 0.f;
+#pragma unroll
+            for (int qq = 0; qq < 2; ++qq) {
+                const int cc = ca + qq, jl = j - cc * bpc;
+                if (cc <= cb && jl >= 0 && jl < p.nbs) acc += dot16(bv[q][qq], fac + cc * 16);
             }
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                const int cc = min(ca + q, cb);
-                const float* f = fac + cc * 16;
-#pragma unroll
-                for (int h4 = 0; h4 < 4; ++h4)
-                    acc += v[q][h4].x * f[h4 * 4] + v[q][h4].y * f[h4 * 4 + 1] + v[q][h4].z * f[h4 * 4 + 2] +
-                           v[q][h4].w * f[h4 * 4 + 3];
-            }
+            pg[j] = acc;
+        }
+    }
+    for (int j = threadIdx.x + 4 * blockDim.x; j < NSs; j += blockDim.x) {   // rows longer than 1024 blocks
+        int ca, cb;
+        block_chunks(j, ca, cb);
+        float acc = 0.f;
+        for (int cc = ca; cc <= cb; ++cc) {
+            const int jl = j - cc * bpc;
+            if (jl < 0 || jl >= p.nbs) continue;
+            const float* bp = bs + ((size_t)cc * kDecNBS + jl) * 16;
+            for (int h = 0; h < p.HG; ++h) acc += bp[h] * fac[cc * 16 + h];
         }
         pg[j] = acc;
     }
     __syncthreads();
-    if (threadIdx.x < 32) topn_row_warp(pg, t, p.n, p.lp, p.fi, p.fl, p.sel_idx + sg * p.n, threadIdx.x);
+    topn_row_cta<8>(pg, t, p.n, p.lp, p.fi, p.fl, p.sel_idx + sg * p.n, tsv, tsi);
 }
 
 // sorted union of the selected blocks (sel: n entries, -1 padded, ascending)
@@ -522,9 +558,18 @@ __global__ void __launch_bounds__(256, 1) dec_slcwin_stream(const DecParams p) {
     __shared__ int ulist[kDecMaxUnits], uflag[kDecMaxUnits];
     __shared__ int selbuf[32];
     __shared__ int nunits;
+    __shared__ uint64_t kbar[kDecW], vbar[kDecW];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tg = lane & 3;
     uint8_t* ks = dsm + warp * STG;
     uint8_t* vs = ks + 32 * KP;
+    if (threadIdx.x < kDecW) {
+        mbar_init(&kbar[threadIdx.x], 1);
+        mbar_init(&vbar[threadIdx.x], 1);
+    }
+    fence_mbar_init();
+    __syncthreads();
+    uint32_t kph = 0, vph = 0;
+    const uint64_t pol = l2_evict_first();
     const long long U = (long long)p.S * p.G * p.NUV;     // unit slots, NUV per (seq, group)
     const int b = blockIdx.x;
     long long x = dec_range_start(b, U, gridDim.x);
@@ -557,13 +602,11 @@ __global__ void __launch_bounds__(256, 1) dec_slcwin_stream(const DecParams p) {
         // rows past the cache are not read; the source stays inside the sequence
         auto issue_k = [&](int i) {
             const int u0 = tok0(i), nv = min(32, L - u0);
-            warp_issue_32rows<DK>(ks, p.kcache + ((size_t)(kvb + (nv > 0 ? u0 : 0)) * p.G + g) * DK, kst, nv);
-            cp_async_commit();
+            warp_bulk_rows<DK>(ks, p.kcache + ((size_t)(kvb + (nv > 0 ? u0 : 0)) * p.G + g) * DK, kst, nv, &kbar[warp], pol);
         };
         auto issue_v = [&](int i) {
             const int u0 = tok0(i), nv = min(32, L - u0);
-            warp_issue_32rows<DV>(vs, p.vcache + ((size_t)(kvb + (nv > 0 ? u0 : 0)) * p.G + g) * DV, vst, nv);
-            cp_async_commit();
+            warp_bulk_rows<DV>(vs, p.vcache + ((size_t)(kvb + (nv > 0 ? u0 : 0)) * p.G + g) * DV, vst, nv, &vbar[warp], pol);
         };
         float m[2][2], l[2][2];
         float o[2][DV / 8][4];
@@ -590,14 +633,15 @@ __global__ void __launch_bounds__(256, 1) dec_slcwin_stream(const DecParams p) {
             // warp-uniform: does the chunk hold keys of each branch?
             const bool has_sel = insel && nval > 0;
             const bool has_win = nval > 0 && u0 + nval - 1 >= wlo;
-            cp_async_wait_1();                          // K of chunk i
+            if (!mbar_wait(&kbar[warp], kph, 0x403)) break;   // K of chunk i
+            kph ^= 1;
             __syncwarp();
             float sf[4][4];
             if (has_sel || has_win) warp_logits_sa<DK>(smem_u32(qs), smem_u32(ks), sf);
             __syncwarp();
             if (more) issue_k(i + kDecW);
-            if (more) cp_async_wait_1();                // V of chunk i
-            else cp_async_wait();
+            if (!mbar_wait(&vbar[warp], vph, 0x404)) break;   // V of chunk i
+            vph ^= 1;
             __syncwarp();
 #pragma unroll
             for (int br = 0; br < 2; ++br) {
@@ -663,10 +707,12 @@ __global__ void __launch_bounds__(256, 1) dec_slcwin_stream(const DecParams p) {
 }
 
 // -------------------------------------------------------------- step 4
+// One thread per output float4: it merges its head's records of both
+// branches itself (one pass, running max), so the only barrier is the one
+// that publishes the record list.
 template <int DV>
 __global__ void __launch_bounds__(256) dec_final(const DecParams p) {
     constexpr int REC = DV + 4;
-    __shared__ float fac[2][kDecMaxUnits][16];
     __shared__ int recb[kDecMaxUnits];
     __shared__ int nrec;
     const int g = blockIdx.x, s = blockIdx.y;
@@ -679,61 +725,47 @@ __global__ void __launch_bounds__(256) dec_final(const DecParams p) {
     }
     __syncthreads();
     const int nr = nrec;
-    auto recp = [&](int i, int br) { return p.part2 + (((size_t)recb[i] + sg) * 2 + br) * 16 * REC; };
-    {   // per branch and head: 8 threads over the records
-        const int bh = threadIdx.x >> 3, sub = threadIdx.x & 7;
-        const int br = bh >> 4, h = bh & 15;
-        float M = -INFINITY;
-        for (int i = sub; i < nr; i += 8) M = fmaxf(M, recp(i, br)[h * REC]);
-#pragma unroll
-        for (int o = 4; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-        float Ls = 0.f;
-        for (int i = sub; i < nr; i += 8) {
-            const float* r = recp(i, br) + h * REC;
-            const float f = r[0] != -INFINITY ? exp2f(r[0] - M) : 0.f;
-            fac[br][i][h] = f;
-            Ls += r[1] * f;
-        }
-#pragma unroll
-        for (int o = 4; o >= 1; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
-        const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-        for (int i = sub; i < nr; i += 8) fac[br][i][h] *= inv;
-        if (sub == 0 && h < p.HG && p.lse) {
-            const size_t row = (size_t)s * p.H + g * p.HG + h;
-            p.lse[row * 3 + 1 + br] = Ls > 0.f ? (M + log2f(Ls)) * kLn2 : -INFINITY;
-            if (br == 0) {
-                const float lc = p.lsecmp[sg * 16 + h];
-                p.lse[row * 3] = lc == -INFINITY ? -INFINITY : lc * kLn2;
-            }
-        }
-    }
-    __syncthreads();
     for (int e = threadIdx.x; e < p.HG * (DV / 4); e += blockDim.x) {
         const int h = e / (DV / 4), c4 = (e % (DV / 4)) * 4;
-        float4 ob[2];
-#pragma unroll
-        for (int br = 0; br < 2; ++br) {
-            float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-            for (int i = 0; i < nr; ++i) {
-                const float4 v = *reinterpret_cast<const float4*>(recp(i, br) + h * REC + 4 + c4);
-                const float f = fac[br][i][h];
-                a.x += v.x * f;
-                a.y += v.y * f;
-                a.z += v.z * f;
-                a.w += v.w * f;
-            }
-            ob[br] = a;
-        }
         const size_t row = (size_t)s * p.H + g * p.HG + h;
         const float4 oc = *reinterpret_cast<const float4*>(p.ocmp + (sg * 16 + h) * DV + c4);
-        const float g0 = p.gates[row * 3], g1 = p.gates[row * 3 + 1], g2 = p.gates[row * 3 + 2];
+        const float gt0 = p.gates[row * 3], gt1 = p.gates[row * 3 + 1], gt2 = p.gates[row * 3 + 2];
+        float M[2] = {-INFINITY, -INFINITY}, Ls[2] = {0.f, 0.f};
+        float4 O[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+#pragma unroll 4
+        for (int i = 0; i < nr; ++i) {
+#pragma unroll
+            for (int br = 0; br < 2; ++br) {
+                const float* r = p.part2 + ((((size_t)recb[i] + sg) * 2 + br) * 16 + h) * REC;
+                const float m = r[0], l = r[1];
+                const float4 v = *reinterpret_cast<const float4*>(r + 4 + c4);
+                if (m == -INFINITY) continue;
+                const float Mn = fmaxf(M[br], m);
+                const float a = exp2f(M[br] - Mn), f = exp2f(m - Mn);   // M = -inf first: a = 0
+                Ls[br] = Ls[br] * a + l * f;
+                O[br].x = O[br].x * a + v.x * f;
+                O[br].y = O[br].y * a + v.y * f;
+                O[br].z = O[br].z * a + v.z * f;
+                O[br].w = O[br].w * a + v.w * f;
+                M[br] = Mn;
+            }
+        }
+        float inv[2];
+#pragma unroll
+        for (int br = 0; br < 2; ++br) inv[br] = Ls[br] > 0.f ? 1.f / Ls[br] : 0.f;
         float4 r;
-        r.x = g0 * oc.x + g1 * ob[0].x + g2 * ob[1].x;
-        r.y = g0 * oc.y + g1 * ob[0].y + g2 * ob[1].y;
-        r.z = g0 * oc.z + g1 * ob[0].z + g2 * ob[1].z;
-        r.w = g0 * oc.w + g1 * ob[0].w + g2 * ob[1].w;
+        r.x = gt0 * oc.x + gt1 * O[0].x * inv[0] + gt2 * O[1].x * inv[1];
+        r.y = gt0 * oc.y + gt1 * O[0].y * inv[0] + gt2 * O[1].y * inv[1];
+        r.z = gt0 * oc.z + gt1 * O[0].z * inv[0] + gt2 * O[1].z * inv[1];
+        r.w = gt0 * oc.w + gt1 * O[0].w * inv[0] + gt2 * O[1].w * inv[1];
         *reinterpret_cast<float4*>(p.out + row * DV + c4) = r;
+        if (c4 == 0 && p.lse) {
+#pragma unroll
+            for (int br = 0; br < 2; ++br)
+                p.lse[row * 3 + 1 + br] = Ls[br] > 0.f ? (M[br] + log2f(Ls[br])) * kLn2 : -INFINITY;
+            const float lc = p.lsecmp[sg * 16 + h];
+            p.lse[row * 3] = lc == -INFINITY ? -INFINITY : lc * kLn2;
+        }
     }
 }
 

@@ -75,6 +75,43 @@ __device__ __forceinline__ void warp_issue_32rows(uint8_t* dst, const __nv_bfloa
     }
 }
 
+// L2 policy for data read once: evicted first, so that small results written
+// meanwhile stay cached for the kernels that read them next
+__device__ __forceinline__ uint64_t l2_evict_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// 32 rows of W bf16 (row stride `stride` elements) into shared memory rows of
+// pitch W*2+16 with one bulk (TMA) copy per lane, completing on `bar`, which
+// this call arms for the min(nrows, 32) valid rows; the others are zero-filled by
+// plain stores.  Bulk copies bypass the L1 miss queue that bounds cp.async
+// streaming.  `policy` is an L2 cache policy (see l2_evict_first) for the
+// copies.  The caller waits on `bar` (phase parity) and then __syncwarp()s
+// before reading.  Earlier generic accesses of the rows are fenced first.
+template <int W>
+__device__ __forceinline__ void warp_bulk_rows(uint8_t* dst, const __nv_bfloat16* src, size_t stride, int nrows,
+                                               uint64_t* bar, uint64_t policy) {
+    constexpr int PITCH = W * 2 + 16, BYTES = W * 2;
+    const int lane = threadIdx.x & 31;
+    nrows = max(0, min(nrows, 32));
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_expect_tx(bar, (uint32_t)(max(nrows, 0) * BYTES));
+    __syncwarp();
+    uint8_t* row = dst + lane * PITCH;
+    if (lane < nrows) {
+        asm volatile(
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+            ::"r"(smem_u32(row)), "l"(src + (size_t)lane * stride), "r"(BYTES), "r"(smem_u32(bar)), "l"(policy)
+            : "memory");
+    } else {   // rows past the valid ones
+#pragma unroll
+        for (int c = 0; c < BYTES / 16; ++c) st_shared_v4(smem_u32(row + c * 16), 0u, 0u, 0u, 0u);
+    }
+}
+
 // issue + commit as one group
 __device__ __forceinline__ void warp_copy_rows(uint8_t* dst, int pitch, const __nv_bfloat16* src,
                                                size_t src_stride, int rows, int nvalid, int width) {

@@ -85,6 +85,114 @@ __device__ __forceinline__ void topn_row_warp(const float* row, int t, int n, in
     if (lane < n) out[lane] = (srt == 0x7fffffff) ? -1 : srt;
 }
 
+// The same selection by a whole CTA of NW warps, for long candidate rows in
+// shared memory: warp w takes the top R of its contiguous slice of the scored
+// candidates, warp 0 then takes the top R of the NW*R survivors (ordered by
+// score, then lower index, exactly as above).  sv/si: NW*16 scratch slots.
+// Called by every thread of the CTA.
+template <int NW>
+__device__ __forceinline__ void topn_row_cta(const float* row, int t, int n, int lp, int fi, int fl,
+                                             int32_t* out, float* sv, int* si) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bt = t / lp;
+    const int ncand = bt + 1;
+    if (ncand <= n) {
+        if (threadIdx.x < n) out[threadIdx.x] = (int)threadIdx.x < ncand ? (int)threadIdx.x : -1;
+        return;
+    }
+    const int lo = fi, hi = bt - fl;
+    const int R = n - fi - fl;
+    const int M = hi - lo + 1;
+    const int per = (M + NW - 1) / NW;
+    constexpr int PL = (kTopnPerLane * 32 / NW + 31) / 32;      // values per lane per slice
+    const int s0 = lo + warp * per, s1 = min(hi + 1, s0 + per);
+    float v[PL];
+#pragma unroll
+    for (int k = 0; k < PL; ++k) {
+        const int j = s0 + lane + 32 * k;
+        v[k] = j < s1 ? row[j] : -1.f;              // scores are >= 0
+    }
+    for (int it = 0; it < R; ++it) {
+        float bv = -2.f;
+        int bk = 0;
+#pragma unroll
+        for (int k = 0; k < PL; ++k)
+            if (v[k] > bv) {
+                bv = v[k];
+                bk = k;
+            }
+        int bj = s0 + lane + 32 * bk;
+        if (bv < -0.5f) bj = 0x7fffffff;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+            if (ov > bv || (ov == bv && oj < bj)) {
+                bv = ov;
+                bj = oj;
+            }
+        }
+        if (bj != 0x7fffffff && ((bj - s0) & 31) == lane) {
+            const int kk = (bj - s0) >> 5;
+#pragma unroll
+            for (int k = 0; k < PL; ++k)
+                if (k == kk) v[k] = -1.f;
+        }
+        if (lane == 0) {
+            sv[warp * 16 + it] = bj == 0x7fffffff ? -2.f : bv;
+            si[warp * 16 + it] = bj;
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        constexpr int Q = (NW * 16 + 31) / 32;
+        float w[Q];
+        int wi[Q];
+#pragma unroll
+        for (int k = 0; k < Q; ++k) {
+            const int e = lane + 32 * k, ww = e / 16, r = e % 16;
+            const bool ok = ww < NW && r < R;
+            w[k] = ok ? sv[e] : -2.f;
+            wi[k] = ok ? si[e] : 0x7fffffff;
+        }
+        int mine = 0x7fffffff;
+        for (int it = 0; it < R; ++it) {
+            float bv = -2.f;
+            int bj = 0x7fffffff, bk = -1;
+#pragma unroll
+            for (int k = 0; k < Q; ++k)
+                if (w[k] > bv || (w[k] == bv && wi[k] < bj)) {
+                    bv = w[k];
+                    bj = wi[k];
+                    bk = k;
+                }
+            if (bv < -0.5f) bj = 0x7fffffff;
+            int owner = bk >= 0 ? lane : 32;
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+                const int oo = __shfl_xor_sync(0xffffffffu, owner, o);
+                if (ov > bv || (ov == bv && oj < bj)) {
+                    bv = ov;
+                    bj = oj;
+                    owner = oo;
+                }
+            }
+            if (bj != 0x7fffffff && owner == lane) {
+#pragma unroll
+                for (int k = 0; k < Q; ++k)
+                    if (wi[k] == bj) w[k] = -2.f;
+            }
+            if (lane == it) mine = bj;
+        }
+        if (lane >= R && lane < R + fi) mine = lane - R;
+        if (lane >= R + fi && lane < R + fi + fl) mine = bt - fl + 1 + (lane - R - fi);
+        const int srt = warp_sort_asc(mine, lane);
+        if (lane < n) out[lane] = (srt == 0x7fffffff) ? -1 : srt;
+    }
+}
+
 // one warp per (batch, token, group) item; scores [items, NSp]
 __global__ void __launch_bounds__(256)
     topn_kernel(const float* __restrict__ pscore, long long items, int T, int G, int NSp, int n,

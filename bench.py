@@ -216,6 +216,8 @@ def main():
     ap.add_argument("--workload", default="prefill_fwd_T65536")
     ap.add_argument("--seq-len", type=int, default=0, help="override T (smaller profiling cases)")
     ap.add_argument("--no-extras", action="store_true", help="skip e2e, CPU, decode, backward")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="run only the batched-decode measurement (profiling the decode kernels)")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
@@ -243,6 +245,9 @@ def main():
     torch.cuda.set_device(dev)
     from sparse_attention_long_phi_b200 import nsa
     peaks, peak_src = load_peaks()
+    if args.decode_only:
+        print(json.dumps(bench_decode(dev, nsa, peaks, peak_src, steps=args.steps, warmup=args.warmup)), flush=True)
+        return
 
     # inputs: per-rank seed (independent sequences), resident in HBM
     cr = dict(c, seed=c["seed"] + 7919 * rank)

@@ -542,17 +542,21 @@ nsa_status_t backward_impl(const Shape& s, const void* q, const void* k, const v
         NSA_LAUNCH("bwd_sel_fill", st, bwd_sel_fill<<<(unsigned)ceil_div(N, 256), 256, 0, st>>>(p));
         NSA_TRY(last_launch());
     }
-    // key-centric dK/dV
+    // key-centric dK/dV (tensor cores, 16 heads = N)
     {
+        constexpr int kvs = bwd_kv_mma_smem<DK, DV>();
+        NSA_TRY(set_smem(bwd_kv_mma<DK, DV, kBrWin>, kvs));
+        NSA_TRY(set_smem(bwd_kv_mma<DK, DV, kBrSlc>, kvs));
+        NSA_TRY(set_smem(bwd_kv_mma<DK, DV, kBrCmp>, kvs));
         dim3 gw((unsigned)ceil_div(s.T, 64), (unsigned)ceil_div(64 + s.w - 1, kBwdChunk), (unsigned)(s.B * s.G));
-        NSA_LAUNCH("bwd_kv_kernel", st, bwd_kv_kernel<DK, DV, kBrWin><<<gw, 256, 0, st>>>(p));
+        NSA_LAUNCH("bwd_kv_mma", st, bwd_kv_mma<DK, DV, kBrWin><<<gw, 128, kvs, st>>>(p));
         NSA_TRY(last_launch());
         const int64_t maxch = NE + ceil_div(s.B * s.T * s.G * s.n, kBwdChunk);
-        NSA_LAUNCH("bwd_kv_kernel", st, bwd_kv_kernel<DK, DV, kBrSlc><<<(unsigned)maxch, 256, 0, st>>>(p));
+        NSA_LAUNCH("bwd_kv_mma", st, bwd_kv_mma<DK, DV, kBrSlc><<<(unsigned)maxch, 128, kvs, st>>>(p));
         NSA_TRY(last_launch());
         if (s.C > 0) {
             dim3 gc((unsigned)ceil_div(s.C, 64), (unsigned)ceil_div(s.T, kBwdChunk), (unsigned)(s.B * s.G));
-            NSA_LAUNCH("bwd_kv_kernel", st, bwd_kv_kernel<DK, DV, kBrCmp><<<gc, 256, 0, st>>>(p));
+            NSA_LAUNCH("bwd_kv_mma", st, bwd_kv_mma<DK, DV, kBrCmp><<<gc, 128, kvs, st>>>(p));
             NSA_TRY(last_launch());
             dim3 gp((unsigned)s.T, (unsigned)s.G, (unsigned)s.B);
             NSA_LAUNCH("bwd_phiT_kernel", st, bwd_phiT_kernel<DK><<<gp, DK, 0, st>>>(p, p.dkc, p.wk, dk));

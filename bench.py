@@ -218,6 +218,8 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip e2e, CPU, decode, backward")
     ap.add_argument("--decode-only", action="store_true",
                     help="run only the batched-decode measurement (profiling the decode kernels)")
+    ap.add_argument("--backward-only", action="store_true",
+                    help="run only the forward+backward training measurement (profiling the backward)")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
@@ -247,6 +249,10 @@ def main():
     peaks, peak_src = load_peaks()
     if args.decode_only:
         print(json.dumps(bench_decode(dev, nsa, peaks, peak_src, steps=args.steps, warmup=args.warmup)), flush=True)
+        return
+    if args.backward_only:
+        print(json.dumps(bench_backward(dev, nsa, peaks, steps=args.steps, warmup=args.warmup,
+                                        seq_len=args.seq_len)), flush=True)
         return
 
     # inputs: per-rank seed (independent sequences), resident in HBM
@@ -434,9 +440,11 @@ def bench_decode(dev, nsa, peaks, peak_src, steps=50, warmup=5):
             "l2": "flushed (512 MB write) before each timed step"}
 
 
-def bench_backward(dev, nsa, peaks, steps=2, warmup=1):
-    """Forward + backward of the training workload (B=2, T=16384)."""
+def bench_backward(dev, nsa, peaks, steps=2, warmup=1, seq_len=0):
+    """Forward + backward of the training workload (B=2, T=16384; T overridable for profiling)."""
     c = dict(I.WORKLOADS["train_fwd_bwd_B2_T16384"])
+    if seq_len:
+        c["T"] = seq_len
     x = I.make_forward_inputs(c, dev, with_dout=True)
     phi = {k: x[k] for k in ("wk", "ek", "wv", "ev")}
     stream = torch.cuda.current_stream(dev)
@@ -463,7 +471,8 @@ def bench_backward(dev, nsa, peaks, steps=2, warmup=1):
     f_ms, b_ms = e0.elapsed_time(e1) / steps, e1.elapsed_time(e2) / steps
     _, fwd = forward_flops(c)
     bwd = 2 * fwd                               # dP, dV, dQ, dK
-    return {"workload": "train_fwd_bwd_B2_T16384", "fwd_ms": round(f_ms, 3), "bwd_ms": round(b_ms, 3),
+    return {"workload": "train_fwd_bwd_B2_T16384" if not seq_len else f"train_fwd_bwd_B2_T{seq_len}",
+            "fwd_ms": round(f_ms, 3), "bwd_ms": round(b_ms, 3),
             "tokens_per_s": round(c["B"] * c["T"] / ((f_ms + b_ms) / 1e3), 1),
             "bwd_tflops_algorithmic": round(bwd / (b_ms / 1e3) / 1e12, 2),
             "bwd_frac_of_peak": round(bwd / (b_ms / 1e3) / 1e12 / peaks.get("bf16_tflops", 1590.0), 4),

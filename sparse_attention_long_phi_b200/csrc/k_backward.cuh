@@ -102,31 +102,34 @@ __global__ void __launch_bounds__(128) bwd_query_mma(const BwdParams p) {
         lo = max(0, t - p.w + 1);
         return t - lo + 1;
     };
-    auto token_of = [&](int br, int lo, int key) -> int {
-        return br == kBrSlc ? units[key / p.lp] * p.lp + key % p.lp : lo + key;
-    };
-    auto stage = [&](int br, int lo, int nk, int k0) {
-        warp_copy_rows_ptr(ks, KP, [&](int r) -> const __nv_bfloat16* {
-            const int key = k0 + r;
-            if (key >= nk) return nullptr;
-            if (br == kBrCmp) return p.kc + (((size_t)b * p.C + key) * p.G + g) * DK;
-            const int u = token_of(br, lo, key);
-            return u > t ? nullptr : p.k + (((size_t)b * p.T + u) * p.G + g) * DK;
-        }, 32, DK);
-        warp_copy_rows_ptr(vs, VP, [&](int r) -> const __nv_bfloat16* {
-            const int key = k0 + r;
-            if (key >= nk) return nullptr;
-            if (br == kBrCmp) return p.vc + (((size_t)b * p.C + key) * p.G + g) * DV;
-            const int u = token_of(br, lo, key);
-            return u > t ? nullptr : p.v + (((size_t)b * p.T + u) * p.G + g) * DV;
-        }, 32, DV);
+    // Stage the 32 keys k0.. of a branch (K rows at ks, V rows at vs) and return
+    // how many of them the query sees: they are a prefix, because a chunk's rows
+    // are consecutive cache rows (a selected block holds whole 32-key chunks) in
+    // increasing token order.
+    auto stage = [&](int br, int lo, int nk, int k0) -> int {
+        int row0, nval = min(32, nk - k0);
+        const __nv_bfloat16 *kb, *vb;
+        if (br == kBrCmp) {
+            row0 = k0;
+            kb = p.kc + (((size_t)b * p.C + row0) * p.G + g) * DK;
+            vb = p.vc + (((size_t)b * p.C + row0) * p.G + g) * DV;
+        } else {
+            if (br == kBrSlc) {
+                const int ui = k0 / p.lp;
+                row0 = units[ui] * p.lp + (k0 - ui * p.lp);
+                nval = min(nval, t - row0 + 1);
+            } else {
+                row0 = lo + k0;
+            }
+            kb = p.k + (((size_t)b * p.T + row0) * p.G + g) * DK;
+            vb = p.v + (((size_t)b * p.T + row0) * p.G + g) * DV;
+        }
+        warp_issue_32rows<DK>(ks, kb, (size_t)p.G * DK, nval);
+        warp_issue_32rows<DV>(vs, vb, (size_t)p.G * DV, nval);
+        cp_async_commit();
         cp_async_wait();
         __syncwarp();
-    };
-    // does key `key` of the branch take part (inside the range, causal)?
-    auto seen = [&](int br, int lo, int nk, int key) -> bool {
-        if (key >= nk) return false;
-        return br != kBrSlc || token_of(br, lo, key) <= t;
+        return nval;
     };
 
     // ---------------- pass 1, every branch: LSE, o_c, dgates, D
@@ -142,7 +145,7 @@ __global__ void __launch_bounds__(128) bwd_query_mma(const BwdParams p) {
             for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
         for (int ch = warp; ch < nch; ch += 4) {
             const int k0 = ch * 32;
-            stage(br, lo, nk, k0);
+            const int nval = stage(br, lo, nk, k0);
             float sf[4][4];
             warp_logits<DK>(qa, smem_u32(ks), sf);
             float cm0 = -INFINITY, cm1 = -INFINITY;
@@ -150,7 +153,7 @@ __global__ void __launch_bounds__(128) bwd_query_mma(const BwdParams p) {
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float v = seen(br, lo, nk, k0 + nt * 8 + tg * 2 + (e & 1)) ? sf[nt][e] * c : -INFINITY;
+                    const float v = nt * 8 + tg * 2 + (e & 1) < nval ? sf[nt][e] * c : -INFINITY;
                     sf[nt][e] = v;
                     if (e < 2) cm0 = fmaxf(cm0, v);
                     else cm1 = fmaxf(cm1, v);
@@ -268,7 +271,7 @@ __global__ void __launch_bounds__(128) bwd_query_mma(const BwdParams p) {
         const float g0 = gs[br][gr], g1 = gs[br][gr + 8];
         for (int ch = warp; ch < nch; ch += 4) {
             const int k0 = ch * 32;
-            stage(br, lo, nk, k0);
+            const int nval = stage(br, lo, nk, k0);
             float sf[4][4], dp[4][4];
             warp_logits<DK>(qa, smem_u32(ks), sf);
             warp_logits_sa<DV>(smem_u32(dos), smem_u32(vs), dp);
@@ -278,7 +281,7 @@ __global__ void __launch_bounds__(128) bwd_query_mma(const BwdParams p) {
                 for (int e = 0; e < 4; ++e) {
                     const bool hi = e >= 2;
                     const float Lr = hi ? L1 : L0;
-                    const bool ok = seen(br, lo, nk, k0 + nt * 8 + tg * 2 + (e & 1)) && Lr != -INFINITY;
+                    const bool ok = nt * 8 + tg * 2 + (e & 1) < nval && Lr != -INFINITY;
                     const float P = ok ? exp2f(sf[nt][e] * c - Lr) : 0.f;
                     sf[nt][e] = P * ((hi ? g1 : g0) * dp[nt][e] - (hi ? D1 : D0));
                 }

@@ -296,6 +296,13 @@ __global__ void __launch_bounds__(320, 1)
             vis_hi = (t + 1 >= p.l) ? (t + 1 - p.l) / p.d + 1 : 0;
         }
         if (!row_ok) vis_hi = vis_lo = -1 << 30;
+        if (MODE == kModeWin && row_ok) {
+            // the epilogue adds into this row of out: start bringing it into L2 now,
+            // so its read does not wait on DRAM after the last key tile
+            const char* orow = reinterpret_cast<const char*>(p.out + rowid * DV);
+#pragma unroll
+            for (int q = 0; q < DV * 4; q += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(orow + q));
+        }
         // bounds shared by every row of this query tile (visibility grows with t)
         const int tile_first = t0 + tile * TOK;
         const int tile_last = min(tile_first + TOK, p.T) - 1;

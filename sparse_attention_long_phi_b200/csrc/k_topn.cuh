@@ -33,6 +33,8 @@ __device__ __forceinline__ int warp_sort_asc(int v, int lane) {
 
 // Top-n of one row of importance scores `row` (global or shared memory) for
 // query t, by one warp; writes n ascending indices (-1 padded) to `out`.
+// PL candidates per lane: rows of at most 32*PL scored candidates.
+template <int PL = kTopnPerLane>
 __device__ __forceinline__ void topn_row_warp(const float* row, int t, int n, int lp, int fi, int fl,
                                               int32_t* out, int lane) {
     const int bt = t / lp;
@@ -43,9 +45,9 @@ __device__ __forceinline__ void topn_row_warp(const float* row, int t, int n, in
     }
     const int lo = fi, hi = bt - fl;             // scored candidates lo..hi
     const int R = n - fi - fl;
-    float v[kTopnPerLane];
+    float v[PL];
 #pragma unroll
-    for (int k = 0; k < kTopnPerLane; ++k) {
+    for (int k = 0; k < PL; ++k) {
         const int j = lo + lane + 32 * k;
         v[k] = (j <= hi) ? row[j] : -1.f;        // scores are >= 0
     }
@@ -54,7 +56,7 @@ __device__ __forceinline__ void topn_row_warp(const float* row, int t, int n, in
         float bv = -2.f;
         int bk = 0;
 #pragma unroll
-        for (int k = 0; k < kTopnPerLane; ++k)
+        for (int k = 0; k < PL; ++k)
             if (v[k] > bv) {                     // strict: first (lowest j) wins ties
                 bv = v[k];
                 bk = k;
@@ -73,7 +75,7 @@ __device__ __forceinline__ void topn_row_warp(const float* row, int t, int n, in
         if (bj != 0x7fffffff && ((bj - lo) & 31) == lane) {
             const int kk = (bj - lo) >> 5;
 #pragma unroll
-            for (int k = 0; k < kTopnPerLane; ++k)
+            for (int k = 0; k < PL; ++k)
                 if (k == kk) v[k] = -1.f;
         }
         if (lane == it) mine = bj;
@@ -193,7 +195,8 @@ __device__ __forceinline__ void topn_row_cta(const float* row, int t, int n, int
     }
 }
 
-// one warp per (batch, token, group) item; scores [items, NSp]
+// one warp per (batch, token, group) item; scores [items, NSp]; NSp <= 32*PL
+template <int PL>
 __global__ void __launch_bounds__(256)
     topn_kernel(const float* __restrict__ pscore, long long items, int T, int G, int NSp, int n,
                 int lp, int fi, int fl, int32_t* __restrict__ idx) {
@@ -201,7 +204,7 @@ __global__ void __launch_bounds__(256)
     const long long item = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
     if (item >= items) return;
     const int t = (int)((item / G) % T);
-    topn_row_warp(pscore + item * NSp, t, n, lp, fi, fl, idx + item * n, lane);
+    topn_row_warp<PL>(pscore + item * NSp, t, n, lp, fi, fl, idx + item * n, lane);
 }
 
 }  // namespace nsa

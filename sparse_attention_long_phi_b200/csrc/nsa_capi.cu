@@ -392,9 +392,16 @@ nsa_status_t forward_impl(const Shape& s, const void* q, const void* k, const vo
     // 5. top-n selection
     {
         const long long items = s.B * s.T * s.G;
-        NSA_LAUNCH("topn_kernel", st, topn_kernel<<<(unsigned)ceil_div(items, 8), 256, 0, st>>>(pscore, items, (int)s.T, (int)s.G,
+        const unsigned grid = (unsigned)ceil_div(items, 8);
+        if (s.NSp <= 32 * 32) {   // rows of at most 1024 blocks: 32 candidates per lane
+            NSA_LAUNCH("topn_kernel", st, topn_kernel<32><<<grid, 256, 0, st>>>(pscore, items, (int)s.T, (int)s.G,
                                                                    (int)s.NSp, (int)s.n, (int)s.lp,
                                                                    (int)s.fi, (int)s.fl, sel_idx));
+        } else {
+            NSA_LAUNCH("topn_kernel", st, topn_kernel<kTopnPerLane><<<grid, 256, 0, st>>>(pscore, items, (int)s.T, (int)s.G,
+                                                                   (int)s.NSp, (int)s.n, (int)s.lp,
+                                                                   (int)s.fi, (int)s.fl, sel_idx));
+        }
         NSA_TRY(last_launch());
     }
     // 6. selected attention

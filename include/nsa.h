@@ -150,6 +150,7 @@ nsa_status_t nsa_forward(const nsa_config_t* cfg, const void* q, const void* k, 
  * cmp_offsets[s+1]), which must number nsa_num_cmp_blocks(cfg, L_s);
  * offsets are int64 device arrays of S+1 entries; gates [S,H,3] fp32.
  * Out: out [S,H,d_v] fp32, sel_idx [S,G,n] int32, lse [S,H,3] fp32 or NULL.
+ * At most 2048 sequences per call (NSA_ERR_UNSUPPORTED beyond).
  * num_seqs must not exceed cfg->batch and no L_s may exceed cfg->seqlen (the
  * workspace was sized from them): a longer context is skipped on the device
  * and reported as NSA_ERR_INVALID_ARG by nsa_sync_status().  A compressed

@@ -65,6 +65,7 @@ def test_forward_argument_validation_on_host(L):
     assert _fwd(L, dict(base, dk=128)) == 2                 # no kernel for d_k = 128
     assert _fwd(L, dict(base, lp=32, l=16)) == 2            # selection block != 64
     assert _fwd(L, dict(base, n=17)) == 2
+    assert _fwd(L, dict(base, T=131073)) == 2                # beyond the largest supported context
     assert _fwd(L, base, ws_bytes=1024) == 3                # workspace too small
 
 
@@ -77,6 +78,8 @@ def test_decode_and_backward_validation_on_host(L):
     assert lib.nsa_decode(ctypes.byref(cfg), 33, *args, 1 << 30, None) == 1   # more seqs than sized
     assert lib.nsa_decode(ctypes.byref(cfg), 8, *args, 16, None) == 3         # workspace too small
     assert lib.nsa_decode(ctypes.byref(cfg), 0, *args, 16, None) == 0         # nothing to do
+    big = L.make_config(dict(c, B=4096), batch=4096, seqlen=8192)
+    assert lib.nsa_decode(ctypes.byref(big), 3000, *args, 1 << 40, None) == 2  # > 2048 sequences per call
     cb = L.make_config(I.WORKLOADS["train_fwd_bwd_B2_T16384"])
     assert lib.nsa_backward(ctypes.byref(cb), fake, fake, fake, fake, None, fake, fake, fake, fake,
                             fake, fake, fake, 64, None) == 3

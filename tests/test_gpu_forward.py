@@ -71,3 +71,11 @@ def test_prefill_T65536_sampled_rows():
     c = wl("prefill_fwd_T65536")
     rows = sample_rows(1, c["T"], 48, seed=2, edge=32)
     check_forward(c, rows=rows)
+
+
+def test_prefill_largest_supported_context_sampled_rows():
+    # T = 131072, the largest context the library accepts (2048 selection blocks,
+    # 64 candidates per top-n lane); first/last tokens and random rows
+    c = wl("prefill_fwd_T65536", T=131072, seed=2131)
+    rows = sample_rows(1, c["T"], 16, seed=3, edge=8)
+    check_forward(c, rows=rows)

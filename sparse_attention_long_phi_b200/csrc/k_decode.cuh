@@ -204,6 +204,7 @@ __global__ void __launch_bounds__(256, 1) dec_cmp_stream(const DecParams p) {
         if (lane == 0) pre[p.S] = run;
     }
     __syncthreads();
+    dep_launch();
     if (blockIdx.x == 0)
         for (int s = threadIdx.x; s <= p.S; s += blockDim.x) p.cpre[s] = pre[s];
     const long long N = pre[p.S];
@@ -389,6 +390,7 @@ __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
     __shared__ float tsv[8 * 16];
     __shared__ int tsi[8 * 16];
     const int g = blockIdx.x, s = blockIdx.y;
+    dep_launch();
     int L, C;
     if (!dec_seq_ok(p, s, L, C)) {
         if (threadIdx.x == 0 && g == 0 && L > 0) atomicOr(&g_nsa_error, 4u);
@@ -397,6 +399,7 @@ __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
     const int t = L - 1;
     const int nch = (C + 31) / 32;
     const size_t sg = (size_t)s * p.G + g;
+    dep_wait();                                        // the compressed stream's records
     if (threadIdx.x == 0) {
         int cnt = 0;
         if (nch > 0) {
@@ -568,6 +571,8 @@ __global__ void __launch_bounds__(256, 1) dec_slcwin_stream(const DecParams p) {
     }
     fence_mbar_init();
     __syncthreads();
+    dep_launch();
+    dep_wait();                                       // sel_idx and o_cmp of the combine
     uint32_t kph = 0, vph = 0;
     const uint64_t pol = l2_evict_first();
     const long long U = (long long)p.S * p.G * p.NUV;     // unit slots, NUV per (seq, group)
@@ -719,6 +724,7 @@ __global__ void __launch_bounds__(256) dec_final(const DecParams p) {
     int L, C;
     if (!dec_seq_ok(p, s, L, C)) return;
     const size_t sg = (size_t)s * p.G + g;
+    dep_wait();                                       // the selected/window records
     if (threadIdx.x == 0) {
         const long long X0 = (long long)sg * p.NUV;
         nrec = dec_record_ctas(X0, X0 + p.NUV, (long long)p.S * p.G * p.NUV, p.grid3, recb, kDecMaxUnits);

@@ -112,6 +112,25 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel on the stream finishes; it reads that kernel's results
+// only after griddepcontrol.wait (dep_wait()).
+template <typename... KArgs, typename... Args>
+nsa_status_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? NSA_OK : NSA_ERR_CUDA;
+}
+
 struct Shape {
     int64_t B, T, H, G, DK, DV, HG, l, d, lp, n, fi, fl, w;
     int64_t C, Cp, Tp, DVP, NS, NSp;
@@ -605,13 +624,15 @@ nsa_status_t decode_launch(DecParams& p, const Shape& s, int S, cudaStream_t st)
     p.grid3 = std::min(kDecMaxGrid, nsm * std::max(1, occ3));
     NSA_LAUNCH("dec_cmp_stream", st, dec_cmp_stream<DK, DV><<<(unsigned)p.grid1, 256, smem, st>>>(p));
     NSA_TRY(last_launch());
+    // the three dependent kernels start while their predecessor drains
     const int smem2 = (kDecMaxChunks * 16 + p.NCH * 16 + p.NSmax) * 4;
     NSA_TRY(set_smem(dec_cmp_combine<DV>, smem2));
-    NSA_LAUNCH("dec_cmp_combine", st, dec_cmp_combine<DV><<<dim3((unsigned)s.G, (unsigned)S), 256, smem2, st>>>(p));
-    NSA_TRY(last_launch());
-    NSA_LAUNCH("dec_slcwin_stream", st, dec_slcwin_stream<DK, DV><<<(unsigned)p.grid3, 256, smem, st>>>(p));
-    NSA_TRY(last_launch());
-    NSA_LAUNCH("dec_final", st, dec_final<DV><<<dim3((unsigned)s.G, (unsigned)S), 256, 0, st>>>(p));
+    NSA_LAUNCH("dec_cmp_combine", st,
+               NSA_TRY(launch_dependent(dec_cmp_combine<DV>, dim3((unsigned)s.G, (unsigned)S), dim3(256), smem2, st, p)));
+    NSA_LAUNCH("dec_slcwin_stream", st,
+               NSA_TRY(launch_dependent(dec_slcwin_stream<DK, DV>, dim3((unsigned)p.grid3), dim3(256), smem, st, p)));
+    NSA_LAUNCH("dec_final", st,
+               NSA_TRY(launch_dependent(dec_final<DV>, dim3((unsigned)s.G, (unsigned)S), dim3(256), 0, st, p)));
     return last_launch();
 }
 

@@ -250,13 +250,14 @@ __global__ void __launch_bounds__(192, 1)
     }
 }
 
-// Exact recomputation of the listed elements: one warp per element, fp64
-// sum of W[o, x] * (x_blk[x] + E[x]) over the l*D inputs (8 per lane and
-// load), rounded once.
+// Exact recomputation of the listed elements: one warp per element, the fp64
+// bias W[o,:]·E (computed once by phi_bias_kernel) plus the fp64 sum of
+// W[o, x] * x_blk[x] over the l*D inputs (8 per lane and load); each bf16
+// product is exact in fp32, so one widening per product remains.  Rounded once.
 template <int D>
 __global__ void __launch_bounds__(256)
     phi_fixup_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ W,
-                     const __nv_bfloat16* __restrict__ E, int T, int G, int l, int d, int C, int Cp,
+                     const double* __restrict__ bias, int T, int G, int l, int d, int C, int Cp,
                      const uint32_t* __restrict__ fix_list, const unsigned int* __restrict__ fix_count,
                      __nv_bfloat16* __restrict__ y, __nv_bfloat16* __restrict__ yT) {
     const int lane = threadIdx.x & 31;
@@ -276,24 +277,20 @@ __global__ void __launch_bounds__(256)
             const int j = xx / D, c = xx % D;
             const uint4 xv = *reinterpret_cast<const uint4*>(
                 x + (((size_t)b * T + (size_t)i * d + j) * G + g) * D + c);
-            const uint4 ev = *reinterpret_cast<const uint4*>(E + xx);
             const uint4 wv = *reinterpret_cast<const uint4*>(wr + xx);
             const __nv_bfloat16* xh = reinterpret_cast<const __nv_bfloat16*>(&xv);
-            const __nv_bfloat16* eh = reinterpret_cast<const __nv_bfloat16*>(&ev);
             const __nv_bfloat16* wh = reinterpret_cast<const __nv_bfloat16*>(&wv);
 #pragma unroll
             for (int q = 0; q < 8; q += 2) {
-                acc0 += (double)__bfloat162float(wh[q]) *
-                        ((double)__bfloat162float(xh[q]) + (double)__bfloat162float(eh[q]));
-                acc1 += (double)__bfloat162float(wh[q + 1]) *
-                        ((double)__bfloat162float(xh[q + 1]) + (double)__bfloat162float(eh[q + 1]));
+                acc0 += (double)(__bfloat162float(wh[q]) * __bfloat162float(xh[q]));
+                acc1 += (double)(__bfloat162float(wh[q + 1]) * __bfloat162float(xh[q + 1]));
             }
         }
         double acc = acc0 + acc1;
 #pragma unroll
         for (int s2 = 16; s2 >= 1; s2 >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s2);
         if (lane == 0) {
-            const __nv_bfloat16 r = d2bf16_rn(acc);
+            const __nv_bfloat16 r = d2bf16_rn(acc + bias[o]);
             if (y) y[(((size_t)b * C + i) * G + g) * D + o] = r;
             if (yT) yT[(((size_t)b * G + g) * D + o) * Cp + i] = r;
         }

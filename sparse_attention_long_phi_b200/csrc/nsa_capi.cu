@@ -255,8 +255,8 @@ nsa_status_t launch_phi_linear(const Shape& s, const void* x, const void* W, con
         reinterpret_cast<__nv_bfloat16*>(y), reinterpret_cast<__nv_bfloat16*>(yT), fix_list, fix_count));
     NSA_TRY(last_launch());
     NSA_LAUNCH("phi_fixup_kernel", st, phi_fixup_kernel<D><<<148 * 4, 256, 0, st>>>(
-        reinterpret_cast<const __nv_bfloat16*>(x), reinterpret_cast<const __nv_bfloat16*>(W),
-        reinterpret_cast<const __nv_bfloat16*>(E), (int)s.T, (int)s.G, (int)s.l, (int)s.d, (int)s.C,
+        reinterpret_cast<const __nv_bfloat16*>(x), reinterpret_cast<const __nv_bfloat16*>(W), bias,
+        (int)s.T, (int)s.G, (int)s.l, (int)s.d, (int)s.C,
         (int)s.Cp, fix_list, fix_count, reinterpret_cast<__nv_bfloat16*>(y),
         reinterpret_cast<__nv_bfloat16*>(yT)));
     return last_launch();

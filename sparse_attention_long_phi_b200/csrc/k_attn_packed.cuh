@@ -50,14 +50,16 @@ struct PackedParams {
 template <int DK, int DV, int HG, int MODE>
 struct PackedCfg {
     static constexpr int TOK = 128 / HG;              // tokens per query tile
-    static constexpr int BN = 64;
+    // keys per tile: 128 in the LSE pass (S only in TMEM, and an N = 128 product
+    // reads Q from shared memory once per 128 keys), 64 where O also lives in TMEM
+    static constexpr int BN = MODE == kModeLse ? 128 : 64;
     static constexpr int NQB = DK / 64;
     static constexpr int kQBytes = 128 * DK * 2;      // one tile
-    static constexpr int kKBox = BN * 128;            // 64 rows x 128 B
+    static constexpr int kKBox = BN * 128;            // BN rows x 128 B
     static constexpr int kKBytes = NQB * kKBox;
     static constexpr int kVBytes = DV * 128;          // DV rows x 64 keys
     static constexpr int kPBytes = 128 * 128;         // 128 rows x 64 keys
-    static constexpr int NSK = MODE == kModeLse ? 3 : 2;
+    static constexpr int NSK = 2;
     static constexpr int NSV = MODE == kModeLse ? 0 : 2;
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + 2 * kQBytes;
@@ -65,8 +67,9 @@ struct PackedCfg {
     static constexpr int kOffP = kOffV + NSV * kVBytes;
     static constexpr int kOffBar = kOffP + (MODE == kModeLse ? 0 : 2 * kPBytes);
     static constexpr int kSmem = kOffBar + 256 + 1024;
-    // TMEM: S tile A [0,128) (2 buffers of 64), S tile B [128,256), O_A, O_B
-    static constexpr uint32_t kTmemCols = (MODE == kModeLse) ? 256 : 512;
+    static_assert(kSmem <= 232448, "shared memory");
+    // TMEM: S tile A [0, 2BN) (2 buffers of BN), S tile B [2BN, 4BN), then O_A, O_B
+    static constexpr uint32_t kTmemCols = 512;
     static constexpr int kThreads = 320;
 };
 
@@ -159,7 +162,7 @@ __global__ void __launch_bounds__(320, 1)
     } else {
         const int kend = (t_last + 1 >= p.l) ? (t_last + 1 - p.l) / p.d + 1 : 0;
         key0 = 0;
-        ntiles = (kend + 63) / 64;
+        ntiles = (kend + Cfg::BN - 1) / Cfg::BN;
     }
 
     if (threadIdx.x == 0) {
@@ -204,7 +207,7 @@ __global__ void __launch_bounds__(320, 1)
                     tma_load_4d(smem + Cfg::kOffQ + tile * Cfg::kQBytes + bx * 16384, &mapQ, qfull,
                                 bx * 64, g * HG, t0 + tile * TOK, b);
             for (int jt = 0; jt < ntiles; ++jt) {
-                const int kb = key0 + jt * 64;
+                const int kb = key0 + jt * Cfg::BN;
                 const int s = jt % NSK;
                 if (jt >= NSK && !wait_or_abort(&kempty[s], ((jt / NSK) - 1) & 1, 0x201, abort_flag))
                     break;
@@ -212,7 +215,9 @@ __global__ void __launch_bounds__(320, 1)
                 mbar_expect_tx(&kfull[s], Cfg::kKBytes);
 #pragma unroll
                 for (int bx = 0; bx < Cfg::NQB; ++bx)
-                    tma_load_4d(ks + bx * Cfg::kKBox, &mapK, &kfull[s], bx * 64, g, kb, b);
+#pragma unroll
+                    for (int hb = 0; hb < Cfg::BN / 64; ++hb)   // boxes of 64 rows
+                        tma_load_4d(ks + bx * Cfg::kKBox + hb * 8192, &mapK, &kfull[s], bx * 64, g, kb + hb * 64, b);
                 if (MODE != kModeLse) {
                     const int sv = jt % NSV;
                     if (jt >= NSV && !wait_or_abort(&vempty[sv], ((jt / NSV) - 1) & 1, 0x202, abort_flag))
@@ -226,7 +231,7 @@ __global__ void __launch_bounds__(320, 1)
     } else if (warp == 9) {
         // ----------------------------------------------------------- MMA
         if (lane == 0 && ntiles > 0) {
-            constexpr uint32_t idS = idesc_bf16(128, 64);
+            constexpr uint32_t idS = idesc_bf16(128, Cfg::BN);
             constexpr uint32_t idO = idesc_bf16(128, DV);
             bool ok = wait_or_abort(qfull, 0, 0x203, abort_flag);
             auto issue_S = [&](int jt) -> bool {
@@ -242,7 +247,7 @@ __global__ void __launch_bounds__(320, 1)
                     const uint32_t sQ = smem_u32(smem + Cfg::kOffQ + tile * Cfg::kQBytes);
 #pragma unroll
                     for (int kk = 0; kk < DK / 16; ++kk)
-                        umma_bf16_ss(tmem + tile * 128 + buf * 64,
+                        umma_bf16_ss(tmem + tile * 2 * Cfg::BN + buf * Cfg::BN,
                                      sdesc_sw128(sQ + (kk / 4) * 16384 + (kk % 4) * 32),
                                      sdesc_sw128(sK + (kk / 4) * Cfg::kKBox + (kk % 4) * 32), idS,
                                      kk > 0 ? 1u : 0u);
@@ -286,7 +291,7 @@ __global__ void __launch_bounds__(320, 1)
         const bool row_ok = t < p.T;
         const size_t rowid = ((size_t)b * p.T + (row_ok ? t : 0)) * p.H + h;
         const uint32_t lanebase = tmem + ((uint32_t)(wq * 32) << 16);
-        const uint32_t sbase = lanebase + tile * 128;         // S buffers of this tile
+        const uint32_t sbase = lanebase + tile * 2 * Cfg::BN; // S buffers of this tile
         const uint32_t obase = lanebase + 256 + tile * DV;    // O of this tile
         int vis_hi, vis_lo = 0;
         if (MODE == kModeWin) {
@@ -318,7 +323,53 @@ __global__ void __launch_bounds__(320, 1)
         for (int c = 0; c < (NC > 0 ? NC : 1); ++c) carry[c] = 0.f;
         bool ok = true;
 
-        for (int jt = 0; jt < ntiles; ++jt) {
+        if (MODE == kModeLse) {
+            // BN = 128 keys per tile, read from TMEM in two halves of 64
+            for (int jt = 0; jt < ntiles; ++jt) {
+                const int buf = jt & 1;
+                if (ok) ok = wait_or_abort(&sfull[2 * tile + buf], (jt >> 1) & 1, 0x208, abort_flag);
+                tc_fence_after();
+#pragma unroll 1
+                for (int hb = 0; hb < Cfg::BN / 64; ++hb) {
+                    const int kb = key0 + jt * Cfg::BN + hb * 64;
+                    uint32_t ra[32], rb[32];
+                    tmem_ld32(sbase + buf * Cfg::BN + hb * 64, ra);
+                    tmem_ld32(sbase + buf * Cfg::BN + hb * 64 + 32, rb);
+                    tmem_wait_ld32(ra);
+                    tmem_wait_ld32(rb);
+                    float s[64];
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        s[k] = __uint_as_float(ra[k]);
+                        s[k + 32] = __uint_as_float(rb[k]);
+                    }
+                    if (!(kb + 64 <= vis_first)) {
+#pragma unroll
+                        for (int k = 0; k < 64; ++k)
+                            if (!(kb + k >= vis_lo && kb + k < vis_hi)) s[k] = -INFINITY;
+                    }
+                    const float c = p.scale_log2;
+                    float mr = -INFINITY;
+#pragma unroll
+                    for (int k = 0; k < 64; ++k) mr = fmaxf(mr, s[k]);
+                    const float mn = fmaxf(m_run, mr * c);
+                    if (mn != -INFINITY) {
+                        float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+                        for (int k = 0; k < 64; k += 2) {
+                            acc0 += ex2a(fmaf(s[k], c, -mn));
+                            acc1 += ex2a(fmaf(s[k + 1], c, -mn));
+                        }
+                        l_run = l_run * ex2a(m_run - mn) + (acc0 + acc1);
+                        m_run = mn;
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sfree[2 * tile + buf]);
+            }
+        }
+        for (int jt = 0; MODE != kModeLse && jt < ntiles; ++jt) {
             const int buf = jt & 1;
             const int kb = key0 + jt * 64;
             if (ok) ok = wait_or_abort(&sfull[2 * tile + buf], (jt >> 1) & 1, 0x208, abort_flag);
@@ -349,23 +400,6 @@ __global__ void __launch_bounds__(320, 1)
                 }
             }
             const float c = p.scale_log2;
-            if (MODE == kModeLse) {
-                float mr = -INFINITY;
-#pragma unroll
-                for (int k = 0; k < 64; ++k) mr = fmaxf(mr, s[k]);
-                const float mn = fmaxf(m_run, mr * c);
-                if (mn != -INFINITY) {
-                    float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-                    for (int k = 0; k < 64; k += 2) {
-                        acc0 += ex2a(fmaf(s[k], c, -mn));
-                        acc1 += ex2a(fmaf(s[k + 1], c, -mn));
-                    }
-                    l_run = l_run * ex2a(m_run - mn) + (acc0 + acc1);
-                    m_run = mn;
-                }
-                continue;
-            }
             float pr[64];
             float alpha = 1.f;
             bool need_rescale = false;

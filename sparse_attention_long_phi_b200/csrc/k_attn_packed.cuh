@@ -22,7 +22,10 @@
 // 4-7 those of tile B (thread = query row), warp 8 is the TMA producer and
 // warp 9 the MMA issuer and TMEM owner.  Key tiles of 64 keys:
 //   S_x = Q_x K^T (M=128, N=64, K=DK) into one of two TMEM buffers per tile,
-//   O_x += P_x V  (M=128, N=DV, K=64) with P_x staged bf16 in shared memory.
+//   O_x += P_x V  (M=128, N=DV, K=64) with P_x written as bf16 over the S
+//   columns it came from and read by the MMA from tensor memory (no shared-
+//   memory round trip for P); S(j+2) is issued into a buffer only once the
+//   P.V product that read P(j) from it has completed.
 // The MMA order S_A(j+1) S_B(j+1) PV_A(j) PV_B(j) lets each tile's softmax
 // overlap the other tile's products.  The softmax is issue-bound, so it is
 // kept to about one FFMA + one MUFU + one add per logit, and the causal /
@@ -65,7 +68,7 @@ struct PackedCfg {
     static constexpr int kOffK = kOffQ + 2 * kQBytes;
     static constexpr int kOffV = kOffK + NSK * kKBytes;
     static constexpr int kOffP = kOffV + NSV * kVBytes;
-    static constexpr int kOffBar = kOffP + (MODE == kModeLse ? 0 : 2 * kPBytes);
+    static constexpr int kOffBar = kOffP;             // P lives in tensor memory
     static constexpr int kSmem = kOffBar + 256 + 1024;
     static_assert(kSmem <= 232448, "shared memory");
     // TMEM: S tile A [0, 2BN) (2 buffers of BN), S tile B [2BN, 4BN), then O_A, O_B
@@ -240,8 +243,14 @@ __global__ void __launch_bounds__(320, 1)
                 const uint32_t sK = smem_u32(smem + Cfg::kOffK + s * Cfg::kKBytes);
 #pragma unroll
                 for (int tile = 0; tile < 2; ++tile) {
-                    if (jt >= 2 &&
+                    if (MODE == kModeLse && jt >= 2 &&
                         !wait_or_abort(&sfree[2 * tile + buf], ((jt - 2) >> 1) & 1, 0x205, abort_flag))
+                        return false;
+                    // the buffer's P(jt-2) must have been read by its P.V product: an MMA
+                    // writing tensor memory is not ordered behind an earlier MMA that
+                    // reads the same columns as its A operand
+                    if (MODE != kModeLse && jt >= 2 &&
+                        !wait_or_abort(&pvdone[tile], (jt - 2) & 1, 0x20B, abort_flag))
                         return false;
                     tc_fence_after();
                     const uint32_t sQ = smem_u32(smem + Cfg::kOffQ + tile * Cfg::kQBytes);
@@ -264,11 +273,11 @@ __global__ void __launch_bounds__(320, 1)
                 for (int tile = 0; tile < 2; ++tile) {
                     if (!wait_or_abort(&pfull[tile], jt & 1, 0x206, abort_flag)) return false;
                     tc_fence_after();
-                    const uint32_t sP = smem_u32(smem + Cfg::kOffP + tile * Cfg::kPBytes);
+                    const uint32_t tP = tmem + tile * 128 + (jt & 1) * 64;    // P over S(jt)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16_ss(tmem + 256 + tile * DV, sdesc_sw128(sP + kk * 32),
-                                     sdesc_sw128(sV + kk * 32), idO, (jt > 0 || kk > 0) ? 1u : 0u);
+                        umma_bf16_ts(tmem + 256 + tile * DV, tP + kk * 8, sdesc_sw128(sV + kk * 32), idO,
+                                     (jt > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&pvdone[tile]);
                 }
                 umma_commit(&vempty[sv]);
@@ -379,9 +388,6 @@ __global__ void __launch_bounds__(320, 1)
             tmem_ld32(sbase + buf * 64 + 32, rb);
             tmem_wait_ld32(ra);
             tmem_wait_ld32(rb);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sfree[2 * tile + buf]);
             float s[64];
 #pragma unroll
             for (int k = 0; k < 32; ++k) {
@@ -456,7 +462,9 @@ __global__ void __launch_bounds__(320, 1)
                         if (j0 + base + v < p.NSp) dst[j0 + base + v] = red[v];
                 }
             }
-            // P -> shared memory (after the previous P.V of this tile has consumed it)
+            // the previous P.V of this tile finished: the window's O rescale needs it,
+            // and it keeps this loop at most one pvdone phase ahead of the MMA warp
+            // (a parity wait cannot tell phases two apart; the epilogue relies on it)
             if (jt > 0 && ok) ok = wait_or_abort(&pvdone[tile], (jt - 1) & 1, 0x209, abort_flag);
             tc_fence_after();
             if (MODE == kModeWin && jt > 0 && __any_sync(0xffffffffu, need_rescale)) {
@@ -472,14 +480,15 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 tmem_wait_st();
             }
-            const uint32_t sP = smem_u32(smem + Cfg::kOffP + tile * Cfg::kPBytes);
+            // P (bf16, two per column) over the first 32 columns of S(jt): the A
+            // operand of this tile's P.V product
+            {
+                uint32_t pk[32];
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-                st_shared_v4(sP + sw128_off(r, c), pack_bf16x2(pr[8 * c + 0], pr[8 * c + 1]),
-                             pack_bf16x2(pr[8 * c + 2], pr[8 * c + 3]),
-                             pack_bf16x2(pr[8 * c + 4], pr[8 * c + 5]),
-                             pack_bf16x2(pr[8 * c + 6], pr[8 * c + 7]));
-            fence_proxy_async_smem();
+                for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pr[2 * c], pr[2 * c + 1]);
+                tmem_st32(sbase + buf * 64, pk);
+                tmem_wait_st();
+            }
             tc_fence_before();
             mbar_arrive(&pfull[tile]);
         }

@@ -13,7 +13,7 @@ buffers, the clocks seen during the timed region, the number of kernel
 launches, the CPU baseline (the fp64 oracle on a bounded sample) and the
 decode and backward measurements of their own workloads.
 
---impl reference times the oracle (the reference of this build) on host cores
+--impl reference times the fp64 CPU oracle (the reference arm) on host cores
 with the same metric, each step a bounded sample extrapolated to a full step.
 """
 from __future__ import annotations

@@ -34,9 +34,23 @@ __device__ __forceinline__ int warp_sort_asc(int v, int lane) {
 // Top-n of one row of importance scores `row` (global or shared memory) for
 // query t, by one warp; writes n ascending indices (-1 padded) to `out`.
 // PL candidates per lane: rows of at most 32*PL scored candidates.
+//
+// Candidate j sits in lane (j - lo) % 32, slot (j - lo) / 32.  Scores are
+// mapped to keys that order like the scores (+0 and -0 equal; a negative
+// score, the padding, or a NaN maps to 0 and is never taken).  Each lane keeps
+// its two best untaken candidates (ties: lower slot = lower j first); a round
+// takes the warp's largest head key (__reduce_max_sync) and, among the lanes
+// holding it, the lowest j (__reduce_min_sync): the highest score, ties to the
+// lower block index.  The winning lane pops its head and rescans its slots
+// when both cached entries are used up.
+__device__ __forceinline__ uint32_t topn_key(float x) {
+    return x > 0.f ? __float_as_uint(x) + 1u : (x == 0.f ? 1u : 0u);
+}
+
 template <int PL = kTopnPerLane>
 __device__ __forceinline__ void topn_row_warp(const float* row, int t, int n, int lp, int fi, int fl,
                                               int32_t* out, int lane) {
+    static_assert(PL <= 64, "taken mask is 64 bits");
     const int bt = t / lp;
     const int ncand = bt + 1;
     if (ncand <= n) {
@@ -45,40 +59,42 @@ __device__ __forceinline__ void topn_row_warp(const float* row, int t, int n, in
     }
     const int lo = fi, hi = bt - fl;             // scored candidates lo..hi
     const int R = n - fi - fl;
-    float v[PL];
+    uint32_t key[PL];
 #pragma unroll
     for (int k = 0; k < PL; ++k) {
         const int j = lo + lane + 32 * k;
-        v[k] = (j <= hi) ? row[j] : -1.f;        // scores are >= 0
+        key[k] = (j <= hi) ? topn_key(row[j]) : 0u;
     }
+    uint64_t taken = 0;
+    uint32_t c0 = 0, c1 = 0;                     // cached keys, c0 >= c1
+    int s0 = 0, s1 = 0;                          // their slots
+    auto rescan = [&]() {
+        c0 = c1 = 0;
+#pragma unroll
+        for (int k = 0; k < PL; ++k) {
+            const uint32_t kk = ((taken >> k) & 1ull) ? 0u : key[k];
+            const bool g0 = kk > c0, g1 = kk > c1;   // strict: the lower slot stays ahead
+            c1 = g0 ? c0 : (g1 ? kk : c1);
+            s1 = g0 ? s0 : (g1 ? k : s1);
+            c0 = g0 ? kk : c0;
+            s0 = g0 ? k : s0;
+        }
+    };
+    rescan();
     int mine = 0x7fffffff;
     for (int it = 0; it < R; ++it) {
-        float bv = -2.f;
-        int bk = 0;
-#pragma unroll
-        for (int k = 0; k < PL; ++k)
-            if (v[k] > bv) {                     // strict: first (lowest j) wins ties
-                bv = v[k];
-                bk = k;
-            }
-        int bj = lo + lane + 32 * bk;
-        if (bv < -0.5f) bj = 0x7fffffff;
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) {
-            float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            int oj = __shfl_xor_sync(0xffffffffu, bj, o);
-            if (ov > bv || (ov == bv && oj < bj)) {
-                bv = ov;
-                bj = oj;
-            }
+        const uint32_t mx = __reduce_max_sync(0xffffffffu, c0);
+        if (mx == 0u) break;                     // warp-uniform: nothing left to take
+        const uint32_t mj = (c0 == mx) ? (uint32_t)(lo + lane + 32 * s0) : 0xffffffffu;
+        const uint32_t bj = __reduce_min_sync(0xffffffffu, mj);
+        if (mj == bj) {                          // this lane holds the winner
+            taken |= 1ull << s0;
+            c0 = c1;
+            s0 = s1;
+            c1 = 0;
+            if (c0 == 0u) rescan();
         }
-        if (bj != 0x7fffffff && ((bj - lo) & 31) == lane) {
-            const int kk = (bj - lo) >> 5;
-#pragma unroll
-            for (int k = 0; k < PL; ++k)
-                if (k == kk) v[k] = -1.f;
-        }
-        if (lane == it) mine = bj;
+        if (lane == it) mine = (int)bj;
     }
     // lanes R .. R+fi+fl-1 carry the forced blocks
     if (lane >= R && lane < R + fi) mine = lane - R;

@@ -175,6 +175,23 @@ nsa_status_t nsa_backward(const nsa_config_t* cfg, const void* q, const void* k,
                           const int32_t* sel_idx, float* dq, float* dk, float* dv, float* dgates,
                           void* workspace, size_t workspace_bytes, void* stream);
 
+/* Top-n block selection alone (page 2, Top-n 块选择; its hyperparameter
+ * paragraph fixes 1 initial and 2 local blocks as always selected), the step
+ * nsa_forward takes between the compressed and the selected branch.
+ * In:  scores [B,T,G,NS] fp32, NS = ceil(T / sel_block): importance score of
+ *      selection block j for query token t and GQA group g.  Only blocks
+ *      0 .. floor(t / sel_block) of row t are read.  Scores are >= 0; a
+ *      negative or NaN score is never selected (the slot stays -1).
+ * Out: sel_idx [B,T,G,n] int32, ascending, -1 padded: all blocks when at most
+ *      n exist; otherwise blocks 0 .. forced_initial-1, the forced_local
+ *      blocks ending at floor(t / sel_block), and the n - forced_initial -
+ *      forced_local highest scores among the remaining blocks, ties to the
+ *      lower block index (decided on the fp32 values).
+ * Needs no workspace.  NSA_ERR_UNSUPPORTED when sel_count > 32 or NS > 2048;
+ * the head dimensions and compression sizes of cfg are not used. */
+nsa_status_t nsa_select_blocks(const nsa_config_t* cfg, const float* scores, int32_t* sel_idx,
+                               void* stream);
+
 /* Synchronise `stream`, then read and clear the device error word of the
  * current device.  Returns NSA_ERR_DEVICE_TIMEOUT if a kernel's bounded wait
  * expired since the last call, NSA_ERR_CUDA if synchronisation failed. */

@@ -31,6 +31,23 @@ __device__ __forceinline__ int warp_sort_asc(int v, int lane) {
     return v;
 }
 
+// bitonic sort of one value per lane across the warp, descending by lane
+template <typename U>
+__device__ __forceinline__ U warp_sort_desc(U v, int lane) {
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const U o = __shfl_xor_sync(0xffffffffu, v, j);
+            const bool up = ((lane & k) == 0);
+            const bool lower = ((lane & j) == 0);
+            const U mn = v < o ? v : o, mx = v < o ? o : v;
+            v = (lower == up) ? mx : mn;
+        }
+    }
+    return v;
+}
+
 // Top-n of one row of importance scores `row` (global or shared memory) for
 // query t, by one warp; writes n ascending indices (-1 padded) to `out`.
 // PL candidates per lane: rows of at most 32*PL scored candidates.
@@ -43,13 +60,20 @@ __device__ __forceinline__ int warp_sort_asc(int v, int lane) {
 // holding it, the lowest j (__reduce_min_sync): the highest score, ties to the
 // lower block index.  The winning lane pops its head and rescans its slots
 // when both cached entries are used up.
+//
+// Most rows skip those rounds: with theta the R-th largest of the 32 lane
+// maxima, at least R candidates have key >= theta, so every winner does.  When
+// at most 32 candidates reach theta they are gathered into `wbuf` (32 slots of
+// this warp) as (key, ~j) and one descending warp sort leaves the winners, in
+// order, in lanes 0..R-1.  The rounds above are the fallback for rows with
+// more (ties at theta) or with theta = 0.
 __device__ __forceinline__ uint32_t topn_key(float x) {
     return x > 0.f ? __float_as_uint(x) + 1u : (x == 0.f ? 1u : 0u);
 }
 
 template <int PL = kTopnPerLane>
 __device__ __forceinline__ void topn_row_warp(const float* row, int t, int n, int lp, int fi, int fl,
-                                              int32_t* out, int lane) {
+                                              int32_t* out, int lane, unsigned long long* wbuf) {
     static_assert(PL <= 64, "taken mask is 64 bits");
     const int bt = t / lp;
     const int ncand = bt + 1;
@@ -60,41 +84,72 @@ __device__ __forceinline__ void topn_row_warp(const float* row, int t, int n, in
     const int lo = fi, hi = bt - fl;             // scored candidates lo..hi
     const int R = n - fi - fl;
     uint32_t key[PL];
+    uint32_t lmax = 0;
 #pragma unroll
     for (int k = 0; k < PL; ++k) {
         const int j = lo + lane + 32 * k;
         key[k] = (j <= hi) ? topn_key(row[j]) : 0u;
+        lmax = max(lmax, key[k]);
     }
-    uint64_t taken = 0;
-    uint32_t c0 = 0, c1 = 0;                     // cached keys, c0 >= c1
-    int s0 = 0, s1 = 0;                          // their slots
-    auto rescan = [&]() {
-        c0 = c1 = 0;
-#pragma unroll
-        for (int k = 0; k < PL; ++k) {
-            const uint32_t kk = ((taken >> k) & 1ull) ? 0u : key[k];
-            const bool g0 = kk > c0, g1 = kk > c1;   // strict: the lower slot stays ahead
-            c1 = g0 ? c0 : (g1 ? kk : c1);
-            s1 = g0 ? s0 : (g1 ? k : s1);
-            c0 = g0 ? kk : c0;
-            s0 = g0 ? k : s0;
-        }
-    };
-    rescan();
     int mine = 0x7fffffff;
-    for (int it = 0; it < R; ++it) {
-        const uint32_t mx = __reduce_max_sync(0xffffffffu, c0);
-        if (mx == 0u) break;                     // warp-uniform: nothing left to take
-        const uint32_t mj = (c0 == mx) ? (uint32_t)(lo + lane + 32 * s0) : 0xffffffffu;
-        const uint32_t bj = __reduce_min_sync(0xffffffffu, mj);
-        if (mj == bj) {                          // this lane holds the winner
-            taken |= 1ull << s0;
-            c0 = c1;
-            s0 = s1;
-            c1 = 0;
-            if (c0 == 0u) rescan();
+    bool done = R <= 0;                          // only forced blocks
+    const uint32_t theta = done ? 0u : __shfl_sync(0xffffffffu, warp_sort_desc(lmax, lane), R - 1);
+    if (theta > 0u) {
+        int cnt = 0;
+#pragma unroll
+        for (int k = 0; k < PL; ++k) cnt += key[k] >= theta;
+        const int total = (int)__reduce_add_sync(0xffffffffu, (unsigned)cnt);
+        if (total <= 32) {
+            int pos = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, pos, o);
+                if (lane >= o) pos += y;
+            }
+            pos -= cnt;                            // exclusive prefix
+#pragma unroll
+            for (int k = 0; k < PL; ++k)
+                if (key[k] >= theta)
+                    wbuf[pos++] = ((unsigned long long)key[k] << 32) | (uint32_t)~(uint32_t)(lo + lane + 32 * k);
+            __syncwarp();
+            unsigned long long c = lane < total ? wbuf[lane] : 0ull;
+            __syncwarp();                          // wbuf is free for the warp's next row
+            c = warp_sort_desc(c, lane);
+            if (lane < R) mine = (int)~(uint32_t)c;
+            done = true;
         }
-        if (lane == it) mine = (int)bj;
+    }
+    if (!done) {
+        uint64_t taken = 0;
+        uint32_t c0 = 0, c1 = 0;                     // cached keys, c0 >= c1
+        int s0 = 0, s1 = 0;                          // their slots
+        auto rescan = [&]() {
+            c0 = c1 = 0;
+#pragma unroll
+            for (int k = 0; k < PL; ++k) {
+                const uint32_t kk = ((taken >> k) & 1ull) ? 0u : key[k];
+                const bool g0 = kk > c0, g1 = kk > c1;   // strict: the lower slot stays ahead
+                c1 = g0 ? c0 : (g1 ? kk : c1);
+                s1 = g0 ? s0 : (g1 ? k : s1);
+                c0 = g0 ? kk : c0;
+                s0 = g0 ? k : s0;
+            }
+        };
+        rescan();
+        for (int it = 0; it < R; ++it) {
+            const uint32_t mx = __reduce_max_sync(0xffffffffu, c0);
+            if (mx == 0u) break;                     // warp-uniform: nothing left to take
+            const uint32_t mj = (c0 == mx) ? (uint32_t)(lo + lane + 32 * s0) : 0xffffffffu;
+            const uint32_t bj = __reduce_min_sync(0xffffffffu, mj);
+            if (mj == bj) {                          // this lane holds the winner
+                taken |= 1ull << s0;
+                c0 = c1;
+                s0 = s1;
+                c1 = 0;
+                if (c0 == 0u) rescan();
+            }
+            if (lane == it) mine = (int)bj;
+        }
     }
     // lanes R .. R+fi+fl-1 carry the forced blocks
     if (lane >= R && lane < R + fi) mine = lane - R;
@@ -216,11 +271,12 @@ template <int PL>
 __global__ void __launch_bounds__(256)
     topn_kernel(const float* __restrict__ pscore, long long items, int T, int G, int NSp, int n,
                 int lp, int fi, int fl, int32_t* __restrict__ idx) {
+    __shared__ unsigned long long wbuf[8][32];
     const int lane = threadIdx.x & 31;
     const long long item = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
     if (item >= items) return;
     const int t = (int)((item / G) % T);
-    topn_row_warp<PL>(pscore + item * NSp, t, n, lp, fi, fl, idx + item * n, lane);
+    topn_row_warp<PL>(pscore + item * NSp, t, n, lp, fi, fl, idx + item * n, lane, wbuf[threadIdx.x >> 5]);
 }
 
 }  // namespace nsa

@@ -764,6 +764,27 @@ nsa_status_t nsa_forward(const nsa_config_t* cfg, const void* q, const void* k, 
     return forward_impl<64, 64, 4>(s, q, k, v, gates, phi, out, sel_idx, lse, kc_out, vc_out, ws, st);
 }
 
+nsa_status_t nsa_select_blocks(const nsa_config_t* cfg, const float* scores, int32_t* sel_idx,
+                               void* stream) {
+    Shape s;
+    NSA_TRY(derive(cfg, s));
+    if (!scores || !sel_idx) return NSA_ERR_INVALID_ARG;
+    if (s.n > 32 || s.NS > 64 * 32) return NSA_ERR_UNSUPPORTED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const long long items = s.B * s.T * s.G;
+    const unsigned grid = (unsigned)ceil_div(items, 8);
+    if (s.NS <= 32 * 32) {
+        NSA_LAUNCH("topn_kernel", st, topn_kernel<32><<<grid, 256, 0, st>>>(scores, items, (int)s.T, (int)s.G,
+                                                               (int)s.NS, (int)s.n, (int)s.lp,
+                                                               (int)s.fi, (int)s.fl, sel_idx));
+    } else {
+        NSA_LAUNCH("topn_kernel", st, topn_kernel<kTopnPerLane><<<grid, 256, 0, st>>>(scores, items, (int)s.T, (int)s.G,
+                                                               (int)s.NS, (int)s.n, (int)s.lp,
+                                                               (int)s.fi, (int)s.fl, sel_idx));
+    }
+    return last_launch();
+}
+
 nsa_status_t nsa_decode(const nsa_config_t* cfg, int32_t num_seqs, const void* q,
                         const void* k_cache, const void* v_cache, const int64_t* kv_offsets,
                         const void* kc_cache, const void* vc_cache, const int64_t* cmp_offsets,

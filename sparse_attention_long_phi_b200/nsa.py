@@ -65,6 +65,8 @@ def lib():
         L.nsa_compress.argtypes = [pc, _P, _P, pp, _P, _P, _P, ctypes.c_size_t, _P]
         L.nsa_forward.restype = ctypes.c_int
         L.nsa_forward.argtypes = [pc, _P, _P, _P, _P, pp, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+        L.nsa_select_blocks.restype = ctypes.c_int
+        L.nsa_select_blocks.argtypes = [pc, _P, _P, _P]
         L.nsa_decode.restype = ctypes.c_int
         L.nsa_decode.argtypes = [pc, ctypes.c_int32] + [_P] * 12 + [ctypes.c_size_t, _P]
         L.nsa_backward.restype = ctypes.c_int
@@ -179,6 +181,18 @@ def compress(c: dict, k, v, phi=None, stream=None):
     _check("nsa_compress", lib().nsa_compress(ctypes.byref(make_config(c)), _p(k), _p(v), _phi(phi),
                                               _p(kc), _p(vc), _p(ws), ws.numel(), _stream(stream)))
     return kc[:, :C], vc[:, :C]
+
+
+def select_blocks(c: dict, scores, stream=None) -> torch.Tensor:
+    """Top-n block selection alone.  scores [B,T,G,NS] fp32 (NS = ceil(T / l')) ->
+    sel_idx [B,T,G,n] int32, ascending, -1 padded."""
+    B, T, G = c["B"], c["T"], c["G"]
+    assert scores.dtype == torch.float32 and scores.is_cuda
+    assert tuple(scores.shape) == (B, T, G, -(-T // c["lp"])), "scores must be [B,T,G,ceil(T/l')]"
+    idx = torch.empty(B, T, G, c["n"], dtype=torch.int32, device=scores.device)
+    _check("nsa_select_blocks", lib().nsa_select_blocks(ctypes.byref(make_config(c)), _p(scores), _p(idx),
+                                                        _stream(stream)))
+    return idx
 
 
 @dataclass

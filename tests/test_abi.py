@@ -69,6 +69,18 @@ def test_forward_argument_validation_on_host(L):
     assert _fwd(L, base, ws_bytes=1024) == 3                # workspace too small
 
 
+def test_select_blocks_validation_on_host(L):
+    lib = L.lib()
+    fake = ctypes.c_void_p(1 << 20)
+    base = dict(I.WORKLOADS["prefill_fwd_T8192"])
+    cfg = L.make_config(base)
+    assert lib.nsa_select_blocks(ctypes.byref(cfg), None, fake, None) == 1       # null scores
+    assert lib.nsa_select_blocks(ctypes.byref(cfg), fake, None, None) == 1       # null output
+    assert lib.nsa_select_blocks(ctypes.byref(L.make_config(dict(base, n=2))), fake, fake, None) == 1
+    assert lib.nsa_select_blocks(ctypes.byref(L.make_config(dict(base, n=33))), fake, fake, None) == 2
+    assert lib.nsa_select_blocks(ctypes.byref(L.make_config(dict(base, T=131073))), fake, fake, None) == 2
+
+
 def test_decode_and_backward_validation_on_host(L):
     lib = L.lib()
     c = dict(I.WORKLOADS["decode_S32_L8k_64k"], B=32, T=65536)

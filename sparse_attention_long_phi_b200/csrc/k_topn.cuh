@@ -83,12 +83,18 @@ __device__ __forceinline__ void topn_row_warp(const float* row, int t, int n, in
     }
     const int lo = fi, hi = bt - fl;             // scored candidates lo..hi
     const int R = n - fi - fl;
+    // every lane loads all its slots from in-bounds addresses (slots past hi
+    // re-read row[hi]) so that the loads carry no predicate and are all in
+    // flight together; the slots past hi are masked afterwards
+    float raw[PL];
+#pragma unroll
+    for (int k = 0; k < PL; ++k) raw[k] = row[min(lo + lane + 32 * k, hi)];
     uint32_t key[PL];
     uint32_t lmax = 0;
 #pragma unroll
     for (int k = 0; k < PL; ++k) {
         const int j = lo + lane + 32 * k;
-        key[k] = (j <= hi) ? topn_key(row[j]) : 0u;
+        key[k] = (j <= hi) ? topn_key(raw[k]) : 0u;
         lmax = max(lmax, key[k]);
     }
     int mine = 0x7fffffff;
@@ -268,15 +274,28 @@ __device__ __forceinline__ void topn_row_cta(const float* row, int t, int n, int
 
 // one warp per (batch, token, group) item; scores [items, NSp]; NSp <= 32*PL
 template <int PL>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, PL <= 32 ? 3 : 1)
     topn_kernel(const float* __restrict__ pscore, long long items, int T, int G, int NSp, int n,
                 int lp, int fi, int fl, int32_t* __restrict__ idx) {
     __shared__ unsigned long long wbuf[8][32];
     const int lane = threadIdx.x & 31;
     const long long item = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
     if (item >= items) return;
-    const int t = (int)((item / G) % T);
-    topn_row_warp<PL>(pscore + item * NSp, t, n, lp, fi, fl, idx + item * n, lane, wbuf[threadIdx.x >> 5]);
+    const int t = items <= 0x7fffffffLL ? (int)(((unsigned)item / (unsigned)G) % (unsigned)T)
+                                        : (int)((item / G) % T);
+    // the fewest slots per lane that hold the row's scored candidates (warp-uniform)
+    const int nsl = (t / lp - fl - fi + 32) / 32;
+    const float* row = pscore + item * NSp;
+    int32_t* out = idx + item * n;
+    unsigned long long* wb = wbuf[threadIdx.x >> 5];
+    if (PL > 8 && nsl <= 8)
+        topn_row_warp<8>(row, t, n, lp, fi, fl, out, lane, wb);
+    else if (PL > 16 && nsl <= 16)
+        topn_row_warp<16>(row, t, n, lp, fi, fl, out, lane, wb);
+    else if (PL > 32 && nsl <= 32)
+        topn_row_warp<32>(row, t, n, lp, fi, fl, out, lane, wb);
+    else
+        topn_row_warp<PL>(row, t, n, lp, fi, fl, out, lane, wb);
 }
 
 }  // namespace nsa

@@ -308,6 +308,10 @@ __global__ void __launch_bounds__(320, 1)
             const size_t rb2 = ((size_t)b * p.T + tb + i) * p.H + (size_t)g * HG;
 #pragma unroll
             for (int h = 0; h < HG; ++h) gate_nx[h] = __ldg(p.gates + (rb2 + h) * 3 + 1);
+            // the token's out rows (HG x DV fp32, contiguous), read-modify-written
+            // by the epilogue: brought into L2 now, two tokens ahead
+            if (kl * 32 < HG * DV)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(p.out + rb2 * DV + kl * 32));
         };
         prefetch(wg);
         for (int i = wg; i < N; i += 2, ++it) {

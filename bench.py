@@ -336,7 +336,7 @@ def main():
         if rank == 0 and world == 1:
             try:
                 hx = host_inputs(x)
-                full, desc = oracle_sample(cr, hx, rows_per_step=384, phi_fraction=1.0, seed=1)
+                full, desc = oracle_sample(cr, hx, rows_per_step=768, phi_fraction=1.0, seed=1)
                 import oracle
                 line["cpu_baseline"] = {"value": round(tokens_per_step / full, 3), "unit": "tokens/s",
                                         "cores": oracle.num_threads(), "kind": "oracle",

@@ -363,13 +363,15 @@ __global__ void __launch_bounds__(320, 1)
                     for (int k = 0; k < 64; ++k) mr = fmaxf(mr, s[k]);
                     const float mn = fmaxf(m_run, mr * c);
                     if (mn != -INFINITY) {
-                        float acc0 = 0.f, acc1 = 0.f;
+                        // even and odd columns summed separately, two per packed instruction
+                        float2 acc = make_float2(0.f, 0.f);
+                        const float2 c2 = make_float2(c, c), nm2 = make_float2(-mn, -mn);
 #pragma unroll
                         for (int k = 0; k < 64; k += 2) {
-                            acc0 += ex2a(fmaf(s[k], c, -mn));
-                            acc1 += ex2a(fmaf(s[k + 1], c, -mn));
+                            const float2 a = __ffma2_rn(make_float2(s[k], s[k + 1]), c2, nm2);
+                            acc = __fadd2_rn(acc, make_float2(ex2a(a.x), ex2a(a.y)));
                         }
-                        l_run = l_run * ex2a(m_run - mn) + (acc0 + acc1);
+                        l_run = l_run * ex2a(m_run - mn) + (acc.x + acc.y);
                         m_run = mn;
                     }
                 }
@@ -412,8 +414,13 @@ __global__ void __launch_bounds__(320, 1)
             if (MODE == kModeCmp) {
                 // a row with no visible key has LSE = -inf and only masked logits
                 const float nl = lse2 == -INFINITY ? 0.f : -lse2;
+                const float2 c2 = make_float2(c, c), nl2 = make_float2(nl, nl);
 #pragma unroll
-                for (int k = 0; k < 64; ++k) pr[k] = ex2a(fmaf(s[k], c, nl));
+                for (int k = 0; k < 64; k += 2) {
+                    const float2 a = __ffma2_rn(make_float2(s[k], s[k + 1]), c2, nl2);
+                    pr[k] = ex2a(a.x);
+                    pr[k + 1] = ex2a(a.y);
+                }
             } else {
                 float mr = -INFINITY;
 #pragma unroll
@@ -427,29 +434,44 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 // m_run stays -inf while every key so far is masked for this row
                 const float nm = m_run == -INFINITY ? 0.f : -m_run;
-                float acc0 = 0.f, acc1 = 0.f;
+                const float2 c2 = make_float2(c, c), nm2 = make_float2(nm, nm);
+                float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int k = 0; k < 64; k += 2) {
-                    pr[k] = ex2a(fmaf(s[k], c, nm));
-                    pr[k + 1] = ex2a(fmaf(s[k + 1], c, nm));
-                    acc0 += pr[k];
-                    acc1 += pr[k + 1];
+                    const float2 a = __ffma2_rn(make_float2(s[k], s[k + 1]), c2, nm2);
+                    pr[k] = ex2a(a.x);
+                    pr[k + 1] = ex2a(a.y);
+                    acc = __fadd2_rn(acc, make_float2(pr[k], pr[k + 1]));
                 }
-                l_run += acc0 + acc1;
+                l_run += acc.x + acc.y;
             }
             if (MODE == kModeCmp) {
                 // importance scores of selection blocks kb/SPB .. kb/SPB + NB - 1
                 float part[NJ];
+                if constexpr (SPB == 4 && CPS == 2) {
+                    // key 4m+u feeds block m twice for u < 3; key 4m+3 feeds blocks m
+                    // and m+1 once: part[m] = 2 (p0+p1+p2+p3) - p3 + p(4m-1), with
+                    // p(-1) the last key of the previous tile (carried)
 #pragma unroll
-                for (int m = 0; m < NJ; ++m) part[m] = 0.f;
+                    for (int m = 0; m < NB; ++m) {
+                        const float2 q = __fadd2_rn(make_float2(pr[4 * m], pr[4 * m + 1]),
+                                                    make_float2(pr[4 * m + 2], pr[4 * m + 3]));
+                        const float prev = m == 0 ? carry[0] : pr[4 * m - 1];
+                        part[m] = fmaf(2.f, q.x + q.y, prev - pr[4 * m + 3]);
+                    }
+                    carry[0] = pr[63];
+                } else {
 #pragma unroll
-                for (int c = 0; c < NC; ++c) part[c] += carry[c];
+                    for (int m = 0; m < NJ; ++m) part[m] = 0.f;
 #pragma unroll
-                for (int k = 0; k < 64; ++k)
+                    for (int c = 0; c < NC; ++c) part[c] += carry[c];
 #pragma unroll
-                    for (int u = 0; u < CPS; ++u) part[(k + u) / SPB] += pr[k];
+                    for (int k = 0; k < 64; ++k)
 #pragma unroll
-                for (int c = 0; c < NC; ++c) carry[c] = part[NB + c];
+                        for (int u = 0; u < CPS; ++u) part[(k + u) / SPB] += pr[k];
+#pragma unroll
+                    for (int c = 0; c < NC; ++c) carry[c] = part[NB + c];
+                }
                 float red[NB];
 #pragma unroll
                 for (int m = 0; m < NB; ++m) red[m] = part[m];

@@ -463,13 +463,47 @@ def bench_decode(dev, nsa, peaks, peak_src, steps=50, warmup=5):
             blocks |= bl
         nbytes += H * dk * 2 + H * 3 * 4 + H * dv * 4
     gbs = nbytes / (ms / 1e3) / 1e9
+    append = bench_append(c, x, kv_off, cmp_off, dev, nsa, stream)
     return {"workload": "decode_S32_L8k_64k", "value": round(c["S"] / (ms / 1e3), 1),
             "unit": "tokens/s", "ms_per_step": round(ms, 4), "unique_bytes_per_step": int(nbytes),
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
                          "peak_source": f"{peak_src} copy bandwidth", "frac_of_8TBs": round(gbs / 8000, 4)},
             "kernels": {k: {"launches": n, "us_per_step": round(1e3 * t / steps, 2)} for k, (n, t) in prof.items()},
-            "l2": "flushed (512 MB write) before each timed step"}
+            "l2": "flushed (512 MB write) before each timed step", "append": append}
+
+
+def bench_append(c, x, kv_off, cmp_off, dev, nsa, stream, reps=50):
+    """Decode-step cache maintenance for the 32 sequences: append the last token of
+    each (into the row it already owns) and compress the block it completes; once
+    with the drawn lengths (few complete a block), once with every sequence
+    completing one (the lengths moved back to the last block boundary)."""
+    L = torch.from_numpy(x["lengths"]).to(dev)
+    l, d = c["l"], c["d"]
+    typical = L - 1
+    all_blocks = L - 1 - ((L - l) % d)
+    k_new = x["k_cache"][kv_off[1:] - 1].contiguous()
+    v_new = x["v_cache"][kv_off[1:] - 1].contiguous()
+    phi = I.make_phi_params(c, dev) if c["phi"] == "linear" else None
+    starts, cstarts = kv_off[:-1].contiguous(), cmp_off[:-1].contiguous()
+
+    def run(lens):
+        for _ in range(3):
+            nsa.decode_append(c, k_new, v_new, x["k_cache"], x["v_cache"], starts, lens, x["kc_cache"],
+                              x["vc_cache"], cstarts, phi, stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            nsa.decode_append(c, k_new, v_new, x["k_cache"], x["v_cache"], starts, lens, x["kc_cache"],
+                              x["vc_cache"], cstarts, phi, stream)
+        e1.record(stream)
+        e1.synchronize()
+        nsa.sync_status()
+        return round(1e3 * e0.elapsed_time(e1) / reps, 2)
+
+    n_typ = int((((typical + 1 - l) % d == 0) & (typical + 1 >= l)).sum())
+    return {"us_per_step": run(typical.contiguous()), "blocks_completed": n_typ,
+            "us_per_step_every_seq_completes_a_block": run(all_blocks.contiguous()), "seqs": int(L.numel())}
 
 
 def bench_backward(dev, nsa, peaks, steps=2, warmup=1, seq_len=0):

@@ -175,6 +175,37 @@ nsa_status_t nsa_backward(const nsa_config_t* cfg, const void* q, const void* k,
                           const int32_t* sel_idx, float* dq, float* dk, float* dv, float* dgates,
                           void* workspace, size_t workspace_bytes, void* stream);
 
+/* Batched decode step over caches with spare capacity per sequence: as
+ * nsa_decode, but sequence s holds kv_len[s] tokens in rows [kv_start[s],
+ * kv_start[s] + kv_len[s]) of k_cache/v_cache and nsa_num_cmp_blocks(cfg,
+ * kv_len[s]) compressed blocks from row cmp_start[s] of kc_cache/vc_cache
+ * (kv_start, kv_len, cmp_start: int64 device arrays of S entries).  With
+ * nsa_decode_append this serves a generation loop without repacking the
+ * caches.  Same limits, workspace and errors as nsa_decode. */
+nsa_status_t nsa_decode_rows(const nsa_config_t* cfg, int32_t num_seqs, const void* q,
+                             const void* k_cache, const void* v_cache, const int64_t* kv_start,
+                             const int64_t* kv_len, const void* kc_cache, const void* vc_cache,
+                             const int64_t* cmp_start, const float* gates, float* out, int32_t* sel_idx,
+                             float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Decode-step cache maintenance (page 2, 令牌压缩: block i covers tokens
+ * [i*d, i*d + l); 效率分析 解码速度: the decode step reads the compressed cache).
+ * Appends one token per sequence and compresses the block it completes.
+ * In:  k_new [S,G,d_k], v_new [S,G,d_v] bf16: the token at position kv_len[s]
+ *      of sequence s; kv_start, kv_len, cmp_start as for nsa_decode_rows
+ *      (lengths BEFORE the append); phi parameters for NSA_PHI_LINEAR.
+ * Out: row kv_start[s] + kv_len[s] of k_cache/v_cache; and when the new length
+ *      L = kv_len[s] + 1 satisfies L >= l and (L - l) % d == 0, row
+ *      cmp_start[s] + (L - l)/d of kc_cache/vc_cache = phi of tokens
+ *      [L - l, L), correctly rounded to bf16 (each output one fp64 sum).
+ * The caller owns the capacity (the rows written must exist) and advances
+ * kv_len itself after the call.  Needs no workspace; S <= 65535; caches, new
+ * rows and phi parameters 16-byte aligned (NSA_ERR_INVALID_ARG otherwise). */
+nsa_status_t nsa_decode_append(const nsa_config_t* cfg, int32_t num_seqs, const void* k_new,
+                               const void* v_new, void* k_cache, void* v_cache, const int64_t* kv_start,
+                               const int64_t* kv_len, void* kc_cache, void* vc_cache,
+                               const int64_t* cmp_start, const nsa_phi_params_t* phi, void* stream);
+
 /* Top-n block selection alone (page 2, Top-n 块选择; its hyperparameter
  * paragraph fixes 1 initial and 2 local blocks as always selected), the step
  * nsa_forward takes between the compressed and the selected branch.

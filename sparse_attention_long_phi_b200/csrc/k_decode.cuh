@@ -48,7 +48,8 @@ struct DecParams {
     int spb, cps, nbs;       // l'/d, l/d, block-sum slots used per chunk
     float scale_log2;
     const __nv_bfloat16 *q, *kcache, *vcache, *kccache, *vccache;
-    const int64_t *kv_off, *cmp_off;
+    const int64_t *kv_off, *cmp_off;   // row starts; [S+1] packed, or [S] with kv_len
+    const int64_t* kv_len;             // [S] tokens per sequence, or null (packed offsets)
     const float* gates;
     float* out;
     int32_t* sel_idx;
@@ -82,8 +83,13 @@ __device__ __forceinline__ void load_q_frags(const DecParams& p, int s, int g, u
 // lengths of sequence s; false when it is empty or exceeds the sizes the
 // workspace was laid out for
 __device__ __forceinline__ bool dec_seq_ok(const DecParams& p, int s, int& L, int& C) {
-    L = (int)(p.kv_off[s + 1] - p.kv_off[s]);
-    C = (int)(p.cmp_off[s + 1] - p.cmp_off[s]);
+    if (p.kv_len) {               // rows from explicit lengths (caches with spare capacity)
+        L = (int)p.kv_len[s];
+        C = L >= p.l ? (L - p.l) / p.d + 1 : 0;
+    } else {
+        L = (int)(p.kv_off[s + 1] - p.kv_off[s]);
+        C = (int)(p.cmp_off[s + 1] - p.cmp_off[s]);
+    }
     return L > 0 && L <= p.Lmax && C <= p.Cmax;
 }
 
@@ -225,7 +231,8 @@ __global__ void __launch_bounds__(256, 1) dec_cmp_stream(const DecParams p) {
         }
         const int s = lo;
         const int64_t cbase = p.cmp_off[s];
-        const int C = (int)(p.cmp_off[s + 1] - cbase);
+        int Ls, C;
+        dec_seq_ok(p, s, Ls, C);                    // s holds chunks, so it passed this check
         const int nch = (C + 31) / 32;
         const int r = (int)(x - pre[s]);
         const int g = r / nch, cfirst = r - g * nch;

@@ -22,6 +22,7 @@
 #include "k_backward.cuh"
 #include "k_phi.cuh"
 #include "k_topn.cuh"
+#include "k_append.cuh"
 
 using namespace nsa;
 
@@ -639,7 +640,7 @@ nsa_status_t decode_launch(DecParams& p, const Shape& s, int S, cudaStream_t st)
 nsa_status_t decode_impl(const Shape& s, int S, const void* q, const void* kcache, const void* vcache,
                          const int64_t* kv_off, const void* kccache, const void* vccache,
                          const int64_t* cmp_off, const float* gates, float* out, int32_t* sel_idx,
-                         float* lse, uint8_t* ws, cudaStream_t st) {
+                         float* lse, uint8_t* ws, cudaStream_t st, const int64_t* kv_len = nullptr) {
     DecParams p{};
     p.S = S;
     p.H = (int)s.H;
@@ -665,6 +666,7 @@ nsa_status_t decode_impl(const Shape& s, int S, const void* q, const void* kcach
     p.vccache = reinterpret_cast<const __nv_bfloat16*>(vccache);
     p.kv_off = kv_off;
     p.cmp_off = cmp_off;
+    p.kv_len = kv_len;
     p.gates = gates;
     p.out = out;
     p.sel_idx = sel_idx;
@@ -808,6 +810,82 @@ nsa_status_t nsa_decode(const nsa_config_t* cfg, int32_t num_seqs, const void* q
     return decode_impl(s, num_seqs, q, k_cache, v_cache, kv_offsets, kc_cache, vc_cache, cmp_offsets,
                        gates, out, sel_idx, lse, reinterpret_cast<uint8_t*>(workspace),
                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+nsa_status_t nsa_decode_rows(const nsa_config_t* cfg, int32_t num_seqs, const void* q,
+                             const void* k_cache, const void* v_cache, const int64_t* kv_start,
+                             const int64_t* kv_len, const void* kc_cache, const void* vc_cache,
+                             const int64_t* cmp_start, const float* gates, float* out, int32_t* sel_idx,
+                             float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+    Shape s;
+    NSA_TRY(derive(cfg, s));
+    NSA_TRY(supported(s));
+    if (cfg->score_map != 0) return NSA_ERR_UNSUPPORTED;
+    if (num_seqs < 0 || num_seqs > cfg->batch) return NSA_ERR_INVALID_ARG;
+    if (num_seqs == 0) return NSA_OK;
+    if (!q || !k_cache || !v_cache || !kv_start || !kv_len || !kc_cache || !vc_cache || !cmp_start ||
+        !gates || !out || !sel_idx)
+        return NSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(kc_cache) ||
+        !aligned16(vc_cache))
+        return NSA_ERR_INVALID_ARG;
+    const size_t need = decode_ws_bytes(s.B, s.T, s.G, s.l, s.d, s.lp, s.w, s.n, s.DV);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return NSA_ERR_WORKSPACE;
+    return decode_impl(s, num_seqs, q, k_cache, v_cache, kv_start, kc_cache, vc_cache, cmp_start,
+                       gates, out, sel_idx, lse, reinterpret_cast<uint8_t*>(workspace),
+                       reinterpret_cast<cudaStream_t>(stream), kv_len);
+}
+
+nsa_status_t nsa_decode_append(const nsa_config_t* cfg, int32_t num_seqs, const void* k_new,
+                               const void* v_new, void* k_cache, void* v_cache, const int64_t* kv_start,
+                               const int64_t* kv_len, void* kc_cache, void* vc_cache,
+                               const int64_t* cmp_start, const nsa_phi_params_t* phi, void* stream) {
+    Shape s;
+    NSA_TRY(derive(cfg, s));
+    NSA_TRY(supported(s));
+    if (num_seqs < 0) return NSA_ERR_INVALID_ARG;
+    if (num_seqs == 0) return NSA_OK;
+    if (num_seqs > 65535) return NSA_ERR_UNSUPPORTED;
+    if (!k_new || !v_new || !k_cache || !v_cache || !kv_start || !kv_len || !kc_cache || !vc_cache ||
+        !cmp_start)
+        return NSA_ERR_INVALID_ARG;
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache))
+        return NSA_ERR_INVALID_ARG;
+    if (s.phi == NSA_PHI_LINEAR && (!phi || !phi->w_k || !phi->e_k || !phi->w_v || !phi->e_v ||
+                                    !aligned16(phi->w_k) || !aligned16(phi->w_v) || !aligned16(phi->e_k) ||
+                                    !aligned16(phi->e_v)))
+        return NSA_ERR_INVALID_ARG;
+    AppendParams p{};
+    p.S = num_seqs;
+    p.G = (int)s.G;
+    p.l = (int)s.l;
+    p.d = (int)s.d;
+    p.phi = s.phi == NSA_PHI_LINEAR ? 1 : 0;
+    p.kv_start = kv_start;
+    p.cmp_start = cmp_start;
+    p.len = kv_len;
+    p.k_new = reinterpret_cast<const __nv_bfloat16*>(k_new);
+    p.v_new = reinterpret_cast<const __nv_bfloat16*>(v_new);
+    p.k_cache = reinterpret_cast<__nv_bfloat16*>(k_cache);
+    p.v_cache = reinterpret_cast<__nv_bfloat16*>(v_cache);
+    p.kc_cache = reinterpret_cast<__nv_bfloat16*>(kc_cache);
+    p.vc_cache = reinterpret_cast<__nv_bfloat16*>(vc_cache);
+    if (p.phi) {
+        p.w_k = reinterpret_cast<const __nv_bfloat16*>(phi->w_k);
+        p.e_k = reinterpret_cast<const __nv_bfloat16*>(phi->e_k);
+        p.w_v = reinterpret_cast<const __nv_bfloat16*>(phi->w_v);
+        p.e_v = reinterpret_cast<const __nv_bfloat16*>(phi->e_v);
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const dim3 grid((unsigned)num_seqs, (unsigned)s.G, 2 * kAppendSplit);
+    const size_t smem = p.phi ? (size_t)s.l * std::max(s.DK, s.DV) * sizeof(double) : 0;
+    if (smem > 48 * 1024) return NSA_ERR_UNSUPPORTED;     // l * d_k <= 6144 for the staged block
+    if (s.DK == 192)
+        NSA_LAUNCH("decode_append_kernel", st, decode_append_kernel<192, 128><<<grid, 256, smem, st>>>(p));
+    else
+        NSA_LAUNCH("decode_append_kernel", st, decode_append_kernel<64, 64><<<grid, 256, smem, st>>>(p));
+    return last_launch();
 }
 
 nsa_status_t nsa_backward(const nsa_config_t* cfg, const void* q, const void* k, const void* v,

@@ -146,15 +146,20 @@ def make_forward_inputs(wl: dict, device="cpu", with_dout: bool = False) -> dict
     z = normal64(s, STREAMS["gates"], B * T * H * 3, device)
     out["gates"] = torch.sigmoid(z).to(torch.float32).view(B, T, H, 3)
     if wl.get("phi", "mean") == "linear":
-        out["wk"] = normal_bf16(s, STREAMS["wk"], (dk, l * dk), std=1.0 / math.sqrt(l * dk),
-                                device=device)
-        out["ek"] = normal_bf16(s, STREAMS["ek"], (l, dk), device=device)
-        out["wv"] = normal_bf16(s, STREAMS["wv"], (dv, l * dv), std=1.0 / math.sqrt(l * dv),
-                                device=device)
-        out["ev"] = normal_bf16(s, STREAMS["ev"], (l, dv), device=device)
+        out.update(make_phi_params(wl, device))
     if with_dout:
         out["dout"] = normal_bf16(s, STREAMS["dout"], (B, T, H, dv), device=device)
     return out
+
+
+def make_phi_params(wl: dict, device="cpu") -> dict:
+    """Linear phi parameters: W_K [dk, l*dk] ~ N(0, 1/(l*dk)), E_K [l, dk] ~ N(0,1),
+    W_V [dv, l*dv] ~ N(0, 1/(l*dv)), E_V [l, dv] ~ N(0,1), bf16."""
+    s, dk, dv, l = wl["seed"], wl["dk"], wl["dv"], wl["l"]
+    return {"wk": normal_bf16(s, STREAMS["wk"], (dk, l * dk), std=1.0 / math.sqrt(l * dk), device=device),
+            "ek": normal_bf16(s, STREAMS["ek"], (l, dk), device=device),
+            "wv": normal_bf16(s, STREAMS["wv"], (dv, l * dv), std=1.0 / math.sqrt(l * dv), device=device),
+            "ev": normal_bf16(s, STREAMS["ev"], (l, dv), device=device)}
 
 
 def decode_lengths(wl: dict) -> np.ndarray:

@@ -63,8 +63,14 @@ def lib():
         L.nsa_num_cmp_blocks.argtypes = [pc, ctypes.c_int64]
         L.nsa_compress.restype = ctypes.c_int
         L.nsa_compress.argtypes = [pc, _P, _P, pp, _P, _P, _P, ctypes.c_size_t, _P]
+        L.nsa_compress_static.restype = ctypes.c_int
+        L.nsa_compress_static.argtypes = [pc, _P, _P, pp, _P, _P, _P]
         L.nsa_forward.restype = ctypes.c_int
         L.nsa_forward.argtypes = [pc, _P, _P, _P, _P, pp, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+        L.nsa_decode_rows.restype = ctypes.c_int
+        L.nsa_decode_rows.argtypes = [pc, ctypes.c_int32] + [_P] * 13 + [ctypes.c_size_t, _P]
+        L.nsa_decode_append.restype = ctypes.c_int
+        L.nsa_decode_append.argtypes = [pc, ctypes.c_int32] + [_P] * 9 + [pp, _P]
         L.nsa_select_blocks.restype = ctypes.c_int
         L.nsa_select_blocks.argtypes = [pc, _P, _P, _P]
         L.nsa_decode.restype = ctypes.c_int
@@ -195,6 +201,18 @@ def select_blocks(c: dict, scores, stream=None) -> torch.Tensor:
     return idx
 
 
+def compress_static(c: dict, k, v, phi=None, stream=None) -> tuple:
+    """Token compression with the library's fixed device scratch (no workspace).
+    Returns (status, kc, vc); status NSA_ERR_WORKSPACE (3) when the sizes exceed it."""
+    B, T, G = c["B"], c["T"], c["G"]
+    C = num_cmp_blocks(c, T)
+    kc = torch.full((B, max(C, 1), G, c["dk"]), float("nan"), dtype=torch.bfloat16, device=k.device)
+    vc = torch.full((B, max(C, 1), G, c["dv"]), float("nan"), dtype=torch.bfloat16, device=k.device)
+    rc = lib().nsa_compress_static(ctypes.byref(make_config(c)), _p(k), _p(v), _phi(phi), _p(kc), _p(vc),
+                                   _stream(stream))
+    return rc, kc[:, :C], vc[:, :C]
+
+
 @dataclass
 class DecodeBuffers:
     out: torch.Tensor
@@ -229,6 +247,31 @@ def decode(c: dict, q, k_cache, v_cache, kv_off, kc_cache, vc_cache, cmp_off, ga
     decode_into(c, max_len, q, k_cache, v_cache, kv_off, kc_cache, vc_cache, cmp_off, gates, buf,
                 stream)
     return {"out": buf.out, "idx": buf.idx, "lse": buf.lse}
+
+
+def decode_rows(c: dict, q, k_cache, v_cache, kv_start, kv_len, kc_cache, vc_cache, cmp_start, gates,
+                max_len: int, want_lse=True, stream=None) -> dict:
+    """One decode step over caches with spare capacity: sequence s holds kv_len[s] tokens
+    from row kv_start[s] and its compressed blocks from row cmp_start[s] (int64 device [S])."""
+    S = q.shape[0]
+    buf = decode_buffers(c, S, max_len, q.device, want_lse)
+    cfg = make_config(c, batch=S, seqlen=max_len)
+    _check("nsa_decode_rows", lib().nsa_decode_rows(
+        ctypes.byref(cfg), S, _p(q), _p(k_cache), _p(v_cache), _p(kv_start), _p(kv_len), _p(kc_cache),
+        _p(vc_cache), _p(cmp_start), _p(gates), _p(buf.out), _p(buf.idx), _p(buf.lse), _p(buf.ws),
+        buf.ws.numel(), _stream(stream)))
+    return {"out": buf.out, "idx": buf.idx, "lse": buf.lse}
+
+
+def decode_append(c: dict, k_new, v_new, k_cache, v_cache, kv_start, kv_len, kc_cache, vc_cache, cmp_start,
+                  phi=None, stream=None):
+    """Append token kv_len[s] of each sequence (k_new [S,G,dk], v_new [S,G,dv]) to the raw caches and
+    write phi of the compressed block it completes, if any.  kv_len is not advanced here."""
+    S = k_new.shape[0]
+    cfg = make_config(c, batch=S, seqlen=c.get("T", 1))   # the context length plays no part here
+    _check("nsa_decode_append", lib().nsa_decode_append(
+        ctypes.byref(cfg), S, _p(k_new), _p(v_new), _p(k_cache), _p(v_cache), _p(kv_start), _p(kv_len),
+        _p(kc_cache), _p(vc_cache), _p(cmp_start), _phi(phi), _stream(stream)))
 
 
 def backward(c: dict, q, k, v, gates, dout, idx, phi=None, stream=None) -> dict:

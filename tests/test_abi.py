@@ -35,6 +35,27 @@ def test_library_exports_every_declared_entry_point(L):
         assert hasattr(lib, n), n
 
 
+def declared_arity():
+    """Parameter count of every function include/nsa.h declares."""
+    txt = open(os.path.join(ROOT, "include", "nsa.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(nsa_[a-z_]+)\s*\(([^()]*)\)\s*;", txt):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_argument_counts_match_the_header(L):
+    lib = L.lib()
+    arity = declared_arity()
+    assert len(arity) >= 14
+    for name, n in arity.items():
+        argtypes = getattr(lib, name).argtypes
+        assert argtypes is not None, f"{name}: no argtypes in the binding"
+        assert len(argtypes) == n, f"{name}: binding has {len(argtypes)} arguments, header {n}"
+
+
 def test_status_strings_and_shape_helpers(L):
     lib = L.lib()
     for code in range(6):
@@ -79,6 +100,24 @@ def test_select_blocks_validation_on_host(L):
     assert lib.nsa_select_blocks(ctypes.byref(L.make_config(dict(base, n=2))), fake, fake, None) == 1
     assert lib.nsa_select_blocks(ctypes.byref(L.make_config(dict(base, n=33))), fake, fake, None) == 2
     assert lib.nsa_select_blocks(ctypes.byref(L.make_config(dict(base, T=131073))), fake, fake, None) == 2
+
+
+def test_decode_append_and_rows_validation_on_host(L):
+    lib = L.lib()
+    c = dict(I.WORKLOADS["decode_S32_L8k_64k"])
+    cfg = L.make_config(c, batch=32, seqlen=65536)
+    fake = ctypes.c_void_p(1 << 20)
+    nine = [fake] * 9
+    assert lib.nsa_decode_append(ctypes.byref(cfg), 4, None, *nine[1:], None, None) == 1     # null k_new
+    assert lib.nsa_decode_append(ctypes.byref(cfg), 4, *nine, None, None) == 1               # linear phi, no params
+    assert lib.nsa_decode_append(ctypes.byref(cfg), 0, *([None] * 9), None, None) == 0      # nothing to do
+    assert lib.nsa_decode_append(ctypes.byref(cfg), -1, *nine, None, None) == 1
+    assert lib.nsa_decode_rows(ctypes.byref(cfg), 33, *([fake] * 13), 1 << 30, None) == 1   # more seqs than sized
+    assert lib.nsa_decode_rows(ctypes.byref(cfg), 8, *([fake] * 13), 16, None) == 3         # workspace too small
+    args = [fake] * 13
+    args[4] = None                                                                           # no lengths
+    assert lib.nsa_decode_rows(ctypes.byref(cfg), 8, *args, 1 << 30, None) == 1
+    assert len(L.lib().nsa_decode_rows.argtypes) == 17 and len(L.lib().nsa_decode.argtypes) == 16
 
 
 def test_decode_and_backward_validation_on_host(L):

@@ -12,28 +12,9 @@ from sparse_attention_long_phi_b200 import inputs as I
 pytestmark = pytest.mark.gpu
 
 
-def _static_fn(nsa):
-    lib = nsa.lib()
-    fn = lib.nsa_compress_static
-    fn.restype = ctypes.c_int
-    fn.argtypes = [ctypes.POINTER(nsa.CConfig)] + [ctypes.c_void_p] * 2 + \
-                  [ctypes.POINTER(nsa.CPhi)] + [ctypes.c_void_p] * 3
-    return fn
-
-
 def _call_static(nsa, c, x):
-    fn = _static_fn(nsa)
-    B, T, G = c["B"], c["T"], c["G"]
-    C = nsa.num_cmp_blocks(c, T)
-    kc = torch.full((B, C, G, c["dk"]), float("nan"), dtype=torch.bfloat16, device="cuda")
-    vc = torch.full((B, C, G, c["dv"]), float("nan"), dtype=torch.bfloat16, device="cuda")
-    phi = None
-    if "wk" in x:
-        phi = ctypes.byref(nsa.CPhi(*(ctypes.c_void_p(x[n].data_ptr()) for n in ("wk", "ek", "wv", "ev"))))
-    rc = fn(ctypes.byref(nsa.make_config(c)), ctypes.c_void_p(x["k"].data_ptr()),
-            ctypes.c_void_p(x["v"].data_ptr()), phi, ctypes.c_void_p(kc.data_ptr()),
-            ctypes.c_void_p(vc.data_ptr()), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
-    return rc, kc, vc
+    phi = {n: x[n] for n in ("wk", "ek", "wv", "ev")} if "wk" in x else None
+    return nsa.compress_static(c, x["k"], x["v"], phi)
 
 
 @pytest.mark.parametrize("name,T,seed", [("prefill_fwd_T8192", 8192, 5000), ("tiny_fwd_T1024", 1024, 5001)])
@@ -55,9 +36,7 @@ def test_static_compress_matches_workspace_compress_twice(name, T, seed):
 def test_static_compress_rejects_sizes_beyond_its_scratch():
     from sparse_attention_long_phi_b200 import nsa
     c = dict(I.WORKLOADS["prefill_fwd_T65536"])     # 5.2M compressed elements > 16 MiB of scratch
-    x = {k: torch.empty(0, device="cuda") for k in ("k", "v", "wk", "ek", "wv", "ev")}
-    fn = _static_fn(nsa)
-    fake = ctypes.c_void_p(1 << 20)
-    rc = fn(ctypes.byref(nsa.make_config(c)), fake, fake,
-            ctypes.byref(nsa.CPhi(fake, fake, fake, fake)), fake, fake, None)
+    fake = ctypes.c_void_p(1 << 20)                  # never dereferenced: rejected first
+    rc = nsa.lib().nsa_compress_static(ctypes.byref(nsa.make_config(c)), fake, fake,
+                                       ctypes.byref(nsa.CPhi(fake, fake, fake, fake)), fake, fake, None)
     assert rc == 3

@@ -552,13 +552,16 @@ def run_reference(args, c, rank, world, tokens_per_step):
     import oracle
     x = I.make_forward_inputs(c, "cuda" if torch.cuda.is_available() else "cpu")
     hx = host_inputs(x)
+    # each step: two rows per host thread (the oracle parallelises over rows, so
+    # every core works) and 1/16 of the phi blocks, about half a second of CPU work
+    rows = 2 * oracle.num_threads()
     for i in range(args.warmup):
-        oracle_sample(c, hx, rows_per_step=2, phi_fraction=1 / 64, seed=100 + i)
+        oracle_sample(c, hx, rows_per_step=rows, phi_fraction=1 / 16, seed=100 + i)
     fulls = []
     t0 = time.perf_counter()
     desc = ""
     for i in range(args.steps):
-        full, desc = oracle_sample(c, hx, rows_per_step=2, phi_fraction=1 / 64, seed=i)
+        full, desc = oracle_sample(c, hx, rows_per_step=rows, phi_fraction=1 / 16, seed=i)
         fulls.append(full)
     wall = time.perf_counter() - t0
     sec = float(np.mean(fulls))

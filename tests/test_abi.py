@@ -120,6 +120,18 @@ def test_decode_append_and_rows_validation_on_host(L):
     assert len(L.lib().nsa_decode_rows.argtypes) == 17 and len(L.lib().nsa_decode.argtypes) == 16
 
 
+@pytest.mark.parametrize("l,d", [(32, 16), (32, 32), (16, 16), (64, 16)])
+def test_append_completion_rule_matches_block_count(L, l, d):
+    # nsa_decode_append compresses block (L - l)/d exactly when the new length L
+    # adds one to nsa_num_cmp_blocks (page 2, 令牌压缩: block i = tokens [i*d, i*d + l))
+    import oracle
+    c = dict(I.WORKLOADS["prefill_fwd_T8192"], l=l, d=d)
+    for n in range(1, 600):
+        grows = L.num_cmp_blocks(c, n) - L.num_cmp_blocks(c, n - 1)
+        assert grows == int(n >= l and (n - l) % d == 0), n
+        assert L.num_cmp_blocks(c, n) == oracle.num_cmp_blocks(c, n)
+
+
 def test_decode_and_backward_validation_on_host(L):
     lib = L.lib()
     c = dict(I.WORKLOADS["decode_S32_L8k_64k"], B=32, T=65536)

@@ -67,7 +67,9 @@ def _load():
         lib.oracle_decode.restype = ctypes.c_int
         lib.oracle_decode.argtypes = [pc, _I64] + [_P] * 12 + [_I64]
         lib.oracle_backward_tail.restype = None
-        lib.oracle_backward_tail.argtypes = [pc] + [_P] * 10 + [_I64] + [_P] * 4
+        lib.oracle_backward_tail.argtypes = [pc] + [_P] * 10 + [_I64] + [_P] * 6
+        lib.oracle_phi_param_grads.restype = None
+        lib.oracle_phi_param_grads.argtypes = [pc, _I64] + [_P] * 6
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
         _lib = lib
@@ -228,21 +230,44 @@ def decode(c: dict, q, k_cache, v_cache, kv_off, kc_cache, vc_cache, cmp_off, ga
 
 
 def backward_tail(c: dict, q, k, v, gates, dout, idx, wk=None, ek=None, wv=None, ev=None,
-                  t_lo: int = 0):
+                  t_lo: int = 0, want_cmp: bool = False):
     """Backward with the selection ``idx`` [B,T,G,n] held fixed.
 
     dk/dv are exact for tokens u >= t_lo, dq/dgates for rows t >= t_lo.
-    Returns dict(dq [B,T,H,dk], dk [B,T,G,dk], dv [B,T,G,dv], dgates [B,T,H,3]).
+    Returns dict(dq [B,T,H,dk], dk [B,T,G,dk], dv [B,T,G,dv], dgates [B,T,H,3]), and with
+    want_cmp the compressed-key gradients dkc [B,C,G,dk], dvc [B,C,G,dv] (exact with t_lo = 0).
     """
     cf = make_cfg(c)
     B, T, H, G = cf.B, cf.T, cf.H, cf.G
+    C = num_cmp_blocks(c, T)
     dq = np.zeros((B, T, H, cf.dk))
     dk = np.zeros((B, T, G, cf.dk))
     dv = np.zeros((B, T, G, cf.dv))
     dg = np.zeros((B, T, H, 3))
+    dkc = np.zeros((B, C, G, cf.dk)) if want_cmp else None
+    dvc = np.zeros((B, C, G, cf.dv)) if want_cmp else None
     _load().oracle_backward_tail(
         ctypes.byref(cf), _ptr(_c(q, np.uint16)), _ptr(_c(k, np.uint16)), _ptr(_c(v, np.uint16)),
         _ptr(_c(gates, np.float32)), _ptr(_c(wk, np.uint16)), _ptr(_c(ek, np.uint16)),
         _ptr(_c(wv, np.uint16)), _ptr(_c(ev, np.uint16)), _ptr(_c(dout, np.uint16)),
-        _ptr(_c(idx, np.int32)), int(t_lo), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg))
-    return {"dq": dq, "dk": dk, "dv": dv, "dgates": dg}
+        _ptr(_c(idx, np.int32)), int(t_lo), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dkc), _ptr(dvc))
+    out = {"dq": dq, "dk": dk, "dv": dv, "dgates": dg}
+    if want_cmp:
+        out.update(dkc=dkc, dvc=dvc)
+    return out
+
+
+def phi_param_grads(c: dict, k, v, wk, ek, wv, ev, dkc, dvc):
+    """Gradients of the linear phi's W_K, E_K, W_V, E_V from dK~ = dkc, dV~ = dvc
+    (token compression: K~[i] = W vec(k_blk + E)).  fp64 dict(dwk, dek, dwv, dev)."""
+    cf = make_cfg(c)
+    lib = _load()
+    out = {}
+    for name, x, W, E, dY, D in (("k", k, wk, ek, dkc, cf.dk), ("v", v, wv, ev, dvc, cf.dv)):
+        dW = np.zeros((D, cf.l * D))
+        dE = np.zeros((cf.l, D))
+        lib.oracle_phi_param_grads(ctypes.byref(cf), int(D), _ptr(_c(x, np.uint16)), _ptr(_c(W, np.uint16)),
+                                   _ptr(_c(E, np.uint16)), _ptr(np.ascontiguousarray(dY, np.float64)),
+                                   _ptr(dW), _ptr(dE))
+        out["dw" + name], out["de" + name] = dW, dE
+    return out

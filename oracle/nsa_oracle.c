@@ -530,7 +530,7 @@ void oracle_backward_tail(const ocfg_t* c, const uint16_t* q, const uint16_t* k,
                           const uint16_t* v, const float* gates, const uint16_t* wk,
                           const uint16_t* ek, const uint16_t* wv, const uint16_t* ev,
                           const uint16_t* dout, const int32_t* idx, int64_t t_lo, double* dq,
-                          double* dk, double* dv, double* dgates)
+                          double* dk, double* dv, double* dgates, double* dkc_out, double* dvc_out)
 {
     const int64_t B = c->B, T = c->T, H = c->H, G = c->G, dK = c->dk, dV = c->dv;
     const int64_t C = oracle_num_cmp_blocks(c, T);
@@ -648,10 +648,50 @@ void oracle_backward_tail(const ocfg_t* c, const uint16_t* q, const uint16_t* k,
                     }
                 }
             }
+    if (dkc_out && C > 0) memcpy(dkc_out, dkc, sizeof(double) * (size_t)(B * C * G * dK));
+    if (dvc_out && C > 0) memcpy(dvc_out, dvc, sizeof(double) * (size_t)(B * C * G * dV));
     free(kc);
     free(vc);
     free(dkc);
     free(dvc);
+}
+
+/* Gradients of the linear phi's parameters (token compression: K~[i] =
+ * W vec(k_blk + E), vec position-major) from the compressed-key gradients
+ * dY = dK~ [B,C,G,D] of the backward above:
+ *   dW[o, x]  = sum over (b, i, g) of dY[b,i,g,o] * X[b,i,g,x],  X = vec(k_blk + E)
+ *   dE[j, ch] = sum over (b, i, g) and o of W[o, j*D + ch] * dY[b,i,g,o]
+ * (the bf16 rounding of K~ treated as the identity, as above).  One call per
+ * tensor: x = k with W_K, E_K (D = d_k) or v with W_V, E_V (D = d_v).
+ * Outputs fp64, zeroed here: dW [D, l*D], dE [l, D]. */
+void oracle_phi_param_grads(const ocfg_t* c, int64_t D, const uint16_t* x, const uint16_t* W,
+                            const uint16_t* E, const double* dY, double* dW, double* dE)
+{
+    const int64_t B = c->B, T = c->T, G = c->G, l = c->l, K = c->l * D;
+    const int64_t C = oracle_num_cmp_blocks(c, T);
+    memset(dW, 0, sizeof(double) * (size_t)(D * K));
+    memset(dE, 0, sizeof(double) * (size_t)K);
+#pragma omp parallel for schedule(static)
+    for (int64_t o = 0; o < D; ++o)
+        for (int64_t b = 0; b < B; ++b)
+            for (int64_t i = 0; i < C; ++i)
+                for (int64_t g = 0; g < G; ++g) {
+                    const double dy = dY[((b * C + i) * G + g) * D + o];
+                    for (int64_t j = 0; j < l; ++j)
+                        for (int64_t ch = 0; ch < D; ++ch)
+                            dW[o * K + j * D + ch] +=
+                                dy * (bf(x[((b * T + i * c->d + j) * G + g) * D + ch]) + bf(E[j * D + ch]));
+                }
+#pragma omp parallel for schedule(static)
+    for (int64_t e = 0; e < K; ++e) {
+        double acc = 0.0;
+        for (int64_t b = 0; b < B; ++b)
+            for (int64_t i = 0; i < C; ++i)
+                for (int64_t g = 0; g < G; ++g)
+                    for (int64_t o = 0; o < D; ++o)
+                        acc += bf(W[o * K + e]) * dY[((b * C + i) * G + g) * D + o];
+        dE[e] = acc;
+    }
 }
 
 int oracle_num_threads(void)

@@ -396,6 +396,39 @@ def test_backward_matches_central_differences(phi):
                                np.einsum("thc,thbc->thb", dO, r["obr"]), atol=1e-12)
 
 
+def test_phi_parameter_gradients_match_central_differences():
+    # token compression: K~[i] = W vec(k_blk + E); dW and dE from the backward's dK~, dV~
+    c = small_cfg(T=56, H=2, G=1, dk=8, dv=8, l=8, d=4, lp=8, n=3, w=9, phi="linear")
+    x = make(c, with_dout=True)
+    idx = oracle.forward_rows(c, x["q"], x["k"], x["v"], x["gates"],
+                              *oracle.phi(c, x["k"], x["v"], x["wk"], x["ek"], x["wv"], x["ev"]),
+                              np.arange(56))["idx"].reshape(1, 56, 1, 3)
+    rng = np.random.default_rng(12)
+    eps = 2.0 ** -10
+    checks = ([("wk", (o, e)) for o, e in zip(rng.integers(0, 8, 5), rng.integers(0, 64, 5))] +
+              [("ek", (j, ch)) for j, ch in zip(rng.integers(0, 8, 5), rng.integers(0, 8, 5))] +
+              [("wv", (o, e)) for o, e in zip(rng.integers(0, 8, 5), rng.integers(0, 64, 5))] +
+              [("ev", (j, ch)) for j, ch in zip(rng.integers(0, 8, 5), rng.integers(0, 8, 5))])
+    for name, pos in checks:
+        xz = {k: (v.copy() if isinstance(v, np.ndarray) else v) for k, v in x.items()}
+        xz[name][pos] = 0                                   # expand around 0 so +-eps is exact
+        g = oracle.backward_tail(dict(c, cmp_exact=1), xz["q"], xz["k"], xz["v"], xz["gates"], xz["dout"],
+                                 idx, xz["wk"], xz["ek"], xz["wv"], xz["ev"], want_cmp=True)
+        pg = oracle.phi_param_grads(c, xz["k"], xz["v"], xz["wk"], xz["ek"], xz["wv"], xz["ev"],
+                                    g["dkc"], g["dvc"])
+        vals = []
+        for sgn in (1, -1):
+            xp = dict(xz)
+            xp[name] = xz[name].copy()
+            xp[name][pos] = oracle.bf16_round(sgn * eps)
+            vals.append(_loss(c, xp, idx))
+        fd = (vals[0] - vals[1]) / (2 * eps)
+        an = pg["d" + name][pos]
+        assert abs(fd - an) <= 1e-6 + 1e-5 * abs(an), (name, pos, fd, an)
+    # dE = sum over blocks of W^T dK~: also the sum over block positions of dk's phi part
+    assert np.abs(pg["dwk"]).max() > 0 and np.abs(pg["dek"]).max() > 0
+
+
 def test_backward_tail_is_exact_above_the_cut():
     c = small_cfg(T=80, H=2, G=1, dk=8, dv=8, l=8, d=4, lp=8, n=3, w=9, phi="linear")
     x = make(c, with_dout=True)

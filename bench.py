@@ -517,7 +517,7 @@ def bench_backward(dev, nsa, peaks, steps=2, warmup=1, seq_len=0):
     fb = nsa.forward_buffers(c, dev, want_lse=False)
     nsa.forward_into(c, x["q"], x["k"], x["v"], x["gates"], phi, fb, stream)
     for _ in range(warmup):
-        nsa.backward(c, x["q"], x["k"], x["v"], x["gates"], x["dout"], fb.idx, phi)
+        nsa.backward(c, x["q"], x["k"], x["v"], x["gates"], x["dout"], fb.idx, phi, want_phi_grads=True)
     torch.cuda.synchronize(dev)
     nsa.sync_status()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -528,8 +528,8 @@ def bench_backward(dev, nsa, peaks, steps=2, warmup=1, seq_len=0):
     e1.record(stream)
     nsa.profile_read()
     nsa.profile_enable(True)
-    for _ in range(steps):
-        nsa.backward(c, x["q"], x["k"], x["v"], x["gates"], x["dout"], fb.idx, phi)
+    for _ in range(steps):   # the full training backward: q, k, v, gates and the phi parameters
+        nsa.backward(c, x["q"], x["k"], x["v"], x["gates"], x["dout"], fb.idx, phi, want_phi_grads=True)
     e2.record(stream)
     torch.cuda.synchronize(dev)
     nsa.profile_enable(False)

@@ -223,6 +223,19 @@ nsa_status_t nsa_decode_append(const nsa_config_t* cfg, int32_t num_seqs, const 
 nsa_status_t nsa_select_blocks(const nsa_config_t* cfg, const float* scores, int32_t* sel_idx,
                                void* stream);
 
+/* Gradients of the linear phi's parameters (page 2, 令牌压缩: a learnable map
+ * with intra-block position encoding, K~[i] = w_k vec(k_blk + e_k), likewise
+ * V~).  Reads the compressed-key gradients dK~/dV~ that the preceding
+ * nsa_backward call with the same cfg left in `workspace` (same stream, the
+ * workspace untouched in between) and k, v, phi as passed to it.
+ * Out (fp32, caller-owned): dw_k [d_k, l*d_k], de_k [l, d_k], dw_v [d_v, l*d_v],
+ * de_v [l, d_v]:  dW[o, x] = sum over (b, block i, g) of dK~[o] * x[x] with
+ * x = vec(k_blk + e_k);  dE[j, c] = sum over o of w[o, j*d + c] * sum dK~[o].
+ * NSA_ERR_INVALID_ARG for the mean phi (no parameters) or missing tensors. */
+nsa_status_t nsa_backward_phi_params(const nsa_config_t* cfg, const void* k, const void* v,
+                                     const nsa_phi_params_t* phi, float* dw_k, float* de_k, float* dw_v,
+                                     float* de_v, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronise `stream`, then read and clear the device error word of the
  * current device.  Returns NSA_ERR_DEVICE_TIMEOUT if a kernel's bounded wait
  * expired since the last call, NSA_ERR_CUDA if synchronisation failed. */

@@ -23,6 +23,7 @@
 #include "k_phi.cuh"
 #include "k_topn.cuh"
 #include "k_append.cuh"
+#include "k_phi_grad.cuh"
 
 using namespace nsa;
 
@@ -952,6 +953,57 @@ int32_t nsa_profile_read(int32_t max_kernels, char* names, int32_t* launches, fl
         ++k;
     }
     return k;
+}
+
+nsa_status_t nsa_backward_phi_params(const nsa_config_t* cfg, const void* k, const void* v,
+                                     const nsa_phi_params_t* phi, float* dw_k, float* de_k, float* dw_v,
+                                     float* de_v, void* workspace, size_t workspace_bytes, void* stream) {
+    Shape s;
+    NSA_TRY(derive(cfg, s));
+    NSA_TRY(supported(s));
+    if (s.phi != NSA_PHI_LINEAR) return NSA_ERR_INVALID_ARG;          // mean phi has no parameters
+    if (!k || !v || !phi || !phi->w_k || !phi->e_k || !phi->w_v || !phi->e_v || !dw_k || !de_k || !dw_v ||
+        !de_v)
+        return NSA_ERR_INVALID_ARG;
+    if (!aligned16(dw_k) || !aligned16(dw_v)) return NSA_ERR_INVALID_ARG;
+    const BwdWs L = bwd_layout(s);
+    if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return NSA_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+    const int64_t KK = s.l * s.DK, KV = s.l * s.DV;
+    if (s.C == 0) {                                      // no compressed block: no gradient
+        if (cudaMemsetAsync(dw_k, 0, (size_t)s.DK * KK * 4, st) != cudaSuccess ||
+            cudaMemsetAsync(de_k, 0, (size_t)KK * 4, st) != cudaSuccess ||
+            cudaMemsetAsync(dw_v, 0, (size_t)s.DV * KV * 4, st) != cudaSuccess ||
+            cudaMemsetAsync(de_v, 0, (size_t)KV * 4, st) != cudaSuccess)
+            return NSA_ERR_CUDA;
+        return NSA_OK;
+    }
+    const float* dkc = reinterpret_cast<const float*>(ws + L.off_dkc);
+    const float* dvc = reinterpret_cast<const float*>(ws + L.off_dvc);
+    float* colsum = reinterpret_cast<float*>(ws + L.off_fix);   // scratch: the fix-up list is done
+    const int N = (int)(s.B * s.C * s.G);
+    auto bf = [](const void* p) { return reinterpret_cast<const __nv_bfloat16*>(p); };
+    NSA_LAUNCH("phi_colsum_kernel", st, phi_colsum_kernel<<<(unsigned)(s.DK / 32), 256, 0, st>>>(dkc, N, (int)s.DK, colsum));
+    NSA_TRY(last_launch());
+    NSA_LAUNCH("phi_colsum_kernel", st, phi_colsum_kernel<<<(unsigned)(s.DV / 32), 256, 0, st>>>(dvc, N, (int)s.DV, colsum + s.DK));
+    NSA_TRY(last_launch());
+    NSA_LAUNCH("phi_de_kernel", st, phi_de_kernel<<<(unsigned)ceil_div(KK, 256), 256, 0, st>>>(bf(phi->w_k), colsum, (int)s.DK, (int)KK, de_k));
+    NSA_TRY(last_launch());
+    NSA_LAUNCH("phi_de_kernel", st, phi_de_kernel<<<(unsigned)ceil_div(KV, 256), 256, 0, st>>>(bf(phi->w_v), colsum + s.DK, (int)s.DV, (int)KV, de_v));
+    NSA_TRY(last_launch());
+    const int B = (int)s.B, T = (int)s.T, G = (int)s.G, C = (int)s.C, l = (int)s.l, d = (int)s.d;
+    if (s.DK == 192) {
+        NSA_LAUNCH("phi_dw_kernel", st, phi_dw_kernel<192><<<dim3((unsigned)(KK / 64), 3), 256, 0, st>>>(dkc, bf(k), bf(phi->e_k), B, T, G, C, l, d, dw_k));
+        NSA_TRY(last_launch());
+        NSA_LAUNCH("phi_dw_kernel", st, phi_dw_kernel<128><<<dim3((unsigned)(KV / 64), 2), 256, 0, st>>>(dvc, bf(v), bf(phi->e_v), B, T, G, C, l, d, dw_v));
+    } else {
+        NSA_LAUNCH("phi_dw_kernel", st, phi_dw_kernel<64><<<dim3((unsigned)(KK / 64), 1), 256, 0, st>>>(dkc, bf(k), bf(phi->e_k), B, T, G, C, l, d, dw_k));
+        NSA_TRY(last_launch());
+        NSA_LAUNCH("phi_dw_kernel", st, phi_dw_kernel<64><<<dim3((unsigned)(KV / 64), 1), 256, 0, st>>>(dvc, bf(v), bf(phi->e_v), B, T, G, C, l, d, dw_v));
+    }
+    return last_launch();
 }
 
 nsa_status_t nsa_sync_status(void* stream) {

@@ -78,6 +78,8 @@ def lib():
         L.nsa_backward.restype = ctypes.c_int
         L.nsa_backward.argtypes = [pc, _P, _P, _P, _P, pp, _P, _P, _P, _P, _P, _P, _P,
                                    ctypes.c_size_t, _P]
+        L.nsa_backward_phi_params.restype = ctypes.c_int
+        L.nsa_backward_phi_params.argtypes = [pc, _P, _P, pp, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
         L.nsa_sync_status.restype = ctypes.c_int
         L.nsa_sync_status.argtypes = [_P]
         L.nsa_profile_enable.restype = ctypes.c_int
@@ -274,17 +276,26 @@ def decode_append(c: dict, k_new, v_new, k_cache, v_cache, kv_start, kv_len, kc_
         _p(kc_cache), _p(vc_cache), _p(cmp_start), _phi(phi), _stream(stream)))
 
 
-def backward(c: dict, q, k, v, gates, dout, idx, phi=None, stream=None) -> dict:
-    """Gradients with the selection idx [B,T,G,n] held fixed: dq, dk, dv, dgates (fp32)."""
+def backward(c: dict, q, k, v, gates, dout, idx, phi=None, stream=None, want_phi_grads=False) -> dict:
+    """Gradients with the selection idx [B,T,G,n] held fixed: dq, dk, dv, dgates (fp32); with
+    want_phi_grads (linear phi) also dwk [dk, l*dk], dek [l, dk], dwv [dv, l*dv], dev [l, dv]."""
     B, T, H, G, dk, dv = c["B"], c["T"], c["H"], c["G"], c["dk"], c["dv"]
     f32 = dict(dtype=torch.float32, device=q.device)
     res = {"dq": torch.empty(B, T, H, dk, **f32), "dk": torch.empty(B, T, G, dk, **f32),
            "dv": torch.empty(B, T, G, dv, **f32), "dgates": torch.empty(B, T, H, 3, **f32)}
     ws = alloc_workspace(c, NSA_MODE_BACKWARD, q.device)
+    cfg = make_config(c)
     _check("nsa_backward", lib().nsa_backward(
-        ctypes.byref(make_config(c)), _p(q), _p(k), _p(v), _p(gates), _phi(phi), _p(dout), _p(idx),
+        ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(gates), _phi(phi), _p(dout), _p(idx),
         _p(res["dq"]), _p(res["dk"]), _p(res["dv"]), _p(res["dgates"]), _p(ws), ws.numel(),
         _stream(stream)))
+    if want_phi_grads:
+        l = c["l"]
+        res.update(dwk=torch.empty(dk, l * dk, **f32), dek=torch.empty(l, dk, **f32),
+                   dwv=torch.empty(dv, l * dv, **f32), dev=torch.empty(l, dv, **f32))
+        _check("nsa_backward_phi_params", lib().nsa_backward_phi_params(
+            ctypes.byref(cfg), _p(k), _p(v), _phi(phi), _p(res["dwk"]), _p(res["dek"]), _p(res["dwv"]),
+            _p(res["dev"]), _p(ws), ws.numel(), _stream(stream)))
     return res
 
 

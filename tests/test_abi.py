@@ -132,6 +132,18 @@ def test_append_completion_rule_matches_block_count(L, l, d):
         assert L.num_cmp_blocks(c, n) == oracle.num_cmp_blocks(c, n)
 
 
+def test_phi_parameter_gradient_validation_on_host(L):
+    lib = L.lib()
+    fake = ctypes.c_void_p(1 << 20)
+    phi = ctypes.byref(L.CPhi(fake, fake, fake, fake))
+    lin = L.make_config(I.WORKLOADS["train_fwd_bwd_B2_T16384"])
+    mean = L.make_config(dict(I.WORKLOADS["train_fwd_bwd_B2_T16384"], phi="mean"))
+    out = [fake] * 4
+    assert lib.nsa_backward_phi_params(ctypes.byref(mean), fake, fake, phi, *out, fake, 1 << 40, None) == 1
+    assert lib.nsa_backward_phi_params(ctypes.byref(lin), fake, fake, None, *out, fake, 1 << 40, None) == 1
+    assert lib.nsa_backward_phi_params(ctypes.byref(lin), fake, fake, phi, *out, fake, 64, None) == 3
+
+
 def test_decode_and_backward_validation_on_host(L):
     lib = L.lib()
     c = dict(I.WORKLOADS["decode_S32_L8k_64k"], B=32, T=65536)

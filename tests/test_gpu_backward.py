@@ -1,5 +1,6 @@
-"""GPU parity of nsa_backward against the fp64 oracle, with the same (valid,
-seeded) block selection on both sides.  Gradients: relative L2 <= 1e-2."""
+"""GPU parity of nsa_backward (and, for the linear phi, nsa_backward_phi_params)
+against the fp64 oracle, with the same (valid, seeded) block selection on both
+sides.  Gradients: relative L2 <= 1e-2."""
 import numpy as np
 import pytest
 import torch
@@ -15,13 +16,30 @@ def run_backward(c, t_lo=0):
     from sparse_attention_long_phi_b200 import nsa
     x = I.make_forward_inputs(c, "cuda", with_dout=True)
     idx = I.random_selection(c, "cuda")
-    r = nsa.backward(c, x["q"], x["k"], x["v"], x["gates"], x["dout"], idx, phi_params(x))
+    # the linear phi's parameter gradients need the complete dK~/dV~ (every row): t_lo = 0
+    phi_grads = c.get("phi") == "linear" and t_lo == 0
+    r = nsa.backward(c, x["q"], x["k"], x["v"], x["gates"], x["dout"], idx, phi_params(x),
+                     want_phi_grads=phi_grads)
     torch.cuda.synchronize()
     nsa.sync_status()
     hx = host(x)
     want = oracle.backward_tail(c, hx["q"], hx["k"], hx["v"], hx["gates"], hx["dout"],
                                 idx.cpu().numpy(), hx.get("wk"), hx.get("ek"), hx.get("wv"),
-                                hx.get("ev"), t_lo=t_lo)
+                                hx.get("ev"), t_lo=t_lo, want_cmp=phi_grads)
+    if phi_grads:
+        want.update(oracle.phi_param_grads(c, hx["k"], hx["v"], hx["wk"], hx["ek"], hx["wv"], hx["ev"],
+                                           want["dkc"], want["dvc"]))
+        for key in ("dwk", "dwv", "dev"):
+            got = r[key].cpu().numpy()
+            assert np.isfinite(got).all(), key
+            err = rel_l2(got, want[key])
+            assert err <= 1e-2, f"{key}: rel L2 {err:.3e}"
+        # E_K adds one vector, w_k vec(E_K), to every compressed key: the softmax does not
+        # see it, so dE_K is zero (each row's dS sums to zero).  The GPU's products take
+        # dS rounded to bf16, which leaves a residual of order 2^-9 of the terms
+        dek = r["dek"].cpu().numpy()
+        assert np.isfinite(dek).all()
+        assert np.abs(dek).max() <= 2e-3 * np.abs(want["dwk"]).max()
     for key in ("dq", "dk", "dv", "dgates"):
         got = r[key].cpu().numpy()[:, t_lo:]
         exp = want[key][:, t_lo:]

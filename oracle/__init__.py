@@ -62,6 +62,8 @@ def _load():
         lib.oracle_forward_rows.restype = None
         lib.oracle_forward_rows.argtypes = [pc, _P, _P, _P, _P, _P, _P, _I64, _P, _P, _P, _P, _P,
                                             _P, _P, _P]
+        lib.oracle_forward_rows_branches.restype = None
+        lib.oracle_forward_rows_branches.argtypes = [pc] + [_P] * 8 + [_I64] + [_P] * 8
         lib.oracle_key_counts.restype = None
         lib.oracle_key_counts.argtypes = [pc, _I64, _P]
         lib.oracle_decode.restype = ctypes.c_int
@@ -161,7 +163,8 @@ def phi(c: dict, k, v, wk=None, ek=None, wv=None, ev=None, exact: bool = False):
     return (kc, vc, kx, vx) if exact else (kc, vc)
 
 
-def forward_rows(c: dict, q, k, v, gates, kc, vc, rows, idx_in=None, want=("out", "idx", "lse")):
+def forward_rows(c: dict, q, k, v, gates, kc, vc, rows, idx_in=None, want=("out", "idx", "lse"),
+                 k_win=None, v_win=None):
     """Forward for the rows r = b*T + t listed in ``rows``.
 
     ``kc``/``vc`` are the compressed keys/values [B,C,G,*], as bf16 bits (the
@@ -171,6 +174,8 @@ def forward_rows(c: dict, q, k, v, gates, kc, vc, rows, idx_in=None, want=("out"
     log, cmp/slc/win), pgrp [R,G,Nsel] (group importance scores), pcmp [R,H,C]
     (compressed probabilities), obr [R,H,3,dv] (per-branch outputs).
     ``idx_in`` ([R,G,n]) replaces the oracle's selection for these rows.
+    ``k_win``/``v_win`` give the window branch its own keys/values (independent
+    K/V per branch); by default it reads k/v like the selected branch.
     """
     cf = make_cfg(c)
     rows = np.ascontiguousarray(rows, np.int64).reshape(-1)
@@ -186,8 +191,12 @@ def forward_rows(c: dict, q, k, v, gates, kc, vc, rows, idx_in=None, want=("out"
         res["pcmp"] = np.zeros((R, cf.H, max(C, 1)))
     if "obr" in want:
         res["obr"] = np.zeros((R, cf.H, 3, cf.dv))
-    _load().oracle_forward_rows(
-        ctypes.byref(cf), _ptr(_c(q, np.uint16)), _ptr(_c(k, np.uint16)), _ptr(_c(v, np.uint16)),
+    kb, vb = _c(k, np.uint16), _c(v, np.uint16)
+    kw = kb if k_win is None else _c(k_win, np.uint16)
+    vw = vb if v_win is None else _c(v_win, np.uint16)
+    assert kw.shape == kb.shape and vw.shape == vb.shape
+    _load().oracle_forward_rows_branches(
+        ctypes.byref(cf), _ptr(_c(q, np.uint16)), _ptr(kb), _ptr(vb), _ptr(kw), _ptr(vw),
         _ptr(_c(gates, np.float32)), _ptr(_vals(kc)), _ptr(_vals(vc)), R,
         _ptr(rows), _ptr(_c(idx_in, np.int32)), _ptr(res["out"]), _ptr(res["idx"]),
         _ptr(res.get("lse")), _ptr(res.get("pgrp")), _ptr(res.get("pcmp")), _ptr(res.get("obr")))

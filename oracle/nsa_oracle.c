@@ -330,7 +330,8 @@ void oracle_topn(const ocfg_t* c, int64_t nrows, const int64_t* rows, const doub
  * out [nrows,H,dv] = g_cmp o_cmp + g_slc o_slc + g_win o_win (final output
  * computation paragraph; gated-fusion section of the explainer). */
 static void forward_rows_impl(const ocfg_t* c, const uint16_t* q, const uint16_t* k,
-                              const uint16_t* v, const float* gates, int64_t qrow0,
+                              const uint16_t* v, const uint16_t* kw, const uint16_t* vw,
+                              const float* gates, int64_t qrow0,
                               const double* kc, const double* vc, int64_t nrows,
                               const int64_t* rows, const int32_t* idx_in, double* out,
                               int32_t* idx_out, double* lse, double* pgrp, double* pcmp,
@@ -397,7 +398,9 @@ static void forward_rows_impl(const ocfg_t* c, const uint16_t* q, const uint16_t
                 double l1 = attend(c->dk, c->dv, sc, qv, K, V, c->G * c->dk, c->G * c->dv, keys, nk,
                                    p, ob + c->dv);
                 nk = win_keys(c, t, keys);
-                double l2 = attend(c->dk, c->dv, sc, qv, K, V, c->G * c->dk, c->G * c->dv, keys, nk,
+                const uint16_t* KW = kw + (b * c->T * c->G + g) * c->dk;
+                const uint16_t* VW = vw + (b * c->T * c->G + g) * c->dv;
+                double l2 = attend(c->dk, c->dv, sc, qv, KW, VW, c->G * c->dk, c->G * c->dv, keys, nk,
                                    p, ob + 2 * c->dv);
                 if (lse) {
                     lse[(a * c->H + h) * 3 + 1] = l1;
@@ -429,7 +432,23 @@ void oracle_forward_rows(const ocfg_t* c, const uint16_t* q, const uint16_t* k, 
                          int64_t nrows, const int64_t* rows, const int32_t* idx_in, double* out,
                          int32_t* idx_out, double* lse, double* pgrp, double* pcmp, double* obr)
 {
-    forward_rows_impl(c, q, k, v, gates, 0, kc, vc, nrows, rows, idx_in, out, idx_out, lse, pgrp,
+    forward_rows_impl(c, q, k, v, k, v, gates, 0, kc, vc, nrows, rows, idx_in, out, idx_out, lse, pgrp,
+                      pcmp, obr);
+}
+
+/* The same rows with independent keys/values per branch (page 2, sliding-window
+ * paragraph: the branches keep separate keys and values so that the window
+ * branch's local patterns do not shortcut the other two): the compressed
+ * branch reads kc/vc (phi of its own k/v, computed by the caller), the
+ * selected branch k/v, the window branch kw/vw ([B,T,G,*] bf16 each).  The
+ * selection still comes from the compressed branch's probabilities. */
+void oracle_forward_rows_branches(const ocfg_t* c, const uint16_t* q, const uint16_t* k,
+                                  const uint16_t* v, const uint16_t* kw, const uint16_t* vw,
+                                  const float* gates, const double* kc, const double* vc, int64_t nrows,
+                                  const int64_t* rows, const int32_t* idx_in, double* out,
+                                  int32_t* idx_out, double* lse, double* pgrp, double* pcmp, double* obr)
+{
+    forward_rows_impl(c, q, k, v, kw, vw, gates, 0, kc, vc, nrows, rows, idx_in, out, idx_out, lse, pgrp,
                       pcmp, obr);
 }
 
@@ -488,6 +507,7 @@ int oracle_decode(const ocfg_t* c0, int64_t S, const uint16_t* q, const uint16_t
         for (int64_t e = 0; e < nc * c.G * c.dk; ++e) kcd[e] = bf(kccache[cmp_off[s] * c.G * c.dk + e]);
         for (int64_t e = 0; e < nc * c.G * c.dv; ++e) vcd[e] = bf(vccache[cmp_off[s] * c.G * c.dv + e]);
         forward_rows_impl(&c, q + s * c.H * c.dk, kcache + kv_off[s] * c.G * c.dk,
+                          vcache + kv_off[s] * c.G * c.dv, kcache + kv_off[s] * c.G * c.dk,
                           vcache + kv_off[s] * c.G * c.dv, gates + s * c.H * 3, t, kcd, vcd, 1,
                           &row, NULL, out + s * c.H * c.dv, idx + s * c.G * c.n,
                           lse ? lse + s * c.H * 3 : NULL, pg, NULL, NULL);

@@ -300,6 +300,33 @@ def test_one_hot_gates_isolate_branches():
 
 # ------------------------------------------------------ pages' token counts
 
+def test_independent_window_keys_and_values():
+    # page 2, sliding-window paragraph: the window branch may keep its own keys/values
+    c = small_cfg(T=96, lp=16, n=6, w=96)                  # w >= T: the window sees every u <= t
+    x = make(c)
+    kw = I.bits(I.normal_bf16(99, 1, (1, 96, 2, 16)))
+    vw = I.bits(I.normal_bf16(99, 2, (1, 96, 2, 8)))
+    kc, vc = oracle.phi(c, x["k"], x["v"])
+    rows = np.arange(96)
+    want = ("out", "idx", "lse", "obr", "pgrp")
+    same = oracle.forward_rows(c, x["q"], x["k"], x["v"], x["gates"], kc, vc, rows, want=want,
+                               k_win=x["k"], v_win=x["v"])
+    base = oracle.forward_rows(c, x["q"], x["k"], x["v"], x["gates"], kc, vc, rows, want=want)
+    for key in want:                                       # passing the shared k/v changes nothing
+        np.testing.assert_array_equal(same[key], base[key])
+    sep = oracle.forward_rows(c, x["q"], x["k"], x["v"], x["gates"], kc, vc, rows, want=want,
+                              k_win=kw, v_win=vw)
+    # the window branch is full causal attention over its own keys/values (library)
+    ref = full_causal(f64(x["q"]), f64(kw), f64(vw), 1 / 4.0).reshape(-1, 4, 8)
+    np.testing.assert_allclose(sep["obr"][:, :, 2], ref, atol=1e-12)
+    # the compressed and selected branches, the scores and the selection do not see them
+    np.testing.assert_array_equal(sep["obr"][:, :, :2], base["obr"][:, :, :2])
+    np.testing.assert_array_equal(sep["idx"], base["idx"])
+    np.testing.assert_array_equal(sep["pgrp"], base["pgrp"])
+    np.testing.assert_array_equal(sep["lse"][:, :, :2], base["lse"][:, :, :2])
+    assert not np.allclose(sep["obr"][:, :, 2], base["obr"][:, :, 2])
+
+
 def test_token_counts_reproduce_the_pages_numbers():
     gold = json.load(open(os.path.join(HERE, "golden", "page_numbers.json")))
     hp = {k: gold["hyperparameters"][k] for k in ("l", "d", "lp", "n", "fi", "fl", "w")}

@@ -99,3 +99,15 @@ def test_throttled_region_is_measured_again(monkeypatch):
 def test_warmup_below_three_is_refused(monkeypatch):
     with pytest.raises(AssertionError):
         _run(monkeypatch, [CLEAN], ["--no-extras", "--steps", "20", "--warmup", "2"])
+
+
+def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
+    # under torchrun every rank but 0 leaves at once, without work or output
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--steps", "2", "--warmup", "3"])
+    monkeypatch.setattr(I, "make_forward_inputs", lambda *a, **k: pytest.fail("rank 1 did work"))
+    out = io.StringIO()
+    with contextlib.redirect_stdout(out):
+        bench.main()
+    assert out.getvalue() == ""

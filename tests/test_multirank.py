@@ -1,6 +1,8 @@
-"""The benchmark's multi-rank bookkeeping on CPU (gloo, world size 2): every
-rank processes its own sequence (no data-path collective); the job time is
-the slowest rank's, and the whole-job throughput counts all ranks' tokens."""
+"""Multi-rank paths on CPU (gloo, world size 2): the benchmark's bookkeeping
+(every rank processes its own sequence, no data-path collective; the job time is
+the slowest rank's, the whole-job throughput counts all ranks' tokens; a
+re-measurement decided by any rank is taken by all), and sharding one sequence
+by GQA group, which needs no exchange and reproduces the single-rank result."""
 import os
 import socket
 
@@ -62,3 +64,62 @@ def test_clock_records_that_force_a_second_measurement():
     assert not bench.clocks_rejected({"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]})
     assert bench.any_rank(True) and not bench.any_rank(False)
 
+
+
+def _group_worker(rank, world, port, q):
+    import numpy as np
+
+    import oracle
+    from sparse_attention_long_phi_b200 import inputs as I
+    from sparse_attention_long_phi_b200 import shard
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        c = dict(B=1, T=200, H=8, G=4, dk=16, dv=8, l=8, d=4, lp=16, n=4, fi=1, fl=2, w=24,
+                 phi="linear", seed=21)
+        x = {k: (I.bits(v) if v.dtype == torch.bfloat16 else v.numpy())
+             for k, v in I.make_forward_inputs(c, "cpu").items()}
+        g0, g1 = shard.group_range(c["G"], rank, world)
+        cs, xs = shard.slice_groups(c, x, g0, g1)
+        kc, vc = oracle.phi(cs, xs["k"], xs["v"], xs["wk"], xs["ek"], xs["wv"], xs["ev"])
+        r = oracle.forward_rows(cs, xs["q"], xs["k"], xs["v"], xs["gates"], kc, vc, np.arange(200))
+        parts = [None] * world
+        dist.all_gather_object(parts, (g0, g1, r["out"], r["idx"]))   # no data-path exchange: results only
+        if rank == 0:
+            kc, vc = oracle.phi(c, x["k"], x["v"], x["wk"], x["ek"], x["wv"], x["ev"])
+            full = oracle.forward_rows(c, x["q"], x["k"], x["v"], x["gates"], kc, vc, np.arange(200))
+            out = np.concatenate([p[2] for p in parts], axis=1)
+            idx = np.concatenate([p[3] for p in parts], axis=1)
+            q.put((np.array_equal(out, full["out"]), np.array_equal(idx, full["idx"]),
+                   [p[:2] for p in parts]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_group_sharding_is_exact_with_two_gloo_ranks():
+    # the operator splits by GQA group with no exchange: two ranks' outputs, concatenated
+    # along the heads, are bit for bit the single-rank result (fp64 oracle as the compute)
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_group_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(180)
+        assert p.exitcode == 0
+    same_out, same_idx, ranges = q.get(timeout=10)
+    assert ranges == [(0, 2), (2, 4)]
+    assert same_out and same_idx
+
+
+def test_group_ranges_cover_every_group_once():
+    from sparse_attention_long_phi_b200 import shard
+    for G in (1, 2, 3, 4, 7, 8):
+        for world in range(1, G + 1):
+            rs = [shard.group_range(G, r, world) for r in range(world)]
+            assert rs[0][0] == 0 and rs[-1][1] == G
+            assert all(a[1] == b[0] for a, b in zip(rs, rs[1:]))
+            assert max(g1 - g0 for g0, g1 in rs) - min(g1 - g0 for g0, g1 in rs) <= 1
+    with pytest.raises(ValueError):
+        shard.group_range(2, 0, 3)

@@ -123,3 +123,16 @@ def test_group_ranges_cover_every_group_once():
             assert max(g1 - g0 for g0, g1 in rs) - min(g1 - g0 for g0, g1 in rs) <= 1
     with pytest.raises(ValueError):
         shard.group_range(2, 0, 3)
+
+
+def test_slice_groups_on_torch_tensors():
+    from sparse_attention_long_phi_b200 import inputs as I
+    from sparse_attention_long_phi_b200 import shard
+    c = dict(I.WORKLOADS["prefill_fwd_T8192"], T=64)
+    x = I.make_forward_inputs(c, "cpu", with_dout=True)
+    cs, xs = shard.slice_groups(c, x, 1, 3)
+    assert (cs["G"], cs["H"]) == (2, 32)
+    assert xs["q"].shape == (1, 64, 32, 192) and xs["q"].is_contiguous()
+    assert torch.equal(xs["q"], x["q"][:, :, 16:48]) and torch.equal(xs["k"], x["k"][:, :, 1:3])
+    assert torch.equal(xs["gates"], x["gates"][:, :, 16:48]) and torch.equal(xs["dout"], x["dout"][:, :, 16:48])
+    assert xs["wk"] is x["wk"]                       # the phi parameters are shared by every group

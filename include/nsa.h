@@ -119,9 +119,9 @@ nsa_status_t nsa_compress(const nsa_config_t* cfg, const void* k, const void* v,
  *     bytes must fit in 16 MiB, otherwise NSA_ERR_WORKSPACE is returned and
  *     nothing is launched (e.g. B=1, G=4, d_k+d_v=320 allows up to about
  *     T=52k tokens);
- *   - the first call on a device looks up the array's device address (once
- *     per device, with that device current); make that first call before
- *     any stream capture;
+ *   - every call looks up the array's device address on the current device
+ *     (a host-side query); the first call on a device may load the library's
+ *     device code there, so make that first call before any stream capture;
  *   - all calls share the array: two calls whose kernels overlap on the GPU
  *     (different streams, or different host threads on one device) race;
  *     serialise them.  Each call clears the counters it needs.
@@ -141,6 +141,19 @@ nsa_status_t nsa_forward(const nsa_config_t* cfg, const void* q, const void* k, 
                          const float* gates, const nsa_phi_params_t* phi, float* out,
                          int32_t* sel_idx, float* lse, void* kc_out, void* vc_out,
                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* Where nsa_forward leaves the group importance scores (page 2, 重要性分数计算:
+ * the compressed branch's probabilities mapped onto selection blocks by the
+ * overlap weights and summed over the heads of a GQA group), the table the
+ * top-n step reads.  Returns the byte offset of the table inside the FORWARD
+ * workspace, or -1 for an invalid cfg; *row_stride (if not NULL) receives NSp,
+ * the padded number of selection blocks per row.  After an nsa_forward call
+ * with this cfg has completed, p'[b,t,g,j] is the fp32 at
+ * workspace + offset + 4*(((b*T + t)*G + g)*NSp + j) for every block
+ * j <= floor(t / sel_block) of a row that sees at least one compressed block
+ * (t >= cmp_block - 1); other entries are unspecified.  The table stays valid
+ * until the workspace is reused.  No device work, no CUDA call. */
+int64_t nsa_forward_score_table(const nsa_config_t* cfg, int64_t* row_stride);
 
 /* Batched decode step (page 2, 效率分析 解码速度): one query per sequence at
  * position t = L_s - 1 over caches that already hold the current token.
@@ -235,6 +248,17 @@ nsa_status_t nsa_select_blocks(const nsa_config_t* cfg, const float* scores, int
 nsa_status_t nsa_backward_phi_params(const nsa_config_t* cfg, const void* k, const void* v,
                                      const nsa_phi_params_t* phi, float* dw_k, float* de_k, float* dw_v,
                                      float* de_v, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Failure-detection self-test: launches one kernel whose single waiting thread
+ * waits, through the same bounded wait every libnsa kernel uses, on an
+ * mbarrier on which nothing ever arrives.  After limit_ns nanoseconds of device
+ * time (1 .. 2e9) the wait gives up, records its site in the device error word
+ * and the kernel returns normally: the next nsa_sync_status() on that stream
+ * reports NSA_ERR_DEVICE_TIMEOUT and clears the word, and the CUDA context
+ * stays usable.  No fault, trap or hang is involved.  NSA_ERR_INVALID_ARG for a
+ * limit outside that range.  Not part of the pages' operator: it lets a caller
+ * (and the test suite) check that an expired wait is reported. */
+nsa_status_t nsa_check_timeout_path(uint64_t limit_ns, void* stream);
 
 /* Synchronise `stream`, then read and clear the device error word of the
  * current device.  Returns NSA_ERR_DEVICE_TIMEOUT if a kernel's bounded wait

@@ -70,6 +70,8 @@ def _load():
         lib.oracle_decode.argtypes = [pc, _I64] + [_P] * 12 + [_I64]
         lib.oracle_backward_tail.restype = None
         lib.oracle_backward_tail.argtypes = [pc] + [_P] * 10 + [_I64] + [_P] * 6
+        lib.oracle_backward_rows.restype = None
+        lib.oracle_backward_rows.argtypes = [pc] + [_P] * 10 + [_I64] + [_P] * 7
         lib.oracle_phi_param_grads.restype = None
         lib.oracle_phi_param_grads.argtypes = [pc, _I64] + [_P] * 6
         lib.oracle_num_threads.restype = ctypes.c_int
@@ -260,6 +262,34 @@ def backward_tail(c: dict, q, k, v, gates, dout, idx, wk=None, ek=None, wv=None,
         _ptr(_c(gates, np.float32)), _ptr(_c(wk, np.uint16)), _ptr(_c(ek, np.uint16)),
         _ptr(_c(wv, np.uint16)), _ptr(_c(ev, np.uint16)), _ptr(_c(dout, np.uint16)),
         _ptr(_c(idx, np.int32)), int(t_lo), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dkc), _ptr(dvc))
+    out = {"dq": dq, "dk": dk, "dv": dv, "dgates": dg}
+    if want_cmp:
+        out.update(dkc=dkc, dvc=dvc)
+    return out
+
+
+def backward_rows(c: dict, q, k, v, gates, dout, idx, rows, wk=None, ek=None, wv=None, ev=None,
+                  want_cmp: bool = False):
+    """Backward restricted to the query rows r = b*T + t in ``rows``: the gradient of the
+    sum over those rows of <dout, out> (rows outside contribute nothing, as if their dout
+    were zero).  Same outputs as backward_tail; dq/dgates are zero outside the listed rows,
+    dk/dv/dkc/dvc hold the listed rows' contributions at every key position."""
+    cf = make_cfg(c)
+    B, T, H, G = cf.B, cf.T, cf.H, cf.G
+    C = num_cmp_blocks(c, T)
+    rows = np.ascontiguousarray(rows, np.int64).reshape(-1)
+    dq = np.zeros((B, T, H, cf.dk))
+    dk = np.zeros((B, T, G, cf.dk))
+    dv = np.zeros((B, T, G, cf.dv))
+    dg = np.zeros((B, T, H, 3))
+    dkc = np.zeros((B, C, G, cf.dk)) if want_cmp else None
+    dvc = np.zeros((B, C, G, cf.dv)) if want_cmp else None
+    _load().oracle_backward_rows(
+        ctypes.byref(cf), _ptr(_c(q, np.uint16)), _ptr(_c(k, np.uint16)), _ptr(_c(v, np.uint16)),
+        _ptr(_c(gates, np.float32)), _ptr(_c(wk, np.uint16)), _ptr(_c(ek, np.uint16)),
+        _ptr(_c(wv, np.uint16)), _ptr(_c(ev, np.uint16)), _ptr(_c(dout, np.uint16)),
+        _ptr(_c(idx, np.int32)), int(rows.size), _ptr(rows), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg),
+        _ptr(dkc), _ptr(dvc))
     out = {"dq": dq, "dk": dk, "dv": dv, "dgates": dg}
     if want_cmp:
         out.update(dkc=dkc, dvc=dvc)

@@ -546,11 +546,12 @@ int oracle_decode(const ocfg_t* c0, int64_t S, const uint16_t* q, const uint16_t
  * t >= t_lo; entries below t_lo hold partial sums.  t_lo = 0 is the full
  * backward.  Outputs (fp64, zeroed here): dq [B,T,H,dk], dk [B,T,G,dk],
  * dv [B,T,G,dv], dgates [B,T,H,3].  idx [B,T,G,n]. */
-void oracle_backward_tail(const ocfg_t* c, const uint16_t* q, const uint16_t* k,
+static void backward_core(const ocfg_t* c, const uint16_t* q, const uint16_t* k,
                           const uint16_t* v, const float* gates, const uint16_t* wk,
                           const uint16_t* ek, const uint16_t* wv, const uint16_t* ev,
-                          const uint16_t* dout, const int32_t* idx, int64_t t_lo, double* dq,
-                          double* dk, double* dv, double* dgates, double* dkc_out, double* dvc_out)
+                          const uint16_t* dout, const int32_t* idx, int64_t t_lo,
+                          const uint8_t* row_on, double* dq, double* dk, double* dv,
+                          double* dgates, double* dkc_out, double* dvc_out)
 {
     const int64_t B = c->B, T = c->T, H = c->H, G = c->G, dK = c->dk, dV = c->dv;
     const int64_t C = oracle_num_cmp_blocks(c, T);
@@ -586,6 +587,7 @@ void oracle_backward_tail(const ocfg_t* c, const uint16_t* q, const uint16_t* k,
             double* dO = (double*)malloc(sizeof(double) * (size_t)dV);
             for (int64_t t = (t_lo > 0 ? t_lo : 0); t < T; ++t) {
                 const int64_t r = b * T + t;
+                if (row_on && !row_on[r]) continue;
                 for (int64_t hh = 0; hh < Hg; ++hh) {
                     const int64_t h = g * Hg + hh;
                     load_q(c, q, r, h, qv);
@@ -674,6 +676,37 @@ void oracle_backward_tail(const ocfg_t* c, const uint16_t* q, const uint16_t* k,
     free(vc);
     free(dkc);
     free(dvc);
+}
+
+void oracle_backward_tail(const ocfg_t* c, const uint16_t* q, const uint16_t* k,
+                          const uint16_t* v, const float* gates, const uint16_t* wk,
+                          const uint16_t* ek, const uint16_t* wv, const uint16_t* ev,
+                          const uint16_t* dout, const int32_t* idx, int64_t t_lo, double* dq,
+                          double* dk, double* dv, double* dgates, double* dkc_out, double* dvc_out)
+{
+    backward_core(c, q, k, v, gates, wk, ek, wv, ev, dout, idx, t_lo, NULL, dq, dk, dv, dgates,
+                  dkc_out, dvc_out);
+}
+
+/* The same backward restricted to the query rows r = b*T + t listed in
+ * rows[0 .. nrows): the gradient of sum over the listed rows of <dout, out>,
+ * i.e. every row outside the list contributes nothing (as if its dout were
+ * zero).  dq/dgates are those of the listed rows (zero elsewhere); dk, dv and
+ * the compressed-key gradients sum the listed rows' contributions over every
+ * key they read, at any position.  Outputs as oracle_backward_tail. */
+void oracle_backward_rows(const ocfg_t* c, const uint16_t* q, const uint16_t* k,
+                          const uint16_t* v, const float* gates, const uint16_t* wk,
+                          const uint16_t* ek, const uint16_t* wv, const uint16_t* ev,
+                          const uint16_t* dout, const int32_t* idx, int64_t nrows,
+                          const int64_t* rows, double* dq, double* dk, double* dv,
+                          double* dgates, double* dkc_out, double* dvc_out)
+{
+    uint8_t* on = (uint8_t*)calloc((size_t)(c->B * c->T), 1);
+    for (int64_t a = 0; a < nrows; ++a)
+        if (rows[a] >= 0 && rows[a] < c->B * c->T) on[rows[a]] = 1;
+    backward_core(c, q, k, v, gates, wk, ek, wv, ev, dout, idx, 0, on, dq, dk, dv, dgates,
+                  dkc_out, dvc_out);
+    free(on);
 }
 
 /* Gradients of the linear phi's parameters (token compression: K~[i] =

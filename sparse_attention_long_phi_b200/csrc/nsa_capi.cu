@@ -302,6 +302,19 @@ nsa_status_t run_phi(const Shape& s, const void* k, const void* v, const nsa_phi
     return launch_phi_linear<64>(s, v, phi->w_v, phi->e_v, bias + s.DK, vc, vcT, lv, cnt + 1, st);
 }
 
+// Failure-detection self-test: lane 0 waits, through the same bounded wait
+// every kernel uses, on an mbarrier on which nothing ever arrives.  The wait
+// expires after limit_ns, records its site in the device error word and the
+// kernel returns; the other lanes return at once (no CTA barrier follows).
+constexpr unsigned kSiteSelftest = 0x7F0;
+__global__ void timeout_selftest_kernel(unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    (void)mbar_wait_for(&bar, 0, kSiteSelftest, limit_ns);
+}
+
 __global__ void cmp_empty_kernel(float* out, float* lse, long long rows, int DV) {
     long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i < rows * DV) out[i] = 0.f;
@@ -729,6 +742,13 @@ size_t nsa_workspace_size(const nsa_config_t* cfg, int32_t mode) {
     return 0;
 }
 
+int64_t nsa_forward_score_table(const nsa_config_t* cfg, int64_t* row_stride) {
+    Shape s;
+    if (derive(cfg, s) != NSA_OK) return -1;
+    if (row_stride) *row_stride = s.NSp;
+    return (int64_t)fwd_layout(s).off_ps;
+}
+
 nsa_status_t nsa_compress(const nsa_config_t* cfg, const void* k, const void* v,
                           const nsa_phi_params_t* phi, void* kc, void* vc, void* workspace,
                           size_t workspace_bytes, void* stream) {
@@ -1006,6 +1026,13 @@ nsa_status_t nsa_backward_phi_params(const nsa_config_t* cfg, const void* k, con
     return last_launch();
 }
 
+nsa_status_t nsa_check_timeout_path(uint64_t limit_ns, void* stream) {
+    if (limit_ns == 0 || limit_ns > kWaitLimitNs) return NSA_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    NSA_LAUNCH("timeout_selftest_kernel", st, timeout_selftest_kernel<<<1, 32, 0, st>>>(limit_ns));
+    return last_launch();
+}
+
 nsa_status_t nsa_sync_status(void* stream) {
     if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return NSA_ERR_CUDA;
     unsigned int v = 0;
@@ -1026,26 +1053,18 @@ nsa_status_t nsa_sync_status(void* stream) {
 // device memory.  Its scratch (the fp64 position-embedding bias and the list
 // of elements re-rounded exactly) lives in the fixed array below instead of a
 // caller workspace.  The array is a host-side stand-in in host code; its
-// device address is fetched with cudaGetSymbolAddress once per device, the
-// first time the entry point runs with that device current.
+// device address on the current device is looked up with cudaGetSymbolAddress
+// on every call (a host-side query, cheap once the module is loaded), so a
+// context that was torn down and re-created never sees a stale address.
 namespace {
 
 constexpr size_t kStaticScratchBytes = size_t(16) << 20;   // 16 MiB on every device that loads the library
 __device__ __align__(256) uint8_t g_compress_scratch[kStaticScratchBytes];
 
-std::mutex g_static_mu;
-void* g_static_scratch[128] = {};
-
 nsa_status_t static_scratch_ptr(void** out) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return NSA_ERR_CUDA;
-    std::lock_guard<std::mutex> lk(g_static_mu);
-    if (!g_static_scratch[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_compress_scratch) != cudaSuccess || !p) return NSA_ERR_CUDA;
-        g_static_scratch[dev] = p;
-    }
-    *out = g_static_scratch[dev];
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_compress_scratch) != cudaSuccess || !p) return NSA_ERR_CUDA;
+    *out = p;
     return NSA_OK;
 }
 

@@ -70,17 +70,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity to complete.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned site) {
+// Bounded wait for the phase with the given parity to complete: gives up after
+// limit_ns of device time (or, as a backstop, 2^30 polls), records `site` in
+// the error word and returns false.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, unsigned site,
+                                              unsigned long long limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     for (uint32_t it = 0;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 63u && globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (((it & 63u) == 63u && globaltimer_ns() - t0 > limit_ns) || it == (1u << 30)) {
             record_timeout(site);
             return false;
         }
     }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned site) {
+    return mbar_wait_for(bar, parity, site, kWaitLimitNs);
 }
 
 // Programmatic dependent launch: let the next kernel on the stream begin its

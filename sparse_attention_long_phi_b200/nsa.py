@@ -61,6 +61,8 @@ def lib():
         L.nsa_workspace_size.argtypes = [pc, ctypes.c_int32]
         L.nsa_num_cmp_blocks.restype = ctypes.c_int64
         L.nsa_num_cmp_blocks.argtypes = [pc, ctypes.c_int64]
+        L.nsa_forward_score_table.restype = ctypes.c_int64
+        L.nsa_forward_score_table.argtypes = [pc, ctypes.POINTER(ctypes.c_int64)]
         L.nsa_compress.restype = ctypes.c_int
         L.nsa_compress.argtypes = [pc, _P, _P, pp, _P, _P, _P, ctypes.c_size_t, _P]
         L.nsa_compress_static.restype = ctypes.c_int
@@ -80,6 +82,8 @@ def lib():
                                    ctypes.c_size_t, _P]
         L.nsa_backward_phi_params.restype = ctypes.c_int
         L.nsa_backward_phi_params.argtypes = [pc, _P, _P, pp, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+        L.nsa_check_timeout_path.restype = ctypes.c_int
+        L.nsa_check_timeout_path.argtypes = [ctypes.c_uint64, _P]
         L.nsa_sync_status.restype = ctypes.c_int
         L.nsa_sync_status.argtypes = [_P]
         L.nsa_profile_enable.restype = ctypes.c_int
@@ -172,12 +176,29 @@ def forward_into(c: dict, q, k, v, gates, phi, buf: ForwardBuffers, stream=None)
         _p(buf.lse), _p(buf.kc), _p(buf.vc), _p(buf.ws), buf.ws.numel(), _stream(stream)))
 
 
-def forward(c: dict, q, k, v, gates, phi=None, want_lse=True, want_kc=False, stream=None) -> dict:
+def score_table(c: dict, ws: torch.Tensor) -> torch.Tensor:
+    """View of the group importance-score table [B,T,G,NSp] fp32 that nsa_forward leaves in
+    its workspace `ws` (valid for blocks j <= t // l' of rows t >= l - 1)."""
+    stride = ctypes.c_int64(0)
+    off = int(lib().nsa_forward_score_table(ctypes.byref(make_config(c)), ctypes.byref(stride)))
+    if off < 0:
+        raise NsaError("nsa_forward_score_table", 1)
+    B, T, G = c["B"], c["T"], c["G"]
+    n = B * T * G * stride.value
+    return ws[off:off + 4 * n].view(torch.float32).view(B, T, G, stride.value)
+
+
+def forward(c: dict, q, k, v, gates, phi=None, want_lse=True, want_kc=False, stream=None,
+            want_scores=False) -> dict:
     """Prefill forward.  q [B,T,H,dk], k [B,T,G,dk], v [B,T,G,dv] bf16; gates [B,T,H,3] fp32;
-    phi = dict(wk, ek, wv, ev) for the linear map.  Returns out, idx, lse, kc, vc."""
+    phi = dict(wk, ek, wv, ev) for the linear map.  Returns out, idx, lse, kc, vc (and with
+    want_scores the importance-score table left in the workspace)."""
     buf = forward_buffers(c, q.device, want_lse, want_kc)
     forward_into(c, q, k, v, gates, phi, buf, stream)
-    return {"out": buf.out, "idx": buf.idx, "lse": buf.lse, "kc": buf.kc, "vc": buf.vc}
+    res = {"out": buf.out, "idx": buf.idx, "lse": buf.lse, "kc": buf.kc, "vc": buf.vc}
+    if want_scores:
+        res["scores"] = score_table(c, buf.ws)
+    return res
 
 
 def compress(c: dict, k, v, phi=None, stream=None):
@@ -297,6 +318,12 @@ def backward(c: dict, q, k, v, gates, dout, idx, phi=None, stream=None, want_phi
             ctypes.byref(cfg), _p(k), _p(v), _phi(phi), _p(res["dwk"]), _p(res["dek"]), _p(res["dwv"]),
             _p(res["dev"]), _p(ws), ws.numel(), _stream(stream)))
     return res
+
+
+def check_timeout_path(limit_ns: int = 1_000_000, stream=None):
+    """Launch the failure-detection self-test: a bounded wait that nothing satisfies
+    expires after limit_ns; the next sync_status() raises NsaError (device timeout)."""
+    _check("nsa_check_timeout_path", lib().nsa_check_timeout_path(int(limit_ns), _stream(stream)))
 
 
 def sync_status(stream=None):

@@ -67,8 +67,49 @@ def phi_params(x):
     return {k: x[k] for k in ("wk", "ek", "wv", "ev")} if "wk" in x else None
 
 
-def selection_ok(c, q_row, pg, got, want, delta):
-    """GPU index row `got` vs oracle `want` for one (row, group); pg = oracle scores."""
+def selection_valid(c, t, row):
+    """Structural check of one selected-block row for query token t (page 2,
+    Top-n 块选择 and its hyperparameter paragraph): min(n, b_t + 1) indices in
+    [0, b_t], strictly ascending, then -1 padding; when more than n candidates
+    exist the forced blocks 0 .. fi-1 and b_t-fl+1 .. b_t are among them.
+    Returns None when valid, else a reason string."""
+    n, lp = c["n"], c["lp"]
+    fi, fl = c.get("fi", 1), c.get("fl", 2)
+    bt = int(t) // lp
+    row = [int(j) for j in row]
+    cnt = min(n, bt + 1)
+    head, tail = row[:cnt], row[cnt:]
+    if any(j != -1 for j in tail):
+        return f"padding {tail}"
+    if any(j < 0 or j > bt for j in head):
+        return f"index outside [0, {bt}]: {head}"
+    if any(head[a] >= head[a + 1] for a in range(len(head) - 1)):
+        return f"not strictly ascending: {head}"
+    if bt + 1 > n:
+        forced = set(range(min(fi, bt + 1))) | set(range(max(0, bt - fl + 1), bt + 1))
+        if not forced <= set(head):
+            return f"forced blocks {sorted(forced - set(head))} missing"
+    return None
+
+
+def selections_valid(c, ts, idx):
+    """selection_valid over rows: ts [R] token positions, idx [R, G, n]; asserts."""
+    bad = []
+    for a in range(len(ts)):
+        for g in range(idx.shape[1]):
+            why = selection_valid(c, ts[a], idx[a, g])
+            if why:
+                bad.append((int(ts[a]), g, why))
+    assert not bad, f"{len(bad)} invalid selection rows, e.g. {bad[:3]}"
+
+
+def selection_ok(c, t, pg, got, want, delta):
+    """GPU index row `got` vs oracle `want` for token t of one group; pg = the
+    oracle's group scores.  The GPU row must be a valid selection; where the
+    sets differ, every block only the GPU chose must score at least (1 - eps)
+    x every block only the oracle chose (a near-tie)."""
+    if selection_valid(c, t, got) is not None:
+        return False
     A = set(int(j) for j in got if j >= 0) - set(int(j) for j in want if j >= 0)
     B = set(int(j) for j in want if j >= 0) - set(int(j) for j in got if j >= 0)
     if not A and not B:
@@ -79,13 +120,51 @@ def selection_ok(c, q_row, pg, got, want, delta):
     return min(pg[j] for j in A) >= max(pg[j] for j in B) * (1 - eps)
 
 
+def near_tie_bound(pairs):
+    """Largest number of (row, group) selections allowed to differ at a near-tie:
+    fp32 against fp64 scores flips the order of two blocks only when their
+    scores agree to about 1e-6, so such rows must stay rare."""
+    return max(2, pairs // 200)
+
+
+def check_scores(c, table, rows, pgrp, report=None, rtol=2e-5):
+    """Importance-score table left by nsa_forward (fp32, from the compressed
+    branch's probabilities) against the oracle's fp64 group scores p', for every
+    candidate block j <= t // l' of the rows that see a compressed block.  Both
+    sides use the same bf16 compressed keys (phi is correctly rounded), so the
+    difference is fp32 arithmetic: logits accumulated over d_k products, one
+    exp2 per probability, sums over the heads and the overlap taps.  Each entry
+    must agree within rtol of the row's largest score."""
+    B, T, G = c["B"], c["T"], c["G"]
+    lp, l = c["lp"], c["l"]
+    tab = table.reshape(B * T, G, -1).cpu().numpy()[rows]
+    worst, checked = 0.0, 0
+    for a, r in enumerate(rows):
+        t = int(r) % T
+        if t < l - 1:
+            continue
+        nb = t // lp + 1
+        got = tab[a, :, :nb].astype(np.float64)
+        want = pgrp[a, :, :nb]
+        assert np.isfinite(got).all(), f"score row {int(r)} not finite"
+        scale = np.maximum(want.max(axis=1, keepdims=True), 1e-30)
+        err = float((np.abs(got - want) / scale).max())
+        worst = max(worst, err)
+        checked += 1
+    assert worst <= rtol, f"importance scores: max error {worst:.3e} of the row maximum"
+    if report is not None:
+        report.update(score_rows=checked, score_err=worst)
+    return worst
+
+
 def check_forward(c: dict, rows=None, device="cuda", x=None, report=None):
     """Run nsa_forward on the workload, compare with the oracle on `rows`."""
     from sparse_attention_long_phi_b200 import nsa
     B, T, H, G, n = c["B"], c["T"], c["H"], c["G"], c["n"]
     if x is None:
         x = I.make_forward_inputs(c, device)
-    r = nsa.forward(c, x["q"], x["k"], x["v"], x["gates"], phi_params(x), want_lse=True, want_kc=True)
+    r = nsa.forward(c, x["q"], x["k"], x["v"], x["gates"], phi_params(x), want_lse=True, want_kc=True,
+                    want_scores=True)
     torch.cuda.synchronize()
     nsa.sync_status()
     hx = host(x)
@@ -107,6 +186,8 @@ def check_forward(c: dict, rows=None, device="cuda", x=None, report=None):
     want = oracle.forward_rows(c, hx["q"], hx["k"], hx["v"], hx["gates"], kc_o, vc_o, rows,
                                want=("out", "idx", "lse", "pgrp"))
     got_idx = r["idx"].reshape(B * T, G, n).cpu().numpy()[rows]
+    selections_valid(c, rows % T, got_idx)
+    check_scores(c, r["scores"], rows, want["pgrp"], report)
     Hg = H // G
     scale = c.get("scale", 0) or 1 / math.sqrt(c["dk"])
     qd = None
@@ -123,11 +204,13 @@ def check_forward(c: dict, rows=None, device="cuda", x=None, report=None):
                     qd = {}
                 qr = f64(hx["q"][b, t, g * Hg:(g + 1) * Hg])
                 delta = scale * float(np.abs(qr @ dK[b, :nv, g].T).max())
-            if selection_ok(c, None, want["pgrp"][a, g], got_idx[a, g], want["idx"][a, g], delta):
+            if selection_ok(c, t, want["pgrp"][a, g], got_idx[a, g], want["idx"][a, g], delta):
                 fixed.append(a)
             else:
                 bad.append((int(rows[a]), g, got_idx[a, g].tolist(), want["idx"][a, g].tolist()))
     assert not bad, f"{len(bad)} selection mismatches beyond near-ties, e.g. {bad[:3]}"
+    print(f"near-tie selections accepted: {len(fixed)} of {rows.size * G} (row, group) pairs")
+    assert len(fixed) <= near_tie_bound(rows.size * G), f"{len(fixed)} near-tie rows"
     if fixed:
         fixed = np.unique(fixed)
         redo = oracle.forward_rows(c, hx["q"], hx["k"], hx["v"], hx["gates"], kc_o, vc_o,

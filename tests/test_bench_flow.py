@@ -29,7 +29,7 @@ class _Event:
         return 660.0          # 20 steps of 33 ms
 
 
-def _run(monkeypatch, clock_records, argv):
+def _run(monkeypatch, clock_records, argv, inputs=None):
     calls = {"forward": 0, "regions": 0}
     monkeypatch.setattr(torch.cuda, "Event", _Event)
     monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
@@ -49,9 +49,9 @@ def _run(monkeypatch, clock_records, argv):
     import sparse_attention_long_phi_b200 as pkg
     monkeypatch.setattr(pkg, "nsa", fake, raising=False)
     monkeypatch.setitem(sys.modules, "sparse_attention_long_phi_b200.nsa", fake)
-    monkeypatch.setattr(I, "make_forward_inputs",
-                        lambda c, dev, with_dout=False: {k: torch.zeros(1) for k in
-                                                         ("q", "k", "v", "gates", "wk", "ek", "wv", "ev")})
+    monkeypatch.setattr(I, "make_forward_inputs", inputs or
+                        (lambda c, dev, with_dout=False: {k: torch.zeros(1) for k in
+                                                          ("q", "k", "v", "gates", "wk", "ek", "wv", "ev")}))
     records = list(clock_records)
 
     def stop(self):
@@ -111,3 +111,29 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
     with contextlib.redirect_stdout(out):
         bench.main()
     assert out.getvalue() == ""
+
+
+def test_roofline_reports_burst_and_sustained(monkeypatch):
+    line, _ = _run(monkeypatch, [CLEAN], ["--no-extras", "--steps", "20", "--warmup", "5"])
+    roof = line["roofline"]
+    peaks, _ = bench.load_peaks()
+    assert roof["peak"] == peaks.get("bf16_tflops", bench.FALLBACK_PEAKS["bf16_tflops"])
+    assert roof["frac_sustained"] == pytest.approx(roof["achieved"] / roof["peak_sustained"], rel=1e-3)
+    assert roof["frac_sustained"] > roof["frac"]
+
+
+def test_group_sharding_is_strong_scaling_over_one_sequence(monkeypatch):
+    # rank 1 of 2 takes groups [2, 4) of the one sequence; the job's tokens per step are
+    # the sequence's, counted once, over the slowest rank's time
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    shapes = {"q": (1, 2, 64, 1), "gates": (1, 2, 64, 3), "k": (1, 2, 4, 1), "v": (1, 2, 4, 1),
+              "wk": (1,), "ek": (1,), "wv": (1,), "ev": (1,)}
+    line, _ = _run(monkeypatch, [CLEAN], ["--no-extras", "--steps", "20", "--warmup", "5",
+                                          "--shard", "groups"],
+                   inputs=lambda c, dev, with_dout=False: {k: torch.zeros(v) for k, v in shapes.items()})
+    assert line["scaling"] == "strong"
+    assert line["value"] == pytest.approx(65536 / 0.033, rel=1e-4)
+    assert bench.strong_scaling_value(65536, 20, 660.0) == pytest.approx(65536 * 20 / 0.66)
+    from sparse_attention_long_phi_b200 import shard
+    assert shard.group_range(4, 1, 2) == (2, 4) and shard.group_range(4, 3, 4) == (3, 4)

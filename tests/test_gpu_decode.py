@@ -7,7 +7,7 @@ import pytest
 import torch
 
 import oracle
-from helpers import assert_close_out, host, selection_ok
+from helpers import assert_close_out, host, near_tie_bound, selection_ok, selections_valid
 from sparse_attention_long_phi_b200 import inputs as I
 
 pytestmark = pytest.mark.gpu
@@ -29,13 +29,17 @@ def run_decode(c, lengths=None):
                          hx["vc_cache"], x["cmp_off"], hx["gates"], want_pgrp=True)
     got_idx = r["idx"].cpu().numpy()
     S, G = got_idx.shape[:2]
+    ts = np.asarray(x["lengths"], np.int64) - 1          # each sequence's query position
+    selections_valid(c, ts, got_idx)
     fixed = []
     for s in range(S):
         for g in range(G):
             if not np.array_equal(got_idx[s, g], want["idx"][s, g]):
-                assert selection_ok(c, None, want["pgrp"][s, g], got_idx[s, g], want["idx"][s, g], 0.0), \
+                assert selection_ok(c, ts[s], want["pgrp"][s, g], got_idx[s, g], want["idx"][s, g], 0.0), \
                     (s, g, got_idx[s, g], want["idx"][s, g])
                 fixed.append(s)
+    print(f"decode near-tie selections accepted: {len(fixed)} of {S * G}")
+    assert len(fixed) <= near_tie_bound(S * G)
     if fixed:
         # recompute those sequences under the GPU's (valid) selection
         for s in sorted(set(fixed)):

@@ -68,9 +68,19 @@ def test_forward_is_deterministic():
 
 
 def test_prefill_T65536_sampled_rows():
+    # 4096 query positions: every t < 1024 (the rows where all blocks are
+    # candidates and the first compressed blocks appear), the last 64, and
+    # seeded uniform draws over the rest
     c = wl("prefill_fwd_T65536")
-    rows = sample_rows(1, c["T"], 48, seed=2, edge=32)
-    check_forward(c, rows=rows)
+    T = c["T"]
+    rng = np.random.default_rng(2)
+    fixed = set(range(1024)) | set(range(T - 64, T))
+    rest = rng.choice(np.arange(1024, T - 64), 4096 - len(fixed), replace=False)
+    rows = np.array(sorted(fixed | set(int(r) for r in rest)), np.int64)
+    assert rows.size == 4096
+    rep = {}
+    check_forward(c, rows=rows, report=rep)
+    print("T=65536 sample:", rep)
 
 
 def test_prefill_largest_supported_context_sampled_rows():

@@ -470,3 +470,63 @@ def test_backward_tail_is_exact_above_the_cut():
                                 x["ek"], x["wv"], x["ev"], t_lo=50)
     for key in ("dq", "dk", "dv", "dgates"):
         np.testing.assert_array_equal(full[key][:, 50:], tail[key][:, 50:])
+
+
+@pytest.mark.parametrize("l,d,lp", [(32, 16, 64), (16, 8, 64), (8, 8, 32)])
+def test_unweighted_score_map_counts_each_overlapping_block_once(l, d, lp):
+    """score_map = 1, the unweighted reading of the blockings-differ paragraph:
+    with p_cmp one-hot at block i*, selection block j scores Hg for every j that
+    block i* overlaps (interval overlap > 0) and 0 elsewhere."""
+    T = 8 * lp
+    c = small_cfg(T=T, l=l, d=d, lp=lp, H=2, G=1, dk=16, dv=8, n=T // lp + 1, phi="linear",
+                  score_map=1)
+    x = make(c)
+    dk, dv = 16, 8
+    sel_k = np.zeros((dk, l * dk), np.float32)
+    sel_k[:, :dk] = np.eye(dk)
+    x["wk"] = I.bits(torch.from_numpy(sel_k).to(torch.bfloat16))
+    x["ek"] = np.zeros((l, dk), np.uint16)
+    x["wv"] = I.bits(torch.zeros(dv, l * dv).to(torch.bfloat16))
+    k = np.zeros((1, T, 1, dk), np.float32)
+    q = np.zeros((1, T, 2, dk), np.float32)
+    q[..., 0] = 4.0
+    C = oracle.num_cmp_blocks(c, T)
+    for i_star in [1, 3, 4, C - 2]:
+        k[:] = 0
+        k[0, i_star * d, 0, 0] = 30.0
+        x["k"] = I.bits(torch.from_numpy(k).to(torch.bfloat16))
+        x["q"] = I.bits(torch.from_numpy(q).to(torch.bfloat16))
+        r = run_rows(c, x, rows=[T - 1])
+        for j in range(T // lp):
+            lo, hi = max(i_star * d, j * lp), min(i_star * d + l, (j + 1) * lp)
+            want = 2.0 if hi > lo else 0.0
+            assert abs(r["pgrp"][0, 0, j] - want) < 1e-9, (i_star, j, r["pgrp"][0, 0, j], want)
+
+
+def test_backward_rows_is_the_backward_of_the_listed_rows_only():
+    """Restricting the backward to a row set R is the backward with dout zeroed
+    outside R (the loss sum_t <dout_t, out_t> is linear in dout): checked against
+    the full backward of such a dout, and the full list equals the full backward."""
+    c = small_cfg(T=96, H=4, G=2, dk=8, dv=8, l=8, d=4, lp=8, n=4, w=11, phi="linear", B=2)
+    x = make(c, with_dout=True)
+    idx = I.random_selection(dict(c, seed=5)).numpy()
+    B, T = c["B"], c["T"]
+    rows = np.array([0, 7, 31, 50, 95, T + 3, T + 64, 2 * T - 1])
+    dz = np.zeros_like(x["dout"]).reshape(B * T, -1)
+    dz[rows] = x["dout"].reshape(B * T, -1)[rows]
+    dz = dz.reshape(x["dout"].shape)
+    args = (x["wk"], x["ek"], x["wv"], x["ev"])
+    full = oracle.backward_tail(c, x["q"], x["k"], x["v"], x["gates"], dz, idx, *args, want_cmp=True)
+    part = oracle.backward_rows(c, x["q"], x["k"], x["v"], x["gates"], x["dout"], idx, rows, *args,
+                                want_cmp=True)
+    for key in ("dq", "dk", "dv", "dkc", "dvc"):
+        np.testing.assert_allclose(part[key], full[key], rtol=1e-12, atol=1e-14, err_msg=key)
+    on = np.zeros(B * T, bool)
+    on[rows] = True
+    ref = oracle.backward_tail(c, x["q"], x["k"], x["v"], x["gates"], x["dout"], idx, *args)
+    dg = part["dgates"].reshape(B * T, -1)
+    np.testing.assert_array_equal(dg[on], ref["dgates"].reshape(B * T, -1)[on])
+    assert not dg[~on].any()
+    every = oracle.backward_rows(c, x["q"], x["k"], x["v"], x["gates"], x["dout"], idx, np.arange(B * T), *args)
+    for key in ("dq", "dk", "dv", "dgates"):
+        np.testing.assert_array_equal(every[key], ref[key])

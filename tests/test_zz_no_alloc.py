@@ -2,8 +2,6 @@
 device memory (graph-captured loops, plugins whose host framework owns all
 device memory).  It must produce exactly what nsa_compress produces, call
 after call, while sharing one fixed device scratch array."""
-import ctypes
-
 import pytest
 import torch
 
@@ -36,7 +34,9 @@ def test_static_compress_matches_workspace_compress_twice(name, T, seed):
 def test_static_compress_rejects_sizes_beyond_its_scratch():
     from sparse_attention_long_phi_b200 import nsa
     c = dict(I.WORKLOADS["prefill_fwd_T65536"])     # 5.2M compressed elements > 16 MiB of scratch
-    fake = ctypes.c_void_p(1 << 20)                  # never dereferenced: rejected first
-    rc = nsa.lib().nsa_compress_static(ctypes.byref(nsa.make_config(c)), fake, fake,
-                                       ctypes.byref(nsa.CPhi(fake, fake, fake, fake)), fake, fake, None)
-    assert rc == 3
+    x = I.make_forward_inputs(c, "cuda")            # real tensors of the right sizes
+    phi = {n: x[n] for n in ("wk", "ek", "wv", "ev")}
+    rc, kc, vc = nsa.compress_static(c, x["k"], x["v"], phi)
+    torch.cuda.synchronize()
+    assert rc == 3                                   # NSA_ERR_WORKSPACE, nothing launched
+    assert torch.isnan(kc.float()).all() and torch.isnan(vc.float()).all()

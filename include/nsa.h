@@ -62,7 +62,12 @@ typedef enum {
 
 typedef enum { NSA_PHI_MEAN = 0, NSA_PHI_LINEAR = 1 } nsa_phi_t;
 
-typedef enum { NSA_MODE_FORWARD = 0, NSA_MODE_DECODE = 1, NSA_MODE_BACKWARD = 2 } nsa_mode_t;
+typedef enum {
+    NSA_MODE_FORWARD = 0,
+    NSA_MODE_DECODE = 1,
+    NSA_MODE_BACKWARD = 2,
+    NSA_MODE_FORWARD_BRANCHES = 3 /* nsa_forward_branches */
+} nsa_mode_t;
 
 /* Operator configuration.  Token compression: block length l = cmp_block,
  * stride d = cmp_stride.  Selection: block length l' = sel_block, n =
@@ -141,6 +146,25 @@ nsa_status_t nsa_forward(const nsa_config_t* cfg, const void* q, const void* k, 
                          const float* gates, const nsa_phi_params_t* phi, float* out,
                          int32_t* sel_idx, float* lse, void* kc_out, void* vc_out,
                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* Prefill forward with independent keys and values per branch (page 2, 滑动窗口:
+ * the three branches are given their own keys and values, so that the local
+ * window cannot take over what compression and selection should learn).
+ * The compressed branch compresses k_cmp [B,T,G,d_k] / v_cmp [B,T,G,d_v]
+ * (phi as in nsa_compress; its probabilities also drive the selection), the
+ * selected branch attends the chosen blocks of k_slc / v_slc, the window the
+ * last w tokens of k_win / v_win; all bf16, same shapes as k / v of
+ * nsa_forward.  Everything else (q, gates, phi, outputs, errors) as in
+ * nsa_forward; with the same tensor passed for all three branches the results
+ * equal nsa_forward's bit for bit.  Needs the NSA_MODE_FORWARD_BRANCHES
+ * workspace (one transposed copy of v_win more than NSA_MODE_FORWARD; the
+ * score table sits at the same offset, see nsa_forward_score_table). */
+nsa_status_t nsa_forward_branches(const nsa_config_t* cfg, const void* q, const void* k_cmp,
+                                  const void* v_cmp, const void* k_slc, const void* v_slc,
+                                  const void* k_win, const void* v_win, const float* gates,
+                                  const nsa_phi_params_t* phi, float* out, int32_t* sel_idx, float* lse,
+                                  void* kc_out, void* vc_out, void* workspace, size_t workspace_bytes,
+                                  void* stream);
 
 /* Where nsa_forward leaves the group importance scores (page 2, 重要性分数计算:
  * the compressed branch's probabilities mapped onto selection blocks by the

@@ -127,15 +127,25 @@ __global__ void __launch_bounds__(320, 1)
 
     if (warp == 8) {
         // ------------------------------------------------------ producer
-        if (lane == 0 && N > 0) {
-            tma_prefetch_desc(&mapQ);
-            tma_prefetch_desc(&mapK);
-            tma_prefetch_desc(&mapV);
+        // The whole warp runs the loop: lane 0 waits for a free slot and posts the
+        // slot's byte count, then the slot's boxes are issued from separate lanes
+        // (one issuing thread alone cannot keep the TMA unit busy).
+        if (N > 0) {
+            if (lane == 0) {
+                tma_prefetch_desc(&mapQ);
+                tma_prefetch_desc(&mapK);
+                tma_prefetch_desc(&mapV);
+            }
             uint32_t cnt = 0;
+            // warp-collective: lane 0 waits, every lane gets the outcome
+            auto lane0_wait = [&](uint64_t* bar, uint32_t parity, unsigned site) -> bool {
+                bool ok = true;
+                if (lane == 0) ok = wait_or_abort(bar, parity, site, abort_flag);
+                return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            };
             auto slot_acquire = [&](uint32_t c) -> uint8_t* {
                 const int sl = c % Cfg::NSLOT;
-                if (c >= Cfg::NSLOT &&
-                    !wait_or_abort(&empty[sl], ((c / Cfg::NSLOT) - 1) & 1, 0x301, abort_flag))
+                if (c >= Cfg::NSLOT && !lane0_wait(&empty[sl], ((c / Cfg::NSLOT) - 1) & 1, 0x301))
                     return nullptr;
                 return smem + Cfg::kOffKV + sl * Cfg::kSlot;
             };
@@ -174,16 +184,17 @@ __global__ void __launch_bounds__(320, 1)
                     uint8_t* sl = slot_acquire(cnt);
                     if (!sl) return false;
                     uint64_t* bar = &full[cnt % Cfg::NSLOT];
+                    if (lane == 0) mbar_expect_tx(bar, kv_is_k ? Cfg::kKPair : Cfg::kVPair);
+                    __syncwarp();
                     if (kv_is_k) {
-                        mbar_expect_tx(bar, Cfg::kKPair);
-                        for (int bx = 0; bx < Cfg::NQB; ++bx) {
-                            tma_load_4d(sl + bx * 16384, &mapK, bar, bx * 64, g, ja * 64, b);
-                            tma_load_4d(sl + bx * 16384 + 8192, &mapK, bar, bx * 64, g, jb * 64, b);
+                        // lane 2*bx + half: 64 channels bx of block ja (half 0) or jb (half 1)
+                        if (lane < 2 * Cfg::NQB) {
+                            const int bx = lane >> 1, half = lane & 1;
+                            tma_load_4d(sl + bx * 16384 + half * 8192, &mapK, bar, bx * 64, g,
+                                        (half ? jb : ja) * 64, b);
                         }
-                    } else {
-                        mbar_expect_tx(bar, Cfg::kVPair);
-                        tma_load_4d(sl, &mapV, bar, ja * 64, 0, g, b);
-                        tma_load_4d(sl + Cfg::DVM * 128, &mapV, bar, jb * 64, 0, g, b);
+                    } else if (lane < 2) {
+                        tma_load_4d(sl + lane * (Cfg::DVM * 128), &mapV, bar, (lane ? jb : ja) * 64, 0, g, b);
                     }
                     ++cnt;
                 }
@@ -191,13 +202,15 @@ __global__ void __launch_bounds__(320, 1)
             };
             auto load_S = [&](int i, const int4 (&r)[4]) -> bool {
                 const int qs = i & 1;
-                if (i >= 2 && !wait_or_abort(&qempty[qs], ((i - 2) >> 1) & 1, 0x302, abort_flag))
-                    return false;
-                npairs_ring[i & 3] = (count_row(r) + 1) / 2;          // read by the MMA warp
-                mbar_expect_tx(&qfull[qs], Cfg::kQSlot);                // (release)
-                for (int bx = 0; bx < Cfg::NQB; ++bx)
-                    tma_load_4d(smem + Cfg::kOffQ + qs * Cfg::kQSlot + bx * 2048, &mapQ, &qfull[qs],
-                                bx * 64, g * HG, tb + i, b);
+                if (i >= 2 && !lane0_wait(&qempty[qs], ((i - 2) >> 1) & 1, 0x302)) return false;
+                if (lane == 0) {
+                    npairs_ring[i & 3] = (count_row(r) + 1) / 2;      // read by the MMA warp
+                    mbar_expect_tx(&qfull[qs], Cfg::kQSlot);            // (release)
+                }
+                __syncwarp();
+                if (lane < Cfg::NQB)
+                    tma_load_4d(smem + Cfg::kOffQ + qs * Cfg::kQSlot + lane * 2048, &mapQ, &qfull[qs],
+                                lane * 64, g * HG, tb + i, b);
                 return load_pairs(r, true);
             };
             int4 cur[4], prev[4], nxt[4];

@@ -189,7 +189,7 @@ nsa_status_t supported(const Shape& s) {
 }
 
 struct FwdWs {
-    size_t off_kc, off_vct, off_vt, off_bias, off_lse, off_ps, off_fix, total;
+    size_t off_kc, off_vct, off_vt, off_bias, off_lse, off_ps, off_fix, off_vt_win, total;
 };
 
 // phi fix-up list: two counters (K, V), then one entry per K~ and V~ element
@@ -214,8 +214,14 @@ FwdWs fwd_layout(const Shape& s) {
     o = align256(o + (size_t)s.B * s.T * s.G * s.NSp * 4);
     w.off_fix = o;
     o = align256(o + fix_bytes(s));
+    w.off_vt_win = o;                 // used only when the window has its own values
     w.total = o;
     return w;
+}
+
+// forward with independent keys/values per branch: a second transposed v
+inline size_t fwd_branches_total(const Shape& s) {
+    return fwd_layout(s).total + align256((size_t)s.B * s.G * s.DVP * s.Tp * 2);
 }
 
 inline nsa_status_t last_launch() {
@@ -346,8 +352,16 @@ nsa_status_t launch_packed_blk(const Shape& s, const CUtensorMap& mQ, const CUte
     return NSA_ERR_UNSUPPORTED;
 }
 
+// Keys and values of the three branches (page 2, 滑动窗口: the branches may
+// have independent keys and values).  The compressed branch compresses
+// (k_cmp, v_cmp); the selected branch reads (k_slc, v_slc) and the window
+// (k_win, v_win).  nsa_forward passes one k/v to all three.
+struct BranchKV {
+    const void *k_cmp, *v_cmp, *k_slc, *v_slc, *k_win, *v_win;
+};
+
 template <int DK, int DV, int HG>
-nsa_status_t forward_impl(const Shape& s, const void* q, const void* k, const void* v,
+nsa_status_t forward_impl(const Shape& s, const void* q, const BranchKV& kv,
                           const float* gates, const nsa_phi_params_t* phi, float* out,
                           int32_t* sel_idx, float* lse, void* kc_out, void* vc_out, uint8_t* ws,
                           cudaStream_t st) {
@@ -355,22 +369,24 @@ nsa_status_t forward_impl(const Shape& s, const void* q, const void* k, const vo
     void* kc = kc_out ? kc_out : ws + L.off_kc;
     void* vcT = ws + L.off_vct;
     void* vT = ws + L.off_vt;
+    const bool own_win_v = kv.v_win != kv.v_slc;
+    void* vTw = own_win_v ? ws + L.off_vt_win : vT;
     double* bias = reinterpret_cast<double*>(ws + L.off_bias);
     float* lse_cmp = reinterpret_cast<float*>(ws + L.off_lse);
     float* pscore = reinterpret_cast<float*>(ws + L.off_ps);
 
     // 1. token compression
-    NSA_TRY(run_phi(s, k, v, phi, kc, vc_out, vcT, bias, ws + L.off_fix, st));
+    NSA_TRY(run_phi(s, kv.k_cmp, kv.v_cmp, phi, kc, vc_out, vcT, bias, ws + L.off_fix, st));
     // 2. v transposed for the P.V products of the selected and window branches
-    {
+    for (int pass = 0; pass < (own_win_v ? 2 : 1); ++pass) {
         dim3 grid((unsigned)ceil_div(s.Tp, 64), (unsigned)s.G, (unsigned)s.B);
-        NSA_LAUNCH("transpose_v_kernel", st, transpose_v_kernel<<<grid, dim3(64, 4), 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(v),
-                                                         (int)s.T, (int)s.G, (int)s.DV, (int)s.DVP,
-                                                         (int)s.Tp, reinterpret_cast<__nv_bfloat16*>(vT)));
+        NSA_LAUNCH("transpose_v_kernel", st, transpose_v_kernel<<<grid, dim3(64, 4), 0, st>>>(
+            reinterpret_cast<const __nv_bfloat16*>(pass ? kv.v_win : kv.v_slc), (int)s.T, (int)s.G, (int)s.DV,
+            (int)s.DVP, (int)s.Tp, reinterpret_cast<__nv_bfloat16*>(pass ? vTw : vT)));
         NSA_TRY(last_launch());
     }
     // tensor maps
-    CUtensorMap mQ, mQs, mKc, mVc, mK, mVT, mVTs;
+    CUtensorMap mQ, mQs, mKc, mVc, mK, mVT, mVTs, mKw;
     {
         const uint64_t dQ[4] = {(uint64_t)s.DK, (uint64_t)s.H, (uint64_t)s.T, (uint64_t)s.B};
         const uint64_t sQ[3] = {(uint64_t)s.DK * 2, (uint64_t)s.H * s.DK * 2, (uint64_t)s.T * s.H * s.DK * 2};
@@ -384,8 +400,8 @@ nsa_status_t forward_impl(const Shape& s, const void* q, const void* k, const vo
         const uint32_t bVT[4] = {64, (uint32_t)s.DV, 1, 1};
         const uint32_t bVTs[4] = {64, 128, 1, 1};
         if (!make_map(&mQ, q, 4, dQ, sQ, bQ) || !make_map(&mQs, q, 4, dQ, sQ, bQs) ||
-            !make_map(&mK, k, 4, dK, sK, bK) || !make_map(&mVT, vT, 4, dVT, sVT, bVT) ||
-            !make_map(&mVTs, vT, 4, dVT, sVT, bVTs))
+            !make_map(&mK, kv.k_slc, 4, dK, sK, bK) || !make_map(&mKw, kv.k_win, 4, dK, sK, bK) ||
+            !make_map(&mVT, vTw, 4, dVT, sVT, bVT) || !make_map(&mVTs, vT, 4, dVT, sVT, bVTs))
             return NSA_ERR_CUDA;
         if (s.C > 0) {
             const uint64_t dKc[4] = {(uint64_t)s.DK, (uint64_t)s.G, (uint64_t)s.C, (uint64_t)s.B};
@@ -461,7 +477,7 @@ nsa_status_t forward_impl(const Shape& s, const void* q, const void* k, const vo
         NSA_TRY(last_launch());
     }
     // 7. sliding window
-    NSA_TRY((launch_packed_blk<DK, DV, HG, kModeWin>(s, mQ, mK, mVT, pp, st)));
+    NSA_TRY((launch_packed_blk<DK, DV, HG, kModeWin>(s, mQ, mKw, mVT, pp, st)));
     return NSA_OK;
 }
 
@@ -737,6 +753,7 @@ size_t nsa_workspace_size(const nsa_config_t* cfg, int32_t mode) {
     Shape s;
     if (derive(cfg, s) != NSA_OK) return 0;
     if (mode == NSA_MODE_FORWARD) return fwd_layout(s).total;
+    if (mode == NSA_MODE_FORWARD_BRANCHES) return fwd_branches_total(s);
     if (mode == NSA_MODE_DECODE) return decode_ws_bytes(s.B, s.T, s.G, s.l, s.d, s.lp, s.w, s.n, s.DV);
     if (mode == NSA_MODE_BACKWARD) return bwd_layout(s).total;
     return 0;
@@ -782,9 +799,36 @@ nsa_status_t nsa_forward(const nsa_config_t* cfg, const void* q, const void* k, 
         return NSA_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+    const BranchKV kv{k, v, k, v, k, v};
     if (s.DK == 192)
-        return forward_impl<192, 128, 16>(s, q, k, v, gates, phi, out, sel_idx, lse, kc_out, vc_out, ws, st);
-    return forward_impl<64, 64, 4>(s, q, k, v, gates, phi, out, sel_idx, lse, kc_out, vc_out, ws, st);
+        return forward_impl<192, 128, 16>(s, q, kv, gates, phi, out, sel_idx, lse, kc_out, vc_out, ws, st);
+    return forward_impl<64, 64, 4>(s, q, kv, gates, phi, out, sel_idx, lse, kc_out, vc_out, ws, st);
+}
+
+nsa_status_t nsa_forward_branches(const nsa_config_t* cfg, const void* q, const void* k_cmp,
+                                  const void* v_cmp, const void* k_slc, const void* v_slc,
+                                  const void* k_win, const void* v_win, const float* gates,
+                                  const nsa_phi_params_t* phi, float* out, int32_t* sel_idx, float* lse,
+                                  void* kc_out, void* vc_out, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+    Shape s;
+    NSA_TRY(derive(cfg, s));
+    NSA_TRY(supported(s));
+    if (cfg->score_map != 0) return NSA_ERR_UNSUPPORTED;
+    if (!q || !k_cmp || !v_cmp || !k_slc || !v_slc || !k_win || !v_win || !gates || !out || !sel_idx)
+        return NSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cmp) || !aligned16(v_cmp) || !aligned16(k_slc) || !aligned16(v_slc) ||
+        !aligned16(k_win) || !aligned16(v_win) || !aligned16(out) || (kc_out && !aligned16(kc_out)) ||
+        (vc_out && !aligned16(vc_out)))
+        return NSA_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < fwd_branches_total(s) || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return NSA_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+    const BranchKV kv{k_cmp, v_cmp, k_slc, v_slc, k_win, v_win};
+    if (s.DK == 192)
+        return forward_impl<192, 128, 16>(s, q, kv, gates, phi, out, sel_idx, lse, kc_out, vc_out, ws, st);
+    return forward_impl<64, 64, 4>(s, q, kv, gates, phi, out, sel_idx, lse, kc_out, vc_out, ws, st);
 }
 
 nsa_status_t nsa_select_blocks(const nsa_config_t* cfg, const float* scores, int32_t* sel_idx,

@@ -16,7 +16,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SO = os.path.join(_HERE, "libnsa.so")
 
-NSA_MODE_FORWARD, NSA_MODE_DECODE, NSA_MODE_BACKWARD = 0, 1, 2
+NSA_MODE_FORWARD, NSA_MODE_DECODE, NSA_MODE_BACKWARD, NSA_MODE_FORWARD_BRANCHES = 0, 1, 2, 3
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "workspace",
           4: "CUDA error", 5: "device timeout"}
 
@@ -69,6 +69,8 @@ def lib():
         L.nsa_compress_static.argtypes = [pc, _P, _P, pp, _P, _P, _P]
         L.nsa_forward.restype = ctypes.c_int
         L.nsa_forward.argtypes = [pc, _P, _P, _P, _P, pp, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+        L.nsa_forward_branches.restype = ctypes.c_int
+        L.nsa_forward_branches.argtypes = [pc] + [_P] * 8 + [pp] + [_P] * 6 + [ctypes.c_size_t, _P]
         L.nsa_decode_rows.restype = ctypes.c_int
         L.nsa_decode_rows.argtypes = [pc, ctypes.c_int32] + [_P] * 13 + [ctypes.c_size_t, _P]
         L.nsa_decode_append.restype = ctypes.c_int
@@ -198,6 +200,30 @@ def forward(c: dict, q, k, v, gates, phi=None, want_lse=True, want_kc=False, str
     res = {"out": buf.out, "idx": buf.idx, "lse": buf.lse, "kc": buf.kc, "vc": buf.vc}
     if want_scores:
         res["scores"] = score_table(c, buf.ws)
+    return res
+
+
+def forward_branches(c: dict, q, kv: dict, gates, phi=None, want_lse=True, want_kc=False,
+                     stream=None, want_scores=False) -> dict:
+    """Prefill forward with independent keys/values per branch: kv = dict(k_cmp, v_cmp,
+    k_slc, v_slc, k_win, v_win), each shaped like k / v.  Returns as forward()."""
+    B, T, H, G, dk, dv = c["B"], c["T"], c["H"], c["G"], c["dk"], c["dv"]
+    C = num_cmp_blocks(c, T)
+    dev = q.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = torch.empty(B, T, H, dv, **f32)
+    idx = torch.empty(B, T, G, c["n"], dtype=torch.int32, device=dev)
+    lse = torch.empty(B, T, H, 3, **f32) if want_lse else None
+    kc = torch.empty(B, max(C, 1), G, dk, dtype=torch.bfloat16, device=dev) if want_kc else None
+    vc = torch.empty(B, max(C, 1), G, dv, dtype=torch.bfloat16, device=dev) if want_kc else None
+    ws = alloc_workspace(c, NSA_MODE_FORWARD_BRANCHES, dev)
+    _check("nsa_forward_branches", lib().nsa_forward_branches(
+        ctypes.byref(make_config(c)), _p(q), _p(kv["k_cmp"]), _p(kv["v_cmp"]), _p(kv["k_slc"]),
+        _p(kv["v_slc"]), _p(kv["k_win"]), _p(kv["v_win"]), _p(gates), _phi(phi), _p(out), _p(idx), _p(lse),
+        _p(kc), _p(vc), _p(ws), ws.numel(), _stream(stream)))
+    res = {"out": out, "idx": idx, "lse": lse, "kc": kc, "vc": vc}
+    if want_scores:
+        res["scores"] = score_table(c, ws)
     return res
 
 

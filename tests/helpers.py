@@ -157,17 +157,37 @@ def check_scores(c, table, rows, pgrp, report=None, rtol=2e-5):
     return worst
 
 
-def check_forward(c: dict, rows=None, device="cuda", x=None, report=None):
-    """Run nsa_forward on the workload, compare with the oracle on `rows`."""
+def branch_inputs(c: dict, x: dict, device="cuda") -> dict:
+    """Independent keys/values per branch (page 2, 滑动窗口): the compressed branch
+    keeps x's k/v, the selected and window branches get k/v drawn with other seeds."""
+    xs = I.make_forward_inputs(dict(c, seed=c["seed"] + 101), device)
+    xw = I.make_forward_inputs(dict(c, seed=c["seed"] + 202), device)
+    return {"k_cmp": x["k"], "v_cmp": x["v"], "k_slc": xs["k"], "v_slc": xs["v"],
+            "k_win": xw["k"], "v_win": xw["v"]}
+
+
+def check_forward(c: dict, rows=None, device="cuda", x=None, report=None, branches=False):
+    """Run nsa_forward (or, with branches, nsa_forward_branches on independent keys and
+    values per branch) on the workload, compare with the oracle on `rows`."""
     from sparse_attention_long_phi_b200 import nsa
     B, T, H, G, n = c["B"], c["T"], c["H"], c["G"], c["n"]
     if x is None:
         x = I.make_forward_inputs(c, device)
-    r = nsa.forward(c, x["q"], x["k"], x["v"], x["gates"], phi_params(x), want_lse=True, want_kc=True,
-                    want_scores=True)
+    if branches:
+        kv = branch_inputs(c, x, device)
+        r = nsa.forward_branches(c, x["q"], kv, x["gates"], phi_params(x), want_lse=True, want_kc=True,
+                                 want_scores=True)
+        hkv = host(kv)
+    else:
+        r = nsa.forward(c, x["q"], x["k"], x["v"], x["gates"], phi_params(x), want_lse=True, want_kc=True,
+                        want_scores=True)
     torch.cuda.synchronize()
     nsa.sync_status()
     hx = host(x)
+    if branches:                    # what each branch reads
+        okv = dict(k=hkv["k_slc"], v=hkv["v_slc"], k_win=hkv["k_win"], v_win=hkv["v_win"])
+    else:
+        okv = dict(k=hx["k"], v=hx["v"], k_win=None, v_win=None)
     C = oracle.num_cmp_blocks(c, T)
     kc_o, vc_o = oracle.phi(c, hx["k"], hx["v"], hx.get("wk"), hx.get("ek"), hx.get("wv"), hx.get("ev"))
     dK = np.zeros(kc_o.shape)
@@ -183,8 +203,8 @@ def check_forward(c: dict, rows=None, device="cuda", x=None, report=None):
     if rows is None:
         rows = np.arange(B * T)
     rows = np.asarray(rows, np.int64)
-    want = oracle.forward_rows(c, hx["q"], hx["k"], hx["v"], hx["gates"], kc_o, vc_o, rows,
-                               want=("out", "idx", "lse", "pgrp"))
+    want = oracle.forward_rows(c, hx["q"], okv["k"], okv["v"], hx["gates"], kc_o, vc_o, rows,
+                               want=("out", "idx", "lse", "pgrp"), k_win=okv["k_win"], v_win=okv["v_win"])
     got_idx = r["idx"].reshape(B * T, G, n).cpu().numpy()[rows]
     selections_valid(c, rows % T, got_idx)
     check_scores(c, r["scores"], rows, want["pgrp"], report)
@@ -213,8 +233,9 @@ def check_forward(c: dict, rows=None, device="cuda", x=None, report=None):
     assert len(fixed) <= near_tie_bound(rows.size * G), f"{len(fixed)} near-tie rows"
     if fixed:
         fixed = np.unique(fixed)
-        redo = oracle.forward_rows(c, hx["q"], hx["k"], hx["v"], hx["gates"], kc_o, vc_o,
-                                   rows[fixed], idx_in=got_idx[fixed], want=("out", "idx", "lse"))
+        redo = oracle.forward_rows(c, hx["q"], okv["k"], okv["v"], hx["gates"], kc_o, vc_o,
+                                   rows[fixed], idx_in=got_idx[fixed], want=("out", "idx", "lse"),
+                                   k_win=okv["k_win"], v_win=okv["v_win"])
         want["out"][fixed] = redo["out"]
         want["lse"][fixed] = redo["lse"]
     out_g = r["out"].reshape(B * T, H, c["dv"]).cpu().numpy()[rows]

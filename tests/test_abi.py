@@ -160,3 +160,26 @@ def test_decode_and_backward_validation_on_host(L):
                             fake, fake, fake, 64, None) == 3
     assert lib.nsa_backward(ctypes.byref(cb), None, fake, fake, fake, None, fake, fake, fake, fake,
                             fake, fake, fake, 1 << 40, None) == 1
+
+
+def test_forward_branches_validation_and_score_table_on_host(L):
+    lib = L.lib()
+    base = dict(I.WORKLOADS["prefill_fwd_T8192"], phi="mean")
+    cfg = L.make_config(base)
+    fake = ctypes.c_void_p(1 << 20)
+    ws = 1 << 34
+    seven = [fake] * 7                     # q, k_cmp, v_cmp, k_slc, v_slc, k_win, v_win
+    missing = list(seven)
+    missing[5] = None                      # no window keys
+    assert lib.nsa_forward_branches(ctypes.byref(cfg), *missing, fake, None, fake, fake, None, None, None,
+                                    fake, ws, None) == 1
+    small = L.workspace_size(base, L.NSA_MODE_FORWARD)
+    assert lib.nsa_forward_branches(ctypes.byref(cfg), *seven, fake, None, fake, fake, None, None, None,
+                                    fake, small, None) == 3          # needs the larger workspace
+    assert L.workspace_size(base, L.NSA_MODE_FORWARD_BRANCHES) > small
+    stride = ctypes.c_int64(0)
+    off = lib.nsa_forward_score_table(ctypes.byref(cfg), ctypes.byref(stride))
+    assert 0 < off < small and off % 256 == 0 and stride.value == 128
+    assert off + 4 * 8192 * 4 * 128 <= small
+    assert lib.nsa_forward_score_table(ctypes.byref(L.make_config(dict(base, d=12))), None) == -1
+    assert lib.nsa_check_timeout_path(0, None) == 1                  # limit outside 1 .. 2e9 ns

@@ -8,19 +8,16 @@
 // The compressed branch's dK~/dV~ go back through phi (mean: /l to each
 // member token; linear: W^T dK~ scattered over the overlapping blocks).
 //
-// Kernels (SIMT, fp32 accumulation):
+// Kernels of this file (the tcgen05 key-centric and dense query-centric
+// passes live in k_bwd_kv.cuh and k_bwd_q.cuh):
 //   bwd_query_mma        one CTA per (b, t, g) on warp-level bf16 tensor cores
-//                        (the 16 heads of the group are the M side): pass 1
-//                        recomputes every branch's LSE and o_c (online softmax
-//                        per warp, merged across warps) and writes dgates and
-//                        D_c; pass 2 recomputes S and dP = dO_c V^T, forms dS
-//                        and accumulates dq = scale dS K.
-//   bwd_kv_mma<BR>       key-centric: a tile of 64 keys (raw tokens for the
-//                        window and selected branches, compressed blocks for
-//                        the compressed one) accumulates over the queries that
-//                        read it, then adds into dk/dv (dK~/dV~) atomically.
-//                        Selected keys find their queries through an inverse
-//                        index (block -> tokens) built by count / scan / fill.
+//                        (the 16 heads of the group are the M side): with the
+//                        row statistics known, recomputes S and dP = dO_c V^T
+//                        over the selected blocks, forms dS and accumulates
+//                        dq = scale dS K (sweep 2); without them it first
+//                        recomputes every branch's LSE and o_c (sweep 1).
+//   bwd_branch_stats     d(gate_c), D_c and the log2 LSE of one branch from its
+//                        output under unit gates.
 //   bwd_phiT_kernel      dk/dv += phi^T(dK~/dV~).
 #pragma once
 #include "nsa_dev.cuh"
@@ -29,7 +26,6 @@
 namespace nsa {
 
 enum { kBrCmp = 0, kBrSlc = 1, kBrWin = 2 };
-constexpr int kBwdChunk = 128;     // tokens per key-centric work item
 
 struct BwdParams {
     int B, T, H, G, HG, DK, DV, l, d, lp, n, w, C, NSb;
@@ -42,6 +38,8 @@ struct BwdParams {
     float *dkc, *dvc;           // [B,C,G,*]
     int *cnt, *cursor, *off, *chunk_off, *list;
     int phi;                    // 0 mean, 1 linear
+    int have_stats;             // lse2 / dlt / dgates already computed: the query pass skips its sweep 1
+    int q_branches;             // bit br set: the query pass accumulates dq of branch br (sweep 2)
 };
 
 __device__ __forceinline__ int ncmp_vis(const BwdParams& p, int t) {
@@ -133,7 +131,15 @@ __global__ void __launch_bounds__(128) bwd_query_mma(const BwdParams p) {
     };
 
     // ---------------- pass 1, every branch: LSE, o_c, dgates, D
-    for (int br = 0; br < 3; ++br) {
+    if (p.have_stats) {
+        if (threadIdx.x < 48) {
+            const int br = threadIdx.x / 16, h = threadIdx.x % 16;
+            lse2s[br][h] = h < p.HG ? p.lse2[(rowbase + h) * 3 + br] : -INFINITY;
+            Ds[br][h] = h < p.HG ? p.dlt[(rowbase + h) * 3 + br] : 0.f;
+        }
+        __syncthreads();
+    }
+    for (int br = 0; br < 3 && !p.have_stats; ++br) {
         int lo;
         const int nk = branch_keys(br, lo);
         const int nch = (nk + 31) / 32;
@@ -263,6 +269,7 @@ __global__ void __launch_bounds__(128) bwd_query_mma(const BwdParams p) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) dq[nt][e] = 0.f;
     for (int br = 0; br < 3; ++br) {
+        if (!((p.q_branches >> br) & 1)) continue;
         int lo;
         const int nk = branch_keys(br, lo);
         const int nch = (nk + 31) / 32;
@@ -306,308 +313,37 @@ __global__ void __launch_bounds__(128) bwd_query_mma(const BwdParams p) {
     }
 }
 
-// --------------------------------------------------------- per key tile
-// One CTA of 4 warps = 64 keys (warp w: keys 16w..16w+15 of the tile) and a
-// run of up to kBwdChunk tokens that attend them; per token, on warp-level
-// bf16 tensor cores (mma.sync m16n8k16) with the 16 heads as the N side:
-//   S^T = K_w Q_t^T,  dP^T = V_w dO_t^T                 (16 keys x 16 heads)
-//   P = exp(S - LSE_h), dS = P (g_h dP - D_h)
-//   dK_w += scale dS^T Q_t,  dV_w += (g P)^T dO_t       (in registers)
-// The tile's K/V rows and the tokens' Q/dO rows (double-buffered) sit in
-// shared memory; dK/dV are added to the fp32 outputs once at the end.
-// grid.z = b*G + g.  WIN: grid (key tiles of 64 tokens, token chunks).
-// CMP: grid (key tiles of 64 compressed blocks, token chunks).
-// SLC: grid.x = chunk id over the inverse index (binary search), b and g
-// from the entry found.
-template <int DK, int DV>
-__host__ __device__ constexpr int bwd_kv_mma_smem() {
-    return 64 * ((DK * 2 + 16) + (DV * 2 + 16)) + 2 * 16 * ((DK * 2 + 16) + (DV * 2 + 16));
-}
-
-template <int DK, int DV, int BR>
-__global__ void __launch_bounds__(128) bwd_kv_mma(const BwdParams p) {
-    constexpr int KP = DK * 2 + 16, VP = DV * 2 + 16;
-    extern __shared__ __align__(16) uint8_t bsm[];
-    uint8_t* kt = bsm;                          // [64][KP]
-    uint8_t* vt = kt + 64 * KP;                 // [64][VP]
-    uint8_t* tokb = vt + 64 * VP;               // 2 x ([16][KP] Q rows, [16][VP] dO rows)
-    __shared__ float sl[2][16], sD[2][16], sg[2][16];
-    __shared__ int stok[2];
-    int b = blockIdx.z / p.G, g = blockIdx.z % p.G;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gr = lane >> 2, tg = lane & 3;
-
-    int key0, tok_lo, tok_hi;           // keys key0..key0+63; tokens (or list entries) [tok_lo, tok_hi)
-    const int* toklist = nullptr;
-    if (BR == kBrSlc) {
-        const int cid = blockIdx.x;
-        if (cid >= p.chunk_off[p.B * p.G * p.NSb]) return;
-        int lo = 0, hi = p.B * p.G * p.NSb;             // entry e with chunk_off[e] <= cid < chunk_off[e+1]
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (p.chunk_off[mid] <= cid) lo = mid;
-            else hi = mid;
-        }
-        const int e = lo;
-        b = e / (p.G * p.NSb);
-        g = (e / p.NSb) % p.G;
-        const int j = e % p.NSb;
-        const int c = cid - p.chunk_off[e];
-        key0 = j * p.lp;
-        tok_lo = p.off[e] + c * kBwdChunk;
-        tok_hi = min(p.off[e] + p.cnt[e], tok_lo + kBwdChunk);
-        toklist = p.list;
-    } else if (BR == kBrWin) {
-        key0 = blockIdx.x * 64;
-        if (key0 >= p.T) return;
-        const int tmax = min(p.T, key0 + 64 + p.w - 1);
-        tok_lo = key0 + blockIdx.y * kBwdChunk;
-        tok_hi = min(tmax, tok_lo + kBwdChunk);
-    } else {
-        key0 = blockIdx.x * 64;
-        if (key0 >= p.C) return;
-        const int tfirst = key0 * p.d + p.l - 1;
-        tok_lo = tfirst + blockIdx.y * kBwdChunk;
-        tok_hi = min(p.T, tok_lo + kBwdChunk);
+// ------------------------------------------------- per-branch statistics
+// From one branch's output o_c (computed with unit gates) and its natural-log
+// LSE: d(gate_c) = <dO, o_c>, D_c = g_c <dO, o_c>, LSE in log2 units.  One
+// warp per query row (b, t, h).
+__global__ void bwd_branch_stats(const float* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
+                                 const float* __restrict__ gates, const float* __restrict__ lse_nat, int br,
+                                 long long rows, int DV, float* dgates, float* dlt, float* lse2) {
+    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    float acc = 0.f;
+    for (int c = lane * 4; c < DV; c += 128) {
+        const float4 ov = *reinterpret_cast<const float4*>(o + row * DV + c);
+        const uint2 dv = *reinterpret_cast<const uint2*>(dout + row * DV + c);
+        const __nv_bfloat162 d01 = *reinterpret_cast<const __nv_bfloat162*>(&dv.x);
+        const __nv_bfloat162 d23 = *reinterpret_cast<const __nv_bfloat162*>(&dv.y);
+        acc += ov.x * __low2float(d01) + ov.y * __high2float(d01) + ov.z * __low2float(d23) +
+               ov.w * __high2float(d23);
     }
-    if (tok_lo >= tok_hi) return;
-    const int nkeys = BR == kBrCmp ? p.C : p.T;
-
-    // the tile's K and V rows (rows past the keys zero-filled)
-    {
-        const __nv_bfloat16* kb = BR == kBrCmp ? p.kc + ((size_t)b * p.C * p.G + g) * DK
-                                               : p.k + ((size_t)b * p.T * p.G + g) * DK;
-        const __nv_bfloat16* vb = BR == kBrCmp ? p.vc + ((size_t)b * p.C * p.G + g) * DV
-                                               : p.v + ((size_t)b * p.T * p.G + g) * DV;
-        const int nv = min(64, nkeys - key0);
-        for (int e = threadIdx.x; e < 64 * (DK / 8); e += 128) {
-            const int r = e / (DK / 8), c8 = e % (DK / 8);
-            const bool ok = r < nv;
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(kt + r * KP + c8 * 16)),
-                         "l"(kb + (size_t)(ok ? key0 + r : key0) * p.G * DK + c8 * 8), "r"(ok ? 16 : 0)
-                         : "memory");
-        }
-        for (int e = threadIdx.x; e < 64 * (DV / 8); e += 128) {
-            const int r = e / (DV / 8), c8 = e % (DV / 8);
-            const bool ok = r < nv;
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(vt + r * VP + c8 * 16)),
-                         "l"(vb + (size_t)(ok ? key0 + r : key0) * p.G * DV + c8 * 8), "r"(ok ? 16 : 0)
-                         : "memory");
-        }
-        cp_async_commit();
-    }
-    // one token's Q / dO rows (heads past HG zero) and statistics into buffer `buf`
-    auto stage = [&](int it, int buf) {
-        const int t = toklist ? toklist[it] : it;
-        const size_t rowbase = ((size_t)b * p.T + t) * p.H + (size_t)g * p.HG;
-        uint8_t* qs = tokb + buf * 16 * (KP + VP);
-        uint8_t* ds = qs + 16 * KP;
-        for (int e = threadIdx.x; e < 16 * (DK / 8); e += 128) {
-            const int h = e / (DK / 8), c8 = e % (DK / 8);
-            const bool ok = h < p.HG;
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(qs + h * KP + c8 * 16)),
-                         "l"(p.q + (rowbase + (ok ? h : 0)) * DK + c8 * 8), "r"(ok ? 16 : 0)
-                         : "memory");
-        }
-        for (int e = threadIdx.x; e < 16 * (DV / 8); e += 128) {
-            const int h = e / (DV / 8), c8 = e % (DV / 8);
-            const bool ok = h < p.HG;
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(ds + h * VP + c8 * 16)),
-                         "l"(p.dout + (rowbase + (ok ? h : 0)) * DV + c8 * 8), "r"(ok ? 16 : 0)
-                         : "memory");
-        }
-        cp_async_commit();
-        if (threadIdx.x < 16) {
-            const int h = threadIdx.x;
-            const bool ok = h < p.HG;
-            sl[buf][h] = ok ? p.lse2[(rowbase + h) * 3 + BR] : -INFINITY;
-            sD[buf][h] = ok ? p.dlt[(rowbase + h) * 3 + BR] : 0.f;
-            sg[buf][h] = ok ? p.gates[(rowbase + h) * 3 + BR] : 0.f;
-        }
-        if (threadIdx.x == 0) stok[buf] = t;
-    };
-
-    float dk[DK / 8][4], dv[DV / 8][4];
 #pragma unroll
-    for (int nt = 0; nt < DK / 8; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dk[nt][e] = 0.f;
-#pragma unroll
-    for (int nt = 0; nt < DV / 8; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dv[nt][e] = 0.f;
-    const int mi = lane >> 3, rr = lane & 7;
-    const uint32_t ka = smem_u32(kt) + (warp * 16 + (mi & 1) * 8 + rr) * KP + (mi >> 1) * 16;   // A rows of this warp
-    const uint32_t va = smem_u32(vt) + (warp * 16 + (mi & 1) * 8 + rr) * VP + (mi >> 1) * 16;
-    // key of accumulator rows gr, gr + 8 (tile-local)
-    const int kr0 = warp * 16 + gr, kr1 = kr0 + 8;
-
-    stage(tok_lo, 0);
-    for (int it = tok_lo; it < tok_hi; ++it) {
-        const int buf = (it - tok_lo) & 1;
-        if (it + 1 < tok_hi) {
-            stage(it + 1, buf ^ 1);
-            cp_async_wait_1();
-        } else {
-            cp_async_wait();
-        }
-        __syncthreads();
-        const int t = stok[buf];
-        const uint32_t qs = smem_u32(tokb + buf * 16 * (KP + VP));
-        const uint32_t ds = qs + 16 * KP;
-        // S^T = K_w Q^T, dP^T = V_w dO^T: two n-tiles of 8 heads
-        float sa[2][4], da[2][4];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) sa[nt][e] = da[nt][e] = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < DK / 16; ++kk) {
-            uint32_t a[4], b0, b1, b2, b3;
-            ldsm_x4(ka + kk * 32, a[0], a[1], a[2], a[3]);
-            // B: heads (mi>>1)*8 + rr, dims kk*16 + (mi&1)*8
-            ldsm_x4(qs + ((mi >> 1) * 8 + rr) * KP + kk * 32 + (mi & 1) * 16, b0, b1, b2, b3);
-            mma16816(sa[0], a, b0, b1);
-            mma16816(sa[1], a, b2, b3);
-        }
-#pragma unroll
-        for (int kk = 0; kk < DV / 16; ++kk) {
-            uint32_t a[4], b0, b1, b2, b3;
-            ldsm_x4(va + kk * 32, a[0], a[1], a[2], a[3]);
-            ldsm_x4(ds + ((mi >> 1) * 8 + rr) * VP + kk * 32 + (mi & 1) * 16, b0, b1, b2, b3);
-            mma16816(da[0], a, b0, b1);
-            mma16816(da[1], a, b2, b3);
-        }
-        // which of this thread's two keys does token t see?
-        auto seen = [&](int kr) -> bool {
-            const int key = key0 + kr;
-            if (key >= nkeys) return false;
-            if (BR == kBrCmp) return key < ncmp_vis(p, t);
-            if (BR == kBrSlc) return key <= t;
-            return key <= t && key >= t - p.w + 1;
-        };
-        const bool v0 = seen(kr0), v1 = seen(kr1);
-        float ps[2][4], pg[2][4];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int h = nt * 8 + tg * 2 + (e & 1);
-                const bool ok = (e < 2 ? v0 : v1) && sl[buf][h] != -INFINITY;
-                const float P = ok ? exp2f(sa[nt][e] * p.scale_log2 - sl[buf][h]) : 0.f;
-                ps[nt][e] = P * (sg[buf][h] * da[nt][e] - sD[buf][h]);
-                pg[nt][e] = P * sg[buf][h];
-            }
-        // dK_w += dS^T Q, dV_w += (gP)^T dO: A = the 16 x 16 (keys x heads) tile, B from
-        // the Q / dO rows (heads = K dimension) via ldmatrix.trans
-        uint32_t as[4], ap[4];
-        as[0] = pack_bf16x2(ps[0][0], ps[0][1]);
-        as[1] = pack_bf16x2(ps[0][2], ps[0][3]);
-        as[2] = pack_bf16x2(ps[1][0], ps[1][1]);
-        as[3] = pack_bf16x2(ps[1][2], ps[1][3]);
-        ap[0] = pack_bf16x2(pg[0][0], pg[0][1]);
-        ap[1] = pack_bf16x2(pg[0][2], pg[0][3]);
-        ap[2] = pack_bf16x2(pg[1][0], pg[1][1]);
-        ap[3] = pack_bf16x2(pg[1][2], pg[1][3]);
-#pragma unroll
-        for (int nt = 0; nt < DK / 8; nt += 2) {
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4_t(qs + ((mi & 1) * 8 + rr) * KP + (nt * 8 + (mi >> 1) * 8) * 2, b0, b1, b2, b3);
-            mma16816(dk[nt], as, b0, b1);
-            mma16816(dk[nt + 1], as, b2, b3);
-        }
-#pragma unroll
-        for (int nt = 0; nt < DV / 8; nt += 2) {
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4_t(ds + ((mi & 1) * 8 + rr) * VP + (nt * 8 + (mi >> 1) * 8) * 2, b0, b1, b2, b3);
-            mma16816(dv[nt], ap, b0, b1);
-            mma16816(dv[nt + 1], ap, b2, b3);
-        }
-        __syncthreads();                        // buffer `buf` is restaged next iteration
-    }
-    // add into the fp32 outputs (several token chunks share a key tile)
-    float* dkb = BR == kBrCmp ? p.dkc + ((size_t)b * p.C * p.G + g) * DK : p.dk + ((size_t)b * p.T * p.G + g) * DK;
-    float* dvb = BR == kBrCmp ? p.dvc + ((size_t)b * p.C * p.G + g) * DV : p.dv + ((size_t)b * p.T * p.G + g) * DV;
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        const int key = key0 + (half ? kr1 : kr0);
-        if (key >= nkeys) continue;
-        float* dkr = dkb + (size_t)key * p.G * DK;
-        float* dvr = dvb + (size_t)key * p.G * DV;
-#pragma unroll
-        for (int nt = 0; nt < DK / 8; ++nt) {
-            atomicAdd(dkr + nt * 8 + tg * 2, p.scale * dk[nt][2 * half]);
-            atomicAdd(dkr + nt * 8 + tg * 2 + 1, p.scale * dk[nt][2 * half + 1]);
-        }
-#pragma unroll
-        for (int nt = 0; nt < DV / 8; ++nt) {
-            atomicAdd(dvr + nt * 8 + tg * 2, dv[nt][2 * half]);
-            atomicAdd(dvr + nt * 8 + tg * 2 + 1, dv[nt][2 * half + 1]);
-        }
+    for (int m = 16; m >= 1; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+    if (lane == 0) {
+        dgates[row * 3 + br] = acc;
+        dlt[row * 3 + br] = gates[row * 3 + br] * acc;
+        lse2[row * 3 + br] = lse_nat[row * 3 + br] * kLog2e;
     }
 }
 
-// -------------------------------------------------- inverse index (slc)
-__global__ void bwd_sel_count(const BwdParams p) {
+__global__ void fill_f32(float* x, long long n, float v) {
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    const long long N = (long long)p.B * p.T * p.G * p.n;
-    if (i >= N) return;
-    const int j = p.idx[i];
-    if (j < 0) return;
-    const long long btg = i / p.n;
-    const int g = (int)(btg % p.G);
-    const int b = (int)(btg / ((long long)p.T * p.G));
-    atomicAdd(&p.cnt[((size_t)b * p.G + g) * p.NSb + j], 1);
-}
-
-// single CTA of 1024 threads: off = exclusive scan of cnt, chunk_off = scan of ceil(cnt/chunk)
-__global__ void __launch_bounds__(1024) bwd_sel_scan(const BwdParams p) {
-    __shared__ int s_cnt[1024], s_ch[1024];
-    const int N = p.B * p.G * p.NSb;
-    const int per = (N + 1023) / 1024;
-    const int beg = min(N, (int)threadIdx.x * per), end = min(N, beg + per);
-    int a = 0, c = 0;
-    for (int i = beg; i < end; ++i) {
-        a += p.cnt[i];
-        c += (p.cnt[i] + kBwdChunk - 1) / kBwdChunk;
-    }
-    s_cnt[threadIdx.x] = a;
-    s_ch[threadIdx.x] = c;
-    __syncthreads();
-    for (int o = 1; o < 1024; o <<= 1) {
-        int va = threadIdx.x >= (unsigned)o ? s_cnt[threadIdx.x - o] : 0;
-        int vc = threadIdx.x >= (unsigned)o ? s_ch[threadIdx.x - o] : 0;
-        __syncthreads();
-        s_cnt[threadIdx.x] += va;
-        s_ch[threadIdx.x] += vc;
-        __syncthreads();
-    }
-    a = s_cnt[threadIdx.x] - a;
-    c = s_ch[threadIdx.x] - c;
-    for (int i = beg; i < end; ++i) {
-        p.off[i] = a;
-        p.chunk_off[i] = c;
-        a += p.cnt[i];
-        c += (p.cnt[i] + kBwdChunk - 1) / kBwdChunk;
-    }
-    if (threadIdx.x == 1023) {
-        p.off[N] = s_cnt[1023];
-        p.chunk_off[N] = s_ch[1023];
-    }
-}
-
-__global__ void bwd_sel_fill(const BwdParams p) {
-    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    const long long N = (long long)p.B * p.T * p.G * p.n;
-    if (i >= N) return;
-    const int j = p.idx[i];
-    if (j < 0) return;
-    const long long btg = i / p.n;
-    const int g = (int)(btg % p.G);
-    const int t = (int)((btg / p.G) % p.T);
-    const int b = (int)(btg / ((long long)p.T * p.G));
-    const size_t e = ((size_t)b * p.G + g) * p.NSb + j;
-    const int pos = atomicAdd(&p.cursor[e], 1);
-    p.list[p.off[e] + pos] = t;
+    if (i < n) x[i] = v;
 }
 
 // ------------------------------------------------------------ phi^T

@@ -20,6 +20,8 @@
 #include "k_attn_sel.cuh"
 #include "k_decode.cuh"
 #include "k_backward.cuh"
+#include "k_bwd_kv.cuh"
+#include "k_bwd_q.cuh"
 #include "k_phi.cuh"
 #include "k_topn.cuh"
 #include "k_append.cuh"
@@ -352,6 +354,113 @@ nsa_status_t launch_packed_blk(const Shape& s, const CUtensorMap& mQ, const CUte
     return NSA_ERR_UNSUPPORTED;
 }
 
+// Tensor maps of the attention kernels: q (packed query tiles and per-token
+// head boxes), raw keys of the selected and window branches, compressed keys,
+// and the transposed value copies (the K-major B operands of the P.V products).
+struct AttnMaps {
+    CUtensorMap mQ, mQs, mKc, mVc, mK, mVT, mVTs, mKw;
+};
+
+template <int DK, int DV, int HG>
+nsa_status_t attn_maps(const Shape& s, const void* q, const void* k_slc, const void* k_win, const void* kc,
+                       const void* vcT, const void* vT, const void* vTw, AttnMaps& m) {
+    const uint64_t dQ[4] = {(uint64_t)s.DK, (uint64_t)s.H, (uint64_t)s.T, (uint64_t)s.B};
+    const uint64_t sQ[3] = {(uint64_t)s.DK * 2, (uint64_t)s.H * s.DK * 2, (uint64_t)s.T * s.H * s.DK * 2};
+    const uint32_t bQ[4] = {64, (uint32_t)HG, (uint32_t)(128 / HG), 1};
+    const uint32_t bQs[4] = {64, 16, 1, 1};
+    const uint64_t dK[4] = {(uint64_t)s.DK, (uint64_t)s.G, (uint64_t)s.T, (uint64_t)s.B};
+    const uint64_t sK[3] = {(uint64_t)s.DK * 2, (uint64_t)s.G * s.DK * 2, (uint64_t)s.T * s.G * s.DK * 2};
+    const uint32_t bK[4] = {64, 1, 64, 1};
+    const uint64_t dVT[4] = {(uint64_t)s.T, (uint64_t)s.DVP, (uint64_t)s.G, (uint64_t)s.B};
+    const uint64_t sVT[3] = {(uint64_t)s.Tp * 2, (uint64_t)s.DVP * s.Tp * 2, (uint64_t)s.G * s.DVP * s.Tp * 2};
+    const uint32_t bVT[4] = {64, (uint32_t)s.DV, 1, 1};
+    const uint32_t bVTs[4] = {64, 128, 1, 1};
+    if (!make_map(&m.mQ, q, 4, dQ, sQ, bQ) || !make_map(&m.mQs, q, 4, dQ, sQ, bQs) ||
+        !make_map(&m.mK, k_slc, 4, dK, sK, bK) || !make_map(&m.mKw, k_win, 4, dK, sK, bK) ||
+        !make_map(&m.mVT, vTw, 4, dVT, sVT, bVT) || !make_map(&m.mVTs, vT, 4, dVT, sVT, bVTs))
+        return NSA_ERR_CUDA;
+    if (s.C > 0) {
+        const uint64_t dKc[4] = {(uint64_t)s.DK, (uint64_t)s.G, (uint64_t)s.C, (uint64_t)s.B};
+        const uint64_t sKc[3] = {(uint64_t)s.DK * 2, (uint64_t)s.G * s.DK * 2, (uint64_t)s.C * s.G * s.DK * 2};
+        const uint64_t dVc[4] = {(uint64_t)s.C, (uint64_t)s.DV, (uint64_t)s.G, (uint64_t)s.B};
+        const uint64_t sVc[3] = {(uint64_t)s.Cp * 2, (uint64_t)s.DV * s.Cp * 2, (uint64_t)s.G * s.DV * s.Cp * 2};
+        const uint32_t bVc[4] = {64, (uint32_t)s.DV, 1, 1};
+        if (!make_map(&m.mKc, kc, 4, dKc, sKc, bK) || !make_map(&m.mVc, vcT, 4, dVc, sVc, bVc))
+            return NSA_ERR_CUDA;
+    }
+    return NSA_OK;
+}
+
+template <int HG>
+PackedParams packed_params(const Shape& s, const float* gates, float* out, float* lse, float* lse_cmp,
+                           float* pscore) {
+    PackedParams pp{};
+    pp.B = (int)s.B;
+    pp.T = (int)s.T;
+    pp.H = (int)s.H;
+    pp.G = (int)s.G;
+    pp.l = (int)s.l;
+    pp.d = (int)s.d;
+    pp.lp = (int)s.lp;
+    pp.w = (int)s.w;
+    pp.scale_log2 = s.scale * kLog2e;
+    pp.gates = gates;
+    pp.out = out;
+    pp.lse_user = lse;
+    pp.lse_cmp = lse_cmp;
+    pp.pscore = pscore;
+    pp.NSp = (int)s.NSp;
+    pp.n_ctas = (int)ceil_div(s.T, 2 * (128 / HG));
+    return pp;
+}
+
+// compressed branch: out = g_cmp o_cmp (stored), lse[..., 0], the score table
+template <int DK, int DV, int HG>
+nsa_status_t launch_cmp(const Shape& s, const AttnMaps& m, const float* gates, float* out, float* lse,
+                        float* lse_cmp, float* pscore, cudaStream_t st) {
+    if (s.C > 0) {
+        const PackedParams pp = packed_params<HG>(s, gates, out, lse, lse_cmp, pscore);
+        NSA_TRY((launch_packed_blk<DK, DV, HG, kModeLse>(s, m.mQ, m.mKc, m.mVc, pp, st)));
+        return launch_packed_blk<DK, DV, HG, kModeCmp>(s, m.mQ, m.mKc, m.mVc, pp, st);
+    }
+    const long long rows = s.B * s.T * s.H;
+    NSA_LAUNCH("cmp_empty_kernel", st, cmp_empty_kernel<<<(unsigned)ceil_div(rows * s.DV, 256), 256, 0, st>>>(out, lse, rows, (int)s.DV));
+    return last_launch();
+}
+
+// selected branch under sel_idx: out += g_slc o_slc, lse[..., 1]
+template <int DK, int DV, int HG>
+nsa_status_t launch_sel(const Shape& s, const AttnMaps& m, const float* gates, float* out, float* lse,
+                        const int32_t* sel_idx, cudaStream_t st) {
+    SelParams sp{};
+    sp.B = (int)s.B;
+    sp.T = (int)s.T;
+    sp.H = (int)s.H;
+    sp.G = (int)s.G;
+    sp.n = (int)s.n;
+    sp.scale_log2 = s.scale * kLog2e;
+    sp.idx = sel_idx;
+    sp.gates = gates;
+    sp.out = out;
+    sp.lse_user = lse;
+    int64_t tpc = (s.B * s.T * s.G) / (148 * 8);
+    sp.tpc = (int)std::min<int64_t>(64, std::max<int64_t>(4, tpc));
+    using Cfg = SelCfg<DK, DV>;
+    NSA_TRY(set_smem(attn_sel_kernel<DK, DV, HG>, Cfg::kSmem));
+    sp.nchunks = (int)ceil_div(s.T, sp.tpc);
+    dim3 grid((unsigned)(sp.nchunks * s.G), 1, (unsigned)s.B);
+    NSA_LAUNCH("attn_sel_kernel", st, attn_sel_kernel<DK, DV, HG><<<grid, Cfg::kThreads, Cfg::kSmem, st>>>(m.mQs, m.mK, m.mVTs, sp));
+    return last_launch();
+}
+
+// sliding window: out += g_win o_win, lse[..., 2]
+template <int DK, int DV, int HG>
+nsa_status_t launch_win(const Shape& s, const AttnMaps& m, const float* gates, float* out, float* lse,
+                        cudaStream_t st) {
+    const PackedParams pp = packed_params<HG>(s, gates, out, lse, nullptr, nullptr);
+    return launch_packed_blk<DK, DV, HG, kModeWin>(s, m.mQ, m.mKw, m.mVT, pp, st);
+}
+
 // Keys and values of the three branches (page 2, 滑动窗口: the branches may
 // have independent keys and values).  The compressed branch compresses
 // (k_cmp, v_cmp); the selected branch reads (k_slc, v_slc) and the window
@@ -385,60 +494,10 @@ nsa_status_t forward_impl(const Shape& s, const void* q, const BranchKV& kv,
             (int)s.DVP, (int)s.Tp, reinterpret_cast<__nv_bfloat16*>(pass ? vTw : vT)));
         NSA_TRY(last_launch());
     }
-    // tensor maps
-    CUtensorMap mQ, mQs, mKc, mVc, mK, mVT, mVTs, mKw;
-    {
-        const uint64_t dQ[4] = {(uint64_t)s.DK, (uint64_t)s.H, (uint64_t)s.T, (uint64_t)s.B};
-        const uint64_t sQ[3] = {(uint64_t)s.DK * 2, (uint64_t)s.H * s.DK * 2, (uint64_t)s.T * s.H * s.DK * 2};
-        const uint32_t bQ[4] = {64, (uint32_t)HG, (uint32_t)(128 / HG), 1};
-        const uint32_t bQs[4] = {64, 16, 1, 1};
-        const uint64_t dK[4] = {(uint64_t)s.DK, (uint64_t)s.G, (uint64_t)s.T, (uint64_t)s.B};
-        const uint64_t sK[3] = {(uint64_t)s.DK * 2, (uint64_t)s.G * s.DK * 2, (uint64_t)s.T * s.G * s.DK * 2};
-        const uint32_t bK[4] = {64, 1, 64, 1};
-        const uint64_t dVT[4] = {(uint64_t)s.T, (uint64_t)s.DVP, (uint64_t)s.G, (uint64_t)s.B};
-        const uint64_t sVT[3] = {(uint64_t)s.Tp * 2, (uint64_t)s.DVP * s.Tp * 2, (uint64_t)s.G * s.DVP * s.Tp * 2};
-        const uint32_t bVT[4] = {64, (uint32_t)s.DV, 1, 1};
-        const uint32_t bVTs[4] = {64, 128, 1, 1};
-        if (!make_map(&mQ, q, 4, dQ, sQ, bQ) || !make_map(&mQs, q, 4, dQ, sQ, bQs) ||
-            !make_map(&mK, kv.k_slc, 4, dK, sK, bK) || !make_map(&mKw, kv.k_win, 4, dK, sK, bK) ||
-            !make_map(&mVT, vTw, 4, dVT, sVT, bVT) || !make_map(&mVTs, vT, 4, dVT, sVT, bVTs))
-            return NSA_ERR_CUDA;
-        if (s.C > 0) {
-            const uint64_t dKc[4] = {(uint64_t)s.DK, (uint64_t)s.G, (uint64_t)s.C, (uint64_t)s.B};
-            const uint64_t sKc[3] = {(uint64_t)s.DK * 2, (uint64_t)s.G * s.DK * 2, (uint64_t)s.C * s.G * s.DK * 2};
-            const uint64_t dVc[4] = {(uint64_t)s.C, (uint64_t)s.DV, (uint64_t)s.G, (uint64_t)s.B};
-            const uint64_t sVc[3] = {(uint64_t)s.Cp * 2, (uint64_t)s.DV * s.Cp * 2, (uint64_t)s.G * s.DV * s.Cp * 2};
-            const uint32_t bVc[4] = {64, (uint32_t)s.DV, 1, 1};
-            if (!make_map(&mKc, kc, 4, dKc, sKc, bK) || !make_map(&mVc, vcT, 4, dVc, sVc, bVc))
-                return NSA_ERR_CUDA;
-        }
-    }
-    PackedParams pp{};
-    pp.B = (int)s.B;
-    pp.T = (int)s.T;
-    pp.H = (int)s.H;
-    pp.G = (int)s.G;
-    pp.l = (int)s.l;
-    pp.d = (int)s.d;
-    pp.lp = (int)s.lp;
-    pp.w = (int)s.w;
-    pp.scale_log2 = s.scale * kLog2e;
-    pp.gates = gates;
-    pp.out = out;
-    pp.lse_user = lse;
-    pp.lse_cmp = lse_cmp;
-    pp.pscore = pscore;
-    pp.NSp = (int)s.NSp;
-    pp.n_ctas = (int)ceil_div(s.T, 2 * (128 / HG));
+    AttnMaps m;
+    NSA_TRY((attn_maps<DK, DV, HG>(s, q, kv.k_slc, kv.k_win, kc, vcT, vT, vTw, m)));
     // 3-4. compressed attention: LSE pass, then P.V~ with importance scores
-    if (s.C > 0) {
-        NSA_TRY((launch_packed_blk<DK, DV, HG, kModeLse>(s, mQ, mKc, mVc, pp, st)));
-        NSA_TRY((launch_packed_blk<DK, DV, HG, kModeCmp>(s, mQ, mKc, mVc, pp, st)));
-    } else {
-        const long long rows = s.B * s.T * s.H;
-        NSA_LAUNCH("cmp_empty_kernel", st, cmp_empty_kernel<<<(unsigned)ceil_div(rows * s.DV, 256), 256, 0, st>>>(out, lse, rows, (int)s.DV));
-        NSA_TRY(last_launch());
-    }
+    NSA_TRY((launch_cmp<DK, DV, HG>(s, m, gates, out, lse, lse_cmp, pscore, st)));
     // 5. top-n selection
     {
         const long long items = s.B * s.T * s.G;
@@ -455,37 +514,17 @@ nsa_status_t forward_impl(const Shape& s, const void* q, const BranchKV& kv,
         NSA_TRY(last_launch());
     }
     // 6. selected attention
-    {
-        SelParams sp{};
-        sp.B = (int)s.B;
-        sp.T = (int)s.T;
-        sp.H = (int)s.H;
-        sp.G = (int)s.G;
-        sp.n = (int)s.n;
-        sp.scale_log2 = s.scale * kLog2e;
-        sp.idx = sel_idx;
-        sp.gates = gates;
-        sp.out = out;
-        sp.lse_user = lse;
-        int64_t tpc = (s.B * s.T * s.G) / (148 * 8);
-        sp.tpc = (int)std::min<int64_t>(64, std::max<int64_t>(4, tpc));
-        using Cfg = SelCfg<DK, DV>;
-        NSA_TRY(set_smem(attn_sel_kernel<DK, DV, HG>, Cfg::kSmem));
-        sp.nchunks = (int)ceil_div(s.T, sp.tpc);
-        dim3 grid((unsigned)(sp.nchunks * s.G), 1, (unsigned)s.B);
-        NSA_LAUNCH("attn_sel_kernel", st, attn_sel_kernel<DK, DV, HG><<<grid, Cfg::kThreads, Cfg::kSmem, st>>>(mQs, mK, mVTs, sp));
-        NSA_TRY(last_launch());
-    }
+    NSA_TRY((launch_sel<DK, DV, HG>(s, m, gates, out, lse, sel_idx, st)));
     // 7. sliding window
-    NSA_TRY((launch_packed_blk<DK, DV, HG, kModeWin>(s, mQ, mKw, mVT, pp, st)));
-    return NSA_OK;
+    return launch_win<DK, DV, HG>(s, m, gates, out, lse, st);
 }
 
 
 // -------------------------------------------------------------- backward
 struct BwdWs {
     size_t off_kc, off_vc, off_vct, off_bias, off_lse2, off_dlt, off_dkc, off_dvc, off_cnt,
-        off_cur, off_off, off_choff, off_list, off_fix, total;
+        off_cur, off_off, off_choff, off_list, off_fix, off_ones, off_obuf, off_lsen, off_lsec, off_ps, off_vt,
+        total;
 };
 
 BwdWs bwd_layout(const Shape& s) {
@@ -521,6 +560,19 @@ BwdWs bwd_layout(const Shape& s) {
     o = align256(o + (size_t)s.B * s.T * s.G * s.n * 4);
     w.off_fix = o;
     o = align256(o + fix_bytes(s));
+    // per-branch statistics through the forward kernels
+    w.off_ones = o;
+    o = align256(o + (size_t)s.B * s.T * s.H * 3 * 4);
+    w.off_obuf = o;
+    o = align256(o + (size_t)s.B * s.T * s.H * s.DV * 4);
+    w.off_lsen = o;
+    o = align256(o + (size_t)s.B * s.T * s.H * 3 * 4);
+    w.off_lsec = o;
+    o = align256(o + (size_t)s.B * s.T * s.H * 4);
+    w.off_ps = o;
+    o = align256(o + (size_t)s.B * s.T * s.G * s.NSp * 4);
+    w.off_vt = o;
+    o = align256(o + (size_t)s.B * s.G * s.DVP * s.Tp * 2);
     w.total = o;
     return w;
 }
@@ -582,38 +634,139 @@ nsa_status_t backward_impl(const Shape& s, const void* q, const void* k, const v
         cudaMemsetAsync(ws + L.off_dkc, 0, L.off_cnt - L.off_dkc, st) != cudaSuccess ||
         cudaMemsetAsync(ws + L.off_cnt, 0, L.off_off - L.off_cnt, st) != cudaSuccess)
         return NSA_ERR_CUDA;
-    // per-query statistics, d(gates), dq (tensor cores, 16 heads = M)
+    // per-branch statistics under the given selection, from the forward kernels:
+    // with unit gates each branch's output is its own o_c, whose dot product with
+    // dO gives d(gate_c) and D_c = g_c <dO, o_c>; the kernels' LSEs come along
     {
+        constexpr int HG = DK == 192 ? 16 : 4;
+        const long long rows = s.B * s.T * s.H;
+        float* ones = reinterpret_cast<float*>(ws + L.off_ones);
+        float* obuf = reinterpret_cast<float*>(ws + L.off_obuf);
+        float* lsen = reinterpret_cast<float*>(ws + L.off_lsen);
+        void* vT = ws + L.off_vt;
+        NSA_LAUNCH("fill_f32", st, fill_f32<<<(unsigned)ceil_div(rows * 3, 256), 256, 0, st>>>(ones, rows * 3, 1.f));
+        NSA_TRY(last_launch());
+        dim3 tg((unsigned)ceil_div(s.Tp, 64), (unsigned)s.G, (unsigned)s.B);
+        NSA_LAUNCH("transpose_v_kernel", st, transpose_v_kernel<<<tg, dim3(64, 4), 0, st>>>(
+            reinterpret_cast<const __nv_bfloat16*>(v), (int)s.T, (int)s.G, (int)s.DV, (int)s.DVP, (int)s.Tp,
+            reinterpret_cast<__nv_bfloat16*>(vT)));
+        NSA_TRY(last_launch());
+        AttnMaps m;
+        NSA_TRY((attn_maps<DK, DV, HG>(s, q, k, k, ws + L.off_kc, ws + L.off_vct, vT, vT, m)));
+        const size_t obytes = (size_t)rows * DV * 4;
+        for (int br = 0; br < 3; ++br) {
+            if (br == 0) {
+                NSA_TRY((launch_cmp<DK, DV, HG>(s, m, ones, obuf, lsen, reinterpret_cast<float*>(ws + L.off_lsec),
+                                                reinterpret_cast<float*>(ws + L.off_ps), st)));
+            } else {
+                if (cudaMemsetAsync(obuf, 0, obytes, st) != cudaSuccess) return NSA_ERR_CUDA;
+                if (br == 1) NSA_TRY((launch_sel<DK, DV, HG>(s, m, ones, obuf, lsen, sel_idx, st)));
+                else NSA_TRY((launch_win<DK, DV, HG>(s, m, ones, obuf, lsen, st)));
+            }
+            NSA_LAUNCH("bwd_branch_stats", st, bwd_branch_stats<<<(unsigned)ceil_div(rows, 8), 256, 0, st>>>(
+                obuf, reinterpret_cast<const __nv_bfloat16*>(dout), gates, lsen, br, rows, DV, dgates, p.dlt, p.lse2));
+            NSA_TRY(last_launch());
+        }
+        p.have_stats = 1;
+    }
+    // dq of the selected branch (warp-level tensor cores, 16 heads = M); it writes dq
+    {
+        p.q_branches = 1 << kBrSlc;
         const int smem = bwd_query_mma_smem<DK, DV>();
         NSA_TRY(set_smem(bwd_query_mma<DK, DV>, smem));
         NSA_LAUNCH("bwd_query_mma", st, bwd_query_mma<DK, DV><<<dim3((unsigned)s.T, (unsigned)s.G, (unsigned)s.B), 128, smem, st>>>(p));
         NSA_TRY(last_launch());
     }
-    // inverse index of the selection: block -> tokens
+    // dq of the window and compressed branches (tcgen05, packed query tiles), added
     {
-        const long long N = s.B * s.T * s.G * s.n;
-        NSA_LAUNCH("bwd_sel_count", st, bwd_sel_count<<<(unsigned)ceil_div(N, 256), 256, 0, st>>>(p));
-        NSA_TRY(last_launch());
-        NSA_LAUNCH("bwd_sel_scan", st, bwd_sel_scan<<<1, 1024, 0, st>>>(p));
-        NSA_TRY(last_launch());
-        NSA_LAUNCH("bwd_sel_fill", st, bwd_sel_fill<<<(unsigned)ceil_div(N, 256), 256, 0, st>>>(p));
-        NSA_TRY(last_launch());
-    }
-    // key-centric dK/dV (tensor cores, 16 heads = N)
-    {
-        constexpr int kvs = bwd_kv_mma_smem<DK, DV>();
-        NSA_TRY(set_smem(bwd_kv_mma<DK, DV, kBrWin>, kvs));
-        NSA_TRY(set_smem(bwd_kv_mma<DK, DV, kBrSlc>, kvs));
-        NSA_TRY(set_smem(bwd_kv_mma<DK, DV, kBrCmp>, kvs));
-        dim3 gw((unsigned)ceil_div(s.T, 64), (unsigned)ceil_div(64 + s.w - 1, kBwdChunk), (unsigned)(s.B * s.G));
-        NSA_LAUNCH("bwd_kv_mma", st, bwd_kv_mma<DK, DV, kBrWin><<<gw, 128, kvs, st>>>(p));
-        NSA_TRY(last_launch());
-        const int64_t maxch = NE + ceil_div(s.B * s.T * s.G * s.n, kBwdChunk);
-        NSA_LAUNCH("bwd_kv_mma", st, bwd_kv_mma<DK, DV, kBrSlc><<<(unsigned)maxch, 128, kvs, st>>>(p));
+        constexpr int HG = DK == 192 ? 16 : 4;
+        using Cfg = BqCfg<DK, DV>;
+        CUtensorMap mQ, mO, mK, mV, mKc, mVc;
+        const uint32_t bQ[4] = {64, (uint32_t)HG, (uint32_t)(128 / HG), 1};
+        const uint32_t bKV[4] = {64, 1, 64, 1};
+        const uint64_t dQ[4] = {(uint64_t)DK, (uint64_t)s.H, (uint64_t)s.T, (uint64_t)s.B};
+        const uint64_t sQ[3] = {(uint64_t)DK * 2, (uint64_t)s.H * DK * 2, (uint64_t)s.T * s.H * DK * 2};
+        const uint64_t dO[4] = {(uint64_t)DV, (uint64_t)s.H, (uint64_t)s.T, (uint64_t)s.B};
+        const uint64_t sO[3] = {(uint64_t)DV * 2, (uint64_t)s.H * DV * 2, (uint64_t)s.T * s.H * DV * 2};
+        const uint64_t dK[4] = {(uint64_t)DK, (uint64_t)s.G, (uint64_t)s.T, (uint64_t)s.B};
+        const uint64_t sK[3] = {(uint64_t)DK * 2, (uint64_t)s.G * DK * 2, (uint64_t)s.T * s.G * DK * 2};
+        const uint64_t dV[4] = {(uint64_t)DV, (uint64_t)s.G, (uint64_t)s.T, (uint64_t)s.B};
+        const uint64_t sV[3] = {(uint64_t)DV * 2, (uint64_t)s.G * DV * 2, (uint64_t)s.T * s.G * DV * 2};
+        if (!make_map(&mQ, q, 4, dQ, sQ, bQ) || !make_map(&mO, dout, 4, dO, sO, bQ) ||
+            !make_map(&mK, k, 4, dK, sK, bKV) || !make_map(&mV, v, 4, dV, sV, bKV))
+            return NSA_ERR_CUDA;
+        NSA_TRY(set_smem(bwd_q_dense<DK, DV, HG, kBrWin>, Cfg::kSmem));
+        NSA_TRY(set_smem(bwd_q_dense<DK, DV, HG, kBrCmp>, Cfg::kSmem));
+        const dim3 grid((unsigned)ceil_div(s.T, 128 / HG), 1, (unsigned)(s.B * s.G));
+        NSA_LAUNCH("bwd_q_dense_win", st, bwd_q_dense<DK, DV, HG, kBrWin><<<grid, Cfg::kThreads, Cfg::kSmem, st>>>(mQ, mO, mK, mV, p));
         NSA_TRY(last_launch());
         if (s.C > 0) {
-            dim3 gc((unsigned)ceil_div(s.C, 64), (unsigned)ceil_div(s.T, kBwdChunk), (unsigned)(s.B * s.G));
-            NSA_LAUNCH("bwd_kv_mma", st, bwd_kv_mma<DK, DV, kBrCmp><<<gc, 128, kvs, st>>>(p));
+            const uint64_t dKc[4] = {(uint64_t)DK, (uint64_t)s.G, (uint64_t)s.C, (uint64_t)s.B};
+            const uint64_t sKc[3] = {(uint64_t)DK * 2, (uint64_t)s.G * DK * 2, (uint64_t)s.C * s.G * DK * 2};
+            const uint64_t dVc[4] = {(uint64_t)DV, (uint64_t)s.G, (uint64_t)s.C, (uint64_t)s.B};
+            const uint64_t sVc[3] = {(uint64_t)DV * 2, (uint64_t)s.G * DV * 2, (uint64_t)s.C * s.G * DV * 2};
+            if (!make_map(&mKc, ws + L.off_kc, 4, dKc, sKc, bKV) || !make_map(&mVc, ws + L.off_vc, 4, dVc, sVc, bKV))
+                return NSA_ERR_CUDA;
+            NSA_LAUNCH("bwd_q_dense_cmp", st, bwd_q_dense<DK, DV, HG, kBrCmp><<<grid, Cfg::kThreads, Cfg::kSmem, st>>>(mQ, mO, mKc, mVc, p));
+            NSA_TRY(last_launch());
+        }
+    }
+    // selected branch: block pairs -> the tokens that chose them (with which halves)
+    const int64_t NP = ceil_div(s.NS, 2);
+    const int64_t NEp = s.B * s.G * NP;
+    BkvParams kp{};
+    kp.bp = p;
+    kp.n_pairs = (int)NP;
+    kp.pcnt = p.cnt;
+    kp.poff = p.off;
+    kp.pchunk = p.chunk_off;
+    kp.plist = p.list;
+    {
+        const long long rows = s.B * s.T * s.G;
+        NSA_LAUNCH("bwd_pair_count", st, bwd_pair_count<<<(unsigned)ceil_div(rows, 256), 256, 0, st>>>(p, (int)NP, p.cnt));
+        NSA_TRY(last_launch());
+        NSA_LAUNCH("bwd_pair_scan", st, bwd_pair_scan<<<1, 1024, 0, st>>>((int)NEp, p.cnt, p.off, p.chunk_off));
+        NSA_TRY(last_launch());
+        NSA_LAUNCH("bwd_pair_fill", st, bwd_pair_fill<<<(unsigned)ceil_div(rows, 256), 256, 0, st>>>(p, (int)NP, p.off, p.cursor, p.list));
+        NSA_TRY(last_launch());
+    }
+    // key-centric dK/dV of the three branches (tcgen05, 128 keys per tile)
+    {
+        constexpr int HG = DK == 192 ? 16 : 4;
+        using Cfg = BkvCfg<DK, DV>;
+        CUtensorMap mK, mV, mKc, mVc, mQ, mO;
+        const uint32_t bKV[4] = {64, 1, 128, 1};
+        const uint64_t dK[4] = {(uint64_t)DK, (uint64_t)s.G, (uint64_t)s.T, (uint64_t)s.B};
+        const uint64_t sK[3] = {(uint64_t)DK * 2, (uint64_t)s.G * DK * 2, (uint64_t)s.T * s.G * DK * 2};
+        const uint64_t dV[4] = {(uint64_t)DV, (uint64_t)s.G, (uint64_t)s.T, (uint64_t)s.B};
+        const uint64_t sV[3] = {(uint64_t)DV * 2, (uint64_t)s.G * DV * 2, (uint64_t)s.T * s.G * DV * 2};
+        const uint32_t bR[4] = {64, (uint32_t)HG, (uint32_t)(kBkvRows / HG), 1};
+        const uint64_t dQ[4] = {(uint64_t)DK, (uint64_t)s.H, (uint64_t)s.T, (uint64_t)s.B};
+        const uint64_t sQ[3] = {(uint64_t)DK * 2, (uint64_t)s.H * DK * 2, (uint64_t)s.T * s.H * DK * 2};
+        const uint64_t dO[4] = {(uint64_t)DV, (uint64_t)s.H, (uint64_t)s.T, (uint64_t)s.B};
+        const uint64_t sO[3] = {(uint64_t)DV * 2, (uint64_t)s.H * DV * 2, (uint64_t)s.T * s.H * DV * 2};
+        if (!make_map(&mK, k, 4, dK, sK, bKV) || !make_map(&mV, v, 4, dV, sV, bKV) ||
+            !make_map(&mQ, q, 4, dQ, sQ, bR) || !make_map(&mO, dout, 4, dO, sO, bR))
+            return NSA_ERR_CUDA;
+        NSA_TRY(set_smem(bwd_kv_tc<DK, DV, HG, kBrWin>, Cfg::kSmem));
+        NSA_TRY(set_smem(bwd_kv_tc<DK, DV, HG, kBrSlc>, Cfg::kSmem));
+        NSA_TRY(set_smem(bwd_kv_tc<DK, DV, HG, kBrCmp>, Cfg::kSmem));
+        const unsigned bg = (unsigned)(s.B * s.G);
+        dim3 gw((unsigned)ceil_div(s.T, 128), (unsigned)ceil_div(128 + s.w - 1, kBkvChunk), bg);
+        NSA_LAUNCH("bwd_kv_tc_win", st, bwd_kv_tc<DK, DV, HG, kBrWin><<<gw, Cfg::kThreads, Cfg::kSmem, st>>>(mK, mV, mQ, mO, kp));
+        NSA_TRY(last_launch());
+        const int64_t maxch = NEp + ceil_div(s.B * s.T * s.G * s.n, kBkvChunk);
+        NSA_LAUNCH("bwd_kv_tc_slc", st, bwd_kv_tc<DK, DV, HG, kBrSlc><<<(unsigned)maxch, Cfg::kThreads, Cfg::kSmem, st>>>(mK, mV, mQ, mO, kp));
+        NSA_TRY(last_launch());
+        if (s.C > 0) {
+            const uint64_t dKc[4] = {(uint64_t)DK, (uint64_t)s.G, (uint64_t)s.C, (uint64_t)s.B};
+            const uint64_t sKc[3] = {(uint64_t)DK * 2, (uint64_t)s.G * DK * 2, (uint64_t)s.C * s.G * DK * 2};
+            const uint64_t dVc[4] = {(uint64_t)DV, (uint64_t)s.G, (uint64_t)s.C, (uint64_t)s.B};
+            const uint64_t sVc[3] = {(uint64_t)DV * 2, (uint64_t)s.G * DV * 2, (uint64_t)s.C * s.G * DV * 2};
+            if (!make_map(&mKc, ws + L.off_kc, 4, dKc, sKc, bKV) || !make_map(&mVc, ws + L.off_vc, 4, dVc, sVc, bKV))
+                return NSA_ERR_CUDA;
+            dim3 gc((unsigned)ceil_div(s.C, 128), (unsigned)ceil_div(s.T, kBkvChunk), bg);
+            NSA_LAUNCH("bwd_kv_tc_cmp", st, bwd_kv_tc<DK, DV, HG, kBrCmp><<<gc, Cfg::kThreads, Cfg::kSmem, st>>>(mKc, mVc, mQ, mO, kp));
             NSA_TRY(last_launch());
             dim3 gp((unsigned)s.T, (unsigned)s.G, (unsigned)s.B);
             NSA_LAUNCH("bwd_phiT_kernel", st, bwd_phiT_kernel<DK><<<gp, DK, 0, st>>>(p, p.dkc, p.wk, dk));

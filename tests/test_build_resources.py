@@ -54,7 +54,8 @@ def report():
 def test_every_kernel_is_reported(report):
     names = " ".join(r[0] for r in report)
     for k in ("attn_packed_kernel", "attn_sel_kernel", "topn_kernel", "phi_linear_kernel", "dec_cmp_stream",
-              "dec_slcwin_stream", "bwd_query_mma", "bwd_kv_mma", "decode_append_kernel", "phi_dw_kernel"):
+              "dec_slcwin_stream", "bwd_query_mma", "bwd_kv_tc", "bwd_q_dense", "decode_append_kernel",
+              "phi_dw_kernel"):
         assert k in names, k
 
 

@@ -205,8 +205,11 @@ nsa_status_t nsa_decode(const nsa_config_t* cfg, int32_t num_seqs, const void* q
  * forward's).  Out (fp32, overwritten): dq [B,T,H,d_k], dk [B,T,G,d_k],
  * dv [B,T,G,d_v] (through all three branches and, for the compressed branch,
  * through phi), dgates [B,T,H,3] = <dout, o_branch>.  The per-branch softmax
- * statistics are recomputed.  No gradient flows into the importance scores,
- * the phi parameters or the gate MLP. */
+ * statistics are recomputed (each branch once more forward under sel_idx), so
+ * any valid selection may be passed.  No gradient flows into the importance
+ * scores, the phi parameters or the gate MLP.  The BACKWARD workspace holds,
+ * besides the compressed keys and their gradients, one fp32 [B,T,H,d_v] branch
+ * output (about 1.1 GB at B=2, T=16384, H=64). */
 nsa_status_t nsa_backward(const nsa_config_t* cfg, const void* q, const void* k, const void* v,
                           const float* gates, const nsa_phi_params_t* phi, const void* dout,
                           const int32_t* sel_idx, float* dq, float* dk, float* dv, float* dgates,

@@ -10,13 +10,14 @@
 // tokens for the window, 128 compressed blocks for the compressed branch, a
 // pair of selection blocks (2m, 2m+1) for the selected branch -- and walks the
 // query rows that read them in steps of 64 rows (64/HG tokens x HG heads):
-//   S^T  = K Q^T       M = 128 keys, N = 64 rows, K = d_k   (TMEM, 2 buffers)
+//   S^T  = K Q^T       M = 128 keys, N = 64 rows, K = d_k   (TMEM)
 //   dP^T = V dO^T      M = 128 keys, N = 64 rows, K = d_v   (TMEM)
-//   softmax warps (thread = key): gP^T = g P^T and dS^T to shared memory (bf16)
+//   softmax warps (thread = key): gP^T = g P^T and dS^T back to TMEM (bf16)
 //   dV  += gP^T dO     M = 128 keys, N = d_v, K = 64 rows   (TMEM accumulator)
 //   dK  += dS^T Q      M = 128 keys, N = d_k, K = 64 rows   (TMEM accumulator)
-// The last two take Q / dO as transposed (MN-major) operands straight from the
-// tiles the first two read K-major, so each row tile is staged once.  The
+// The last two read gP^T / dS^T from tensor memory and take Q / dO as
+// transposed (MN-major) operands straight from the tiles the first two read
+// K-major, so each row tile is staged once (three stages in flight).  The
 // accumulated tile is added into dk/dv (dK~/dV~ for the compressed branch) in
 // fp32 at the end; several CTAs can share a key tile (token chunks).
 //
@@ -26,8 +27,9 @@
 // their rows).  A row's statistics (log2-domain LSE, D = g <dO, o>, g) come
 // from the per-query pass of the backward.
 //
-// Warps 0-3: softmax and epilogue (thread = key = TMEM lane); warp 4: loader
-// (TMA, or gather with warp 6); warp 5: MMA issuer and TMEM owner.
+// Warps 0-7: softmax and epilogue (a key per TMEM lane, warps 4-7 taking the
+// second half of each step's rows); warp 8: loader (TMA, or gather with warp
+// 10); warp 9: MMA issuer and TMEM owner.
 #pragma once
 #include "nsa_dev.cuh"
 #include "k_attn_packed.cuh"
@@ -60,6 +62,10 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
                  : "memory");
 }
 
+__device__ __forceinline__ void red_add_v1(float* p, float a) {
+    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(a) : "memory");
+}
+
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
@@ -67,25 +73,24 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
 template <int DK, int DV>
 struct BkvCfg {
     static constexpr int NQB = DK / 64, NVB = DV / 64;
+    static constexpr int NST = 3;                      // stages of query rows in flight
     static constexpr int kKTile = 128 * DK * 2;        // NQB boxes [128 keys][64]
     static constexpr int kVTile = 128 * DV * 2;
     static constexpr int kQStage = kBkvRows * DK * 2;  // NQB boxes [64 rows][64]
     static constexpr int kOStage = kBkvRows * DV * 2;
-    static constexpr int kPT = 128 * kBkvRows * 2;     // gP^T / dS^T: [128 keys][64 rows]
     static constexpr int kOffK = 0;
     static constexpr int kOffV = kOffK + kKTile;
     static constexpr int kOffQ = kOffV + kVTile;
-    static constexpr int kOffO = kOffQ + 2 * kQStage;
-    static constexpr int kOffGP = kOffO + 2 * kOStage;
-    static constexpr int kOffDS = kOffGP + kPT;
-    static constexpr int kOffStat = kOffDS + kPT;      // 2 stages x 5 arrays x 64
+    static constexpr int kOffO = kOffQ + NST * kQStage;
+    static constexpr int kOffStat = kOffO + NST * kOStage;   // NST stages x 5 arrays x 64
     static constexpr int kStatBytes = 5 * kBkvRows * 4;
-    static constexpr int kOffBar = kOffStat + 2 * kStatBytes;
+    static constexpr int kOffBar = kOffStat + NST * kStatBytes;
     static constexpr int kSmem = kOffBar + 256 + 1024;
     static_assert(kSmem <= 232448, "shared memory");
-    static constexpr int kThreads = 224;
-    // TMEM columns: S^T buffers 0 / 64, dP^T 128, dV 192, dK 192 + DV
-    static constexpr uint32_t kColDP = 128, kColDV = 192, kColDK = 192 + DV;
+    static constexpr int kThreads = 352;
+    // TMEM columns: S^T 0, gP^T 64 and dS^T 96 (bf16 pairs: the A operands of the
+    // gradient products), dP^T 128, dV 192, dK 192 + DV
+    static constexpr uint32_t kColGP = 64, kColDS = 96, kColDP = 128, kColDV = 192, kColDK = 192 + DV;
     static_assert(kColDK + DK <= 512, "tensor memory");
 };
 
@@ -99,7 +104,7 @@ struct BkvParams {
 };
 
 template <int DK, int DV, int HG, int BR>
-__global__ void __launch_bounds__(224, 1)
+__global__ void __launch_bounds__(352, 1)
     bwd_kv_tc(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
               const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapO,
               const BkvParams P) {
@@ -149,10 +154,10 @@ __global__ void __launch_bounds__(224, 1)
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
     uint64_t* kvfull = bars + 0;
-    uint64_t* stfull = bars + 1;    // [2]
-    uint64_t* stempty = bars + 3;   // [2]
-    uint64_t* sfull = bars + 5;     // [2]
-    uint64_t* sfree = bars + 7;     // [2]
+    uint64_t* stfull = bars + 1;    // [NST]
+    uint64_t* stempty = bars + 4;   // [NST]
+    uint64_t* sfull = bars + 7;
+    uint64_t* sfree = bars + 8;
     uint64_t* dpfull = bars + 9;
     uint64_t* dpfree = bars + 10;
     uint64_t* pfull = bars + 11;
@@ -164,21 +169,21 @@ __global__ void __launch_bounds__(224, 1)
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     if (threadIdx.x == 0) {
         mbar_init(kvfull, 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < Cfg::NST; ++s) {
             mbar_init(&stfull[s], BR == kBrSlc ? 2 : 1);
             mbar_init(&stempty[s], 1);
-            mbar_init(&sfull[s], 1);
-            mbar_init(&sfree[s], 4);
         }
+        mbar_init(sfull, 1);
+        mbar_init(sfree, 8);
         mbar_init(dpfull, 1);
-        mbar_init(dpfree, 4);
-        mbar_init(pfull, 4);
+        mbar_init(dpfree, 8);
+        mbar_init(pfull, 8);
         mbar_init(pempty, 1);
         mbar_init(accfull, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == 9) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
@@ -187,7 +192,7 @@ __global__ void __launch_bounds__(224, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    float* st_lse = reinterpret_cast<float*>(smem + Cfg::kOffStat);      // [2][5][64]
+    float* st_lse = reinterpret_cast<float*>(smem + Cfg::kOffStat);      // [NST][5][64]
     auto stat = [&](int st, int a) -> float* { return st_lse + (st * 5 + a) * kBkvRows; };
     // warp-collective wait: lane 0 polls, every lane gets the outcome
     auto lane0_wait = [&](uint64_t* bar, uint32_t parity, unsigned site) -> bool {
@@ -196,9 +201,9 @@ __global__ void __launch_bounds__(224, 1)
         return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     };
 
-    if (warp == 4 || (BR == kBrSlc && warp == 6)) {
+    if (warp == 8 || (BR == kBrSlc && warp == 10)) {
         // -------------------------------------------------------- loader
-        if (warp == 4) {                            // the key tile (rows past the keys: zeros)
+        if (warp == 8) {                            // the key tile (rows past the keys: zeros)
             if (lane == 0) mbar_expect_tx(kvfull, Cfg::kKTile + Cfg::kVTile);
             __syncwarp();
             if (lane < Cfg::NQB)
@@ -208,9 +213,11 @@ __global__ void __launch_bounds__(224, 1)
                             (lane - Cfg::NQB) * 64, g, key0, b);
         }
         if (BR != kBrSlc) {
-            for (int j = 0; j < nsteps; ++j) {
-                const int st = j & 1;
-                if (j >= 2 && !lane0_wait(&stempty[st], ((j - 2) >> 1) & 1, 0x401)) break;
+            // a step's row statistics are read into registers one step ahead, so
+            // their latency overlaps the previous step
+            float rl[2], rd[2], rg[2];
+            int rt[2];
+            auto load_stats = [&](int j) {
                 const int t0 = tok_lo + j * TPS;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
@@ -218,10 +225,24 @@ __global__ void __launch_bounds__(224, 1)
                     const int t = t0 + cc / HG, h = cc % HG;
                     const bool valid = t < tok_hi;
                     const size_t r3 = (((size_t)b * p.T + (valid ? t : 0)) * p.H + (size_t)g * HG + h) * 3 + BR;
-                    stat(st, 0)[cc] = valid ? p.lse2[r3] : INFINITY;
-                    stat(st, 1)[cc] = valid ? p.dlt[r3] : 0.f;
-                    stat(st, 2)[cc] = valid ? p.gates[r3] : 0.f;
-                    reinterpret_cast<int*>(stat(st, 3))[cc] = valid ? t : -1;
+                    rl[half] = valid ? p.lse2[r3] : INFINITY;
+                    rd[half] = valid ? p.dlt[r3] : 0.f;
+                    rg[half] = valid ? p.gates[r3] : 0.f;
+                    rt[half] = valid ? t : -1;
+                }
+            };
+            load_stats(0);
+            for (int j = 0; j < nsteps; ++j) {
+                const int st = j % Cfg::NST;
+                const int t0 = tok_lo + j * TPS;
+                if (j >= Cfg::NST && !lane0_wait(&stempty[st], ((j / Cfg::NST) - 1) & 1, 0x401)) break;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const int cc = lane + 32 * half;
+                    stat(st, 0)[cc] = rl[half];
+                    stat(st, 1)[cc] = rd[half];
+                    stat(st, 2)[cc] = rg[half];
+                    reinterpret_cast<int*>(stat(st, 3))[cc] = rt[half];
                     reinterpret_cast<int*>(stat(st, 4))[cc] = 3;
                 }
                 __syncwarp();
@@ -233,32 +254,44 @@ __global__ void __launch_bounds__(224, 1)
                 else if (lane < Cfg::NQB + Cfg::NVB)
                     tma_load_4d(smem + Cfg::kOffO + st * Cfg::kOStage + (lane - Cfg::NQB) * 8192, &mapO,
                                 &stfull[st], (lane - Cfg::NQB) * 64, g * HG, t0, b);
+                if (j + 1 < nsteps) load_stats(j + 1);
             }
         } else {
             // gather: thread cc (0..63) stages query row cc of each step with 16-byte
             // copies into the 128-byte-swizzled tiles.  A step is posted as soon as its
             // copies land, before the wait for the next stage: the MMA that frees that
-            // stage runs only after the posted step's products have been issued.
-            const int cc = (warp == 4 ? 0 : 32) + lane;
+            // stage runs only after the posted step's products have been issued.  The
+            // list entry and row statistics of a step are read one step ahead.
+            const int cc = (warp == 8 ? 0 : 32) + lane;
             const int tk = cc / HG, h = cc % HG;
+            bool valid;
+            int ent;
+            float rl, rd, rg;
+            auto load_entry = [&](int j) {
+                const int e = tok_lo + j * TPS + tk;
+                valid = e < tok_hi;
+                ent = valid ? __ldg(P.plist + e) : 0;
+                const size_t row = ((size_t)b * p.T + (ent & 0x3FFFFFFF)) * p.H + (size_t)g * HG + h;
+                rl = valid ? p.lse2[row * 3 + BR] : INFINITY;
+                rd = valid ? p.dlt[row * 3 + BR] : 0.f;
+                rg = valid ? p.gates[row * 3 + BR] : 0.f;
+            };
+            load_entry(0);
             for (int j = 0; j <= nsteps; ++j) {
                 if (j >= 1) {
                     asm volatile("cp.async.wait_group 0;" ::: "memory");
                     fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&stfull[(j - 1) & 1]);
+                    if (lane == 0) mbar_arrive(&stfull[(j - 1) % Cfg::NST]);
                 }
                 if (j == nsteps) break;
-                const int st = j & 1;
-                if (j >= 2 && !lane0_wait(&stempty[st], ((j - 2) >> 1) & 1, 0x402)) break;
-                const int e = tok_lo + j * TPS + tk;
-                const bool valid = e < tok_hi;
-                const int ent = valid ? P.plist[e] : 0;
+                const int st = j % Cfg::NST;
+                if (j >= Cfg::NST && !lane0_wait(&stempty[st], ((j / Cfg::NST) - 1) & 1, 0x402)) break;
                 const int t = ent & 0x3FFFFFFF;
                 const size_t row = ((size_t)b * p.T + t) * p.H + (size_t)g * HG + h;
-                stat(st, 0)[cc] = valid ? p.lse2[row * 3 + BR] : INFINITY;
-                stat(st, 1)[cc] = valid ? p.dlt[row * 3 + BR] : 0.f;
-                stat(st, 2)[cc] = valid ? p.gates[row * 3 + BR] : 0.f;
+                stat(st, 0)[cc] = rl;
+                stat(st, 1)[cc] = rd;
+                stat(st, 2)[cc] = rg;
                 reinterpret_cast<int*>(stat(st, 3))[cc] = valid ? t : -1;
                 reinterpret_cast<int*>(stat(st, 4))[cc] = (int)((unsigned)ent >> 30);
                 const uint32_t sq = smem_u32(smem + Cfg::kOffQ + st * Cfg::kQStage);
@@ -285,86 +318,120 @@ __global__ void __launch_bounds__(224, 1)
                         for (int c = 0; c < 8; ++c) st_shared_v4(so + bx * 8192 + sw128_off(cc, c), 0, 0, 0, 0);
                 }
                 asm volatile("cp.async.commit_group;" ::: "memory");
+                if (j + 1 < nsteps) load_entry(j + 1);
             }
             asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ----------------------------------------------------------- MMA
         if (lane == 0) {
             constexpr uint32_t idS = idesc_bf16(128, kBkvRows);
             constexpr uint32_t idV = idesc_bf16_bmn(128, DV);
             constexpr uint32_t idK = idesc_bf16_bmn(128, DK);
             const uint32_t sK = smem_u32(smem + Cfg::kOffK), sV = smem_u32(smem + Cfg::kOffV);
-            const uint32_t sGP = smem_u32(smem + Cfg::kOffGP), sDS = smem_u32(smem + Cfg::kOffDS);
             bool ok = wait_or_abort(kvfull, 0, 0x403, abort_flag);
-            auto grad = [&](int i) -> bool {
-                const int st = i & 1;
-                if (!wait_or_abort(pfull, i & 1, 0x404, abort_flag)) return false;
-                tc_fence_after();
-                const uint32_t sQ = smem_u32(smem + Cfg::kOffQ + st * Cfg::kQStage);
-                const uint32_t sO = smem_u32(smem + Cfg::kOffO + st * Cfg::kOStage);
+            // Two independent streams of products: S^T/dP^T of step js (when its rows
+            // are staged and its TMEM buffers free) and dV/dK of step jg (when its
+            // gP^T/dS^T are written).  Each is issued as soon as it is ready, so the
+            // gradient products of a step never wait for the next step's rows.
+            int js = 0, jg = 0;
+            unsigned long long t_idle = 0;
+            uint32_t spins = 0;
+            while (ok && jg < nsteps) {
+                bool progressed = false;
+                if (js < nsteps) {
+                    const int st = js % Cfg::NST;
+                    const bool ready = mbar_test_wait(&stfull[st], (js / Cfg::NST) & 1) &&
+                                       (js < 1 || (mbar_test_wait(sfree, (js - 1) & 1) &&
+                                                   mbar_test_wait(dpfree, (js - 1) & 1)));
+                    if (ready) {
+                        tc_fence_after();
+                        const uint32_t sQ = smem_u32(smem + Cfg::kOffQ + st * Cfg::kQStage);
+                        const uint32_t sO = smem_u32(smem + Cfg::kOffO + st * Cfg::kOStage);
 #pragma unroll
-                for (int kk = 0; kk < kBkvRows / 16; ++kk)
-                    umma_bf16_ss(tmem + Cfg::kColDV, sdesc_sw128(sGP + kk * 32),
-                                 sdesc_sw128_mn(sO + kk * 2048, 8192, 1024), idV, (i > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < DK / 16; ++kk)
+                            umma_bf16_ss(tmem, sdesc_sw128(sK + (kk / 4) * 16384 + (kk % 4) * 32),
+                                         sdesc_sw128(sQ + (kk / 4) * 8192 + (kk % 4) * 32), idS, kk > 0 ? 1u : 0u);
+                        umma_commit(sfull);
 #pragma unroll
-                for (int kk = 0; kk < kBkvRows / 16; ++kk)
-                    umma_bf16_ss(tmem + Cfg::kColDK, sdesc_sw128(sDS + kk * 32),
-                                 sdesc_sw128_mn(sQ + kk * 2048, 8192, 1024), idK, (i > 0 || kk > 0) ? 1u : 0u);
-                umma_commit(&stempty[st]);
-                umma_commit(pempty);
-                return true;
-            };
-            for (int j = 0; j < nsteps && ok; ++j) {
-                const int st = j & 1;
-                if (!(ok = wait_or_abort(&stfull[st], (j >> 1) & 1, 0x405, abort_flag))) break;
-                if (j >= 2 && !(ok = wait_or_abort(&sfree[st], ((j - 2) >> 1) & 1, 0x406, abort_flag))) break;
-                tc_fence_after();
-                const uint32_t sQ = smem_u32(smem + Cfg::kOffQ + st * Cfg::kQStage);
-                const uint32_t sO = smem_u32(smem + Cfg::kOffO + st * Cfg::kOStage);
+                        for (int kk = 0; kk < DV / 16; ++kk)
+                            umma_bf16_ss(tmem + Cfg::kColDP, sdesc_sw128(sV + (kk / 4) * 16384 + (kk % 4) * 32),
+                                         sdesc_sw128(sO + (kk / 4) * 8192 + (kk % 4) * 32), idS, kk > 0 ? 1u : 0u);
+                        umma_commit(dpfull);
+                        ++js;
+                        progressed = true;
+                    }
+                }
+                if (jg < js && mbar_test_wait(pfull, jg & 1)) {
+                    const int st = jg % Cfg::NST;
+                    tc_fence_after();
+                    const uint32_t sQ = smem_u32(smem + Cfg::kOffQ + st * Cfg::kQStage);
+                    const uint32_t sO = smem_u32(smem + Cfg::kOffO + st * Cfg::kOStage);
 #pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk)
-                    umma_bf16_ss(tmem + st * 64, sdesc_sw128(sK + (kk / 4) * 16384 + (kk % 4) * 32),
-                                 sdesc_sw128(sQ + (kk / 4) * 8192 + (kk % 4) * 32), idS, kk > 0 ? 1u : 0u);
-                umma_commit(&sfull[st]);
-                if (j >= 1 && !(ok = wait_or_abort(dpfree, (j - 1) & 1, 0x407, abort_flag))) break;
-                tc_fence_after();
+                    for (int kk = 0; kk < kBkvRows / 16; ++kk)
+                        umma_bf16_ts(tmem + Cfg::kColDV, tmem + Cfg::kColGP + kk * 8,
+                                     sdesc_sw128_mn(sO + kk * 2048, 8192, 1024), idV, (jg > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-                for (int kk = 0; kk < DV / 16; ++kk)
-                    umma_bf16_ss(tmem + Cfg::kColDP, sdesc_sw128(sV + (kk / 4) * 16384 + (kk % 4) * 32),
-                                 sdesc_sw128(sO + (kk / 4) * 8192 + (kk % 4) * 32), idS, kk > 0 ? 1u : 0u);
-                umma_commit(dpfull);
-                if (j >= 1) ok = grad(j - 1);
+                    for (int kk = 0; kk < kBkvRows / 16; ++kk)
+                        umma_bf16_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDS + kk * 8,
+                                     sdesc_sw128_mn(sQ + kk * 2048, 8192, 1024), idK, (jg > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&stempty[st]);
+                    umma_commit(pempty);
+                    ++jg;
+                    progressed = true;
+                }
+                // bounded: no progress for the wait limit ends the CTA with an error
+                if (progressed) {
+                    spins = 0;
+                } else if ((++spins & 63u) == 0u) {
+                    if (*abort_flag) {
+                        ok = false;
+                    } else {
+                        const unsigned long long now = globaltimer_ns();
+                        if (t_idle == 0) t_idle = now;
+                        else if (now - t_idle > kWaitLimitNs) {
+                            record_timeout(0x404);
+                            *abort_flag = 1;
+                            ok = false;
+                        }
+                    }
+                }
+                if (progressed) t_idle = 0;
             }
-            if (ok) ok = grad(nsteps - 1);
             umma_commit(accfull);               // also on the abort path: the epilogue waits on it
         }
-    } else if (warp < 4) {
+    } else if (warp < 8) {
         // ------------------------------------------------- softmax, epilogue
-        const int kl = warp * 32 + lane;                     // key within the tile = TMEM lane
+        // warp w: keys 32 (w % 4) .. +31 (its TMEM lane quadrant), query rows
+        // 32 (w / 4) .. +31 of each step
+        const int quad = warp & 3, hc = warp >> 2;
+        const int kl = quad * 32 + lane;                     // key within the tile = TMEM lane
         const int u = key0 + kl;
         const bool key_ok = u < nkeys;
         const int half = kl >> 6;                            // selected branch: block 2m or 2m+1
-        const uint32_t lanebase = tmem + ((uint32_t)(warp * 32) << 16);
-        const uint32_t rowGP = smem_u32(smem + Cfg::kOffGP), rowDS = smem_u32(smem + Cfg::kOffDS);
+        const uint32_t lanebase = tmem + ((uint32_t)(quad * 32) << 16);
         const float c = p.scale_log2;
+        constexpr int TPH = 32 / HG > 0 ? 32 / HG : 1;       // tokens among this warp's 32 rows
         bool ok = true;
         for (int j = 0; j < nsteps; ++j) {
-            const int st = j & 1;
+            const int st = j % Cfg::NST;
             // the step's row statistics (written by the loader before it posted the stage)
-            if (!(ok = lane0_wait(&stfull[st], (j >> 1) & 1, 0x40C))) break;
-            if (!(ok = lane0_wait(&sfull[st], (j >> 1) & 1, 0x408))) break;
+            if (!(ok = lane0_wait(&stfull[st], (j / Cfg::NST) & 1, 0x40C))) break;
+            if (!(ok = lane0_wait(sfull, j & 1, 0x408))) break;
             if (!(ok = lane0_wait(dpfull, j & 1, 0x409))) break;
             tc_fence_after();
-            const float4* L4 = reinterpret_cast<const float4*>(stat(st, 0));
-            const float4* D4 = reinterpret_cast<const float4*>(stat(st, 1));
-            const float4* G4 = reinterpret_cast<const float4*>(stat(st, 2));
-            const int* TK = reinterpret_cast<const int*>(stat(st, 3));
-            const int* BT = reinterpret_cast<const int*>(stat(st, 4));
-            // does each of the step's tokens see this key?
-            bool vt[TPS];
+            uint32_t sr[32], dr[32];
+            tmem_ld32(lanebase + hc * 32, sr);
+            tmem_ld32(lanebase + Cfg::kColDP + hc * 32, dr);
+            const float4* L4 = reinterpret_cast<const float4*>(stat(st, 0) + hc * 32);
+            const float4* D4 = reinterpret_cast<const float4*>(stat(st, 1) + hc * 32);
+            const float4* G4 = reinterpret_cast<const float4*>(stat(st, 2) + hc * 32);
+            const int* TK = reinterpret_cast<const int*>(stat(st, 3)) + hc * 32;
+            const int* BT = reinterpret_cast<const int*>(stat(st, 4)) + hc * 32;
+            // does each of this warp's tokens see this key?
+            bool vt[TPH];
 #pragma unroll
-            for (int tk = 0; tk < TPS; ++tk) {
+            for (int tk = 0; tk < TPH; ++tk) {
                 const int t = TK[tk * HG];
                 bool v = key_ok && t >= 0;
                 if constexpr (BR == kBrWin) v = v && u <= t && u > t - p.w;
@@ -372,91 +439,63 @@ __global__ void __launch_bounds__(224, 1)
                 else v = v && u <= t && ((BT[tk * HG] >> half) & 1);
                 vt[tk] = v;
             }
-            // two halves of 32 rows: S^T and dP^T columns, then gP^T and dS^T in bf16
-            // pairs, stored as soon as the previous step's dV / dK products have read
-            // the tiles
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                uint32_t sr[32], dr[32];
-                tmem_ld32(lanebase + st * 64 + hf * 32, sr);
-                tmem_ld32(lanebase + Cfg::kColDP + hf * 32, dr);
-                tmem_wait_ld32(sr);
-                tmem_wait_ld32(dr);
-                if (hf == 1) {                      // both TMEM buffers read: release them
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) {
-                        mbar_arrive(&sfree[st]);
-                        mbar_arrive(dpfree);
-                    }
-                }
-                uint32_t gp[16], dsv[16];
-#pragma unroll
-                for (int q4 = 0; q4 < 8; ++q4) {    // 4 columns per statistics load
-                    const int c0 = hf * 32 + q4 * 4;
-                    const float4 l4 = L4[c0 / 4], d4 = D4[c0 / 4], g4 = G4[c0 / 4];
-                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-                    const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
-                    const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
-                    float pv[4], dsn[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int col = c0 + e;
-                        const float sv = __uint_as_float(sr[q4 * 4 + e]);
-                        const float dpv = __uint_as_float(dr[q4 * 4 + e]);
-                        const float pr = vt[col / HG] ? ex2a(fmaf(sv, c, -lv[e])) : 0.f;
-                        pv[e] = gv[e] * pr;
-                        dsn[e] = pr * fmaf(gv[e], dpv, -dv[e]);
-                    }
-                    gp[q4 * 2] = pack_bf16x2(pv[0], pv[1]);
-                    gp[q4 * 2 + 1] = pack_bf16x2(pv[2], pv[3]);
-                    dsv[q4 * 2] = pack_bf16x2(dsn[0], dsn[1]);
-                    dsv[q4 * 2 + 1] = pack_bf16x2(dsn[2], dsn[3]);
-                }
-                if (hf == 0 && j >= 1 && !(ok = lane0_wait(pempty, (j - 1) & 1, 0x40A))) break;
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    st_shared_v4(rowGP + sw128_off(kl, hf * 4 + ch), gp[4 * ch], gp[4 * ch + 1], gp[4 * ch + 2],
-                                 gp[4 * ch + 3]);
-                    st_shared_v4(rowDS + sw128_off(kl, hf * 4 + ch), dsv[4 * ch], dsv[4 * ch + 1], dsv[4 * ch + 2],
-                                 dsv[4 * ch + 3]);
-                }
+            tmem_wait_ld32(sr);
+            tmem_wait_ld32(dr);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {                                 // this warp's columns are read
+                mbar_arrive(sfree);
+                mbar_arrive(dpfree);
             }
-            if (!ok) break;
-            fence_proxy_async_smem();
+            uint32_t gp[16], dsv[16];
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4) {                 // 4 rows per statistics load
+                const float4 l4 = L4[q4], d4 = D4[q4], g4 = G4[q4];
+                const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+                const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
+                float pv[4], dsn[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int col = q4 * 4 + e;
+                    const float pr = vt[col / HG] ? ex2a(fmaf(__uint_as_float(sr[col]), c, -lv[e])) : 0.f;
+                    pv[e] = gv[e] * pr;
+                    dsn[e] = pr * fmaf(gv[e], __uint_as_float(dr[col]), -dv[e]);
+                }
+                gp[q4 * 2] = pack_bf16x2(pv[0], pv[1]);
+                gp[q4 * 2 + 1] = pack_bf16x2(pv[2], pv[3]);
+                dsv[q4 * 2] = pack_bf16x2(dsn[0], dsn[1]);
+                dsv[q4 * 2 + 1] = pack_bf16x2(dsn[2], dsn[3]);
+            }
+            // the previous step's dV / dK products have read gP^T / dS^T
+            if (j >= 1 && !(ok = lane0_wait(pempty, (j - 1) & 1, 0x40A))) break;
+            tc_fence_after();
+            // this warp's 32 rows: K-steps 2 hc and 2 hc + 1 of the gradient products
+            tmem_st16(lanebase + Cfg::kColGP + hc * 16, gp);
+            tmem_st16(lanebase + Cfg::kColDS + hc * 16, dsv);
+            tmem_wait_st();
+            tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(pfull);
         }
-        // epilogue: add the tile's dV and scale * dK into the fp32 gradients
+        // epilogue: the tile's dV (warps 0-3) and scale * dK (warps 4-7) added into
+        // the fp32 gradients
         if (lane0_wait(accfull, 0, 0x40B) && ok) {
             tc_fence_after();
-            float* dvb = BR == kBrCmp ? p.dvc : p.dv;
-            float* dkb = BR == kBrCmp ? p.dkc : p.dk;
             const size_t rowk = ((size_t)b * nkeys + (key_ok ? u : 0)) * p.G + g;
+            const int ncol = hc == 0 ? DV : DK;
+            const uint32_t col0 = hc == 0 ? Cfg::kColDV : Cfg::kColDK;
+            float* dst = (hc == 0 ? (BR == kBrCmp ? p.dvc : p.dv) : (BR == kBrCmp ? p.dkc : p.dk)) + rowk * ncol;
+            const float sc = hc == 0 ? 1.f : p.scale;
 #pragma unroll 1
-            for (int c0 = 0; c0 < DV; c0 += 32) {
+            for (int c0 = 0; c0 < ncol; c0 += 32) {
                 uint32_t r[32];
-                tmem_ld32(lanebase + Cfg::kColDV + c0, r);
+                tmem_ld32(lanebase + col0 + c0, r);
                 tmem_wait_ld32(r);
                 if (key_ok) {
-                    float* dst = dvb + rowk * DV + c0;
 #pragma unroll
                     for (int e = 0; e < 32; e += 4)
-                        red_add_v4(dst + e, __uint_as_float(r[e]), __uint_as_float(r[e + 1]),
-                                   __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
-                }
-            }
-#pragma unroll 1
-            for (int c0 = 0; c0 < DK; c0 += 32) {
-                uint32_t r[32];
-                tmem_ld32(lanebase + Cfg::kColDK + c0, r);
-                tmem_wait_ld32(r);
-                if (key_ok) {
-                    float* dst = dkb + rowk * DK + c0;
-                    const float sc = p.scale;
-#pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        red_add_v4(dst + e, sc * __uint_as_float(r[e]), sc * __uint_as_float(r[e + 1]),
+                        red_add_v4(dst + c0 + e, sc * __uint_as_float(r[e]), sc * __uint_as_float(r[e + 1]),
                                    sc * __uint_as_float(r[e + 2]), sc * __uint_as_float(r[e + 3]));
                 }
             }
@@ -464,7 +503,7 @@ __global__ void __launch_bounds__(224, 1)
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
@@ -472,22 +511,23 @@ __global__ void __launch_bounds__(224, 1)
 
 // ------------------------------------ selected branch: block pairs -> tokens
 // For every (b, t, g) row of the selection, each distinct pair m = j/2 of its
-// selected blocks j, with bit h set when block 2m + h was chosen.
-__device__ __forceinline__ int pair_entries(const int32_t* r, int n, int nsb, int (&pr)[16], int (&bits)[16]) {
-    int np = 0;
-    for (int a = 0; a < n && a < 16; ++a) {
+// selected blocks j, with bit h set when block 2m + h was chosen: emit(m, bits)
+// once per pair (the row is ascending, so a pair's blocks are adjacent).
+template <typename F>
+__device__ __forceinline__ void for_each_pair(const int32_t* r, int n, int nsb, F&& emit) {
+    int cur = -1, bits = 0;
+    for (int a = 0; a < n; ++a) {
         const int j = r[a];
         if (j < 0 || j >= nsb) break;
         const int m = j >> 1;
-        if (np > 0 && pr[np - 1] == m) {
-            bits[np - 1] |= 1 << (j & 1);
-        } else {
-            pr[np] = m;
-            bits[np] = 1 << (j & 1);
-            ++np;
+        if (m != cur) {
+            if (cur >= 0) emit(cur, bits);
+            cur = m;
+            bits = 0;
         }
+        bits |= 1 << (j & 1);
     }
-    return np;
+    if (cur >= 0) emit(cur, bits);
 }
 
 __global__ void bwd_pair_count(const BwdParams p, int n_pairs, int* pcnt) {
@@ -495,9 +535,8 @@ __global__ void bwd_pair_count(const BwdParams p, int n_pairs, int* pcnt) {
     if (i >= (long long)p.B * p.T * p.G) return;
     const int g = (int)(i % p.G);
     const int b = (int)(i / ((long long)p.T * p.G));
-    int pr[16], bits[16];
-    const int np = pair_entries(p.idx + i * p.n, p.n, p.NSb, pr, bits);
-    for (int a = 0; a < np; ++a) atomicAdd(&pcnt[((size_t)b * p.G + g) * n_pairs + pr[a]], 1);
+    int* base = pcnt + ((size_t)b * p.G + g) * n_pairs;
+    for_each_pair(p.idx + i * p.n, p.n, p.NSb, [&](int m, int) { atomicAdd(base + m, 1); });
 }
 
 // single CTA: poff = exclusive scan of pcnt, pchunk = scan of ceil(pcnt / chunk)
@@ -541,13 +580,11 @@ __global__ void bwd_pair_fill(const BwdParams p, int n_pairs, const int* poff, i
     const int g = (int)(i % p.G);
     const int t = (int)((i / p.G) % p.T);
     const int b = (int)(i / ((long long)p.T * p.G));
-    int pr[16], bits[16];
-    const int np = pair_entries(p.idx + i * p.n, p.n, p.NSb, pr, bits);
-    for (int a = 0; a < np; ++a) {
-        const size_t e = ((size_t)b * p.G + g) * n_pairs + pr[a];
-        const int pos = atomicAdd(&cursor[e], 1);
-        plist[poff[e] + pos] = (int)((unsigned)t | ((unsigned)bits[a] << 30));
-    }
+    const size_t e0 = ((size_t)b * p.G + g) * n_pairs;
+    for_each_pair(p.idx + i * p.n, p.n, p.NSb, [&](int m, int bits) {
+        const int pos = atomicAdd(&cursor[e0 + m], 1);
+        plist[poff[e0 + m] + pos] = (int)((unsigned)t | ((unsigned)bits << 30));
+    });
 }
 
 }  // namespace nsa

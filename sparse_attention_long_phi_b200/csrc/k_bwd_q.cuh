@@ -7,12 +7,13 @@
 // group, the packed layout of the forward) and walks its keys in tiles of 64:
 //   S  = Q K^T    M = 128 rows, N = 64 keys, K = d_k   (TMEM, 2 buffers)
 //   dP = dO V^T   M = 128 rows, N = 64 keys, K = d_v   (TMEM, 2 buffers)
-//   softmax warps (thread = row): dS in bf16 over the first 32 columns of S
+//   softmax warps (thread = row): dS in bf16 over S columns already read
 //   dQ += dS K    M = 128 rows, N = d_k, K = 64 keys   (A from tensor memory,
 //                 K as a transposed operand from the tile S read K-major)
 // Keys: the window's last w tokens, or the compressed blocks complete at t.
 // dq rows are disjoint between CTAs; the result is added into dq (fp32).
-// Warps 0-3 softmax and epilogue, warp 4 TMA, warp 5 MMA and TMEM owner.
+// Warps 0-7 softmax and epilogue (two per TMEM lane quadrant, each half of a
+// key tile), warp 8 TMA, warp 9 MMA and TMEM owner.
 #pragma once
 #include "nsa_dev.cuh"
 #include "k_attn_packed.cuh"
@@ -30,19 +31,20 @@ struct BqCfg {
     static constexpr int kVT = 64 * DV * 2;
     static constexpr int kOffQ = 0;
     static constexpr int kOffO = kOffQ + kQTile;
-    static constexpr int kOffK = kOffO + kOTile;     // 2 slots
-    static constexpr int kOffV = kOffK + 2 * kKT;    // 2 slots
-    static constexpr int kOffBar = kOffV + 2 * kVT;
+    static constexpr int NSLOT = 3;                  // key tiles in flight
+    static constexpr int kOffK = kOffO + kOTile;
+    static constexpr int kOffV = kOffK + NSLOT * kKT;
+    static constexpr int kOffBar = kOffV + NSLOT * kVT;
     static constexpr int kSmem = kOffBar + 256 + 1024;
     static_assert(kSmem <= 232448, "shared memory");
-    static constexpr int kThreads = 192;
+    static constexpr int kThreads = 320;
     // TMEM: S buffers 0 / 64, dP buffers 128 / 192, dQ 256
     static constexpr uint32_t kColDP = 128, kColDQ = 256;
     static_assert(kColDQ + DK <= 512, "tensor memory");
 };
 
 template <int DK, int DV, int HG, int BR>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     bwd_q_dense(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapO,
                 const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
                 const BwdParams p) {
@@ -68,30 +70,32 @@ __global__ void __launch_bounds__(192, 1)
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
     uint64_t* qfull = bars + 0;
-    uint64_t* kvfull = bars + 1;    // [2]
-    uint64_t* kvempty = bars + 3;   // [2]
-    uint64_t* sfull = bars + 5;     // [2]  S and dP of a tile
-    uint64_t* dpfree = bars + 7;    // [2]
-    uint64_t* pfull = bars + 9;     // [2]  dS written
-    uint64_t* dqdone = bars + 11;   // [2]  dQ product of a tile complete (S buffer free)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 14);
+    uint64_t* kvfull = bars + 1;    // [NSLOT] key tile slots
+    uint64_t* kvempty = bars + 4;   // [NSLOT]
+    uint64_t* sfull = bars + 7;     // [2]  S and dP of a tile (TMEM buffer j & 1)
+    uint64_t* dpfree = bars + 9;    // [2]
+    uint64_t* pfull = bars + 11;    // [2]  dS written
+    uint64_t* dqdone = bars + 13;   // [2]  dQ product of a tile complete (S buffer free)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 16);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     if (threadIdx.x == 0) {
         mbar_init(qfull, 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < Cfg::NSLOT; ++s) {
             mbar_init(&kvfull[s], 1);
             mbar_init(&kvempty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
             mbar_init(&sfull[s], 1);
-            mbar_init(&dpfree[s], 4);
-            mbar_init(&pfull[s], 4);
+            mbar_init(&dpfree[s], 8);
+            mbar_init(&pfull[s], 8);
             mbar_init(&dqdone[s], 1);
         }
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == 9) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
@@ -100,7 +104,7 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ------------------------------------------------------------ TMA
         auto lane0_wait = [&](uint64_t* bar, uint32_t parity, unsigned site) -> bool {
             bool ok = true;
@@ -115,8 +119,8 @@ __global__ void __launch_bounds__(192, 1)
             tma_load_4d(smem + Cfg::kOffO + (lane - Cfg::NQB) * 16384, &mapO, qfull, (lane - Cfg::NQB) * 64,
                         g * HG, t0, b);
         for (int j = 0; j < ntiles; ++j) {
-            const int sl = j & 1;
-            if (j >= 2 && !lane0_wait(&kvempty[sl], ((j - 2) >> 1) & 1, 0x501)) break;
+            const int sl = j % Cfg::NSLOT;
+            if (j >= Cfg::NSLOT && !lane0_wait(&kvempty[sl], ((j / Cfg::NSLOT) - 1) & 1, 0x501)) break;
             const int kb = k_lo + j * 64;
             if (lane == 0) mbar_expect_tx(&kvfull[sl], Cfg::kKT + Cfg::kVT);
             __syncwarp();
@@ -126,51 +130,81 @@ __global__ void __launch_bounds__(192, 1)
                 tma_load_4d(smem + Cfg::kOffV + sl * Cfg::kVT + (lane - Cfg::NQB) * 8192, &mapV, &kvfull[sl],
                             (lane - Cfg::NQB) * 64, g, kb, b);
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ------------------------------------------------------------ MMA
         if (lane == 0) {
             constexpr uint32_t idS = idesc_bf16(128, 64);
             constexpr uint32_t idQ = idesc_bf16_bmn(128, DK);
             const uint32_t sQ = smem_u32(smem + Cfg::kOffQ), sO = smem_u32(smem + Cfg::kOffO);
             bool ok = wait_or_abort(qfull, 0, 0x502, abort_flag);
-            auto dq_of = [&](int i) -> bool {          // dQ += dS(i) K(i)
-                const int sl = i & 1;
-                if (!wait_or_abort(&pfull[sl], (i >> 1) & 1, 0x503, abort_flag)) return false;
-                tc_fence_after();
-                const uint32_t sK = smem_u32(smem + Cfg::kOffK + sl * Cfg::kKT);
+            // Two streams: S/dP of tile js (its keys staged, its TMEM buffers free) and the
+            // dQ product of tile jq (its dS written), each issued as soon as it is ready.
+            int js = 0, jq = 0;
+            unsigned long long t_idle = 0;
+            uint32_t spins = 0;
+            while (ok && jq < ntiles) {
+                bool progressed = false;
+                if (js < ntiles) {
+                    const int sl = js % Cfg::NSLOT, bf = js & 1;
+                    // S(js) overwrites the buffer whose dS fed dQ(js-2); dP(js) the one softmax(js-2) read
+                    const bool ready = mbar_test_wait(&kvfull[sl], (js / Cfg::NSLOT) & 1) &&
+                                       (js < 2 || (mbar_test_wait(&dqdone[bf], ((js - 2) >> 1) & 1) &&
+                                                   mbar_test_wait(&dpfree[bf], ((js - 2) >> 1) & 1)));
+                    if (ready) {
+                        tc_fence_after();
+                        const uint32_t sK = smem_u32(smem + Cfg::kOffK + sl * Cfg::kKT);
+                        const uint32_t sV = smem_u32(smem + Cfg::kOffV + sl * Cfg::kVT);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_bf16_ts(tmem + Cfg::kColDQ, tmem + sl * 64 + kk * 8,
-                                 sdesc_sw128_mn(sK + kk * 2048, 8192, 1024), idQ, (i > 0 || kk > 0) ? 1u : 0u);
-                umma_commit(&dqdone[sl]);
-                umma_commit(&kvempty[sl]);
-                return true;
-            };
-            for (int j = 0; j < ntiles && ok; ++j) {
-                const int sl = j & 1;
-                if (!(ok = wait_or_abort(&kvfull[sl], (j >> 1) & 1, 0x504, abort_flag))) break;
-                // S(j) overwrites the buffer whose dS fed dQ(j-2); dP(j) the one softmax(j-2) read
-                if (j >= 2 && !(ok = wait_or_abort(&dqdone[sl], ((j - 2) >> 1) & 1, 0x505, abort_flag))) break;
-                if (j >= 2 && !(ok = wait_or_abort(&dpfree[sl], ((j - 2) >> 1) & 1, 0x506, abort_flag))) break;
-                tc_fence_after();
-                const uint32_t sK = smem_u32(smem + Cfg::kOffK + sl * Cfg::kKT);
-                const uint32_t sV = smem_u32(smem + Cfg::kOffV + sl * Cfg::kVT);
+                        for (int kk = 0; kk < DK / 16; ++kk)
+                            umma_bf16_ss(tmem + bf * 64, sdesc_sw128(sQ + (kk / 4) * 16384 + (kk % 4) * 32),
+                                         sdesc_sw128(sK + (kk / 4) * 8192 + (kk % 4) * 32), idS, kk > 0 ? 1u : 0u);
 #pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk)
-                    umma_bf16_ss(tmem + sl * 64, sdesc_sw128(sQ + (kk / 4) * 16384 + (kk % 4) * 32),
-                                 sdesc_sw128(sK + (kk / 4) * 8192 + (kk % 4) * 32), idS, kk > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < DV / 16; ++kk)
+                            umma_bf16_ss(tmem + Cfg::kColDP + bf * 64, sdesc_sw128(sO + (kk / 4) * 16384 + (kk % 4) * 32),
+                                         sdesc_sw128(sV + (kk / 4) * 8192 + (kk % 4) * 32), idS, kk > 0 ? 1u : 0u);
+                        umma_commit(&sfull[bf]);
+                        ++js;
+                        progressed = true;
+                    }
+                }
+                if (jq < js && mbar_test_wait(&pfull[jq & 1], (jq >> 1) & 1)) {   // dQ += dS(jq) K(jq)
+                    const int sl = jq % Cfg::NSLOT, bf = jq & 1;
+                    tc_fence_after();
+                    const uint32_t sK = smem_u32(smem + Cfg::kOffK + sl * Cfg::kKT);
 #pragma unroll
-                for (int kk = 0; kk < DV / 16; ++kk)
-                    umma_bf16_ss(tmem + Cfg::kColDP + sl * 64, sdesc_sw128(sO + (kk / 4) * 16384 + (kk % 4) * 32),
-                                 sdesc_sw128(sV + (kk / 4) * 8192 + (kk % 4) * 32), idS, kk > 0 ? 1u : 0u);
-                umma_commit(&sfull[sl]);
-                if (j >= 1) ok = dq_of(j - 1);
+                    for (int kk = 0; kk < 4; ++kk)  // keys 16kk.. : packed by warp kk / 2 in its own columns
+                        umma_bf16_ts(tmem + Cfg::kColDQ, tmem + bf * 64 + (kk >> 1) * 32 + (kk & 1) * 8,
+                                     sdesc_sw128_mn(sK + kk * 2048, 8192, 1024), idQ, (jq > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&dqdone[bf]);
+                    umma_commit(&kvempty[sl]);
+                    ++jq;
+                    progressed = true;
+                }
+                // bounded: no progress for the wait limit ends the CTA with an error
+                if (progressed) {
+                    spins = 0;
+                    t_idle = 0;
+                } else if ((++spins & 63u) == 0u) {
+                    if (*abort_flag) {
+                        ok = false;
+                    } else {
+                        const unsigned long long now = globaltimer_ns();
+                        if (t_idle == 0) t_idle = now;
+                        else if (now - t_idle > kWaitLimitNs) {
+                            record_timeout(0x503);
+                            *abort_flag = 1;
+                            ok = false;
+                        }
+                    }
+                }
             }
-            if (ok) ok = dq_of(ntiles - 1);
         }
-    } else if (warp < 4) {
+    } else if (warp < 8) {
         // ------------------------------------------------- softmax, epilogue
-        const int r = warp * 32 + lane;                  // row = TMEM lane
+        // warp w: rows 32 (w % 4) .. +31 (its TMEM lane quadrant), keys 32 (w / 4)
+        // .. +31 of each key tile
+        const int quad = warp & 3, hc = warp >> 2;
+        const int r = quad * 32 + lane;                  // row = TMEM lane
         const int t = t0 + r / HG, h = g * HG + r % HG;
         const bool row_ok = t < p.T;
         const size_t row = ((size_t)b * p.T + (row_ok ? t : 0)) * p.H + h;
@@ -186,7 +220,7 @@ __global__ void __launch_bounds__(192, 1)
             vis_hi = (t + 1 >= p.l) ? (t + 1 - p.l) / p.d + 1 : 0;
         }
         if (!row_ok || L == -INFINITY) vis_lo = vis_hi = 0;
-        const uint32_t lanebase = tmem + ((uint32_t)(warp * 32) << 16);
+        const uint32_t lanebase = tmem + ((uint32_t)(quad * 32) << 16);
         const float c = p.scale_log2;
         bool ok = true;
         for (int j = 0; j < ntiles; ++j) {
@@ -195,52 +229,53 @@ __global__ void __launch_bounds__(192, 1)
             if (lane == 0) w_ok = wait_or_abort(&sfull[sl], (j >> 1) & 1, 0x507, abort_flag);
             if (!(ok = __shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0) != 0)) break;
             tc_fence_after();
-            const int kb = k_lo + j * 64;
-            uint32_t ds[32];
+            const int kb = k_lo + j * 64 + hc * 32;
+            uint32_t sr[32], dr[32];
+            tmem_ld32(lanebase + sl * 64 + hc * 32, sr);
+            tmem_ld32(lanebase + Cfg::kColDP + sl * 64 + hc * 32, dr);
+            tmem_wait_ld32(sr);
+            tmem_wait_ld32(dr);
+            uint32_t ds[16];
+            // the whole key range of the tile inside the row's: no masks
+            const bool inner = kb >= vis_lo && kb + 32 <= vis_hi;
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                uint32_t sr[32], dr[32];
-                tmem_ld32(lanebase + sl * 64 + hf * 32, sr);
-                tmem_ld32(lanebase + Cfg::kColDP + sl * 64 + hf * 32, dr);
-                tmem_wait_ld32(sr);
-                tmem_wait_ld32(dr);
+            for (int cp = 0; cp < 16; ++cp) {
+                float v2[2];
 #pragma unroll
-                for (int cp = 0; cp < 16; ++cp) {
-                    float v2[2];
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int key = kb + hf * 32 + 2 * cp + e;
-                        const bool vis = key >= vis_lo && key < vis_hi;
-                        const float pr = vis ? ex2a(fmaf(__uint_as_float(sr[2 * cp + e]), c, -L)) : 0.f;
-                        v2[e] = pr * fmaf(gr, __uint_as_float(dr[2 * cp + e]), -Dr);
-                    }
-                    ds[hf * 16 + cp] = pack_bf16x2(v2[0], v2[1]);
+                for (int e = 0; e < 2; ++e) {
+                    const int key = kb + 2 * cp + e;
+                    const bool vis = inner || (key >= vis_lo && key < vis_hi);
+                    const float pr = vis ? ex2a(fmaf(__uint_as_float(sr[2 * cp + e]), c, -L)) : 0.f;
+                    v2[e] = pr * fmaf(gr, __uint_as_float(dr[2 * cp + e]), -Dr);
                 }
+                ds[cp] = pack_bf16x2(v2[0], v2[1]);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&dpfree[sl]);
-            // dS (bf16 pairs) over the first 32 columns of this tile's S buffer:
-            // the A operand of dQ += dS K, read from tensor memory
-            tmem_st32(lanebase + sl * 64, ds);
+            // dS (bf16 pairs) over the first 16 of the 32 S columns this warp read (the
+            // other warp of the quadrant may still be reading its own): the A operand
+            // of dQ += dS K, read from tensor memory
+            tmem_st16(lanebase + sl * 64 + hc * 32, ds);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&pfull[sl]);
         }
-        // epilogue: scale * dQ added into dq
+        // epilogue: scale * dQ added into dq (columns split between the two warps of a quadrant)
         bool w_ok = true;
         const int last = ntiles - 1;
         if (lane == 0) w_ok = ok && wait_or_abort(&dqdone[last & 1], (last >> 1) & 1, 0x508, abort_flag);
         if (__shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0) != 0) {
             tc_fence_after();
             float* dst = p.dq + row * DK;
+            constexpr int HALF = DK / 2;
 #pragma unroll 1
-            for (int c0 = 0; c0 < DK; c0 += 32) {
+            for (int c0 = hc * HALF; c0 < (hc + 1) * HALF; c0 += 32) {
                 uint32_t rq[32];
                 tmem_ld32(lanebase + Cfg::kColDQ + c0, rq);
                 tmem_wait_ld32(rq);
-                if (row_ok && h < p.H) {
+                if (row_ok) {
 #pragma unroll
                     for (int e = 0; e < 32; e += 4)
                         red_add_v4(dst + c0 + e, p.scale * __uint_as_float(rq[e]), p.scale * __uint_as_float(rq[e + 1]),
@@ -251,7 +286,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }

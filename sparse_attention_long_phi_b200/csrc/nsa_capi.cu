@@ -22,6 +22,7 @@
 #include "k_backward.cuh"
 #include "k_bwd_kv.cuh"
 #include "k_bwd_q.cuh"
+#include "k_bwd_qsel.cuh"
 #include "k_phi.cuh"
 #include "k_topn.cuh"
 #include "k_append.cuh"
@@ -667,14 +668,34 @@ nsa_status_t backward_impl(const Shape& s, const void* q, const void* k, const v
                 obuf, reinterpret_cast<const __nv_bfloat16*>(dout), gates, lsen, br, rows, DV, dgates, p.dlt, p.lse2));
             NSA_TRY(last_launch());
         }
-        p.have_stats = 1;
     }
-    // dq of the selected branch (warp-level tensor cores, 16 heads = M); it writes dq
+    // dq of the selected branch (tcgen05, per token and group, transposed products), added
+    if (cudaMemsetAsync(dq, 0, (size_t)s.B * s.T * s.H * DK * 4, st) != cudaSuccess) return NSA_ERR_CUDA;
     {
-        p.q_branches = 1 << kBrSlc;
-        const int smem = bwd_query_mma_smem<DK, DV>();
-        NSA_TRY(set_smem(bwd_query_mma<DK, DV>, smem));
-        NSA_LAUNCH("bwd_query_mma", st, bwd_query_mma<DK, DV><<<dim3((unsigned)s.T, (unsigned)s.G, (unsigned)s.B), 128, smem, st>>>(p));
+        constexpr int HG = DK == 192 ? 16 : 4;
+        using Cfg = BqsCfg<DK, DV>;
+        CUtensorMap mQs, mOs, mK, mV;
+        const uint32_t bH[4] = {64, 16, 1, 1};
+        const uint32_t bKV[4] = {64, 1, 64, 1};
+        const uint64_t dQ[4] = {(uint64_t)DK, (uint64_t)s.H, (uint64_t)s.T, (uint64_t)s.B};
+        const uint64_t sQ[3] = {(uint64_t)DK * 2, (uint64_t)s.H * DK * 2, (uint64_t)s.T * s.H * DK * 2};
+        const uint64_t dO[4] = {(uint64_t)DV, (uint64_t)s.H, (uint64_t)s.T, (uint64_t)s.B};
+        const uint64_t sO[3] = {(uint64_t)DV * 2, (uint64_t)s.H * DV * 2, (uint64_t)s.T * s.H * DV * 2};
+        const uint64_t dK[4] = {(uint64_t)DK, (uint64_t)s.G, (uint64_t)s.T, (uint64_t)s.B};
+        const uint64_t sK[3] = {(uint64_t)DK * 2, (uint64_t)s.G * DK * 2, (uint64_t)s.T * s.G * DK * 2};
+        const uint64_t dV[4] = {(uint64_t)DV, (uint64_t)s.G, (uint64_t)s.T, (uint64_t)s.B};
+        const uint64_t sV[3] = {(uint64_t)DV * 2, (uint64_t)s.G * DV * 2, (uint64_t)s.T * s.G * DV * 2};
+        if (!make_map(&mQs, q, 4, dQ, sQ, bH) || !make_map(&mOs, dout, 4, dO, sO, bH) ||
+            !make_map(&mK, k, 4, dK, sK, bKV) || !make_map(&mV, v, 4, dV, sV, bKV))
+            return NSA_ERR_CUDA;
+        BqsParams qp{};
+        qp.bp = p;
+        const int64_t tpc = (s.B * s.T * s.G) / (148 * 8);
+        qp.tpc = (int)std::min<int64_t>(64, std::max<int64_t>(4, tpc));
+        qp.nchunks = (int)ceil_div(s.T, qp.tpc);
+        NSA_TRY(set_smem(bwd_q_sel<DK, DV, HG>, Cfg::kSmem));
+        const dim3 grid((unsigned)(qp.nchunks * s.G), 1, (unsigned)s.B);
+        NSA_LAUNCH("bwd_q_sel", st, bwd_q_sel<DK, DV, HG><<<grid, Cfg::kThreads, Cfg::kSmem, st>>>(mQs, mOs, mK, mV, qp));
         NSA_TRY(last_launch());
     }
     // dq of the window and compressed branches (tcgen05, packed query tiles), added

@@ -76,21 +76,26 @@ def forward_flops(c):
     return f, total_attn
 
 
-def csrc_sha():
+# the source files that define each kernel whose traffic is recorded (its own file and
+# the device primitives it includes)
+KERNEL_SOURCES = {"attn_sel_kernel": ("k_attn_sel.cuh", "k_attn_packed.cuh", "nsa_dev.cuh")}
+
+
+def csrc_sha(files=None):
     h = hashlib.sha256()
     d = os.path.join(ROOT, "sparse_attention_long_phi_b200", "csrc")
-    for n in sorted(os.listdir(d)):
+    for n in sorted(files if files else os.listdir(d)):
         h.update(open(os.path.join(d, n), "rb").read())
     return h.hexdigest()[:16]
 
 
 def ncu_traffic(kernel):
     """DRAM bytes per launch of `kernel` from the committed ncu summary, if the
-    kernel sources have not changed since it was captured (else None)."""
+    kernel's sources have not changed since it was captured (else None)."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.md")
     if not os.path.exists(p):
         return None
-    sha = csrc_sha()
+    sha = csrc_sha(KERNEL_SOURCES.get(kernel))
     for line in open(p):
         parts = line.strip().split()
         if len(parts) == 4 and parts[0] == "traffic:" and parts[1] == kernel and parts[3] == sha:

@@ -583,41 +583,65 @@ def bench_append(c, x, kv_off, cmp_off, dev, nsa, stream, reps=50):
 
 
 def bench_backward(dev, nsa, peaks, steps=2, warmup=1, seq_len=0):
-    """Forward + backward of the training workload (B=2, T=16384; T overridable for profiling)."""
+    """Forward + backward of the training workload (B=2, T=16384; T overridable for profiling):
+    the training forward (which keeps each branch's output and LSE) and the backward from
+    those saved statistics, with the phi parameter gradients.  The backward that recomputes
+    the statistics itself (nsa_backward) is timed beside it."""
     c = dict(I.WORKLOADS["train_fwd_bwd_B2_T16384"])
     if seq_len:
         c["T"] = seq_len
     x = I.make_forward_inputs(c, dev, with_dout=True)
     phi = {k: x[k] for k in ("wk", "ek", "wv", "ev")}
     stream = torch.cuda.current_stream(dev)
-    fb = nsa.forward_buffers(c, dev, want_lse=False)
-    nsa.forward_into(c, x["q"], x["k"], x["v"], x["gates"], phi, fb, stream)
+    ws_f = nsa.alloc_workspace(c, nsa.NSA_MODE_FORWARD, dev)
+    ws_b = nsa.alloc_workspace(c, nsa.NSA_MODE_BACKWARD, dev)
+
+    def fwd():
+        return nsa.forward_train(c, x["q"], x["k"], x["v"], x["gates"], phi, stream, ws=ws_f)
+
+    def bwd(f):
+        return nsa.backward_saved(c, x["q"], x["k"], x["v"], x["gates"], x["dout"], f["idx"], f["lse"],
+                                  f["o_branch"], phi, stream, ws=ws_b, want_phi_grads=True)
+
+    def bwd_recompute(f):
+        return nsa.backward(c, x["q"], x["k"], x["v"], x["gates"], x["dout"], f["idx"], phi, stream,
+                            want_phi_grads=True, ws=ws_b)
+
     for _ in range(warmup):
-        nsa.backward(c, x["q"], x["k"], x["v"], x["gates"], x["dout"], fb.idx, phi, want_phi_grads=True)
+        f = fwd()
+        bwd(f)
+        bwd_recompute(f)
     torch.cuda.synchronize(dev)
     nsa.sync_status()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    ev[0].record(stream)
     for _ in range(steps):
-        nsa.forward_into(c, x["q"], x["k"], x["v"], x["gates"], phi, fb, stream)
-    e1.record(stream)
+        f = fwd()
+    ev[1].record(stream)
     nsa.profile_read()
     nsa.profile_enable(True)
     for _ in range(steps):   # the full training backward: q, k, v, gates and the phi parameters
-        nsa.backward(c, x["q"], x["k"], x["v"], x["gates"], x["dout"], fb.idx, phi, want_phi_grads=True)
-    e2.record(stream)
+        bwd(f)
+    ev[2].record(stream)
     torch.cuda.synchronize(dev)
     nsa.profile_enable(False)
     prof = nsa.profile_read()
-    f_ms, b_ms = e0.elapsed_time(e1) / steps, e1.elapsed_time(e2) / steps
-    _, fwd = forward_flops(c)
-    bwd = 2 * fwd                               # dP, dV, dQ, dK
+    for _ in range(steps):
+        bwd_recompute(f)
+    ev[3].record(stream)
+    torch.cuda.synchronize(dev)
+    nsa.sync_status()
+    f_ms, b_ms = ev[0].elapsed_time(ev[1]) / steps, ev[1].elapsed_time(ev[2]) / steps
+    r_ms = ev[2].elapsed_time(ev[3]) / steps
+    _, fwd_flop = forward_flops(c)
+    bwd_flop = 2 * fwd_flop                     # dP, dV, dQ, dK
     return {"workload": "train_fwd_bwd_B2_T16384" if not seq_len else f"train_fwd_bwd_B2_T{seq_len}",
             "fwd_ms": round(f_ms, 3), "bwd_ms": round(b_ms, 3),
+            "path": "nsa_forward_train + nsa_backward_saved (+ nsa_backward_phi_params)",
+            "bwd_recompute_ms": round(r_ms, 3),
             "tokens_per_s": round(c["B"] * c["T"] / ((f_ms + b_ms) / 1e3), 1),
-            "bwd_tflops_algorithmic": round(bwd / (b_ms / 1e3) / 1e12, 2),
-            "bwd_frac_of_peak": round(bwd / (b_ms / 1e3) / 1e12 / peaks.get("bf16_tflops", 1590.0), 4),
+            "bwd_tflops_algorithmic": round(bwd_flop / (b_ms / 1e3) / 1e12, 2),
+            "bwd_frac_of_peak": round(bwd_flop / (b_ms / 1e3) / 1e12 / peaks.get("bf16_tflops", 1590.0), 4),
             "kernels": {k: {"launches": n, "ms_per_step": round(t / steps, 3)} for k, (n, t) in prof.items()}}
 
 

@@ -215,6 +215,35 @@ nsa_status_t nsa_backward(const nsa_config_t* cfg, const void* q, const void* k,
                           const int32_t* sel_idx, float* dq, float* dk, float* dv, float* dgates,
                           void* workspace, size_t workspace_bytes, void* stream);
 
+/* Training forward (pages: natively trainable design; 最终输出计算 for the
+ * gated sum): exactly nsa_forward (same kernels, same out, sel_idx and lse,
+ * bit for bit), and in addition each branch's own output before its gate,
+ * which is what the backward's per-branch statistics are made of.
+ * Out: out, sel_idx as nsa_forward; lse [B,T,H,3] fp32 (required);
+ *      o_branch [3,B,T,H,d_v] fp32 (required, 16-byte aligned): o_cmp, o_slc,
+ *      o_win in that order, each normalised by its own softmax, so that
+ *      out = sum_c gates[..., c] * o_branch[c] up to rounding.
+ * Same FORWARD workspace as nsa_forward; the compressed keys are not
+ * returned (the backward recomputes them). */
+nsa_status_t nsa_forward_train(const nsa_config_t* cfg, const void* q, const void* k, const void* v,
+                               const float* gates, const nsa_phi_params_t* phi, float* out, int32_t* sel_idx,
+                               float* lse, float* o_branch, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/* Backward from the training forward's saved statistics: as nsa_backward, but
+ * the per-branch outputs and LSEs are read from `o_branch` and `lse` as
+ * nsa_forward_train wrote them for the same q, k, v, phi and sel_idx,
+ * instead of being recomputed by three more forward passes (the usual
+ * attention-training split: the forward keeps what the softmax backward
+ * needs).  Results equal nsa_backward's up to the order of floating-point
+ * additions.  Passing statistics that belong to other inputs gives wrong
+ * gradients; nothing checks them.  BACKWARD workspace, as nsa_backward. */
+nsa_status_t nsa_backward_saved(const nsa_config_t* cfg, const void* q, const void* k, const void* v,
+                                const float* gates, const nsa_phi_params_t* phi, const void* dout,
+                                const int32_t* sel_idx, const float* lse, const float* o_branch, float* dq,
+                                float* dk, float* dv, float* dgates, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
 /* Batched decode step over caches with spare capacity per sequence: as
  * nsa_decode, but sequence s holds kv_len[s] tokens in rows [kv_start[s],
  * kv_start[s] + kv_len[s]) of k_cache/v_cache and nsa_num_cmp_blocks(cfg,

@@ -43,6 +43,7 @@ struct PackedParams {
     float scale_log2;          // softmax scale * log2(e)
     const float* gates;        // [B,T,H,3]
     float* out;                // [B,T,H,DV]
+    float* obranch;            // [B,T,H,DV] this branch's own output o_c (before the gate), or null
     float* lse_user;           // [B,T,H,3] or null
     float* lse_cmp;            // [B,T,H] natural log (pass 1 writes, pass 2 reads)
     float* pscore;             // [B,T,G,NSp]
@@ -548,6 +549,13 @@ __global__ void __launch_bounds__(320, 1)
                 } else {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) o[e] = 0u;
+                }
+                if (row_ok && ok && p.obranch) {
+                    float4* dsto = reinterpret_cast<float4*>(p.obranch + rowid * DV + c0);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        dsto[e] = make_float4(__uint_as_float(o[4 * e + 0]) * inv, __uint_as_float(o[4 * e + 1]) * inv,
+                                              __uint_as_float(o[4 * e + 2]) * inv, __uint_as_float(o[4 * e + 3]) * inv);
                 }
                 if (row_ok && ok) {
                     float4* dst = reinterpret_cast<float4*>(p.out + rowid * DV + c0);

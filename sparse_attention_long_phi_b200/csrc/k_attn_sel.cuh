@@ -31,6 +31,7 @@ struct SelParams {
     const int32_t* idx;         // [B,T,G,n]
     const float* gates;         // [B,T,H,3]
     float* out;                 // [B,T,H,DV] accumulated
+    float* obranch;             // [B,T,H,DV] the branch's own output o_slc (before the gate), or null
     float* lse_user;            // [B,T,H,3] or null
     int tpc;                    // tokens per CTA
     int nchunks;                // token chunks per group: grid.x = G * nchunks, group-major
@@ -50,7 +51,7 @@ struct SelCfg {
     static constexpr int kOffP = kOffKV + NSLOT * kSlot;
     static constexpr int kPBytes = 16 * 2048;             // 16 heads x 1024 keys
     static constexpr int kOffRed = kOffP + 2 * kPBytes;   // one P^T tile per warpgroup
-    static constexpr int kRedBytes = 2 * (2 * 4 * 16 * 4 + 16 * 4);
+    static constexpr int kRedBytes = 2 * (2 * 4 * 16 * 4 + 2 * 16 * 4);
     static constexpr int kOffBar = kOffRed + kRedBytes;
     static constexpr int kSmem = kOffBar + 256 + 1024;
     static constexpr int kThreads = 320;
@@ -307,20 +308,20 @@ __global__ void __launch_bounds__(320, 1)
         float* redm = reinterpret_cast<float*>(smem + Cfg::kOffRed + wg * (Cfg::kRedBytes / 2));
         float* redl = redm + 64;
         int* su = reinterpret_cast<int*>(redl + 64);          // [16] block ids of the token
+        float* sg = redl + 80;                                 // [16] the token's selected-branch gates
         const uint32_t bar_id = 1 + wg;
         bool ok = true;
         int it = 0;
         // the token's selection entry (threads kl < 16) and gates, prefetched
         // one token ahead so their latency overlaps the previous token
         int idx_nx = -1;
-        float gate_nx[HG];
+        float gate_nx = 0.f;
         auto prefetch = [&](int i) {
             if (i >= N) return;
             const int32_t* row = idx_base + (size_t)(tb + i) * p.G * p.n;
             if (kl < 16) idx_nx = kl < p.n ? __ldg(row + kl) : -1;
             const size_t rb2 = ((size_t)b * p.T + tb + i) * p.H + (size_t)g * HG;
-#pragma unroll
-            for (int h = 0; h < HG; ++h) gate_nx[h] = __ldg(p.gates + (rb2 + h) * 3 + 1);
+            if (kl < HG) gate_nx = __ldg(p.gates + (rb2 + kl) * 3 + 1);
             // the token's out rows (HG x DV fp32, contiguous), read-modify-written
             // by the epilogue: brought into L2 now, two tokens ahead
             if (kl * 32 < HG * DV)
@@ -329,10 +330,10 @@ __global__ void __launch_bounds__(320, 1)
         prefetch(wg);
         for (int i = wg; i < N; i += 2, ++it) {
             const int t = tb + i;
-            if (kl < 16) su[kl] = idx_nx;
-            float gate[HG];
-#pragma unroll
-            for (int h = 0; h < HG; ++h) gate[h] = gate_nx[h];
+            if (kl < 16) {
+                su[kl] = idx_nx;
+                sg[kl] = gate_nx;
+            }
             const size_t rowbase = ((size_t)b * p.T + t) * p.H + (size_t)g * HG;
             named_bar_sync(bar_id, 128);
             prefetch(i + 2);
@@ -420,7 +421,8 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
                 for (int h = 0; h < HG; ++h) {
                     const float o = ls[h] > 0.f ? __uint_as_float(r[h]) / ls[h] : 0.f;
-                    p.out[(rowbase + h) * DV + kl] = prev[h] + gate[h] * o;
+                    p.out[(rowbase + h) * DV + kl] = prev[h] + sg[h] * o;
+                    if (p.obranch) p.obranch[(rowbase + h) * DV + kl] = o;
                 }
             }
             if (ok && p.lse_user && kl < HG) {

@@ -15,7 +15,11 @@
 //                           K tile read as a transposed operand), N = 16, K = 128
 // A CTA walks a range of tokens of one group; two softmax warpgroups take
 // alternate tokens with their own TMEM buffers, so one token's softmax
-// overlaps the other's products.  Warp 8: TMA producer, warp 9: MMA issuer.
+// overlaps the other's products.  K and V of a pair sit in separate rings:
+// V is needed only by dP^T and is released as soon as that product is done,
+// while K stays for the dQ^T products, so the K ring is the deeper one.
+// Warp 8 stages Q_t/dO_t and the K pairs, warp 10 the V pairs (each waits
+// only on its own ring), warp 9 issues the MMAs.
 #pragma once
 #include "nsa_dev.cuh"
 #include "k_attn_packed.cuh"
@@ -35,17 +39,20 @@ struct BqsCfg {
     static constexpr int kO = NVB * 2048;             // dO_t
     static constexpr int kKPair = NQB * 16384;        // per box: [128 keys][64]
     static constexpr int kVPair = NVB * 16384;
-    static constexpr int kSlot = kKPair + kVPair;
-    static constexpr int NSLOT = 2;
+    static constexpr int NK = 3;                      // K pair slots
     static constexpr int kDS = 16 * 256;              // dS^T [16 heads][128 keys], two 64-key atoms
     static constexpr int kOffQ = 0;                   // 2 token slots of Q_t then dO_t
     static constexpr int kOffO = kOffQ + 2 * kQ;
-    static constexpr int kOffKV = ((kOffO + 2 * kO + 1023) / 1024) * 1024;
-    static constexpr int kOffDS = kOffKV + NSLOT * kSlot;   // [2 warpgroups][2 buffers]
+    static constexpr int kOffK = ((kOffO + 2 * kO + 1023) / 1024) * 1024;
+    static constexpr int kOffDS = kOffK + NK * kKPair;      // [2 warpgroups][2 buffers]
     static constexpr int kOffBar = kOffDS + 4 * kDS;
-    static constexpr int kSmem = kOffBar + 512 + 1024;
-    static_assert(kSmem <= 232448, "shared memory");
-    static constexpr int kThreads = 320;
+    static constexpr int kOffV = kOffBar + 1024;            // V pair slots: what is left, 1..4
+    static constexpr int kSmemMax = 232448;
+    static constexpr int NVfit = (kSmemMax - 1024 - kOffV) / kVPair;
+    static constexpr int NV = NVfit > 4 ? 4 : NVfit;
+    static constexpr int kSmem = kOffV + NV * kVPair + 1024;
+    static_assert(NV >= 1 && kSmem <= kSmemMax, "shared memory");
+    static constexpr int kThreads = 352;
     // TMEM per warpgroup (128 columns apart): S^T buffers 0 / 16, dP^T 32 / 48, dQ^T 64 (+16)
     static constexpr uint32_t kColDP = 32, kColDQ = 64;
 };
@@ -57,7 +64,7 @@ struct BqsParams {
 };
 
 template <int DK, int DV, int HG>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     bwd_q_sel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapO,
               const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
               const BqsParams P) {
@@ -70,17 +77,19 @@ __global__ void __launch_bounds__(320, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
     uint64_t* qfull = bars + 0;     // [2] token slots
     uint64_t* qempty = bars + 2;    // [2]
-    uint64_t* full = bars + 4;      // [NSLOT] K/V pair slots
-    uint64_t* empty = bars + 6;     // [NSLOT]
-    uint64_t* sdfull = bars + 8;    // [2 wg][2 buf]  S^T and dP^T of a pair
-    uint64_t* sdfree = bars + 12;   // [2][2]
-    uint64_t* dsfull = bars + 16;   // [2][2]         dS^T tile written
-    uint64_t* dsfree = bars + 20;   // [2][2]         dS^T tile read by the dQ^T products
-    uint64_t* dqfull = bars + 24;   // [2]
-    uint64_t* dqfree = bars + 26;   // [2]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 28);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 29);
-    int* npairs_ring = reinterpret_cast<int*>(bars + 30);     // [4] producer -> MMA
+    uint64_t* kfull = bars + 4;     // [NK] K pair slots
+    uint64_t* kempty = bars + 8;    // [NK]
+    uint64_t* vfull = bars + 12;    // [NV] V pair slots
+    uint64_t* vempty = bars + 16;   // [NV]
+    uint64_t* sdfull = bars + 20;   // [2 wg][2 buf]  S^T and dP^T of a pair
+    uint64_t* sdfree = bars + 24;   // [2][2]
+    uint64_t* dsfull = bars + 28;   // [2][2]         dS^T tile written
+    uint64_t* dsfree = bars + 32;   // [2][2]         dS^T tile read by the dQ^T products
+    uint64_t* dqfull = bars + 36;   // [2]
+    uint64_t* dqfree = bars + 38;   // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 40);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 41);
+    int* npairs_ring = reinterpret_cast<int*>(bars + 42);     // [8] producer -> MMA
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int g = blockIdx.x / P.nchunks, b = blockIdx.z;
@@ -96,9 +105,13 @@ __global__ void __launch_bounds__(320, 1)
             mbar_init(&dqfull[s], 1);
             mbar_init(&dqfree[s], 4);
         }
-        for (int s = 0; s < Cfg::NSLOT; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+        for (int s = 0; s < Cfg::NK; ++s) {
+            mbar_init(&kfull[s], 1);
+            mbar_init(&kempty[s], 1);
+        }
+        for (int s = 0; s < Cfg::NV; ++s) {
+            mbar_init(&vfull[s], 1);
+            mbar_init(&vempty[s], 1);
         }
         for (int s = 0; s < 4; ++s) {
             mbar_init(&sdfull[s], 1);
@@ -137,13 +150,13 @@ __global__ void __launch_bounds__(320, 1)
         return nu;
     };
 
+    auto lane0_wait = [&](uint64_t* bar, uint32_t parity, unsigned site) -> bool {
+        bool ok = true;
+        if (lane == 0) ok = wait_or_abort(bar, parity, site, abort_flag);
+        return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    };
     if (warp == 8) {
-        // ------------------------------------------------------ producer
-        auto lane0_wait = [&](uint64_t* bar, uint32_t parity, unsigned site) -> bool {
-            bool ok = true;
-            if (lane == 0) ok = wait_or_abort(bar, parity, site, abort_flag);
-            return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        };
+        // ----------------------------------------- producer: Q_t, dO_t, K pairs
         uint32_t cnt = 0;
         bool ok = true;
         for (int i = 0; i < N && ok; ++i) {
@@ -153,7 +166,7 @@ __global__ void __launch_bounds__(320, 1)
             const int nu = count_row(r);
             if (i >= 2 && !(ok = lane0_wait(&qempty[qs], ((i - 2) >> 1) & 1, 0x601))) break;
             if (lane == 0) {
-                npairs_ring[i & 3] = (nu + 1) / 2;           // read by the MMA warp after qfull
+                npairs_ring[i & 7] = (nu + 1) / 2;           // read by the MMA warp after qfull
                 mbar_expect_tx(&qfull[qs], Cfg::kQ + Cfg::kO);
             }
             __syncwarp();
@@ -165,89 +178,169 @@ __global__ void __launch_bounds__(320, 1)
                             (lane - Cfg::NQB) * 64, g * HG, tb + i, b);
             for (int pp = 0; pp < (nu + 1) / 2; ++pp) {
                 const int ja = pick(r, 2 * pp), jb = 2 * pp + 1 < nu ? pick(r, 2 * pp + 1) : ja;
-                const int sl = cnt % Cfg::NSLOT;
-                if (cnt >= Cfg::NSLOT && !(ok = lane0_wait(&empty[sl], ((cnt / Cfg::NSLOT) - 1) & 1, 0x602))) break;
-                uint8_t* base = smem + Cfg::kOffKV + sl * Cfg::kSlot;
-                if (lane == 0) mbar_expect_tx(&full[sl], Cfg::kSlot);
+                const int sl = cnt % Cfg::NK;
+                if (cnt >= Cfg::NK && !(ok = lane0_wait(&kempty[sl], ((cnt / Cfg::NK) - 1) & 1, 0x602))) break;
+                uint8_t* base = smem + Cfg::kOffK + sl * Cfg::kKPair;
+                if (lane == 0) mbar_expect_tx(&kfull[sl], Cfg::kKPair);
                 __syncwarp();
-                // lane 2 box + half: K boxes (64 channels) of block ja / jb; then V
+                // lane 2 box + half: 64 channels (box) of block ja (half 0) or jb (half 1)
                 if (lane < 2 * Cfg::NQB) {
                     const int bx = lane >> 1, half = lane & 1;
-                    tma_load_4d(base + bx * 16384 + half * 8192, &mapK, &full[sl], bx * 64, g, (half ? jb : ja) * 64, b);
-                } else if (lane < 2 * (Cfg::NQB + Cfg::NVB)) {
-                    const int l2 = lane - 2 * Cfg::NQB, bx = l2 >> 1, half = l2 & 1;
-                    tma_load_4d(base + Cfg::kKPair + bx * 16384 + half * 8192, &mapV, &full[sl], bx * 64, g,
-                                (half ? jb : ja) * 64, b);
+                    tma_load_4d(base + bx * 16384 + half * 8192, &mapK, &kfull[sl], bx * 64, g, (half ? jb : ja) * 64, b);
+                }
+                ++cnt;
+            }
+        }
+    } else if (warp == 10) {
+        // ------------------------------------------------- producer: V pairs
+        uint32_t cnt = 0;
+        bool ok = true;
+        for (int i = 0; i < N && ok; ++i) {
+            int r[16];
+            load_row(i, r);
+            const int nu = count_row(r);
+            for (int pp = 0; pp < (nu + 1) / 2; ++pp) {
+                const int ja = pick(r, 2 * pp), jb = 2 * pp + 1 < nu ? pick(r, 2 * pp + 1) : ja;
+                const int sl = cnt % Cfg::NV;
+                if (cnt >= Cfg::NV && !(ok = lane0_wait(&vempty[sl], ((cnt / Cfg::NV) - 1) & 1, 0x60B))) break;
+                uint8_t* base = smem + Cfg::kOffV + sl * Cfg::kVPair;
+                if (lane == 0) mbar_expect_tx(&vfull[sl], Cfg::kVPair);
+                __syncwarp();
+                if (lane < 2 * Cfg::NVB) {
+                    const int bx = lane >> 1, half = lane & 1;
+                    tma_load_4d(base + bx * 16384 + half * 8192, &mapV, &vfull[sl], bx * 64, g, (half ? jb : ja) * 64, b);
                 }
                 ++cnt;
             }
         }
     } else if (warp == 9) {
         // ----------------------------------------------------------- MMA
+        // Two streams issued by one thread, each as soon as it is ready:
+        //   A  dP^T then S^T of the next pair (its V / K staged, its TMEM buffer read
+        //      by the softmax), token after token;
+        //   B  dQ^T of the oldest pair whose dS^T tile is written.
+        // So a pair's dQ^T products never wait for the next pair's rows, and its K
+        // slot returns to the producer as soon as they are done.  Every wait is a
+        // test; no progress for the wait limit ends the CTA with an error.
         if (lane == 0) {
             constexpr uint32_t id16 = idesc_bf16(128, 16);
             constexpr uint32_t idT = idesc_bf16_amn(128, 16);
-            uint32_t cnt = 0;
-            // per (warpgroup, buffer) q: bit q of `par` = parity of its S/dP issues so far,
-            // bit q of `used` = at least one issue
-            uint32_t par = 0, used = 0;
+            uint32_t ck = 0, cv = 0, cb = 0;      // K, V slots used by A; K slots released by B
+            // per (warpgroup, buffer) q: bit q = parity of A's S/dP issues, any issue; of B's dQ^T issues
+            uint32_t parA = 0, usedA = 0, parB = 0;
+            int ia = 0, pa = 0, npa = -1;         // A: token, pair, its pairs (-1: not started)
+            int ib = 0, pb = 0, npb = -1;         // B
+            bool dp_done = false, dqfree_ok = false;
             bool ok = true;
-            for (int i = 0; i < N && ok; ++i) {
-                const int qs = i & 1, wg = i & 1;
-                const uint32_t tw = tmem + wg * 128;
-                if (!(ok = wait_or_abort(&qfull[qs], (i >> 1) & 1, 0x603, abort_flag))) break;
-                const int np = npairs_ring[i & 3];
-                // this warpgroup's previous token has read its dQ^T
-                if (i >= 2 && !(ok = wait_or_abort(&dqfree[wg], ((i - 2) >> 1) & 1, 0x604, abort_flag))) break;
-                tc_fence_after();
-                const uint32_t sQ = smem_u32(smem + Cfg::kOffQ + qs * Cfg::kQ);
-                const uint32_t sO = smem_u32(smem + Cfg::kOffO + qs * Cfg::kO);
-                // pair k of this warpgroup's token stream: buffers and phases counted per warpgroup
-                auto dq_pair = [&](int pp, uint32_t c) -> bool {
-                    const int bf = pp & 1, q = wg * 2 + bf;
-                    if (!wait_or_abort(&dsfull[q], ((par >> q) & 1) ^ 1, 0x605, abort_flag)) return false;
-                    tc_fence_after();
-                    const uint32_t sK = smem_u32(smem + Cfg::kOffKV + (c % Cfg::NSLOT) * Cfg::kSlot);
-                    const uint32_t sD = smem_u32(smem + Cfg::kOffDS + q * Cfg::kDS);
+            unsigned long long t_idle = 0;
+            uint32_t spins = 0;
+            while (ok && ib < N) {
+                bool progressed = false;
+                if (ia < N) {
+                    if (npa < 0 && mbar_test_wait(&qfull[ia & 1], (ia >> 1) & 1)) npa = npairs_ring[ia & 7];
+                    if (npa >= 0 && pa < npa) {
+                        const int wg = ia & 1, bf = pa & 1, q = wg * 2 + bf;
+                        const uint32_t tw = tmem + wg * 128;
+                        if (!dp_done) {
+                            const int sv = cv % Cfg::NV;
+                            if (mbar_test_wait(&vfull[sv], (cv / Cfg::NV) & 1) &&
+                                (!((usedA >> q) & 1) || mbar_test_wait(&sdfree[q], ((parA >> q) & 1) ^ 1))) {
+                                tc_fence_after();
+                                const uint32_t sO = smem_u32(smem + Cfg::kOffO + (ia & 1) * Cfg::kO);
+                                const uint32_t sV = smem_u32(smem + Cfg::kOffV + sv * Cfg::kVPair);
 #pragma unroll
-                    for (int hh = 0; hh < NH; ++hh)
+                                for (int kk = 0; kk < DV / 16; ++kk)
+                                    umma_bf16_ss(tw + Cfg::kColDP + bf * 16,
+                                                 sdesc_sw128(sV + (kk / 4) * 16384 + (kk % 4) * 32),
+                                                 sdesc_sw128(sO + (kk / 4) * 2048 + (kk % 4) * 32), id16,
+                                                 kk > 0 ? 1u : 0u);
+                                umma_commit(&vempty[sv]);
+                                ++cv;
+                                dp_done = true;
+                                progressed = true;
+                            }
+                        }
+                        const int sk = ck % Cfg::NK;
+                        if (dp_done && mbar_test_wait(&kfull[sk], (ck / Cfg::NK) & 1)) {
+                            tc_fence_after();
+                            const uint32_t sQ = smem_u32(smem + Cfg::kOffQ + (ia & 1) * Cfg::kQ);
+                            const uint32_t sK = smem_u32(smem + Cfg::kOffK + sk * Cfg::kKPair);
 #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)
-                            umma_bf16_ss(tw + Cfg::kColDQ + hh * 16,
-                                         sdesc_sw128_mn(sK + hh * 2 * 16384 + kk * 2048, 16384, 1024),
-                                         sdesc_sw128(sD + (kk / 4) * 2048 + (kk % 4) * 32), idT,
-                                         (pp > 0 || kk > 0) ? 1u : 0u);
-                    umma_commit(&dsfree[q]);
-                    umma_commit(&empty[c % Cfg::NSLOT]);
-                    return true;
-                };
-                for (int pp = 0; pp < np && ok; ++pp) {
-                    const int bf = pp & 1, q = wg * 2 + bf;
-                    const int sl = cnt % Cfg::NSLOT;
-                    if (!(ok = wait_or_abort(&full[sl], (cnt / Cfg::NSLOT) & 1, 0x606, abort_flag))) break;
-                    if (((used >> q) & 1) &&
-                        !(ok = wait_or_abort(&sdfree[q], ((par >> q) & 1) ^ 1, 0x607, abort_flag)))
-                        break;
-                    tc_fence_after();
-                    const uint32_t sK = smem_u32(smem + Cfg::kOffKV + sl * Cfg::kSlot);
-                    const uint32_t sV = sK + Cfg::kKPair;
-#pragma unroll
-                    for (int kk = 0; kk < DK / 16; ++kk)
-                        umma_bf16_ss(tw + bf * 16, sdesc_sw128(sK + (kk / 4) * 16384 + (kk % 4) * 32),
-                                     sdesc_sw128(sQ + (kk / 4) * 2048 + (kk % 4) * 32), id16, kk > 0 ? 1u : 0u);
-#pragma unroll
-                    for (int kk = 0; kk < DV / 16; ++kk)
-                        umma_bf16_ss(tw + Cfg::kColDP + bf * 16, sdesc_sw128(sV + (kk / 4) * 16384 + (kk % 4) * 32),
-                                     sdesc_sw128(sO + (kk / 4) * 2048 + (kk % 4) * 32), id16, kk > 0 ? 1u : 0u);
-                    umma_commit(&sdfull[q]);
-                    par ^= 1u << q;
-                    used |= 1u << q;
-                    if (pp >= 1) ok = dq_pair(pp - 1, cnt - 1);
-                    ++cnt;
+                            for (int kk = 0; kk < DK / 16; ++kk)
+                                umma_bf16_ss(tw + bf * 16, sdesc_sw128(sK + (kk / 4) * 16384 + (kk % 4) * 32),
+                                             sdesc_sw128(sQ + (kk / 4) * 2048 + (kk % 4) * 32), id16,
+                                             kk > 0 ? 1u : 0u);
+                            umma_commit(&sdfull[q]);
+                            parA ^= 1u << q;
+                            usedA |= 1u << q;
+                            ++ck;
+                            ++pa;
+                            dp_done = false;
+                            progressed = true;
+                        }
+                    }
+                    if (npa >= 0 && pa == npa) {          // every product of token ia issued
+                        umma_commit(&qempty[ia & 1]);
+                        ++ia;
+                        pa = 0;
+                        npa = -1;
+                        progressed = true;
+                    }
                 }
-                if (ok && np > 0) ok = dq_pair(np - 1, cnt - 1);
-                umma_commit(&dqfull[wg]);
-                umma_commit(&qempty[qs]);
+                if (ib < ia || (ib == ia && pb < pa)) {   // pair (ib, pb) has its S^T / dP^T issued
+                    const int wg = ib & 1;
+                    if (npb < 0) npb = npairs_ring[ib & 7];
+                    if (!dqfree_ok)                       // this warpgroup's last token read its dQ^T
+                        dqfree_ok = ib < 2 || mbar_test_wait(&dqfree[wg], ((ib - 2) >> 1) & 1);
+                    if (dqfree_ok && pb < npb) {
+                        const int bf = pb & 1, q = wg * 2 + bf;
+                        if (mbar_test_wait(&dsfull[q], (parB >> q) & 1)) {
+                            tc_fence_after();
+                            const uint32_t tw = tmem + wg * 128;
+                            const uint32_t sK = smem_u32(smem + Cfg::kOffK + (cb % Cfg::NK) * Cfg::kKPair);
+                            const uint32_t sD = smem_u32(smem + Cfg::kOffDS + q * Cfg::kDS);
+#pragma unroll
+                            for (int hh = 0; hh < NH; ++hh)
+#pragma unroll
+                                for (int kk = 0; kk < 8; ++kk)
+                                    umma_bf16_ss(tw + Cfg::kColDQ + hh * 16,
+                                                 sdesc_sw128_mn(sK + hh * 2 * 16384 + kk * 2048, 16384, 1024),
+                                                 sdesc_sw128(sD + (kk / 4) * 2048 + (kk % 4) * 32), idT,
+                                                 (pb > 0 || kk > 0) ? 1u : 0u);
+                            umma_commit(&dsfree[q]);
+                            umma_commit(&kempty[cb % Cfg::NK]);
+                            ++cb;
+                            parB ^= 1u << q;
+                            ++pb;
+                            progressed = true;
+                        }
+                    }
+                    if (dqfree_ok && pb == npb) {         // token ib complete
+                        umma_commit(&dqfull[wg]);
+                        ++ib;
+                        pb = 0;
+                        npb = -1;
+                        dqfree_ok = false;
+                        progressed = true;
+                    }
+                }
+                if (progressed) {
+                    spins = 0;
+                    t_idle = 0;
+                } else if ((++spins & 63u) == 0u) {
+                    if (*abort_flag) {
+                        ok = false;
+                    } else {
+                        const unsigned long long now = globaltimer_ns();
+                        if (t_idle == 0) {
+                            t_idle = now;
+                        } else if (now - t_idle > kWaitLimitNs) {
+                            record_timeout(0x606);
+                            *abort_flag = 1;
+                            ok = false;
+                        }
+                    }
+                }
             }
         }
     } else {

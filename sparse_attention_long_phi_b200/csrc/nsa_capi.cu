@@ -27,6 +27,7 @@
 #include "k_topn.cuh"
 #include "k_append.cuh"
 #include "k_phi_grad.cuh"
+#include "k_phi_bwd.cuh"
 
 using namespace nsa;
 
@@ -415,24 +416,27 @@ PackedParams packed_params(const Shape& s, const float* gates, float* out, float
     return pp;
 }
 
-// compressed branch: out = g_cmp o_cmp (stored), lse[..., 0], the score table
+// compressed branch: out = g_cmp o_cmp (stored), lse[..., 0], the score table;
+// with obranch, o_cmp itself too
 template <int DK, int DV, int HG>
 nsa_status_t launch_cmp(const Shape& s, const AttnMaps& m, const float* gates, float* out, float* lse,
-                        float* lse_cmp, float* pscore, cudaStream_t st) {
+                        float* lse_cmp, float* pscore, cudaStream_t st, float* obranch = nullptr) {
     if (s.C > 0) {
-        const PackedParams pp = packed_params<HG>(s, gates, out, lse, lse_cmp, pscore);
+        PackedParams pp = packed_params<HG>(s, gates, out, lse, lse_cmp, pscore);
+        pp.obranch = obranch;
         NSA_TRY((launch_packed_blk<DK, DV, HG, kModeLse>(s, m.mQ, m.mKc, m.mVc, pp, st)));
         return launch_packed_blk<DK, DV, HG, kModeCmp>(s, m.mQ, m.mKc, m.mVc, pp, st);
     }
     const long long rows = s.B * s.T * s.H;
+    if (obranch && cudaMemsetAsync(obranch, 0, (size_t)rows * s.DV * 4, st) != cudaSuccess) return NSA_ERR_CUDA;
     NSA_LAUNCH("cmp_empty_kernel", st, cmp_empty_kernel<<<(unsigned)ceil_div(rows * s.DV, 256), 256, 0, st>>>(out, lse, rows, (int)s.DV));
     return last_launch();
 }
 
-// selected branch under sel_idx: out += g_slc o_slc, lse[..., 1]
+// selected branch under sel_idx: out += g_slc o_slc, lse[..., 1]; with obranch, o_slc too
 template <int DK, int DV, int HG>
 nsa_status_t launch_sel(const Shape& s, const AttnMaps& m, const float* gates, float* out, float* lse,
-                        const int32_t* sel_idx, cudaStream_t st) {
+                        const int32_t* sel_idx, cudaStream_t st, float* obranch = nullptr) {
     SelParams sp{};
     sp.B = (int)s.B;
     sp.T = (int)s.T;
@@ -443,6 +447,7 @@ nsa_status_t launch_sel(const Shape& s, const AttnMaps& m, const float* gates, f
     sp.idx = sel_idx;
     sp.gates = gates;
     sp.out = out;
+    sp.obranch = obranch;
     sp.lse_user = lse;
     int64_t tpc = (s.B * s.T * s.G) / (148 * 8);
     sp.tpc = (int)std::min<int64_t>(64, std::max<int64_t>(4, tpc));
@@ -454,11 +459,12 @@ nsa_status_t launch_sel(const Shape& s, const AttnMaps& m, const float* gates, f
     return last_launch();
 }
 
-// sliding window: out += g_win o_win, lse[..., 2]
+// sliding window: out += g_win o_win, lse[..., 2]; with obranch, o_win too
 template <int DK, int DV, int HG>
 nsa_status_t launch_win(const Shape& s, const AttnMaps& m, const float* gates, float* out, float* lse,
-                        cudaStream_t st) {
-    const PackedParams pp = packed_params<HG>(s, gates, out, lse, nullptr, nullptr);
+                        cudaStream_t st, float* obranch = nullptr) {
+    PackedParams pp = packed_params<HG>(s, gates, out, lse, nullptr, nullptr);
+    pp.obranch = obranch;
     return launch_packed_blk<DK, DV, HG, kModeWin>(s, m.mQ, m.mKw, m.mVT, pp, st);
 }
 
@@ -470,11 +476,18 @@ struct BranchKV {
     const void *k_cmp, *v_cmp, *k_slc, *v_slc, *k_win, *v_win;
 };
 
+// obranch (optional): [3][B,T,H,DV], each branch's own output o_c before its
+// gate, in the order compressed, selected, window (what the backward's
+// statistics need, saved by a training forward)
 template <int DK, int DV, int HG>
 nsa_status_t forward_impl(const Shape& s, const void* q, const BranchKV& kv,
                           const float* gates, const nsa_phi_params_t* phi, float* out,
                           int32_t* sel_idx, float* lse, void* kc_out, void* vc_out, uint8_t* ws,
-                          cudaStream_t st) {
+                          cudaStream_t st, float* obranch = nullptr) {
+    const size_t ob_stride = (size_t)s.B * s.T * s.H * s.DV;
+    float* ob_cmp = obranch;
+    float* ob_slc = obranch ? obranch + ob_stride : nullptr;
+    float* ob_win = obranch ? obranch + 2 * ob_stride : nullptr;
     const FwdWs L = fwd_layout(s);
     void* kc = kc_out ? kc_out : ws + L.off_kc;
     void* vcT = ws + L.off_vct;
@@ -498,7 +511,7 @@ nsa_status_t forward_impl(const Shape& s, const void* q, const BranchKV& kv,
     AttnMaps m;
     NSA_TRY((attn_maps<DK, DV, HG>(s, q, kv.k_slc, kv.k_win, kc, vcT, vT, vTw, m)));
     // 3-4. compressed attention: LSE pass, then P.V~ with importance scores
-    NSA_TRY((launch_cmp<DK, DV, HG>(s, m, gates, out, lse, lse_cmp, pscore, st)));
+    NSA_TRY((launch_cmp<DK, DV, HG>(s, m, gates, out, lse, lse_cmp, pscore, st, ob_cmp)));
     // 5. top-n selection
     {
         const long long items = s.B * s.T * s.G;
@@ -515,17 +528,74 @@ nsa_status_t forward_impl(const Shape& s, const void* q, const BranchKV& kv,
         NSA_TRY(last_launch());
     }
     // 6. selected attention
-    NSA_TRY((launch_sel<DK, DV, HG>(s, m, gates, out, lse, sel_idx, st)));
+    NSA_TRY((launch_sel<DK, DV, HG>(s, m, gates, out, lse, sel_idx, st, ob_slc)));
     // 7. sliding window
-    return launch_win<DK, DV, HG>(s, m, gates, out, lse, st);
+    return launch_win<DK, DV, HG>(s, m, gates, out, lse, st, ob_win);
 }
 
+
+// ---------------------------------------------- linear phi backward (tcgen05)
+// The products need whole 256-column tiles of the l*D inputs.
+bool phi_bwd_tensor_ok(const Shape& s) { return (s.l * s.DK) % 256 == 0 && (s.l * s.DV) % 256 == 0; }
+
+// kPhiT: dX[b, i*d + j, g, :] += (dY[b,i,g,:] W)[j*D ..]; kPhiDW: dW = dY^T X + s E
+template <int D, int MODE>
+nsa_status_t launch_phi_bwd(const Shape& s, const void* dyb, const void* src, float* dX, float* dW,
+                            const float* colsum, const void* E, cudaStream_t st) {
+    CUtensorMap mY, mB;
+    const uint64_t dY[4] = {(uint64_t)D, (uint64_t)s.G, (uint64_t)s.C, (uint64_t)s.B};
+    const uint64_t sY[3] = {(uint64_t)D * 2, (uint64_t)s.G * D * 2, (uint64_t)s.C * s.G * D * 2};
+    const uint32_t bY[4] = {64, 1, MODE == kPhiT ? 128u : 64u, 1};
+    if (!make_map(&mY, dyb, 4, dY, sY, bY)) return NSA_ERR_CUDA;
+    if (MODE == kPhiT) {
+        const uint64_t dW2[2] = {(uint64_t)s.l * D, (uint64_t)D};
+        const uint64_t sW2[1] = {(uint64_t)s.l * D * 2};
+        const uint32_t bW2[2] = {64, 64};
+        if (!make_map(&mB, src, 2, dW2, sW2, bW2)) return NSA_ERR_CUDA;
+    } else {
+        const uint64_t dX5[5] = {(uint64_t)D, (uint64_t)s.G, (uint64_t)s.d, (uint64_t)(s.T / s.d), (uint64_t)s.B};
+        const uint64_t sX5[4] = {(uint64_t)D * 2, (uint64_t)s.G * D * 2, (uint64_t)s.d * s.G * D * 2,
+                                 (uint64_t)s.T * s.G * D * 2};
+        const uint32_t bX5[5] = {64, 1, 1, 64, 1};
+        if (!make_map(&mB, src, 5, dX5, sX5, bX5)) return NSA_ERR_CUDA;
+    }
+    PhiBwdParams pp{};
+    pp.B = (int)s.B;
+    pp.T = (int)s.T;
+    pp.G = (int)s.G;
+    pp.C = (int)s.C;
+    pp.D = D;
+    pp.l = (int)s.l;
+    pp.d = (int)s.d;
+    pp.dX = dX;
+    pp.dW = dW;
+    pp.s = colsum;
+    pp.E = reinterpret_cast<const __nv_bfloat16*>(E);
+    NSA_TRY(set_smem(phi_bwd_gemm<MODE>, PhiBwdCfg::kSmem));
+    const dim3 grid((unsigned)(s.l * D / PhiBwdCfg::NT),
+                    (unsigned)(MODE == kPhiT ? ceil_div(s.C, 128) : ceil_div(D, 128)),
+                    (unsigned)(MODE == kPhiT ? s.B * s.G : 1));
+    NSA_LAUNCH(MODE == kPhiT ? "phi_bwd_gemm_dx" : "phi_bwd_gemm_dw", st,
+               phi_bwd_gemm<MODE><<<grid, PhiBwdCfg::kThreads, PhiBwdCfg::kSmem, st>>>(mY, mB, pp));
+    return last_launch();
+}
+
+// dK~ and dV~ (fp32 [B,C,G,D]) rounded to bf16 into the workspace
+nsa_status_t phi_bwd_operands(const Shape& s, const float* dkc, const float* dvc, __nv_bfloat16* dyb,
+                              cudaStream_t st) {
+    const long long nk4 = s.B * s.C * s.G * s.DK / 4, nv4 = s.B * s.C * s.G * s.DV / 4;
+    NSA_LAUNCH("f32_to_bf16_kernel", st, f32_to_bf16_kernel<<<(unsigned)ceil_div(nk4, 256), 256, 0, st>>>(dkc, dyb, nk4));
+    NSA_TRY(last_launch());
+    NSA_LAUNCH("f32_to_bf16_kernel", st, f32_to_bf16_kernel<<<(unsigned)ceil_div(nv4, 256), 256, 0, st>>>(
+        dvc, dyb + (size_t)s.B * s.C * s.G * s.DK, nv4));
+    return last_launch();
+}
 
 // -------------------------------------------------------------- backward
 struct BwdWs {
     size_t off_kc, off_vc, off_vct, off_bias, off_lse2, off_dlt, off_dkc, off_dvc, off_cnt,
         off_cur, off_off, off_choff, off_list, off_fix, off_ones, off_obuf, off_lsen, off_lsec, off_ps, off_vt,
-        total;
+        off_dyb, total;
 };
 
 BwdWs bwd_layout(const Shape& s) {
@@ -574,6 +644,9 @@ BwdWs bwd_layout(const Shape& s) {
     o = align256(o + (size_t)s.B * s.T * s.G * s.NSp * 4);
     w.off_vt = o;
     o = align256(o + (size_t)s.B * s.G * s.DVP * s.Tp * 2);
+    // bf16 copies of dK~ and dV~ for the linear phi's tensor-core products
+    w.off_dyb = o;
+    o = align256(o + (size_t)s.B * C1 * s.G * (s.DK + s.DV) * 2);
     w.total = o;
     return w;
 }
@@ -582,7 +655,8 @@ template <int DK, int DV>
 nsa_status_t backward_impl(const Shape& s, const void* q, const void* k, const void* v,
                            const float* gates, const nsa_phi_params_t* phi, const void* dout,
                            const int32_t* sel_idx, float* dq, float* dk, float* dv, float* dgates,
-                           uint8_t* ws, cudaStream_t st) {
+                           uint8_t* ws, cudaStream_t st, const float* saved_lse = nullptr,
+                           const float* saved_o = nullptr) {
     const BwdWs L = bwd_layout(s);
     const int64_t NE = s.B * s.G * s.NS;
     BwdParams p{};
@@ -637,8 +711,17 @@ nsa_status_t backward_impl(const Shape& s, const void* q, const void* k, const v
         return NSA_ERR_CUDA;
     // per-branch statistics under the given selection, from the forward kernels:
     // with unit gates each branch's output is its own o_c, whose dot product with
-    // dO gives d(gate_c) and D_c = g_c <dO, o_c>; the kernels' LSEs come along
-    {
+    // dO gives d(gate_c) and D_c = g_c <dO, o_c>; the kernels' LSEs come along.
+    // A training forward that saved o_c and the LSEs spares these passes.
+    if (saved_o) {
+        const long long rows = s.B * s.T * s.H;
+        for (int br = 0; br < 3; ++br) {
+            NSA_LAUNCH("bwd_branch_stats", st, bwd_branch_stats<<<(unsigned)ceil_div(rows, 8), 256, 0, st>>>(
+                saved_o + (size_t)br * rows * DV, reinterpret_cast<const __nv_bfloat16*>(dout), gates, saved_lse, br,
+                rows, DV, dgates, p.dlt, p.lse2));
+            NSA_TRY(last_launch());
+        }
+    } else {
         constexpr int HG = DK == 192 ? 16 : 4;
         const long long rows = s.B * s.T * s.H;
         float* ones = reinterpret_cast<float*>(ws + L.off_ones);
@@ -789,11 +872,19 @@ nsa_status_t backward_impl(const Shape& s, const void* q, const void* k, const v
             dim3 gc((unsigned)ceil_div(s.C, 128), (unsigned)ceil_div(s.T, kBkvChunk), bg);
             NSA_LAUNCH("bwd_kv_tc_cmp", st, bwd_kv_tc<DK, DV, HG, kBrCmp><<<gc, Cfg::kThreads, Cfg::kSmem, st>>>(mKc, mVc, mQ, mO, kp));
             NSA_TRY(last_launch());
-            dim3 gp((unsigned)s.T, (unsigned)s.G, (unsigned)s.B);
-            NSA_LAUNCH("bwd_phiT_kernel", st, bwd_phiT_kernel<DK><<<gp, DK, 0, st>>>(p, p.dkc, p.wk, dk));
-            NSA_TRY(last_launch());
-            NSA_LAUNCH("bwd_phiT_kernel", st, bwd_phiT_kernel<DV><<<gp, DV, 0, st>>>(p, p.dvc, p.wv, dv));
-            NSA_TRY(last_launch());
+            if (s.phi == NSA_PHI_LINEAR && phi_bwd_tensor_ok(s)) {
+                __nv_bfloat16* dyb = reinterpret_cast<__nv_bfloat16*>(ws + L.off_dyb);
+                NSA_TRY(phi_bwd_operands(s, p.dkc, p.dvc, dyb, st));
+                NSA_TRY((launch_phi_bwd<DK, kPhiT>(s, dyb, p.wk, dk, nullptr, nullptr, nullptr, st)));
+                NSA_TRY((launch_phi_bwd<DV, kPhiT>(s, dyb + (size_t)s.B * s.C * s.G * DK, p.wv, dv, nullptr,
+                                                   nullptr, nullptr, st)));
+            } else {
+                dim3 gp((unsigned)s.T, (unsigned)s.G, (unsigned)s.B);
+                NSA_LAUNCH("bwd_phiT_kernel", st, bwd_phiT_kernel<DK><<<gp, DK, 0, st>>>(p, p.dkc, p.wk, dk));
+                NSA_TRY(last_launch());
+                NSA_LAUNCH("bwd_phiT_kernel", st, bwd_phiT_kernel<DV><<<gp, DV, 0, st>>>(p, p.dvc, p.wv, dv));
+                NSA_TRY(last_launch());
+            }
         }
     }
     return NSA_OK;
@@ -979,6 +1070,29 @@ nsa_status_t nsa_forward(const nsa_config_t* cfg, const void* q, const void* k, 
     return forward_impl<64, 64, 4>(s, q, kv, gates, phi, out, sel_idx, lse, kc_out, vc_out, ws, st);
 }
 
+nsa_status_t nsa_forward_train(const nsa_config_t* cfg, const void* q, const void* k, const void* v,
+                               const float* gates, const nsa_phi_params_t* phi, float* out, int32_t* sel_idx,
+                               float* lse, float* o_branch, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+    Shape s;
+    NSA_TRY(derive(cfg, s));
+    NSA_TRY(supported(s));
+    if (cfg->score_map != 0) return NSA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !gates || !out || !sel_idx || !lse || !o_branch) return NSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(o_branch))
+        return NSA_ERR_INVALID_ARG;
+    const FwdWs L = fwd_layout(s);
+    if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return NSA_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+    const BranchKV kv{k, v, k, v, k, v};
+    if (s.DK == 192)
+        return forward_impl<192, 128, 16>(s, q, kv, gates, phi, out, sel_idx, lse, nullptr, nullptr, ws, st,
+                                          o_branch);
+    return forward_impl<64, 64, 4>(s, q, kv, gates, phi, out, sel_idx, lse, nullptr, nullptr, ws, st, o_branch);
+}
+
 nsa_status_t nsa_forward_branches(const nsa_config_t* cfg, const void* q, const void* k_cmp,
                                   const void* v_cmp, const void* k_slc, const void* v_slc,
                                   const void* k_win, const void* v_win, const float* gates,
@@ -1147,6 +1261,29 @@ nsa_status_t nsa_backward(const nsa_config_t* cfg, const void* q, const void* k,
     return backward_impl<64, 64>(s, q, k, v, gates, phi, dout, sel_idx, dq, dk, dv, dgates, ws, st);
 }
 
+nsa_status_t nsa_backward_saved(const nsa_config_t* cfg, const void* q, const void* k, const void* v,
+                                const float* gates, const nsa_phi_params_t* phi, const void* dout,
+                                const int32_t* sel_idx, const float* lse, const float* o_branch, float* dq,
+                                float* dk, float* dv, float* dgates, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+    Shape s;
+    NSA_TRY(derive(cfg, s));
+    NSA_TRY(supported(s));
+    if (!q || !k || !v || !gates || !dout || !sel_idx || !lse || !o_branch || !dq || !dk || !dv || !dgates)
+        return NSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(o_branch))
+        return NSA_ERR_INVALID_ARG;
+    const BwdWs L = bwd_layout(s);
+    if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return NSA_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+    if (s.DK == 192)
+        return backward_impl<192, 128>(s, q, k, v, gates, phi, dout, sel_idx, dq, dk, dv, dgates, ws, st, lse,
+                                       o_branch);
+    return backward_impl<64, 64>(s, q, k, v, gates, phi, dout, sel_idx, dq, dk, dv, dgates, ws, st, lse, o_branch);
+}
+
 nsa_status_t nsa_profile_enable(int32_t on) {
     std::lock_guard<std::mutex> lk(g_prof_mu);
     g_prof_on = on != 0;
@@ -1231,6 +1368,17 @@ nsa_status_t nsa_backward_phi_params(const nsa_config_t* cfg, const void* k, con
     NSA_TRY(last_launch());
     NSA_LAUNCH("phi_de_kernel", st, phi_de_kernel<<<(unsigned)ceil_div(KV, 256), 256, 0, st>>>(bf(phi->w_v), colsum + s.DK, (int)s.DV, (int)KV, de_v));
     NSA_TRY(last_launch());
+    if (phi_bwd_tensor_ok(s)) {
+        __nv_bfloat16* dyb = reinterpret_cast<__nv_bfloat16*>(ws + L.off_dyb);
+        const __nv_bfloat16* dybv = dyb + (size_t)s.B * s.C * s.G * s.DK;
+        NSA_TRY(phi_bwd_operands(s, dkc, dvc, dyb, st));
+        if (s.DK == 192) {
+            NSA_TRY((launch_phi_bwd<192, kPhiDW>(s, dyb, k, nullptr, dw_k, colsum, phi->e_k, st)));
+            return launch_phi_bwd<128, kPhiDW>(s, dybv, v, nullptr, dw_v, colsum + s.DK, phi->e_v, st);
+        }
+        NSA_TRY((launch_phi_bwd<64, kPhiDW>(s, dyb, k, nullptr, dw_k, colsum, phi->e_k, st)));
+        return launch_phi_bwd<64, kPhiDW>(s, dybv, v, nullptr, dw_v, colsum + s.DK, phi->e_v, st);
+    }
     const int B = (int)s.B, T = (int)s.T, G = (int)s.G, C = (int)s.C, l = (int)s.l, d = (int)s.d;
     if (s.DK == 192) {
         NSA_LAUNCH("phi_dw_kernel", st, phi_dw_kernel<192><<<dim3((unsigned)(KK / 64), 3), 256, 0, st>>>(dkc, bf(k), bf(phi->e_k), B, T, G, C, l, d, dw_k));

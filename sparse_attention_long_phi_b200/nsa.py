@@ -69,6 +69,11 @@ def lib():
         L.nsa_compress_static.argtypes = [pc, _P, _P, pp, _P, _P, _P]
         L.nsa_forward.restype = ctypes.c_int
         L.nsa_forward.argtypes = [pc, _P, _P, _P, _P, pp, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+        L.nsa_forward_train.restype = ctypes.c_int
+        L.nsa_forward_train.argtypes = [pc, _P, _P, _P, _P, pp, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+        L.nsa_backward_saved.restype = ctypes.c_int
+        L.nsa_backward_saved.argtypes = [pc, _P, _P, _P, _P, pp, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                         ctypes.c_size_t, _P]
         L.nsa_forward_branches.restype = ctypes.c_int
         L.nsa_forward_branches.argtypes = [pc] + [_P] * 8 + [pp] + [_P] * 6 + [ctypes.c_size_t, _P]
         L.nsa_decode_rows.restype = ctypes.c_int
@@ -203,6 +208,53 @@ def forward(c: dict, q, k, v, gates, phi=None, want_lse=True, want_kc=False, str
     return res
 
 
+def forward_train(c: dict, q, k, v, gates, phi=None, stream=None, ws=None) -> dict:
+    """Training forward: forward()'s out, idx, lse plus o_branch [3,B,T,H,dv] fp32, each
+    branch's own output before its gate (compressed, selected, window), for backward_saved."""
+    B, T, H, G, dv = c["B"], c["T"], c["H"], c["G"], c["dv"]
+    f32 = dict(dtype=torch.float32, device=q.device)
+    res = {"out": torch.empty(B, T, H, dv, **f32),
+           "idx": torch.empty(B, T, G, c["n"], dtype=torch.int32, device=q.device),
+           "lse": torch.empty(B, T, H, 3, **f32), "o_branch": torch.empty(3, B, T, H, dv, **f32)}
+    if ws is None:
+        ws = alloc_workspace(c, NSA_MODE_FORWARD, q.device)
+    _check("nsa_forward_train", lib().nsa_forward_train(
+        ctypes.byref(make_config(c)), _p(q), _p(k), _p(v), _p(gates), _phi(phi), _p(res["out"]),
+        _p(res["idx"]), _p(res["lse"]), _p(res["o_branch"]), _p(ws), ws.numel(), _stream(stream)))
+    return res
+
+
+def backward_saved(c: dict, q, k, v, gates, dout, idx, lse, o_branch, phi=None, stream=None,
+                   ws=None, want_phi_grads=False) -> dict:
+    """backward() from the statistics forward_train saved (lse, o_branch) for the same inputs
+    and selection idx: dq, dk, dv, dgates (fp32), and the phi parameter gradients as backward()."""
+    B, T, H, G, dk, dv = c["B"], c["T"], c["H"], c["G"], c["dk"], c["dv"]
+    f32 = dict(dtype=torch.float32, device=q.device)
+    res = {"dq": torch.empty(B, T, H, dk, **f32), "dk": torch.empty(B, T, G, dk, **f32),
+           "dv": torch.empty(B, T, G, dv, **f32), "dgates": torch.empty(B, T, H, 3, **f32)}
+    if ws is None:
+        ws = alloc_workspace(c, NSA_MODE_BACKWARD, q.device)
+    cfg = make_config(c)
+    _check("nsa_backward_saved", lib().nsa_backward_saved(
+        ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(gates), _phi(phi), _p(dout), _p(idx),
+        _p(lse), _p(o_branch), _p(res["dq"]), _p(res["dk"]), _p(res["dv"]), _p(res["dgates"]), _p(ws),
+        ws.numel(), _stream(stream)))
+    if want_phi_grads:
+        _phi_grads(c, cfg, k, v, phi, ws, stream, res)
+    return res
+
+
+def _phi_grads(c, cfg, k, v, phi, ws, stream, res):
+    """nsa_backward_phi_params after a backward that left dK~/dV~ in ws."""
+    dk, dv, l = c["dk"], c["dv"], c["l"]
+    f32 = dict(dtype=torch.float32, device=k.device)
+    res.update(dwk=torch.empty(dk, l * dk, **f32), dek=torch.empty(l, dk, **f32),
+               dwv=torch.empty(dv, l * dv, **f32), dev=torch.empty(l, dv, **f32))
+    _check("nsa_backward_phi_params", lib().nsa_backward_phi_params(
+        ctypes.byref(cfg), _p(k), _p(v), _phi(phi), _p(res["dwk"]), _p(res["dek"]), _p(res["dwv"]),
+        _p(res["dev"]), _p(ws), ws.numel(), _stream(stream)))
+
+
 def forward_branches(c: dict, q, kv: dict, gates, phi=None, want_lse=True, want_kc=False,
                      stream=None, want_scores=False) -> dict:
     """Prefill forward with independent keys/values per branch: kv = dict(k_cmp, v_cmp,
@@ -323,26 +375,23 @@ def decode_append(c: dict, k_new, v_new, k_cache, v_cache, kv_start, kv_len, kc_
         _p(kc_cache), _p(vc_cache), _p(cmp_start), _phi(phi), _stream(stream)))
 
 
-def backward(c: dict, q, k, v, gates, dout, idx, phi=None, stream=None, want_phi_grads=False) -> dict:
+def backward(c: dict, q, k, v, gates, dout, idx, phi=None, stream=None, want_phi_grads=False,
+             ws=None) -> dict:
     """Gradients with the selection idx [B,T,G,n] held fixed: dq, dk, dv, dgates (fp32); with
     want_phi_grads (linear phi) also dwk [dk, l*dk], dek [l, dk], dwv [dv, l*dv], dev [l, dv]."""
     B, T, H, G, dk, dv = c["B"], c["T"], c["H"], c["G"], c["dk"], c["dv"]
     f32 = dict(dtype=torch.float32, device=q.device)
     res = {"dq": torch.empty(B, T, H, dk, **f32), "dk": torch.empty(B, T, G, dk, **f32),
            "dv": torch.empty(B, T, G, dv, **f32), "dgates": torch.empty(B, T, H, 3, **f32)}
-    ws = alloc_workspace(c, NSA_MODE_BACKWARD, q.device)
+    if ws is None:
+        ws = alloc_workspace(c, NSA_MODE_BACKWARD, q.device)
     cfg = make_config(c)
     _check("nsa_backward", lib().nsa_backward(
         ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(gates), _phi(phi), _p(dout), _p(idx),
         _p(res["dq"]), _p(res["dk"]), _p(res["dv"]), _p(res["dgates"]), _p(ws), ws.numel(),
         _stream(stream)))
     if want_phi_grads:
-        l = c["l"]
-        res.update(dwk=torch.empty(dk, l * dk, **f32), dek=torch.empty(l, dk, **f32),
-                   dwv=torch.empty(dv, l * dv, **f32), dev=torch.empty(l, dv, **f32))
-        _check("nsa_backward_phi_params", lib().nsa_backward_phi_params(
-            ctypes.byref(cfg), _p(k), _p(v), _phi(phi), _p(res["dwk"]), _p(res["dek"]), _p(res["dwv"]),
-            _p(res["dev"]), _p(ws), ws.numel(), _stream(stream)))
+        _phi_grads(c, cfg, k, v, phi, ws, stream, res)
     return res
 
 

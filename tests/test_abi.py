@@ -183,3 +183,28 @@ def test_forward_branches_validation_and_score_table_on_host(L):
     assert off + 4 * 8192 * 4 * 128 <= small
     assert lib.nsa_forward_score_table(ctypes.byref(L.make_config(dict(base, d=12))), None) == -1
     assert lib.nsa_check_timeout_path(0, None) == 1                  # limit outside 1 .. 2e9 ns
+
+
+def test_training_forward_and_saved_backward_validation_on_host(L):
+    lib = L.lib()
+    cb = L.make_config(dict(I.WORKLOADS["train_fwd_bwd_B2_T16384"]))
+    fake = ctypes.c_void_p(1 << 20)
+    big = 1 << 40
+    # nsa_forward_train(cfg, q, k, v, gates, phi, out, sel_idx, lse, o_branch, ws, bytes, stream)
+    assert lib.nsa_forward_train(ctypes.byref(cb), fake, fake, fake, fake, None, fake, fake, None, fake,
+                                 fake, big, None) == 1                  # lse is required
+    assert lib.nsa_forward_train(ctypes.byref(cb), fake, fake, fake, fake, None, fake, fake, fake, None,
+                                 fake, big, None) == 1                  # o_branch is required
+    assert lib.nsa_forward_train(ctypes.byref(cb), fake, fake, fake, fake, None, fake, fake, fake,
+                                 ctypes.c_void_p((1 << 20) + 4), fake, big, None) == 1   # misaligned
+    assert lib.nsa_forward_train(ctypes.byref(cb), fake, fake, fake, fake, None, fake, fake, fake, fake,
+                                 fake, 64, None) == 3                   # workspace too small
+    # nsa_backward_saved(cfg, q, k, v, gates, phi, dout, sel_idx, lse, o_branch, dq, dk, dv, dgates,
+    #                    ws, bytes, stream)
+    args = [fake] * 4
+    assert lib.nsa_backward_saved(ctypes.byref(cb), *args, None, fake, fake, None, fake, *args, fake, big,
+                                  None) == 1                            # no saved LSE
+    assert lib.nsa_backward_saved(ctypes.byref(cb), *args, None, fake, fake, fake, None, *args, fake, big,
+                                  None) == 1                            # no saved branch outputs
+    assert lib.nsa_backward_saved(ctypes.byref(cb), *args, None, fake, fake, fake, fake, *args, fake, 64,
+                                  None) == 3

@@ -215,132 +215,79 @@ __global__ void __launch_bounds__(352, 1)
         }
     } else if (warp == 9) {
         // ----------------------------------------------------------- MMA
-        // Two streams issued by one thread, each as soon as it is ready:
-        //   A  dP^T then S^T of the next pair (its V / K staged, its TMEM buffer read
-        //      by the softmax), token after token;
-        //   B  dQ^T of the oldest pair whose dS^T tile is written.
-        // So a pair's dQ^T products never wait for the next pair's rows, and its K
-        // slot returns to the producer as soon as they are done.  Every wait is a
-        // test; no progress for the wait limit ends the CTA with an error.
+        // Per pair: dP^T first (its V slot returns to the producer as soon as it is
+        // done), S^T, then the dQ^T products of the previous pair, whose dS^T the
+        // softmax has written meanwhile.  (Issuing the two streams by readiness
+        // instead measured no faster: the N = 16 products keep the pipe busy.)
         if (lane == 0) {
             constexpr uint32_t id16 = idesc_bf16(128, 16);
             constexpr uint32_t idT = idesc_bf16_amn(128, 16);
-            uint32_t ck = 0, cv = 0, cb = 0;      // K, V slots used by A; K slots released by B
-            // per (warpgroup, buffer) q: bit q = parity of A's S/dP issues, any issue; of B's dQ^T issues
-            uint32_t parA = 0, usedA = 0, parB = 0;
-            int ia = 0, pa = 0, npa = -1;         // A: token, pair, its pairs (-1: not started)
-            int ib = 0, pb = 0, npb = -1;         // B
-            bool dp_done = false, dqfree_ok = false;
+            uint32_t ck = 0, cv = 0;      // K and V pair slots consumed
+            // per (warpgroup, buffer) q: bit q of `par` = parity of its S/dP issues so far,
+            // bit q of `used` = at least one issue
+            uint32_t par = 0, used = 0;
             bool ok = true;
-            unsigned long long t_idle = 0;
-            uint32_t spins = 0;
-            while (ok && ib < N) {
-                bool progressed = false;
-                if (ia < N) {
-                    if (npa < 0 && mbar_test_wait(&qfull[ia & 1], (ia >> 1) & 1)) npa = npairs_ring[ia & 7];
-                    if (npa >= 0 && pa < npa) {
-                        const int wg = ia & 1, bf = pa & 1, q = wg * 2 + bf;
-                        const uint32_t tw = tmem + wg * 128;
-                        if (!dp_done) {
-                            const int sv = cv % Cfg::NV;
-                            if (mbar_test_wait(&vfull[sv], (cv / Cfg::NV) & 1) &&
-                                (!((usedA >> q) & 1) || mbar_test_wait(&sdfree[q], ((parA >> q) & 1) ^ 1))) {
-                                tc_fence_after();
-                                const uint32_t sO = smem_u32(smem + Cfg::kOffO + (ia & 1) * Cfg::kO);
-                                const uint32_t sV = smem_u32(smem + Cfg::kOffV + sv * Cfg::kVPair);
+            for (int i = 0; i < N && ok; ++i) {
+                const int qs = i & 1, wg = i & 1;
+                const uint32_t tw = tmem + wg * 128;
+                if (!(ok = wait_or_abort(&qfull[qs], (i >> 1) & 1, 0x603, abort_flag))) break;
+                const int np = npairs_ring[i & 7];
+                // this warpgroup's previous token has read its dQ^T
+                if (i >= 2 && !(ok = wait_or_abort(&dqfree[wg], ((i - 2) >> 1) & 1, 0x604, abort_flag))) break;
+                tc_fence_after();
+                const uint32_t sQ = smem_u32(smem + Cfg::kOffQ + qs * Cfg::kQ);
+                const uint32_t sO = smem_u32(smem + Cfg::kOffO + qs * Cfg::kO);
+                // pair k of this warpgroup's token stream: buffers and phases counted per warpgroup
+                auto dq_pair = [&](int pp, uint32_t c) -> bool {
+                    const int bf = pp & 1, q = wg * 2 + bf;
+                    if (!wait_or_abort(&dsfull[q], ((par >> q) & 1) ^ 1, 0x605, abort_flag)) return false;
+                    tc_fence_after();
+                    const uint32_t sK = smem_u32(smem + Cfg::kOffK + (c % Cfg::NK) * Cfg::kKPair);
+                    const uint32_t sD = smem_u32(smem + Cfg::kOffDS + q * Cfg::kDS);
 #pragma unroll
-                                for (int kk = 0; kk < DV / 16; ++kk)
-                                    umma_bf16_ss(tw + Cfg::kColDP + bf * 16,
-                                                 sdesc_sw128(sV + (kk / 4) * 16384 + (kk % 4) * 32),
-                                                 sdesc_sw128(sO + (kk / 4) * 2048 + (kk % 4) * 32), id16,
-                                                 kk > 0 ? 1u : 0u);
-                                umma_commit(&vempty[sv]);
-                                ++cv;
-                                dp_done = true;
-                                progressed = true;
-                            }
-                        }
-                        const int sk = ck % Cfg::NK;
-                        if (dp_done && mbar_test_wait(&kfull[sk], (ck / Cfg::NK) & 1)) {
-                            tc_fence_after();
-                            const uint32_t sQ = smem_u32(smem + Cfg::kOffQ + (ia & 1) * Cfg::kQ);
-                            const uint32_t sK = smem_u32(smem + Cfg::kOffK + sk * Cfg::kKPair);
+                    for (int hh = 0; hh < NH; ++hh)
 #pragma unroll
-                            for (int kk = 0; kk < DK / 16; ++kk)
-                                umma_bf16_ss(tw + bf * 16, sdesc_sw128(sK + (kk / 4) * 16384 + (kk % 4) * 32),
-                                             sdesc_sw128(sQ + (kk / 4) * 2048 + (kk % 4) * 32), id16,
-                                             kk > 0 ? 1u : 0u);
-                            umma_commit(&sdfull[q]);
-                            parA ^= 1u << q;
-                            usedA |= 1u << q;
-                            ++ck;
-                            ++pa;
-                            dp_done = false;
-                            progressed = true;
-                        }
-                    }
-                    if (npa >= 0 && pa == npa) {          // every product of token ia issued
-                        umma_commit(&qempty[ia & 1]);
-                        ++ia;
-                        pa = 0;
-                        npa = -1;
-                        progressed = true;
-                    }
+                        for (int kk = 0; kk < 8; ++kk)
+                            umma_bf16_ss(tw + Cfg::kColDQ + hh * 16,
+                                         sdesc_sw128_mn(sK + hh * 2 * 16384 + kk * 2048, 16384, 1024),
+                                         sdesc_sw128(sD + (kk / 4) * 2048 + (kk % 4) * 32), idT,
+                                         (pp > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&dsfree[q]);
+                    umma_commit(&kempty[c % Cfg::NK]);
+                    return true;
+                };
+                for (int pp = 0; pp < np && ok; ++pp) {
+                    const int bf = pp & 1, q = wg * 2 + bf;
+                    const int sv = cv % Cfg::NV;
+                    if (!(ok = wait_or_abort(&vfull[sv], (cv / Cfg::NV) & 1, 0x606, abort_flag))) break;
+                    if (((used >> q) & 1) &&
+                        !(ok = wait_or_abort(&sdfree[q], ((par >> q) & 1) ^ 1, 0x607, abort_flag)))
+                        break;
+                    tc_fence_after();
+                    const uint32_t sV = smem_u32(smem + Cfg::kOffV + sv * Cfg::kVPair);
+#pragma unroll
+                    for (int kk = 0; kk < DV / 16; ++kk)
+                        umma_bf16_ss(tw + Cfg::kColDP + bf * 16, sdesc_sw128(sV + (kk / 4) * 16384 + (kk % 4) * 32),
+                                     sdesc_sw128(sO + (kk / 4) * 2048 + (kk % 4) * 32), id16, kk > 0 ? 1u : 0u);
+                    umma_commit(&vempty[sv]);
+                    ++cv;
+                    const int sk = ck % Cfg::NK;
+                    if (!(ok = wait_or_abort(&kfull[sk], (ck / Cfg::NK) & 1, 0x60C, abort_flag))) break;
+                    tc_fence_after();
+                    const uint32_t sK = smem_u32(smem + Cfg::kOffK + sk * Cfg::kKPair);
+#pragma unroll
+                    for (int kk = 0; kk < DK / 16; ++kk)
+                        umma_bf16_ss(tw + bf * 16, sdesc_sw128(sK + (kk / 4) * 16384 + (kk % 4) * 32),
+                                     sdesc_sw128(sQ + (kk / 4) * 2048 + (kk % 4) * 32), id16, kk > 0 ? 1u : 0u);
+                    umma_commit(&sdfull[q]);
+                    par ^= 1u << q;
+                    used |= 1u << q;
+                    if (pp >= 1) ok = dq_pair(pp - 1, ck - 1);
+                    ++ck;
                 }
-                if (ib < ia || (ib == ia && pb < pa)) {   // pair (ib, pb) has its S^T / dP^T issued
-                    const int wg = ib & 1;
-                    if (npb < 0) npb = npairs_ring[ib & 7];
-                    if (!dqfree_ok)                       // this warpgroup's last token read its dQ^T
-                        dqfree_ok = ib < 2 || mbar_test_wait(&dqfree[wg], ((ib - 2) >> 1) & 1);
-                    if (dqfree_ok && pb < npb) {
-                        const int bf = pb & 1, q = wg * 2 + bf;
-                        if (mbar_test_wait(&dsfull[q], (parB >> q) & 1)) {
-                            tc_fence_after();
-                            const uint32_t tw = tmem + wg * 128;
-                            const uint32_t sK = smem_u32(smem + Cfg::kOffK + (cb % Cfg::NK) * Cfg::kKPair);
-                            const uint32_t sD = smem_u32(smem + Cfg::kOffDS + q * Cfg::kDS);
-#pragma unroll
-                            for (int hh = 0; hh < NH; ++hh)
-#pragma unroll
-                                for (int kk = 0; kk < 8; ++kk)
-                                    umma_bf16_ss(tw + Cfg::kColDQ + hh * 16,
-                                                 sdesc_sw128_mn(sK + hh * 2 * 16384 + kk * 2048, 16384, 1024),
-                                                 sdesc_sw128(sD + (kk / 4) * 2048 + (kk % 4) * 32), idT,
-                                                 (pb > 0 || kk > 0) ? 1u : 0u);
-                            umma_commit(&dsfree[q]);
-                            umma_commit(&kempty[cb % Cfg::NK]);
-                            ++cb;
-                            parB ^= 1u << q;
-                            ++pb;
-                            progressed = true;
-                        }
-                    }
-                    if (dqfree_ok && pb == npb) {         // token ib complete
-                        umma_commit(&dqfull[wg]);
-                        ++ib;
-                        pb = 0;
-                        npb = -1;
-                        dqfree_ok = false;
-                        progressed = true;
-                    }
-                }
-                if (progressed) {
-                    spins = 0;
-                    t_idle = 0;
-                } else if ((++spins & 63u) == 0u) {
-                    if (*abort_flag) {
-                        ok = false;
-                    } else {
-                        const unsigned long long now = globaltimer_ns();
-                        if (t_idle == 0) {
-                            t_idle = now;
-                        } else if (now - t_idle > kWaitLimitNs) {
-                            record_timeout(0x606);
-                            *abort_flag = 1;
-                            ok = false;
-                        }
-                    }
-                }
+                if (ok && np > 0) ok = dq_pair(np - 1, ck - 1);
+                umma_commit(&dqfull[wg]);
+                umma_commit(&qempty[qs]);
             }
         }
     } else {

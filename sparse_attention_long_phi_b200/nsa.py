@@ -208,14 +208,16 @@ def forward(c: dict, q, k, v, gates, phi=None, want_lse=True, want_kc=False, str
     return res
 
 
-def forward_train(c: dict, q, k, v, gates, phi=None, stream=None, ws=None) -> dict:
+def forward_train(c: dict, q, k, v, gates, phi=None, stream=None, ws=None, res=None) -> dict:
     """Training forward: forward()'s out, idx, lse plus o_branch [3,B,T,H,dv] fp32, each
-    branch's own output before its gate (compressed, selected, window), for backward_saved."""
+    branch's own output before its gate (compressed, selected, window), for backward_saved.
+    `res` (a previous result) is written in place instead of allocating new tensors."""
     B, T, H, G, dv = c["B"], c["T"], c["H"], c["G"], c["dv"]
     f32 = dict(dtype=torch.float32, device=q.device)
-    res = {"out": torch.empty(B, T, H, dv, **f32),
-           "idx": torch.empty(B, T, G, c["n"], dtype=torch.int32, device=q.device),
-           "lse": torch.empty(B, T, H, 3, **f32), "o_branch": torch.empty(3, B, T, H, dv, **f32)}
+    if res is None:
+        res = {"out": torch.empty(B, T, H, dv, **f32),
+               "idx": torch.empty(B, T, G, c["n"], dtype=torch.int32, device=q.device),
+               "lse": torch.empty(B, T, H, 3, **f32), "o_branch": torch.empty(3, B, T, H, dv, **f32)}
     if ws is None:
         ws = alloc_workspace(c, NSA_MODE_FORWARD, q.device)
     _check("nsa_forward_train", lib().nsa_forward_train(
@@ -225,13 +227,15 @@ def forward_train(c: dict, q, k, v, gates, phi=None, stream=None, ws=None) -> di
 
 
 def backward_saved(c: dict, q, k, v, gates, dout, idx, lse, o_branch, phi=None, stream=None,
-                   ws=None, want_phi_grads=False) -> dict:
+                   ws=None, want_phi_grads=False, res=None) -> dict:
     """backward() from the statistics forward_train saved (lse, o_branch) for the same inputs
-    and selection idx: dq, dk, dv, dgates (fp32), and the phi parameter gradients as backward()."""
+    and selection idx: dq, dk, dv, dgates (fp32), and the phi parameter gradients as backward().
+    `res` (a previous result) is written in place instead of allocating new tensors."""
     B, T, H, G, dk, dv = c["B"], c["T"], c["H"], c["G"], c["dk"], c["dv"]
     f32 = dict(dtype=torch.float32, device=q.device)
-    res = {"dq": torch.empty(B, T, H, dk, **f32), "dk": torch.empty(B, T, G, dk, **f32),
-           "dv": torch.empty(B, T, G, dv, **f32), "dgates": torch.empty(B, T, H, 3, **f32)}
+    if res is None:
+        res = {"dq": torch.empty(B, T, H, dk, **f32), "dk": torch.empty(B, T, G, dk, **f32),
+               "dv": torch.empty(B, T, G, dv, **f32), "dgates": torch.empty(B, T, H, 3, **f32)}
     if ws is None:
         ws = alloc_workspace(c, NSA_MODE_BACKWARD, q.device)
     cfg = make_config(c)
@@ -245,11 +249,13 @@ def backward_saved(c: dict, q, k, v, gates, dout, idx, lse, o_branch, phi=None, 
 
 
 def _phi_grads(c, cfg, k, v, phi, ws, stream, res):
-    """nsa_backward_phi_params after a backward that left dK~/dV~ in ws."""
+    """nsa_backward_phi_params after a backward that left dK~/dV~ in ws (into res's
+    dwk/dek/dwv/dev when it has them)."""
     dk, dv, l = c["dk"], c["dv"], c["l"]
     f32 = dict(dtype=torch.float32, device=k.device)
-    res.update(dwk=torch.empty(dk, l * dk, **f32), dek=torch.empty(l, dk, **f32),
-               dwv=torch.empty(dv, l * dv, **f32), dev=torch.empty(l, dv, **f32))
+    if "dwk" not in res:
+        res.update(dwk=torch.empty(dk, l * dk, **f32), dek=torch.empty(l, dk, **f32),
+                   dwv=torch.empty(dv, l * dv, **f32), dev=torch.empty(l, dv, **f32))
     _check("nsa_backward_phi_params", lib().nsa_backward_phi_params(
         ctypes.byref(cfg), _p(k), _p(v), _phi(phi), _p(res["dwk"]), _p(res["dek"]), _p(res["dwv"]),
         _p(res["dev"]), _p(ws), ws.numel(), _stream(stream)))

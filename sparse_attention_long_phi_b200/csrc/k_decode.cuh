@@ -6,15 +6,15 @@
 // HBM-bound: every cache row is read once.  The 16 heads of a GQA group are
 // the M = 16 side of warp-level bf16 tensor-core products (mma.sync
 // m16n8k16, fp32 accumulate).  The two streaming kernels are persistent (one
-// CTA of 8 warps per SM).  The chunks of 32 cache rows of all (seq, group)
-// pairs form one sequence that is cut into equal contiguous ranges, one per
-// CTA; a CTA walks its range one (seq, group) segment at a time, its warps
-// taking the segment's chunks round-robin.  Each warp pipelines K and V
-// separately (the next chunk's K is in flight while this chunk's softmax and
-// P.V run, its V while the next logits run) and keeps an online softmax; the
-// warps merge once per segment into one record, stored at slot
-// (CTA index + seq*G + group), which is unique because consecutive pairs
-// share at most one CTA.
+// CTA of 8 warps per SM).  Each warp pipelines K and V separately (the next
+// chunk's K is in flight while this chunk's softmax and P.V run, its V while
+// the next logits run) and keeps an online softmax.  Compressed stream: the
+// chunks of 32 cache rows of all (seq, group) pairs form one sequence cut into
+// equal contiguous ranges, one per warp; a warp streams its range across pair
+// boundaries and writes a record per pair it touched at slot (warp index +
+// seq*G + group), unique because consecutive pairs share at most one warp.
+// Selected/window stream: the same with ranges per CTA, whose warps take a
+// pair's chunks round-robin and merge once per pair into one record.
 //   1. dec_cmp_stream   compressed cache: per segment (max, sum, unnormalised
 //                       O); per chunk the head max and the per-head selection-
 //                       block sums of exp(logit - chunk max), mapped with the
@@ -56,7 +56,7 @@ struct DecParams {
     float* lse;
     float* cmax;     // [S*G][NCH][16]            chunk max per head (log2 units)
     float* bsum;     // [S*G][NCH][kDecNBS][16]   per-head block sums of exp2(s - chunk max)
-    float* part1;    // [grid1 + S*G][16][DV+4]   segment max, sum, -, -, unnormalised O
+    float* part1;    // [grid1*8 + S*G][16][DV+4] per warp and pair: max, sum, -, -, unnormalised O
     float* ocmp;     // [S*G][16][DV]             normalised compressed-branch output
     float* lsecmp;   // [S*G][16]                 log2 units
     float* part2;    // [grid3 + S*G][2][16][DV+4] per segment and branch (selected, window)
@@ -174,10 +174,10 @@ template <int DK, int DV>
 __global__ void __launch_bounds__(256, 1) dec_cmp_stream(const DecParams p) {
     constexpr int KP = DK * 2 + 16, STG = dec_stage_bytes<DK, DV>();
     extern __shared__ __align__(16) uint8_t dsm[];
-    float* mrg = reinterpret_cast<float*>(dsm);                                  // [8][16][DV] at merges
     float(*pt)[16][33] = reinterpret_cast<float(*)[16][33]>(dsm + kDecW * STG);  // [8][16][33]
-    __shared__ float wm[kDecW][16], wl[kDecW][16];
     __shared__ int pre[kDecMaxSeqs + 1];
+    __shared__ int64_t cbs[kDecMaxSeqs];             // compressed row start of sequence s
+    __shared__ int ccs[kDecMaxSeqs];                 // compressed rows of sequence s
     __shared__ uint64_t kbar[kDecW], vbar[kDecW];    // per warp: its K / V rows landed
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gr = lane >> 2, tg = lane & 3;
     uint8_t* ks = dsm + warp * STG;
@@ -197,6 +197,8 @@ __global__ void __launch_bounds__(256, 1) dec_cmp_stream(const DecParams p) {
             if (s < p.S) {
                 int L, C;
                 if (dec_seq_ok(p, s, L, C)) cnt = p.G * ((C + 31) / 32);
+                ccs[s] = C;
+                cbs[s] = p.cmp_off[s];
             }
             int inc = cnt;
 #pragma unroll
@@ -214,59 +216,79 @@ __global__ void __launch_bounds__(256, 1) dec_cmp_stream(const DecParams p) {
     if (blockIdx.x == 0)
         for (int s = threadIdx.x; s <= p.S; s += blockDim.x) p.cpre[s] = pre[s];
     const long long N = pre[p.S];
-    const int b = blockIdx.x;
-    long long x = dec_range_start(b, N, gridDim.x);
-    const long long x1 = dec_range_start(b + 1, N, gridDim.x);
+    // Each warp owns a contiguous, equal range of the chunk sequence and streams it
+    // on its own: a chunk's K and V copies are issued as soon as the previous
+    // chunk has read its staging rows, across (seq, group) boundaries too, and
+    // the warp writes one online-softmax record per (seq, group) it touched, at
+    // slot (warp index + seq*G + group), unique because consecutive pairs share
+    // at most one warp.  No CTA-wide barrier after the prefix.
+    const int gw = blockIdx.x * kDecW + warp, W = gridDim.x * kDecW;
+    long long x = dec_range_start(gw, N, W);
+    const long long x1 = dec_range_start(gw + 1, N, W);
     const float cl = p.scale_log2;
     const bool fast = p.spb == 4 && p.cps == 2;
     uint32_t kph = 0, vph = 0;
     const uint64_t pol = l2_evict_first();
-    while (x < x1) {
-        // segment: consecutive chunks of one (seq, group)
-        int lo = 0, hi = p.S;                       // largest lo with pre[lo] <= x
+    const size_t kst = (size_t)p.G * DK, vst = (size_t)p.G * DV;
+    struct Seg {
+        int s, g, c, C, nch;
+        int64_t cbase;
+    };
+    // (seq, group, chunk) of item xx
+    auto locate = [&](long long xx, Seg& q) {
+        int lo = 0, hi = p.S;                       // largest lo with pre[lo] <= xx
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
-            if (pre[mid] <= x) lo = mid;
+            if (pre[mid] <= xx) lo = mid;
             else hi = mid;
         }
-        const int s = lo;
-        const int64_t cbase = p.cmp_off[s];
-        int Ls, C;
-        dec_seq_ok(p, s, Ls, C);                    // s holds chunks, so it passed this check
-        const int nch = (C + 31) / 32;
-        const int r = (int)(x - pre[s]);
-        const int g = r / nch, cfirst = r - g * nch;
-        const int n = (int)min((long long)(nch - cfirst), x1 - x);
-        const size_t sg = (size_t)s * p.G + g;
-        const size_t kst = (size_t)p.G * DK, vst = (size_t)p.G * DV;
-        const __nv_bfloat16* kb = p.kccache + ((size_t)cbase * p.G + g) * DK;
-        const __nv_bfloat16* vb = p.vccache + ((size_t)cbase * p.G + g) * DV;
-        auto issue_k = [&](int c) { warp_bulk_rows<DK>(ks, kb + (size_t)c * 32 * kst, kst, C - c * 32, &kbar[warp], pol); };
-        auto issue_v = [&](int c) { warp_bulk_rows<DV>(vs, vb + (size_t)c * 32 * vst, vst, C - c * 32, &vbar[warp], pol); };
+        q.s = lo;                                   // lo holds chunks, so it passed the length checks
+        q.C = ccs[lo];
+        q.nch = (q.C + 31) / 32;
+        const int r = (int)(xx - pre[lo]);
+        q.g = r / q.nch;
+        q.c = r - q.g * q.nch;
+        q.cbase = cbs[lo];
+    };
+    auto issue_k = [&](const Seg& q) {
+        warp_bulk_rows<DK>(ks, p.kccache + ((size_t)(q.cbase + (int64_t)q.c * 32) * p.G + q.g) * DK, kst,
+                           q.C - q.c * 32, &kbar[warp], pol);
+    };
+    auto issue_v = [&](const Seg& q) {
+        warp_bulk_rows<DV>(vs, p.vccache + ((size_t)(q.cbase + (int64_t)q.c * 32) * p.G + q.g) * DV, vst,
+                           q.C - q.c * 32, &vbar[warp], pol);
+    };
+    if (x < x1) {
+        Seg cur;
+        locate(x, cur);
+        issue_k(cur);
+        issue_v(cur);
         uint32_t qa[DK / 16][4];
-        load_q_frags<DK>(p, s, g, qa);
+        load_q_frags<DK>(p, cur.s, cur.g, qa);
         float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
         float o[DV / 8][4];
 #pragma unroll
         for (int nt = 0; nt < DV / 8; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
-        int i = warp;
-        if (i < n) {
-            issue_k(cfirst + i);
-            issue_v(cfirst + i);
-        }
-        for (; i < n; i += kDecW) {
-            const int c = cfirst + i;
-            const bool more = i + kDecW < n;
+        for (;;) {
+            const int c = cur.c;
             if (!mbar_wait(&kbar[warp], kph, 0x401)) break;   // K of chunk c
             kph ^= 1;
             __syncwarp();
             float sf[4][4];
             warp_logits<DK>(qa, smem_u32(ks), sf);
             __syncwarp();
-            if (more) issue_k(c + kDecW);
-            const int nval = min(32, C - c * 32);
+            // the next item: the following chunk of this pair, or the next pair's first
+            const bool more = x + 1 < x1;
+            Seg nxt = cur;
+            const bool same = c + 1 < cur.nch;
+            if (more) {
+                if (same) nxt.c = c + 1;
+                else locate(x + 1, nxt);
+                issue_k(nxt);
+            }
+            const int nval = min(32, cur.C - c * 32);
             float mc0 = -INFINITY, mc1 = -INFINITY;
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt)
@@ -301,7 +323,7 @@ __global__ void __launch_bounds__(256, 1) dec_cmp_stream(const DecParams p) {
             }
             // per-head selection-block sums of this chunk: slot jl = block 32c/spb + jl
             // takes chunk key i with weight |[i, i+cps) n [jl*spb, jl*spb+spb)|
-            const size_t cr = sg * p.NCH + c;
+            const size_t cr = ((size_t)cur.s * p.G + cur.g) * p.NCH + c;
             float* bdst = p.bsum + cr * kDecNBS * 16;
             if (fast) {
                 // spb = 4, cps = 2: slot jl = 2 A_jl - P(4jl+3) + P(4jl-1), A = sum of the
@@ -375,11 +397,36 @@ __global__ void __launch_bounds__(256, 1) dec_cmp_stream(const DecParams p) {
             }
             warp_pv<DV>(sf, smem_u32(vs), o);
             __syncwarp();
-            if (more) issue_v(c + kDecW);
+            if (more) issue_v(nxt);
+            if (!more || !same) {
+                // this warp's record of (seq, group): (max, sum, -, -, O relative to max)
+                constexpr int REC = DV + 4;
+                const size_t sg = (size_t)cur.s * p.G + cur.g;
+                float* rec = p.part1 + ((size_t)gw + sg) * 16 * REC;
+                if (tg == 0) {
+                    rec[gr * REC] = m0;
+                    rec[gr * REC + 1] = l0;
+                    rec[(gr + 8) * REC] = m1;
+                    rec[(gr + 8) * REC + 1] = l1;
+                }
+#pragma unroll
+                for (int nt = 0; nt < DV / 8; ++nt) {
+                    const int cc = 4 + nt * 8 + tg * 2;
+                    *reinterpret_cast<float2*>(rec + gr * REC + cc) = make_float2(o[nt][0], o[nt][1]);
+                    *reinterpret_cast<float2*>(rec + (gr + 8) * REC + cc) = make_float2(o[nt][2], o[nt][3]);
+                }
+                m0 = m1 = -INFINITY;
+                l0 = l1 = 0.f;
+#pragma unroll
+                for (int nt = 0; nt < DV / 8; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+                if (more) load_q_frags<DK>(p, nxt.s, nxt.g, qa);
+            }
+            if (!more) break;
+            cur = nxt;
+            ++x;
         }
-        // no copy is in flight: the staging area becomes the merge scratch
-        dec_merge_record<DV>(m0, m1, l0, l1, o, mrg, wm, wl, p.part1 + ((size_t)b + sg) * 16 * (DV + 4));
-        x += n;
     }
 }
 
@@ -394,8 +441,7 @@ __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
     __shared__ float lse2[16];
     __shared__ int recb[kDecMaxChunks];
     __shared__ int nrec;
-    __shared__ float tsv[8 * 16];
-    __shared__ int tsi[8 * 16];
+    __shared__ int tsm[256 + 16 + 8 * 8 + 32];       // top-n scratch
     const int g = blockIdx.x, s = blockIdx.y;
     dep_launch();
     int L, C;
@@ -411,7 +457,7 @@ __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
         int cnt = 0;
         if (nch > 0) {
             const long long X0 = (long long)p.cpre[s] + (long long)g * nch;
-            cnt = dec_record_ctas(X0, X0 + nch, p.cpre[p.S], p.grid1, recb, kDecMaxChunks);
+            cnt = dec_record_ctas(X0, X0 + nch, p.cpre[p.S], p.grid1 * kDecW, recb, kDecMaxChunks);
         }
         nrec = cnt;
     }
@@ -448,19 +494,34 @@ __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
     }
     __syncthreads();                                   // nrec, recb, fac (raw)
     const int nr = nrec;
-    {   // LSE per head over the records: 16 threads per head
+    {   // LSE per head over the records: 16 threads per head, each thread's records
+        // (i = sub, sub + 16, ...) read once, up to four at a time
         const int h = threadIdx.x >> 4, sub = threadIdx.x & 15;
-        float M = -INFINITY;
-        for (int i = sub; i < nr; i += 16) M = fmaxf(M, p.part1[((size_t)(recb[i] + sg) * 16 + h) * REC]);
+        float M = -INFINITY, Ls = 0.f;
+        for (int i0 = sub; i0 < nr; i0 += 64) {
+            float rm[4], rl[4];
 #pragma unroll
-        for (int o = 8; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-        float Ls = 0.f;
-        for (int i = sub; i < nr; i += 16) {
-            const float* r = p.part1 + ((size_t)(recb[i] + sg) * 16 + h) * REC;
-            if (r[0] != -INFINITY) Ls += r[1] * exp2f(r[0] - M);
+            for (int k = 0; k < 4; ++k) {
+                const int i = i0 + 16 * k;
+                const float* r = p.part1 + ((size_t)(recb[i < nr ? i : 0] + sg) * 16 + h) * REC;
+                rm[k] = i < nr ? r[0] : -INFINITY;
+                rl[k] = i < nr ? r[1] : 0.f;
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                if (rm[k] == -INFINITY) continue;
+                const float Mn = fmaxf(M, rm[k]);
+                Ls = Ls * exp2f(M - Mn) + rl[k] * exp2f(rm[k] - Mn);      // M = -inf first: factor 0
+                M = Mn;
+            }
         }
 #pragma unroll
-        for (int o = 8; o >= 1; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
+        for (int o = 8; o >= 1; o >>= 1) {
+            const float Mo = __shfl_xor_sync(0xffffffffu, M, o), Lo = __shfl_xor_sync(0xffffffffu, Ls, o);
+            const float Mn = fmaxf(M, Mo);
+            Ls = (Mn == -INFINITY) ? 0.f : Ls * exp2f(M - Mn) + Lo * exp2f(Mo - Mn);
+            M = Mn;
+        }
         const float l2 = Ls > 0.f ? M + log2f(Ls) : -INFINITY;
         if (sub == 0) {
             lse2[h] = l2;
@@ -481,14 +542,20 @@ __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
     for (int e = threadIdx.x; e < 16 * (DV / 4); e += blockDim.x) {
         const int h = e / (DV / 4), c4 = (e % (DV / 4)) * 4;
         float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-        for (int i = 0; i < nr; ++i) {
-            const float4 v = *reinterpret_cast<const float4*>(p.part1 + ((size_t)(recb[i] + sg) * 16 + h) * REC + 4 + c4);
-            const float f = ifac[i * 16 + h];
-            a.x += v.x * f;
-            a.y += v.y * f;
-            a.z += v.z * f;
-            a.w += v.w * f;
+        for (int i0 = 0; i0 < nr; i0 += 8) {
+            float4 v[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                v[k] = i0 + k < nr ? *reinterpret_cast<const float4*>(p.part1 + ((size_t)(recb[i0 + k] + sg) * 16 + h) * REC + 4 + c4)
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const float f = i0 + k < nr ? ifac[(i0 + k) * 16 + h] : 0.f;
+                a.x += v[k].x * f;
+                a.y += v[k].y * f;
+                a.z += v[k].z * f;
+                a.w += v[k].w * f;
+            }
         }
         *reinterpret_cast<float4*>(p.ocmp + (sg * 16 + h) * DV + c4) = a;
     }
@@ -528,7 +595,7 @@ __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
         pg[j] = acc;
     }
     __syncthreads();
-    topn_row_cta<8>(pg, t, p.n, p.lp, p.fi, p.fl, p.sel_idx + sg * p.n, tsv, tsi);
+    topn_row_cta_radix<256>(pg, t, p.n, p.lp, p.fi, p.fl, p.sel_idx + sg * p.n, tsm);
 }
 
 // sorted union of the selected blocks (sel: n entries, -1 padded, ascending)
@@ -745,23 +812,36 @@ __global__ void __launch_bounds__(256) dec_final(const DecParams p) {
         const float gt0 = p.gates[row * 3], gt1 = p.gates[row * 3 + 1], gt2 = p.gates[row * 3 + 2];
         float M[2] = {-INFINITY, -INFINITY}, Ls[2] = {0.f, 0.f};
         float4 O[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
-#pragma unroll 4
-        for (int i = 0; i < nr; ++i) {
+        for (int i0 = 0; i0 < nr; i0 += 4) {
+            // every load of four records (both branches) in flight before the merge
+            float rm[4][2], rl[4][2];
+            float4 rv[4][2];
 #pragma unroll
-            for (int br = 0; br < 2; ++br) {
-                const float* r = p.part2 + ((((size_t)recb[i] + sg) * 2 + br) * 16 + h) * REC;
-                const float m = r[0], l = r[1];
-                const float4 v = *reinterpret_cast<const float4*>(r + 4 + c4);
-                if (m == -INFINITY) continue;
-                const float Mn = fmaxf(M[br], m);
-                const float a = exp2f(M[br] - Mn), f = exp2f(m - Mn);   // M = -inf first: a = 0
-                Ls[br] = Ls[br] * a + l * f;
-                O[br].x = O[br].x * a + v.x * f;
-                O[br].y = O[br].y * a + v.y * f;
-                O[br].z = O[br].z * a + v.z * f;
-                O[br].w = O[br].w * a + v.w * f;
-                M[br] = Mn;
-            }
+            for (int k = 0; k < 4; ++k)
+#pragma unroll
+                for (int br = 0; br < 2; ++br) {
+                    const bool in = i0 + k < nr;
+                    const float* r = p.part2 + ((((size_t)recb[in ? i0 + k : 0] + sg) * 2 + br) * 16 + h) * REC;
+                    rm[k][br] = in ? r[0] : -INFINITY;
+                    rl[k][br] = in ? r[1] : 0.f;
+                    rv[k][br] = in ? *reinterpret_cast<const float4*>(r + 4 + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+#pragma unroll
+                for (int br = 0; br < 2; ++br) {
+                    const float m = rm[k][br];
+                    if (m == -INFINITY) continue;
+                    const float4 v = rv[k][br];
+                    const float Mn = fmaxf(M[br], m);
+                    const float a = exp2f(M[br] - Mn), f = exp2f(m - Mn);   // M = -inf first: a = 0
+                    Ls[br] = Ls[br] * a + rl[k][br] * f;
+                    O[br].x = O[br].x * a + v.x * f;
+                    O[br].y = O[br].y * a + v.y * f;
+                    O[br].z = O[br].z * a + v.z * f;
+                    O[br].w = O[br].w * a + v.w * f;
+                    M[br] = Mn;
+                }
         }
         float inv[2];
 #pragma unroll
@@ -792,7 +872,7 @@ inline size_t decode_ws_bytes(int64_t S, int64_t Lmax, int64_t G, int64_t l, int
     size_t o = 0;
     o += a((size_t)S * G * NCH * 16 * 4);
     o += a((size_t)S * G * NCH * kDecNBS * 16 * 4);
-    o += a((size_t)(kDecMaxGrid + S * G) * 16 * (DV + 4) * 4);
+    o += a((size_t)(kDecMaxGrid * kDecW + S * G) * 16 * (DV + 4) * 4);
     o += a((size_t)S * G * 16 * DV * 4);
     o += a((size_t)S * G * 16 * 4);
     o += a((size_t)(kDecMaxGrid + S * G) * 2 * 16 * (DV + 4) * 4);

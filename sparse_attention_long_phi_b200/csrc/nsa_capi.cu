@@ -982,7 +982,7 @@ nsa_status_t decode_impl(const Shape& s, int S, const void* q, const void* kcach
     const size_t SG = (size_t)S * s.G;
     p.cmax = carve(SG * p.NCH * 16 * 4);
     p.bsum = carve(SG * p.NCH * kDecNBS * 16 * 4);
-    p.part1 = carve((kDecMaxGrid + SG) * 16 * (s.DV + 4) * 4);
+    p.part1 = carve((kDecMaxGrid * kDecW + SG) * 16 * (s.DV + 4) * 4);
     p.ocmp = carve(SG * 16 * s.DV * 4);
     p.lsecmp = carve(SG * 16 * 4);
     p.part2 = carve((kDecMaxGrid + SG) * 2 * 16 * (s.DV + 4) * 4);
@@ -1132,8 +1132,8 @@ nsa_status_t nsa_select_blocks(const nsa_config_t* cfg, const float* scores, int
         NSA_LAUNCH("topn_kernel", st, topn_kernel<32><<<grid, 256, 0, st>>>(scores, items, (int)s.T, (int)s.G,
                                                                (int)s.NS, (int)s.n, (int)s.lp,
                                                                (int)s.fi, (int)s.fl, sel_idx));
-    } else {
-        NSA_LAUNCH("topn_kernel", st, topn_kernel<kTopnPerLane><<<grid, 256, 0, st>>>(scores, items, (int)s.T, (int)s.G,
+    } else {   // longer rows: one CTA per row, radix select (the decode step's routine)
+        NSA_LAUNCH("topn_cta_kernel", st, topn_cta_kernel<<<(unsigned)items, 256, 0, st>>>(scores, (int)s.T, (int)s.G,
                                                                (int)s.NS, (int)s.n, (int)s.lp,
                                                                (int)s.fi, (int)s.fl, sel_idx));
     }

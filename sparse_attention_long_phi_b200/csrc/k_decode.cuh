@@ -57,10 +57,10 @@ struct DecParams {
     float* cmax;     // [S*G][NCH][16]            chunk max per head (log2 units)
     float* bsum;     // [S*G][NCH][kDecNBS][16]   per-head block sums of exp2(s - chunk max)
     float* part1;    // [grid1*8 + S*G][16][DV+4] per warp and pair: max, sum, -, -, unnormalised O
-    float* ocmp;     // [S*G][16][DV]             normalised compressed-branch output
     float* lsecmp;   // [S*G][16]                 log2 units
     float* part2;    // [grid3 + S*G][2][16][DV+4] per segment and branch (selected, window)
     int* cpre;       // [S+1] compressed chunks (x G) before sequence s
+    int* units;      // [S*G][NUV] selected U window blocks of a pair: block*2 + selected, -1 empty
     int Lmax, Cmax, NCH, NUV, NSmax;
     int grid1, grid3;
 };
@@ -70,7 +70,7 @@ __host__ __device__ constexpr int dec_stage_bytes() {      // one warp: 32 K row
     return 32 * ((DK * 2 + 16) + (DV * 2 + 16));
 }
 template <int DK, int DV>
-__host__ __device__ constexpr int dec_stream_smem() {      // staging (merge area aliased) + P tiles
+__host__ __device__ constexpr int dec_stream_smem() {      // staging + P tiles (block sums)
     return kDecW * dec_stage_bytes<DK, DV>() + kDecW * 16 * 33 * 4;
 }
 
@@ -101,72 +101,23 @@ __device__ __forceinline__ long long dec_range_start(int b, long long N, int gri
 __device__ __forceinline__ int dec_cta_of(long long x, long long N, int grid) {
     return (int)(((x + 1) * grid - 1) / N);
 }
-// record slots of items [X0, X1) (X1 > X0): CTAs with a non-empty range
-// among those holding them; returns the count, slots b + sg into out[]
-__device__ __forceinline__ int dec_record_ctas(long long X0, long long X1, long long N, int grid, int* out, int cap) {
+// Record slots of items [X0, X1) (X1 > X0): the ranges (warps) that are not
+// empty among those holding them, written to out[] (at most cap), found by one
+// warp (lane k tests candidate bf + k, 32 at a time); every lane returns the count
+__device__ __forceinline__ int dec_record_list_warp(long long X0, long long X1, long long N, int grid, int* out,
+                                                    int cap) {
+    const int lane = threadIdx.x & 31;
     const int bf = dec_cta_of(X0, N, grid), bl = dec_cta_of(X1 - 1, N, grid);
     int cnt = 0;
-    for (int b = bf; b <= bl && cnt < cap; ++b)
-        if (dec_range_start(b + 1, N, grid) > dec_range_start(b, N, grid)) out[cnt++] = b;
-    return cnt;
-}
-
-// Merge the 8 warps' online-softmax states (rows gr, gr+8 per lane) into one
-// record [16][DV+4] = (max, sum, -, -, O relative to max).  `mrg` is a
-// [8][16][DV] fp32 scratch; wm/wl [8][16].  Ends with a barrier.
-template <int DV>
-__device__ __forceinline__ void dec_merge_record(float m0, float m1, float l0, float l1, const float (&o)[DV / 8][4],
-                                                 float* mrg, float (*wm)[16], float (*wl)[16], float* rec) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gr = lane >> 2, tg = lane & 3;
-    if (tg == 0) {
-        wm[warp][gr] = m0;
-        wm[warp][gr + 8] = m1;
-        wl[warp][gr] = l0;
-        wl[warp][gr + 8] = l1;
+    for (int base = bf; base <= bl; base += 32) {
+        const int b = base + lane;
+        const bool use = b <= bl && dec_range_start(b + 1, N, grid) > dec_range_start(b, N, grid);
+        const unsigned m = __ballot_sync(0xffffffffu, use);
+        const int pos = cnt + __popc(m & ((1u << lane) - 1u));
+        if (use && pos < cap) out[pos] = b;
+        cnt += __popc(m);
     }
-    __syncthreads();
-    {
-        float M0 = -INFINITY, M1 = -INFINITY;
-#pragma unroll
-        for (int w2 = 0; w2 < kDecW; ++w2) {
-            M0 = fmaxf(M0, wm[w2][gr]);
-            M1 = fmaxf(M1, wm[w2][gr + 8]);
-        }
-        const float f0 = m0 == -INFINITY ? 0.f : exp2f(m0 - M0);
-        const float f1 = m1 == -INFINITY ? 0.f : exp2f(m1 - M1);
-#pragma unroll
-        for (int nt = 0; nt < DV / 8; ++nt) {
-            const int cc = nt * 8 + tg * 2;
-            *reinterpret_cast<float2*>(mrg + (warp * 16 + gr) * DV + cc) = make_float2(o[nt][0] * f0, o[nt][1] * f0);
-            *reinterpret_cast<float2*>(mrg + (warp * 16 + gr + 8) * DV + cc) = make_float2(o[nt][2] * f1, o[nt][3] * f1);
-        }
-    }
-    __syncthreads();
-    constexpr int REC = DV + 4;
-    for (int e = threadIdx.x; e < 16 * (DV / 4); e += blockDim.x) {
-        const int h = e / (DV / 4), c4 = (e % (DV / 4)) * 4;
-        float4 a = *reinterpret_cast<const float4*>(mrg + h * DV + c4);
-#pragma unroll
-        for (int w2 = 1; w2 < kDecW; ++w2) {       // fixed order: deterministic
-            const float4 b = *reinterpret_cast<const float4*>(mrg + (w2 * 16 + h) * DV + c4);
-            a.x += b.x;
-            a.y += b.y;
-            a.z += b.z;
-            a.w += b.w;
-        }
-        *reinterpret_cast<float4*>(rec + h * REC + 4 + c4) = a;
-    }
-    if (threadIdx.x < 16) {
-        const int h = threadIdx.x;
-        float M = -INFINITY;
-        for (int w2 = 0; w2 < kDecW; ++w2) M = fmaxf(M, wm[w2][h]);
-        float Ls = 0.f;
-        for (int w2 = 0; w2 < kDecW; ++w2)
-            if (wm[w2][h] != -INFINITY) Ls += wl[w2][h] * exp2f(wm[w2][h] - M);
-        rec[h * REC] = M;
-        rec[h * REC + 1] = Ls;
-    }
-    __syncthreads();
+    return min(cnt, cap);
 }
 
 // -------------------------------------------------------------- step 1
@@ -430,18 +381,77 @@ __global__ void __launch_bounds__(256, 1) dec_cmp_stream(const DecParams p) {
     }
 }
 
+// sorted union of the selected blocks (sel: n entries, -1 padded, ascending)
+// and the blocks overlapping the window; flag[i] = 1 when list[i] is selected
+__device__ __forceinline__ int dec_units(const DecParams& p, const int32_t* sel, int L, int* list, int* flag) {
+    const int wlo = max(0, L - p.w) / p.lp, whi = (L - 1) / p.lp;
+    int i = 0, j = wlo, cnt = 0, last = -1;
+    while (cnt < kDecMaxUnits) {
+        const int a = (i < p.n && sel[i] >= 0) ? sel[i] : 0x7fffffff;
+        const int b = j <= whi ? j : 0x7fffffff;
+        const int m = min(a, b);
+        if (m == 0x7fffffff) break;
+        const bool from_sel = m == a;
+        if (m == a) ++i;
+        if (m == b) ++j;
+        if (m != last) {
+            list[cnt] = m;
+            flag[cnt] = from_sel ? 1 : 0;
+            ++cnt;
+        } else if (from_sel) {
+            flag[cnt - 1] = 1;
+        }
+        last = m;
+    }
+    return cnt;
+}
+
+// dec_units by one warp, written as units[i] = block*2 + selected (-1 past the
+// end, NUV slots): lane i holds selected block i, lane k window block wlo + k;
+// a block's place is the number of list entries below it.
+// scratch: >= 32 + 2 * kDecMaxUnits ints of shared memory (the one-lane path).
+__device__ __forceinline__ void dec_units_warp(const DecParams& p, const int32_t* sel, int L, int* units,
+                                               int* scratch) {
+    const int lane = threadIdx.x & 31;
+    const int wlo = max(0, L - p.w) / p.lp, whi = (L - 1) / p.lp, nw = whi - wlo + 1;
+    if (nw > 32) {                                     // windows of more than 32 blocks: one lane
+        if (lane == 0) {
+            int* sb = scratch;
+            int* list = scratch + 32;
+            int* flag = scratch + 32 + kDecMaxUnits;
+            for (int i = 0; i < p.n; ++i) sb[i] = sel[i];
+            const int cnt = dec_units(p, sb, L, list, flag);
+            for (int i = 0; i < p.NUV; ++i) units[i] = i < cnt ? list[i] * 2 + flag[i] : -1;
+        }
+        return;
+    }
+    const int a = lane < p.n ? sel[lane] : -1;        // ascending, -1 padded
+    const bool va = a >= 0;
+    const bool inw = va && a >= wlo && a <= whi;
+    const bool out = va && !inw;
+    const unsigned mout = __ballot_sync(0xffffffffu, out);
+    const unsigned mbelow = __ballot_sync(0xffffffffu, out && a < wlo);
+    const unsigned selw = __reduce_or_sync(0xffffffffu, inw ? 1u << (a - wlo) : 0u);   // window blocks selected
+    const unsigned lt = (1u << lane) - 1u;
+    if (out) units[__popc(mout & lt) + (a > whi ? nw : 0)] = a * 2 + 1;
+    if (lane < nw) units[lane + __popc(mbelow)] = (wlo + lane) * 2 + ((selw >> lane) & 1u);
+    const int cnt = nw + __popc(mout);
+    for (int i = cnt + lane; i < p.NUV; i += 32) units[i] = -1;
+}
+
 // -------------------------------------------------------------- step 2
-// Every load that does not need the row LSE (records, chunk maxima, this
-// thread's block sums) is issued before the first barrier, so the kernel
-// waits about one memory round trip; the top-n runs on all 8 warps.
+// Every load that does not need the row LSE (chunk maxima, this thread's block
+// sums) is issued before the first barrier; the records give the LSE in one
+// round of loads (their O is merged by the final step); the top-n and the unit
+// list run on all warps.
 template <int DV>
 __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
     constexpr int REC = DV + 4;
-    extern __shared__ float csm[];                     // ifac [256][16], fac [NCH][16], pg [NSmax]
+    extern __shared__ float csm[];                     // fac [NCH][16], pg [NSmax]
     __shared__ float lse2[16];
     __shared__ int recb[kDecMaxChunks];
     __shared__ int nrec;
-    __shared__ int tsm[256 + 16 + 8 * 8 + 32];       // top-n scratch
+    __shared__ int tsm[2 * 8 * 32];                   // top-n scratch
     const int g = blockIdx.x, s = blockIdx.y;
     dep_launch();
     int L, C;
@@ -453,16 +463,15 @@ __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
     const int nch = (C + 31) / 32;
     const size_t sg = (size_t)s * p.G + g;
     dep_wait();                                        // the compressed stream's records
-    if (threadIdx.x == 0) {
+    if (threadIdx.x < 32) {
         int cnt = 0;
         if (nch > 0) {
             const long long X0 = (long long)p.cpre[s] + (long long)g * nch;
-            cnt = dec_record_ctas(X0, X0 + nch, p.cpre[p.S], p.grid1 * kDecW, recb, kDecMaxChunks);
+            cnt = dec_record_list_warp(X0, X0 + nch, p.cpre[p.S], p.grid1 * kDecW, recb, kDecMaxChunks);
         }
-        nrec = cnt;
+        if (threadIdx.x == 0) nrec = cnt;
     }
-    float* ifac = csm;
-    float* fac = csm + kDecMaxChunks * 16;
+    float* fac = csm;
     float* pg = fac + p.NCH * 16;
     // chunk maxima (log2 units) and this thread's block sums: independent of the LSE
     const float* cm = p.cmax + sg * p.NCH * 16;
@@ -527,37 +536,12 @@ __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
             lse2[h] = l2;
             p.lsecmp[sg * 16 + h] = l2;
         }
-        for (int i = sub; i < nr; i += 16) {
-            const float m = p.part1[((size_t)(recb[i] + sg) * 16 + h) * REC];
-            ifac[i * 16 + h] = (m != -INFINITY && l2 != -INFINITY) ? exp2f(m - l2) : 0.f;
-        }
     }
     __syncthreads();
     // per chunk and head: exp2(chunk max - LSE); heads past HG do not score
     for (int e = threadIdx.x; e < nch * 16; e += blockDim.x) {
         const int h = e & 15;
         fac[e] = (h < p.HG && lse2[h] != -INFINITY) ? exp2f(fac[e] - lse2[h]) : 0.f;
-    }
-    // o_cmp = sum over records of O exp2(m - LSE)
-    for (int e = threadIdx.x; e < 16 * (DV / 4); e += blockDim.x) {
-        const int h = e / (DV / 4), c4 = (e % (DV / 4)) * 4;
-        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int i0 = 0; i0 < nr; i0 += 8) {
-            float4 v[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                v[k] = i0 + k < nr ? *reinterpret_cast<const float4*>(p.part1 + ((size_t)(recb[i0 + k] + sg) * 16 + h) * REC + 4 + c4)
-                                   : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const float f = i0 + k < nr ? ifac[(i0 + k) * 16 + h] : 0.f;
-                a.x += v[k].x * f;
-                a.y += v[k].y * f;
-                a.z += v[k].z * f;
-                a.w += v[k].w * f;
-            }
-        }
-        *reinterpret_cast<float4*>(p.ocmp + (sg * 16 + h) * DV + c4) = a;
     }
     __syncthreads();
     auto dot16 = [&](const float4 (&v)[4], const float* f) {
@@ -595,50 +579,34 @@ __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
         pg[j] = acc;
     }
     __syncthreads();
-    topn_row_cta_radix<256>(pg, t, p.n, p.lp, p.fi, p.fl, p.sel_idx + sg * p.n, tsm);
-}
-
-// sorted union of the selected blocks (sel: n entries, -1 padded, ascending)
-// and the blocks overlapping the window; flag[i] = 1 when list[i] is selected
-__device__ __forceinline__ int dec_units(const DecParams& p, const int32_t* sel, int L, int* list, int* flag) {
-    const int wlo = max(0, L - p.w) / p.lp, whi = (L - 1) / p.lp;
-    int i = 0, j = wlo, cnt = 0, last = -1;
-    while (cnt < kDecMaxUnits) {
-        const int a = (i < p.n && sel[i] >= 0) ? sel[i] : 0x7fffffff;
-        const int b = j <= whi ? j : 0x7fffffff;
-        const int m = min(a, b);
-        if (m == 0x7fffffff) break;
-        const bool from_sel = m == a;
-        if (m == a) ++i;
-        if (m == b) ++j;
-        if (m != last) {
-            list[cnt] = m;
-            flag[cnt] = from_sel ? 1 : 0;
-            ++cnt;
-        } else if (from_sel) {
-            flag[cnt - 1] = 1;
-        }
-        last = m;
-    }
-    return cnt;
+    topn_row_cta_redux<256>(pg, t, p.n, p.lp, p.fi, p.fl, p.sel_idx + sg * p.n, tsm);
+    // the pair's units for the selected/window stream: the sorted union of the
+    // selected blocks and the window's blocks, each flagged when selected
+    __syncthreads();                                   // the selection row is written
+    if (threadIdx.x < 32) dec_units_warp(p, p.sel_idx + sg * p.n, L, p.units + sg * p.NUV, tsm);
 }
 
 // -------------------------------------------------------------- step 3
 template <int DK, int DV>
+__host__ __device__ constexpr int dec_slcwin_smem() {        // staging + one Q tile per warp
+    return kDecW * dec_stage_bytes<DK, DV>() + kDecW * 16 * (DK * 2 + 16);
+}
+
+// Each warp owns a contiguous, equal range of the unit slots (NUV per pair, the
+// combine's sorted union of selected and window blocks, -1 when empty); per pair
+// it loads its own copy of Q and streams the chunks of the pair's units in its
+// range, then writes one record per branch at slot (warp index + seq*G + group),
+// unique because consecutive pairs share at most one warp.
+template <int DK, int DV>
 __global__ void __launch_bounds__(256, 1) dec_slcwin_stream(const DecParams p) {
     constexpr int KP = DK * 2 + 16, STG = dec_stage_bytes<DK, DV>();
     extern __shared__ __align__(16) uint8_t dsm[];
-    float* mrg = reinterpret_cast<float*>(dsm);
-    uint8_t* qs = dsm + kDecW * STG;                      // [16][DK] Q tile, pitch DK*2+16
-    static_assert(16 * (DK * 2 + 16) <= kDecW * 16 * 33 * 4, "Q tile");
-    __shared__ float wm[kDecW][16], wl[kDecW][16];
-    __shared__ int ulist[kDecMaxUnits], uflag[kDecMaxUnits];
-    __shared__ int selbuf[32];
-    __shared__ int nunits;
     __shared__ uint64_t kbar[kDecW], vbar[kDecW];
+    __shared__ int ulw[kDecW][33];                    // per warp: a batch's non-empty units, their count
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tg = lane & 3;
     uint8_t* ks = dsm + warp * STG;
     uint8_t* vs = ks + 32 * KP;
+    uint8_t* qs = dsm + kDecW * STG + warp * 16 * KP;   // this warp's [16][DK] Q tile
     if (threadIdx.x < kDecW) {
         mbar_init(&kbar[threadIdx.x], 1);
         mbar_init(&vbar[threadIdx.x], 1);
@@ -646,14 +614,15 @@ __global__ void __launch_bounds__(256, 1) dec_slcwin_stream(const DecParams p) {
     fence_mbar_init();
     __syncthreads();
     dep_launch();
-    dep_wait();                                       // sel_idx and o_cmp of the combine
+    dep_wait();                                       // the combine's units and selections
     uint32_t kph = 0, vph = 0;
     const uint64_t pol = l2_evict_first();
-    const long long U = (long long)p.S * p.G * p.NUV;     // unit slots, NUV per (seq, group)
-    const int b = blockIdx.x;
-    long long x = dec_range_start(b, U, gridDim.x);
-    const long long x1 = dec_range_start(b + 1, U, gridDim.x);
+    const long long U = (long long)p.S * p.G * p.NUV;
+    const int gw = blockIdx.x * kDecW + warp, W = gridDim.x * kDecW;
+    long long x = dec_range_start(gw, U, W);
+    const long long x1 = dec_range_start(gw + 1, U, W);
     const float cl = p.scale_log2;
+    constexpr int REC = DV + 4;
     while (x < x1) {
         const size_t sg = (size_t)(x / p.NUV);
         const int ua = (int)(x % p.NUV);
@@ -661,30 +630,17 @@ __global__ void __launch_bounds__(256, 1) dec_slcwin_stream(const DecParams p) {
         const int s = (int)(sg / p.G), g = (int)(sg % p.G);
         int L, C;
         const bool ok = dec_seq_ok(p, s, L, C);
-        if (warp == 0) {                                  // unit list of (s, g)
-            if (ok && lane < p.n) selbuf[lane] = p.sel_idx[sg * p.n + lane];
-            __syncwarp();
-            if (lane == 0) nunits = ok ? dec_units(p, selbuf, L, ulist, uflag) : 0;
-        }
-        // Q of the group as a [16][DK] tile (rows >= HG zero), read with ldmatrix
-        for (int e = threadIdx.x; e < 16 * (DK / 8); e += blockDim.x) {
-            const int h = e / (DK / 8), c8 = e % (DK / 8);
-            int4 v = make_int4(0, 0, 0, 0);
-            if (h < p.HG) v = *reinterpret_cast<const int4*>(p.q + ((size_t)s * p.H + (size_t)g * p.HG + h) * DK + c8 * 8);
-            *reinterpret_cast<int4*>(qs + h * KP + c8 * 16) = v;
-        }
-        __syncthreads();
-        const int n = 2 * max(0, min(ua + nslot, nunits) - ua);   // chunks of 32 tokens
         const int64_t kvb = ok ? p.kv_off[s] : 0;
         const size_t kst = (size_t)p.G * DK, vst = (size_t)p.G * DV;
-        auto tok0 = [&](int i) { return ulist[ua + (i >> 1)] * p.lp + (i & 1) * 32; };
+
+        auto tok0 = [&](int u, int i) { return (u >> 1) * p.lp + (i & 1) * 32; };
         // rows past the cache are not read; the source stays inside the sequence
-        auto issue_k = [&](int i) {
-            const int u0 = tok0(i), nv = min(32, L - u0);
+        auto issue_k = [&](int u0) {
+            const int nv = min(32, L - u0);
             warp_bulk_rows<DK>(ks, p.kcache + ((size_t)(kvb + (nv > 0 ? u0 : 0)) * p.G + g) * DK, kst, nv, &kbar[warp], pol);
         };
-        auto issue_v = [&](int i) {
-            const int u0 = tok0(i), nv = min(32, L - u0);
+        auto issue_v = [&](int u0) {
+            const int nv = min(32, L - u0);
             warp_bulk_rows<DV>(vs, p.vcache + ((size_t)(kvb + (nv > 0 ? u0 : 0)) * p.G + g) * DV, vst, nv, &vbar[warp], pol);
         };
         float m[2][2], l[2][2];
@@ -699,27 +655,60 @@ __global__ void __launch_bounds__(256, 1) dec_slcwin_stream(const DecParams p) {
                 for (int e = 0; e < 4; ++e) o[br][nt][e] = 0.f;
         }
         const int wlo = L - p.w;
-        int i = warp;
-        if (i < n) {
-            issue_k(i);
-            issue_v(i);
+        bool live = true, qready = false;
+        // this range's units of the pair, 32 slots at a time (lane i: slot ua + b0 + i)
+        for (int b0 = 0; b0 < nslot && live; b0 += 32) {
+        {
+            const int myu = (ok && b0 + lane < nslot) ? p.units[sg * p.NUV + ua + b0 + lane] : -1;
+            const unsigned umask = __ballot_sync(0xffffffffu, myu >= 0);
+            if (myu >= 0) ulw[warp][__popc(umask & ((1u << lane) - 1u))] = myu;
+            if (lane == 0) ulw[warp][32] = __popc(umask);
         }
-        for (; i < n; i += kDecW) {
-            const bool more = i + kDecW < n;
-            const int u0 = tok0(i);
-            const bool insel = uflag[ua + (i >> 1)] != 0;
+        __syncwarp();
+        const int n = 2 * ulw[warp][32];                   // chunks of 32 tokens
+        // unit of chunk i: the (i/2)-th non-empty slot of the batch
+        auto unit_of = [&](int i) { return ulw[warp][i >> 1]; };
+        int ucur = n > 0 ? unit_of(0) : 0;
+        if (n > 0) {
+            issue_k(tok0(ucur, 0));
+            issue_v(tok0(ucur, 0));
+            if (!qready) {
+                // Q of the group as a [16][DK] tile (rows >= HG zero), read with ldmatrix;
+                // loaded while the first rows are in flight
+                for (int e = lane; e < 16 * (DK / 8); e += 32) {
+                    const int h = e / (DK / 8), c8 = e % (DK / 8);
+                    int4 v = make_int4(0, 0, 0, 0);
+                    if (h < p.HG)
+                        v = *reinterpret_cast<const int4*>(p.q + ((size_t)s * p.H + (size_t)g * p.HG + h) * DK + c8 * 8);
+                    *reinterpret_cast<int4*>(qs + h * KP + c8 * 16) = v;
+                }
+                __syncwarp();
+                qready = true;
+            }
+        }
+        for (int i = 0; i < n; ++i) {
+            const bool more = i + 1 < n;
+            const int unxt = more ? ((i & 1) ? unit_of(i + 1) : ucur) : ucur;
+            const int u0 = tok0(ucur, i);
+            const bool insel = (ucur & 1) != 0;
             const int nval = min(32, L - u0);
             // warp-uniform: does the chunk hold keys of each branch?
             const bool has_sel = insel && nval > 0;
             const bool has_win = nval > 0 && u0 + nval - 1 >= wlo;
-            if (!mbar_wait(&kbar[warp], kph, 0x403)) break;   // K of chunk i
+            if (!mbar_wait(&kbar[warp], kph, 0x403)) {   // K of chunk i
+                live = false;
+                break;
+            }
             kph ^= 1;
             __syncwarp();
             float sf[4][4];
             if (has_sel || has_win) warp_logits_sa<DK>(smem_u32(qs), smem_u32(ks), sf);
             __syncwarp();
-            if (more) issue_k(i + kDecW);
-            if (!mbar_wait(&vbar[warp], vph, 0x404)) break;   // V of chunk i
+            if (more) issue_k(tok0(unxt, i + 1));
+            if (!mbar_wait(&vbar[warp], vph, 0x404)) {   // V of chunk i
+                live = false;
+                break;
+            }
             vph ^= 1;
             __syncwarp();
 #pragma unroll
@@ -776,86 +765,175 @@ __global__ void __launch_bounds__(256, 1) dec_slcwin_stream(const DecParams p) {
                 warp_pv<DV>(pf4, smem_u32(vs), o[br]);
             }
             __syncwarp();
-            if (more) issue_v(i + kDecW);
+            if (more) issue_v(tok0(unxt, i + 1));
+            ucur = unxt;
         }
-        float* rec = p.part2 + ((size_t)b + sg) * 2 * 16 * (DV + 4);
-        dec_merge_record<DV>(m[0][0], m[0][1], l[0][0], l[0][1], o[0], mrg, wm, wl, rec);
-        dec_merge_record<DV>(m[1][0], m[1][1], l[1][0], l[1][1], o[1], mrg, wm, wl, rec + 16 * (DV + 4));
+        }
+        if (!live) break;
+        // this warp's records of the pair, one per branch: (max, sum, -, -, O relative to max)
+        float* rec = p.part2 + ((size_t)gw + sg) * 2 * 16 * REC;
+        const int gr = lane >> 2;
+#pragma unroll
+        for (int br = 0; br < 2; ++br) {
+            float* rb = rec + br * 16 * REC;
+            if (tg == 0) {
+                rb[gr * REC] = m[br][0];
+                rb[gr * REC + 1] = l[br][0];
+                rb[(gr + 8) * REC] = m[br][1];
+                rb[(gr + 8) * REC + 1] = l[br][1];
+            }
+#pragma unroll
+            for (int nt = 0; nt < DV / 8; ++nt) {
+                const int cc = 4 + nt * 8 + tg * 2;
+                *reinterpret_cast<float2*>(rb + gr * REC + cc) = make_float2(o[br][nt][0], o[br][nt][1]);
+                *reinterpret_cast<float2*>(rb + (gr + 8) * REC + cc) = make_float2(o[br][nt][2], o[br][nt][3]);
+            }
+        }
+        __syncwarp();                                  // the Q tile is reloaded for the next pair
         x += nslot;
     }
 }
 
 // -------------------------------------------------------------- step 4
-// One thread per output float4: it merges its head's records of both
-// branches itself (one pass, running max), so the only barrier is the one
-// that publishes the record list.
+// Per (seq, group): the records of all three branches merged in two rounds of
+// loads.  Round 1: each selected/window record's (max, sum) per head, 8 threads
+// per (branch, head), gives the branch's max M, sum L and the weight
+// exp2(m - M) / L of every record; each compressed record's max gives its
+// weight exp2(m - LSE) under the combine's LSE.  Round 2: one thread per output
+// float4 sums the records' O weighted, all loads of a batch in flight; then
+// out = sum_c g_c o_c and the LSEs.
 template <int DV>
 __global__ void __launch_bounds__(256) dec_final(const DecParams p) {
     constexpr int REC = DV + 4;
     __shared__ int recb[kDecMaxUnits];
-    __shared__ int nrec;
+    __shared__ int recc[kDecMaxChunks];
+    __shared__ int nrec, nrecc;
+    __shared__ float wgt[kDecMaxUnits][2][16];      // record weight per branch and head
+    __shared__ float wgc[kDecMaxChunks][16];        // compressed record weight per head
+    __shared__ float lsb[2][16];                    // branch LSE (log2 units)
     const int g = blockIdx.x, s = blockIdx.y;
     int L, C;
     if (!dec_seq_ok(p, s, L, C)) return;
     const size_t sg = (size_t)s * p.G + g;
+    const int nch = (C + 31) / 32;
     dep_wait();                                       // the selected/window records
-    if (threadIdx.x == 0) {
+    if (threadIdx.x < 32) {
         const long long X0 = (long long)sg * p.NUV;
-        nrec = dec_record_ctas(X0, X0 + p.NUV, (long long)p.S * p.G * p.NUV, p.grid3, recb, kDecMaxUnits);
+        const int cnt = dec_record_list_warp(X0, X0 + p.NUV, (long long)p.S * p.G * p.NUV, p.grid3 * kDecW, recb,
+                                             kDecMaxUnits);
+        if (threadIdx.x == 0) nrec = cnt;
+    } else if (threadIdx.x < 64) {
+        int cnt = 0;
+        if (nch > 0) {
+            const long long X0 = (long long)p.cpre[s] + (long long)g * nch;
+            cnt = dec_record_list_warp(X0, X0 + nch, p.cpre[p.S], p.grid1 * kDecW, recc, kDecMaxChunks);
+        }
+        if (threadIdx.x == 32) nrecc = cnt;
     }
     __syncthreads();
-    const int nr = nrec;
+    const int nr = nrec, nrc = nrecc;
+    {   // compressed records: weight exp2(m - LSE) per head, 16 threads per head
+        const int h = threadIdx.x >> 4, sub = threadIdx.x & 15;
+        const float lc = p.lsecmp[sg * 16 + h];
+        for (int i0 = sub; i0 < nrc; i0 += 64) {
+            float rm[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int i = i0 + 16 * k;
+                rm[k] = i < nrc ? p.part1[((size_t)(recc[i] + sg) * 16 + h) * REC] : -INFINITY;
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int i = i0 + 16 * k;
+                if (i < nrc) wgc[i][h] = (rm[k] != -INFINITY && lc != -INFINITY) ? exp2f(rm[k] - lc) : 0.f;
+            }
+        }
+    }
+    {
+        const int bh = threadIdx.x >> 3, sub = threadIdx.x & 7;   // 32 (branch, head) x 8 threads
+        const int br = bh >> 4, h = bh & 15;
+        constexpr int PR = (kDecMaxUnits + 7) / 8;                 // records per thread
+        float rm[PR], rl[PR];
+#pragma unroll
+        for (int k = 0; k < PR; ++k) {
+            const int i = sub + 8 * k;
+            const float* r = p.part2 + ((((size_t)recb[i < nr ? i : 0] + sg) * 2 + br) * 16 + h) * REC;
+            rm[k] = i < nr ? r[0] : -INFINITY;
+            rl[k] = i < nr ? r[1] : 0.f;
+        }
+        float M = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < PR; ++k) M = fmaxf(M, rm[k]);
+#pragma unroll
+        for (int o = 4; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float Ls = 0.f;
+#pragma unroll
+        for (int k = 0; k < PR; ++k)
+            if (rm[k] != -INFINITY) Ls += rl[k] * exp2f(rm[k] - M);
+#pragma unroll
+        for (int o = 4; o >= 1; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
+        const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+#pragma unroll
+        for (int k = 0; k < PR; ++k) {
+            const int i = sub + 8 * k;
+            if (i < nr) wgt[i][br][h] = rm[k] == -INFINITY ? 0.f : exp2f(rm[k] - M) * inv;
+        }
+        if (sub == 0) lsb[br][h] = Ls > 0.f ? M + log2f(Ls) : -INFINITY;
+    }
+    __syncthreads();
     for (int e = threadIdx.x; e < p.HG * (DV / 4); e += blockDim.x) {
         const int h = e / (DV / 4), c4 = (e % (DV / 4)) * 4;
         const size_t row = (size_t)s * p.H + g * p.HG + h;
-        const float4 oc = *reinterpret_cast<const float4*>(p.ocmp + (sg * 16 + h) * DV + c4);
         const float gt0 = p.gates[row * 3], gt1 = p.gates[row * 3 + 1], gt2 = p.gates[row * 3 + 2];
-        float M[2] = {-INFINITY, -INFINITY}, Ls[2] = {0.f, 0.f};
+        float4 oc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i0 = 0; i0 < nrc; i0 += 8) {
+            float4 v[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                v[k] = i0 + k < nrc ? *reinterpret_cast<const float4*>(p.part1 + ((size_t)(recc[i0 + k] + sg) * 16 + h) * REC + 4 + c4)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const float w = i0 + k < nrc ? wgc[i0 + k][h] : 0.f;
+                oc.x += v[k].x * w;
+                oc.y += v[k].y * w;
+                oc.z += v[k].z * w;
+                oc.w += v[k].w * w;
+            }
+        }
         float4 O[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
-        for (int i0 = 0; i0 < nr; i0 += 4) {
-            // every load of four records (both branches) in flight before the merge
-            float rm[4][2], rl[4][2];
-            float4 rv[4][2];
+        for (int i0 = 0; i0 < nr; i0 += 8) {
+            float4 v[8][2];
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
+            for (int k = 0; k < 8; ++k)
 #pragma unroll
-                for (int br = 0; br < 2; ++br) {
-                    const bool in = i0 + k < nr;
-                    const float* r = p.part2 + ((((size_t)recb[in ? i0 + k : 0] + sg) * 2 + br) * 16 + h) * REC;
-                    rm[k][br] = in ? r[0] : -INFINITY;
-                    rl[k][br] = in ? r[1] : 0.f;
-                    rv[k][br] = in ? *reinterpret_cast<const float4*>(r + 4 + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
+                for (int br = 0; br < 2; ++br)
+                    v[k][br] = i0 + k < nr ? *reinterpret_cast<const float4*>(
+                                                 p.part2 + ((((size_t)recb[i0 + k] + sg) * 2 + br) * 16 + h) * REC + 4 + c4)
+                                           : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
+            for (int k = 0; k < 8; ++k)
 #pragma unroll
                 for (int br = 0; br < 2; ++br) {
-                    const float m = rm[k][br];
-                    if (m == -INFINITY) continue;
-                    const float4 v = rv[k][br];
-                    const float Mn = fmaxf(M[br], m);
-                    const float a = exp2f(M[br] - Mn), f = exp2f(m - Mn);   // M = -inf first: a = 0
-                    Ls[br] = Ls[br] * a + rl[k][br] * f;
-                    O[br].x = O[br].x * a + v.x * f;
-                    O[br].y = O[br].y * a + v.y * f;
-                    O[br].z = O[br].z * a + v.z * f;
-                    O[br].w = O[br].w * a + v.w * f;
-                    M[br] = Mn;
+                    const float w = i0 + k < nr ? wgt[i0 + k][br][h] : 0.f;
+                    O[br].x += v[k][br].x * w;
+                    O[br].y += v[k][br].y * w;
+                    O[br].z += v[k][br].z * w;
+                    O[br].w += v[k][br].w * w;
                 }
         }
-        float inv[2];
-#pragma unroll
-        for (int br = 0; br < 2; ++br) inv[br] = Ls[br] > 0.f ? 1.f / Ls[br] : 0.f;
         float4 r;
-        r.x = gt0 * oc.x + gt1 * O[0].x * inv[0] + gt2 * O[1].x * inv[1];
-        r.y = gt0 * oc.y + gt1 * O[0].y * inv[0] + gt2 * O[1].y * inv[1];
-        r.z = gt0 * oc.z + gt1 * O[0].z * inv[0] + gt2 * O[1].z * inv[1];
-        r.w = gt0 * oc.w + gt1 * O[0].w * inv[0] + gt2 * O[1].w * inv[1];
+        r.x = gt0 * oc.x + gt1 * O[0].x + gt2 * O[1].x;
+        r.y = gt0 * oc.y + gt1 * O[0].y + gt2 * O[1].y;
+        r.z = gt0 * oc.z + gt1 * O[0].z + gt2 * O[1].z;
+        r.w = gt0 * oc.w + gt1 * O[0].w + gt2 * O[1].w;
         *reinterpret_cast<float4*>(p.out + row * DV + c4) = r;
         if (c4 == 0 && p.lse) {
 #pragma unroll
-            for (int br = 0; br < 2; ++br)
-                p.lse[row * 3 + 1 + br] = Ls[br] > 0.f ? (M[br] + log2f(Ls[br])) * kLn2 : -INFINITY;
+            for (int br = 0; br < 2; ++br) {
+                const float lb = lsb[br][h];
+                p.lse[row * 3 + 1 + br] = lb == -INFINITY ? -INFINITY : lb * kLn2;
+            }
             const float lc = p.lsecmp[sg * 16 + h];
             p.lse[row * 3] = lc == -INFINITY ? -INFINITY : lc * kLn2;
         }
@@ -873,11 +951,10 @@ inline size_t decode_ws_bytes(int64_t S, int64_t Lmax, int64_t G, int64_t l, int
     o += a((size_t)S * G * NCH * 16 * 4);
     o += a((size_t)S * G * NCH * kDecNBS * 16 * 4);
     o += a((size_t)(kDecMaxGrid * kDecW + S * G) * 16 * (DV + 4) * 4);
-    o += a((size_t)S * G * 16 * DV * 4);
     o += a((size_t)S * G * 16 * 4);
-    o += a((size_t)(kDecMaxGrid + S * G) * 2 * 16 * (DV + 4) * 4);
+    o += a((size_t)(kDecMaxGrid * kDecW + S * G) * 2 * 16 * (DV + 4) * 4);
     o += a((size_t)(S + 1) * 4);
-    (void)NUV;
+    o += a((size_t)S * G * NUV * 4);
     return o;
 }
 

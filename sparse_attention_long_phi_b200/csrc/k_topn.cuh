@@ -272,22 +272,22 @@ __device__ __forceinline__ void topn_row_cta(const float* row, int t, int n, int
     }
 }
 
-// The same selection by a whole CTA of NT threads through a radix select: for
-// scores >= 0 the fp32 bit pattern orders like the value (-0 counts as +0), so
-// four rounds of 8-bit histograms over the candidates still in the running find
-// the key of the R-th largest score; every candidate above it is selected, and
-// among those equal to it the lowest indices, counted in index order (the same
-// set the iterative maximum with ties to the lower index picks).  Negative and
-// NaN scores are never selected.  Candidates lo .. hi <= lo + PL*NT - 1.
-// sm: >= 256 + 16 + PL*NT/32 + 32 ints of shared memory.
+// The same selection by a whole CTA of NT threads, for rows of up to 2048
+// candidates.  For scores >= 0 the fp32 bit pattern orders like the value (-0
+// counts as +0); a candidate's key is that pattern + 1, and 0 marks a score
+// that is never selected (negative, NaN, or already taken).  Each warp takes
+// the top R of its candidates (j = lo + thread + NT*k) one at a time: the
+// warp-wide maximum key and, among the candidates holding it, the lowest block
+// index are single reductions (redux.sync); warp 0 then takes the top R of the
+// warps' lists the same way.  Ties therefore go to the lower block index, the
+// rule of the iterative maximum above.
+// sm: >= NT/32 * 32 * 2 + 2 ints of shared memory.
 template <int NT>
-__device__ __forceinline__ void topn_row_cta_radix(const float* row, int t, int n, int lp, int fi, int fl,
+__device__ __forceinline__ void topn_row_cta_redux(const float* row, int t, int n, int lp, int fi, int fl,
                                                    int32_t* out, int* sm) {
     constexpr int NW = NT / 32, PL = (32 * kTopnPerLane + NT - 1) / NT;
-    int* hist = sm;                     // [256]
-    int* misc = sm + 256;               // prefix, need, selected count, valid count
-    int* wcnt = sm + 272;               // [PL][NW] equal-to-threshold counts per warp
-    int* sel = sm + 272 + PL * NW;      // [32] selected blocks, in no order
+    unsigned* wkey = reinterpret_cast<unsigned*>(sm);   // [NW][32] each warp's picks (key)
+    int* widx = sm + NW * 32;                           // [NW][32]                (block)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int bt = t / lp;
     const int ncand = bt + 1;
@@ -297,97 +297,69 @@ __device__ __forceinline__ void topn_row_cta_radix(const float* row, int t, int 
     }
     const int lo = fi, hi = bt - fl;
     const int R = n - fi - fl;
-    uint32_t key[PL];
-    bool val[PL];
-    int nv = 0;
+    unsigned key[PL];
 #pragma unroll
     for (int k = 0; k < PL; ++k) {
         const int j = lo + tid + NT * k;
         const float v = j <= hi ? row[j] : -1.f;
-        val[k] = v >= 0.f;                                   // false for NaN
-        key[k] = val[k] ? (__float_as_uint(v) & 0x7fffffffu) : 0u;
-        nv += val[k] ? 1 : 0;
+        key[k] = v >= 0.f ? (__float_as_uint(v) & 0x7fffffffu) + 1u : 0u;   // 0 for negative or NaN
     }
-    if (tid < 256) hist[tid] = 0;
-    if (tid == 0) {
-        misc[0] = 0;
-        misc[1] = R;
-        misc[2] = 0;
-        misc[3] = 0;
-    }
-    __syncthreads();
-    if (nv) atomicAdd(&misc[3], nv);
-    __syncthreads();
-    const bool none = R <= 0;                                // only forced blocks
-    const bool take_all = !none && misc[3] <= R;
-    uint32_t prefix = 0, mask = 0;
-    int need = R;
-    if (!none && !take_all) {
-#pragma unroll 1
-        for (int shift = 24; shift >= 0; shift -= 8) {
+    // the warp's top R, best first
+    for (int it = 0; it < R; ++it) {
+        unsigned lm = 0;
+#pragma unroll
+        for (int k = 0; k < PL; ++k) lm = max(lm, key[k]);
+        const unsigned M = __reduce_max_sync(0xffffffffu, lm);
+        unsigned jm = 0xffffffffu;
+        if (M != 0u) {
+#pragma unroll
+            for (int k = PL - 1; k >= 0; --k)
+                if (key[k] == M) jm = (unsigned)(lo + tid + NT * k);
+        }
+        const unsigned J = __reduce_min_sync(0xffffffffu, jm);
+        if (M != 0u && jm == J) {
 #pragma unroll
             for (int k = 0; k < PL; ++k)
-                if (val[k] && (key[k] & mask) == prefix) atomicAdd(&hist[(key[k] >> shift) & 255u], 1);
-            __syncthreads();
-            if (warp == 0) {
-                // bins from the top: lane l holds bins 255 - 8l .. 248 - 8l
-                int c[8], tot = 0;
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    c[q] = hist[255 - 8 * lane - q];
-                    tot += c[q];
-                }
-                int incl = tot;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-                    if (lane >= o) incl += v;
-                }
-                const unsigned hit = __ballot_sync(0xffffffffu, incl >= need);
-                const int f = __ffs(hit) - 1;                    // the R-th largest lies in lane f's bins
-                if (lane == f) {
-                    int above = incl - tot, q = 0;
-                    while (q < 7 && above + c[q] < need) above += c[q++];
-                    misc[0] = (int)(prefix | ((uint32_t)(255 - 8 * lane - q) << shift));
-                    misc[1] = need - above;
-                }
-            }
-            __syncthreads();
-            prefix = (uint32_t)misc[0];
-            need = misc[1];
-            mask |= 255u << shift;
-            if (tid < 256) hist[tid] = 0;
-            __syncthreads();
+                if ((unsigned)(lo + tid + NT * k) == J) key[k] = 0u;
         }
-    }
-    // selected: everything above the threshold key, then the lowest-index ties
-    int tie_before = 0;                                      // ties in earlier index rounds k
-#pragma unroll
-    for (int k = 0; k < PL; ++k) {
-        const bool tie = !none && !take_all && val[k] && key[k] == prefix;
-        const unsigned bal = __ballot_sync(0xffffffffu, tie);
-        if (lane == 0) wcnt[k * NW + warp] = __popc(bal);
-    }
-    __syncthreads();
-#pragma unroll
-    for (int k = 0; k < PL; ++k) {
-        const bool tie = !none && !take_all && val[k] && key[k] == prefix;
-        const unsigned bal = __ballot_sync(0xffffffffu, tie);
-        int rank = tie_before + __popc(bal & ((1u << lane) - 1u));
-        int roundtot = 0;
-        for (int w = 0; w < NW; ++w) {
-            const int cw = wcnt[k * NW + w];
-            if (w < warp) rank += cw;
-            roundtot += cw;
+        if (lane == 0) {
+            wkey[warp * 32 + it] = M;
+            widx[warp * 32 + it] = M != 0u ? (int)J : 0x7fffffff;
         }
-        tie_before += roundtot;
-        const bool pick = !none && (take_all ? val[k] : (val[k] && (key[k] > prefix || (tie && rank < need))));
-        if (pick) sel[atomicAdd(&misc[2], 1)] = lo + tid + NT * k;
     }
     __syncthreads();
     if (warp == 0) {
-        const int ns = misc[2];
-        int mine = lane < ns ? sel[lane] : 0x7fffffff;
+        // the warps' lists: lane l holds entries l, l + 32, ... of the NW x R candidates
+        constexpr int Q = (NW * 32 + 31) / 32;
+        unsigned ck[Q];
+        int ci[Q];
+#pragma unroll
+        for (int q = 0; q < Q; ++q) {
+            const int e = lane + 32 * q, ww = e / 32, r = e % 32;
+            const bool ok = ww < NW && r < R;
+            ck[q] = ok ? wkey[e] : 0u;
+            ci[q] = ok ? widx[e] : 0x7fffffff;
+        }
+        int mine = 0x7fffffff;
+        for (int it = 0; it < R; ++it) {
+            unsigned lm = 0;
+#pragma unroll
+            for (int q = 0; q < Q; ++q) lm = max(lm, ck[q]);
+            const unsigned M = __reduce_max_sync(0xffffffffu, lm);
+            unsigned jm = 0xffffffffu;
+            if (M != 0u) {
+#pragma unroll
+                for (int q = 0; q < Q; ++q)
+                    if (ck[q] == M) jm = min(jm, (unsigned)ci[q]);
+            }
+            const unsigned J = __reduce_min_sync(0xffffffffu, jm);
+            if (M != 0u && jm == J) {
+#pragma unroll
+                for (int q = 0; q < Q; ++q)
+                    if ((unsigned)ci[q] == J) ck[q] = 0u;
+            }
+            if (lane == it) mine = M != 0u ? (int)J : 0x7fffffff;
+        }
         if (lane >= R && lane < R + fi) mine = lane - R;
         if (lane >= R + fi && lane < R + fi + fl) mine = bt - fl + 1 + (lane - R - fi);
         const int srt = warp_sort_asc(mine, lane);
@@ -399,10 +371,10 @@ __device__ __forceinline__ void topn_row_cta_radix(const float* row, int t, int 
 // blocks: scores [items, NSp], NSp <= 2048
 __global__ void __launch_bounds__(256) topn_cta_kernel(const float* __restrict__ pscore, int T, int G, int NSp,
                                                        int n, int lp, int fi, int fl, int32_t* __restrict__ idx) {
-    __shared__ int sm[256 + 16 + 8 * 8 + 32];
+    __shared__ int sm[2 * 8 * 32];
     const long long item = blockIdx.x;
     const int t = (int)((item / G) % T);
-    topn_row_cta_radix<256>(pscore + item * NSp, t, n, lp, fi, fl, idx + item * n, sm);
+    topn_row_cta_redux<256>(pscore + item * NSp, t, n, lp, fi, fl, idx + item * n, sm);
 }
 
 // one warp per (batch, token, group) item; scores [items, NSp]; NSp <= 32*PL

@@ -907,26 +907,26 @@ int device_sm_count() {
 
 template <int DK, int DV>
 nsa_status_t decode_launch(DecParams& p, const Shape& s, int S, cudaStream_t st) {
-    constexpr int smem = dec_stream_smem<DK, DV>();
+    constexpr int smem = dec_stream_smem<DK, DV>(), smem3 = dec_slcwin_smem<DK, DV>();
     const int nsm = device_sm_count();
     // persistent streaming kernels: as many CTAs as fit on the device at once
     int occ1 = 1, occ3 = 1;
     NSA_TRY(set_smem(dec_cmp_stream<DK, DV>, smem));
-    NSA_TRY(set_smem(dec_slcwin_stream<DK, DV>, smem));
+    NSA_TRY(set_smem(dec_slcwin_stream<DK, DV>, smem3));
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ1, dec_cmp_stream<DK, DV>, 256, smem) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ3, dec_slcwin_stream<DK, DV>, 256, smem) != cudaSuccess)
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ3, dec_slcwin_stream<DK, DV>, 256, smem3) != cudaSuccess)
         return NSA_ERR_CUDA;
     p.grid1 = std::min(kDecMaxGrid, nsm * std::max(1, occ1));
     p.grid3 = std::min(kDecMaxGrid, nsm * std::max(1, occ3));
     NSA_LAUNCH("dec_cmp_stream", st, dec_cmp_stream<DK, DV><<<(unsigned)p.grid1, 256, smem, st>>>(p));
     NSA_TRY(last_launch());
     // the three dependent kernels start while their predecessor drains
-    const int smem2 = (kDecMaxChunks * 16 + p.NCH * 16 + p.NSmax) * 4;
+    const int smem2 = (p.NCH * 16 + p.NSmax) * 4;
     NSA_TRY(set_smem(dec_cmp_combine<DV>, smem2));
     NSA_LAUNCH("dec_cmp_combine", st,
                NSA_TRY(launch_dependent(dec_cmp_combine<DV>, dim3((unsigned)s.G, (unsigned)S), dim3(256), smem2, st, p)));
     NSA_LAUNCH("dec_slcwin_stream", st,
-               NSA_TRY(launch_dependent(dec_slcwin_stream<DK, DV>, dim3((unsigned)p.grid3), dim3(256), smem, st, p)));
+               NSA_TRY(launch_dependent(dec_slcwin_stream<DK, DV>, dim3((unsigned)p.grid3), dim3(256), smem3, st, p)));
     NSA_LAUNCH("dec_final", st,
                NSA_TRY(launch_dependent(dec_final<DV>, dim3((unsigned)s.G, (unsigned)S), dim3(256), 0, st, p)));
     return last_launch();
@@ -983,10 +983,10 @@ nsa_status_t decode_impl(const Shape& s, int S, const void* q, const void* kcach
     p.cmax = carve(SG * p.NCH * 16 * 4);
     p.bsum = carve(SG * p.NCH * kDecNBS * 16 * 4);
     p.part1 = carve((kDecMaxGrid * kDecW + SG) * 16 * (s.DV + 4) * 4);
-    p.ocmp = carve(SG * 16 * s.DV * 4);
     p.lsecmp = carve(SG * 16 * 4);
-    p.part2 = carve((kDecMaxGrid + SG) * 2 * 16 * (s.DV + 4) * 4);
+    p.part2 = carve((kDecMaxGrid * kDecW + SG) * 2 * 16 * (s.DV + 4) * 4);
     p.cpre = reinterpret_cast<int*>(carve((size_t)(S + 1) * 4));
+    p.units = reinterpret_cast<int*>(carve(SG * p.NUV * 4));
     if (s.DK == 192) return decode_launch<192, 128>(p, s, S, st);
     return decode_launch<64, 64>(p, s, S, st);
 }
@@ -1132,7 +1132,7 @@ nsa_status_t nsa_select_blocks(const nsa_config_t* cfg, const float* scores, int
         NSA_LAUNCH("topn_kernel", st, topn_kernel<32><<<grid, 256, 0, st>>>(scores, items, (int)s.T, (int)s.G,
                                                                (int)s.NS, (int)s.n, (int)s.lp,
                                                                (int)s.fi, (int)s.fl, sel_idx));
-    } else {   // longer rows: one CTA per row, radix select (the decode step's routine)
+    } else {   // longer rows: one CTA per row (the decode step's selection routine)
         NSA_LAUNCH("topn_cta_kernel", st, topn_cta_kernel<<<(unsigned)items, 256, 0, st>>>(scores, (int)s.T, (int)s.G,
                                                                (int)s.NS, (int)s.n, (int)s.lp,
                                                                (int)s.fi, (int)s.fl, sel_idx));

@@ -76,7 +76,7 @@ def test_select_blocks_counts_and_forced_blocks(n, fi, fl):
 
 @pytest.mark.parametrize("kind", ["uniform", "ties", "one_lane", "zeros", "sparse", "tiny", "heavy"])
 def test_select_blocks_rows_beyond_1024_blocks(kind):
-    # up to 1563 candidate blocks per row: one CTA per row, the radix select the
+    # up to 1563 candidate blocks per row: one CTA per row, the selection routine the
     # decode step also uses (ties at the threshold, all-equal rows, subnormals)
     _check(dict(BASE, B=1, T=100000, G=1), kind, seed=5, nrows=1500)
 
@@ -96,7 +96,7 @@ def _select_valid_only(c, t, row):
 
 
 def test_select_blocks_long_rows_skip_negative_and_nan_scores():
-    # the radix select on rows of up to 1563 blocks with negative and NaN scores mixed
+    # the CTA selection on rows of up to 1563 blocks with negative and NaN scores mixed
     # in, and rows where fewer valid scores than slots remain
     nsa = _nsa()
     c = dict(BASE, B=1, T=100000, G=1)

@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(320, 1)
         if (lane == 0 && N > 0) {
             constexpr uint32_t id16 = idesc_bf16(128, 16);
             uint32_t cnt = 0;
-            int np_of[2] = {0, 0};
+            int np_even = 0, np_odd = 0;   // pair counts of the last even / odd token (registers)
             auto slot_wait = [&](uint32_t c) -> uint32_t {
                 const int sl = c % Cfg::NSLOT;
                 if (!wait_or_abort(&full[sl], (c / Cfg::NSLOT) & 1, 0x303, abort_flag)) return 0;
@@ -246,7 +246,8 @@ __global__ void __launch_bounds__(320, 1)
                 const int qs = i & 1, wg = i & 1;
                 if (!wait_or_abort(&qfull[qs], (i >> 1) & 1, 0x304, abort_flag)) return false;
                 const int np = npairs_ring[i & 3];
-                np_of[i & 1] = np;
+                if (i & 1) np_odd = np;
+                else np_even = np;
                 if (i >= 2 && !wait_or_abort(&sfree[wg], ((i - 2) >> 1) & 1, 0x305, abort_flag))
                     return false;
                 tc_fence_after();
@@ -274,7 +275,7 @@ __global__ void __launch_bounds__(320, 1)
                     return false;
                 tc_fence_after();
                 const uint32_t sP = smem_u32(smem + Cfg::kOffP + wg * Cfg::kPBytes);
-                const int np = np_of[i & 1];
+                const int np = (i & 1) ? np_odd : np_even;
                 for (int pp = 0; pp < np; ++pp) {
                     const uint32_t sV = slot_wait(cnt);
                     if (!sV) return false;

@@ -66,6 +66,39 @@ __global__ void bwd_branch_stats(const float* __restrict__ o, const __nv_bfloat1
     }
 }
 
+// All three branches at once from their saved outputs o_c [3][rows][DV] (the
+// training forward's): dO is read once per row instead of once per branch.
+__global__ void bwd_branch_stats3(const float* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
+                                  const float* __restrict__ gates, const float* __restrict__ lse_nat, long long rows,
+                                  int DV, float* dgates, float* dlt, float* lse2) {
+    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    float acc[3] = {0.f, 0.f, 0.f};
+    for (int c = lane * 4; c < DV; c += 128) {
+        const uint2 dv = *reinterpret_cast<const uint2*>(dout + row * DV + c);
+        const __nv_bfloat162 d01 = *reinterpret_cast<const __nv_bfloat162*>(&dv.x);
+        const __nv_bfloat162 d23 = *reinterpret_cast<const __nv_bfloat162*>(&dv.y);
+#pragma unroll
+        for (int br = 0; br < 3; ++br) {
+            const float4 ov = *reinterpret_cast<const float4*>(o + ((size_t)br * rows + row) * DV + c);
+            acc[br] += ov.x * __low2float(d01) + ov.y * __high2float(d01) + ov.z * __low2float(d23) +
+                       ov.w * __high2float(d23);
+        }
+    }
+#pragma unroll
+    for (int br = 0; br < 3; ++br)
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) acc[br] += __shfl_xor_sync(0xffffffffu, acc[br], m);
+    if (lane < 3) {
+        const int br = lane;
+        const float a = br == 0 ? acc[0] : br == 1 ? acc[1] : acc[2];
+        dgates[row * 3 + br] = a;
+        dlt[row * 3 + br] = gates[row * 3 + br] * a;
+        lse2[row * 3 + br] = lse_nat[row * 3 + br] * kLog2e;
+    }
+}
+
 __global__ void fill_f32(float* x, long long n, float v) {
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i < n) x[i] = v;

@@ -10,14 +10,20 @@
 // channels:
 //   S^T  = K_pair Q_t^T     M = 128 keys, N = 16 heads, K = d_k
 //   dP^T = V_pair dO_t^T    M = 128 keys, N = 16 heads, K = d_v
-//   softmax warps (thread = key): dS^T in bf16 to shared memory [16 heads][128 keys]
-//   dQ^T += K_pair^T dS^T   M = 128 channels (two products for d_k > 128, the
-//                           K tile read as a transposed operand), N = 16, K = 128
+//   softmax warps (thread = key): dS in bf16 to shared memory [16 heads][128 keys]
+//   dQ  += dS K_pair        M = 64 (the 16 heads in rows 0-15), N = d_k channels
+//                           (the K tile read as a transposed operand), K = 128 keys:
+//                           one product per 16 keys for all channels
+// An M = 64 accumulator keeps row r in TMEM lane 32 (r / 16) + r % 16, so the
+// heads sit in lanes 0-15 of the first lane quadrant, read by the first warp of
+// the warpgroup.  Rows 16-63 of the dS operand run past its 16-row tile into
+// the neighbouring shared memory; their products land in accumulator rows no
+// one reads.
 // A CTA walks a range of tokens of one group; two softmax warpgroups take
 // alternate tokens with their own TMEM buffers, so one token's softmax
 // overlaps the other's products.  K and V of a pair sit in separate rings:
 // V is needed only by dP^T and is released as soon as that product is done,
-// while K stays for the dQ^T products, so the K ring is the deeper one.
+// while K stays for the dQ products, so the K ring is the deeper one.
 // Warp 8 stages Q_t/dO_t and the K pairs, warp 10 the V pairs (each waits
 // only on its own ring), warp 9 issues the MMAs.
 #pragma once
@@ -29,9 +35,6 @@
 
 namespace nsa {
 
-// kind::f16 instruction descriptor with the A operand MN-major (transposed)
-__host__ __device__ constexpr uint32_t idesc_bf16_amn(int M, int N) { return idesc_bf16(M, N) | (1u << 15); }
-
 template <int DK, int DV>
 struct BqsCfg {
     static constexpr int NQB = DK / 64, NVB = DV / 64;
@@ -40,7 +43,7 @@ struct BqsCfg {
     static constexpr int kKPair = NQB * 16384;        // per box: [128 keys][64]
     static constexpr int kVPair = NVB * 16384;
     static constexpr int NK = 3;                      // K pair slots
-    static constexpr int kDS = 16 * 256;              // dS^T [16 heads][128 keys], two 64-key atoms
+    static constexpr int kDS = 16 * 256;              // dS [16 heads][128 keys], two 64-key atoms
     static constexpr int kOffQ = 0;                   // 2 token slots of Q_t then dO_t
     static constexpr int kOffO = kOffQ + 2 * kQ;
     static constexpr int kOffK = ((kOffO + 2 * kO + 1023) / 1024) * 1024;
@@ -53,7 +56,7 @@ struct BqsCfg {
     static constexpr int kSmem = kOffV + NV * kVPair + 1024;
     static_assert(NV >= 1 && kSmem <= kSmemMax, "shared memory");
     static constexpr int kThreads = 352;
-    // TMEM per warpgroup (128 columns apart): S^T buffers 0 / 16, dP^T 32 / 48, dQ^T 64 (+16)
+    // TMEM per warpgroup (256 columns apart): S^T buffers 0 / 16, dP^T 32 / 48, dQ 64 .. 64 + d_k
     static constexpr uint32_t kColDP = 32, kColDQ = 64;
 };
 
@@ -69,7 +72,7 @@ __global__ void __launch_bounds__(352, 1)
               const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
               const BqsParams P) {
     using Cfg = BqsCfg<DK, DV>;
-    constexpr int NH = DK > 128 ? 2 : 1;              // dQ^T products (channel halves of 128)
+    static_assert(Cfg::kColDQ + DK <= 256 && DK % 32 == 0, "dQ columns of a warpgroup");
     const BwdParams& p = P.bp;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -83,8 +86,8 @@ __global__ void __launch_bounds__(352, 1)
     uint64_t* vempty = bars + 16;   // [NV]
     uint64_t* sdfull = bars + 20;   // [2 wg][2 buf]  S^T and dP^T of a pair
     uint64_t* sdfree = bars + 24;   // [2][2]
-    uint64_t* dsfull = bars + 28;   // [2][2]         dS^T tile written
-    uint64_t* dsfree = bars + 32;   // [2][2]         dS^T tile read by the dQ^T products
+    uint64_t* dsfull = bars + 28;   // [2][2]         dS tile written
+    uint64_t* dsfree = bars + 32;   // [2][2]         dS tile read by the dQ products
     uint64_t* dqfull = bars + 36;   // [2]
     uint64_t* dqfree = bars + 38;   // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 40);
@@ -123,7 +126,7 @@ __global__ void __launch_bounds__(352, 1)
         fence_mbar_init();
     }
     if (warp == 9) {
-        tmem_alloc(tmem_slot, 256);
+        tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -216,12 +219,12 @@ __global__ void __launch_bounds__(352, 1)
     } else if (warp == 9) {
         // ----------------------------------------------------------- MMA
         // Per pair: dP^T first (its V slot returns to the producer as soon as it is
-        // done), S^T, then the dQ^T products of the previous pair, whose dS^T the
+        // done), S^T, then the dQ products of the previous pair, whose dS the
         // softmax has written meanwhile.  (Issuing the two streams by readiness
         // instead measured no faster: the N = 16 products keep the pipe busy.)
         if (lane == 0) {
             constexpr uint32_t id16 = idesc_bf16(128, 16);
-            constexpr uint32_t idT = idesc_bf16_amn(128, 16);
+            constexpr uint32_t idQ = idesc_bf16_bmn(64, DK);
             uint32_t ck = 0, cv = 0;      // K and V pair slots consumed
             // per (warpgroup, buffer) q: bit q of `par` = parity of its S/dP issues so far,
             // bit q of `used` = at least one issue
@@ -229,10 +232,10 @@ __global__ void __launch_bounds__(352, 1)
             bool ok = true;
             for (int i = 0; i < N && ok; ++i) {
                 const int qs = i & 1, wg = i & 1;
-                const uint32_t tw = tmem + wg * 128;
+                const uint32_t tw = tmem + wg * 256;
                 if (!(ok = wait_or_abort(&qfull[qs], (i >> 1) & 1, 0x603, abort_flag))) break;
                 const int np = npairs_ring[i & 7];
-                // this warpgroup's previous token has read its dQ^T
+                // this warpgroup's previous token has read its dQ
                 if (i >= 2 && !(ok = wait_or_abort(&dqfree[wg], ((i - 2) >> 1) & 1, 0x604, abort_flag))) break;
                 tc_fence_after();
                 const uint32_t sQ = smem_u32(smem + Cfg::kOffQ + qs * Cfg::kQ);
@@ -245,13 +248,9 @@ __global__ void __launch_bounds__(352, 1)
                     const uint32_t sK = smem_u32(smem + Cfg::kOffK + (c % Cfg::NK) * Cfg::kKPair);
                     const uint32_t sD = smem_u32(smem + Cfg::kOffDS + q * Cfg::kDS);
 #pragma unroll
-                    for (int hh = 0; hh < NH; ++hh)
-#pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)
-                            umma_bf16_ss(tw + Cfg::kColDQ + hh * 16,
-                                         sdesc_sw128_mn(sK + hh * 2 * 16384 + kk * 2048, 16384, 1024),
-                                         sdesc_sw128(sD + (kk / 4) * 2048 + (kk % 4) * 32), idT,
-                                         (pp > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_bf16_ss(tw + Cfg::kColDQ, sdesc_sw128(sD + (kk / 4) * 2048 + (kk % 4) * 32),
+                                     sdesc_sw128_mn(sK + kk * 2048, 16384, 1024), idQ, (pp > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&dsfree[q]);
                     umma_commit(&kempty[c % Cfg::NK]);
                     return true;
@@ -293,8 +292,8 @@ __global__ void __launch_bounds__(352, 1)
     } else {
         // --------------------------------- softmax / epilogue (2 warpgroups)
         const int wg = warp >> 2, wq = warp & 3;
-        const int kl = wq * 32 + lane;                 // key of a pair / channel of dQ^T
-        const uint32_t lanebase = tmem + wg * 128 + ((uint32_t)(wq * 32) << 16);
+        const int kl = wq * 32 + lane;                 // key of a pair
+        const uint32_t lanebase = tmem + wg * 256 + ((uint32_t)(wq * 32) << 16);
         const float c = p.scale_log2;
         bool ok = true;
         int it = 0;
@@ -330,7 +329,7 @@ __global__ void __launch_bounds__(352, 1)
                 if (lane == 0) mbar_arrive(&sdfree[q]);
                 const int un = 2 * pp + (kl >> 6);
                 const bool valid = un < nu && pick(r, un) * 64 + (kl & 63) <= t;
-                // the dQ^T products of this buffer's previous pair have read its dS^T tile
+                // the dQ products of this buffer's previous pair have read its dS tile
                 if ((used >> bf) & 1) {
                     w_ok = true;
                     if (lane == 0) w_ok = wait_or_abort(&dsfree[q], ((par >> bf) & 1) ^ 1, 0x609, abort_flag);
@@ -354,21 +353,25 @@ __global__ void __launch_bounds__(352, 1)
                 par ^= 1u << bf;
                 used |= 1u << bf;
             }
-            // epilogue: thread = channel kl (and 128 + kl), columns = heads
+            // epilogue: the first warp of the warpgroup, lane = head, columns = channels
             bool w_ok = true;
             if (lane == 0) w_ok = ok && wait_or_abort(&dqfull[wg], it & 1, 0x60A, abort_flag);
             if (!(ok = __shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0) != 0)) break;
             tc_fence_after();
+            if (wq == 0) {
+                float* dst = p.dq + (rowbase + (lane < HG ? lane : 0)) * DK;
+#pragma unroll 1
+                for (int c0 = 0; c0 < DK; c0 += 32) {
+                    uint32_t rq[32];
+                    tmem_ld32(lanebase + Cfg::kColDQ + c0, rq);
+                    tmem_wait_ld32(rq);
+                    if (np > 0 && lane < HG) {
 #pragma unroll
-            for (int hh = 0; hh < NH; ++hh) {
-                uint32_t rq[16];
-                tmem_ld16(lanebase + Cfg::kColDQ + hh * 16, rq);
-                tmem_wait_ld16(rq);
-                const int ch = hh * 128 + kl;
-                if (np > 0 && ch < DK) {
-#pragma unroll
-                    for (int h = 0; h < HG; ++h)
-                        red_add_v1(p.dq + (rowbase + h) * DK + ch, p.scale * __uint_as_float(rq[h]));
+                        for (int e = 0; e < 32; e += 4)
+                            red_add_v4(dst + c0 + e, p.scale * __uint_as_float(rq[e]),
+                                       p.scale * __uint_as_float(rq[e + 1]), p.scale * __uint_as_float(rq[e + 2]),
+                                       p.scale * __uint_as_float(rq[e + 3]));
+                    }
                 }
             }
             tc_fence_before();
@@ -380,7 +383,7 @@ __global__ void __launch_bounds__(352, 1)
     __syncthreads();
     if (warp == 9) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 512);
     }
 }
 

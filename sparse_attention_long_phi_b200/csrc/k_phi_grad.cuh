@@ -64,23 +64,33 @@ __global__ void __launch_bounds__(256) phi_dw_kernel(const float* __restrict__ d
             make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
 }
 
-// s[o] = sum_n dY[n, o]: grid D/32, block 256 (lane = column, warp w takes rows
-// n = w mod 8); the eight warps' partial sums are added in a fixed order.
-__global__ void __launch_bounds__(256) phi_colsum_kernel(const float* __restrict__ dY, int N, int D,
-                                                         float* __restrict__ s) {
-    __shared__ float part[8][32];
+// s[o] = sum_n dY[n, o] in two steps.  phi_colsum_kernel: grid (D/32, NB), block
+// 256 (lane = column); CTA y takes rows n = y, y + NB, ..., warp w of them every
+// eighth, and writes its sum to part[y][o] (the eight warps added in a fixed
+// order).  phi_colsum_fold: s[o] = part[0][o] + ... + part[NB-1][o] in order.
+__global__ void __launch_bounds__(256) phi_colsum_kernel(const float* __restrict__ dY, int N, int D, int NB,
+                                                         float* __restrict__ part) {
+    __shared__ float red[8][32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, o = blockIdx.x * 32 + lane;
     float acc = 0.f;
 #pragma unroll 8
-    for (int n = warp; n < N; n += 8) acc += dY[(size_t)n * D + o];
-    part[warp][lane] = acc;
+    for (int n = blockIdx.y + NB * warp; n < N; n += NB * 8) acc += dY[(size_t)n * D + o];
+    red[warp][lane] = acc;
     __syncthreads();
     if (warp == 0) {
         float t = 0.f;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) t += part[w][lane];
-        s[o] = t;
+        for (int w = 0; w < 8; ++w) t += red[w][lane];
+        part[(size_t)blockIdx.y * D + o] = t;
     }
+}
+
+__global__ void phi_colsum_fold(const float* __restrict__ part, int NB, int D, float* __restrict__ s) {
+    const int o = blockIdx.x * blockDim.x + threadIdx.x;
+    if (o >= D) return;
+    float t = 0.f;
+    for (int y = 0; y < NB; ++y) t += part[(size_t)y * D + o];
+    s[o] = t;
 }
 
 // dE[x] = sum_o W[o, x] s[o]: one thread per x of the l*D inputs.

@@ -715,12 +715,9 @@ nsa_status_t backward_impl(const Shape& s, const void* q, const void* k, const v
     // A training forward that saved o_c and the LSEs spares these passes.
     if (saved_o) {
         const long long rows = s.B * s.T * s.H;
-        for (int br = 0; br < 3; ++br) {
-            NSA_LAUNCH("bwd_branch_stats", st, bwd_branch_stats<<<(unsigned)ceil_div(rows, 8), 256, 0, st>>>(
-                saved_o + (size_t)br * rows * DV, reinterpret_cast<const __nv_bfloat16*>(dout), gates, saved_lse, br,
-                rows, DV, dgates, p.dlt, p.lse2));
-            NSA_TRY(last_launch());
-        }
+        NSA_LAUNCH("bwd_branch_stats", st, bwd_branch_stats3<<<(unsigned)ceil_div(rows, 8), 256, 0, st>>>(
+            saved_o, reinterpret_cast<const __nv_bfloat16*>(dout), gates, saved_lse, rows, DV, dgates, p.dlt, p.lse2));
+        NSA_TRY(last_launch());
     } else {
         constexpr int HG = DK == 192 ? 16 : 4;
         const long long rows = s.B * s.T * s.H;
@@ -1360,10 +1357,23 @@ nsa_status_t nsa_backward_phi_params(const nsa_config_t* cfg, const void* k, con
     float* colsum = reinterpret_cast<float*>(ws + L.off_fix);   // scratch: the fix-up list is done
     const int N = (int)(s.B * s.C * s.G);
     auto bf = [](const void* p) { return reinterpret_cast<const __nv_bfloat16*>(p); };
-    NSA_LAUNCH("phi_colsum_kernel", st, phi_colsum_kernel<<<(unsigned)(s.DK / 32), 256, 0, st>>>(dkc, N, (int)s.DK, colsum));
-    NSA_TRY(last_launch());
-    NSA_LAUNCH("phi_colsum_kernel", st, phi_colsum_kernel<<<(unsigned)(s.DV / 32), 256, 0, st>>>(dvc, N, (int)s.DV, colsum + s.DK));
-    NSA_TRY(last_launch());
+    // column sums in NB row slices (NB + 1 <= N when NB > 1, so the partial sums
+    // after the (DK + DV) sums fit in the fix-up scratch of N (DK + DV) floats)
+    const int NB = (int)std::min<int64_t>(32, std::max<int64_t>(1, N / 256));
+    {
+        float* pk = NB > 1 ? colsum + s.DK + s.DV : colsum;
+        float* pv = NB > 1 ? pk + (size_t)NB * s.DK : colsum + s.DK;
+        NSA_LAUNCH("phi_colsum_kernel", st, phi_colsum_kernel<<<dim3((unsigned)(s.DK / 32), (unsigned)NB), 256, 0, st>>>(dkc, N, (int)s.DK, NB, pk));
+        NSA_TRY(last_launch());
+        NSA_LAUNCH("phi_colsum_kernel", st, phi_colsum_kernel<<<dim3((unsigned)(s.DV / 32), (unsigned)NB), 256, 0, st>>>(dvc, N, (int)s.DV, NB, pv));
+        NSA_TRY(last_launch());
+        if (NB > 1) {
+            NSA_LAUNCH("phi_colsum_fold", st, phi_colsum_fold<<<(unsigned)ceil_div(s.DK, 64), 64, 0, st>>>(pk, NB, (int)s.DK, colsum));
+            NSA_TRY(last_launch());
+            NSA_LAUNCH("phi_colsum_fold", st, phi_colsum_fold<<<(unsigned)ceil_div(s.DV, 64), 64, 0, st>>>(pv, NB, (int)s.DV, colsum + s.DK));
+            NSA_TRY(last_launch());
+        }
+    }
     NSA_LAUNCH("phi_de_kernel", st, phi_de_kernel<<<(unsigned)ceil_div(KK, 256), 256, 0, st>>>(bf(phi->w_k), colsum, (int)s.DK, (int)KK, de_k));
     NSA_TRY(last_launch());
     NSA_LAUNCH("phi_de_kernel", st, phi_de_kernel<<<(unsigned)ceil_div(KV, 256), 256, 0, st>>>(bf(phi->w_v), colsum + s.DK, (int)s.DV, (int)KV, de_v));

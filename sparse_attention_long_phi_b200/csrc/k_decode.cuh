@@ -448,7 +448,6 @@ template <int DV>
 __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
     constexpr int REC = DV + 4;
     extern __shared__ float csm[];                     // fac [NCH][16], pg [NSmax]
-    __shared__ float lse2[16];
     __shared__ int recb[kDecMaxChunks];
     __shared__ int nrec;
     __shared__ int tsm[2 * 8 * 32];                   // top-n scratch
@@ -532,16 +531,10 @@ __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
             M = Mn;
         }
         const float l2 = Ls > 0.f ? M + log2f(Ls) : -INFINITY;
-        if (sub == 0) {
-            lse2[h] = l2;
-            p.lsecmp[sg * 16 + h] = l2;
-        }
-    }
-    __syncthreads();
-    // per chunk and head: exp2(chunk max - LSE); heads past HG do not score
-    for (int e = threadIdx.x; e < nch * 16; e += blockDim.x) {
-        const int h = e & 15;
-        fac[e] = (h < p.HG && lse2[h] != -INFINITY) ? exp2f(fac[e] - lse2[h]) : 0.f;
+        if (sub == 0) p.lsecmp[sg * 16 + h] = l2;
+        // per chunk of this head: exp2(chunk max - LSE); heads past HG do not score
+        for (int c = sub; c < nch; c += 16)
+            fac[c * 16 + h] = (h < p.HG && l2 != -INFINITY) ? exp2f(fac[c * 16 + h] - l2) : 0.f;
     }
     __syncthreads();
     auto dot16 = [&](const float4 (&v)[4], const float* f) {
@@ -795,143 +788,166 @@ __global__ void __launch_bounds__(256, 1) dec_slcwin_stream(const DecParams p) {
 }
 
 // -------------------------------------------------------------- step 4
-// Per (seq, group): the records of all three branches merged in two rounds of
-// loads.  Round 1: each selected/window record's (max, sum) per head, 8 threads
-// per (branch, head), gives the branch's max M, sum L and the weight
-// exp2(m - M) / L of every record; each compressed record's max gives its
-// weight exp2(m - LSE) under the combine's LSE.  Round 2: one thread per output
-// float4 sums the records' O weighted, all loads of a batch in flight; then
-// out = sum_c g_c o_c and the LSEs.
+// Per (seq, group) and eight heads (grid z): the records of all three
+// branches merged in two rounds of loads, each round issued at once.  Round 1:
+// warp w takes the compressed records of head w (weight exp2(m - LSE) under
+// the combine's LSE) and the selected/window records of two (branch, head)
+// groups, 16 lanes per group (the branch max M, sum L and the weight
+// exp2(m - M) / L of every record).  Round 2: one thread per output float4
+// (two for d_v = 64, each taking every other record) sums the weighted O of
+// the records, eight of each kind per batch of loads; then
+// out = sum_c g_c o_c and the LSEs.  256 CTAs of at most 128 registers per
+// thread fit the GPU in one wave.
+constexpr int kDecFinalHeads = 8;      // heads per dec_final CTA
+
 template <int DV>
-__global__ void __launch_bounds__(256) dec_final(const DecParams p) {
-    constexpr int REC = DV + 4;
+__global__ void __launch_bounds__(256, 2) dec_final(const DecParams p) {
+    constexpr int REC = DV + 4, HQ = kDecFinalHeads, NOUT = HQ * DV / 4, NHALF = 256 / NOUT;
+    static_assert(NHALF >= 1 && NHALF <= 2 && NHALF * NOUT == 256, "threads per output float4");
     __shared__ int recb[kDecMaxUnits];
     __shared__ int recc[kDecMaxChunks];
     __shared__ int nrec, nrecc;
-    __shared__ float wgt[kDecMaxUnits][2][16];      // record weight per branch and head
-    __shared__ float wgc[kDecMaxChunks][16];        // compressed record weight per head
-    __shared__ float lsb[2][16];                    // branch LSE (log2 units)
-    const int g = blockIdx.x, s = blockIdx.y;
+    __shared__ float wgt[kDecMaxUnits][2][HQ];      // selected/window record weight per branch and head
+    __shared__ float wgc[kDecMaxChunks][HQ];        // compressed record weight per head
+    __shared__ float lsb[2][HQ];                    // branch LSE (log2 units)
+    __shared__ float4 part[NHALF > 1 ? NOUT : 1][3];   // the second thread's sums per output
+    const int g = blockIdx.x, s = blockIdx.y, h0 = blockIdx.z * HQ;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int L, C;
-    if (!dec_seq_ok(p, s, L, C)) return;
+    if (h0 >= p.HG || !dec_seq_ok(p, s, L, C)) return;
     const size_t sg = (size_t)s * p.G + g;
     const int nch = (C + 31) / 32;
     dep_wait();                                       // the selected/window records
-    if (threadIdx.x < 32) {
+    if (warp == 0) {
         const long long X0 = (long long)sg * p.NUV;
         const int cnt = dec_record_list_warp(X0, X0 + p.NUV, (long long)p.S * p.G * p.NUV, p.grid3 * kDecW, recb,
                                              kDecMaxUnits);
-        if (threadIdx.x == 0) nrec = cnt;
-    } else if (threadIdx.x < 64) {
+        if (lane == 0) nrec = cnt;
+    } else if (warp == 1) {
         int cnt = 0;
         if (nch > 0) {
             const long long X0 = (long long)p.cpre[s] + (long long)g * nch;
             cnt = dec_record_list_warp(X0, X0 + nch, p.cpre[p.S], p.grid1 * kDecW, recc, kDecMaxChunks);
         }
-        if (threadIdx.x == 32) nrecc = cnt;
+        if (lane == 0) nrecc = cnt;
     }
     __syncthreads();
     const int nr = nrec, nrc = nrecc;
-    {   // compressed records: weight exp2(m - LSE) per head, 16 threads per head
-        const int h = threadIdx.x >> 4, sub = threadIdx.x & 15;
-        const float lc = p.lsecmp[sg * 16 + h];
-        for (int i0 = sub; i0 < nrc; i0 += 64) {
-            float rm[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int i = i0 + 16 * k;
-                rm[k] = i < nrc ? p.part1[((size_t)(recc[i] + sg) * 16 + h) * REC] : -INFINITY;
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int i = i0 + 16 * k;
-                if (i < nrc) wgc[i][h] = (rm[k] != -INFINITY && lc != -INFINITY) ? exp2f(rm[k] - lc) : 0.f;
-            }
-        }
-    }
     {
-        const int bh = threadIdx.x >> 3, sub = threadIdx.x & 7;   // 32 (branch, head) x 8 threads
-        const int br = bh >> 4, h = bh & 15;
-        constexpr int PR = (kDecMaxUnits + 7) / 8;                 // records per thread
-        float rm[PR], rl[PR];
+        // compressed records of head h0 + warp (lane: records lane, lane + 32, ...) and
+        // selected/window records of group (branch, head) gi (16 lanes), loads first
+        const int hc = h0 + warp;
+        const float lc = hc < p.HG ? p.lsecmp[sg * 16 + hc] : -INFINITY;
+        const int gi = warp * 2 + (lane >> 4), sub = lane & 15;
+        const int br = gi / HQ, hl = gi % HQ, h = h0 + hl;
+        constexpr int PC = kDecMaxChunks / 32, PR = (kDecMaxUnits + 15) / 16;
+        float cm[PC], rm[PR], rl[PR];
+#pragma unroll
+        for (int k = 0; k < PC; ++k) {
+            const int i = lane + 32 * k;
+            cm[k] = (i < nrc && lc != -INFINITY) ? p.part1[((size_t)(recc[i] + sg) * 16 + hc) * REC] : -INFINITY;
+        }
 #pragma unroll
         for (int k = 0; k < PR; ++k) {
-            const int i = sub + 8 * k;
-            const float* r = p.part2 + ((((size_t)recb[i < nr ? i : 0] + sg) * 2 + br) * 16 + h) * REC;
-            rm[k] = i < nr ? r[0] : -INFINITY;
-            rl[k] = i < nr ? r[1] : 0.f;
+            const int i = sub + 16 * k;
+            const bool use = i < nr && h < p.HG;
+            const float* r = p.part2 + ((((size_t)recb[use ? i : 0] + sg) * 2 + br) * 16 + (use ? h : 0)) * REC;
+            rm[k] = use ? r[0] : -INFINITY;
+            rl[k] = use ? r[1] : 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < PC; ++k) {
+            const int i = lane + 32 * k;
+            if (i < nrc) wgc[i][warp] = cm[k] != -INFINITY ? exp2f(cm[k] - lc) : 0.f;
         }
         float M = -INFINITY;
 #pragma unroll
         for (int k = 0; k < PR; ++k) M = fmaxf(M, rm[k]);
 #pragma unroll
-        for (int o = 4; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        for (int o = 8; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
         float Ls = 0.f;
 #pragma unroll
         for (int k = 0; k < PR; ++k)
             if (rm[k] != -INFINITY) Ls += rl[k] * exp2f(rm[k] - M);
 #pragma unroll
-        for (int o = 4; o >= 1; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
+        for (int o = 8; o >= 1; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
         const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
 #pragma unroll
         for (int k = 0; k < PR; ++k) {
-            const int i = sub + 8 * k;
-            if (i < nr) wgt[i][br][h] = rm[k] == -INFINITY ? 0.f : exp2f(rm[k] - M) * inv;
+            const int i = sub + 16 * k;
+            if (i < nr) wgt[i][br][hl] = rm[k] == -INFINITY ? 0.f : exp2f(rm[k] - M) * inv;
         }
-        if (sub == 0) lsb[br][h] = Ls > 0.f ? M + log2f(Ls) : -INFINITY;
+        if (sub == 0) lsb[br][hl] = Ls > 0.f ? M + log2f(Ls) : -INFINITY;
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < p.HG * (DV / 4); e += blockDim.x) {
-        const int h = e / (DV / 4), c4 = (e % (DV / 4)) * 4;
-        const size_t row = (size_t)s * p.H + g * p.HG + h;
-        const float gt0 = p.gates[row * 3], gt1 = p.gates[row * 3 + 1], gt2 = p.gates[row * 3 + 2];
-        float4 oc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int i0 = 0; i0 < nrc; i0 += 8) {
-            float4 v[8];
+    // round 2: output e (head h0 + e / (DV/4), channels c4 .. c4+3)
+    const int e = threadIdx.x % NOUT, half = threadIdx.x / NOUT;
+    const int hl = e / (DV / 4), c4 = (e % (DV / 4)) * 4, h = h0 + hl;
+    const bool active = h < p.HG;
+    float4 acc[3];
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-                v[k] = i0 + k < nrc ? *reinterpret_cast<const float4*>(p.part1 + ((size_t)(recc[i0 + k] + sg) * 16 + h) * REC + 4 + c4)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int q = 0; q < 3; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto fma4 = [](float4& a, const float4& v, float w) {
+        a.x = fmaf(v.x, w, a.x);
+        a.y = fmaf(v.y, w, a.y);
+        a.z = fmaf(v.z, w, a.z);
+        a.w = fmaf(v.w, w, a.w);
+    };
+    const int nmax = max(nr, nrc);
+    for (int i0 = half; active && i0 < nmax; i0 += 8 * NHALF) {
+        float4 vc[8], vs[8], vw[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const float w = i0 + k < nrc ? wgc[i0 + k][h] : 0.f;
-                oc.x += v[k].x * w;
-                oc.y += v[k].y * w;
-                oc.z += v[k].z * w;
-                oc.w += v[k].w * w;
+        for (int k = 0; k < 8; ++k) {
+            const int i = i0 + NHALF * k;
+            const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+            vc[k] = (i < nrc && wgc[i][hl] != 0.f)
+                        ? *reinterpret_cast<const float4*>(p.part1 + ((size_t)(recc[i] + sg) * 16 + h) * REC + 4 + c4)
+                        : z;
+            vs[k] = (i < nr && wgt[i][0][hl] != 0.f)
+                        ? *reinterpret_cast<const float4*>(p.part2 + ((((size_t)recb[i] + sg) * 2 + 0) * 16 + h) * REC + 4 + c4)
+                        : z;
+            vw[k] = (i < nr && wgt[i][1][hl] != 0.f)
+                        ? *reinterpret_cast<const float4*>(p.part2 + ((((size_t)recb[i] + sg) * 2 + 1) * 16 + h) * REC + 4 + c4)
+                        : z;
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int i = i0 + NHALF * k;
+            fma4(acc[0], vc[k], i < nrc ? wgc[i][hl] : 0.f);
+            fma4(acc[1], vs[k], i < nr ? wgt[i][0][hl] : 0.f);
+            fma4(acc[2], vw[k], i < nr ? wgt[i][1][hl] : 0.f);
+        }
+    }
+    if (NHALF > 1) {
+        if (half == 1) {
+#pragma unroll
+            for (int q = 0; q < 3; ++q) part[e][q] = acc[q];
+        }
+        __syncthreads();
+    }
+    if (half == 0 && active) {
+        if (NHALF > 1) {
+#pragma unroll
+            for (int q = 0; q < 3; ++q) {
+                const float4 o = part[e][q];
+                acc[q].x += o.x;
+                acc[q].y += o.y;
+                acc[q].z += o.z;
+                acc[q].w += o.w;
             }
         }
-        float4 O[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
-        for (int i0 = 0; i0 < nr; i0 += 8) {
-            float4 v[8][2];
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-#pragma unroll
-                for (int br = 0; br < 2; ++br)
-                    v[k][br] = i0 + k < nr ? *reinterpret_cast<const float4*>(
-                                                 p.part2 + ((((size_t)recb[i0 + k] + sg) * 2 + br) * 16 + h) * REC + 4 + c4)
-                                           : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-#pragma unroll
-                for (int br = 0; br < 2; ++br) {
-                    const float w = i0 + k < nr ? wgt[i0 + k][br][h] : 0.f;
-                    O[br].x += v[k][br].x * w;
-                    O[br].y += v[k][br].y * w;
-                    O[br].z += v[k][br].z * w;
-                    O[br].w += v[k][br].w * w;
-                }
-        }
+        const size_t row = (size_t)s * p.H + (size_t)g * p.HG + h;
+        const float gt0 = p.gates[row * 3], gt1 = p.gates[row * 3 + 1], gt2 = p.gates[row * 3 + 2];
         float4 r;
-        r.x = gt0 * oc.x + gt1 * O[0].x + gt2 * O[1].x;
-        r.y = gt0 * oc.y + gt1 * O[0].y + gt2 * O[1].y;
-        r.z = gt0 * oc.z + gt1 * O[0].z + gt2 * O[1].z;
-        r.w = gt0 * oc.w + gt1 * O[0].w + gt2 * O[1].w;
+        r.x = gt0 * acc[0].x + gt1 * acc[1].x + gt2 * acc[2].x;
+        r.y = gt0 * acc[0].y + gt1 * acc[1].y + gt2 * acc[2].y;
+        r.z = gt0 * acc[0].z + gt1 * acc[1].z + gt2 * acc[2].z;
+        r.w = gt0 * acc[0].w + gt1 * acc[1].w + gt2 * acc[2].w;
         *reinterpret_cast<float4*>(p.out + row * DV + c4) = r;
         if (c4 == 0 && p.lse) {
 #pragma unroll
             for (int br = 0; br < 2; ++br) {
-                const float lb = lsb[br][h];
+                const float lb = lsb[br][hl];
                 p.lse[row * 3 + 1 + br] = lb == -INFINITY ? -INFINITY : lb * kLn2;
             }
             const float lc = p.lsecmp[sg * 16 + h];

@@ -925,7 +925,7 @@ nsa_status_t decode_launch(DecParams& p, const Shape& s, int S, cudaStream_t st)
     NSA_LAUNCH("dec_slcwin_stream", st,
                NSA_TRY(launch_dependent(dec_slcwin_stream<DK, DV>, dim3((unsigned)p.grid3), dim3(256), smem3, st, p)));
     NSA_LAUNCH("dec_final", st,
-               NSA_TRY(launch_dependent(dec_final<DV>, dim3((unsigned)s.G, (unsigned)S), dim3(256), 0, st, p)));
+               NSA_TRY(launch_dependent(dec_final<DV>, dim3((unsigned)s.G, (unsigned)S, (unsigned)ceil_div(s.HG, kDecFinalHeads)), dim3(256), 0, st, p)));
     return last_launch();
 }
 

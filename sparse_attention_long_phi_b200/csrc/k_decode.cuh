@@ -470,6 +470,28 @@ __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
         }
         if (threadIdx.x == 0) nrec = cnt;
     }
+    // When no warp range is empty (at least as many chunks as warps), the pair's records
+    // are those of the consecutive warps bf .. bl: the LSE's record loads (this
+    // thread's first four) are issued now, before the list is shared.
+    const int hh = threadIdx.x >> 4, hsub = threadIdx.x & 15;
+    float rm0[4], rl0[4];
+    int nr_direct = -1;
+    {
+        const long long NN = p.cpre[p.S];
+        const int W1 = p.grid1 * kDecW;
+        if (nch > 0 && NN >= W1) {
+            const long long X0 = (long long)p.cpre[s] + (long long)g * nch;
+            const int bf = dec_cta_of(X0, NN, W1);
+            nr_direct = dec_cta_of(X0 + nch - 1, NN, W1) - bf + 1;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int i = hsub + 16 * k;
+                const float* r = p.part1 + ((size_t)(bf + (i < nr_direct ? i : 0)) + sg) * 16 * REC + (size_t)hh * REC;
+                rm0[k] = i < nr_direct ? r[0] : -INFINITY;
+                rl0[k] = i < nr_direct ? r[1] : 0.f;
+            }
+        }
+    }
     float* fac = csm;
     float* pg = fac + p.NCH * 16;
     // chunk maxima (log2 units) and this thread's block sums: independent of the LSE
@@ -504,16 +526,21 @@ __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
     const int nr = nrec;
     {   // LSE per head over the records: 16 threads per head, each thread's records
         // (i = sub, sub + 16, ...) read once, up to four at a time
-        const int h = threadIdx.x >> 4, sub = threadIdx.x & 15;
+        const int h = hh, sub = hsub;
         float M = -INFINITY, Ls = 0.f;
         for (int i0 = sub; i0 < nr; i0 += 64) {
             float rm[4], rl[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const int i = i0 + 16 * k;
-                const float* r = p.part1 + ((size_t)(recb[i < nr ? i : 0] + sg) * 16 + h) * REC;
-                rm[k] = i < nr ? r[0] : -INFINITY;
-                rl[k] = i < nr ? r[1] : 0.f;
+                if (i0 == sub && nr_direct >= 0) {      // loaded before the barrier
+                    rm[k] = rm0[k];
+                    rl[k] = rl0[k];
+                } else {
+                    const float* r = p.part1 + ((size_t)(recb[i < nr ? i : 0] + sg) * 16 + h) * REC;
+                    rm[k] = i < nr ? r[0] : -INFINITY;
+                    rl[k] = i < nr ? r[1] : 0.f;
+                }
             }
 #pragma unroll
             for (int k = 0; k < 4; ++k) {

@@ -5,28 +5,29 @@
 // One query per sequence at t = L-1 over packed varlen caches.  The step is
 // HBM-bound: every cache row is read once.  The 16 heads of a GQA group are
 // the M = 16 side of warp-level bf16 tensor-core products (mma.sync
-// m16n8k16, fp32 accumulate).  The two streaming kernels are persistent (one
-// CTA of 8 warps per SM).  Each warp pipelines K and V separately (the next
+// m16n8k16, fp32 accumulate).  The streaming kernels are persistent (one CTA
+// per SM: 8 warps, 4 for the window stream).  Each warp pipelines K and V separately (the next
 // chunk's K is in flight while this chunk's softmax and P.V run, its V while
 // the next logits run) and keeps an online softmax.  Compressed stream: the
 // chunks of 32 cache rows of all (seq, group) pairs form one sequence cut into
 // equal contiguous ranges, one per warp; a warp streams its range across pair
 // boundaries and writes a record per pair it touched at slot (warp index +
 // seq*G + group), unique because consecutive pairs share at most one warp.
-// Selected/window stream: the same with ranges per CTA, whose warps take a
-// pair's chunks round-robin and merge once per pair into one record.
+// The window stream takes the same per-warp ranges over the chunks that meet
+// each pair's window, the selected stream over the pairs' selected blocks.
 //   1. dec_cmp_stream   compressed cache: per segment (max, sum, unnormalised
 //                       O); per chunk the head max and the per-head selection-
 //                       block sums of exp(logit - chunk max), mapped with the
 //                       overlap weights, so the importance scores can be
 //                       normalised exactly once the row LSE is known.
-//   2. dec_cmp_combine  per (seq, group): LSE, o_cmp, group importance scores
-//                       (sum over heads and chunks of the block sums rescaled
-//                       by exp(chunk max - LSE)), top-n by one warp.
-//   3. dec_slcwin_stream  the sorted union of the selected blocks and the
-//                       window blocks (a fixed number of unit slots per pair,
-//                       the unused ones empty): logits once, online softmax of
-//                       the selected and the window branch.
+//   2. dec_cmp_combine  per (seq, group): LSE, group importance scores (sum over
+//                       heads and chunks of the block sums rescaled by
+//                       exp(chunk max - LSE)), top-n by the CTA.
+//   2b. dec_win_stream  the window's 32-token chunks, beside the combine (it does
+//                       not need the selection; it waits for the combine before
+//                       it exits).
+//   3. dec_slcwin_stream  the selected blocks' chunks: logits, online softmax,
+//                       P.V per warp.
 //   4. dec_final        merge the records per branch; out = sum_c g_c o_c; lse.
 #pragma once
 #include "nsa_dev.cuh"
@@ -39,7 +40,7 @@ constexpr int kDecW = 8;             // warps per streaming CTA
 constexpr int kDecNBS = 33;          // block-sum slots per chunk (>= (31 + l/d - 1) / (l'/d) + 1)
 constexpr int kDecMaxSeqs = 2048;    // sequences per call (chunk prefix held in shared memory)
 constexpr int kDecMaxChunks = 256;   // compressed chunks per sequence (T <= 131072, d = 16)
-constexpr int kDecMaxUnits = 48;     // units in a (selected U window) list
+constexpr int kDecMaxRecs = 64;      // records of a pair in the selected or the window stream
 constexpr int kDecMaxGrid = 1024;    // CTAs of a streaming kernel
 
 struct DecParams {
@@ -58,11 +59,12 @@ struct DecParams {
     float* bsum;     // [S*G][NCH][kDecNBS][16]   per-head block sums of exp2(s - chunk max)
     float* part1;    // [grid1*8 + S*G][16][DV+4] per warp and pair: max, sum, -, -, unnormalised O
     float* lsecmp;   // [S*G][16]                 log2 units
-    float* part2;    // [grid3 + S*G][2][16][DV+4] per segment and branch (selected, window)
+    float* part2;    // [grid3*8 + S*G][16][DV+4] per warp and pair of the selected stream
+    float* partw;    // [gridw*4 + S*G][16][DV+4] per warp and pair of the window stream
     int* cpre;       // [S+1] compressed chunks (x G) before sequence s
-    int* units;      // [S*G][NUV] selected U window blocks of a pair: block*2 + selected, -1 empty
-    int Lmax, Cmax, NCH, NUV, NSmax;
-    int grid1, grid3;
+    int* wpre;       // [S+1] window chunks (x G) before sequence s
+    int Lmax, Cmax, NCH, NSmax;
+    int grid1, grid3, gridw;
 };
 
 template <int DK, int DV>
@@ -381,64 +383,6 @@ __global__ void __launch_bounds__(256, 1) dec_cmp_stream(const DecParams p) {
     }
 }
 
-// sorted union of the selected blocks (sel: n entries, -1 padded, ascending)
-// and the blocks overlapping the window; flag[i] = 1 when list[i] is selected
-__device__ __forceinline__ int dec_units(const DecParams& p, const int32_t* sel, int L, int* list, int* flag) {
-    const int wlo = max(0, L - p.w) / p.lp, whi = (L - 1) / p.lp;
-    int i = 0, j = wlo, cnt = 0, last = -1;
-    while (cnt < kDecMaxUnits) {
-        const int a = (i < p.n && sel[i] >= 0) ? sel[i] : 0x7fffffff;
-        const int b = j <= whi ? j : 0x7fffffff;
-        const int m = min(a, b);
-        if (m == 0x7fffffff) break;
-        const bool from_sel = m == a;
-        if (m == a) ++i;
-        if (m == b) ++j;
-        if (m != last) {
-            list[cnt] = m;
-            flag[cnt] = from_sel ? 1 : 0;
-            ++cnt;
-        } else if (from_sel) {
-            flag[cnt - 1] = 1;
-        }
-        last = m;
-    }
-    return cnt;
-}
-
-// dec_units by one warp, written as units[i] = block*2 + selected (-1 past the
-// end, NUV slots): lane i holds selected block i, lane k window block wlo + k;
-// a block's place is the number of list entries below it.
-// scratch: >= 32 + 2 * kDecMaxUnits ints of shared memory (the one-lane path).
-__device__ __forceinline__ void dec_units_warp(const DecParams& p, const int32_t* sel, int L, int* units,
-                                               int* scratch) {
-    const int lane = threadIdx.x & 31;
-    const int wlo = max(0, L - p.w) / p.lp, whi = (L - 1) / p.lp, nw = whi - wlo + 1;
-    if (nw > 32) {                                     // windows of more than 32 blocks: one lane
-        if (lane == 0) {
-            int* sb = scratch;
-            int* list = scratch + 32;
-            int* flag = scratch + 32 + kDecMaxUnits;
-            for (int i = 0; i < p.n; ++i) sb[i] = sel[i];
-            const int cnt = dec_units(p, sb, L, list, flag);
-            for (int i = 0; i < p.NUV; ++i) units[i] = i < cnt ? list[i] * 2 + flag[i] : -1;
-        }
-        return;
-    }
-    const int a = lane < p.n ? sel[lane] : -1;        // ascending, -1 padded
-    const bool va = a >= 0;
-    const bool inw = va && a >= wlo && a <= whi;
-    const bool out = va && !inw;
-    const unsigned mout = __ballot_sync(0xffffffffu, out);
-    const unsigned mbelow = __ballot_sync(0xffffffffu, out && a < wlo);
-    const unsigned selw = __reduce_or_sync(0xffffffffu, inw ? 1u << (a - wlo) : 0u);   // window blocks selected
-    const unsigned lt = (1u << lane) - 1u;
-    if (out) units[__popc(mout & lt) + (a > whi ? nw : 0)] = a * 2 + 1;
-    if (lane < nw) units[lane + __popc(mbelow)] = (wlo + lane) * 2 + ((selw >> lane) & 1u);
-    const int cnt = nw + __popc(mout);
-    for (int i = cnt + lane; i < p.NUV; i += 32) units[i] = -1;
-}
-
 // -------------------------------------------------------------- step 2
 // Every load that does not need the row LSE (chunk maxima, this thread's block
 // sums) is issued before the first barrier; the records give the LSE in one
@@ -600,10 +544,237 @@ __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
     }
     __syncthreads();
     topn_row_cta_redux<256>(pg, t, p.n, p.lp, p.fi, p.fl, p.sel_idx + sg * p.n, tsm);
-    // the pair's units for the selected/window stream: the sorted union of the
-    // selected blocks and the window's blocks, each flagged when selected
-    __syncthreads();                                   // the selection row is written
-    if (threadIdx.x < 32) dec_units_warp(p, p.sel_idx + sg * p.n, L, p.units + sg * p.NUV, tsm);
+}
+
+// -------------------------------------------------------------- step 2b
+// The sliding window over the last w tokens of every (seq, group).  It does not
+// depend on the selection, so it runs beside the combine: launched after it,
+// small enough (four warps, one branch, at most 168 registers) to share an SM with a
+// combine CTA, and waiting for the combine only before it exits, so that the
+// kernels after it see the selection.  Items: the 32-token chunks meeting the
+// window, of all (seq, group) pairs in one sequence cut into equal contiguous
+// ranges, one per warp; per chunk the logits once, the window mask, an online
+// softmax and P.V; a record per (warp, pair) at slot (warp index + seq*G + group).
+// Shared memory: per warp two K/V stages (two chunks in flight) and a Q tile.
+constexpr int kDecWinW = 4;          // warps per window-stream CTA
+
+// 32-token chunks of a length-L sequence that meet its window [L-w, L-1]
+__device__ __forceinline__ int dec_win_chunks(const DecParams& p, int L) {
+    return (L - 1) / 32 - max(0, L - p.w) / 32 + 1;
+}
+
+template <int DK, int DV>
+__host__ __device__ constexpr int dec_win_smem() {          // per warp: two K/V stages and a Q tile
+    return kDecWinW * (2 * dec_stage_bytes<DK, DV>() + 16 * (DK * 2 + 16));
+}
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(128, 3) dec_win_stream(const DecParams p) {
+    constexpr int KP = DK * 2 + 16, STG = dec_stage_bytes<DK, DV>(), REC = DV + 4;
+    extern __shared__ __align__(16) uint8_t dsm[];
+    __shared__ int pre[kDecMaxSeqs + 1];
+    __shared__ uint64_t kbar[kDecWinW][2], vbar[kDecWinW][2];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gr = lane >> 2, tg = lane & 3;
+    uint8_t* stg0 = dsm + warp * 2 * STG;                 // stage b: K rows at stg0 + b*STG, V after them
+    uint8_t* qs = dsm + kDecWinW * 2 * STG + warp * 16 * KP;   // this warp's [16][DK] Q tile
+    if (threadIdx.x < kDecWinW * 2) {
+        mbar_init(&kbar[threadIdx.x >> 1][threadIdx.x & 1], 1);
+        mbar_init(&vbar[threadIdx.x >> 1][threadIdx.x & 1], 1);
+    }
+    fence_mbar_init();
+    if (warp == 0) {
+        int run = 0;
+        for (int b0 = 0; b0 < p.S; b0 += 32) {
+            const int s = b0 + lane;
+            int cnt = 0, L, C;
+            if (s < p.S && dec_seq_ok(p, s, L, C)) cnt = p.G * dec_win_chunks(p, L);
+            int inc = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += v;
+            }
+            if (s < p.S) pre[s] = run + inc - cnt;
+            run += __shfl_sync(0xffffffffu, inc, 31);
+        }
+        if (lane == 0) pre[p.S] = run;
+    }
+    __syncthreads();
+    dep_launch();
+    if (blockIdx.x == 0)
+        for (int s = threadIdx.x; s <= p.S; s += blockDim.x) p.wpre[s] = pre[s];
+    const long long N = pre[p.S];
+    const int gw = blockIdx.x * kDecWinW + warp, W = gridDim.x * kDecWinW;
+    long long x = dec_range_start(gw, N, W);
+    const long long x1 = dec_range_start(gw + 1, N, W);
+    const float cl = p.scale_log2;
+    uint32_t kph = 0, vph = 0;                             // bit b: phase of stage b
+    const uint64_t pol = l2_evict_first();
+    const size_t kst = (size_t)p.G * DK, vst = (size_t)p.G * DV;
+    struct Seg {
+        int s, g, L, c, nw, u0;                      // chunk c of the pair's nw; its first token u0
+        int64_t kvb;
+    };
+    auto locate = [&](long long xx, Seg& q) {
+        int lo = 0, hi = p.S;                        // largest lo with pre[lo] <= xx
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (pre[mid] <= xx) lo = mid;
+            else hi = mid;
+        }
+        int L, C;
+        dec_seq_ok(p, lo, L, C);                     // lo holds chunks: its lengths passed
+        const int nw = dec_win_chunks(p, L);
+        const int r = (int)(xx - pre[lo]);
+        q.s = lo;
+        q.g = r / nw;
+        q.L = L;
+        q.c = r - q.g * nw;
+        q.nw = nw;
+        q.u0 = (max(0, L - p.w) / 32 + q.c) * 32;
+        q.kvb = p.kv_off[lo];
+    };
+    // the item after q (x of q given): the pair's next chunk, or the next pair's first
+    auto advance = [&](const Seg& q, long long xq, Seg& nx) {
+        if (q.c + 1 < q.nw) {
+            nx = q;
+            ++nx.c;
+            nx.u0 += 32;
+        } else {
+            locate(xq + 1, nx);
+        }
+    };
+    auto issue = [&](const Seg& q, int b) {
+        uint8_t* ks = stg0 + b * STG;
+        warp_bulk_rows<DK>(ks, p.kcache + ((size_t)(q.kvb + q.u0) * p.G + q.g) * DK, kst, q.L - q.u0, &kbar[warp][b], pol);
+        warp_bulk_rows<DV>(ks + 32 * KP, p.vcache + ((size_t)(q.kvb + q.u0) * p.G + q.g) * DV, vst, q.L - q.u0,
+                           &vbar[warp][b], pol);
+    };
+    // Q of the group as a [16][DK] tile (rows >= HG zero), read with ldmatrix
+    auto load_q_tile = [&](const Seg& q) {
+        for (int e = lane; e < 16 * (DK / 8); e += 32) {
+            const int h = e / (DK / 8), c8 = e % (DK / 8);
+            int4 v = make_int4(0, 0, 0, 0);
+            if (h < p.HG) v = *reinterpret_cast<const int4*>(p.q + ((size_t)q.s * p.H + (size_t)q.g * p.HG + h) * DK + c8 * 8);
+            *reinterpret_cast<int4*>(qs + h * KP + c8 * 16) = v;
+        }
+        __syncwarp();
+    };
+    if (x < x1) {
+        // two chunks in flight: chunk i in stage i & 1
+        Seg cur, nx1;
+        locate(x, cur);
+        issue(cur, 0);
+        if (x + 1 < x1) {
+            advance(cur, x, nx1);
+            issue(nx1, 1);
+        }
+        load_q_tile(cur);
+        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+        float o[DV / 8][4];
+#pragma unroll
+        for (int nt = 0; nt < DV / 8; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+        for (int i = 0;; ++i) {
+            const int b = i & 1;
+            uint8_t* ks = stg0 + b * STG;
+            if (!mbar_wait(&kbar[warp][b], (kph >> b) & 1, 0x405)) break;   // K of chunk i
+            kph ^= 1u << b;
+            __syncwarp();
+            float sf[4][4];
+            warp_logits_sa<DK>(smem_u32(qs), smem_u32(ks), sf);
+            // keys u0 + k inside [L - w, L - 1]
+            const int klo = cur.L - p.w - cur.u0, khi = cur.L - cur.u0;
+            float mc0 = -INFINITY, mc1 = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int key = nt * 8 + tg * 2 + (e & 1);
+                    const float v = (key >= klo && key < khi) ? sf[nt][e] * cl : -INFINITY;
+                    sf[nt][e] = v;
+                    if (e < 2) mc0 = fmaxf(mc0, v);
+                    else mc1 = fmaxf(mc1, v);
+                }
+#pragma unroll
+            for (int q2 = 1; q2 <= 2; q2 <<= 1) {
+                mc0 = fmaxf(mc0, __shfl_xor_sync(0xffffffffu, mc0, q2));
+                mc1 = fmaxf(mc1, __shfl_xor_sync(0xffffffffu, mc1, q2));
+            }
+            const float mn0 = fmaxf(m0, mc0), mn1 = fmaxf(m1, mc1);
+            float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float v = sf[nt][e];
+                    const float pv = v == -INFINITY ? 0.f : exp2f(v - (e < 2 ? mn0 : mn1));
+                    sf[nt][e] = pv;
+                    if (e < 2) s0 += pv;
+                    else s1 += pv;
+                }
+#pragma unroll
+            for (int q2 = 1; q2 <= 2; q2 <<= 1) {
+                s0 += __shfl_xor_sync(0xffffffffu, s0, q2);
+                s1 += __shfl_xor_sync(0xffffffffu, s1, q2);
+            }
+            const float a0 = mn0 == -INFINITY ? 1.f : exp2f(m0 - mn0);
+            const float a1 = mn1 == -INFINITY ? 1.f : exp2f(m1 - mn1);
+            m0 = mn0;
+            m1 = mn1;
+            l0 = l0 * a0 + s0;
+            l1 = l1 * a1 + s1;
+#pragma unroll
+            for (int nt = 0; nt < DV / 8; ++nt) {
+                o[nt][0] *= a0;
+                o[nt][1] *= a0;
+                o[nt][2] *= a1;
+                o[nt][3] *= a1;
+            }
+            if (!mbar_wait(&vbar[warp][b], (vph >> b) & 1, 0x406)) break;   // V of chunk i
+            vph ^= 1u << b;
+            __syncwarp();
+            warp_pv<DV>(sf, smem_u32(ks + 32 * KP), o);
+            __syncwarp();
+            const long long xi = x + i;
+            const bool more = xi + 1 < x1;
+            // stage b is free: chunk i + 2 goes there
+            Seg nx2;
+            if (xi + 2 < x1) {
+                advance(nx1, xi + 1, nx2);
+                issue(nx2, b);
+            }
+            if (!more || !(cur.s == nx1.s && cur.g == nx1.g)) {
+                // this warp's record of (seq, group): (max, sum, -, -, O relative to max)
+                const size_t sg = (size_t)cur.s * p.G + cur.g;
+                float* rec = p.partw + ((size_t)gw + sg) * 16 * REC;
+                if (tg == 0) {
+                    rec[gr * REC] = m0;
+                    rec[gr * REC + 1] = l0;
+                    rec[(gr + 8) * REC] = m1;
+                    rec[(gr + 8) * REC + 1] = l1;
+                }
+#pragma unroll
+                for (int nt = 0; nt < DV / 8; ++nt) {
+                    const int cc = 4 + nt * 8 + tg * 2;
+                    *reinterpret_cast<float2*>(rec + gr * REC + cc) = make_float2(o[nt][0], o[nt][1]);
+                    *reinterpret_cast<float2*>(rec + (gr + 8) * REC + cc) = make_float2(o[nt][2], o[nt][3]);
+                }
+                m0 = m1 = -INFINITY;
+                l0 = l1 = 0.f;
+#pragma unroll
+                for (int nt = 0; nt < DV / 8; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+                if (more) load_q_tile(nx1);
+            }
+            if (!more) break;
+            cur = nx1;
+            nx1 = nx2;
+        }
+    }
+    dep_wait();                                       // the combine: the kernels after this one read its selection
 }
 
 // -------------------------------------------------------------- step 3
@@ -612,17 +783,17 @@ __host__ __device__ constexpr int dec_slcwin_smem() {        // staging + one Q 
     return kDecW * dec_stage_bytes<DK, DV>() + kDecW * 16 * (DK * 2 + 16);
 }
 
-// Each warp owns a contiguous, equal range of the unit slots (NUV per pair, the
-// combine's sorted union of selected and window blocks, -1 when empty); per pair
-// it loads its own copy of Q and streams the chunks of the pair's units in its
-// range, then writes one record per branch at slot (warp index + seq*G + group),
-// unique because consecutive pairs share at most one warp.
+// The selected branch.  Each warp owns a contiguous, equal range of the block
+// slots (n per pair: the selection row, ascending, -1 padded); per pair it loads
+// its own copy of Q and streams the chunks of the pair's blocks in its range,
+// then writes one record at slot (warp index + seq*G + group), unique because
+// consecutive pairs share at most one warp.
 template <int DK, int DV>
 __global__ void __launch_bounds__(256, 1) dec_slcwin_stream(const DecParams p) {
     constexpr int KP = DK * 2 + 16, STG = dec_stage_bytes<DK, DV>();
     extern __shared__ __align__(16) uint8_t dsm[];
     __shared__ uint64_t kbar[kDecW], vbar[kDecW];
-    __shared__ int ulw[kDecW][33];                    // per warp: a batch's non-empty units, their count
+    __shared__ int ulw[kDecW][33];                    // per warp: a batch's selected blocks, their count
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tg = lane & 3;
     uint8_t* ks = dsm + warp * STG;
     uint8_t* vs = ks + 32 * KP;
@@ -634,26 +805,26 @@ __global__ void __launch_bounds__(256, 1) dec_slcwin_stream(const DecParams p) {
     fence_mbar_init();
     __syncthreads();
     dep_launch();
-    dep_wait();                                       // the combine's units and selections
+    dep_wait();                                       // the combine's selections (through the window stream)
     uint32_t kph = 0, vph = 0;
     const uint64_t pol = l2_evict_first();
-    const long long U = (long long)p.S * p.G * p.NUV;
+    const long long U = (long long)p.S * p.G * p.n;
     const int gw = blockIdx.x * kDecW + warp, W = gridDim.x * kDecW;
     long long x = dec_range_start(gw, U, W);
     const long long x1 = dec_range_start(gw + 1, U, W);
     const float cl = p.scale_log2;
     constexpr int REC = DV + 4;
     while (x < x1) {
-        const size_t sg = (size_t)(x / p.NUV);
-        const int ua = (int)(x % p.NUV);
-        const int nslot = (int)min((long long)(p.NUV - ua), x1 - x);
+        const size_t sg = (size_t)(x / p.n);
+        const int ua = (int)(x % p.n);
+        const int nslot = (int)min((long long)(p.n - ua), x1 - x);
         const int s = (int)(sg / p.G), g = (int)(sg % p.G);
         int L, C;
         const bool ok = dec_seq_ok(p, s, L, C);
         const int64_t kvb = ok ? p.kv_off[s] : 0;
         const size_t kst = (size_t)p.G * DK, vst = (size_t)p.G * DV;
 
-        auto tok0 = [&](int u, int i) { return (u >> 1) * p.lp + (i & 1) * 32; };
+        auto tok0 = [&](int blk, int i) { return blk * p.lp + (i & 1) * 32; };
         // rows past the cache are not read; the source stays inside the sequence
         auto issue_k = [&](int u0) {
             const int nv = min(32, L - u0);
@@ -663,35 +834,29 @@ __global__ void __launch_bounds__(256, 1) dec_slcwin_stream(const DecParams p) {
             const int nv = min(32, L - u0);
             warp_bulk_rows<DV>(vs, p.vcache + ((size_t)(kvb + (nv > 0 ? u0 : 0)) * p.G + g) * DV, vst, nv, &vbar[warp], pol);
         };
-        float m[2][2], l[2][2];
-        float o[2][DV / 8][4];
+        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+        float o[DV / 8][4];
 #pragma unroll
-        for (int br = 0; br < 2; ++br) {
-            m[br][0] = m[br][1] = -INFINITY;
-            l[br][0] = l[br][1] = 0.f;
+        for (int nt = 0; nt < DV / 8; ++nt)
 #pragma unroll
-            for (int nt = 0; nt < DV / 8; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) o[br][nt][e] = 0.f;
-        }
-        const int wlo = L - p.w;
+            for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
         bool live = true, qready = false;
-        // this range's units of the pair, 32 slots at a time (lane i: slot ua + b0 + i)
+        // this range's blocks of the pair, 32 slots at a time (lane i: slot ua + b0 + i)
         for (int b0 = 0; b0 < nslot && live; b0 += 32) {
         {
-            const int myu = (ok && b0 + lane < nslot) ? p.units[sg * p.NUV + ua + b0 + lane] : -1;
+            const int myu = (ok && b0 + lane < nslot) ? p.sel_idx[sg * p.n + ua + b0 + lane] : -1;
             const unsigned umask = __ballot_sync(0xffffffffu, myu >= 0);
             if (myu >= 0) ulw[warp][__popc(umask & ((1u << lane) - 1u))] = myu;
             if (lane == 0) ulw[warp][32] = __popc(umask);
         }
         __syncwarp();
         const int n = 2 * ulw[warp][32];                   // chunks of 32 tokens
-        // unit of chunk i: the (i/2)-th non-empty slot of the batch
-        auto unit_of = [&](int i) { return ulw[warp][i >> 1]; };
-        int ucur = n > 0 ? unit_of(0) : 0;
+        // block of chunk i: the (i/2)-th selected block of the batch
+        auto block_of = [&](int i) { return ulw[warp][i >> 1]; };
+        int bcur = n > 0 ? block_of(0) : 0;
         if (n > 0) {
-            issue_k(tok0(ucur, 0));
-            issue_v(tok0(ucur, 0));
+            issue_k(tok0(bcur, 0));
+            issue_v(tok0(bcur, 0));
             if (!qready) {
                 // Q of the group as a [16][DK] tile (rows >= HG zero), read with ldmatrix;
                 // loaded while the first rows are in flight
@@ -708,13 +873,9 @@ __global__ void __launch_bounds__(256, 1) dec_slcwin_stream(const DecParams p) {
         }
         for (int i = 0; i < n; ++i) {
             const bool more = i + 1 < n;
-            const int unxt = more ? ((i & 1) ? unit_of(i + 1) : ucur) : ucur;
-            const int u0 = tok0(ucur, i);
-            const bool insel = (ucur & 1) != 0;
+            const int bnxt = more ? ((i & 1) ? block_of(i + 1) : bcur) : bcur;
+            const int u0 = tok0(bcur, i);
             const int nval = min(32, L - u0);
-            // warp-uniform: does the chunk hold keys of each branch?
-            const bool has_sel = insel && nval > 0;
-            const bool has_win = nval > 0 && u0 + nval - 1 >= wlo;
             if (!mbar_wait(&kbar[warp], kph, 0x403)) {   // K of chunk i
                 live = false;
                 break;
@@ -722,28 +883,24 @@ __global__ void __launch_bounds__(256, 1) dec_slcwin_stream(const DecParams p) {
             kph ^= 1;
             __syncwarp();
             float sf[4][4];
-            if (has_sel || has_win) warp_logits_sa<DK>(smem_u32(qs), smem_u32(ks), sf);
+            if (nval > 0) warp_logits_sa<DK>(smem_u32(qs), smem_u32(ks), sf);
             __syncwarp();
-            if (more) issue_k(tok0(unxt, i + 1));
+            if (more) issue_k(tok0(bnxt, i + 1));
             if (!mbar_wait(&vbar[warp], vph, 0x404)) {   // V of chunk i
                 live = false;
                 break;
             }
             vph ^= 1;
             __syncwarp();
-#pragma unroll
-            for (int br = 0; br < 2; ++br) {
-                if (br == 0 ? !has_sel : !has_win) continue;
-                float pf4[4][4];
+            if (nval > 0) {
                 float mc0 = -INFINITY, mc1 = -INFINITY;
 #pragma unroll
                 for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int key = nt * 8 + tg * 2 + (e & 1);
-                        const bool okk = key < nval && (br == 0 || u0 + key >= wlo);
-                        const float v = okk ? sf[nt][e] * cl : -INFINITY;
-                        pf4[nt][e] = v;
+                        const float v = key < nval ? sf[nt][e] * cl : -INFINITY;
+                        sf[nt][e] = v;
                         if (e < 2) mc0 = fmaxf(mc0, v);
                         else mc1 = fmaxf(mc1, v);
                     }
@@ -752,15 +909,15 @@ __global__ void __launch_bounds__(256, 1) dec_slcwin_stream(const DecParams p) {
                     mc0 = fmaxf(mc0, __shfl_xor_sync(0xffffffffu, mc0, q2));
                     mc1 = fmaxf(mc1, __shfl_xor_sync(0xffffffffu, mc1, q2));
                 }
-                const float mn0 = fmaxf(m[br][0], mc0), mn1 = fmaxf(m[br][1], mc1);
+                const float mn0 = fmaxf(m0, mc0), mn1 = fmaxf(m1, mc1);
                 float s0 = 0.f, s1 = 0.f;
 #pragma unroll
                 for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float v = pf4[nt][e];
+                        const float v = sf[nt][e];
                         const float pv = v == -INFINITY ? 0.f : exp2f(v - (e < 2 ? mn0 : mn1));
-                        pf4[nt][e] = pv;
+                        sf[nt][e] = pv;
                         if (e < 2) s0 += pv;
                         else s1 += pv;
                     }
@@ -769,45 +926,41 @@ __global__ void __launch_bounds__(256, 1) dec_slcwin_stream(const DecParams p) {
                     s0 += __shfl_xor_sync(0xffffffffu, s0, q2);
                     s1 += __shfl_xor_sync(0xffffffffu, s1, q2);
                 }
-                const float a0 = mn0 == -INFINITY ? 1.f : exp2f(m[br][0] - mn0);
-                const float a1 = mn1 == -INFINITY ? 1.f : exp2f(m[br][1] - mn1);
-                m[br][0] = mn0;
-                m[br][1] = mn1;
-                l[br][0] = l[br][0] * a0 + s0;
-                l[br][1] = l[br][1] * a1 + s1;
+                const float a0 = mn0 == -INFINITY ? 1.f : exp2f(m0 - mn0);
+                const float a1 = mn1 == -INFINITY ? 1.f : exp2f(m1 - mn1);
+                m0 = mn0;
+                m1 = mn1;
+                l0 = l0 * a0 + s0;
+                l1 = l1 * a1 + s1;
 #pragma unroll
                 for (int nt = 0; nt < DV / 8; ++nt) {
-                    o[br][nt][0] *= a0;
-                    o[br][nt][1] *= a0;
-                    o[br][nt][2] *= a1;
-                    o[br][nt][3] *= a1;
+                    o[nt][0] *= a0;
+                    o[nt][1] *= a0;
+                    o[nt][2] *= a1;
+                    o[nt][3] *= a1;
                 }
-                warp_pv<DV>(pf4, smem_u32(vs), o[br]);
+                warp_pv<DV>(sf, smem_u32(vs), o);
             }
             __syncwarp();
-            if (more) issue_v(tok0(unxt, i + 1));
-            ucur = unxt;
+            if (more) issue_v(tok0(bnxt, i + 1));
+            bcur = bnxt;
         }
         }
         if (!live) break;
-        // this warp's records of the pair, one per branch: (max, sum, -, -, O relative to max)
-        float* rec = p.part2 + ((size_t)gw + sg) * 2 * 16 * REC;
+        // this warp's record of the pair: (max, sum, -, -, O relative to max)
+        float* rec = p.part2 + ((size_t)gw + sg) * 16 * REC;
         const int gr = lane >> 2;
+        if (tg == 0) {
+            rec[gr * REC] = m0;
+            rec[gr * REC + 1] = l0;
+            rec[(gr + 8) * REC] = m1;
+            rec[(gr + 8) * REC + 1] = l1;
+        }
 #pragma unroll
-        for (int br = 0; br < 2; ++br) {
-            float* rb = rec + br * 16 * REC;
-            if (tg == 0) {
-                rb[gr * REC] = m[br][0];
-                rb[gr * REC + 1] = l[br][0];
-                rb[(gr + 8) * REC] = m[br][1];
-                rb[(gr + 8) * REC + 1] = l[br][1];
-            }
-#pragma unroll
-            for (int nt = 0; nt < DV / 8; ++nt) {
-                const int cc = 4 + nt * 8 + tg * 2;
-                *reinterpret_cast<float2*>(rb + gr * REC + cc) = make_float2(o[br][nt][0], o[br][nt][1]);
-                *reinterpret_cast<float2*>(rb + (gr + 8) * REC + cc) = make_float2(o[br][nt][2], o[br][nt][3]);
-            }
+        for (int nt = 0; nt < DV / 8; ++nt) {
+            const int cc = 4 + nt * 8 + tg * 2;
+            *reinterpret_cast<float2*>(rec + gr * REC + cc) = make_float2(o[nt][0], o[nt][1]);
+            *reinterpret_cast<float2*>(rec + (gr + 8) * REC + cc) = make_float2(o[nt][2], o[nt][3]);
         }
         __syncwarp();                                  // the Q tile is reloaded for the next pair
         x += nslot;
@@ -831,10 +984,10 @@ template <int DV>
 __global__ void __launch_bounds__(256, 2) dec_final(const DecParams p) {
     constexpr int REC = DV + 4, HQ = kDecFinalHeads, NOUT = HQ * DV / 4, NHALF = 256 / NOUT;
     static_assert(NHALF >= 1 && NHALF <= 2 && NHALF * NOUT == 256, "threads per output float4");
-    __shared__ int recb[kDecMaxUnits];
+    __shared__ int recb[2][kDecMaxRecs];            // selected / window stream records
     __shared__ int recc[kDecMaxChunks];
-    __shared__ int nrec, nrecc;
-    __shared__ float wgt[kDecMaxUnits][2][HQ];      // selected/window record weight per branch and head
+    __shared__ int nrec[2], nrecc;
+    __shared__ float wgt[kDecMaxRecs][2][HQ];       // selected/window record weight per branch and head
     __shared__ float wgc[kDecMaxChunks][HQ];        // compressed record weight per head
     __shared__ float lsb[2][HQ];                    // branch LSE (log2 units)
     __shared__ float4 part[NHALF > 1 ? NOUT : 1][3];   // the second thread's sums per output
@@ -844,12 +997,18 @@ __global__ void __launch_bounds__(256, 2) dec_final(const DecParams p) {
     if (h0 >= p.HG || !dec_seq_ok(p, s, L, C)) return;
     const size_t sg = (size_t)s * p.G + g;
     const int nch = (C + 31) / 32;
-    dep_wait();                                       // the selected/window records
+    dep_wait();                                       // the selected branch's records
     if (warp == 0) {
-        const long long X0 = (long long)sg * p.NUV;
-        const int cnt = dec_record_list_warp(X0, X0 + p.NUV, (long long)p.S * p.G * p.NUV, p.grid3 * kDecW, recb,
-                                             kDecMaxUnits);
-        if (lane == 0) nrec = cnt;
+        const long long X0 = (long long)sg * p.n;
+        const int cnt = dec_record_list_warp(X0, X0 + p.n, (long long)p.S * p.G * p.n, p.grid3 * kDecW, recb[0],
+                                             kDecMaxRecs);
+        if (lane == 0) nrec[0] = cnt;
+    } else if (warp == 2) {
+        const int nw = dec_win_chunks(p, L);
+        const long long X0 = (long long)p.wpre[s] + (long long)g * nw;
+        const int cnt = dec_record_list_warp(X0, X0 + nw, (long long)p.wpre[p.S], p.gridw * kDecWinW, recb[1],
+                                             kDecMaxRecs);
+        if (lane == 0) nrec[1] = cnt;
     } else if (warp == 1) {
         int cnt = 0;
         if (nch > 0) {
@@ -859,7 +1018,7 @@ __global__ void __launch_bounds__(256, 2) dec_final(const DecParams p) {
         if (lane == 0) nrecc = cnt;
     }
     __syncthreads();
-    const int nr = nrec, nrc = nrecc;
+    const int nrs = nrec[0], nrw = nrec[1], nrc = nrecc;
     {
         // compressed records of head h0 + warp (lane: records lane, lane + 32, ...) and
         // selected/window records of group (branch, head) gi (16 lanes), loads first
@@ -867,7 +1026,7 @@ __global__ void __launch_bounds__(256, 2) dec_final(const DecParams p) {
         const float lc = hc < p.HG ? p.lsecmp[sg * 16 + hc] : -INFINITY;
         const int gi = warp * 2 + (lane >> 4), sub = lane & 15;
         const int br = gi / HQ, hl = gi % HQ, h = h0 + hl;
-        constexpr int PC = kDecMaxChunks / 32, PR = (kDecMaxUnits + 15) / 16;
+        constexpr int PC = kDecMaxChunks / 32, PR = kDecMaxRecs / 16;
         float cm[PC], rm[PR], rl[PR];
 #pragma unroll
         for (int k = 0; k < PC; ++k) {
@@ -877,8 +1036,8 @@ __global__ void __launch_bounds__(256, 2) dec_final(const DecParams p) {
 #pragma unroll
         for (int k = 0; k < PR; ++k) {
             const int i = sub + 16 * k;
-            const bool use = i < nr && h < p.HG;
-            const float* r = p.part2 + ((((size_t)recb[use ? i : 0] + sg) * 2 + br) * 16 + (use ? h : 0)) * REC;
+            const bool use = i < (br ? nrw : nrs) && h < p.HG;
+            const float* r = (br ? p.partw : p.part2) + (((size_t)recb[br][use ? i : 0] + sg) * 16 + (use ? h : 0)) * REC;
             rm[k] = use ? r[0] : -INFINITY;
             rl[k] = use ? r[1] : 0.f;
         }
@@ -902,7 +1061,7 @@ __global__ void __launch_bounds__(256, 2) dec_final(const DecParams p) {
 #pragma unroll
         for (int k = 0; k < PR; ++k) {
             const int i = sub + 16 * k;
-            if (i < nr) wgt[i][br][hl] = rm[k] == -INFINITY ? 0.f : exp2f(rm[k] - M) * inv;
+            if (i < (br ? nrw : nrs)) wgt[i][br][hl] = rm[k] == -INFINITY ? 0.f : exp2f(rm[k] - M) * inv;
         }
         if (sub == 0) lsb[br][hl] = Ls > 0.f ? M + log2f(Ls) : -INFINITY;
     }
@@ -920,7 +1079,7 @@ __global__ void __launch_bounds__(256, 2) dec_final(const DecParams p) {
         a.z = fmaf(v.z, w, a.z);
         a.w = fmaf(v.w, w, a.w);
     };
-    const int nmax = max(nr, nrc);
+    const int nmax = max(max(nrs, nrw), nrc);
     for (int i0 = half; active && i0 < nmax; i0 += 8 * NHALF) {
         float4 vc[8], vs[8], vw[8];
 #pragma unroll
@@ -930,19 +1089,19 @@ __global__ void __launch_bounds__(256, 2) dec_final(const DecParams p) {
             vc[k] = (i < nrc && wgc[i][hl] != 0.f)
                         ? *reinterpret_cast<const float4*>(p.part1 + ((size_t)(recc[i] + sg) * 16 + h) * REC + 4 + c4)
                         : z;
-            vs[k] = (i < nr && wgt[i][0][hl] != 0.f)
-                        ? *reinterpret_cast<const float4*>(p.part2 + ((((size_t)recb[i] + sg) * 2 + 0) * 16 + h) * REC + 4 + c4)
+            vs[k] = (i < nrs && wgt[i][0][hl] != 0.f)
+                        ? *reinterpret_cast<const float4*>(p.part2 + (((size_t)recb[0][i] + sg) * 16 + h) * REC + 4 + c4)
                         : z;
-            vw[k] = (i < nr && wgt[i][1][hl] != 0.f)
-                        ? *reinterpret_cast<const float4*>(p.part2 + ((((size_t)recb[i] + sg) * 2 + 1) * 16 + h) * REC + 4 + c4)
+            vw[k] = (i < nrw && wgt[i][1][hl] != 0.f)
+                        ? *reinterpret_cast<const float4*>(p.partw + (((size_t)recb[1][i] + sg) * 16 + h) * REC + 4 + c4)
                         : z;
         }
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
             const int i = i0 + NHALF * k;
             fma4(acc[0], vc[k], i < nrc ? wgc[i][hl] : 0.f);
-            fma4(acc[1], vs[k], i < nr ? wgt[i][0][hl] : 0.f);
-            fma4(acc[2], vw[k], i < nr ? wgt[i][1][hl] : 0.f);
+            fma4(acc[1], vs[k], i < nrs ? wgt[i][0][hl] : 0.f);
+            fma4(acc[2], vw[k], i < nrw ? wgt[i][1][hl] : 0.f);
         }
     }
     if (NHALF > 1) {
@@ -988,16 +1147,19 @@ inline size_t decode_ws_bytes(int64_t S, int64_t Lmax, int64_t G, int64_t l, int
                               int64_t w, int64_t n, int64_t DV) {
     const int64_t Cmax = Lmax >= l ? (Lmax - l) / d + 1 : 1;
     const int64_t NCH = (Cmax + 31) / 32;
-    const int64_t NUV = n + (w + lp - 1) / lp + 1;
+    (void)lp;
+    (void)w;
+    (void)n;
     auto a = [](size_t x) { return (x + 255) & ~size_t(255); };
     size_t o = 0;
     o += a((size_t)S * G * NCH * 16 * 4);
     o += a((size_t)S * G * NCH * kDecNBS * 16 * 4);
     o += a((size_t)(kDecMaxGrid * kDecW + S * G) * 16 * (DV + 4) * 4);
     o += a((size_t)S * G * 16 * 4);
-    o += a((size_t)(kDecMaxGrid * kDecW + S * G) * 2 * 16 * (DV + 4) * 4);
+    o += a((size_t)(kDecMaxGrid * kDecW + S * G) * 16 * (DV + 4) * 4);
+    o += a((size_t)(kDecMaxGrid * kDecWinW + S * G) * 16 * (DV + 4) * 4);
     o += a((size_t)(S + 1) * 4);
-    o += a((size_t)S * G * NUV * 4);
+    o += a((size_t)(S + 1) * 4);
     return o;
 }
 

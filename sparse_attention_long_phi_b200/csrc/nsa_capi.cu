@@ -905,16 +905,19 @@ int device_sm_count() {
 template <int DK, int DV>
 nsa_status_t decode_launch(DecParams& p, const Shape& s, int S, cudaStream_t st) {
     constexpr int smem = dec_stream_smem<DK, DV>(), smem3 = dec_slcwin_smem<DK, DV>();
+    constexpr int smemw = dec_win_smem<DK, DV>();
     const int nsm = device_sm_count();
     // persistent streaming kernels: as many CTAs as fit on the device at once
     int occ1 = 1, occ3 = 1;
     NSA_TRY(set_smem(dec_cmp_stream<DK, DV>, smem));
     NSA_TRY(set_smem(dec_slcwin_stream<DK, DV>, smem3));
+    NSA_TRY(set_smem(dec_win_stream<DK, DV>, smemw));
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ1, dec_cmp_stream<DK, DV>, 256, smem) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ3, dec_slcwin_stream<DK, DV>, 256, smem3) != cudaSuccess)
         return NSA_ERR_CUDA;
     p.grid1 = std::min(kDecMaxGrid, nsm * std::max(1, occ1));
     p.grid3 = std::min(kDecMaxGrid, nsm * std::max(1, occ3));
+    p.gridw = std::min(kDecMaxGrid, nsm);
     NSA_LAUNCH("dec_cmp_stream", st, dec_cmp_stream<DK, DV><<<(unsigned)p.grid1, 256, smem, st>>>(p));
     NSA_TRY(last_launch());
     // the three dependent kernels start while their predecessor drains
@@ -922,6 +925,10 @@ nsa_status_t decode_launch(DecParams& p, const Shape& s, int S, cudaStream_t st)
     NSA_TRY(set_smem(dec_cmp_combine<DV>, smem2));
     NSA_LAUNCH("dec_cmp_combine", st,
                NSA_TRY(launch_dependent(dec_cmp_combine<DV>, dim3((unsigned)s.G, (unsigned)S), dim3(256), smem2, st, p)));
+    // the window stream runs beside the combine (one CTA per SM next to a combine CTA)
+    // and waits for it before exiting; the selected stream after it sees the selection
+    NSA_LAUNCH("dec_win_stream", st,
+               NSA_TRY(launch_dependent(dec_win_stream<DK, DV>, dim3((unsigned)p.gridw), dim3(kDecWinW * 32), smemw, st, p)));
     NSA_LAUNCH("dec_slcwin_stream", st,
                NSA_TRY(launch_dependent(dec_slcwin_stream<DK, DV>, dim3((unsigned)p.grid3), dim3(256), smem3, st, p)));
     NSA_LAUNCH("dec_final", st,
@@ -966,9 +973,10 @@ nsa_status_t decode_impl(const Shape& s, int S, const void* q, const void* kcach
     p.Lmax = (int)s.T;
     p.Cmax = (int)(s.T >= s.l ? (s.T - s.l) / s.d + 1 : 1);
     p.NCH = (int)ceil_div(p.Cmax, 32);
-    p.NUV = (int)(s.n + ceil_div(s.w, s.lp) + 1);
     p.NSmax = (int)ceil_div(s.T, s.lp);
-    if (S > kDecMaxSeqs || p.NCH > kDecMaxChunks || p.NUV > kDecMaxUnits || p.nbs > kDecNBS || 32 % p.spb != 0)
+    // records of a pair: at most n (selected stream) and w/32 + 2 (window stream)
+    if (S > kDecMaxSeqs || p.NCH > kDecMaxChunks || s.n > kDecMaxRecs || s.w / 32 + 2 > kDecMaxRecs ||
+        p.nbs > kDecNBS || 32 % p.spb != 0)
         return NSA_ERR_UNSUPPORTED;
     size_t o = 0;
     auto carve = [&](size_t bytes) {
@@ -981,9 +989,10 @@ nsa_status_t decode_impl(const Shape& s, int S, const void* q, const void* kcach
     p.bsum = carve(SG * p.NCH * kDecNBS * 16 * 4);
     p.part1 = carve((kDecMaxGrid * kDecW + SG) * 16 * (s.DV + 4) * 4);
     p.lsecmp = carve(SG * 16 * 4);
-    p.part2 = carve((kDecMaxGrid * kDecW + SG) * 2 * 16 * (s.DV + 4) * 4);
+    p.part2 = carve((kDecMaxGrid * kDecW + SG) * 16 * (s.DV + 4) * 4);
+    p.partw = carve((kDecMaxGrid * kDecWinW + SG) * 16 * (s.DV + 4) * 4);
     p.cpre = reinterpret_cast<int*>(carve((size_t)(S + 1) * 4));
-    p.units = reinterpret_cast<int*>(carve(SG * p.NUV * 4));
+    p.wpre = reinterpret_cast<int*>(carve((size_t)(S + 1) * 4));
     if (s.DK == 192) return decode_launch<192, 128>(p, s, S, st);
     return decode_launch<64, 64>(p, s, S, st);
 }

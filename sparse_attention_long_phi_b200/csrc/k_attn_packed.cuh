@@ -54,17 +54,21 @@ struct PackedParams {
 template <int DK, int DV, int HG, int MODE>
 struct PackedCfg {
     static constexpr int TOK = 128 / HG;              // tokens per query tile
-    // keys per tile: 128 in the LSE pass (S only in TMEM, and an N = 128 product
-    // reads Q from shared memory once per 128 keys), 64 where O also lives in TMEM
-    static constexpr int BN = MODE == kModeLse ? 128 : 64;
+    // keys per tile: 128 in the compressed passes (an N = 128 product reads Q from
+    // shared memory once per 128 keys), 64 for the window.  Pass 2 keeps one S
+    // buffer per query tile (S 2 x 128 + O 2 x 128 TMEM columns); the LSE pass,
+    // with no O, and the window keep two.
+    static constexpr int BN = MODE == kModeWin ? 64 : 128;
+    static constexpr int NBUF = MODE == kModeCmp ? 1 : 2;
     static constexpr int NQB = DK / 64;
     static constexpr int kQBytes = 128 * DK * 2;      // one tile
     static constexpr int kKBox = BN * 128;            // BN rows x 128 B
     static constexpr int kKBytes = NQB * kKBox;
-    static constexpr int kVBytes = DV * 128;          // DV rows x 64 keys
+    static constexpr int kVBox = DV * 128;            // DV rows x 64 keys
+    static constexpr int kVBytes = kVBox * (BN / 64);
     static constexpr int kPBytes = 128 * 128;         // 128 rows x 64 keys
     static constexpr int NSK = 2;
-    static constexpr int NSV = MODE == kModeLse ? 0 : 2;
+    static constexpr int NSV = MODE == kModeLse ? 0 : (MODE == kModeCmp ? 1 : 2);
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + 2 * kQBytes;
     static constexpr int kOffV = kOffK + NSK * kKBytes;
@@ -72,7 +76,8 @@ struct PackedCfg {
     static constexpr int kOffBar = kOffP;             // P lives in tensor memory
     static constexpr int kSmem = kOffBar + 256 + 1024;
     static_assert(kSmem <= 232448, "shared memory");
-    // TMEM: S tile A [0, 2BN) (2 buffers of BN), S tile B [2BN, 4BN), then O_A, O_B
+    // TMEM: S tile A [0, NBUF BN) (NBUF buffers of BN), S tile B [NBUF BN, 2 NBUF BN),
+    // then O_A, O_B from column 256
     static constexpr uint32_t kTmemCols = 512;
     static constexpr int kThreads = 320;
 };
@@ -228,7 +233,9 @@ __global__ void __launch_bounds__(320, 1)
                         break;
                     uint8_t* vs = smem + Cfg::kOffV + sv * Cfg::kVBytes;
                     mbar_expect_tx(&vfull[sv], Cfg::kVBytes);
-                    tma_load_4d(vs, &mapV, &vfull[sv], kb, 0, g, b);
+#pragma unroll
+                    for (int hb = 0; hb < Cfg::BN / 64; ++hb)
+                        tma_load_4d(vs + hb * Cfg::kVBox, &mapV, &vfull[sv], kb + hb * 64, 0, g, b);
                 }
             }
         }
@@ -238,56 +245,77 @@ __global__ void __launch_bounds__(320, 1)
             constexpr uint32_t idS = idesc_bf16(128, Cfg::BN);
             constexpr uint32_t idO = idesc_bf16(128, DV);
             bool ok = wait_or_abort(qfull, 0, 0x203, abort_flag);
-            auto issue_S = [&](int jt) -> bool {
-                const int s = jt % NSK, buf = jt & 1;
-                if (!wait_or_abort(&kfull[s], (jt / NSK) & 1, 0x204, abort_flag)) return false;
+            // S of key tile jt for query tile `tile` (and both tiles when tile < 0)
+            auto issue_S = [&](int jt, int only) -> bool {
+                const int s = jt % NSK, buf = Cfg::NBUF == 2 ? (jt & 1) : 0;
+                if (only <= 0 && !wait_or_abort(&kfull[s], (jt / NSK) & 1, 0x204, abort_flag)) return false;
                 const uint32_t sK = smem_u32(smem + Cfg::kOffK + s * Cfg::kKBytes);
 #pragma unroll
                 for (int tile = 0; tile < 2; ++tile) {
+                    if (only >= 0 && tile != only) continue;
                     if (MODE == kModeLse && jt >= 2 &&
                         !wait_or_abort(&sfree[2 * tile + buf], ((jt - 2) >> 1) & 1, 0x205, abort_flag))
                         return false;
-                    // the buffer's P(jt-2) must have been read by its P.V product: an MMA
-                    // writing tensor memory is not ordered behind an earlier MMA that
+                    // the buffer's P(jt - NBUF) must have been read by its P.V product: an
+                    // MMA writing tensor memory is not ordered behind an earlier MMA that
                     // reads the same columns as its A operand
-                    if (MODE != kModeLse && jt >= 2 &&
-                        !wait_or_abort(&pvdone[tile], (jt - 2) & 1, 0x20B, abort_flag))
+                    if (MODE != kModeLse && jt >= Cfg::NBUF &&
+                        !wait_or_abort(&pvdone[tile], (jt - Cfg::NBUF) & 1, 0x20B, abort_flag))
                         return false;
                     tc_fence_after();
                     const uint32_t sQ = smem_u32(smem + Cfg::kOffQ + tile * Cfg::kQBytes);
 #pragma unroll
                     for (int kk = 0; kk < DK / 16; ++kk)
-                        umma_bf16_ss(tmem + tile * 2 * Cfg::BN + buf * Cfg::BN,
+                        umma_bf16_ss(tmem + tile * Cfg::NBUF * Cfg::BN + buf * Cfg::BN,
                                      sdesc_sw128(sQ + (kk / 4) * 16384 + (kk % 4) * 32),
                                      sdesc_sw128(sK + (kk / 4) * Cfg::kKBox + (kk % 4) * 32), idS,
                                      kk > 0 ? 1u : 0u);
                     umma_commit(&sfull[2 * tile + buf]);
                 }
-                umma_commit(&kempty[s]);
+                if (only != 0) umma_commit(&kempty[s]);       // both tiles have read the K stage
                 return true;
             };
-            auto issue_PV = [&](int jt) -> bool {
+            // P.V of key tile jt for query tile `tile` (and both tiles when tile < 0)
+            auto issue_PV = [&](int jt, int only) -> bool {
                 const int sv = jt % NSV;
-                if (!wait_or_abort(&vfull[sv], (jt / NSV) & 1, 0x207, abort_flag)) return false;
+                if (only <= 0 && !wait_or_abort(&vfull[sv], (jt / NSV) & 1, 0x207, abort_flag)) return false;
                 const uint32_t sV = smem_u32(smem + Cfg::kOffV + sv * Cfg::kVBytes);
 #pragma unroll
                 for (int tile = 0; tile < 2; ++tile) {
+                    if (only >= 0 && tile != only) continue;
                     if (!wait_or_abort(&pfull[tile], jt & 1, 0x206, abort_flag)) return false;
                     tc_fence_after();
-                    const uint32_t tP = tmem + tile * 128 + (jt & 1) * 64;    // P over S(jt)
+                    // P (bf16 pairs) over the first BN/2 columns of S(jt)
+                    const uint32_t tP = tmem + tile * Cfg::NBUF * Cfg::BN + (Cfg::NBUF == 2 ? (jt & 1) : 0) * Cfg::BN;
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16_ts(tmem + 256 + tile * DV, tP + kk * 8, sdesc_sw128(sV + kk * 32), idO,
+                    for (int kk = 0; kk < Cfg::BN / 16; ++kk)
+                        umma_bf16_ts(tmem + 256 + tile * DV, tP + kk * 8,
+                                     sdesc_sw128(sV + (kk / 4) * Cfg::kVBox + (kk % 4) * 32), idO,
                                      (jt > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&pvdone[tile]);
                 }
-                umma_commit(&vempty[sv]);
+                if (only != 0) umma_commit(&vempty[sv]);      // both tiles have read the V stage
                 return true;
             };
-            if (ok) ok = issue_S(0);
-            for (int jt = 0; jt < ntiles && ok; ++jt) {
-                if (jt + 1 < ntiles) ok = issue_S(jt + 1);
-                if (ok && MODE != kModeLse) ok = issue_PV(jt);
+            if (Cfg::NBUF == 2) {
+                // S(jt+1) into the other buffer while the softmax works on S(jt)
+                if (ok) ok = issue_S(0, -1);
+                for (int jt = 0; jt < ntiles && ok; ++jt) {
+                    if (jt + 1 < ntiles) ok = issue_S(jt + 1, -1);
+                    if (ok && MODE != kModeLse) ok = issue_PV(jt, -1);
+                }
+            } else {
+                // one S buffer per query tile: P.V(jt) of a tile, then its S(jt+1) into
+                // the same columns; the two tiles alternate so that one tile's products
+                // run while the other's softmax does
+                if (ok) ok = issue_S(0, 0);
+                if (ok) ok = issue_S(0, 1);
+                for (int jt = 0; jt < ntiles && ok; ++jt) {
+                    ok = issue_PV(jt, 0);
+                    if (ok && jt + 1 < ntiles) ok = issue_S(jt + 1, 0);
+                    if (ok) ok = issue_PV(jt, 1);
+                    if (ok && jt + 1 < ntiles) ok = issue_S(jt + 1, 1);
+                }
             }
         }
     } else {
@@ -301,7 +329,7 @@ __global__ void __launch_bounds__(320, 1)
         const bool row_ok = t < p.T;
         const size_t rowid = ((size_t)b * p.T + (row_ok ? t : 0)) * p.H + h;
         const uint32_t lanebase = tmem + ((uint32_t)(wq * 32) << 16);
-        const uint32_t sbase = lanebase + tile * 2 * Cfg::BN; // S buffers of this tile
+        const uint32_t sbase = lanebase + tile * Cfg::NBUF * Cfg::BN; // S buffers of this tile
         const uint32_t obase = lanebase + 256 + tile * DV;    // O of this tile
         int vis_hi, vis_lo = 0;
         if (MODE == kModeWin) {
@@ -382,13 +410,16 @@ __global__ void __launch_bounds__(320, 1)
             }
         }
         for (int jt = 0; MODE != kModeLse && jt < ntiles; ++jt) {
-            const int buf = jt & 1;
-            const int kb = key0 + jt * 64;
-            if (ok) ok = wait_or_abort(&sfull[2 * tile + buf], (jt >> 1) & 1, 0x208, abort_flag);
+            const int buf = Cfg::NBUF == 2 ? (jt & 1) : 0;
+            if (ok) ok = wait_or_abort(&sfull[2 * tile + buf], (Cfg::NBUF == 2 ? (jt >> 1) : jt) & 1, 0x208, abort_flag);
             tc_fence_after();
+            // the key tile in halves of 64 keys (one half for the window)
+#pragma unroll 1
+            for (int hb = 0; hb < Cfg::BN / 64; ++hb) {
+            const int kb = key0 + jt * Cfg::BN + hb * 64;
             uint32_t ra[32], rb[32];
-            tmem_ld32(sbase + buf * 64, ra);
-            tmem_ld32(sbase + buf * 64 + 32, rb);
+            tmem_ld32(sbase + buf * Cfg::BN + hb * 64, ra);
+            tmem_ld32(sbase + buf * Cfg::BN + hb * 64 + 32, rb);
             tmem_wait_ld32(ra);
             tmem_wait_ld32(rb);
             float s[64];
@@ -488,7 +519,7 @@ __global__ void __launch_bounds__(320, 1)
             // the previous P.V of this tile finished: the window's O rescale needs it,
             // and it keeps this loop at most one pvdone phase ahead of the MMA warp
             // (a parity wait cannot tell phases two apart; the epilogue relies on it)
-            if (jt > 0 && ok) ok = wait_or_abort(&pvdone[tile], (jt - 1) & 1, 0x209, abort_flag);
+            if (hb == 0 && jt > 0 && ok) ok = wait_or_abort(&pvdone[tile], (jt - 1) & 1, 0x209, abort_flag);
             tc_fence_after();
             if (MODE == kModeWin && jt > 0 && __any_sync(0xffffffffu, need_rescale)) {
                 const float a = need_rescale ? alpha : 1.f;
@@ -503,14 +534,16 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 tmem_wait_st();
             }
-            // P (bf16, two per column) over the first 32 columns of S(jt): the A
-            // operand of this tile's P.V product
+            // P (bf16, two per column) over the first BN/2 columns of S(jt), 32 per
+            // half: the A operand of this tile's P.V product (half 1's columns 32-63
+            // held keys of half 0, already read)
             {
                 uint32_t pk[32];
 #pragma unroll
                 for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pr[2 * c], pr[2 * c + 1]);
-                tmem_st32(sbase + buf * 64, pk);
+                tmem_st32(sbase + buf * Cfg::BN + hb * 32, pk);
                 tmem_wait_st();
+            }
             }
             tc_fence_before();
             mbar_arrive(&pfull[tile]);
@@ -526,7 +559,7 @@ __global__ void __launch_bounds__(320, 1)
         } else {
             if (MODE == kModeCmp && NC > 0) {
                 // flush the carried partial scores of the block after the last tile
-                const int jn = (key0 + ntiles * 64) / SPB;
+                const int jn = (key0 + ntiles * Cfg::BN) / SPB;
 #pragma unroll
                 for (int c = 0; c < (NC > 0 ? NC : 1); ++c) {
                     float v = carry[c];

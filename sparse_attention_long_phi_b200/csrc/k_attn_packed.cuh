@@ -20,14 +20,18 @@
 // One CTA takes two adjacent query tiles A and B (256 rows) that read the
 // same key tiles.  Warps 0-3 run the softmax and epilogue of tile A, warps
 // 4-7 those of tile B (thread = query row), warp 8 is the TMA producer and
-// warp 9 the MMA issuer and TMEM owner.  Key tiles of 64 keys:
+// warp 9 the MMA issuer and TMEM owner.  The window takes key tiles of 64 keys:
 //   S_x = Q_x K^T (M=128, N=64, K=DK) into one of two TMEM buffers per tile,
 //   O_x += P_x V  (M=128, N=DV, K=64) with P_x written as bf16 over the S
 //   columns it came from and read by the MMA from tensor memory (no shared-
 //   memory round trip for P); S(j+2) is issued into a buffer only once the
-//   P.V product that read P(j) from it has completed.
-// The MMA order S_A(j+1) S_B(j+1) PV_A(j) PV_B(j) lets each tile's softmax
-// overlap the other tile's products.  The softmax is issue-bound, so it is
+//   P.V product that read P(j) from it has completed, and the MMA order
+//   S_A(j+1) S_B(j+1) PV_A(j) PV_B(j) lets each tile's softmax overlap the
+//   other tile's products.  The compressed passes take 128 keys per tile (Q is
+//   read from shared memory once per 128 keys): pass 1 with two S buffers per
+//   tile (no O), pass 2 with one (S 128 + O 128 columns per tile), in the order
+//   PV_A(j) S_A(j+1) PV_B(j) S_B(j+1); the softmax reads a tile in two halves of
+//   64 keys.  The softmax is issue-bound, so it is
 // kept to about one FFMA + one MUFU + one add per logit, and the causal /
 // window masks are applied only on the key tiles that cross a row's bound.
 #pragma once

@@ -52,7 +52,7 @@ struct PackedParams {
     float* lse_cmp;            // [B,T,H] natural log (pass 1 writes, pass 2 reads)
     float* pscore;             // [B,T,G,NSp]
     int NSp;
-    int n_ctas;                // CTAs along the token axis (two query tiles each)
+    int n_ctas;                // query tile pairs along the token axis (two query tiles each)
 };
 
 template <int DK, int DV, int HG, int MODE>
@@ -158,24 +158,51 @@ __global__ void __launch_bounds__(320, 1)
     uint64_t* pvdone = bars + 21;         // [tile]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 23);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 24);
+    uint64_t* qempty = bars + 25;         // the item's S products have read Q (persistent)
+    uint64_t* ofree = bars + 26;          // [tile] the epilogue has read O (persistent)
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int cta = p.n_ctas - 1 - (int)blockIdx.x;   // heavy tiles first
-    const int g = blockIdx.y, b = blockIdx.z;
-    const int t0 = cta * 2 * TOK;                       // first token of tile A
-    if (t0 >= p.T) return;
-    const int t_last = min(t0 + 2 * TOK, p.T) - 1;      // last token of tile B
-
-    // key range shared by both tiles
-    int key0, ntiles;
-    if (MODE == kModeWin) {
-        const int klo = max(0, t0 - p.w + 1);
-        key0 = (klo / 64) * 64;
-        ntiles = (t_last - key0) / 64 + 1;
-    } else {
-        const int kend = (t_last + 1 >= p.l) ? (t_last + 1 - p.l) / p.d + 1 : 0;
-        key0 = 0;
-        ntiles = (kend + Cfg::BN - 1) / Cfg::BN;
+    // Work items: a pair of query tiles of one (batch, group).  One item per CTA, heavy
+    // tiles first; or, for the window (persistent launch), the CTAs stride over all items
+    // so that one item's epilogue overlaps the next item's loads and products.  Every role
+    // walks the same items in the same order and counts key tiles across them (jbase).
+    constexpr bool kPersist = MODE == kModeWin;
+    struct Item {
+        int g, b, t0, t_last, key0, ntiles;
+    };
+    const int n_items = kPersist ? p.n_ctas * p.G * p.B : 1;
+    auto item_of = [&](int iter, Item& it) -> bool {
+        int cta;
+        if (kPersist) {
+            const int i = (int)blockIdx.x + iter * (int)gridDim.x;
+            if (i >= n_items) return false;
+            cta = i % p.n_ctas;
+            it.g = (i / p.n_ctas) % p.G;
+            it.b = i / (p.n_ctas * p.G);
+        } else {
+            if (iter > 0) return false;
+            cta = p.n_ctas - 1 - (int)blockIdx.x;
+            it.g = blockIdx.y;
+            it.b = blockIdx.z;
+        }
+        it.t0 = cta * 2 * TOK;                         // first token of tile A
+        if (it.t0 >= p.T) return false;
+        it.t_last = min(it.t0 + 2 * TOK, p.T) - 1;     // last token of tile B
+        // key range shared by both tiles
+        if (MODE == kModeWin) {
+            const int klo = max(0, it.t0 - p.w + 1);
+            it.key0 = (klo / 64) * 64;
+            it.ntiles = (it.t_last - it.key0) / 64 + 1;
+        } else {
+            const int kend = (it.t_last + 1 >= p.l) ? (it.t_last + 1 - p.l) / p.d + 1 : 0;
+            it.key0 = 0;
+            it.ntiles = (kend + Cfg::BN - 1) / Cfg::BN;
+        }
+        return true;
+    };
+    {
+        Item it0;
+        if (!item_of(0, it0)) return;                  // no work: leave before any setup
     }
 
     if (threadIdx.x == 0) {
@@ -194,6 +221,9 @@ __global__ void __launch_bounds__(320, 1)
             mbar_init(&sfull[s], 1);
             mbar_init(&sfree[s], 4);
         }
+        mbar_init(qempty, 1);
+        mbar_init(&ofree[0], 128);
+        mbar_init(&ofree[1], 128);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -208,118 +238,152 @@ __global__ void __launch_bounds__(320, 1)
 
     if (warp == 8) {
         // ------------------------------------------------------ producer
-        if (lane == 0 && ntiles > 0) {
+        if (lane == 0) {
             tma_prefetch_desc(&mapQ);
             tma_prefetch_desc(&mapK);
             if (MODE != kModeLse) tma_prefetch_desc(&mapV);
-            mbar_expect_tx(qfull, 2 * Cfg::kQBytes);
+            int jbase = 0, qi = 0;                      // key tiles and Q loads before this item
+            bool ok = true;
+            Item it;
+            for (int iter = 0; ok && item_of(iter, it); ++iter) {
+                const int g = it.g, b = it.b, t0 = it.t0, key0 = it.key0, ntiles = it.ntiles;
+                if (ntiles == 0) continue;
+                // the previous item's S products have read Q
+                if (qi > 0 && !(ok = wait_or_abort(qempty, (qi - 1) & 1, 0x20C, abort_flag))) break;
+                mbar_expect_tx(qfull, 2 * Cfg::kQBytes);
 #pragma unroll
-            for (int tile = 0; tile < 2; ++tile)
+                for (int tile = 0; tile < 2; ++tile)
 #pragma unroll
-                for (int bx = 0; bx < Cfg::NQB; ++bx)
-                    tma_load_4d(smem + Cfg::kOffQ + tile * Cfg::kQBytes + bx * 16384, &mapQ, qfull,
-                                bx * 64, g * HG, t0 + tile * TOK, b);
-            for (int jt = 0; jt < ntiles; ++jt) {
-                const int kb = key0 + jt * Cfg::BN;
-                const int s = jt % NSK;
-                if (jt >= NSK && !wait_or_abort(&kempty[s], ((jt / NSK) - 1) & 1, 0x201, abort_flag))
-                    break;
-                uint8_t* ks = smem + Cfg::kOffK + s * Cfg::kKBytes;
-                mbar_expect_tx(&kfull[s], Cfg::kKBytes);
-#pragma unroll
-                for (int bx = 0; bx < Cfg::NQB; ++bx)
-#pragma unroll
-                    for (int hb = 0; hb < Cfg::BN / 64; ++hb)   // boxes of 64 rows
-                        tma_load_4d(ks + bx * Cfg::kKBox + hb * 8192, &mapK, &kfull[s], bx * 64, g, kb + hb * 64, b);
-                if (MODE != kModeLse) {
-                    const int sv = jt % NSV;
-                    if (jt >= NSV && !wait_or_abort(&vempty[sv], ((jt / NSV) - 1) & 1, 0x202, abort_flag))
+                    for (int bx = 0; bx < Cfg::NQB; ++bx)
+                        tma_load_4d(smem + Cfg::kOffQ + tile * Cfg::kQBytes + bx * 16384, &mapQ, qfull,
+                                    bx * 64, g * HG, t0 + tile * TOK, b);
+                ++qi;
+                for (int jt = 0; jt < ntiles; ++jt) {
+                    const int kb = key0 + jt * Cfg::BN, jg = jbase + jt;
+                    const int s = jg % NSK;
+                    if (jg >= NSK && !(ok = wait_or_abort(&kempty[s], ((jg / NSK) - 1) & 1, 0x201, abort_flag)))
                         break;
-                    uint8_t* vs = smem + Cfg::kOffV + sv * Cfg::kVBytes;
-                    mbar_expect_tx(&vfull[sv], Cfg::kVBytes);
+                    uint8_t* ks = smem + Cfg::kOffK + s * Cfg::kKBytes;
+                    mbar_expect_tx(&kfull[s], Cfg::kKBytes);
 #pragma unroll
-                    for (int hb = 0; hb < Cfg::BN / 64; ++hb)
-                        tma_load_4d(vs + hb * Cfg::kVBox, &mapV, &vfull[sv], kb + hb * 64, 0, g, b);
+                    for (int bx = 0; bx < Cfg::NQB; ++bx)
+#pragma unroll
+                        for (int hb = 0; hb < Cfg::BN / 64; ++hb)   // boxes of 64 rows
+                            tma_load_4d(ks + bx * Cfg::kKBox + hb * 8192, &mapK, &kfull[s], bx * 64, g, kb + hb * 64, b);
+                    if (MODE != kModeLse) {
+                        const int sv = jg % NSV;
+                        if (jg >= NSV && !(ok = wait_or_abort(&vempty[sv], ((jg / NSV) - 1) & 1, 0x202, abort_flag)))
+                            break;
+                        uint8_t* vs = smem + Cfg::kOffV + sv * Cfg::kVBytes;
+                        mbar_expect_tx(&vfull[sv], Cfg::kVBytes);
+#pragma unroll
+                        for (int hb = 0; hb < Cfg::BN / 64; ++hb)
+                            tma_load_4d(vs + hb * Cfg::kVBox, &mapV, &vfull[sv], kb + hb * 64, 0, g, b);
+                    }
                 }
+                jbase += ntiles;
             }
         }
     } else if (warp == 9) {
         // ----------------------------------------------------------- MMA
-        if (lane == 0 && ntiles > 0) {
+        if (lane == 0) {
             constexpr uint32_t idS = idesc_bf16(128, Cfg::BN);
             constexpr uint32_t idO = idesc_bf16(128, DV);
-            bool ok = wait_or_abort(qfull, 0, 0x203, abort_flag);
-            // S of key tile jt for query tile `tile` (and both tiles when tile < 0)
-            auto issue_S = [&](int jt, int only) -> bool {
-                const int s = jt % NSK, buf = Cfg::NBUF == 2 ? (jt & 1) : 0;
-                if (only <= 0 && !wait_or_abort(&kfull[s], (jt / NSK) & 1, 0x204, abort_flag)) return false;
-                const uint32_t sK = smem_u32(smem + Cfg::kOffK + s * Cfg::kKBytes);
+            int jbase = 0, qi = 0;
+            bool ok = true;
+            Item it;
+            for (int iter = 0; ok && item_of(iter, it); ++iter) {
+                const int ntiles = it.ntiles;
+                if (ntiles == 0) continue;
+                if (!(ok = wait_or_abort(qfull, qi & 1, 0x203, abort_flag))) break;
+                // the previous item's last P.V products have completed: its S buffers are
+                // free, and every pvdone phase waited for below belongs to this item
+                if (MODE != kModeLse && qi > 0)
+                    for (int tile = 0; tile < 2 && ok; ++tile)
+                        ok = wait_or_abort(&pvdone[tile], (jbase - 1) & 1, 0x20D, abort_flag);
+                if (!ok) break;
+                // S of key tile jt for query tile `tile` (and both tiles when tile < 0)
+                auto issue_S = [&](int jt, int only) -> bool {
+                    const int jg = jbase + jt;
+                    const int s = jg % NSK, buf = Cfg::NBUF == 2 ? (jg & 1) : 0;
+                    if (only <= 0 && !wait_or_abort(&kfull[s], (jg / NSK) & 1, 0x204, abort_flag)) return false;
+                    const uint32_t sK = smem_u32(smem + Cfg::kOffK + s * Cfg::kKBytes);
 #pragma unroll
-                for (int tile = 0; tile < 2; ++tile) {
-                    if (only >= 0 && tile != only) continue;
-                    if (MODE == kModeLse && jt >= 2 &&
-                        !wait_or_abort(&sfree[2 * tile + buf], ((jt - 2) >> 1) & 1, 0x205, abort_flag))
-                        return false;
-                    // the buffer's P(jt - NBUF) must have been read by its P.V product: an
-                    // MMA writing tensor memory is not ordered behind an earlier MMA that
-                    // reads the same columns as its A operand
-                    if (MODE != kModeLse && jt >= Cfg::NBUF &&
-                        !wait_or_abort(&pvdone[tile], (jt - Cfg::NBUF) & 1, 0x20B, abort_flag))
-                        return false;
-                    tc_fence_after();
-                    const uint32_t sQ = smem_u32(smem + Cfg::kOffQ + tile * Cfg::kQBytes);
+                    for (int tile = 0; tile < 2; ++tile) {
+                        if (only >= 0 && tile != only) continue;
+                        if (MODE == kModeLse && jg >= 2 &&
+                            !wait_or_abort(&sfree[2 * tile + buf], ((jg - 2) >> 1) & 1, 0x205, abort_flag))
+                            return false;
+                        // the buffer's P(jt - NBUF) must have been read by its P.V product: an
+                        // MMA writing tensor memory is not ordered behind an earlier MMA that
+                        // reads the same columns as its A operand
+                        if (MODE != kModeLse && jt >= Cfg::NBUF &&
+                            !wait_or_abort(&pvdone[tile], (jg - Cfg::NBUF) & 1, 0x20B, abort_flag))
+                            return false;
+                        tc_fence_after();
+                        const uint32_t sQ = smem_u32(smem + Cfg::kOffQ + tile * Cfg::kQBytes);
 #pragma unroll
-                    for (int kk = 0; kk < DK / 16; ++kk)
-                        umma_bf16_ss(tmem + tile * Cfg::NBUF * Cfg::BN + buf * Cfg::BN,
-                                     sdesc_sw128(sQ + (kk / 4) * 16384 + (kk % 4) * 32),
-                                     sdesc_sw128(sK + (kk / 4) * Cfg::kKBox + (kk % 4) * 32), idS,
-                                     kk > 0 ? 1u : 0u);
-                    umma_commit(&sfull[2 * tile + buf]);
-                }
-                if (only != 0) umma_commit(&kempty[s]);       // both tiles have read the K stage
-                return true;
-            };
-            // P.V of key tile jt for query tile `tile` (and both tiles when tile < 0)
-            auto issue_PV = [&](int jt, int only) -> bool {
-                const int sv = jt % NSV;
-                if (only <= 0 && !wait_or_abort(&vfull[sv], (jt / NSV) & 1, 0x207, abort_flag)) return false;
-                const uint32_t sV = smem_u32(smem + Cfg::kOffV + sv * Cfg::kVBytes);
+                        for (int kk = 0; kk < DK / 16; ++kk)
+                            umma_bf16_ss(tmem + tile * Cfg::NBUF * Cfg::BN + buf * Cfg::BN,
+                                         sdesc_sw128(sQ + (kk / 4) * 16384 + (kk % 4) * 32),
+                                         sdesc_sw128(sK + (kk / 4) * Cfg::kKBox + (kk % 4) * 32), idS,
+                                         kk > 0 ? 1u : 0u);
+                        umma_commit(&sfull[2 * tile + buf]);
+                    }
+                    if (only != 0) umma_commit(&kempty[s]);       // both tiles have read the K stage
+                    // after the item's last S products the Q tiles may be replaced
+                    if (only != 0 && jt == ntiles - 1) umma_commit(qempty);
+                    return true;
+                };
+                // P.V of key tile jt for query tile `tile` (and both tiles when tile < 0)
+                auto issue_PV = [&](int jt, int only) -> bool {
+                    const int jg = jbase + jt;
+                    const int sv = jg % NSV;
+                    if (only <= 0 && !wait_or_abort(&vfull[sv], (jg / NSV) & 1, 0x207, abort_flag)) return false;
+                    const uint32_t sV = smem_u32(smem + Cfg::kOffV + sv * Cfg::kVBytes);
 #pragma unroll
-                for (int tile = 0; tile < 2; ++tile) {
-                    if (only >= 0 && tile != only) continue;
-                    if (!wait_or_abort(&pfull[tile], jt & 1, 0x206, abort_flag)) return false;
-                    tc_fence_after();
-                    // P (bf16 pairs) over the first BN/2 columns of S(jt)
-                    const uint32_t tP = tmem + tile * Cfg::NBUF * Cfg::BN + (Cfg::NBUF == 2 ? (jt & 1) : 0) * Cfg::BN;
+                    for (int tile = 0; tile < 2; ++tile) {
+                        if (only >= 0 && tile != only) continue;
+                        if (!wait_or_abort(&pfull[tile], jg & 1, 0x206, abort_flag)) return false;
+                        // the first product of an item overwrites O: the previous item's
+                        // epilogue must have read it
+                        if (jt == 0 && qi > 0 && !wait_or_abort(&ofree[tile], (qi - 1) & 1, 0x20E, abort_flag))
+                            return false;
+                        tc_fence_after();
+                        // P (bf16 pairs) over the first BN/2 columns of S(jt)
+                        const uint32_t tP = tmem + tile * Cfg::NBUF * Cfg::BN + (Cfg::NBUF == 2 ? (jg & 1) : 0) * Cfg::BN;
 #pragma unroll
-                    for (int kk = 0; kk < Cfg::BN / 16; ++kk)
-                        umma_bf16_ts(tmem + 256 + tile * DV, tP + kk * 8,
-                                     sdesc_sw128(sV + (kk / 4) * Cfg::kVBox + (kk % 4) * 32), idO,
-                                     (jt > 0 || kk > 0) ? 1u : 0u);
-                    umma_commit(&pvdone[tile]);
+                        for (int kk = 0; kk < Cfg::BN / 16; ++kk)
+                            umma_bf16_ts(tmem + 256 + tile * DV, tP + kk * 8,
+                                         sdesc_sw128(sV + (kk / 4) * Cfg::kVBox + (kk % 4) * 32), idO,
+                                         (jt > 0 || kk > 0) ? 1u : 0u);
+                        umma_commit(&pvdone[tile]);
+                    }
+                    if (only != 0) umma_commit(&vempty[sv]);      // both tiles have read the V stage
+                    return true;
+                };
+                if (Cfg::NBUF == 2) {
+                    // S(jt+1) into the other buffer while the softmax works on S(jt)
+                    ok = issue_S(0, -1);
+                    for (int jt = 0; jt < ntiles && ok; ++jt) {
+                        if (jt + 1 < ntiles) ok = issue_S(jt + 1, -1);
+                        if (ok && MODE != kModeLse) ok = issue_PV(jt, -1);
+                    }
+                } else {
+                    // one S buffer per query tile: P.V(jt) of a tile, then its S(jt+1) into
+                    // the same columns; the two tiles alternate so that one tile's products
+                    // run while the other's softmax does
+                    ok = issue_S(0, 0);
+                    if (ok) ok = issue_S(0, 1);
+                    for (int jt = 0; jt < ntiles && ok; ++jt) {
+                        ok = issue_PV(jt, 0);
+                        if (ok && jt + 1 < ntiles) ok = issue_S(jt + 1, 0);
+                        if (ok) ok = issue_PV(jt, 1);
+                        if (ok && jt + 1 < ntiles) ok = issue_S(jt + 1, 1);
+                    }
                 }
-                if (only != 0) umma_commit(&vempty[sv]);      // both tiles have read the V stage
-                return true;
-            };
-            if (Cfg::NBUF == 2) {
-                // S(jt+1) into the other buffer while the softmax works on S(jt)
-                if (ok) ok = issue_S(0, -1);
-                for (int jt = 0; jt < ntiles && ok; ++jt) {
-                    if (jt + 1 < ntiles) ok = issue_S(jt + 1, -1);
-                    if (ok && MODE != kModeLse) ok = issue_PV(jt, -1);
-                }
-            } else {
-                // one S buffer per query tile: P.V(jt) of a tile, then its S(jt+1) into
-                // the same columns; the two tiles alternate so that one tile's products
-                // run while the other's softmax does
-                if (ok) ok = issue_S(0, 0);
-                if (ok) ok = issue_S(0, 1);
-                for (int jt = 0; jt < ntiles && ok; ++jt) {
-                    ok = issue_PV(jt, 0);
-                    if (ok && jt + 1 < ntiles) ok = issue_S(jt + 1, 0);
-                    if (ok) ok = issue_PV(jt, 1);
-                    if (ok && jt + 1 < ntiles) ok = issue_S(jt + 1, 1);
-                }
+                ++qi;
+                jbase += ntiles;
             }
         }
     } else {
@@ -327,6 +391,10 @@ __global__ void __launch_bounds__(320, 1)
         const int tile = warp >> 2;                 // 0: tile A, 1: tile B
         const int wq = warp & 3;                    // TMEM lane quadrant
         const int r = wq * 32 + lane;               // row within the tile
+        int jbase = 0;                              // key tiles before this item
+        Item it;
+        for (int iter = 0; item_of(iter, it); ++iter) {
+        const int g = it.g, b = it.b, t0 = it.t0, key0 = it.key0, ntiles = it.ntiles;
         const int t = t0 + tile * TOK + r / HG;
         const int hh = r % HG;
         const int h = g * HG + hh;
@@ -368,8 +436,8 @@ __global__ void __launch_bounds__(320, 1)
         if (MODE == kModeLse) {
             // BN = 128 keys per tile, read from TMEM in two halves of 64
             for (int jt = 0; jt < ntiles; ++jt) {
-                const int buf = jt & 1;
-                if (ok) ok = wait_or_abort(&sfull[2 * tile + buf], (jt >> 1) & 1, 0x208, abort_flag);
+                const int jg = jbase + jt, buf = jg & 1;
+                if (ok) ok = wait_or_abort(&sfull[2 * tile + buf], (jg >> 1) & 1, 0x208, abort_flag);
                 tc_fence_after();
 #pragma unroll 1
                 for (int hb = 0; hb < Cfg::BN / 64; ++hb) {
@@ -414,8 +482,9 @@ __global__ void __launch_bounds__(320, 1)
             }
         }
         for (int jt = 0; MODE != kModeLse && jt < ntiles; ++jt) {
-            const int buf = Cfg::NBUF == 2 ? (jt & 1) : 0;
-            if (ok) ok = wait_or_abort(&sfull[2 * tile + buf], (Cfg::NBUF == 2 ? (jt >> 1) : jt) & 1, 0x208, abort_flag);
+            const int jg = jbase + jt;
+            const int buf = Cfg::NBUF == 2 ? (jg & 1) : 0;
+            if (ok) ok = wait_or_abort(&sfull[2 * tile + buf], (Cfg::NBUF == 2 ? (jg >> 1) : jg) & 1, 0x208, abort_flag);
             tc_fence_after();
             // the key tile in halves of 64 keys (one half for the window)
 #pragma unroll 1
@@ -523,7 +592,7 @@ __global__ void __launch_bounds__(320, 1)
             // the previous P.V of this tile finished: the window's O rescale needs it,
             // and it keeps this loop at most one pvdone phase ahead of the MMA warp
             // (a parity wait cannot tell phases two apart; the epilogue relies on it)
-            if (hb == 0 && jt > 0 && ok) ok = wait_or_abort(&pvdone[tile], (jt - 1) & 1, 0x209, abort_flag);
+            if (hb == 0 && jt > 0 && ok) ok = wait_or_abort(&pvdone[tile], (jg - 1) & 1, 0x209, abort_flag);
             tc_fence_after();
             if (MODE == kModeWin && jt > 0 && __any_sync(0xffffffffu, need_rescale)) {
                 const float a = need_rescale ? alpha : 1.f;
@@ -573,7 +642,7 @@ __global__ void __launch_bounds__(320, 1)
                         p.pscore[(((size_t)b * p.T + t) * p.G + g) * p.NSp + jn + c] = v;
                 }
             }
-            if (ntiles > 0 && ok) ok = wait_or_abort(&pvdone[tile], (ntiles - 1) & 1, 0x20A, abort_flag);
+            if (ntiles > 0 && ok) ok = wait_or_abort(&pvdone[tile], (jbase + ntiles - 1) & 1, 0x20A, abort_flag);
             tc_fence_after();
             const float gate = row_ok ? p.gates[rowid * 3 + (MODE == kModeCmp ? 0 : 2)] : 0.f;
             const float inv = (MODE == kModeWin) ? (l_run > 0.f ? 1.f / l_run : 0.f) : 1.f;
@@ -620,6 +689,13 @@ __global__ void __launch_bounds__(320, 1)
             }
             if (MODE == kModeWin && row_ok && p.lse_user)
                 p.lse_user[rowid * 3 + 2] = (m_run + log2f(l_run)) * kLn2;
+            if (ntiles > 0) {
+                // this tile's O has been read: the next item's first P.V may overwrite it
+                tc_fence_before();
+                mbar_arrive(&ofree[tile]);
+            }
+        }
+        jbase += ntiles;
         }
     }
     tc_fence_before();

@@ -332,6 +332,8 @@ __global__ void cmp_empty_kernel(float* out, float* lse, long long rows, int DV)
 }
 
 // ----------------------------------------------------------- attention
+int device_sm_count();   // SMs of the current device (decode section)
+
 template <int DK, int DV, int HG, int MODE, int CPS, int SPB>
 nsa_status_t launch_packed(const Shape& s, const CUtensorMap& mQ, const CUtensorMap& mK,
                            const CUtensorMap& mV, const PackedParams& p, cudaStream_t st) {
@@ -340,6 +342,12 @@ nsa_status_t launch_packed(const Shape& s, const CUtensorMap& mQ, const CUtensor
     const char* kern_name = MODE == kModeLse ? "attn_cmp_lse" : MODE == kModeCmp ? "attn_cmp_pv_scores" : "attn_window";
     NSA_TRY(set_smem(kern, Cfg::kSmem));
     dim3 grid((unsigned)p.n_ctas, (unsigned)s.G, (unsigned)s.B);
+    if (MODE == kModeWin) {
+        // persistent: one CTA per SM walks the (tile pair, group, batch) items, so that one
+        // item's epilogue overlaps the next item's loads and products
+        const int64_t items = (int64_t)p.n_ctas * s.G * s.B;
+        grid = dim3((unsigned)std::min<int64_t>(items, device_sm_count()), 1, 1);
+    }
     NSA_LAUNCH(kern_name, st, kern<<<grid, Cfg::kThreads, Cfg::kSmem, st>>>(mQ, mK, mV, p));
     return last_launch();
 }

@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(320, 1)
     // tiles first; or, for the window (persistent launch), the CTAs stride over all items
     // so that one item's epilogue overlaps the next item's loads and products.  Every role
     // walks the same items in the same order and counts key tiles across them (jbase).
-    constexpr bool kPersist = MODE == kModeWin;
+    constexpr bool kPersist = MODE != kModeLse;
     struct Item {
         int g, b, t0, t_last, key0, ntiles;
     };

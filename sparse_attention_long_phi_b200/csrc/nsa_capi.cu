@@ -342,7 +342,7 @@ nsa_status_t launch_packed(const Shape& s, const CUtensorMap& mQ, const CUtensor
     const char* kern_name = MODE == kModeLse ? "attn_cmp_lse" : MODE == kModeCmp ? "attn_cmp_pv_scores" : "attn_window";
     NSA_TRY(set_smem(kern, Cfg::kSmem));
     dim3 grid((unsigned)p.n_ctas, (unsigned)s.G, (unsigned)s.B);
-    if (MODE == kModeWin) {
+    if (MODE != kModeLse) {
         // persistent: one CTA per SM walks the (tile pair, group, batch) items, so that one
         // item's epilogue overlaps the next item's loads and products
         const int64_t items = (int64_t)p.n_ctas * s.G * s.B;

@@ -162,10 +162,11 @@ __global__ void __launch_bounds__(320, 1)
     uint64_t* ofree = bars + 26;          // [tile] the epilogue has read O (persistent)
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    // Work items: a pair of query tiles of one (batch, group).  One item per CTA, heavy
-    // tiles first; or, for the window (persistent launch), the CTAs stride over all items
-    // so that one item's epilogue overlaps the next item's loads and products.  Every role
-    // walks the same items in the same order and counts key tiles across them (jbase).
+    // Work items: a pair of query tiles of one (batch, group).  Pass 1 takes one item per
+    // CTA, heavy tiles first; pass 2 and the window (persistent launch, one CTA per SM)
+    // stride over all items so that one item's epilogue overlaps the next item's loads and
+    // products.  Every role walks the same items in the same order and counts key tiles
+    // across them (jbase).
     constexpr bool kPersist = MODE != kModeLse;
     struct Item {
         int g, b, t0, t_last, key0, ntiles;

@@ -386,8 +386,8 @@ __global__ void __launch_bounds__(256, 1) dec_cmp_stream(const DecParams p) {
 // -------------------------------------------------------------- step 2
 // Every load that does not need the row LSE (chunk maxima, this thread's block
 // sums) is issued before the first barrier; the records give the LSE in one
-// round of loads (their O is merged by the final step); the top-n and the unit
-// list run on all warps.
+// batch of loads (their O is merged by the final step); the top-n runs on all
+// warps and writes the row's selected block indices.
 template <int DV>
 __global__ void __launch_bounds__(256) dec_cmp_combine(const DecParams p) {
     constexpr int REC = DV + 4;
@@ -969,11 +969,11 @@ __global__ void __launch_bounds__(256, 1) dec_slcwin_stream(const DecParams p) {
 
 // -------------------------------------------------------------- step 4
 // Per (seq, group) and eight heads (grid z): the records of all three
-// branches merged in two rounds of loads, each round issued at once.  Round 1:
+// branches merged in two phases of loads, each phase issued at once.  Phase 1:
 // warp w takes the compressed records of head w (weight exp2(m - LSE) under
 // the combine's LSE) and the selected/window records of two (branch, head)
 // groups, 16 lanes per group (the branch max M, sum L and the weight
-// exp2(m - M) / L of every record).  Round 2: one thread per output float4
+// exp2(m - M) / L of every record).  Phase 2: one thread per output float4
 // (two for d_v = 64, each taking every other record) sums the weighted O of
 // the records, eight of each kind per batch of loads; then
 // out = sum_c g_c o_c and the LSEs.  256 CTAs of at most 128 registers per
@@ -1066,7 +1066,7 @@ __global__ void __launch_bounds__(256, 2) dec_final(const DecParams p) {
         if (sub == 0) lsb[br][hl] = Ls > 0.f ? M + log2f(Ls) : -INFINITY;
     }
     __syncthreads();
-    // round 2: output e (head h0 + e / (DV/4), channels c4 .. c4+3)
+    // phase 2: output e (head h0 + e / (DV/4), channels c4 .. c4+3)
     const int e = threadIdx.x % NOUT, half = threadIdx.x / NOUT;
     const int hl = e / (DV / 4), c4 = (e % (DV / 4)) * 4, h = h0 + hl;
     const bool active = h < p.HG;
